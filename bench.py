@@ -1,0 +1,453 @@
+"""KDA throughput on B200: tokens/s and fraction of roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is the production training pass of the recurrence: the chunked
+prefill forward (which also stores the chunk states) and the chunked
+backward that reuses them, on B=2, H=HV=96, T=4096, K=V=128, bf16 inputs,
+fp32 state (all hot-path kernels except the decode step).  The prefill-only
+workloads and the batched decode step are timed the same way and reported
+under "paths".  A token is one (batch, time) position with all value heads.
+
+With N > 1 (torchrun, one process per GPU) every rank runs its own replica of
+the per-GPU workload (independent batches, no data-path collective): weak
+scaling; the timed region is bracketed by barriers and the slowest rank's
+device time is reported.
+
+``--impl reference`` times the float64 CPU oracle (the only reference this
+method has) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import multiprocessing as mp
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from gated_delta_rule_66_b200.inputs import BY_NAME, make_inputs  # noqa: E402
+
+HEADLINE = "fwdbwd"
+PATHS = ("twin", "prefill_gqa", "fwdbwd", "decode")
+METRIC = "KDA tokens/s at 1 B200 (prefill fwd, fwd+bwd, decode) + % of roofline"
+L2_BYTES = 126 * 2 ** 20
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------- algorithmic work
+
+def esize(w):
+    return 4 if w.dtype == "fp32" else 2
+
+
+def algorithmic_bytes(w, kind):
+    """Bytes a kernel must move at least once (inputs read, outputs written)."""
+    B, T, H, HV, K, V, e = w.B, w.T, w.H, w.HV, w.K, w.V, esize(w)
+    state = B * HV * K * V * 4
+    if kind == "decode":
+        return 2 * state + B * (2 * H * K * e + HV * V * e + HV * K * 4 + HV * 4 + HV * V * e)
+    fwd_in = B * T * (2 * H * K * e + HV * V * e + HV * K * 4 + HV * 4)
+    fwd_out = B * T * HV * V * e + state                      # o, S_T
+    s0 = state if w.s0_std > 0 else 0
+    if kind == "fwd":
+        return fwd_in + fwd_out + s0
+    # backward: reads the forward inputs and dO, writes dq, dk, dv, dg, dbeta, dS0
+    bwd = fwd_in + B * T * HV * V * e + B * T * (2 * H * K * e + HV * V * e + HV * K * 4 + HV * 4) + state
+    return fwd_in + fwd_out + s0 + bwd
+
+
+def chunk_flops_per_head_token(K, V, C):
+    """Flops of the chunked form per (head, token): three K x V state
+    contractions (residual, readout, carry), the two C x C x K interaction
+    products, and the C x C x V solve and readout products (dense tiles)."""
+    return 2 * (3 * K * V + 2 * C * K + 2 * C * V)
+
+
+# ---------------------------------------------------------------------------- GPU arm
+
+class Clocks:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[4:8]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def _flush_l2(buf):
+    buf.add_(1)
+
+
+def gpu_path(kda, name, steps, warmup, rank_barrier):
+    """Times one workload on this rank's GPU.  Returns a result dict."""
+    w = BY_NAME[name]
+    inp = make_inputs(w, with_do=(w.path == "fwdbwd"))
+    dev = torch.device("cuda")
+    d = {n: (None if t is None else t.to(dev)) for n, t in inp.items()}
+    flush = None
+    in_bytes = sum(t.numel() * t.element_size() for t in inp.values() if t is not None)
+    if in_bytes < 2 * L2_BYTES:
+        flush = torch.zeros(256 * 2 ** 20 // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    launches_per_step = 0
+    ws = None
+
+    if w.path == "fwd":
+        def step():
+            if flush is not None:
+                _flush_l2(flush)
+            kda.fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], scale=w.scale, initial_state=d["S0"])
+        launches_per_step = 1
+        tokens = w.B * w.T
+    elif w.path == "fwdbwd":
+        ws = torch.empty(kda.workspace_bytes("bwd", w.B, w.T, w.H, w.HV, w.K, w.V), dtype=torch.uint8,
+                         device=dev)
+
+        def step():
+            kda.fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], scale=w.scale, initial_state=d["S0"],
+                    workspace=ws)
+            kda.bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["dO"], scale=w.scale,
+                    initial_state=d["S0"], workspace=ws, states_from_fwd=True)
+        launches_per_step = 3 + (2 if w.HV > w.H else 0)
+        tokens = w.B * w.T
+    else:
+        S = d["S"]
+
+        def step():
+            kda.decode_step(d["q"], d["k"], d["v"], d["g"], d["beta"], S, scale=w.scale)
+        launches_per_step = 1
+        tokens = w.B
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    rank_barrier()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1) / steps
+    res = {"workload": name, "ms_per_step": ms, "tokens_per_step": tokens,
+           "launches_per_step": launches_per_step, "l2": "flushed" if flush is not None else "inputs > L2"}
+
+    # per-call kernel timing (each C-ABI call below is the launch(es) named)
+    calls = {}
+    if w.path in ("fwd", "decode"):
+        calls["kernel_ms"] = ms  # one kernel per step
+    else:
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        t_f, t_b = 0.0, 0.0
+        for _ in range(steps):
+            e[0].record(stream)
+            kda.fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], scale=w.scale, initial_state=d["S0"],
+                    workspace=ws)
+            e[1].record(stream)
+            kda.bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["dO"], scale=w.scale,
+                    initial_state=d["S0"], workspace=ws, states_from_fwd=True)
+            e[2].record(stream)
+            torch.cuda.synchronize()
+            t_f += e[0].elapsed_time(e[1])
+            t_b += e[1].elapsed_time(e[2])
+        calls["fwd_ms"] = t_f / steps
+        calls["bwd_ms"] = t_b / steps
+    res["calls"] = calls
+
+    # end to end through the public API with host buffers (pinned), copies inside
+    pinned = {n: (None if t is None else t.pin_memory()) for n, t in inp.items()}
+    h2d = sum(t.numel() * t.element_size() for t in pinned.values() if t is not None)
+
+    def e2e_step():
+        dd = {n: (None if t is None else t.to(dev, non_blocking=True)) for n, t in pinned.items()}
+        if w.path == "fwd":
+            outs = kda.fwd(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], scale=w.scale,
+                           initial_state=dd["S0"])
+        elif w.path == "fwdbwd":
+            o, S_T = kda.fwd(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], scale=w.scale,
+                             initial_state=dd["S0"], workspace=ws)
+            outs = (o, S_T) + kda.bwd(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["dO"],
+                                      scale=w.scale, initial_state=dd["S0"], workspace=ws,
+                                      states_from_fwd=True)
+        else:
+            outs = (kda.decode_step(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["S"],
+                                    scale=w.scale), dd["S"])
+        host = [t.to("cpu", non_blocking=True) for t in outs if t is not None]
+        return host
+
+    e2e_steps = max(1, min(steps, 5))
+    e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        host = e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    d2h = sum(t.numel() * t.element_size() for t in host)
+    res["e2e_ms"] = e0.elapsed_time(e1) / e2e_steps
+    res["h2d_bytes"] = h2d
+    res["d2h_bytes"] = d2h
+    del ws
+    return res, w
+
+
+def roofline_for(res, w, peaks):
+    hbm = peaks["hbm_gbs"]
+    if w.path == "decode":
+        byts = algorithmic_bytes(w, "decode")
+        t = res["calls"]["kernel_ms"] * 1e-3
+        return {"bound": "hbm", "kernel": "kda_decode_kernel", "achieved": byts / t / 1e9,
+                "peak": hbm, "unit": "GB/s", "frac": byts / t / 1e9 / hbm, "algorithmic_bytes": byts}
+    if w.path == "fwd":
+        byts = algorithmic_bytes(w, "fwd")
+        t = res["calls"]["kernel_ms"] * 1e-3
+        return {"bound": "hbm", "kernel": "kda_fwd_chunk_kernel", "achieved": byts / t / 1e9,
+                "peak": hbm, "unit": "GB/s", "frac": byts / t / 1e9 / hbm, "algorithmic_bytes": byts}
+    byts = algorithmic_bytes(w, "fwd")
+    t = res["calls"]["fwd_ms"] * 1e-3
+    return {"bound": "hbm", "kernel": "kda_fwd_chunk_kernel (state-storing forward of the step)",
+            "achieved": byts / t / 1e9, "peak": hbm, "unit": "GB/s", "frac": byts / t / 1e9 / hbm,
+            "algorithmic_bytes": byts}
+
+
+def run_gpu(args):
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    from gated_delta_rule_66_b200 import kda
+    peaks = load_peaks()
+    results = {}
+    for name in [HEADLINE] + [p for p in PATHS if p != HEADLINE and args.all_paths]:
+        if name == HEADLINE:
+            with Clocks(local) as clk:
+                res, w = gpu_path(kda, name, args.steps, args.warmup, barrier)
+            res["clocks"] = clk.summary()
+        else:
+            res, w = gpu_path(kda, name, args.steps, args.warmup, barrier)
+        res["roofline"] = roofline_for(res, w, peaks)
+        ms = res["ms_per_step"]
+        if world > 1:
+            t = torch.tensor([ms], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+            res["ms_per_step"] = ms
+        res["tokens_per_s"] = res["tokens_per_step"] * world / (ms * 1e-3)
+        res["e2e_tokens_per_s"] = res["tokens_per_step"] * world / (res["e2e_ms"] * 1e-3)
+        results[name] = (res, w)
+        torch.cuda.empty_cache()
+
+    head, w = results[HEADLINE]
+    line = {
+        "metric": METRIC,
+        "value": head["tokens_per_s"],
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": head["ms_per_step"],
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded; q,k L2-normalised, g = -5 sigmoid(N(0,1)), beta = sigmoid(N(0,1)))",
+        "config": {"workload": "fwdbwd: B=2 H=HV=96 T=4096 K=V=128, bf16 q/k/v/dO, fp32 g/beta/state; "
+                               "step = kda_fwd (stores chunk states) + kda_bwd (reuses them)",
+                   "global_batch": w.B * world, "seq_len": w.T, "parallelism": f"replicas x{world}",
+                   "l2": head["l2"]},
+        "roofline": dict(head["roofline"], traffic=None),
+        "e2e": {"value": head["e2e_tokens_per_s"], "unit": "tokens/s",
+                "h2d_bytes_per_step": head["h2d_bytes"], "d2h_bytes_per_step": head["d2h_bytes"]},
+        "gpu_launches": head["launches_per_step"] * args.steps,
+        "clocks": head.get("clocks"),
+        "peaks": peaks,
+        "paths": {n: {"tokens_per_s": r["tokens_per_s"], "ms_per_step": r["ms_per_step"],
+                      "e2e_tokens_per_s": r["e2e_tokens_per_s"], "calls_ms": r["calls"],
+                      "roofline": r["roofline"], "l2": r["l2"]} for n, (r, _) in results.items()},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_seconds)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------- CPU oracle arm
+
+def _oracle_head(job):
+    """Runs the float64 oracle fwd (+bwd) on one value head of a sample."""
+    import numpy as np
+    sys.path.insert(0, ROOT)
+    import oracle
+    path, arrays, scale = job
+    q, k, v, g, beta, S0, dO = arrays
+    t0 = time.perf_counter()
+    o, S = oracle.kda_forward(q, k, v, g, beta, scale, S0)
+    if path == "fwdbwd":
+        oracle.kda_backward(q, k, v, g, beta, scale, S0, dO)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(w, budget_s=20.0):
+    """Times the oracle on a bounded sample of workload ``w`` on the host's
+    cores: whole value heads (one per worker process) over the first T_s
+    tokens of batch row 0; tokens/s is scaled to all HV heads."""
+    import numpy as np
+    cores = len(os.sched_getaffinity(0))
+    Ts = {"fwdbwd": 256, "fwd": 512, "decode": 1}[w.path]
+    T_s = min(w.T, Ts)
+    sub = w.with_sizes(B=1, T=T_s) if w.path != "decode" else w
+    inp = make_inputs(sub, with_do=(w.path == "fwdbwd")) if w.path != "decode" else None
+    if w.path == "decode":
+        nheads = min(w.HV, cores * 4)
+        sub = w.with_sizes(B=1)
+        inp = make_inputs(sub)
+    f64 = lambda t: None if t is None else t.to(torch.float64).numpy()
+    G = w.HV // w.H
+    jobs = []
+    nheads = min(w.HV, max(cores, 1) * 2)
+    for hv in range(nheads):
+        h = hv // G
+        if w.path == "decode":
+            arrays = (f64(inp["q"][:, None, h:h + 1]), f64(inp["k"][:, None, h:h + 1]),
+                      f64(inp["v"][:, None, hv:hv + 1]), f64(inp["g"][:, None, hv:hv + 1]),
+                      f64(inp["beta"][:, None, hv:hv + 1]), f64(inp["S"][:, hv:hv + 1]), None)
+        else:
+            arrays = (f64(inp["q"][:, :, h:h + 1]), f64(inp["k"][:, :, h:h + 1]),
+                      f64(inp["v"][:, :, hv:hv + 1]), f64(inp["g"][:, :, hv:hv + 1]),
+                      f64(inp["beta"][:, :, hv:hv + 1]),
+                      None if inp["S0"] is None else f64(inp["S0"][:, hv:hv + 1]),
+                      None if inp.get("dO") is None else f64(inp["dO"][:, :, hv:hv + 1]))
+        jobs.append((w.path, arrays, w.scale))
+    ctx = mp.get_context("spawn")
+    t0 = time.perf_counter()
+    with ctx.Pool(processes=cores) as pool:
+        pool.map(_oracle_head, jobs)
+    elapsed = time.perf_counter() - t0
+    head_tokens = nheads * T_s
+    tokens_per_s = head_tokens / w.HV / elapsed
+    return {"value": tokens_per_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{nheads} of {w.HV} value heads x {T_s} tokens of batch row 0 "
+                      f"({'fwd+bwd' if w.path == 'fwdbwd' else w.path}), float64 NumPy, one process per "
+                      f"core; tokens/s scaled to all {w.HV} heads", "seconds": elapsed}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = BY_NAME[HEADLINE]
+    times = []
+    cb = None
+    for _ in range(args.warmup + args.steps):
+        cb = cpu_baseline(w, budget_s=args.cpu_seconds)
+        times.append(cb)
+    timed = times[args.warmup:]
+    val = statistics.median(c["value"] for c in timed)
+    line = {"metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": BY_NAME[HEADLINE].B * BY_NAME[HEADLINE].T / val * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": "fwdbwd: B=2 H=HV=96 T=4096 K=V=128 (oracle on a bounded sample)",
+                       "global_batch": w.B, "seq_len": w.T, "parallelism": "none"},
+            "cpu_baseline": {"kind": "oracle", "cores": cb["cores"], "sample": cb["sample"], "value": val,
+                             "unit": "tokens/s"},
+            "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--headline-only", dest="all_paths", action="store_false")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,151 @@
+// C ABI of the KDA library: argument validation, workspace carving and
+// dispatch to the kernels.  See include/kda.h for the contract.
+#include <math.h>
+#include <stdint.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "../../include/kda.h"
+#include "kda_internal.h"
+
+namespace kda {
+
+static thread_local char g_err[512] = "";
+
+int set_error(int code, const char* msg) {
+  snprintf(g_err, sizeof(g_err), "%s", msg);
+  return code;
+}
+
+int set_cuda_error(const char* where, cudaError_t e) {
+  snprintf(g_err, sizeof(g_err), "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
+  return KDA_ERR_CUDA;
+}
+
+static bool supported_dim(int d) { return d == 32 || d == 64 || d == 128; }
+
+static int check_common(const char* fn, int B, int T, int H, int HV, int K, int V, int dtype,
+                        float scale) {
+  char buf[256];
+  if (B < 1 || T < 1 || H < 1 || HV < 1 || K < 1 || V < 1) {
+    snprintf(buf, sizeof(buf), "%s: sizes must be >= 1 (B=%d T=%d H=%d HV=%d K=%d V=%d)", fn, B, T, H,
+             HV, K, V);
+    return set_error(KDA_ERR_SHAPE, buf);
+  }
+  if (HV % H != 0) {
+    snprintf(buf, sizeof(buf), "%s: HV=%d is not a multiple of H=%d", fn, HV, H);
+    return set_error(KDA_ERR_SHAPE, buf);
+  }
+  if (B > 65535 || HV > 65535) {
+    snprintf(buf, sizeof(buf), "%s: B=%d or HV=%d exceeds 65535", fn, B, HV);
+    return set_error(KDA_ERR_SHAPE, buf);
+  }
+  if (!supported_dim(K) || !supported_dim(V)) {
+    snprintf(buf, sizeof(buf), "%s: K=%d, V=%d; each must be 32, 64 or 128", fn, K, V);
+    return set_error(KDA_ERR_UNSUPPORTED, buf);
+  }
+  if (dtype != KDA_DTYPE_FP32 && dtype != KDA_DTYPE_BF16) {
+    snprintf(buf, sizeof(buf), "%s: dtype=%d is not KDA_DTYPE_FP32 (0) or KDA_DTYPE_BF16 (1)", fn, dtype);
+    return set_error(KDA_ERR_DTYPE, buf);
+  }
+  if (!(scale > 0.f) || !isfinite(scale)) {
+    snprintf(buf, sizeof(buf), "%s: scale=%g must be finite and > 0", fn, (double)scale);
+    return set_error(KDA_ERR_ARG, buf);
+  }
+  return KDA_OK;
+}
+
+static size_t states_bytes(int B, int T, int HV, int K, int V) {
+  const size_t NT = (size_t)(T + FWD_CHUNK - 1) / FWD_CHUNK;
+  return (size_t)B * HV * NT * K * V * sizeof(float);
+}
+
+static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+}  // namespace kda
+
+using namespace kda;
+
+extern "C" {
+
+const char* kda_last_error(void) { return g_err; }
+
+size_t kda_fwd_workspace_bytes(int B, int T, int HV, int K, int V) {
+  if (B < 1 || T < 1 || HV < 1 || K < 1 || V < 1) return 0;
+  return states_bytes(B, T, HV, K, V);
+}
+
+size_t kda_bwd_workspace_bytes(int B, int T, int H, int HV, int K, int V) {
+  if (B < 1 || T < 1 || H < 1 || HV < 1 || K < 1 || V < 1 || HV % H) return 0;
+  size_t bytes = 2 * states_bytes(B, T, HV, K, V);
+  if (HV > H) bytes += 2 * (size_t)B * T * HV * K * sizeof(float);
+  return bytes;
+}
+
+int kda_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+            const float* S0, float scale, int B, int T, int H, int HV, int K, int V, int dtype,
+            void* o, float* S_T, void* workspace, size_t workspace_bytes, void* stream) {
+  g_err[0] = 0;
+  int rc = check_common("kda_fwd", B, T, H, HV, K, V, dtype, scale);
+  if (rc) return rc;
+  if (!q || !k || !v || !g || !beta || !o)
+    return set_error(KDA_ERR_NULL, "kda_fwd: q, k, v, g, beta and o must be non-NULL");
+  if (workspace) {
+    if (workspace_bytes < states_bytes(B, T, HV, K, V))
+      return set_error(KDA_ERR_WORKSPACE, "kda_fwd: workspace smaller than kda_fwd_workspace_bytes()");
+    if (!aligned16(workspace)) return set_error(KDA_ERR_ARG, "kda_fwd: workspace must be 16-byte aligned");
+  }
+  FwdArgs a{q, k, v, g, beta, S0, o, S_T, static_cast<float*>(workspace), scale, B, T, H, HV, K, V};
+  return launch_fwd(a, dtype, static_cast<cudaStream_t>(stream));
+}
+
+int kda_decode_step(const void* q, const void* k, const void* v, const float* g,
+                    const float* beta, float* S, float scale, int B, int H, int HV, int K, int V,
+                    int dtype, void* o, void* stream) {
+  g_err[0] = 0;
+  int rc = check_common("kda_decode_step", B, 1, H, HV, K, V, dtype, scale);
+  if (rc) return rc;
+  if (!q || !k || !v || !g || !beta || !S || !o)
+    return set_error(KDA_ERR_NULL, "kda_decode_step: q, k, v, g, beta, S and o must be non-NULL");
+  if (!aligned16(S)) return set_error(KDA_ERR_ARG, "kda_decode_step: S must be 16-byte aligned");
+  DecodeArgs a{q, k, v, g, beta, S, o, scale, B, H, HV};
+  return launch_decode(a, K, V, dtype, static_cast<cudaStream_t>(stream));
+}
+
+int kda_bwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+            const float* S0, const void* dO, const float* dS_T, float scale, int B, int T, int H,
+            int HV, int K, int V, int dtype, void* dq, void* dk, void* dv, float* dg,
+            float* dbeta, float* dS0, void* workspace, size_t workspace_bytes, int flags,
+            void* stream) {
+  g_err[0] = 0;
+  int rc = check_common("kda_bwd", B, T, H, HV, K, V, dtype, scale);
+  if (rc) return rc;
+  if (!q || !k || !v || !g || !beta || !dO || !dq || !dk || !dv || !dg || !dbeta)
+    return set_error(KDA_ERR_NULL,
+                     "kda_bwd: q, k, v, g, beta, dO, dq, dk, dv, dg and dbeta must be non-NULL");
+  if (flags & ~KDA_BWD_STATES_FROM_FWD) return set_error(KDA_ERR_ARG, "kda_bwd: unknown flags");
+  if (!workspace) return set_error(KDA_ERR_WORKSPACE, "kda_bwd: workspace is required");
+  if (workspace_bytes < kda_bwd_workspace_bytes(B, T, H, HV, K, V))
+    return set_error(KDA_ERR_WORKSPACE, "kda_bwd: workspace smaller than kda_bwd_workspace_bytes()");
+  if (!aligned16(workspace)) return set_error(KDA_ERR_ARG, "kda_bwd: workspace must be 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t sb = states_bytes(B, T, HV, K, V);
+  char* ws = static_cast<char*>(workspace);
+  float* states = reinterpret_cast<float*>(ws);
+  float* dstates = reinterpret_cast<float*>(ws + sb);
+  float *dq_part = nullptr, *dk_part = nullptr;
+  if (HV > H) {
+    dq_part = reinterpret_cast<float*>(ws + 2 * sb);
+    dk_part = dq_part + (size_t)B * T * HV * K;
+  }
+  if (!(flags & KDA_BWD_STATES_FROM_FWD)) {
+    FwdArgs fa{q, k, v, g, beta, S0, nullptr, nullptr, states, scale, B, T, H, HV, K, V};
+    rc = launch_fwd(fa, dtype, st);
+    if (rc) return rc;
+  }
+  BwdArgs a{q, k, v, dO, g, beta, dS_T, states, dstates, dq, dk, dv, dg, dbeta, dS0,
+            dq_part, dk_part, scale, B, T, H, HV, K, V};
+  return launch_bwd(a, dtype, st);
+}
+
+}  // extern "C"

@@ -1,0 +1,52 @@
+// Internal declarations shared by the KDA library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+namespace kda {
+
+constexpr int FWD_CHUNK = 32;    // chunk length of the chunked kernels
+constexpr int FWD_VBLOCK = 32;   // V columns per CTA in the chunked kernels
+
+struct FwdArgs {
+  const void *q, *k, *v;
+  const float *g, *beta, *S0;
+  void* o;          // may be null (state pass only)
+  float* S_T;       // may be null
+  float* states;    // may be null; [B, HV, NT, K, V] state entering each chunk
+  float scale;
+  int B, T, H, HV, K, V;
+};
+
+struct BwdArgs {
+  const void *q, *k, *v, *dO;
+  const float *g, *beta, *dS_T;
+  const float* states;   // [B, HV, NT, K, V]
+  float* dstates;        // [B, HV, NT, K, V] gradient of the state leaving each chunk
+  void *dq, *dk, *dv;    // dtype of q/k/v
+  float *dg, *dbeta, *dS0;
+  float *dq_part, *dk_part;  // fp32 [B, T, HV, K] per value head when HV > H, else null
+  float scale;
+  int B, T, H, HV, K, V;
+};
+
+struct DecodeArgs {
+  const void *q, *k, *v;
+  const float *g, *beta;
+  float* S;
+  void* o;
+  float scale;
+  int B, H, HV;
+};
+
+// error reporting (thread-local message; returns the code)
+int set_error(int code, const char* msg);
+int set_cuda_error(const char* where, cudaError_t e);
+
+int launch_fwd(const FwdArgs& a, int dtype, cudaStream_t stream);
+size_t fwd_smem_bytes(int K);
+int launch_bwd(const BwdArgs& a, int dtype, cudaStream_t stream);
+int launch_decode(const DecodeArgs& a, int K, int V, int dtype, cudaStream_t stream);
+
+}  // namespace kda

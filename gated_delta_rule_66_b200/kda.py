@@ -1,0 +1,198 @@
+"""Thin Python binding of libkda.so (include/kda.h).
+
+Argument marshalling only: every step of the recurrence runs in the CUDA
+kernels behind the C ABI.  Tensors must be CUDA, contiguous and of the
+documented dtypes; outputs are allocated here with torch (device memory is
+torch's job) and the call is enqueued on torch's current stream.  There is no
+CPU fallback: if the compiled library is missing the import fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libkda.so")
+
+KDA_DTYPE_FP32 = 0
+KDA_DTYPE_BF16 = 1
+KDA_BWD_STATES_FROM_FWD = 1
+CHUNK = 32  # chunk length of the library's chunked kernels (workspace layout)
+
+SYMBOLS = ("kda_last_error", "kda_fwd_workspace_bytes", "kda_bwd_workspace_bytes", "kda_fwd",
+           "kda_decode_step", "kda_bwd")
+
+
+class KdaError(RuntimeError):
+    """A non-zero status from the KDA library, with its message."""
+
+    def __init__(self, fn, code, msg):
+        super().__init__(f"{fn} failed with status {code}: {msg}")
+        self.code = code
+
+
+def _load():
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(
+            f"{_LIB_PATH} is missing: build it with `python -m gated_delta_rule_66_b200.build` "
+            "(the KDA library has no CPU fallback)")
+    lib = ctypes.CDLL(_LIB_PATH)
+    vp, f, i, sz = ctypes.c_void_p, ctypes.c_float, ctypes.c_int, ctypes.c_size_t
+    lib.kda_last_error.restype = ctypes.c_char_p
+    lib.kda_last_error.argtypes = []
+    lib.kda_fwd_workspace_bytes.restype = sz
+    lib.kda_fwd_workspace_bytes.argtypes = [i, i, i, i, i]
+    lib.kda_bwd_workspace_bytes.restype = sz
+    lib.kda_bwd_workspace_bytes.argtypes = [i, i, i, i, i, i]
+    lib.kda_fwd.restype = i
+    lib.kda_fwd.argtypes = [vp, vp, vp, vp, vp, vp, f, i, i, i, i, i, i, i, vp, vp, vp, sz, vp]
+    lib.kda_decode_step.restype = i
+    lib.kda_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, f, i, i, i, i, i, i, vp, vp]
+    lib.kda_bwd.restype = i
+    lib.kda_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, f, i, i, i, i, i, i, i,
+                            vp, vp, vp, vp, vp, vp, vp, sz, i, vp]
+    return lib
+
+
+_lib = _load()
+
+
+def library():
+    """The loaded ctypes handle of libkda.so (raw C-ABI access)."""
+    return _lib
+
+
+def _check(fn, rc):
+    if rc != 0:
+        raise KdaError(fn, rc, _lib.kda_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype_code(t):
+    if t.dtype == torch.float32:
+        return KDA_DTYPE_FP32
+    if t.dtype == torch.bfloat16:
+        return KDA_DTYPE_BF16
+    raise TypeError(f"q/k/v must be float32 or bfloat16, got {t.dtype}")
+
+
+def _req(name, t, dtype=None, ndim=None):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {tuple(t.shape)}")
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def workspace_bytes(kind, B, T, H, HV, K, V):
+    """Workspace bytes of ``kind`` = "fwd" (chunk states) or "bwd"."""
+    if kind == "fwd":
+        return int(_lib.kda_fwd_workspace_bytes(B, T, HV, K, V))
+    return int(_lib.kda_bwd_workspace_bytes(B, T, H, HV, K, V))
+
+
+def fwd(q, k, v, g, beta, scale=None, initial_state=None, output_final_state=True,
+        workspace=None, out=None):
+    """Prefill forward.  Returns (o [B,T,HV,V] in v's dtype, S_T or None).
+
+    q, k [B,T,H,K]; v [B,T,HV,V] (same dtype); g [B,T,HV,K], beta [B,T,HV] and
+    initial_state [B,HV,K,V] float32.  ``workspace`` (a uint8 CUDA tensor of
+    at least workspace_bytes("fwd", ...)) receives the chunk states for a
+    later ``bwd(..., workspace=..., states_from_fwd=True)``.
+    """
+    B, T, H, K = q.shape
+    HV, V = v.shape[2], v.shape[3]
+    scale = 1.0 / math.sqrt(K) if scale is None else float(scale)
+    dt = q.dtype
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _req(n, t, dt, 4)
+    _req("g", g, torch.float32, 4)
+    _req("beta", beta, torch.float32, 3)
+    _req("initial_state", initial_state, torch.float32, 4)
+    _req("workspace", workspace)
+    o = torch.empty(B, T, HV, V, dtype=dt, device=q.device) if out is None else out
+    _req("out", o, dt, 4)
+    S_T = torch.empty(B, HV, K, V, dtype=torch.float32, device=q.device) if output_final_state else None
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = _lib.kda_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state), scale,
+                      B, T, H, HV, K, V, _dtype_code(q), _ptr(o), _ptr(S_T), _ptr(workspace),
+                      ws_bytes, _stream())
+    _check("kda_fwd", rc)
+    return o, S_T
+
+
+def decode_step(q, k, v, g, beta, state, scale=None, out=None):
+    """One decode token; ``state`` [B,HV,K,V] float32 is updated in place.
+
+    q, k [B,H,K]; v [B,HV,V] (same dtype); g [B,HV,K], beta [B,HV] float32.
+    Returns o [B,HV,V] in v's dtype.
+    """
+    B, H, K = q.shape
+    HV, V = v.shape[1], v.shape[2]
+    scale = 1.0 / math.sqrt(K) if scale is None else float(scale)
+    dt = q.dtype
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _req(n, t, dt, 3)
+    _req("g", g, torch.float32, 3)
+    _req("beta", beta, torch.float32, 2)
+    _req("state", state, torch.float32, 4)
+    o = torch.empty(B, HV, V, dtype=dt, device=q.device) if out is None else out
+    _req("out", o, dt, 3)
+    rc = _lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state), scale,
+                              B, H, HV, K, V, _dtype_code(q), _ptr(o), _stream())
+    _check("kda_decode_step", rc)
+    return o
+
+
+def bwd(q, k, v, g, beta, dO, scale=None, initial_state=None, dS_T=None, workspace=None,
+        states_from_fwd=False, want_dS0=True):
+    """Backward.  Returns (dq, dk, dv, dg, dbeta, dS0 or None).
+
+    dq, dk [B,T,H,K] and dv [B,T,HV,V] in the input dtype; dg, dbeta, dS0
+    float32.  ``workspace`` defaults to a fresh allocation of
+    workspace_bytes("bwd", ...); pass the tensor given to ``fwd`` together
+    with ``states_from_fwd=True`` to reuse its chunk states.
+    """
+    B, T, H, K = q.shape
+    HV, V = v.shape[2], v.shape[3]
+    scale = 1.0 / math.sqrt(K) if scale is None else float(scale)
+    dt = q.dtype
+    for n, t in (("q", q), ("k", k), ("v", v), ("dO", dO)):
+        _req(n, t, dt, 4)
+    _req("g", g, torch.float32, 4)
+    _req("beta", beta, torch.float32, 3)
+    _req("initial_state", initial_state, torch.float32, 4)
+    _req("dS_T", dS_T, torch.float32, 4)
+    need = workspace_bytes("bwd", B, T, H, HV, K, V)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _req("workspace", workspace)
+    dev = q.device
+    dq = torch.empty(B, T, H, K, dtype=dt, device=dev)
+    dk = torch.empty(B, T, H, K, dtype=dt, device=dev)
+    dv = torch.empty(B, T, HV, V, dtype=dt, device=dev)
+    dg = torch.empty(B, T, HV, K, dtype=torch.float32, device=dev)
+    dbeta = torch.empty(B, T, HV, dtype=torch.float32, device=dev)
+    dS0 = torch.empty(B, HV, K, V, dtype=torch.float32, device=dev) if want_dS0 else None
+    rc = _lib.kda_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state),
+                      _ptr(dO), _ptr(dS_T), scale, B, T, H, HV, K, V, _dtype_code(q),
+                      _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(dbeta), _ptr(dS0),
+                      _ptr(workspace), workspace.numel() * workspace.element_size(),
+                      KDA_BWD_STATES_FROM_FWD if states_from_fwd else 0, _stream())
+    _check("kda_bwd", rc)
+    return dq, dk, dv, dg, dbeta, dS0

@@ -1,0 +1,132 @@
+/*
+ * kda.h -- C ABI of the B200 (sm_100a) Kimi Delta Attention (KDA) library
+ * (libkda.so).
+ *
+ * The recurrence (per batch b and value head hv, for t = 0 .. T-1):
+ *
+ *     S_dec = exp(g_t) (.) S_{t-1}            decay, exp(g_t) broadcast along V
+ *     r_t   = v_t - k_t^T S_dec               delta-rule residual
+ *     S_t   = S_dec + (beta_t k_t) (x) r_t    rank-1 write
+ *     o_t   = (scale q_t)^T S_t               readout after the write
+ *
+ * Defined by "K3/kda/ops/reference/recurrent.py" (naive_kda_fwd and the
+ * module docstring), restated step by step in "K3/notes/sections/sec-01.tex"
+ * (section "KDA recurrence core", the four-step update), and for one decode
+ * token by "kimi_k3_host/kda.rs" (kda_recurrent_step).  Value head hv reads
+ * query/key head hv / (HV / H) (repeat-interleave of the head axis).
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are caller-owned DEVICE pointers to dense row-major
+ *     arrays with the stated shapes.  The library never frees or retains them.
+ *   - dtype selects the element type of q, k, v, o, dO, dq, dk, dv:
+ *     KDA_DTYPE_FP32 (float) or KDA_DTYPE_BF16 (bfloat16).  g, beta, states
+ *     and their gradients are always float.
+ *   - g is the log-space per-channel decay (both gates of the host model give
+ *     g <= 0); beta is the write strength after the sigmoid, in (0, 1).
+ *   - scale multiplies q; it must be finite and > 0 (the usual 1/sqrt(K) is
+ *     the caller's choice).
+ *   - K and V must each be 32, 64 or 128; HV must be a multiple of H.
+ *   - stream is a cudaStream_t (NULL = the legacy default stream).  Every
+ *     call only enqueues work on it and returns; results are ready when the
+ *     stream reaches that point.
+ *   - Return value: KDA_OK (0) or one of the KDA_ERR_* codes below; the
+ *     arguments are validated before anything is enqueued, so a non-zero
+ *     return from validation leaves all buffers untouched.  kda_last_error()
+ *     returns a message for the calling thread's most recent failure.
+ *   - The library allocates no device memory; the backward takes its scratch
+ *     from the caller's workspace.
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  KDA_OK = 0,
+  KDA_ERR_NULL = 1,        /* a required pointer is NULL */
+  KDA_ERR_SHAPE = 2,       /* a size is < 1, HV % H != 0, or a grid limit is exceeded */
+  KDA_ERR_DTYPE = 3,       /* dtype is not KDA_DTYPE_FP32 / KDA_DTYPE_BF16 */
+  KDA_ERR_UNSUPPORTED = 4, /* K or V not in {32, 64, 128} */
+  KDA_ERR_WORKSPACE = 5,   /* workspace missing or smaller than required */
+  KDA_ERR_CUDA = 6,        /* a CUDA call failed (launch or attribute) */
+  KDA_ERR_ARG = 7,         /* scale not finite/positive, misaligned pointer, bad flags */
+};
+
+enum { KDA_DTYPE_FP32 = 0, KDA_DTYPE_BF16 = 1 };
+
+/* Flags of kda_bwd. */
+enum {
+  /* The first kda_fwd_workspace_bytes() bytes of the workspace already hold
+   * the chunk states written by kda_fwd on the same inputs (same q, k, v, g,
+   * beta, S0, scale and sizes); kda_bwd then skips its own state pass. */
+  KDA_BWD_STATES_FROM_FWD = 1,
+};
+
+/* Message for the calling thread's most recent non-zero return ("" if none).
+ * The pointer stays valid until the next call from the same thread. */
+const char* kda_last_error(void);
+
+/* Bytes of the optional kda_fwd workspace: the fp32 state entering every
+ * chunk, laid out [B, HV, ceil(T / chunk), K, V]; 0 if a size is invalid. */
+size_t kda_fwd_workspace_bytes(int B, int T, int HV, int K, int V);
+
+/* Bytes kda_bwd needs: the chunk states, the gradients of the state leaving
+ * every chunk (same layout), and, when HV > H, fp32 per-value-head partials
+ * of dq and dk [B, T, HV, K] each; 0 if a size is invalid. */
+size_t kda_bwd_workspace_bytes(int B, int T, int H, int HV, int K, int V);
+
+/* Chunk-parallel prefill forward ("recurrent.py", naive_kda_fwd; the chunk
+ * form is the triangular-solve algebra of "research_layers.py",
+ * delta_recurrence).
+ *   q, k  [B, T, H, K]   dtype      v   [B, T, HV, V] dtype
+ *   g     [B, T, HV, K]  float      beta [B, T, HV]   float
+ *   S0    [B, HV, K, V]  float, or NULL for a zero initial state
+ *   o     [B, T, HV, V]  dtype (output)
+ *   S_T   [B, HV, K, V]  float (output), or NULL to skip the final state
+ *   workspace: NULL, or at least kda_fwd_workspace_bytes(B, T, HV, K, V)
+ *     bytes, 16-byte aligned; when given, the state entering every chunk is
+ *     stored there for a later kda_bwd with KDA_BWD_STATES_FROM_FWD.
+ * o and S_T must not alias any input.  S_T may alias S0 only if S0 is not
+ * needed afterwards (S0 is read before S_T is written, per value column). */
+int kda_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+            const float* S0, float scale, int B, int T, int H, int HV, int K, int V, int dtype,
+            void* o, float* S_T, void* workspace, size_t workspace_bytes, void* stream);
+
+/* One decode token on a state updated IN PLACE ("kimi_k3_host/kda.rs",
+ * kda_recurrent_step, with the q/k L2 normalisation and the sigmoid of beta
+ * left to the caller).
+ *   q, k  [B, H, K]   dtype      v    [B, HV, V] dtype
+ *   g     [B, HV, K]  float      beta [B, HV]    float
+ *   S     [B, HV, K, V] float, read and overwritten with the new state;
+ *         16-byte aligned
+ *   o     [B, HV, V]  dtype (output) */
+int kda_decode_step(const void* q, const void* k, const void* v, const float* g,
+                    const float* beta, float* S, float scale, int B, int H, int HV, int K, int V,
+                    int dtype, void* o, void* stream);
+
+/* Backward of kda_fwd ("recurrent.py", KDAFunction.backward), returning
+ * also the gradient of the initial state.
+ *   inputs as kda_fwd; dO [B, T, HV, V] dtype; dS_T [B, HV, K, V] float or
+ *   NULL (zero upstream gradient of the final state)
+ *   dq, dk [B, T, H, K] dtype; dv [B, T, HV, V] dtype (grouped heads summed)
+ *   dg [B, T, HV, K] float; dbeta [B, T, HV] float
+ *   dS0 [B, HV, K, V] float, or NULL to skip it
+ *   workspace: at least kda_bwd_workspace_bytes(B, T, H, HV, K, V) bytes,
+ *     16-byte aligned, reused as scratch (contents on return are unspecified
+ *     except that the chunk states stay valid).
+ *   flags: 0 or KDA_BWD_STATES_FROM_FWD. */
+int kda_bwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+            const float* S0, const void* dO, const float* dS_T, float scale, int B, int T, int H,
+            int HV, int K, int V, int dtype, void* dq, void* dk, void* dv, float* dg,
+            float* dbeta, float* dS0, void* workspace, size_t workspace_bytes, int flags,
+            void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H_ */

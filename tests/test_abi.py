@@ -1,0 +1,112 @@
+"""CPU checks of the C ABI: the library loads, exports every entry point that
+include/kda.h declares, sizes its workspaces as documented, and rejects bad
+arguments before it touches a GPU (no compute call is made here)."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from gated_delta_rule_66_b200 import build as kbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kda.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    kbuild.build()
+    from gated_delta_rule_66_b200 import kda
+    return kda.library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kda_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("kda_fwd", "kda_decode_step", "kda_bwd", "kda_fwd_workspace_bytes",
+              "kda_bwd_workspace_bytes", "kda_last_error"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+
+
+def test_workspace_sizes(lib):
+    B, T, H, HV, K, V = 2, 100, 2, 6, 64, 32
+    NT = (T + 31) // 32
+    states = B * HV * NT * K * V * 4
+    assert lib.kda_fwd_workspace_bytes(B, T, HV, K, V) == states
+    assert lib.kda_bwd_workspace_bytes(B, T, H, HV, K, V) == 2 * states + 2 * B * T * HV * K * 4
+    assert lib.kda_bwd_workspace_bytes(B, T, HV, HV, K, V) == 2 * states
+    assert lib.kda_fwd_workspace_bytes(0, T, HV, K, V) == 0
+    assert lib.kda_bwd_workspace_bytes(B, T, 4, HV, K, V) == 0   # HV % H != 0
+
+
+FAKE = ctypes.c_void_p(0x1000)  # never dereferenced: validation fails first
+
+
+def fwd_call(lib, **over):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, S0=None, scale=0.5, B=1, T=8, H=1, HV=2,
+             K=32, V=32, dtype=0, o=FAKE, S_T=None, ws=None, ws_bytes=0, stream=None)
+    a.update(over)
+    return lib.kda_fwd(a["q"], a["k"], a["v"], a["g"], a["beta"], a["S0"], a["scale"], a["B"],
+                       a["T"], a["H"], a["HV"], a["K"], a["V"], a["dtype"], a["o"], a["S_T"],
+                       a["ws"], a["ws_bytes"], a["stream"])
+
+
+@pytest.mark.parametrize("over,code,needle", [
+    (dict(T=0), 2, "sizes"),
+    (dict(B=-1), 2, "sizes"),
+    (dict(H=4, HV=6), 2, "multiple"),
+    (dict(K=48), 4, "K=48"),
+    (dict(V=256), 4, "V=256"),
+    (dict(dtype=2), 3, "dtype"),
+    (dict(scale=0.0), 7, "scale"),
+    (dict(scale=float("nan")), 7, "scale"),
+    (dict(q=None), 1, "non-NULL"),
+    (dict(o=None), 1, "non-NULL"),
+    (dict(ws=FAKE, ws_bytes=16), 5, "workspace"),
+    (dict(ws=ctypes.c_void_p(0x1004), ws_bytes=1 << 30), 7, "aligned"),
+    (dict(B=70000), 2, "65535"),
+])
+def test_fwd_rejects_bad_arguments(lib, over, code, needle):
+    assert fwd_call(lib, **over) == code
+    assert needle in lib.kda_last_error().decode()
+
+
+def test_decode_rejects_bad_arguments(lib):
+    rc = lib.kda_decode_step(FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.c_void_p(0x1008), 0.5, 1, 1, 1,
+                             32, 32, 0, FAKE, None)
+    assert rc == 7 and "aligned" in lib.kda_last_error().decode()
+    rc = lib.kda_decode_step(FAKE, FAKE, FAKE, FAKE, FAKE, None, 0.5, 1, 1, 1, 32, 32, 0, FAKE, None)
+    assert rc == 1
+    rc = lib.kda_decode_step(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0.5, 1, 1, 1, 32, 96, 0, FAKE, None)
+    assert rc == 4
+
+
+def test_bwd_rejects_bad_arguments(lib):
+    args = [FAKE] * 5 + [None, FAKE, None, 0.5, 1, 8, 1, 1, 32, 32, 0] + [FAKE] * 5 + [None]
+    rc = lib.kda_bwd(*args, None, 0, 0, None)
+    assert rc == 5 and "workspace" in lib.kda_last_error().decode()
+    rc = lib.kda_bwd(*args, FAKE, 1 << 40, 2, None)
+    assert rc == 7 and "flags" in lib.kda_last_error().decode()
+    bad = list(args)
+    bad[6] = None  # dO
+    rc = lib.kda_bwd(*bad, FAKE, 1 << 40, 0, None)
+    assert rc == 1
+
+
+def test_last_error_clears_on_next_call(lib):
+    fwd_call(lib, T=0)
+    assert lib.kda_last_error().decode() != ""
+    fwd_call(lib, K=48)
+    assert "K=48" in lib.kda_last_error().decode()

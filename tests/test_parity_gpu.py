@@ -1,0 +1,266 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle.
+
+Every case draws its inputs with the seeded generator, runs the library on
+the GPU, upcasts the exact bits it consumed to float64, runs the oracle on
+them, and compares whole tensors by relative L2 (1e-5 for fp32 inputs,
+2e-3 for bf16 inputs).  Full-size workloads are checked on a seeded subset
+of whole grouped-query blocks (or batch rows for decode).
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gated_delta_rule_66_b200.inputs import BY_NAME, head_subset, make_inputs
+from kda_testlib import f64, rel_l2, report, to_cuda, tol_for
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def kda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    import gated_delta_rule_66_b200 as pkg
+    from gated_delta_rule_66_b200 import kda as mod
+    return mod
+
+
+def run_fwd(kda, inp, scale):
+    d = to_cuda(inp)
+    o, S = kda.fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], scale=scale, initial_state=d["S0"])
+    torch.cuda.synchronize()
+    return o, S
+
+
+def oracle_fwd(inp, scale):
+    return oracle.kda_forward(f64(inp["q"]), f64(inp["k"]), f64(inp["v"]), f64(inp["g"]),
+                              f64(inp["beta"]), scale, f64(inp["S0"]))
+
+
+def check_fwd(kda, inp, scale, dtype, label):
+    o, S = run_fwd(kda, inp, scale)
+    o_ref, S_ref = oracle_fwd(inp, scale)
+    tol = tol_for(dtype)
+    report(f"{label} o", f64(o), o_ref, tol, dtype)
+    report(f"{label} S_T", f64(S), S_ref, tol, torch.float32)
+
+
+# ----------------------------------------------------------------------------- forward
+
+def test_fwd_tiny_workload(kda):
+    w = BY_NAME["tiny"]
+    check_fwd(kda, make_inputs(w), w.scale, w.torch_dtype, "tiny")
+
+
+def test_fwd_twin_workload(kda):
+    w = BY_NAME["twin"]
+    check_fwd(kda, make_inputs(w), w.scale, w.torch_dtype, "twin")
+
+
+FWD_CASES = [
+    # name, base workload, overrides
+    ("T1", "tiny", dict(T=1)),
+    ("T31", "tiny", dict(T=31)),
+    ("T33_s0", "twin", dict(B=1, T=33, H=2, HV=2)),
+    ("K64V64_gqa_ragged", "twin", dict(B=2, T=77, H=2, HV=4, K=64, V=64)),
+    ("K32V128", "twin", dict(B=1, T=70, H=1, HV=2, K=32, V=128)),
+    ("K128V32_bf16", "prefill_gqa", dict(T=90, H=1, HV=3, K=128, V=32)),
+    ("K128_bf16_gqa", "prefill_gqa", dict(T=200, H=2, HV=6)),
+    ("K128_fp32", "prefill_gqa", dict(T=100, H=1, HV=2, dtype="fp32", s0_std=0.02)),
+    ("K64V128_bf16", "fwdbwd", dict(B=1, T=65, H=2, HV=2, K=64, V=128, path="fwd")),
+]
+
+
+@pytest.mark.parametrize("name,base,over", FWD_CASES, ids=[c[0] for c in FWD_CASES])
+def test_fwd_shapes(kda, name, base, over):
+    w = BY_NAME[base].with_sizes(**over)
+    check_fwd(kda, make_inputs(w), w.scale, w.torch_dtype, name)
+
+
+def test_fwd_strong_unbounded_decay(kda):
+    """Very strong decays (|g| up to 40 per step) take the pair-by-pair path
+    for diagonal blocks; results stay finite and match."""
+    w = BY_NAME["twin"].with_sizes(B=1, T=96, H=1, HV=2, K=32, V=32)
+    inp = make_inputs(w)
+    inp["g"] = inp["g"] * 20.0
+    check_fwd(kda, inp, w.scale, w.torch_dtype, "strong_decay")
+
+
+def test_fwd_prefill_gqa_full_size(kda):
+    """Production-head GQA prefill (B=1, H=16 -> HV=96, T=8192, K=V=128,
+    bf16) on the GPU in full; the oracle checks grouped-query block 5."""
+    w = BY_NAME["prefill_gqa"]
+    inp = make_inputs(w)
+    o, S = run_fwd(kda, inp, w.scale)
+    sub, hv_idx = head_subset(inp, w.H, w.HV, [5])
+    o_ref, S_ref = oracle_fwd(sub, w.scale)
+    report("prefill_gqa o[group 5]", f64(o[:, :, hv_idx]), o_ref, tol_for(w.torch_dtype), w.torch_dtype)
+    report("prefill_gqa S_T[group 5]", f64(S[:, hv_idx]), S_ref, tol_for(w.torch_dtype), torch.float32)
+    assert torch.isfinite(o.float()).all() and torch.isfinite(S).all()
+
+
+def test_fwd_split_time_state_passing(kda):
+    w = BY_NAME["prefill_gqa"].with_sizes(T=150, H=2, HV=4)
+    inp = to_cuda(make_inputs(w))
+    o, S = kda.fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], scale=w.scale)
+    T1 = 70
+    sl = lambda x, a, b: x[:, a:b].contiguous()
+    oa, Sa = kda.fwd(*(sl(inp[n], 0, T1) for n in ("q", "k", "v", "g", "beta")), scale=w.scale)
+    ob, Sb = kda.fwd(*(sl(inp[n], T1, 150) for n in ("q", "k", "v", "g", "beta")), scale=w.scale,
+                     initial_state=Sa)
+    assert rel_l2(f64(torch.cat([oa, ob], 1)), f64(o)) < 2e-3
+    assert rel_l2(f64(Sb), f64(S)) < 1e-5
+
+
+def test_fwd_deterministic(kda):
+    w = BY_NAME["prefill_gqa"].with_sizes(T=100, H=2, HV=4)
+    inp = make_inputs(w)
+    o1, S1 = run_fwd(kda, inp, w.scale)
+    o2, S2 = run_fwd(kda, inp, w.scale)
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
+
+
+# ----------------------------------------------------------------------------- backward
+
+def run_bwd(kda, inp, scale, dS_T=None, reuse=False):
+    d = to_cuda(inp)
+    ws = None
+    if reuse:
+        B, T, H, K = d["q"].shape
+        HV, V = d["v"].shape[2], d["v"].shape[3]
+        ws = torch.empty(kda.workspace_bytes("bwd", B, T, H, HV, K, V), dtype=torch.uint8, device="cuda")
+        kda.fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], scale=scale, initial_state=d["S0"],
+                workspace=ws)
+    grads = kda.bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["dO"], scale=scale,
+                    initial_state=d["S0"], dS_T=None if dS_T is None else dS_T.cuda(),
+                    workspace=ws, states_from_fwd=reuse)
+    torch.cuda.synchronize()
+    return grads
+
+
+def oracle_bwd(inp, scale, dS_T=None):
+    return oracle.kda_backward(f64(inp["q"]), f64(inp["k"]), f64(inp["v"]), f64(inp["g"]),
+                               f64(inp["beta"]), scale, f64(inp["S0"]), f64(inp["dO"]),
+                               None if dS_T is None else f64(dS_T))
+
+
+GRAD_NAMES = ("dq", "dk", "dv", "dg", "dbeta", "dS0")
+
+
+def check_bwd(kda, inp, scale, dtype, label, dS_T=None, reuse=False):
+    got = run_bwd(kda, inp, scale, dS_T, reuse)
+    ref = oracle_bwd(inp, scale, dS_T)
+    tol = tol_for(dtype)
+    for n, x, r in zip(GRAD_NAMES, got, ref):
+        out_dtype = dtype if n in ("dq", "dk", "dv") else torch.float32
+        report(f"{label} {n}", f64(x), r, tol, out_dtype)
+
+
+BWD_CASES = [
+    ("fp32_K32_s0_dST", "twin", dict(B=1, T=70, H=1, HV=2)),
+    ("fp32_K64_gqa", "twin", dict(B=2, T=64, H=1, HV=3, K=64, V=64)),
+    ("bf16_K128_gqa_ragged", "prefill_gqa", dict(T=45, H=2, HV=4)),
+    ("bf16_K128", "fwdbwd", dict(B=1, T=130, H=2, HV=2)),
+    ("fp32_K128V32", "fwdbwd", dict(B=1, T=40, H=1, HV=1, V=32, dtype="fp32", s0_std=0.05)),
+]
+
+
+@pytest.mark.parametrize("name,base,over", BWD_CASES, ids=[c[0] for c in BWD_CASES])
+def test_bwd_shapes(kda, name, base, over):
+    w = BY_NAME[base].with_sizes(**over)
+    inp = make_inputs(w, with_do=True)
+    dS_T = None
+    if "dST" in name:
+        dS_T = torch.randn(w.B, w.HV, w.K, w.V, generator=torch.Generator().manual_seed(5))
+    check_bwd(kda, inp, w.scale, w.torch_dtype, name, dS_T)
+
+
+def test_bwd_reuses_forward_states(kda):
+    w = BY_NAME["fwdbwd"].with_sizes(B=1, T=100, H=2, HV=2)
+    inp = make_inputs(w, with_do=True)
+    a = run_bwd(kda, inp, w.scale, reuse=False)
+    b = run_bwd(kda, inp, w.scale, reuse=True)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
+def test_fwdbwd_full_size(kda):
+    """Production fwd+bwd (B=2, H=HV=96, T=4096, K=V=128, bf16) on the GPU in
+    full; the oracle checks value heads 17 and 60 of both batch rows."""
+    w = BY_NAME["fwdbwd"]
+    inp = make_inputs(w)
+    d = to_cuda(inp)
+    o, S = kda.fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], scale=w.scale, initial_state=d["S0"])
+    grads = kda.bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["dO"], scale=w.scale,
+                    initial_state=d["S0"])
+    torch.cuda.synchronize()
+    sub, hv_idx = head_subset(inp, w.H, w.HV, [17, 60])
+    o_ref, S_ref = oracle_fwd(sub, w.scale)
+    tol = tol_for(w.torch_dtype)
+    report("fwdbwd o", f64(o[:, :, hv_idx]), o_ref, tol, w.torch_dtype)
+    report("fwdbwd S_T", f64(S[:, hv_idx]), S_ref, tol, torch.float32)
+    ref = oracle_bwd(sub, w.scale)
+    sel = {"dq": lambda x: x[:, :, [17, 60]], "dk": lambda x: x[:, :, [17, 60]],
+           "dv": lambda x: x[:, :, hv_idx], "dg": lambda x: x[:, :, hv_idx],
+           "dbeta": lambda x: x[:, :, hv_idx], "dS0": lambda x: x[:, hv_idx]}
+    for n, x, r in zip(GRAD_NAMES, grads, ref):
+        out_dtype = w.torch_dtype if n in ("dq", "dk", "dv") else torch.float32
+        report(f"fwdbwd {n}", f64(sel[n](x)), r, tol, out_dtype)
+    for x in grads:
+        assert torch.isfinite(x.float()).all()
+
+
+# ----------------------------------------------------------------------------- decode
+
+def check_decode(kda, inp, scale, dtype, label, rows=None):
+    d = to_cuda(inp)
+    S = d["S"].clone()
+    o = kda.decode_step(d["q"], d["k"], d["v"], d["g"], d["beta"], S, scale=scale)
+    torch.cuda.synchronize()
+    sel = slice(None) if rows is None else rows
+    sub = {n: inp[n][sel] for n in ("q", "k", "v", "g", "beta", "S")}
+    o_ref, S_ref = oracle.kda_decode_step(f64(sub["q"]), f64(sub["k"]), f64(sub["v"]), f64(sub["g"]),
+                                          f64(sub["beta"]), f64(sub["S"]), scale)
+    tol = tol_for(dtype)
+    report(f"{label} o", f64(o[sel]), o_ref, tol, dtype)
+    report(f"{label} S", f64(S[sel]), S_ref, tol, torch.float32)
+
+
+def test_decode_full_size(kda):
+    """Batched decode (B=256, HV=96, K=V=128, bf16 inputs, fp32 state, in
+    place); the oracle checks batch rows 0, 131 and 255."""
+    w = BY_NAME["decode"]
+    check_decode(kda, make_inputs(w), w.scale, w.torch_dtype, "decode", rows=[0, 131, 255])
+
+
+DEC_CASES = [
+    ("K32V32_fp32", dict(B=3, H=2, HV=4, K=32, V=32, dtype="fp32")),
+    ("K64V128_bf16", dict(B=2, H=1, HV=3, K=64, V=128)),
+    ("K128V64_fp32_gqa", dict(B=2, H=2, HV=6, K=128, V=64, dtype="fp32")),
+    ("K32V128_bf16", dict(B=5, H=4, HV=4, K=32, V=128)),
+]
+
+
+@pytest.mark.parametrize("name,over", DEC_CASES, ids=[c[0] for c in DEC_CASES])
+def test_decode_shapes(kda, name, over):
+    w = BY_NAME["decode"].with_sizes(**over)
+    check_decode(kda, make_inputs(w), w.scale, w.torch_dtype, name)
+
+
+def test_decode_sequence_equals_prefill(kda):
+    """T decode steps from S0 equal one prefill over the same T tokens."""
+    w = BY_NAME["prefill_gqa"].with_sizes(T=40, H=2, HV=4, dtype="fp32", s0_std=0.02)
+    inp = to_cuda(make_inputs(w))
+    o, S = kda.fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], scale=w.scale,
+                   initial_state=inp["S0"])
+    St = inp["S0"].clone()
+    outs = []
+    for t in range(w.T):
+        outs.append(kda.decode_step(*(inp[n][:, t].contiguous() for n in ("q", "k", "v", "g", "beta")),
+                                    St, scale=w.scale))
+    torch.cuda.synchronize()
+    assert rel_l2(f64(torch.stack(outs, 1)), f64(o)) < 1e-5
+    assert rel_l2(f64(St), f64(S)) < 1e-5
