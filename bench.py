@@ -363,6 +363,12 @@ def _oracle_head(job):
     return time.perf_counter() - t0
 
 
+def _warm(_):
+    sys.path.insert(0, ROOT)
+    import oracle  # noqa: F401
+    return 0
+
+
 def cpu_baseline(w, budget_s=20.0):
     """Times the oracle on a bounded sample of workload ``w`` on the host's
     cores: whole value heads (one per worker process) over the first T_s
@@ -394,11 +400,14 @@ def cpu_baseline(w, budget_s=20.0):
                       None if inp["S0"] is None else f64(inp["S0"][:, hv:hv + 1]),
                       None if inp.get("dO") is None else f64(inp["dO"][:, :, hv:hv + 1]))
         jobs.append((w.path, arrays, w.scale))
+    for var in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS"):
+        os.environ[var] = "1"   # one thread per worker: `cores` threads in total
     ctx = mp.get_context("spawn")
-    t0 = time.perf_counter()
     with ctx.Pool(processes=cores) as pool:
+        pool.map(_warm, range(cores))          # worker start-up stays outside the timing
+        t0 = time.perf_counter()
         pool.map(_oracle_head, jobs)
-    elapsed = time.perf_counter() - t0
+        elapsed = time.perf_counter() - t0
     head_tokens = nheads * T_s
     tokens_per_s = head_tokens / w.HV / elapsed
     return {"value": tokens_per_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
