@@ -125,6 +125,31 @@ int kda_bwd(const void* q, const void* k, const void* v, const float* g, const f
             float* dbeta, float* dS0, void* workspace, size_t workspace_bytes, int flags,
             void* stream);
 
+/* Size in bytes of the fixed device array that kda_bwd_noalloc uses as its
+ * scratch (64 MiB, held on every GPU that loads the library until exit). */
+#define KDA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+
+/* kda_bwd for callers that cannot allocate device memory: a plugin whose host
+ * framework owns all device memory and gives it no workspace, or a running
+ * loop that forbids allocator calls (cudaMalloc/cudaFree synchronise the
+ * device and fail once another allocator has reserved the memory).  The paper
+ * has no counterpart to this entry point; it is a deployment convenience.
+ *   Arguments, layouts and results are those of kda_bwd (flags = 0); the
+ *   caller still owns every input and output.  The scratch is a file-scope
+ *   __device__ array of KDA_NOALLOC_SCRATCH_BYTES; a problem whose
+ *   kda_bwd_workspace_bytes() exceeds it returns KDA_ERR_WORKSPACE with a
+ *   message and enqueues nothing.  Nothing is allocated: the first call on a
+ *   device looks up the array's device address (cudaGetSymbolAddress) with
+ *   that device current and caches it, so make that first call before any
+ *   stream capture.  All calls share the one array: calls whose work overlaps
+ *   on the GPU (other streams or threads on the same device) race and must be
+ *   ordered by the caller.  Each call writes every scratch byte it reads, so
+ *   stale contents from an earlier call are never used. */
+int kda_bwd_noalloc(const void* q, const void* k, const void* v, const float* g,
+                    const float* beta, const float* S0, const void* dO, const float* dS_T,
+                    float scale, int B, int T, int H, int HV, int K, int V, int dtype, void* dq,
+                    void* dk, void* dv, float* dg, float* dbeta, float* dS0, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
