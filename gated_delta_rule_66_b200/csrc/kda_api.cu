@@ -70,6 +70,11 @@ extern "C" {
 
 const char* kda_last_error(void) { return g_err; }
 
+int kda_device_status(unsigned* flags) {
+  if (!flags) return set_error(KDA_ERR_NULL, "kda_device_status: flags must be non-NULL");
+  return take_device_error(flags);
+}
+
 size_t kda_fwd_workspace_bytes(int B, int T, int HV, int K, int V) {
   if (B < 1 || T < 1 || HV < 1 || K < 1 || V < 1) return 0;
   return states_bytes(B, T, HV, K, V);

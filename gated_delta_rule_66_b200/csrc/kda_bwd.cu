@@ -468,7 +468,10 @@ template <int K, typename TIn>
 static int launch_bwd_t(const BwdArgs& a, cudaStream_t stream) {
   constexpr int C = FWD_CHUNK, VB = FWD_VBLOCK;
   const int NT = (a.T + C - 1) / C;
-  {
+  if (bwd_tc_eligible(a, sizeof(TIn) == 2 ? 1 : 0)) {
+    const int rc = launch_bwd_dstate_tc(a, stream);
+    if (rc) return rc;
+  } else {
     using S = DstSmem<K, C, VB>;
     auto kern = kda_bwd_dstate_kernel<K, C, VB, TIn>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::bytes);

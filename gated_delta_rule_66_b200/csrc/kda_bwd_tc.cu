@@ -1,0 +1,267 @@
+// Tensor-core (tcgen05) reverse pass of the KDA backward for K = V = 128,
+// bf16 q/k/dO, fp32 g/beta: the gradient of the state leaving every 32-step
+// block, and dS0.
+//
+// From the chunk algebra (kda_tc_chunk.cuh) the gradient of the state entering
+// a chunk, given the gradient dM of the state leaving it, is
+//   dU  = P^T dO + (K o e^{c_last - c}) dM
+//   dX  = diag(beta) T^T dU
+//   dM_in = diag(e^{c_last}) dM + (Q~ o e^c)^T dO - (K o e^c)^T dX
+// ("recurrent.py", KDAFunction.backward, taken a chunk at a time; dM needs no
+// forward state).  One CTA per (b, hv) walks the chunks in reverse with dM^T
+// held in TMEM (lane = value column n, column = key channel f):
+//   dU^T  = dO^T P + dM^T (K o e^{c_last-c})^T      (A = dO^T or dM^T, both in TMEM)
+//   dX^T  = dU^T (diag(beta) T^T)^T
+//   dM_in^T = dM^T diag(e^{c_last}) + dO^T (Q~ o e^c) - dX^T (K o e^c)
+// The state gradient at the chunk's midpoint (leaving step 31), needed for the
+// 32-step granularity of the per-chunk gradient kernel, is the same formula
+// over the second half alone:
+//   dM_mid^T = dM^T diag(e^{c_last - c_31}) + dO^T[:,32:] (Q~ o e^{c-c_31})[32:]
+//              - dX^T[:,32:] (K o e^{c-c_31})[32:].
+#include <cuda_bf16.h>
+
+#include "kda_internal.h"
+#include "kda_tc_chunk.cuh"
+
+namespace kda {
+
+extern __device__ unsigned int g_kda_device_error;
+
+namespace tcb {
+using namespace tcc;
+constexpr uint32_t OP_KED = OP, OP_QET = OP + 32768, OP_NKET = OP + 65536, OP_Q2T = OP + 98304,
+                   OP_NK2T = OP + 114688;
+constexpr uint32_t TM_S = 0, TM_DU = 128, TM_DX = 192, TM_DOT = 256, TM_APA = 320, TM_APB = 384,
+                   TM_MID = 384;  // mid-chunk gradient (the interaction tile is read by then)
+}  // namespace tcb
+
+__global__ void __launch_bounds__(256, 1) kda_bwd_dstate_tc_kernel(BwdArgs a) {
+  using namespace tcb;
+  using namespace tc;
+  extern __shared__ __align__(1024) unsigned char sm[];
+  Ctx cx;
+  cx.sm = sm;
+  cx.sb = smem_u32(sm);
+  cx.tid = threadIdx.x;
+  cx.warp = cx.tid >> 5;
+  cx.lane = cx.tid & 31;
+  cx.sub = cx.warp & 3;
+  cx.hcol = cx.warp >> 2;
+  cx.Lr = cx.sub * 32 + cx.lane;
+  cx.lo = (uint32_t)(cx.sub * 32) << 16;
+  const int tid = cx.tid, hcol = cx.hcol, Lr = cx.Lr;
+  const uint32_t lo = cx.lo, sb = cx.sb;
+
+  const int hv = blockIdx.x, b = blockIdx.y;
+  const int G = a.HV / a.H, h = hv / G, T = a.T, NT = (T + C - 1) / C, NT32 = (T + 31) / 32;
+  const size_t head = (size_t)b * a.HV + hv;
+  const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(a.q);
+  const __nv_bfloat16* kg = static_cast<const __nv_bfloat16*>(a.k);
+  const __nv_bfloat16* dog = static_cast<const __nv_bfloat16*>(a.dO);
+  float* sBeta = cx.beta();
+  float* sEl = reinterpret_cast<float*>(sm + S_EL);
+  float* sEh = reinterpret_cast<float*>(sm + S_EMID);  // e^{c_last - c_31}
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + S_BAR);
+  uint32_t* sTm = reinterpret_cast<uint32_t*>(sm + S_TMEM);
+  const float* sC = cx.c();
+
+  if (cx.warp == 0) tmem_alloc(sTm, 512);
+  if (tid == 0) mbar_init(bar, 1);
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tm = *sTm;
+  cx.tm = tm;
+  uint32_t phase = 0;
+  bool failed = false;
+
+  {  // gradient of the final state, transposed
+    for (int cb = 0; cb < 2; ++cb) {
+      const int f0 = hcol * 64 + cb * 32;
+      uint32_t r[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        r[j] = __float_as_uint(a.dS_T ? a.dS_T[(head * KD + f0 + j) * VD + Lr] : 0.f);
+      tmem_st32(tm + lo + TM_S + f0, r);
+    }
+    tmem_wait_st();
+  }
+  fence_before();
+  __syncthreads();
+
+  for (int ch = NT - 1; ch >= 0; --ch) {
+    const int t0 = ch * C, L = min(C, T - t0);
+    load_raw(cx, qg, kg, dog, a.g, a.beta, b, T, t0, L, a.H, a.HV, h, hv);
+    const bool wide = cumsum_span(cx);
+    build_op1_and_issue(cx, a.scale, tm + TM_APA, tm + TM_APB, bar);
+    if (!wait_mma(bar, phase)) { failed = true; break; }
+
+    // ---------------------------------------------------------------- operands of the gradient products
+    const int fq = item_f(cx);
+    {
+      const float4 c63v = ld4(sC + 63 * LDCF + fq), r31 = ld4(sC + 31 * LDCF + fq);
+      const float c63[4] = {c63v.x, c63v.y, c63v.z, c63v.w}, c31[4] = {r31.x, r31.y, r31.z, r31.w};
+      for (int m = 0; m < 8; ++m) {
+        const int i = item_row(cx, m);
+        const float4 c4 = ld4(sC + i * LDCF + fq);
+        const float c[4] = {c4.x, c4.y, c4.z, c4.w};
+        float kf[4], qf[4];
+        bf16x4(sm + RAW_K + i * 256 + fq * 2, kf);
+        bf16x4(sm + RAW_Q + i * 256 + fq * 2, qf);
+        float e[4], ed[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          qf[u] *= a.scale;
+          e[u] = ex2(c[u]);
+          ed[u] = ex2(c63[u] - c[u]);
+        }
+        st_tf32x4(sm, OP_KED + kmaj(i, fq, 128), kf[0] * ed[0], kf[1] * ed[1], kf[2] * ed[2], kf[3] * ed[3]);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          st_tf32(sm, OP_QET + kmaj(fq + u, i, 64), qf[u] * e[u]);
+          st_tf32(sm, OP_NKET + kmaj(fq + u, i, 64), -kf[u] * e[u]);
+        }
+        if (i >= 32) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float x2 = ex2(c[u] - c31[u]);
+            st_tf32(sm, OP_Q2T + kmaj(fq + u, i - 32, 32), qf[u] * x2);
+            st_tf32(sm, OP_NK2T + kmaj(fq + u, i - 32, 32), -kf[u] * x2);
+          }
+        }
+      }
+      if (tid < KD) {
+        sEl[tid] = ex2(sC[63 * LDCF + tid]);
+        sEh[tid] = ex2(sC[63 * LDCF + tid] - sC[31 * LDCF + tid]);
+      }
+      // dO^T into TMEM: lane n, columns j
+      {
+        uint32_t r[32];
+        const unsigned char* col = sm + RAW_X + Lr * 2;
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj)
+          r[jj] = tf32_rna(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(col + (hcol * 32 + jj) * 256)));
+        tmem_st32(tm + lo + TM_DOT + hcol * 32, r);
+        tmem_wait_st();
+      }
+    }
+    Pairwise pw;
+    if (wide) pairwise_compute(cx, a.scale, pw);
+    fence_async_smem();
+    fence_before();
+    __syncthreads();  // raw inputs consumed; the raw region is reused below
+
+    readout_ap(cx, tm + TM_APA, tm + TM_APB, true, wide, pw);  // P^T at R_P
+    invert(cx);
+    {  // (diag(beta) T^T)^T as a K-major operand: element (i, j) = beta_i T[j][i]
+      const float* tr = reinterpret_cast<const float*>(sm + R_TROW);
+      for (int x = tid; x < C * 16; x += NTH) {
+        const int i = x >> 4, j4 = (x & 15) * 4;
+        const float bi = sBeta[i];
+        st_tf32x4(sm, R_T + kmaj(i, j4, 64), bi * tr[j4 * 65 + i], bi * tr[(j4 + 1) * 65 + i],
+                  bi * tr[(j4 + 2) * 65 + i], bi * tr[(j4 + 3) * 65 + i]);
+      }
+    }
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 0) {  // dU^T = dO^T P + dM^T (K o e^{c_last-c})^T
+      fence_after();
+      const uint32_t id = idesc_tf32(128, 64);
+      for (int ks = 0; ks < 8; ++ks)
+        mma_ts(tm + TM_DU, tm + TM_DOT + ks * 8, desc(sb + R_P + ks * 256, 2048), id, ks > 0);
+      for (int ks = 0; ks < 16; ++ks)
+        mma_ts(tm + TM_DU, tm + TM_S + ks * 8, desc(sb + OP_KED + ks * 256, 4096), id, 1);
+      commit(bar);
+    }
+    if (!wait_mma(bar, phase)) { failed = true; break; }
+    if (tid == 0) {  // dX^T = dU^T (diag(beta) T^T)^T
+      const uint32_t id = idesc_tf32(128, 64);
+      for (int ks = 0; ks < 8; ++ks)
+        mma_ts(tm + TM_DX, tm + TM_DU + ks * 8, desc(sb + R_T + ks * 256, 2048), id, ks > 0);
+      commit(bar);
+    }
+    if (!wait_mma(bar, phase)) { failed = true; break; }
+
+    // ---------------------------------------------------------------- store dM (leaving this chunk); start dM_in and dM_mid
+    {
+      uint32_t r[32];
+      for (int cb = 0; cb < 2; ++cb) {
+        const int f0 = hcol * 64 + cb * 32;
+        float s[32];
+        tmem_ld32(tm + lo + TM_S + f0, s);
+        if (2 * ch + 1 < NT32) {
+          float* dst = a.dstates + ((head * NT32 + 2 * ch + 1) * KD + f0) * VD + Lr;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) dst[(size_t)j * VD] = s[j];
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(s[j] * sEh[f0 + j]);
+        tmem_st32(tm + lo + TM_MID + f0, r);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(s[j] * sEl[f0 + j]);
+        tmem_st32(tm + lo + TM_S + f0, r);
+      }
+      tmem_wait_st();
+    }
+    fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      fence_after();
+      const uint32_t id = idesc_tf32(128, 128);
+      for (int ks = 0; ks < 8; ++ks) {
+        mma_ts(tm + TM_S, tm + TM_DOT + ks * 8, desc(sb + OP_QET + ks * 256, 2048), id, 1);
+        mma_ts(tm + TM_S, tm + TM_DX + ks * 8, desc(sb + OP_NKET + ks * 256, 2048), id, 1);
+      }
+      for (int ks = 0; ks < 4; ++ks) {
+        mma_ts(tm + TM_MID, tm + TM_DOT + 32 + ks * 8, desc(sb + OP_Q2T + ks * 256, 1024), id, 1);
+        mma_ts(tm + TM_MID, tm + TM_DX + 32 + ks * 8, desc(sb + OP_NK2T + ks * 256, 1024), id, 1);
+      }
+      commit(bar);
+    }
+    if (!wait_mma(bar, phase)) { failed = true; break; }
+    {  // gradient of the state leaving step 31 of this chunk
+      for (int cb = 0; cb < 2; ++cb) {
+        const int f0 = hcol * 64 + cb * 32;
+        float s[32];
+        tmem_ld32(tm + lo + TM_MID + f0, s);
+        float* dst = a.dstates + ((head * NT32 + 2 * ch) * KD + f0) * VD + Lr;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) dst[(size_t)j * VD] = s[j];
+      }
+    }
+    fence_before();
+    __syncthreads();
+  }
+
+  if (!failed && a.dS0) {
+    fence_after();
+    for (int cb = 0; cb < 2; ++cb) {
+      const int f0 = hcol * 64 + cb * 32;
+      float s[32];
+      tmem_ld32(tm + lo + TM_S + f0, s);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) a.dS0[(head * KD + f0 + j) * VD + Lr] = s[j];
+    }
+  }
+  fence_before();
+  __syncthreads();
+  if (cx.warp == 0) tmem_dealloc(tm, 512);
+  if (failed && tid == 0) atomicOr(&g_kda_device_error, 1u);
+}
+
+bool bwd_tc_eligible(const BwdArgs& a, int dtype) {
+  auto al16 = [](const void* p) { return ((uintptr_t)p & 15u) == 0; };
+  return dtype == 1 && a.K == 128 && a.V == 128 && al16(a.q) && al16(a.k) && al16(a.dO) && al16(a.g);
+}
+
+int launch_bwd_dstate_tc(const BwdArgs& a, cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(kda_bwd_dstate_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)tcc::SMEM_BYTES);
+  if (e != cudaSuccess) return set_cuda_error("kda_bwd: cudaFuncSetAttribute", e);
+  kda_bwd_dstate_tc_kernel<<<dim3(a.HV, a.B), tcc::NTH, tcc::SMEM_BYTES, stream>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return set_cuda_error("kda_bwd: tensor-core state-gradient launch", e);
+  return 0;
+}
+
+}  // namespace kda

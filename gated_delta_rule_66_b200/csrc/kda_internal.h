@@ -45,8 +45,13 @@ int set_error(int code, const char* msg);
 int set_cuda_error(const char* where, cudaError_t e);
 
 int launch_fwd(const FwdArgs& a, int dtype, cudaStream_t stream);
+bool fwd_tc_eligible(const FwdArgs& a, int dtype);
+int launch_fwd_tc(const FwdArgs& a, cudaStream_t stream);
+int take_device_error(unsigned* out);
 size_t fwd_smem_bytes(int K);
 int launch_bwd(const BwdArgs& a, int dtype, cudaStream_t stream);
+bool bwd_tc_eligible(const BwdArgs& a, int dtype);
+int launch_bwd_dstate_tc(const BwdArgs& a, cudaStream_t stream);
 int launch_decode(const DecodeArgs& a, int K, int V, int dtype, cudaStream_t stream);
 
 }  // namespace kda

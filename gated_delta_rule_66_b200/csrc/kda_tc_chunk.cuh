@@ -1,0 +1,286 @@
+// Per-chunk building blocks shared by the tensor-core KDA kernels (K = V =
+// 128, chunk C = 64, bf16 q/k/v/dO, fp32 g/beta): loading a chunk, the
+// in-chunk cumulative decay, the interaction products Ah and P on the tensor
+// cores, and their read-out for the triangular solve.
+//
+// Chunk algebra ("research_layers.py", delta_recurrence, erase = write = k,
+// beta folded into the residual): with c_i = sum_{s<=i} g_s inside the chunk,
+//   Ah[i][j] = sum_f k_if k_jf exp(c_if - c_jf)   (j < i)
+//   P [i][j] = sum_f q~_if k_jf exp(c_if - c_jf)  (j <= i),  q~ = scale q.
+// Both come out of two tf32 products of split-exponent operands:
+//   product a: [K o x; Q~ o x] (K o y)^T with x_i = e^{c_i - c_r}, y_j = e^{c_r - c_j}
+//              and r the middle row (15 or 47) of the 32-row half holding i and j;
+//              it gives the two diagonal 32 x 32 blocks;
+//   product b: rows i >= 32 against columns j < 32 with r = 31 (both factors <= 1).
+// When the decay from a half's middle row to either end exceeds 80 (only an
+// unbounded gate can do that) the same-half entries are formed pair by pair.
+//
+// Shared-memory map (bytes):
+//   [0, 82944)       raw chunk: q, k, a third bf16 row tensor (v or dO), and the
+//                    cumulative decay c (log2 units, row stride LDCF floats);
+//                    reused after the raw data is consumed for Ah, T, P and W
+//   [82944, 230400)  operand region: the interaction operands, then the
+//                    kernel's own product operands
+//   [230400, ...)    beta, per-channel decay constants, barrier, TMEM base
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "kda_chunk.cuh"
+#include "kda_tc.cuh"
+
+namespace kda {
+namespace tcc {
+
+constexpr int C = 64, KD = 128, VD = 128, NTH = 256;
+constexpr uint32_t RAW_Q = 0, RAW_K = 16384, RAW_X = 32768, RAW_C = 49152;
+constexpr int LDCF = 132;
+constexpr uint32_t R_AH = 0, R_TROW = 16640, R_SW = 33280, R_P = 37888, R_T = 54272, R_WOP = 0;
+constexpr uint32_t OP = 82944;
+constexpr uint32_t OP_XA = OP, OP_YA = OP + 65536, OP_XB = OP + 98304, OP_YB = OP + 131072;
+constexpr uint32_t SMALL = OP + 147456;
+constexpr uint32_t S_BETA = SMALL, S_EL = SMALL + 256, S_EMID = S_EL + 512, S_CARRY = S_EMID + 512,
+                   S_BAR = S_CARRY + 512, S_TMEM = S_BAR + 8, SMEM_BYTES = S_TMEM + 16;
+constexpr float LOG2E = 1.4426950408889634f;
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+static_assert(R_T + 16384 <= OP && R_P + 16384 <= R_T && R_WOP + 32768 <= R_SW, "raw-region reuse");
+
+struct Ctx {
+  unsigned char* sm;
+  uint32_t sb;      // shared address of sm
+  uint32_t tm;      // TMEM base
+  uint32_t lo;      // this warp's TMEM lane base (<< 16)
+  int tid, warp, lane, sub, hcol, Lr;
+  __device__ float* c() const { return reinterpret_cast<float*>(sm + RAW_C); }
+  __device__ float* beta() const { return reinterpret_cast<float*>(sm + S_BETA); }
+};
+
+__device__ __forceinline__ void st_tf32x4(unsigned char* base, uint32_t off, float a, float b, float c, float d) {
+  uint4 v = make_uint4(tc::tf32_rna(a), tc::tf32_rna(b), tc::tf32_rna(c), tc::tf32_rna(d));
+  *reinterpret_cast<uint4*>(base + off) = v;
+}
+__device__ __forceinline__ void st_tf32(unsigned char* base, uint32_t off, float a) {
+  *reinterpret_cast<uint32_t*>(base + off) = tc::tf32_rna(a);
+}
+__device__ __forceinline__ void bf16x4(const unsigned char* p, float (&o)[4]) {
+  const uint2 r = *reinterpret_cast<const uint2*>(p);
+  const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&r.x);
+  const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&r.y);
+  o[0] = __low2float(lo); o[1] = __high2float(lo); o[2] = __low2float(hi); o[3] = __high2float(hi);
+}
+__device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+
+// Asynchronous load of one chunk: q, k rows of query/key head h, x rows of
+// value head hv (v or dO), g rows and beta; rows past the sequence end are
+// zero.  Completes (wait + barrier) before returning.
+__device__ __forceinline__ void load_raw(const Ctx& c, const __nv_bfloat16* q, const __nv_bfloat16* k,
+                                         const __nv_bfloat16* x, const float* g, const float* beta,
+                                         int b, int T, int t0, int L, int H, int HV, int h, int hv) {
+  using namespace tc;
+  for (int e = c.tid; e < C * 16; e += NTH) {
+    const int i = e >> 4, vec = e & 15;
+    const bool ok = i < L;
+    const size_t t = (size_t)b * T + t0 + (ok ? i : 0);  // row 0 of the chunk is always valid
+    cp_async16(c.sb + RAW_Q + i * 256 + vec * 16, q + (t * H + h) * KD + vec * 8, ok);
+    cp_async16(c.sb + RAW_K + i * 256 + vec * 16, k + (t * H + h) * KD + vec * 8, ok);
+    cp_async16(c.sb + RAW_X + i * 256 + vec * 16, x + (t * HV + hv) * VD + vec * 8, ok);
+  }
+  for (int e = c.tid; e < C * 32; e += NTH) {
+    const int i = e >> 5, vec = e & 31;
+    const bool ok = i < L;
+    const size_t t = (size_t)b * T + t0 + (ok ? i : 0);
+    cp_async16(c.sb + RAW_C + (i * LDCF + vec * 4) * 4, g + (t * HV + hv) * KD + vec * 4, ok);
+  }
+  if (c.tid < C) c.beta()[c.tid] = (c.tid < L) ? beta[((size_t)b * T + t0 + c.tid) * HV + hv] : 0.f;
+  cp_async_wait_all();
+  __syncthreads();
+}
+
+// In-chunk cumulative decay (natural log summed, stored times log2(e)).
+// Returns, block-uniformly, whether some half's decay from its middle row to
+// either end exceeds 80 (the split exponents would then leave fp32 range).
+__device__ __forceinline__ bool cumsum_span(const Ctx& c) {
+  float* sC = c.c();
+  float* sCarry = reinterpret_cast<float*>(c.sm + S_CARRY);
+  const int f = c.tid & 127, hh = c.tid >> 7;
+  float v[32];
+  float run = 0.f;
+#pragma unroll
+  for (int r = 0; r < 32; ++r) {
+    run += sC[(hh * 32 + r) * LDCF + f];
+    v[r] = run;
+  }
+  if (hh == 0) sCarry[f] = run;
+  __syncthreads();
+  const float carry = hh ? sCarry[f] : 0.f;
+#pragma unroll
+  for (int r = 0; r < 32; ++r) sC[(hh * 32 + r) * LDCF + f] = (v[r] + carry) * LOG2E;
+  __syncthreads();
+  bool w = false;
+  if (c.tid < KD) {
+    const float lim = 80.f * LOG2E;
+    const int t = c.tid;
+    const float c0 = sC[t], c15 = sC[15 * LDCF + t], c31 = sC[31 * LDCF + t];
+    const float c32 = sC[32 * LDCF + t], c47 = sC[47 * LDCF + t], c63 = sC[63 * LDCF + t];
+    w = fabsf(c0 - c15) > lim || fabsf(c15 - c31) > lim || fabsf(c32 - c47) > lim || fabsf(c47 - c63) > lim;
+  }
+  return __syncthreads_or(w);
+}
+
+// Item mapping of the element-wise operand builders: thread t owns key
+// channels 4*((t>>3)&31) .. +3 and rows m*8 + (t&7), m = 0..7.
+__device__ __forceinline__ int item_f(const Ctx& c) { return ((c.tid >> 3) & 31) * 4; }
+__device__ __forceinline__ int item_row(const Ctx& c, int m) { return m * 8 + (c.tid & 7); }
+
+// Interaction operands into the operand region, then the two products on
+// the tensor cores (issued by thread 0, completion on `bar`).
+__device__ __forceinline__ void build_op1_and_issue(const Ctx& c, float scale, uint32_t tm_apa,
+                                                    uint32_t tm_apb, uint64_t* bar) {
+  using namespace tc;
+  const float* sC = c.c();
+  const int fq = item_f(c);
+  const float4 r15 = ld4(sC + 15 * LDCF + fq), r47 = ld4(sC + 47 * LDCF + fq), r31 = ld4(sC + 31 * LDCF + fq);
+  const float c31[4] = {r31.x, r31.y, r31.z, r31.w};
+  for (int m = 0; m < 8; ++m) {
+    const int i = item_row(c, m);
+    const float4 c4 = ld4(sC + i * LDCF + fq);
+    const float cc[4] = {c4.x, c4.y, c4.z, c4.w};
+    float kf[4], qf[4];
+    bf16x4(c.sm + RAW_K + i * 256 + fq * 2, kf);
+    bf16x4(c.sm + RAW_Q + i * 256 + fq * 2, qf);
+    const float4 rr = (i < 32) ? r15 : r47;
+    const float cr[4] = {rr.x, rr.y, rr.z, rr.w};
+    float xa[4], ya[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      qf[u] *= scale;
+      xa[u] = ex2(cc[u] - cr[u]);
+      ya[u] = ex2(cr[u] - cc[u]);
+    }
+    st_tf32x4(c.sm, OP_XA + kmaj(i, fq, 128), kf[0] * xa[0], kf[1] * xa[1], kf[2] * xa[2], kf[3] * xa[3]);
+    st_tf32x4(c.sm, OP_XA + kmaj(64 + i, fq, 128), qf[0] * xa[0], qf[1] * xa[1], qf[2] * xa[2], qf[3] * xa[3]);
+    st_tf32x4(c.sm, OP_YA + kmaj(i, fq, 128), kf[0] * ya[0], kf[1] * ya[1], kf[2] * ya[2], kf[3] * ya[3]);
+    if (i >= 32) {
+      float xb[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) xb[u] = ex2(cc[u] - c31[u]);
+      st_tf32x4(c.sm, OP_XB + kmaj(i - 32, fq, 128), kf[0] * xb[0], kf[1] * xb[1], kf[2] * xb[2], kf[3] * xb[3]);
+      st_tf32x4(c.sm, OP_XB + kmaj(i, fq, 128), qf[0] * xb[0], qf[1] * xb[1], qf[2] * xb[2], qf[3] * xb[3]);
+    } else {
+      float yb[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) yb[u] = ex2(c31[u] - cc[u]);
+      st_tf32x4(c.sm, OP_YB + kmaj(i, fq, 128), kf[0] * yb[0], kf[1] * yb[1], kf[2] * yb[2], kf[3] * yb[3]);
+    }
+  }
+  fence_async_smem();
+  __syncthreads();
+  if (c.tid == 0) {
+    fence_after();
+    const uint32_t idA = idesc_tf32(128, 64), idB = idesc_tf32(64, 32);
+    for (int ks = 0; ks < 16; ++ks)
+      mma_ss(tm_apa, desc(c.sb + OP_XA + ks * 256, 4096), desc(c.sb + OP_YA + ks * 256, 4096), idA, ks > 0);
+    for (int ks = 0; ks < 16; ++ks)
+      mma_ss(tm_apb, desc(c.sb + OP_XB + ks * 256, 4096), desc(c.sb + OP_YB + ks * 256, 4096), idB, ks > 0);
+    commit(bar);
+  }
+}
+
+// Waits for the tensor-core work committed to `bar` (phase parity toggled
+// here).  Returns false, block-uniformly, if the bounded wait ran out.
+__device__ __forceinline__ bool wait_mma(uint64_t* bar, uint32_t& phase) {
+  const bool ok = tc::mbar_wait(bar, phase);
+  phase ^= 1;
+  const bool bad = __syncthreads_or(!ok);
+  tc::fence_after();
+  return !bad;
+}
+
+// Same-half Ah/P entries pair by pair (only when cumsum_span said so); must
+// run while the raw chunk is still in shared memory.
+struct Pairwise {
+  float v[16];
+  int kind, i, j0;
+};
+__device__ __forceinline__ void pairwise_compute(const Ctx& c, float scale, Pairwise& pw) {
+  const float* sC = c.c();
+  pw.kind = c.tid >> 7;
+  pw.i = (c.tid >> 1) & 63;
+  pw.j0 = (pw.i & 32) + (c.tid & 1) * 16;
+  const unsigned char* rowi = c.sm + (pw.kind ? RAW_Q : RAW_K) + pw.i * 256;
+  for (int jj = 0; jj < 16; ++jj) {
+    const int j = pw.j0 + jj;
+    float acc = 0.f;
+    if (pw.kind ? (j <= pw.i) : (j < pw.i)) {
+      const unsigned char* rowj = c.sm + RAW_K + j * 256;
+      for (int f = 0; f < KD; ++f) {
+        const float xi = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(rowi + 2 * f));
+        const float kj = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(rowj + 2 * f));
+        acc = fmaf(xi * kj, tc::ex2(sC[pw.i * LDCF + f] - sC[j * LDCF + f]), acc);
+      }
+      if (pw.kind) acc *= scale;
+    }
+    pw.v[jj] = acc;
+  }
+}
+
+// byte offset of P[i][j] in its operand tile: P itself (rows i, K = j) for the
+// forward readout, P^T (rows j, K = i) for the backward
+__device__ __forceinline__ uint32_t p_off(int i, int j, bool transP) {
+  return R_P + (transP ? tc::kmaj(j, i, 64) : tc::kmaj(i, j, 64));
+}
+
+// Reads Ah (row-major, stride 65, at R_AH) and P (tf32 operand at R_P) out of
+// the two interaction products; the raw region must be free.  Ends with a
+// barrier.
+__device__ __forceinline__ void readout_ap(const Ctx& c, uint32_t tm_apa, uint32_t tm_apb, bool transP,
+                                           bool wide, const Pairwise& pw) {
+  using namespace tc;
+  float* sAh = reinterpret_cast<float*>(c.sm + R_AH);
+  {
+    float v[32];
+    tmem_ld32(tm_apa + c.lo + c.hcol * 32, v);
+    const bool isA = c.Lr < 64;
+    const int i = isA ? c.Lr : c.Lr - 64;
+#pragma unroll
+    for (int jj = 0; jj < 32; ++jj) {
+      const int j = c.hcol * 32 + jj;
+      const bool same = (i >> 5) == (j >> 5);
+      if (!same && i >= 32) continue;  // lower-left block comes from product b
+      const float val = (same && (isA ? j < i : j <= i)) ? v[jj] : 0.f;
+      if (isA) sAh[i * 65 + j] = val;
+      else st_tf32(c.sm, p_off(i, j, transP), val);
+    }
+  }
+  {
+    float v[16];
+    tmem_ld16(tm_apb + c.lo + c.hcol * 16, v);
+    if (c.lane < 16) {
+      const int r = c.sub * 16 + c.lane;  // row of the 64-row product (M = 64 accumulator layout)
+#pragma unroll
+      for (int jj = 0; jj < 16; ++jj) {
+        const int j = c.hcol * 16 + jj;
+        if (r < 32) sAh[(32 + r) * 65 + j] = v[jj];
+        else st_tf32(c.sm, p_off(r, j, transP), v[jj]);
+      }
+    }
+  }
+  __syncthreads();
+  if (wide) {
+    for (int jj = 0; jj < 16; ++jj) {
+      const int j = pw.j0 + jj;
+      if (pw.kind == 0 && j < pw.i) sAh[pw.i * 65 + j] = pw.v[jj];
+      if (pw.kind == 1 && j <= pw.i) st_tf32(c.sm, p_off(pw.i, j, transP), pw.v[jj]);
+    }
+    __syncthreads();
+  }
+}
+
+// T = (I + diag(beta) Ah)^-1, row-major at R_TROW (stride 65).
+__device__ __forceinline__ void invert(const Ctx& c) {
+  invert_unit_lower<C>(reinterpret_cast<float*>(c.sm + R_AH), c.beta(), reinterpret_cast<float*>(c.sm + R_TROW),
+                       reinterpret_cast<float*>(c.sm + R_SW));
+}
+
+}  // namespace tcc
+}  // namespace kda

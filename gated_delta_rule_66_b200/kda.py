@@ -22,8 +22,8 @@ KDA_DTYPE_BF16 = 1
 KDA_BWD_STATES_FROM_FWD = 1
 CHUNK = 32  # chunk length of the library's chunked kernels (workspace layout)
 
-SYMBOLS = ("kda_last_error", "kda_fwd_workspace_bytes", "kda_bwd_workspace_bytes", "kda_fwd",
-           "kda_decode_step", "kda_bwd")
+SYMBOLS = ("kda_last_error", "kda_device_status", "kda_fwd_workspace_bytes",
+           "kda_bwd_workspace_bytes", "kda_fwd", "kda_decode_step", "kda_bwd")
 
 
 class KdaError(RuntimeError):
@@ -43,6 +43,8 @@ def _load():
     vp, f, i, sz = ctypes.c_void_p, ctypes.c_float, ctypes.c_int, ctypes.c_size_t
     lib.kda_last_error.restype = ctypes.c_char_p
     lib.kda_last_error.argtypes = []
+    lib.kda_device_status.restype = i
+    lib.kda_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint)]
     lib.kda_fwd_workspace_bytes.restype = sz
     lib.kda_fwd_workspace_bytes.argtypes = [i, i, i, i, i]
     lib.kda_bwd_workspace_bytes.restype = sz
@@ -97,6 +99,14 @@ def _req(name, t, dtype=None, ndim=None):
 
 def _stream():
     return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def device_status():
+    """Reads and clears the kernels' device-side error bits on the current
+    device (synchronises it); 0 means no kernel gave up on a bounded wait."""
+    flags = ctypes.c_uint(0)
+    _check("kda_device_status", _lib.kda_device_status(ctypes.byref(flags)))
+    return int(flags.value)
 
 
 def workspace_bytes(kind, B, T, H, HV, K, V):

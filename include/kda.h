@@ -70,6 +70,13 @@ enum {
  * The pointer stays valid until the next call from the same thread. */
 const char* kda_last_error(void);
 
+/* Reads and clears the device-side error bits of the library's kernels on the
+ * current device, synchronising it first.  Bit 0: a tensor-core kernel gave
+ * up waiting for its own tensor-core work (a bounded wait ran out) and
+ * skipped the rest of its launch; its outputs are then undefined.  Returns
+ * KDA_OK or KDA_ERR_CUDA; *flags receives the bits (0 = none). */
+int kda_device_status(unsigned* flags);
+
 /* Bytes of the optional kda_fwd workspace: the fp32 state entering every
  * chunk, laid out [B, HV, ceil(T / chunk), K, V]; 0 if a size is invalid. */
 size_t kda_fwd_workspace_bytes(int B, int T, int HV, int K, int V);
