@@ -80,11 +80,17 @@ size_t kda_fwd_workspace_bytes(int B, int T, int HV, int K, int V) {
   return states_bytes(B, T, HV, K, V);
 }
 
+static size_t grads_record_bytes(int B, int T, int HV, int K, int V) {
+  if (K != 128 || V != 128) return 0;
+  const size_t NT64 = (size_t)(T + 63) / 64;
+  return (size_t)B * HV * NT64 * GREC * sizeof(float);
+}
+
 size_t kda_bwd_workspace_bytes(int B, int T, int H, int HV, int K, int V) {
   if (B < 1 || T < 1 || H < 1 || HV < 1 || K < 1 || V < 1 || HV % H) return 0;
   size_t bytes = 2 * states_bytes(B, T, HV, K, V);
   if (HV > H) bytes += 2 * (size_t)B * T * HV * K * sizeof(float);
-  return bytes;
+  return bytes + grads_record_bytes(B, T, HV, K, V);
 }
 
 int kda_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
@@ -139,17 +145,20 @@ int kda_bwd(const void* q, const void* k, const void* v, const float* g, const f
   float* states = reinterpret_cast<float*>(ws);
   float* dstates = reinterpret_cast<float*>(ws + sb);
   float *dq_part = nullptr, *dk_part = nullptr;
+  size_t off = 2 * sb;
   if (HV > H) {
-    dq_part = reinterpret_cast<float*>(ws + 2 * sb);
+    dq_part = reinterpret_cast<float*>(ws + off);
     dk_part = dq_part + (size_t)B * T * HV * K;
+    off += 2 * (size_t)B * T * HV * K * sizeof(float);
   }
+  float* gws = grads_record_bytes(B, T, HV, K, V) ? reinterpret_cast<float*>(ws + off) : nullptr;
   if (!(flags & KDA_BWD_STATES_FROM_FWD)) {
     FwdArgs fa{q, k, v, g, beta, S0, nullptr, nullptr, states, scale, B, T, H, HV, K, V};
     rc = launch_fwd(fa, dtype, st);
     if (rc) return rc;
   }
   BwdArgs a{q, k, v, dO, g, beta, dS_T, states, dstates, dq, dk, dv, dg, dbeta, dS0,
-            dq_part, dk_part, scale, B, T, H, HV, K, V};
+            dq_part, dk_part, gws, scale, B, T, H, HV, K, V};
   return launch_bwd(a, dtype, st);
 }
 

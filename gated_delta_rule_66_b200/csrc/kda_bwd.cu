@@ -363,62 +363,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) kda_bwd_grads_kernel(BwdArgs a) {
   __syncthreads();
   float *sDq = sdQE, *sDk = sdKE, *sDc = sdKEd;
 
-  for (int J = 0; J < NB; ++J) {
-    const bool pairwise = block_factors<K, C, PRECISE>(J, sC, sE1, sE2o, sE2d, sFlag);
-    const int r0 = J * BS;
-    // row terms: rows i >= r0 against the columns of block J
-    for (int idx = threadIdx.x; idx < (C - r0) * K; idx += NTHREADS) {
-      const int i = r0 + idx / K, f = idx % K;
-      const bool diag = i < r0 + BS;
-      const int jmax = diag ? i : r0 + BS - 1;   // j <= i
-      float rA = 0.f, rP = 0.f;
-      if (diag && pairwise) {
-        for (int j = r0; j <= jmax; ++j) {
-          const float w = sK[j * LDK + f] * kexp<PRECISE>(sC[i * LDK + f] - sC[j * LDK + f]);
-          rA = fmaf(sdA[i * LDC + j], w, rA);
-          rP = fmaf(sdP[i * LDC + j], w, rP);
-        }
-      } else {
-        const float* e2 = diag ? sE2d : sE2o;
-        for (int j = r0; j <= jmax; ++j) {
-          const float w = sK[j * LDK + f] * e2[(j - r0) * LDK + f];
-          rA = fmaf(sdA[i * LDC + j], w, rA);
-          rP = fmaf(sdP[i * LDC + j], w, rP);
-        }
-        const float e1 = sE1[i * LDK + f];
-        rA *= e1;
-        rP *= e1;
-      }
-      const int o = i * LDK + f;
-      sDk[o] += rA;
-      sDq[o] += rP;
-      sDc[o] += sK[o] * rA + sQ[o] * rP;
-    }
-    __syncthreads();
-    // column terms: columns j of block J against rows i >= j
-    for (int idx = threadIdx.x; idx < BS * K; idx += NTHREADS) {
-      const int jj = idx / K, f = idx % K, j = r0 + jj;
-      float cAd = 0.f, cPd = 0.f, cAo = 0.f, cPo = 0.f;
-      for (int i = j; i < r0 + BS; ++i) {
-        const int o = i * LDK + f;
-        const float x = (pairwise) ? kexp<PRECISE>(sC[o] - sC[j * LDK + f]) : sE1[o];
-        cAd = fmaf(sdA[i * LDC + j], sK[o] * x, cAd);
-        cPd = fmaf(sdP[i * LDC + j], sQ[o] * x, cPd);
-      }
-      for (int i = r0 + BS; i < C; ++i) {
-        const int o = i * LDK + f;
-        const float x = sE1[o];
-        cAo = fmaf(sdA[i * LDC + j], sK[o] * x, cAo);
-        cPo = fmaf(sdP[i * LDC + j], sQ[o] * x, cPo);
-      }
-      const float e2d = pairwise ? 1.f : sE2d[jj * LDK + f], e2o = sE2o[jj * LDK + f];
-      const float col = (cAd + cPd) * e2d + (cAo + cPo) * e2o;
-      const int o = j * LDK + f;
-      sDk[o] += col;
-      sDc[o] -= sK[o] * col;
-    }
-    __syncthreads();
-  }
+  factored_terms<K, C, PRECISE, false>(sK, sQ, sC, sdA, sdP, sE1, sE2o, sE2d, sFlag, sDq, sDk, sDc);
 
   // dg = reverse cumulative sum of dc over the chunk (plus the chunk-end terms)
   for (int f = threadIdx.x; f < K; f += NTHREADS) {
@@ -464,12 +409,199 @@ __global__ void kda_group_sum_kernel(const float* __restrict__ part, TIn* __rest
   }
 }
 
+
+// Assembles dq, dk, dg and dbeta of one 64-step chunk from the record that
+// kda_bwd_grads_tc_kernel wrote (Ah, [dP; dA], [dQE; dKE'], dKEd, dbeta_R,
+// dEl): dbeta = dbeta_R + sum_j dA_ij Ah_ij; dq~ = dQE o e^c; dk = dKE o e^c +
+// dKEd o e^{c_last-c}; dc = (dQE o q~ + dKE o k) o e^c - dKEd o k o e^{c_last-c};
+// then the interaction terms (factored_terms) and dg = reverse cumsum of dc.
+// Everything here is independent across key channels, so one CTA handles one
+// (b, hv, chunk, half of the 128 key channels).
+struct AsmSmem {
+  static constexpr int C = 64, KH = 64, LDK = KH + 1, LDC = C + 1;
+  static constexpr int oK = 0, oQ = oK + C * LDK, oC = oQ + C * LDK, oDq = oC + C * LDK, oDk = oDq + C * LDK,
+                       oDc = oDk + C * LDK, oE1 = oDc + C * LDK, oE2o = oE1 + C * LDK, oE2d = oE2o + BS * LDK,
+                       oAh = oE2d + BS * LDK, odA = oAh + C * LDC, odP = odA + C * LDC, oBeta = odP + C * LDC,
+                       oLast = oBeta + C, oFlag = oLast + KH, total = oFlag + 4;
+  static constexpr size_t bytes = (size_t)total * sizeof(float);
+};
+
+template <typename TIn>
+__global__ void __launch_bounds__(NTHREADS, 1) kda_bwd_assemble_kernel(BwdArgs a) {
+  using S = AsmSmem;
+  constexpr int C = S::C, KH = S::KH, LDK = S::LDK, LDC = S::LDC, KD = 128;
+  extern __shared__ float smem[];
+  float *sK = smem + S::oK, *sQ = smem + S::oQ, *sC = smem + S::oC, *sDq = smem + S::oDq,
+        *sDk = smem + S::oDk, *sDc = smem + S::oDc, *sE1 = smem + S::oE1, *sE2o = smem + S::oE2o,
+        *sE2d = smem + S::oE2d, *sAh = smem + S::oAh, *sdA = smem + S::odA, *sdP = smem + S::odP,
+        *sBeta = smem + S::oBeta, *sLast = smem + S::oLast;
+  int* sFlag = reinterpret_cast<int*>(smem + S::oFlag);
+  const int ch = blockIdx.x >> 1, fh = blockIdx.x & 1, hv = blockIdx.y, b = blockIdx.z;
+  const int G = a.HV / a.H, h = hv / G, T = a.T, NT = (T + C - 1) / C;
+  const int t0 = ch * C, L = min(C, T - t0), f0 = fh * KH;
+  const size_t head = (size_t)b * a.HV + hv;
+  const float* rec = a.gws + (head * NT + ch) * GREC;
+  const TIn* q = static_cast<const TIn*>(a.q);
+  const TIn* k = static_cast<const TIn*>(a.k);
+
+  // inputs of this channel half: 4 channels per item, all loads issued before use
+  {
+    float4 gv[4];
+    float qv[4][4], kv[4][4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int idx = threadIdx.x + m * NTHREADS, i = idx >> 4, f4 = (idx & 15) * 4;
+      gv[m] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) qv[m][u] = kv[m][u] = 0.f;
+      if (i < L) {
+        const size_t rq = (((size_t)b * T + t0 + i) * a.H + h) * KD + f0 + f4;
+        gv[m] = *reinterpret_cast<const float4*>(a.g + (((size_t)b * T + t0 + i) * a.HV + hv) * KD + f0 + f4);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          qv[m][u] = to_f(q[rq + u]);
+          kv[m][u] = to_f(k[rq + u]);
+        }
+      }
+    }
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int idx = threadIdx.x + m * NTHREADS, i = idx >> 4, f4 = (idx & 15) * 4;
+      const float gg[4] = {gv[m].x, gv[m].y, gv[m].z, gv[m].w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        sQ[i * LDK + f4 + u] = qv[m][u] * a.scale;
+        sK[i * LDK + f4 + u] = kv[m][u];
+        sC[i * LDK + f4 + u] = gg[u];
+      }
+    }
+  }
+  for (int i = threadIdx.x; i < C; i += NTHREADS)
+    sBeta[i] = (i < L) ? a.beta[((size_t)b * T + t0 + i) * a.HV + hv] : 0.f;
+  {  // Ah, dP, dA (float4 rows of the record)
+    float4 ah[4], dp[4], da[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int idx = threadIdx.x + m * NTHREADS, i = idx >> 4, j4 = (idx & 15) * 4;
+      ah[m] = *reinterpret_cast<const float4*>(rec + G_AH + i * 64 + j4);
+      dp[m] = *reinterpret_cast<const float4*>(rec + G_PA + i * 64 + j4);
+      da[m] = *reinterpret_cast<const float4*>(rec + G_PA + (64 + i) * 64 + j4);
+    }
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int idx = threadIdx.x + m * NTHREADS, i = idx >> 4, j4 = (idx & 15) * 4;
+      const float vah[4] = {ah[m].x, ah[m].y, ah[m].z, ah[m].w}, vdp[4] = {dp[m].x, dp[m].y, dp[m].z, dp[m].w},
+                  vda[4] = {da[m].x, da[m].y, da[m].z, da[m].w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = j4 + u;
+        sAh[i * LDC + j] = vah[u];
+        sdP[i * LDC + j] = (j <= i) ? vdp[u] : 0.f;
+        sdA[i * LDC + j] = (j < i) ? vda[u] : 0.f;
+      }
+    }
+  }
+  __syncthreads();
+  for (int f = threadIdx.x; f < KH; f += NTHREADS) {
+    float run = 0.f;
+    for (int i = 0; i < C; ++i) {
+      run += sC[i * LDK + f];
+      sC[i * LDK + f] = run;
+    }
+  }
+  if (fh == 0) {
+    for (int i = threadIdx.x; i < L; i += NTHREADS) {
+      float s = rec[G_DBR + i];
+      for (int j = 0; j < i; ++j) s = fmaf(sdA[i * LDC + j], sAh[i * LDC + j], s);
+      a.dbeta[((size_t)b * T + t0 + i) * a.HV + hv] = s;
+    }
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < C * C; idx += NTHREADS) {
+    const int i = idx >> 6, j = idx & 63;
+    sdA[i * LDC + j] *= sBeta[i];
+  }
+  {  // element-wise terms; the chunk-end sum of dKEd o k o e^{c_last-c} goes through sE1
+    float4 qe[4], ke[4], kd[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int idx = threadIdx.x + m * NTHREADS, i = idx >> 4, f4 = (idx & 15) * 4;
+      qe[m] = *reinterpret_cast<const float4*>(rec + G_QK + i * 128 + f0 + f4);
+      ke[m] = *reinterpret_cast<const float4*>(rec + G_QK + (64 + i) * 128 + f0 + f4);
+      kd[m] = *reinterpret_cast<const float4*>(rec + G_KED + i * 128 + f0 + f4);
+    }
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int idx = threadIdx.x + m * NTHREADS, i = idx >> 4, f4 = (idx & 15) * 4;
+      const float vq[4] = {qe[m].x, qe[m].y, qe[m].z, qe[m].w}, vk[4] = {ke[m].x, ke[m].y, ke[m].z, ke[m].w},
+                  vd[4] = {kd[m].x, kd[m].y, kd[m].z, kd[m].w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int f = f4 + u, o = i * LDK + f;
+        const float c = sC[o], e = __expf(c), ed = __expf(sC[(C - 1) * LDK + f] - c);
+        const float dqe = vq[u], dke = sBeta[i] * vk[u], dked = vd[u];
+        const float kk = sK[o], qq = sQ[o];
+        sDq[o] = dqe * e;
+        sDk[o] = dke * e + dked * ed;
+        sDc[o] = (dqe * qq + dke * kk) * e - dked * kk * ed;
+        sE1[o] = dked * kk * ed;
+      }
+    }
+  }
+  __syncthreads();
+  for (int f = threadIdx.x; f < KH; f += NTHREADS) {
+    float s = rec[G_DEL + f0 + f] * __expf(sC[(C - 1) * LDK + f]);
+    for (int i = 0; i < C; ++i) s += sE1[i * LDK + f];
+    sLast[f] = s;
+  }
+  __syncthreads();
+  factored_terms<KH, C, false, true>(sK, sQ, sC, sdA, sdP, sE1, sE2o, sE2d, sFlag, sDq, sDk, sDc);
+  for (int f = threadIdx.x; f < KH; f += NTHREADS) {
+    float run = sLast[f];
+    for (int i = C - 1; i >= 0; --i) {
+      run += sDc[i * LDK + f];
+      sDc[i * LDK + f] = run;
+    }
+  }
+  __syncthreads();
+  TIn* dq = static_cast<TIn*>(a.dq);
+  TIn* dk = static_cast<TIn*>(a.dk);
+  for (int idx = threadIdx.x; idx < L * KH; idx += NTHREADS) {
+    const int i = idx / KH, f = idx % KH, o = i * LDK + f;
+    const size_t row_v = ((size_t)b * T + t0 + i) * a.HV + hv;
+    a.dg[row_v * KD + f0 + f] = sDc[o];
+    if (G == 1) {
+      const size_t row_h = ((size_t)b * T + t0 + i) * a.H + h;
+      dq[row_h * KD + f0 + f] = from_f<TIn>(a.scale * sDq[o]);
+      dk[row_h * KD + f0 + f] = from_f<TIn>(sDk[o]);
+    } else {
+      a.dq_part[row_v * KD + f0 + f] = a.scale * sDq[o];
+      a.dk_part[row_v * KD + f0 + f] = sDk[o];
+    }
+  }
+}
+
+template <typename TIn>
+static int launch_assemble(const BwdArgs& a, cudaStream_t stream) {
+  auto kern = kda_bwd_assemble_kernel<TIn>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)AsmSmem::bytes);
+  if (e != cudaSuccess) return set_cuda_error("kda_bwd: cudaFuncSetAttribute", e);
+  const int NT = (a.T + 63) / 64;
+  kern<<<dim3(NT * 2, a.HV, a.B), NTHREADS, AsmSmem::bytes, stream>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return set_cuda_error("kda_bwd: assemble launch", e);
+  return 0;
+}
+
 template <int K, typename TIn>
 static int launch_bwd_t(const BwdArgs& a, cudaStream_t stream) {
   constexpr int C = FWD_CHUNK, VB = FWD_VBLOCK;
   const int NT = (a.T + C - 1) / C;
-  if (bwd_tc_eligible(a, sizeof(TIn) == 2 ? 1 : 0)) {
-    const int rc = launch_bwd_dstate_tc(a, stream);
+  const bool tc = bwd_tc_eligible(a, sizeof(TIn) == 2 ? 1 : 0);
+  if (tc) {
+    int rc = launch_bwd_dstate_tc(a, stream);
+    if (!rc) rc = launch_bwd_grads_tc(a, stream);
+    if (!rc) rc = launch_assemble<TIn>(a, stream);
     if (rc) return rc;
   } else {
     using S = DstSmem<K, C, VB>;
@@ -479,13 +611,11 @@ static int launch_bwd_t(const BwdArgs& a, cudaStream_t stream) {
     kern<<<dim3(a.V / VB, a.HV, a.B), NTHREADS, S::bytes, stream>>>(a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return set_cuda_error("kda_bwd: state-gradient launch", e);
-  }
-  {
-    using S = GradSmem<K, C, VB>;
-    auto kern = kda_bwd_grads_kernel<K, C, VB, TIn>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::bytes);
+    using S2 = GradSmem<K, C, VB>;
+    auto kern2 = kda_bwd_grads_kernel<K, C, VB, TIn>;
+    e = cudaFuncSetAttribute(kern2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S2::bytes);
     if (e != cudaSuccess) return set_cuda_error("kda_bwd: cudaFuncSetAttribute", e);
-    kern<<<dim3(NT, a.HV, a.B), NTHREADS, S::bytes, stream>>>(a);
+    kern2<<<dim3(NT, a.HV, a.B), NTHREADS, S2::bytes, stream>>>(a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return set_cuda_error("kda_bwd: gradient launch", e);
   }

@@ -251,7 +251,8 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_dstate_tc_kernel(BwdArgs a) {
 
 bool bwd_tc_eligible(const BwdArgs& a, int dtype) {
   auto al16 = [](const void* p) { return ((uintptr_t)p & 15u) == 0; };
-  return dtype == 1 && a.K == 128 && a.V == 128 && al16(a.q) && al16(a.k) && al16(a.dO) && al16(a.g);
+  return dtype == 1 && a.K == 128 && a.V == 128 && a.gws != nullptr && al16(a.q) && al16(a.k) &&
+         al16(a.dO) && al16(a.g);
 }
 
 int launch_bwd_dstate_tc(const BwdArgs& a, cudaStream_t stream) {
@@ -261,6 +262,304 @@ int launch_bwd_dstate_tc(const BwdArgs& a, cudaStream_t stream) {
   kda_bwd_dstate_tc_kernel<<<dim3(a.HV, a.B), tcc::NTH, tcc::SMEM_BYTES, stream>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return set_cuda_error("kda_bwd: tensor-core state-gradient launch", e);
+  return 0;
+}
+
+
+// ============================================================================
+// Per-chunk gradient products on the tensor cores (K = V = 128, C = 64).
+//
+// One CTA per (b, hv, chunk), all chunks in parallel.  With M the state
+// entering the chunk and dM the gradient of the state leaving it (both from
+// the workspace), it recomputes
+//   X = V - (K o e^c) M,  U = T diag(beta) X,  dU = P^T dO + (K o e^{c_last-c}) dM,
+//   dR = T^T dU,  dv = diag(beta) dR,
+// and forms every product that sums over the value columns n:
+//   dP = dO U^T,  dA = -dR U^T,  dQE = dO M^T,  dKE' = -dR M^T (dKE = diag(beta) dKE'),
+//   dKEd = U dM^T,  dbeta_R_i = sum_n dR_in X_in,  dEl_f = sum_n M_fn dM_fn,
+// writing them (with Ah) to a per-chunk record that kda_bwd_assemble_kernel
+// turns into dq, dk, dg and dbeta.  Lane-n products use the transposed forms
+// (A operands M^T, dM^T, dO^T, X^T, dU^T in TMEM); the sums over n contract
+// [dO; -dR] against U, M and dM staged in shared memory.
+// ============================================================================
+namespace tcg {
+using namespace tcc;
+constexpr uint32_t OP_KE = OP, OP_U = OP, OP_KED = OP + 32768, OP_DO = OP + 65536, OP_TT = OP + 131072;
+constexpr uint32_t R_MB = 0;  // M or dM staged as [f][n] once the raw region is free
+constexpr uint32_t TM_M = 0, TM_U = 0, TM_QK = 0, TM_DM = 128, TM_DR = 128, TM_KED = 128, TM_DOT = 256,
+                   TM_PA = 256, TM_APA = 320, TM_APB = 384, TM_X = 320, TM_DU = 384;
+}  // namespace tcg
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+  return x;
+}
+
+__global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
+  using namespace tcg;
+  using namespace tc;
+  extern __shared__ __align__(1024) unsigned char sm[];
+  Ctx cx;
+  cx.sm = sm;
+  cx.sb = smem_u32(sm);
+  cx.tid = threadIdx.x;
+  cx.warp = cx.tid >> 5;
+  cx.lane = cx.tid & 31;
+  cx.sub = cx.warp & 3;
+  cx.hcol = cx.warp >> 2;
+  cx.Lr = cx.sub * 32 + cx.lane;
+  cx.lo = (uint32_t)(cx.sub * 32) << 16;
+  const int tid = cx.tid, hcol = cx.hcol, Lr = cx.Lr, lane = cx.lane;
+  const uint32_t lo = cx.lo, sb = cx.sb;
+
+  const int ch = blockIdx.x, hv = blockIdx.y, b = blockIdx.z;
+  const int G = a.HV / a.H, h = hv / G, T = a.T, NT = (T + C - 1) / C, NT32 = (T + 31) / 32;
+  const int t0 = ch * C, L = min(C, T - t0);
+  const size_t head = (size_t)b * a.HV + hv;
+  float* rec = a.gws + (head * NT + ch) * GREC;
+  const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(a.q);
+  const __nv_bfloat16* kg = static_cast<const __nv_bfloat16*>(a.k);
+  const __nv_bfloat16* vg = static_cast<const __nv_bfloat16*>(a.v);
+  const __nv_bfloat16* dog = static_cast<const __nv_bfloat16*>(a.dO);
+  __nv_bfloat16* dvg = static_cast<__nv_bfloat16*>(a.dv);
+  float* sBeta = cx.beta();
+  float* sDEl = reinterpret_cast<float*>(sm + S_EL);    // 128 floats
+  float* sDbR = reinterpret_cast<float*>(sm + S_EMID);  // 64 floats
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + S_BAR);
+  uint32_t* sTm = reinterpret_cast<uint32_t*>(sm + S_TMEM);
+  const float* sC = cx.c();
+  // per-subpartition partial sums, added in a fixed order (deterministic)
+  float* partEl = reinterpret_cast<float*>(sm + R_AH);   // [4][128], once Ah is in the record
+  float* partBr = reinterpret_cast<float*>(sm + OP_TT);  // [4][64], once T^T is consumed
+
+  if (cx.warp == 0) tmem_alloc(sTm, 512);
+  if (tid == 0) mbar_init(bar, 1);
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tm = *sTm;
+  cx.tm = tm;
+  uint32_t phase = 0;
+  bool failed = false;
+
+  do {
+    // ---------------------------------------------------------------- interaction products
+    load_raw(cx, qg, kg, dog, a.g, a.beta, b, T, t0, L, a.H, a.HV, h, hv);
+    const bool wide = cumsum_span(cx);
+    build_op1_and_issue(cx, a.scale, tm + TM_APA, tm + TM_APB, bar);
+    if (!wait_mma(bar, phase)) { failed = true; break; }
+
+    // ---------------------------------------------------------------- K o e^c, K o e^{c_last-c}, dO, dO^T
+    {
+      const int fq = item_f(cx);
+      const float4 c63v = ld4(sC + 63 * LDCF + fq);
+      const float c63[4] = {c63v.x, c63v.y, c63v.z, c63v.w};
+      for (int m = 0; m < 8; ++m) {
+        const int i = item_row(cx, m);
+        const float4 c4 = ld4(sC + i * LDCF + fq);
+        const float c[4] = {c4.x, c4.y, c4.z, c4.w};
+        float kf[4], df[4];
+        bf16x4(sm + RAW_K + i * 256 + fq * 2, kf);
+        bf16x4(sm + RAW_X + i * 256 + fq * 2, df);
+        float e[4], ed[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          e[u] = ex2(c[u]);
+          ed[u] = ex2(c63[u] - c[u]);
+        }
+        st_tf32x4(sm, OP_KE + kmaj(i, fq, 128), kf[0] * e[0], kf[1] * e[1], kf[2] * e[2], kf[3] * e[3]);
+        st_tf32x4(sm, OP_KED + kmaj(i, fq, 128), kf[0] * ed[0], kf[1] * ed[1], kf[2] * ed[2], kf[3] * ed[3]);
+        st_tf32x4(sm, OP_DO + kmaj(i, fq, 128), df[0], df[1], df[2], df[3]);
+      }
+      uint32_t r[32];
+      const unsigned char* col = sm + RAW_X + Lr * 2;
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj)
+        r[jj] = tf32_rna(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(col + (hcol * 32 + jj) * 256)));
+      tmem_st32(tm + lo + TM_DOT + hcol * 32, r);
+      tmem_wait_st();
+    }
+    Pairwise pw;
+    if (wide) pairwise_compute(cx, a.scale, pw);
+    fence_async_smem();
+    fence_before();
+    __syncthreads();
+
+    readout_ap(cx, tm + TM_APA, tm + TM_APB, true, wide, pw);  // Ah at R_AH, P^T at R_P
+    {
+      const float* sAh = reinterpret_cast<const float*>(sm + R_AH);
+      for (int x = tid; x < C * C; x += NTH) rec[G_AH + x] = sAh[(x >> 6) * 65 + (x & 63)];
+    }
+    invert(cx);
+    {  // T diag(beta) at R_T and T^T at OP_TT, both as (row i, K = j) operands
+      const float* tr = reinterpret_cast<const float*>(sm + R_TROW);
+      for (int x = tid; x < C * 16; x += NTH) {
+        const int i = x >> 4, j4 = (x & 15) * 4;
+        const float* p = tr + i * 65 + j4;
+        st_tf32x4(sm, R_T + kmaj(i, j4, 64), p[0] * sBeta[j4], p[1] * sBeta[j4 + 1], p[2] * sBeta[j4 + 2],
+                  p[3] * sBeta[j4 + 3]);
+        st_tf32x4(sm, OP_TT + kmaj(i, j4, 64), tr[j4 * 65 + i], tr[(j4 + 1) * 65 + i], tr[(j4 + 2) * 65 + i],
+                  tr[(j4 + 3) * 65 + i]);
+      }
+    }
+
+    // ---------------------------------------------------------------- M^T, dM^T into TMEM; dEl
+    {
+      const int dm_idx = (2 * ch + 1 < NT32) ? 2 * ch + 1 : 2 * ch;
+      for (int cb = 0; cb < 2; ++cb) {
+        const int f0 = hcol * 64 + cb * 32;
+        uint32_t rm[32], rd[32];
+        const float* ms = a.states + ((head * NT32 + 2 * ch) * KD + f0) * VD + Lr;
+        const float* ds = a.dstates + ((head * NT32 + dm_idx) * KD + f0) * VD + Lr;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float mv = ms[(size_t)j * VD], dv = ds[(size_t)j * VD];
+          rm[j] = __float_as_uint(mv);
+          rd[j] = __float_as_uint(dv);
+          const float s = warp_sum(mv * dv);
+          if (lane == 0) partEl[cx.sub * KD + f0 + j] = s;
+        }
+        tmem_st32(tm + lo + TM_M + f0, rm);
+        tmem_st32(tm + lo + TM_DM + f0, rd);
+      }
+      tmem_wait_st();
+    }
+    float vT[32];  // V^T: lane n, rows i of this warp half
+#pragma unroll
+    for (int jj = 0; jj < 32; ++jj) {
+      const int i = hcol * 32 + jj;
+      vT[jj] = (i < L) ? __bfloat162float(vg[(((size_t)b * T + t0 + i) * a.HV + hv) * VD + Lr]) : 0.f;
+    }
+    fence_async_smem();
+    fence_before();
+    __syncthreads();
+    if (tid < KD) sDEl[tid] = ((partEl[tid] + partEl[KD + tid]) + partEl[2 * KD + tid]) + partEl[3 * KD + tid];
+    if (tid == 0) {  // X'^T = M^T (K o e^c)^T ; dU^T = dO^T P + dM^T (K o e^{c_last-c})^T
+      fence_after();
+      const uint32_t id = idesc_tf32(128, 64);
+      for (int ks = 0; ks < 16; ++ks)
+        mma_ts(tm + TM_X, tm + TM_M + ks * 8, desc(sb + OP_KE + ks * 256, 4096), id, ks > 0);
+      for (int ks = 0; ks < 8; ++ks)
+        mma_ts(tm + TM_DU, tm + TM_DOT + ks * 8, desc(sb + R_P + ks * 256, 2048), id, ks > 0);
+      for (int ks = 0; ks < 16; ++ks)
+        mma_ts(tm + TM_DU, tm + TM_DM + ks * 8, desc(sb + OP_KED + ks * 256, 4096), id, 1);
+      commit(bar);
+    }
+    if (!wait_mma(bar, phase)) { failed = true; break; }
+    {  // X^T = V^T - X'^T
+      float x[32];
+      uint32_t r[32];
+      tmem_ld32(tm + lo + TM_X + hcol * 32, x);
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) r[jj] = tf32_rna(vT[jj] - x[jj]);
+      tmem_st32(tm + lo + TM_X + hcol * 32, r);
+      tmem_wait_st();
+    }
+    fence_before();
+    __syncthreads();
+    if (tid == 0) {  // U^T = X^T (T diag(beta))^T ; dR^T = dU^T T
+      fence_after();
+      const uint32_t id = idesc_tf32(128, 64);
+      for (int ks = 0; ks < 8; ++ks) {
+        mma_ts(tm + TM_U, tm + TM_X + ks * 8, desc(sb + R_T + ks * 256, 2048), id, ks > 0);
+        mma_ts(tm + TM_DR, tm + TM_DU + ks * 8, desc(sb + OP_TT + ks * 256, 2048), id, ks > 0);
+      }
+      commit(bar);
+    }
+    if (!wait_mma(bar, phase)) { failed = true; break; }
+
+    // ---------------------------------------------------------------- dv, dbeta_R; U and -dR as [i][n] operands
+    {
+      float u[32], dr[32], x[32];
+      tmem_ld32(tm + lo + TM_U + hcol * 32, u);
+      tmem_ld32(tm + lo + TM_DR + hcol * 32, dr);
+      tmem_ld32(tm + lo + TM_X + hcol * 32, x);
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) {
+        const int i = hcol * 32 + jj;
+        if (i < L) dvg[(((size_t)b * T + t0 + i) * a.HV + hv) * VD + Lr] = __float2bfloat16_rn(sBeta[i] * dr[jj]);
+        const float s = warp_sum(dr[jj] * x[jj]);
+        if (lane == 0) partBr[cx.sub * C + i] = s;
+        st_tf32(sm, OP_U + kmaj(i, Lr, 128), u[jj]);
+        st_tf32(sm, OP_DO + kmaj(64 + i, Lr, 128), -dr[jj]);
+      }
+    }
+    // M as [f][n] for the sums over n
+    for (int e = tid; e < KD * 32; e += NTH) {
+      const int f = e >> 5, n4 = (e & 31) * 4;
+      cp_async16(sb + R_MB + kmaj(f, n4, 128), a.states + ((head * NT32 + 2 * ch) * KD + f) * VD + n4, true);
+    }
+    cp_async_wait_all();
+    fence_async_smem();
+    __syncthreads();
+    if (tid < C) sDbR[tid] = ((partBr[tid] + partBr[C + tid]) + partBr[2 * C + tid]) + partBr[3 * C + tid];
+    if (tid == 0) {  // [dP; dA] = [dO; -dR] U^T ; [dQE; dKE'] = [dO; -dR] M^T
+      fence_after();
+      for (int ks = 0; ks < 16; ++ks) {
+        const uint64_t aD = desc(sb + OP_DO + ks * 256, 4096);
+        mma_ss(tm + TM_PA, aD, desc(sb + OP_U + ks * 256, 4096), idesc_tf32(128, 64), ks > 0);
+        mma_ss(tm + TM_QK, aD, desc(sb + R_MB + ks * 256, 4096), idesc_tf32(128, 128), ks > 0);
+      }
+      commit(bar);
+    }
+    if (!wait_mma(bar, phase)) { failed = true; break; }
+    {  // dM as [f][n]
+      const int dm_idx = (2 * ch + 1 < NT32) ? 2 * ch + 1 : 2 * ch;
+      for (int e = tid; e < KD * 32; e += NTH) {
+        const int f = e >> 5, n4 = (e & 31) * 4;
+        cp_async16(sb + R_MB + kmaj(f, n4, 128), a.dstates + ((head * NT32 + dm_idx) * KD + f) * VD + n4, true);
+      }
+      cp_async_wait_all();
+    }
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 0) {  // dKEd = U dM^T
+      fence_after();
+      for (int ks = 0; ks < 16; ++ks)
+        mma_ss(tm + TM_KED, desc(sb + OP_U + ks * 256, 4096), desc(sb + R_MB + ks * 256, 4096), idesc_tf32(64, 128),
+               ks > 0);
+      commit(bar);
+    }
+    if (!wait_mma(bar, phase)) { failed = true; break; }
+
+    // ---------------------------------------------------------------- record
+    {
+      float v[32];
+      tmem_ld32(tm + lo + TM_PA + hcol * 32, v);
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) rec[G_PA + Lr * 64 + hcol * 32 + jj] = v[jj];
+      for (int cb = 0; cb < 2; ++cb) {
+        const int f0 = hcol * 64 + cb * 32;
+        tmem_ld32(tm + lo + TM_QK + f0, v);
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) rec[G_QK + Lr * 128 + f0 + jj] = v[jj];
+        tmem_ld32(tm + lo + TM_KED + f0, v);
+        if (lane < 16) {
+          const int r = cx.sub * 16 + lane;  // M = 64 accumulator layout
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj) rec[G_KED + r * 128 + f0 + jj] = v[jj];
+        }
+      }
+      if (tid < C) rec[G_DBR + tid] = sDbR[tid];
+      if (tid < KD) rec[G_DEL + tid] = sDEl[tid];
+    }
+  } while (false);
+
+  fence_before();
+  __syncthreads();
+  if (cx.warp == 0) tmem_dealloc(tm, 512);
+  if (failed && tid == 0) atomicOr(&g_kda_device_error, 1u);
+}
+
+int launch_bwd_grads_tc(const BwdArgs& a, cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(kda_bwd_grads_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)tcc::SMEM_BYTES);
+  if (e != cudaSuccess) return set_cuda_error("kda_bwd: cudaFuncSetAttribute", e);
+  const int NT = (a.T + tcc::C - 1) / tcc::C;
+  kda_bwd_grads_tc_kernel<<<dim3(NT, a.HV, a.B), tcc::NTH, tcc::SMEM_BYTES, stream>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return set_cuda_error("kda_bwd: tensor-core gradient launch", e);
   return 0;
 }
 

@@ -236,4 +236,206 @@ __device__ void invert_unit_lower(const float* sAh, const float* sBeta, float* s
   }
 }
 
+
+// Adds to dq~, dk and the decay adjoint dc the terms that flow through the
+// interaction matrices (dA_hat = beta_i dA, strict lower; dP, lower incl.
+// diagonal; both C x C with row stride C+1):
+//   row terms    rowA_i = sum_j dA_hat_ij (k_j o e^{c_i - c_j}),  rowP_i likewise with dP
+//   column terms colA_j = sum_i dA_hat_ij (k_i o e^{c_i - c_j}),  colP_j with q~_i
+//   dk += rowA + colA + colP,  dq~ += rowP,
+//   dc += k o rowA + q~ o rowP - k o (colA + colP)
+// with every exp(c_i - c_j) split at the 16-row sub-block references of
+// block_factors (pair by pair for a diagonal block whose span is too wide).
+// sK, sQ, sC, sDq, sDk, sDc are C x K with row stride K+1; sE1 / sE2o / sE2d
+// are the scratch of block_factors.  One column block J at a time:
+// factored_block_scalar with fp32 FMA (any block), factored_block_mma with
+// 3xTF32 warp MMAs (blocks whose exponents split, K a multiple of 8).
+template <int K, int C, bool PRECISE>
+__device__ void factored_block_scalar(int J, bool pairwise, const float* sK, const float* sQ, const float* sC,
+                                      const float* sdA, const float* sdP, const float* sE1, const float* sE2o,
+                                      const float* sE2d, float* sDq, float* sDk, float* sDc) {
+  constexpr int LDK = K + 1, LDC = C + 1;
+    const int r0 = J * BS;
+    // row terms: rows i >= r0 against the columns of block J
+    for (int idx = threadIdx.x; idx < (C - r0) * K; idx += NTHREADS) {
+      const int i = r0 + idx / K, f = idx % K;
+      const bool diag = i < r0 + BS;
+      const int jmax = diag ? i : r0 + BS - 1;   // j <= i
+      float rA = 0.f, rP = 0.f;
+      if (diag && pairwise) {
+        for (int j = r0; j <= jmax; ++j) {
+          const float w = sK[j * LDK + f] * kexp<PRECISE>(sC[i * LDK + f] - sC[j * LDK + f]);
+          rA = fmaf(sdA[i * LDC + j], w, rA);
+          rP = fmaf(sdP[i * LDC + j], w, rP);
+        }
+      } else {
+        const float* e2 = diag ? sE2d : sE2o;
+        for (int j = r0; j <= jmax; ++j) {
+          const float w = sK[j * LDK + f] * e2[(j - r0) * LDK + f];
+          rA = fmaf(sdA[i * LDC + j], w, rA);
+          rP = fmaf(sdP[i * LDC + j], w, rP);
+        }
+        const float e1 = sE1[i * LDK + f];
+        rA *= e1;
+        rP *= e1;
+      }
+      const int o = i * LDK + f;
+      sDk[o] += rA;
+      sDq[o] += rP;
+      sDc[o] += sK[o] * rA + sQ[o] * rP;
+    }
+    __syncthreads();
+    // column terms: columns j of block J against rows i >= j
+    for (int idx = threadIdx.x; idx < BS * K; idx += NTHREADS) {
+      const int jj = idx / K, f = idx % K, j = r0 + jj;
+      float cAd = 0.f, cPd = 0.f, cAo = 0.f, cPo = 0.f;
+      for (int i = j; i < r0 + BS; ++i) {
+        const int o = i * LDK + f;
+        const float x = (pairwise) ? kexp<PRECISE>(sC[o] - sC[j * LDK + f]) : sE1[o];
+        cAd = fmaf(sdA[i * LDC + j], sK[o] * x, cAd);
+        cPd = fmaf(sdP[i * LDC + j], sQ[o] * x, cPd);
+      }
+      for (int i = r0 + BS; i < C; ++i) {
+        const int o = i * LDK + f;
+        const float x = sE1[o];
+        cAo = fmaf(sdA[i * LDC + j], sK[o] * x, cAo);
+        cPo = fmaf(sdP[i * LDC + j], sQ[o] * x, cPo);
+      }
+      const float e2d = pairwise ? 1.f : sE2d[jj * LDK + f], e2o = sE2o[jj * LDK + f];
+      const float col = (cAd + cPd) * e2d + (cAo + cPo) * e2o;
+      const int o = j * LDK + f;
+      sDk[o] += col;
+      sDc[o] -= sK[o] * col;
+    }
+    __syncthreads();
+}
+
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+
+// d += a (16 x 8, row-major) * b (8 x 8), tf32 inputs, fp32 accumulate.
+// Fragments (g = lane / 4, t = lane % 4): a0 (g, t), a1 (g+8, t), a2 (g, t+4),
+// a3 (g+8, t+4); b0 (k = t, n = g), b1 (k = t+4, n = g); d0 (g, 2t),
+// d1 (g, 2t+1), d2 (g+8, 2t), d3 (g+8, 2t+1).
+__device__ __forceinline__ void mma_16x8x8(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// x = hi + lo with both halves exactly representable in tf32; three tf32
+// products hi*hi + hi*lo + lo*hi carry ~fp32 accuracy (the lo*lo term is
+// below fp32 rounding).
+struct Split {
+  uint32_t hi, lo;
+};
+__device__ __forceinline__ Split split_tf32(float x) {
+  const uint32_t h = to_tf32(x);
+  return {h, to_tf32(x - __uint_as_float(h))};
+}
+__device__ __forceinline__ void mma3(float (&d)[4], const Split (&a)[4], const Split (&b)[2]) {
+  const uint32_t ah[4] = {a[0].hi, a[1].hi, a[2].hi, a[3].hi}, al[4] = {a[0].lo, a[1].lo, a[2].lo, a[3].lo};
+  const uint32_t bh[2] = {b[0].hi, b[1].hi}, bl[2] = {b[0].lo, b[1].lo};
+  mma_16x8x8(d, al, bh);
+  mma_16x8x8(d, ah, bl);
+  mma_16x8x8(d, ah, bh);
+}
+
+template <int K, int C>
+__device__ void factored_block_mma(int J, const float* sK, const float* sQ, const float* sdA, const float* sdP,
+                                   const float* sE1, const float* sE2o, const float* sE2d, float* sDq, float* sDk,
+                                   float* sDc) {
+  constexpr int LDK = K + 1, LDC = C + 1, NB = C / BS, NTL = K / 8;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const int r0 = J * BS;
+  // row terms: row block I >= J, 8 key channels per tile
+  for (int x = warp; x < (NB - J) * NTL; x += NTHREADS / 32) {
+    const int I = J + x / NTL, f0 = (x % NTL) * 8, i0 = I * BS;
+    const float* e2 = (I == J) ? sE2d : sE2o;
+    float accA[4] = {0.f, 0.f, 0.f, 0.f}, accP[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+      const int j = r0 + ks * 8 + t;
+      Split aA[4], aP[4], bw[2];
+      aA[0] = split_tf32(sdA[(i0 + g) * LDC + j]);
+      aA[1] = split_tf32(sdA[(i0 + g + 8) * LDC + j]);
+      aA[2] = split_tf32(sdA[(i0 + g) * LDC + j + 4]);
+      aA[3] = split_tf32(sdA[(i0 + g + 8) * LDC + j + 4]);
+      aP[0] = split_tf32(sdP[(i0 + g) * LDC + j]);
+      aP[1] = split_tf32(sdP[(i0 + g + 8) * LDC + j]);
+      aP[2] = split_tf32(sdP[(i0 + g) * LDC + j + 4]);
+      aP[3] = split_tf32(sdP[(i0 + g + 8) * LDC + j + 4]);
+      bw[0] = split_tf32(sK[j * LDK + f0 + g] * e2[(j - r0) * LDK + f0 + g]);
+      bw[1] = split_tf32(sK[(j + 4) * LDK + f0 + g] * e2[(j + 4 - r0) * LDK + f0 + g]);
+      mma3(accA, aA, bw);
+      mma3(accP, aP, bw);
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int i = i0 + g + ((e & 2) ? 8 : 0), f = f0 + 2 * t + (e & 1), o = i * LDK + f;
+      const float e1 = sE1[o], rA = accA[e] * e1, rP = accP[e] * e1;
+      sDk[o] += rA;
+      sDq[o] += rP;
+      sDc[o] += sK[o] * rA + sQ[o] * rP;
+    }
+  }
+  __syncthreads();
+  // column terms: columns of block J against rows i of J (diagonal) and below
+  for (int x = warp; x < NTL; x += NTHREADS / 32) {
+    const int f0 = x * 8;
+    float accD[4] = {0.f, 0.f, 0.f, 0.f}, accO[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int ks = 0; ks < (C - r0) / 8; ++ks) {
+      const int i = r0 + ks * 8 + t;
+      Split aA[4], aP[4], bk[2], bq[2];
+      aA[0] = split_tf32(sdA[i * LDC + r0 + g]);
+      aA[1] = split_tf32(sdA[i * LDC + r0 + g + 8]);
+      aA[2] = split_tf32(sdA[(i + 4) * LDC + r0 + g]);
+      aA[3] = split_tf32(sdA[(i + 4) * LDC + r0 + g + 8]);
+      aP[0] = split_tf32(sdP[i * LDC + r0 + g]);
+      aP[1] = split_tf32(sdP[i * LDC + r0 + g + 8]);
+      aP[2] = split_tf32(sdP[(i + 4) * LDC + r0 + g]);
+      aP[3] = split_tf32(sdP[(i + 4) * LDC + r0 + g + 8]);
+      const int o0 = i * LDK + f0 + g, o1 = (i + 4) * LDK + f0 + g;
+      bk[0] = split_tf32(sK[o0] * sE1[o0]);
+      bk[1] = split_tf32(sK[o1] * sE1[o1]);
+      bq[0] = split_tf32(sQ[o0] * sE1[o0]);
+      bq[1] = split_tf32(sQ[o1] * sE1[o1]);
+      if (ks < 2) {
+        mma3(accD, aA, bk);
+        mma3(accD, aP, bq);
+      } else {
+        mma3(accO, aA, bk);
+        mma3(accO, aP, bq);
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int jj = g + ((e & 2) ? 8 : 0), j = r0 + jj, f = f0 + 2 * t + (e & 1), o = j * LDK + f;
+      const float col = accD[e] * sE2d[jj * LDK + f] + accO[e] * sE2o[jj * LDK + f];
+      sDk[o] += col;
+      sDc[o] -= sK[o] * col;
+    }
+  }
+  __syncthreads();
+}
+
+template <int K, int C, bool PRECISE, bool USE_MMA>
+__device__ void factored_terms(const float* sK, const float* sQ, const float* sC, const float* sdA,
+                               const float* sdP, float* sE1, float* sE2o, float* sE2d, int* sFlag,
+                               float* sDq, float* sDk, float* sDc) {
+  constexpr int NB = C / BS;
+  for (int J = 0; J < NB; ++J) {
+    const bool pairwise = block_factors<K, C, PRECISE>(J, sC, sE1, sE2o, sE2d, sFlag);
+    if (USE_MMA && !pairwise)
+      factored_block_mma<K, C>(J, sK, sQ, sdA, sdP, sE1, sE2o, sE2d, sDq, sDk, sDc);
+    else
+      factored_block_scalar<K, C, PRECISE>(J, pairwise, sK, sQ, sC, sdA, sdP, sE1, sE2o, sE2d, sDq, sDk, sDc);
+  }
+}
+
 }  // namespace kda

@@ -9,6 +9,12 @@ namespace kda {
 constexpr int FWD_CHUNK = 32;    // chunk length of the chunked kernels
 constexpr int FWD_VBLOCK = 32;   // V columns per CTA in the chunked kernels
 
+// Per-(b, hv, 64-step chunk) record of the tensor-core backward (floats):
+// Ah [64][64], [dP; dA] [128][64], [dQE; dKE'] [128][128], dKEd [64][128],
+// dbeta_R [64], dEl [128].
+constexpr int G_AH = 0, G_PA = 4096, G_QK = 12288, G_KED = 28672, G_DBR = 36864, G_DEL = 36928,
+              GREC = 37120;
+
 struct FwdArgs {
   const void *q, *k, *v;
   const float *g, *beta, *S0;
@@ -27,6 +33,7 @@ struct BwdArgs {
   void *dq, *dk, *dv;    // dtype of q/k/v
   float *dg, *dbeta, *dS0;
   float *dq_part, *dk_part;  // fp32 [B, T, HV, K] per value head when HV > H, else null
+  float* gws;                // per-chunk records of the tensor-core backward (K = V = 128), else null
   float scale;
   int B, T, H, HV, K, V;
 };
@@ -52,6 +59,7 @@ size_t fwd_smem_bytes(int K);
 int launch_bwd(const BwdArgs& a, int dtype, cudaStream_t stream);
 bool bwd_tc_eligible(const BwdArgs& a, int dtype);
 int launch_bwd_dstate_tc(const BwdArgs& a, cudaStream_t stream);
+int launch_bwd_grads_tc(const BwdArgs& a, cudaStream_t stream);
 int launch_decode(const DecodeArgs& a, int K, int V, int dtype, cudaStream_t stream);
 
 }  // namespace kda
