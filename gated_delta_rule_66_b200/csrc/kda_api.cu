@@ -72,7 +72,11 @@ const char* kda_last_error(void) { return g_err; }
 
 int kda_device_status(unsigned* flags) {
   if (!flags) return set_error(KDA_ERR_NULL, "kda_device_status: flags must be non-NULL");
-  return take_device_error(flags);
+  unsigned f1 = 0, f2 = 0;
+  int rc = take_device_error(&f1);
+  if (!rc) rc = take_bwd_device_error(&f2);
+  *flags = f1 | f2;
+  return rc;
 }
 
 size_t kda_fwd_workspace_bytes(int B, int T, int HV, int K, int V) {

@@ -170,7 +170,7 @@ template <int K, int C, int VB, typename TIn>
 __global__ void __launch_bounds__(NTHREADS, 1) kda_bwd_grads_kernel(BwdArgs a) {
   using S = GradSmem<K, C, VB>;
   constexpr bool PRECISE = sizeof(TIn) == 4;
-  constexpr int LDK = S::LDK, LDC = S::LDC, LDV = S::LDV, NB = C / BS;
+  constexpr int LDK = S::LDK, LDC = S::LDC, LDV = S::LDV;
   extern __shared__ float smem[];
   float *sK = smem + S::oK, *sQ = smem + S::oQ, *sC = smem + S::oC, *sE = smem + S::oE,
         *sEd = smem + S::oEd, *sAh = smem + S::oAh, *sT = smem + S::oT, *sP = smem + S::oP,

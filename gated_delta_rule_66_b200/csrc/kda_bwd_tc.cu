@@ -25,7 +25,7 @@
 
 namespace kda {
 
-extern __device__ unsigned int g_kda_device_error;
+__device__ unsigned int g_kda_bwd_device_error;  // this file's kernels (one flag per translation unit)
 
 namespace tcb {
 using namespace tcc;
@@ -246,7 +246,7 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_dstate_tc_kernel(BwdArgs a) {
   fence_before();
   __syncthreads();
   if (cx.warp == 0) tmem_dealloc(tm, 512);
-  if (failed && tid == 0) atomicOr(&g_kda_device_error, 1u);
+  if (failed && tid == 0) atomicOr(&g_kda_bwd_device_error, 1u);
 }
 
 bool bwd_tc_eligible(const BwdArgs& a, int dtype) {
@@ -549,7 +549,7 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
   fence_before();
   __syncthreads();
   if (cx.warp == 0) tmem_dealloc(tm, 512);
-  if (failed && tid == 0) atomicOr(&g_kda_device_error, 1u);
+  if (failed && tid == 0) atomicOr(&g_kda_bwd_device_error, 1u);
 }
 
 int launch_bwd_grads_tc(const BwdArgs& a, cudaStream_t stream) {
@@ -563,4 +563,16 @@ int launch_bwd_grads_tc(const BwdArgs& a, cudaStream_t stream) {
   return 0;
 }
 
+}  // namespace kda
+
+namespace kda {
+int take_bwd_device_error(unsigned* out) {
+  unsigned v = 0, zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_kda_bwd_device_error, sizeof(v));
+  if (e != cudaSuccess) return set_cuda_error("kda_device_status", e);
+  e = cudaMemcpyToSymbol(g_kda_bwd_device_error, &zero, sizeof(zero));
+  if (e != cudaSuccess) return set_cuda_error("kda_device_status", e);
+  *out = v;
+  return 0;
+}
 }  // namespace kda

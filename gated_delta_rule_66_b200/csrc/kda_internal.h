@@ -55,6 +55,7 @@ int launch_fwd(const FwdArgs& a, int dtype, cudaStream_t stream);
 bool fwd_tc_eligible(const FwdArgs& a, int dtype);
 int launch_fwd_tc(const FwdArgs& a, cudaStream_t stream);
 int take_device_error(unsigned* out);
+int take_bwd_device_error(unsigned* out);
 size_t fwd_smem_bytes(int K);
 int launch_bwd(const BwdArgs& a, int dtype, cudaStream_t stream);
 bool bwd_tc_eligible(const BwdArgs& a, int dtype);
