@@ -416,41 +416,68 @@ __global__ void kda_group_sum_kernel(const float* __restrict__ part, TIn* __rest
 // dKEd o e^{c_last-c}; dc = (dQE o q~ + dKE o k) o e^c - dKEd o k o e^{c_last-c};
 // then the interaction terms (factored_terms) and dg = reverse cumsum of dc.
 // Everything here is independent across key channels, so one CTA handles one
-// (b, hv, chunk, half of the 128 key channels).
+// (b, hv, chunk, quarter of the 128 key channels); two CTAs fit on an SM.
 struct AsmSmem {
-  static constexpr int C = 64, KH = 64, LDK = KH + 1, LDC = C + 1;
+  static constexpr int C = 64, KQ = 32, LDK = KQ + 1, LDC = C + 1;
   static constexpr int oK = 0, oQ = oK + C * LDK, oC = oQ + C * LDK, oDq = oC + C * LDK, oDk = oDq + C * LDK,
                        oDc = oDk + C * LDK, oE1 = oDc + C * LDK, oE2o = oE1 + C * LDK, oE2d = oE2o + BS * LDK,
-                       oAh = oE2d + BS * LDK, odA = oAh + C * LDC, odP = odA + C * LDC, oBeta = odP + C * LDC,
-                       oLast = oBeta + C, oFlag = oLast + KH, total = oFlag + 4;
+                       odA = oE2d + BS * LDK, odP = odA + C * LDC, oBeta = odP + C * LDC, oSeg = oBeta + C,
+                       oLast = oSeg + 8 * KQ, oFlag = oLast + KQ, total = oFlag + 4;
   static constexpr size_t bytes = (size_t)total * sizeof(float);
 };
 
+// Inclusive (forward) or reverse cumulative sum over the C = 64 rows of each
+// of the KQ = 32 columns of a [64][LDK] array, by 8 segments of 8 rows
+// (256 threads; seg is 8 x KQ scratch; `base` is added to every element of a
+// reverse sum).  Ends with a barrier.
+template <bool REVERSE>
+__device__ __forceinline__ void cumsum64(float* a, float* seg, const float* base) {
+  constexpr int LDK = AsmSmem::LDK, KQ = AsmSmem::KQ;
+  const int f = threadIdx.x % KQ, sg = threadIdx.x / KQ;  // 8 segments
+  float v[8], run = 0.f;
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    const int i = REVERSE ? (63 - (sg * 8 + r)) : (sg * 8 + r);
+    run += a[i * LDK + f];
+    v[r] = run;
+  }
+  seg[sg * KQ + f] = run;
+  __syncthreads();
+  float carry = REVERSE && base ? base[f] : 0.f;
+  for (int s2 = 0; s2 < sg; ++s2) carry += seg[s2 * KQ + f];
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    const int i = REVERSE ? (63 - (sg * 8 + r)) : (sg * 8 + r);
+    a[i * LDK + f] = v[r] + carry;
+  }
+  __syncthreads();
+}
+
 template <typename TIn>
-__global__ void __launch_bounds__(NTHREADS, 1) kda_bwd_assemble_kernel(BwdArgs a) {
+__global__ void __launch_bounds__(NTHREADS, 2) kda_bwd_assemble_kernel(BwdArgs a) {
   using S = AsmSmem;
-  constexpr int C = S::C, KH = S::KH, LDK = S::LDK, LDC = S::LDC, KD = 128;
+  constexpr int C = S::C, KQ = S::KQ, LDK = S::LDK, LDC = S::LDC, KD = 128;
   extern __shared__ float smem[];
   float *sK = smem + S::oK, *sQ = smem + S::oQ, *sC = smem + S::oC, *sDq = smem + S::oDq,
         *sDk = smem + S::oDk, *sDc = smem + S::oDc, *sE1 = smem + S::oE1, *sE2o = smem + S::oE2o,
-        *sE2d = smem + S::oE2d, *sAh = smem + S::oAh, *sdA = smem + S::odA, *sdP = smem + S::odP,
-        *sBeta = smem + S::oBeta, *sLast = smem + S::oLast;
+        *sE2d = smem + S::oE2d, *sdA = smem + S::odA, *sdP = smem + S::odP, *sBeta = smem + S::oBeta,
+        *sSeg = smem + S::oSeg, *sLast = smem + S::oLast;
   int* sFlag = reinterpret_cast<int*>(smem + S::oFlag);
-  const int ch = blockIdx.x >> 1, fh = blockIdx.x & 1, hv = blockIdx.y, b = blockIdx.z;
+  const int ch = blockIdx.x >> 2, fq4 = blockIdx.x & 3, hv = blockIdx.y, b = blockIdx.z;
   const int G = a.HV / a.H, h = hv / G, T = a.T, NT = (T + C - 1) / C;
-  const int t0 = ch * C, L = min(C, T - t0), f0 = fh * KH;
+  const int t0 = ch * C, L = min(C, T - t0), f0 = fq4 * KQ;
   const size_t head = (size_t)b * a.HV + hv;
   const float* rec = a.gws + (head * NT + ch) * GREC;
   const TIn* q = static_cast<const TIn*>(a.q);
   const TIn* k = static_cast<const TIn*>(a.k);
+  const int tid = threadIdx.x;
 
-  // inputs of this channel half: 4 channels per item, all loads issued before use
-  {
-    float4 gv[4];
-    float qv[4][4], kv[4][4];
+  {  // inputs of this channel quarter (4 channels per item) and the C x C adjoints; loads first
+    float4 gv[2], dp[4], da[4];
+    float qv[2][4], kv[2][4];
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const int idx = threadIdx.x + m * NTHREADS, i = idx >> 4, f4 = (idx & 15) * 4;
+    for (int m = 0; m < 2; ++m) {
+      const int idx = tid + m * NTHREADS, i = idx >> 3, f4 = (idx & 7) * 4;
       gv[m] = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int u = 0; u < 4; ++u) qv[m][u] = kv[m][u] = 0.f;
@@ -465,8 +492,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) kda_bwd_assemble_kernel(BwdArgs a
       }
     }
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const int idx = threadIdx.x + m * NTHREADS, i = idx >> 4, f4 = (idx & 15) * 4;
+    for (int m = 0; m < 4; ++m) {  // column j of [dP; dA], four rows per item
+      const int idx = tid + m * NTHREADS, j = idx >> 4, i4 = (idx & 15) * 4;
+      dp[m] = *reinterpret_cast<const float4*>(rec + G_PA + j * 128 + i4);
+      da[m] = *reinterpret_cast<const float4*>(rec + G_PA + j * 128 + 64 + i4);
+    }
+    if (tid < C) sBeta[tid] = (tid < L) ? a.beta[((size_t)b * T + t0 + tid) * a.HV + hv] : 0.f;
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+      const int idx = tid + m * NTHREADS, i = idx >> 3, f4 = (idx & 7) * 4;
       const float gg[4] = {gv[m].x, gv[m].y, gv[m].z, gv[m].w};
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
@@ -475,69 +509,58 @@ __global__ void __launch_bounds__(NTHREADS, 1) kda_bwd_assemble_kernel(BwdArgs a
         sC[i * LDK + f4 + u] = gg[u];
       }
     }
-  }
-  for (int i = threadIdx.x; i < C; i += NTHREADS)
-    sBeta[i] = (i < L) ? a.beta[((size_t)b * T + t0 + i) * a.HV + hv] : 0.f;
-  {  // Ah, dP, dA (float4 rows of the record)
-    float4 ah[4], dp[4], da[4];
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
-      const int idx = threadIdx.x + m * NTHREADS, i = idx >> 4, j4 = (idx & 15) * 4;
-      ah[m] = *reinterpret_cast<const float4*>(rec + G_AH + i * 64 + j4);
-      dp[m] = *reinterpret_cast<const float4*>(rec + G_PA + i * 64 + j4);
-      da[m] = *reinterpret_cast<const float4*>(rec + G_PA + (64 + i) * 64 + j4);
-    }
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const int idx = threadIdx.x + m * NTHREADS, i = idx >> 4, j4 = (idx & 15) * 4;
-      const float vah[4] = {ah[m].x, ah[m].y, ah[m].z, ah[m].w}, vdp[4] = {dp[m].x, dp[m].y, dp[m].z, dp[m].w},
-                  vda[4] = {da[m].x, da[m].y, da[m].z, da[m].w};
+      const int idx = tid + m * NTHREADS, j = idx >> 4, i4 = (idx & 15) * 4;
+      const float vdp[4] = {dp[m].x, dp[m].y, dp[m].z, dp[m].w}, vda[4] = {da[m].x, da[m].y, da[m].z, da[m].w};
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const int j = j4 + u;
-        sAh[i * LDC + j] = vah[u];
+        const int i = i4 + u;
         sdP[i * LDC + j] = (j <= i) ? vdp[u] : 0.f;
         sdA[i * LDC + j] = (j < i) ? vda[u] : 0.f;
       }
     }
   }
   __syncthreads();
-  for (int f = threadIdx.x; f < KH; f += NTHREADS) {
-    float run = 0.f;
-    for (int i = 0; i < C; ++i) {
-      run += sC[i * LDK + f];
-      sC[i * LDK + f] = run;
+  cumsum64<false>(sC, sSeg, nullptr);
+  if (fq4 == 0 && tid < L) {  // dbeta = dbeta_R + sum_{j<i} dA_ij Ah_ij (Ah read straight from the record)
+    const int i = tid;
+    const float4* arow = reinterpret_cast<const float4*>(rec + G_AH + i * 64);
+    float s0 = rec[G_DBR + i], s1 = 0.f;
+    for (int j4 = 0; j4 < 16; ++j4) {
+      const float4 ah = arow[j4];
+      const float vah[4] = {ah.x, ah.y, ah.z, ah.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = j4 * 4 + u;
+        if (u & 1) s1 = fmaf(sdA[i * LDC + j], vah[u], s1);
+        else s0 = fmaf(sdA[i * LDC + j], vah[u], s0);
+      }
     }
-  }
-  if (fh == 0) {
-    for (int i = threadIdx.x; i < L; i += NTHREADS) {
-      float s = rec[G_DBR + i];
-      for (int j = 0; j < i; ++j) s = fmaf(sdA[i * LDC + j], sAh[i * LDC + j], s);
-      a.dbeta[((size_t)b * T + t0 + i) * a.HV + hv] = s;
-    }
+    a.dbeta[((size_t)b * T + t0 + i) * a.HV + hv] = s0 + s1;
   }
   __syncthreads();
-  for (int idx = threadIdx.x; idx < C * C; idx += NTHREADS) {
+  for (int idx = tid; idx < C * C; idx += NTHREADS) {
     const int i = idx >> 6, j = idx & 63;
     sdA[i * LDC + j] *= sBeta[i];
   }
   {  // element-wise terms; the chunk-end sum of dKEd o k o e^{c_last-c} goes through sE1
-    float4 qe[4], ke[4], kd[4];
+    float4 qe[2], ke[2], kd[2];
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const int idx = threadIdx.x + m * NTHREADS, i = idx >> 4, f4 = (idx & 15) * 4;
-      qe[m] = *reinterpret_cast<const float4*>(rec + G_QK + i * 128 + f0 + f4);
-      ke[m] = *reinterpret_cast<const float4*>(rec + G_QK + (64 + i) * 128 + f0 + f4);
-      kd[m] = *reinterpret_cast<const float4*>(rec + G_KED + i * 128 + f0 + f4);
+    for (int m = 0; m < 2; ++m) {  // channel f of the quarter, four rows per item
+      const int idx = tid + m * NTHREADS, f = idx >> 4, i4 = (idx & 15) * 4;
+      qe[m] = *reinterpret_cast<const float4*>(rec + G_QK + (f0 + f) * 128 + i4);
+      ke[m] = *reinterpret_cast<const float4*>(rec + G_QK + (f0 + f) * 128 + 64 + i4);
+      kd[m] = *reinterpret_cast<const float4*>(rec + G_KED + (f0 + f) * 64 + i4);
     }
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const int idx = threadIdx.x + m * NTHREADS, i = idx >> 4, f4 = (idx & 15) * 4;
+    for (int m = 0; m < 2; ++m) {
+      const int idx = tid + m * NTHREADS, f = idx >> 4, i4 = (idx & 15) * 4;
       const float vq[4] = {qe[m].x, qe[m].y, qe[m].z, qe[m].w}, vk[4] = {ke[m].x, ke[m].y, ke[m].z, ke[m].w},
                   vd[4] = {kd[m].x, kd[m].y, kd[m].z, kd[m].w};
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const int f = f4 + u, o = i * LDK + f;
+        const int i = i4 + u, o = i * LDK + f;
         const float c = sC[o], e = __expf(c), ed = __expf(sC[(C - 1) * LDK + f] - c);
         const float dqe = vq[u], dke = sBeta[i] * vk[u], dked = vd[u];
         const float kk = sK[o], qq = sQ[o];
@@ -549,25 +572,26 @@ __global__ void __launch_bounds__(NTHREADS, 1) kda_bwd_assemble_kernel(BwdArgs a
     }
   }
   __syncthreads();
-  for (int f = threadIdx.x; f < KH; f += NTHREADS) {
-    float s = rec[G_DEL + f0 + f] * __expf(sC[(C - 1) * LDK + f]);
-    for (int i = 0; i < C; ++i) s += sE1[i * LDK + f];
-    sLast[f] = s;
-  }
-  __syncthreads();
-  factored_terms<KH, C, false, true>(sK, sQ, sC, sdA, sdP, sE1, sE2o, sE2d, sFlag, sDq, sDk, sDc);
-  for (int f = threadIdx.x; f < KH; f += NTHREADS) {
-    float run = sLast[f];
-    for (int i = C - 1; i >= 0; --i) {
-      run += sDc[i * LDK + f];
-      sDc[i * LDK + f] = run;
+  {  // chunk-end terms: dEl o e^{c_last} + sum_i dKEd o k o e^{c_last - c}
+    const int f = tid % KQ, sg = tid / KQ;
+    float s = 0.f;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) s += sE1[(sg * 8 + r) * LDK + f];
+    sSeg[sg * KQ + f] = s;
+    __syncthreads();
+    if (tid < KQ) {
+      float t = rec[G_DEL + f0 + tid] * __expf(sC[(C - 1) * LDK + tid]);
+      for (int s2 = 0; s2 < 8; ++s2) t += sSeg[s2 * KQ + tid];
+      sLast[tid] = t;
     }
+    __syncthreads();
   }
-  __syncthreads();
+  factored_terms<KQ, C, false, true>(sK, sQ, sC, sdA, sdP, sE1, sE2o, sE2d, sFlag, sDq, sDk, sDc);
+  cumsum64<true>(sDc, sSeg, sLast);
   TIn* dq = static_cast<TIn*>(a.dq);
   TIn* dk = static_cast<TIn*>(a.dk);
-  for (int idx = threadIdx.x; idx < L * KH; idx += NTHREADS) {
-    const int i = idx / KH, f = idx % KH, o = i * LDK + f;
+  for (int idx = tid; idx < L * KQ; idx += NTHREADS) {
+    const int i = idx / KQ, f = idx % KQ, o = i * LDK + f;
     const size_t row_v = ((size_t)b * T + t0 + i) * a.HV + hv;
     a.dg[row_v * KD + f0 + f] = sDc[o];
     if (G == 1) {
@@ -587,7 +611,7 @@ static int launch_assemble(const BwdArgs& a, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)AsmSmem::bytes);
   if (e != cudaSuccess) return set_cuda_error("kda_bwd: cudaFuncSetAttribute", e);
   const int NT = (a.T + 63) / 64;
-  kern<<<dim3(NT * 2, a.HV, a.B), NTHREADS, AsmSmem::bytes, stream>>>(a);
+  kern<<<dim3(NT * 4, a.HV, a.B), NTHREADS, AsmSmem::bytes, stream>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return set_cuda_error("kda_bwd: assemble launch", e);
   return 0;

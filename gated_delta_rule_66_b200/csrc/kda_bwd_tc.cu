@@ -528,17 +528,17 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
       float v[32];
       tmem_ld32(tm + lo + TM_PA + hcol * 32, v);
 #pragma unroll
-      for (int jj = 0; jj < 32; ++jj) rec[G_PA + Lr * 64 + hcol * 32 + jj] = v[jj];
+      for (int jj = 0; jj < 32; ++jj) rec[G_PA + (hcol * 32 + jj) * 128 + Lr] = v[jj];
       for (int cb = 0; cb < 2; ++cb) {
         const int f0 = hcol * 64 + cb * 32;
         tmem_ld32(tm + lo + TM_QK + f0, v);
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) rec[G_QK + Lr * 128 + f0 + jj] = v[jj];
+        for (int jj = 0; jj < 32; ++jj) rec[G_QK + (f0 + jj) * 128 + Lr] = v[jj];
         tmem_ld32(tm + lo + TM_KED + f0, v);
         if (lane < 16) {
           const int r = cx.sub * 16 + lane;  // M = 64 accumulator layout
 #pragma unroll
-          for (int jj = 0; jj < 32; ++jj) rec[G_KED + r * 128 + f0 + jj] = v[jj];
+          for (int jj = 0; jj < 32; ++jj) rec[G_KED + (f0 + jj) * 64 + r] = v[jj];
         }
       }
       if (tid < C) rec[G_DBR + tid] = sDbR[tid];

@@ -9,8 +9,10 @@ namespace kda {
 constexpr int FWD_CHUNK = 32;    // chunk length of the chunked kernels
 constexpr int FWD_VBLOCK = 32;   // V columns per CTA in the chunked kernels
 
-// Per-(b, hv, 64-step chunk) record of the tensor-core backward (floats):
-// Ah [64][64], [dP; dA] [128][64], [dQE; dKE'] [128][128], dKEd [64][128],
+// Per-(b, hv, 64-step chunk) record of the tensor-core backward (floats),
+// column-major so that the TMEM lanes (rows) are contiguous:
+// Ah [i][j] (row-major 64 x 64), [dP; dA] as [j][i'] (64 x 128, i' < 64 dP),
+// [dQE; dKE'] as [f][i'] (128 x 128, i' < 64 dQE), dKEd as [f][i] (128 x 64),
 // dbeta_R [64], dEl [128].
 constexpr int G_AH = 0, G_PA = 4096, G_QK = 12288, G_KED = 28672, G_DBR = 36864, G_DEL = 36928,
               GREC = 37120;
