@@ -586,7 +586,17 @@ __global__ void __launch_bounds__(NTHREADS, 2) kda_bwd_assemble_kernel(BwdArgs a
     }
     __syncthreads();
   }
-  factored_terms<KQ, C, false, true>(sK, sQ, sC, sdA, sdP, sE1, sE2o, sE2d, sFlag, sDq, sDk, sDc);
+  {  // split exponents hold when every 16-row block's decay span is at most 80
+    bool wide = false;
+    if (tid < 4 * KQ) {
+      const int J = tid / KQ, f = tid % KQ;
+      wide = sC[(16 * J) * LDK + f] - sC[(16 * J + 15) * LDK + f] > DIAG_SPAN_MAX;
+    }
+    if (__syncthreads_or(wide))
+      factored_terms<KQ, C, false, false>(sK, sQ, sC, sdA, sdP, sE1, sE2o, sE2d, sFlag, sDq, sDk, sDc);
+    else
+      factored_terms_fused<KQ>(sK, sQ, sC, sdA, sdP, sDq, sDk, sDc);
+  }
   cumsum64<true>(sDc, sSeg, sLast);
   TIn* dq = static_cast<TIn*>(a.dq);
   TIn* dk = static_cast<TIn*>(a.dk);
