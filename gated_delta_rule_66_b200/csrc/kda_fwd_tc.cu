@@ -105,41 +105,42 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_tc_kernel(FwdArgs a) {
     if (!wait_mma(bar, phase)) { failed = true; break; }
 
     // ---------------------------------------------------------------- state-product operands
-    const int fq = item_f(cx);
-    {
-      const float4 c63v = ld4(sC + 63 * LDCF + fq), r31 = ld4(sC + 31 * LDCF + fq);
-      const float c63[4] = {c63v.x, c63v.y, c63v.z, c63v.w}, c31[4] = {r31.x, r31.y, r31.z, r31.w};
+    {  // Q~ o e^c as [i][f]: thread items of 4 channels, 16-byte stores
+      const int fq = item_f(cx);
       for (int m = 0; m < 8; ++m) {
         const int i = item_row(cx, m);
         const float4 c4 = ld4(sC + i * LDCF + fq);
-        const float c[4] = {c4.x, c4.y, c4.z, c4.w};
-        float kf[4], qf[4], vf[4];
-        bf16x4(sm + RAW_K + i * 256 + fq * 2, kf);
+        float qf[4];
         bf16x4(sm + RAW_Q + i * 256 + fq * 2, qf);
-        bf16x4(sm + RAW_X + i * 256 + fq * 2, vf);
-        const float bi = sBeta[i];
-        float e[4], ed[4];
+        st_tf32x4(sm, OP_QE + kmaj(i, fq, 128), a.scale * qf[0] * ex2(c4.x), a.scale * qf[1] * ex2(c4.y),
+                  a.scale * qf[2] * ex2(c4.z), a.scale * qf[3] * ex2(c4.w));
+      }
+    }
+    {  // transposed operands [f][i]: thread items of one channel x 4 rows, 16-byte stores
+      const int f = tid & 127;
+      const float c63 = sC[63 * LDCF + f], c31 = sC[31 * LDCF + f];
+      const __nv_bfloat16* kcol = reinterpret_cast<const __nv_bfloat16*>(sm + RAW_K) + f;
+      const __nv_bfloat16* vcol = reinterpret_cast<const __nv_bfloat16*>(sm + RAW_X) + f;
+      for (int m = 0; m < 8; ++m) {
+        const int i0 = ((tid >> 7) + 2 * m) * 4;
+        float bke[4], ked[4], bv[4], kmid[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          e[u] = ex2(c[u]);
-          ed[u] = ex2(c63[u] - c[u]);
+          const int i = i0 + u;
+          const float c = sC[i * LDCF + f], kk = __bfloat162float(kcol[i * 128]), bi = sBeta[i];
+          bke[u] = bi * kk * ex2(c);
+          ked[u] = kk * ex2(c63 - c);
+          bv[u] = bi * __bfloat162float(vcol[i * 128]);
+          if (a.states && i0 < 32) kmid[u] = kk * ex2(c31 - c);
         }
-        st_tf32x4(sm, OP_QE + kmaj(i, fq, 128), a.scale * qf[0] * e[0], a.scale * qf[1] * e[1],
-                  a.scale * qf[2] * e[2], a.scale * qf[3] * e[3]);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          st_tf32(sm, OP_BKET + kmaj(fq + u, i, 64), bi * kf[u] * e[u]);
-          st_tf32(sm, OP_KEDT + kmaj(fq + u, i, 64), kf[u] * ed[u]);
-          st_tf32(sm, OP_BVT + kmaj(fq + u, i, 64), bi * vf[u]);
-        }
-        if (a.states && i < 32) {  // (K o e^{c_31 - c})^T over the first half: the mid-chunk state
-#pragma unroll
-          for (int u = 0; u < 4; ++u) st_tf32(sm, OP_KMID + kmaj(fq + u, i, 32), kf[u] * ex2(c31[u] - c[u]));
-        }
+        st_tf32x4(sm, OP_BKET + kmaj(f, i0, 64), bke[0], bke[1], bke[2], bke[3]);
+        st_tf32x4(sm, OP_KEDT + kmaj(f, i0, 64), ked[0], ked[1], ked[2], ked[3]);
+        st_tf32x4(sm, OP_BVT + kmaj(f, i0, 64), bv[0], bv[1], bv[2], bv[3]);
+        if (a.states && i0 < 32) st_tf32x4(sm, OP_KMID + kmaj(f, i0, 32), kmid[0], kmid[1], kmid[2], kmid[3]);
       }
       if (tid < KD) {
-        sEl[tid] = ex2(sC[63 * LDCF + tid]);
-        sE31[tid] = ex2(sC[31 * LDCF + tid]);
+        sEl[tid] = ex2(c63);
+        sE31[tid] = ex2(c31);
       }
     }
     Pairwise pw;
@@ -175,7 +176,7 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_tc_kernel(FwdArgs a) {
       float v[32];
       tmem_ld32(tm + lo + TM_W + hcol * 32, v);
 #pragma unroll
-      for (int jj = 0; jj < 32; ++jj) st_tf32(sm, R_WOP + kmaj(hcol * 32 + jj, Lr, 128), v[jj]);
+      for (int jj = 0; jj < 32; ++jj) st_tf32(sm, R_WOP + kmaj_pad(hcol * 32 + jj, Lr, 128), v[jj]);
     }
     fence_async_smem();
     __syncthreads();
@@ -183,7 +184,7 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_tc_kernel(FwdArgs a) {
       fence_after();
       const uint32_t id = idesc_tf32(128, 64);
       for (int ks = 0; ks < 16; ++ks) {
-        mma_ts(tm + TM_X, tm + TM_S + ks * 8, desc(sb + R_WOP + ks * 256, 4096), id, ks > 0);
+        mma_ts(tm + TM_X, tm + TM_S + ks * 8, desc(sb + R_WOP + ks * 288, 4608, 144), id, ks > 0);
         mma_ts(tm + TM_O, tm + TM_S + ks * 8, desc(sb + OP_QE + ks * 256, 4096), id, ks > 0);
       }
       commit(bar);

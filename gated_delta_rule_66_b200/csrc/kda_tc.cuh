@@ -25,11 +25,18 @@ __device__ __forceinline__ uint32_t kmaj(int r, int k, int kt) {
   return (uint32_t)((r >> 3) * (kt * 32) + (k >> 2) * 128 + (r & 7) * 16 + (k & 3) * 4);
 }
 
+// The same layout with K-adjacent core matrices 144 bytes apart (LBO = 144,
+// SBO = KT * 36): a warp whose lanes hold 32 consecutive k of one row stores
+// into 32 distinct banks.  A K step then advances the start by 288 bytes.
+__device__ __forceinline__ uint32_t kmaj_pad(int r, int k, int kt) {
+  return (uint32_t)((r >> 3) * (kt * 36) + (k >> 2) * 144 + (r & 7) * 16 + (k & 3) * 4);
+}
+
 // shared-memory matrix descriptor (no swizzle, version 1 for sm_100)
-__device__ __forceinline__ uint64_t desc(uint32_t saddr, uint32_t sbo) {
+__device__ __forceinline__ uint64_t desc(uint32_t saddr, uint32_t sbo, uint32_t lbo = 128) {
   uint64_t d = 0;
   d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
-  d |= (uint64_t)((128u >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
   d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
   d |= (uint64_t)1 << 46;
   return d;

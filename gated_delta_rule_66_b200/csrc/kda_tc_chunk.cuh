@@ -43,8 +43,8 @@ constexpr uint32_t S_BETA = SMALL, S_EL = SMALL + 256, S_EMID = S_EL + 512, S_CA
                    S_BAR = S_CARRY + 512, S_TMEM = S_BAR + 8, SMEM_BYTES = S_TMEM + 16;
 constexpr float LOG2E = 1.4426950408889634f;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-static_assert(R_T + 16384 <= OP && R_P + 16384 <= R_T && R_WOP + 32768 <= R_SW && R_SW + 3072 <= R_P,
-              "raw-region reuse");
+static_assert(R_T + 16384 <= OP && R_P + 16384 <= R_T && R_SW + 3072 <= R_P && R_WOP + 36864 <= R_P,
+              "raw-region reuse (the padded W overlaps only the dead inverse scratch)");
 
 struct Ctx {
   unsigned char* sm;
@@ -280,19 +280,20 @@ __device__ __forceinline__ void readout_ap(const Ctx& c, uint32_t tm_apa, uint32
 // T = (I + diag(beta) Ah)^-1 for the 64 x 64 unit lower-triangular system,
 // row-major at R_TROW (stride 65).  The four 16 x 16 diagonal blocks are
 // solved by forward substitution with a whole column per thread in
-// registers; the blocks below them follow in three levels of block
-// substitution, T_IJ = -T_II sum_{J<=L<I} A_IL T_LJ, one level per block
-// distance I - J (each level's blocks are independent).
+// registers; the blocks below follow in three levels of block substitution,
+// T_IJ = -T_II sum_{J<=L<I} A_IL T_LJ (level = block distance I - J), one
+// warp per block, as 3xTF32 warp MMAs (fp32-accurate).
 __device__ __forceinline__ void invert(const Ctx& c) {
   constexpr int LD = 65;
   const float* sAh = reinterpret_cast<const float*>(c.sm + R_AH);
   float* sT = reinterpret_cast<float*>(c.sm + R_TROW);
-  float* sW = reinterpret_cast<float*>(c.sm + R_SW);  // 3 blocks of 16 x 16
+  float* sW = reinterpret_cast<float*>(c.sm + R_SW);  // one 16 x 16 scratch per warp (3 warps)
   const float* sB = c.beta();
   const int tid = c.tid;
-  for (int x = tid; x < 64 * 64; x += NTH) {
-    const int i = x >> 6, j = x & 63;
-    if ((i >> 4) != (j >> 4)) sT[i * LD + j] = 0.f;  // diagonal blocks are written below
+  for (int x = tid; x < 6 * 256; x += NTH) {  // strictly upper blocks
+    const int blk = x >> 8, r = (x >> 4) & 15, col = x & 15;
+    const int I = blk < 3 ? 0 : (blk < 5 ? 1 : 2), J = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+    sT[(16 * I + r) * LD + 16 * J + col] = 0.f;
   }
   if (tid < 64) {
     const int o = (tid >> 4) * 16, col = tid & 15;
@@ -311,32 +312,57 @@ __device__ __forceinline__ void invert(const Ctx& c) {
     for (int r = 0; r < 16; ++r) sT[(o + r) * LD + o + col] = t[r];
   }
   __syncthreads();
+  const int warp = c.warp, g = c.lane >> 2, t4 = c.lane & 3;
   for (int d = 1; d < 4; ++d) {
-    const int nb = 4 - d;
-    // W = sum_{L=J}^{I-1} diag(beta_I) Ah_IL T_LJ for the blocks (I, J) = (J + d, J)
-    for (int x = tid; x < nb * 256; x += NTH) {
-      const int J = x >> 8, r = (x >> 4) & 15, col = x & 15, I = J + d;
-      const float* arow = sAh + (16 * I + r) * LD;
-      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-      for (int l = 16 * J; l < 16 * I; l += 4) {
-        a0 = fmaf(arow[l], sT[l * LD + 16 * J + col], a0);
-        a1 = fmaf(arow[l + 1], sT[(l + 1) * LD + 16 * J + col], a1);
-        a2 = fmaf(arow[l + 2], sT[(l + 2) * LD + 16 * J + col], a2);
-        a3 = fmaf(arow[l + 3], sT[(l + 3) * LD + 16 * J + col], a3);
+    if (warp < 4 - d) {
+      const int J = warp, I = J + d, ri = 16 * I;
+      // W = sum_{L=J}^{I-1} diag(beta_I) Ah_IL T_LJ  (16 x 16, K = 16 d)
+      float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      const float bg = sB[ri + g], bg8 = sB[ri + g + 8];
+      for (int ks = 0; ks < 2 * d; ++ks) {
+        const int l = 16 * J + 8 * ks + t4;
+        Split a[4];
+        a[0] = split_tf32(bg * sAh[(ri + g) * LD + l]);
+        a[1] = split_tf32(bg8 * sAh[(ri + g + 8) * LD + l]);
+        a[2] = split_tf32(bg * sAh[(ri + g) * LD + l + 4]);
+        a[3] = split_tf32(bg8 * sAh[(ri + g + 8) * LD + l + 4]);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          Split bb[2];
+          bb[0] = split_tf32(sT[l * LD + 16 * J + nt * 8 + g]);
+          bb[1] = split_tf32(sT[(l + 4) * LD + 16 * J + nt * 8 + g]);
+          mma3(acc[nt], a, bb);
+        }
       }
-      sW[J * 256 + r * 16 + col] = sB[16 * I + r] * ((a0 + a1) + (a2 + a3));
-    }
-    __syncthreads();
-    // T_IJ = -T_II W
-    for (int x = tid; x < nb * 256; x += NTH) {
-      const int J = x >> 8, r = (x >> 4) & 15, col = x & 15, I = J + d;
-      const float* trow = sT + (16 * I + r) * LD + 16 * I;
-      float a0 = 0.f, a1 = 0.f;
-      for (int m = 0; m <= r; m += 2) {
-        a0 = fmaf(trow[m], sW[J * 256 + m * 16 + col], a0);
-        if (m + 1 <= r) a1 = fmaf(trow[m + 1], sW[J * 256 + (m + 1) * 16 + col], a1);
+      float* w = sW + warp * 256;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) w[(g + ((e & 2) ? 8 : 0)) * 16 + nt * 8 + 2 * t4 + (e & 1)] = acc[nt][e];
+      __syncwarp();
+      // T_IJ = -T_II W
+      float tt[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+      for (int ks = 0; ks < 2; ++ks) {
+        const int m = 8 * ks + t4;
+        Split a[4];
+        a[0] = split_tf32(sT[(ri + g) * LD + ri + m]);
+        a[1] = split_tf32(sT[(ri + g + 8) * LD + ri + m]);
+        a[2] = split_tf32(sT[(ri + g) * LD + ri + m + 4]);
+        a[3] = split_tf32(sT[(ri + g + 8) * LD + ri + m + 4]);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          Split bb[2];
+          bb[0] = split_tf32(w[m * 16 + nt * 8 + g]);
+          bb[1] = split_tf32(w[(m + 4) * 16 + nt * 8 + g]);
+          mma3(tt[nt], a, bb);
+        }
       }
-      sT[(16 * I + r) * LD + 16 * J + col] = -(a0 + a1);
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          sT[(ri + g + ((e & 2) ? 8 : 0)) * LD + 16 * J + nt * 8 + 2 * t4 + (e & 1)] = -tt[nt][e];
     }
     __syncthreads();
   }
