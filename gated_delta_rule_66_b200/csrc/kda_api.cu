@@ -62,6 +62,17 @@ static size_t states_bytes(int B, int T, int HV, int K, int V) {
 
 static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
+// interaction records stored by the tensor-core forward (K = V = 128)
+static size_t inter_bytes(int B, int T, int HV, int K, int V) {
+  if (K != 128 || V != 128) return 0;
+  const size_t NT64 = (size_t)(T + 63) / 64;
+  return (size_t)B * HV * NT64 * INTER_REC * sizeof(float);
+}
+
+static size_t fwd_ws_bytes(int B, int T, int HV, int K, int V) {
+  return states_bytes(B, T, HV, K, V) + inter_bytes(B, T, HV, K, V);
+}
+
 }  // namespace kda
 
 using namespace kda;
@@ -81,7 +92,7 @@ int kda_device_status(unsigned* flags) {
 
 size_t kda_fwd_workspace_bytes(int B, int T, int HV, int K, int V) {
   if (B < 1 || T < 1 || HV < 1 || K < 1 || V < 1) return 0;
-  return states_bytes(B, T, HV, K, V);
+  return fwd_ws_bytes(B, T, HV, K, V);
 }
 
 static size_t grads_record_bytes(int B, int T, int HV, int K, int V) {
@@ -92,7 +103,7 @@ static size_t grads_record_bytes(int B, int T, int HV, int K, int V) {
 
 size_t kda_bwd_workspace_bytes(int B, int T, int H, int HV, int K, int V) {
   if (B < 1 || T < 1 || H < 1 || HV < 1 || K < 1 || V < 1 || HV % H) return 0;
-  size_t bytes = 2 * states_bytes(B, T, HV, K, V);
+  size_t bytes = fwd_ws_bytes(B, T, HV, K, V) + states_bytes(B, T, HV, K, V);
   if (HV > H) bytes += 2 * (size_t)B * T * HV * K * sizeof(float);
   return bytes + grads_record_bytes(B, T, HV, K, V);
 }
@@ -106,11 +117,14 @@ int kda_fwd(const void* q, const void* k, const void* v, const float* g, const f
   if (!q || !k || !v || !g || !beta || !o)
     return set_error(KDA_ERR_NULL, "kda_fwd: q, k, v, g, beta and o must be non-NULL");
   if (workspace) {
-    if (workspace_bytes < states_bytes(B, T, HV, K, V))
+    if (workspace_bytes < fwd_ws_bytes(B, T, HV, K, V))
       return set_error(KDA_ERR_WORKSPACE, "kda_fwd: workspace smaller than kda_fwd_workspace_bytes()");
     if (!aligned16(workspace)) return set_error(KDA_ERR_ARG, "kda_fwd: workspace must be 16-byte aligned");
   }
-  FwdArgs a{q, k, v, g, beta, S0, o, S_T, static_cast<float*>(workspace), scale, B, T, H, HV, K, V};
+  float* inter = (workspace && inter_bytes(B, T, HV, K, V))
+                     ? reinterpret_cast<float*>(static_cast<char*>(workspace) + states_bytes(B, T, HV, K, V))
+                     : nullptr;
+  FwdArgs a{q, k, v, g, beta, S0, o, S_T, static_cast<float*>(workspace), inter, scale, B, T, H, HV, K, V};
   return launch_fwd(a, dtype, static_cast<cudaStream_t>(stream));
 }
 
@@ -147,9 +161,11 @@ int kda_bwd(const void* q, const void* k, const void* v, const float* g, const f
   const size_t sb = states_bytes(B, T, HV, K, V);
   char* ws = static_cast<char*>(workspace);
   float* states = reinterpret_cast<float*>(ws);
-  float* dstates = reinterpret_cast<float*>(ws + sb);
+  const size_t fb = fwd_ws_bytes(B, T, HV, K, V);
+  float* inter = inter_bytes(B, T, HV, K, V) ? reinterpret_cast<float*>(ws + sb) : nullptr;
+  float* dstates = reinterpret_cast<float*>(ws + fb);
   float *dq_part = nullptr, *dk_part = nullptr;
-  size_t off = 2 * sb;
+  size_t off = fb + sb;
   if (HV > H) {
     dq_part = reinterpret_cast<float*>(ws + off);
     dk_part = dq_part + (size_t)B * T * HV * K;
@@ -157,11 +173,11 @@ int kda_bwd(const void* q, const void* k, const void* v, const float* g, const f
   }
   float* gws = grads_record_bytes(B, T, HV, K, V) ? reinterpret_cast<float*>(ws + off) : nullptr;
   if (!(flags & KDA_BWD_STATES_FROM_FWD)) {
-    FwdArgs fa{q, k, v, g, beta, S0, nullptr, nullptr, states, scale, B, T, H, HV, K, V};
+    FwdArgs fa{q, k, v, g, beta, S0, nullptr, nullptr, states, inter, scale, B, T, H, HV, K, V};
     rc = launch_fwd(fa, dtype, st);
     if (rc) return rc;
   }
-  BwdArgs a{q, k, v, dO, g, beta, dS_T, states, dstates, dq, dk, dv, dg, dbeta, dS0,
+  BwdArgs a{q, k, v, dO, g, beta, dS_T, states, inter, dstates, dq, dk, dv, dg, dbeta, dS0,
             dq_part, dk_part, gws, scale, B, T, H, HV, K, V};
   return launch_bwd(a, dtype, st);
 }

@@ -525,7 +525,7 @@ __global__ void __launch_bounds__(NTHREADS, 2) kda_bwd_assemble_kernel(BwdArgs a
   cumsum64<false>(sC, sSeg, nullptr);
   if (fq4 == 0 && tid < L) {  // dbeta = dbeta_R + sum_{j<i} dA_ij Ah_ij (Ah read straight from the record)
     const int i = tid;
-    const float4* arow = reinterpret_cast<const float4*>(rec + G_AH + i * 64);
+    const float4* arow = reinterpret_cast<const float4*>(a.inter + (head * NT + ch) * INTER_REC + INTER_AH + i * 64);
     float s0 = rec[G_DBR + i], s1 = 0.f;
     for (int j4 = 0; j4 < 16; ++j4) {
       const float4 ah = arow[j4];

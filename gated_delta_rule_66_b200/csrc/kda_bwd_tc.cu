@@ -91,10 +91,9 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_dstate_tc_kernel(BwdArgs a) {
 
   for (int ch = NT - 1; ch >= 0; --ch) {
     const int t0 = ch * C, L = min(C, T - t0);
+    const float* irec = a.inter + (head * NT + ch) * INTER_REC;  // P^T, T of this chunk (forward)
     load_raw(cx, qg, kg, dog, a.g, a.beta, b, T, t0, L, a.H, a.HV, h, hv);
-    const bool wide = cumsum_span(cx);
-    build_op1_and_issue(cx, a.scale, tm + TM_APA, tm + TM_APB, bar);
-    if (!wait_mma(bar, phase)) { failed = true; break; }
+    cumsum_span(cx);
 
     // ---------------------------------------------------------------- operands of the gradient products
     const int fq = item_f(cx);
@@ -145,22 +144,20 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_dstate_tc_kernel(BwdArgs a) {
         tmem_wait_st();
       }
     }
-    Pairwise pw;
-    if (wide) pairwise_compute(cx, a.scale, pw);
     fence_async_smem();
     fence_before();
     __syncthreads();  // raw inputs consumed; the raw region is reused below
-
-    readout_ap(cx, tm + TM_APA, tm + TM_APB, true, wide, pw);  // P^T at R_P
-    invert(cx);
-    {  // (diag(beta) T^T)^T as a K-major operand: element (i, j) = beta_i T[j][i]
-      const float* tr = reinterpret_cast<const float*>(sm + R_TROW);
-      for (int x = tid; x < C * 16; x += NTH) {
-        const int i = x >> 4, j4 = (x & 15) * 4;
-        const float bi = sBeta[i];
-        st_tf32x4(sm, R_T + kmaj(i, j4, 64), bi * tr[j4 * 65 + i], bi * tr[(j4 + 1) * 65 + i],
-                  bi * tr[(j4 + 2) * 65 + i], bi * tr[(j4 + 3) * 65 + i]);
-      }
+    for (int x = tid; x < C * 16; x += NTH) {  // P^T (row i, K j) = P[j][i], from the record's P^T
+      const int i = x >> 4, j4 = (x & 15) * 4;
+      const float4 p = *reinterpret_cast<const float4*>(irec + i * 64 + j4);
+      st_tf32x4(sm, R_P + kmaj(i, j4, 64), p.x, p.y, p.z, p.w);
+    }
+    for (int x = tid; x < C * 16; x += NTH) {  // (diag(beta) T^T)^T: element (i, j) = beta_i T[j][i]
+      const int i = x & 63, j4 = (x >> 6) * 4;
+      const float bi = sBeta[i];
+      const float* tcol = irec + INTER_T + i;
+      st_tf32x4(sm, R_T + kmaj(i, j4, 64), bi * tcol[j4 * 64], bi * tcol[(j4 + 1) * 64], bi * tcol[(j4 + 2) * 64],
+                bi * tcol[(j4 + 3) * 64]);
     }
     fence_async_smem();
     __syncthreads();
@@ -251,8 +248,8 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_dstate_tc_kernel(BwdArgs a) {
 
 bool bwd_tc_eligible(const BwdArgs& a, int dtype) {
   auto al16 = [](const void* p) { return ((uintptr_t)p & 15u) == 0; };
-  return dtype == 1 && a.K == 128 && a.V == 128 && a.gws != nullptr && al16(a.q) && al16(a.k) &&
-         al16(a.dO) && al16(a.g);
+  return dtype == 1 && a.K == 128 && a.V == 128 && a.gws != nullptr && a.inter != nullptr && al16(a.q) &&
+         al16(a.k) && al16(a.v) && al16(a.dO) && al16(a.g);
 }
 
 int launch_bwd_dstate_tc(const BwdArgs& a, cudaStream_t stream) {
@@ -346,9 +343,8 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
   do {
     // ---------------------------------------------------------------- interaction products
     load_raw(cx, qg, kg, dog, a.g, a.beta, b, T, t0, L, a.H, a.HV, h, hv);
-    const bool wide = cumsum_span(cx);
-    build_op1_and_issue(cx, a.scale, tm + TM_APA, tm + TM_APB, bar);
-    if (!wait_mma(bar, phase)) { failed = true; break; }
+    cumsum_span(cx);
+    const float* irec = a.inter + (head * NT + ch) * INTER_REC;  // P^T, T of this chunk (forward)
 
     // ---------------------------------------------------------------- K o e^c, K o e^{c_last-c}, dO, dO^T
     {
@@ -380,28 +376,22 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
       tmem_st32(tm + lo + TM_DOT + hcol * 32, r);
       tmem_wait_st();
     }
-    Pairwise pw;
-    if (wide) pairwise_compute(cx, a.scale, pw);
     fence_async_smem();
     fence_before();
-    __syncthreads();
-
-    readout_ap(cx, tm + TM_APA, tm + TM_APB, true, wide, pw);  // Ah at R_AH, P^T at R_P
-    {
-      const float* sAh = reinterpret_cast<const float*>(sm + R_AH);
-      for (int x = tid; x < C * C; x += NTH) rec[G_AH + x] = sAh[(x >> 6) * 65 + (x & 63)];
+    __syncthreads();  // raw inputs consumed
+    for (int x = tid; x < C * 16; x += NTH) {  // P^T and T diag(beta), (row i, K = j) operands
+      const int i = x >> 4, j4 = (x & 15) * 4;
+      const float4 p = *reinterpret_cast<const float4*>(irec + i * 64 + j4);
+      st_tf32x4(sm, R_P + kmaj(i, j4, 64), p.x, p.y, p.z, p.w);
+      const float4 t = *reinterpret_cast<const float4*>(irec + INTER_T + i * 64 + j4);
+      st_tf32x4(sm, R_T + kmaj(i, j4, 64), t.x * sBeta[j4], t.y * sBeta[j4 + 1], t.z * sBeta[j4 + 2],
+                t.w * sBeta[j4 + 3]);
     }
-    invert(cx);
-    {  // T diag(beta) at R_T and T^T at OP_TT, both as (row i, K = j) operands
-      const float* tr = reinterpret_cast<const float*>(sm + R_TROW);
-      for (int x = tid; x < C * 16; x += NTH) {
-        const int i = x >> 4, j4 = (x & 15) * 4;
-        const float* p = tr + i * 65 + j4;
-        st_tf32x4(sm, R_T + kmaj(i, j4, 64), p[0] * sBeta[j4], p[1] * sBeta[j4 + 1], p[2] * sBeta[j4 + 2],
-                  p[3] * sBeta[j4 + 3]);
-        st_tf32x4(sm, OP_TT + kmaj(i, j4, 64), tr[j4 * 65 + i], tr[(j4 + 1) * 65 + i], tr[(j4 + 2) * 65 + i],
-                  tr[(j4 + 3) * 65 + i]);
-      }
+    for (int x = tid; x < C * 16; x += NTH) {  // T^T: element (i, j) = T[j][i]
+      const int i = x & 63, j4 = (x >> 6) * 4;
+      const float* tcol = irec + INTER_T + i;
+      st_tf32x4(sm, OP_TT + kmaj(i, j4, 64), tcol[j4 * 64], tcol[(j4 + 1) * 64], tcol[(j4 + 2) * 64],
+                tcol[(j4 + 3) * 64]);
     }
 
     // ---------------------------------------------------------------- M^T, dM^T into TMEM; dEl

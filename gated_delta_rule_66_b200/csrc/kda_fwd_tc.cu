@@ -147,8 +147,18 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_tc_kernel(FwdArgs a) {
     if (wide) pairwise_compute(cx, a.scale, pw);
     __syncthreads();  // raw inputs consumed; the raw region is reused below
 
-    readout_ap(cx, tm + TM_APA, tm + TM_APB, false, wide, pw);
+    float* irec = a.inter ? a.inter + (head * NT + ch) * INTER_REC : nullptr;
+    readout_ap(cx, tm + TM_APA, tm + TM_APB, false, wide, pw, irec);
     invert(cx);
+    if (irec) {  // T and Ah for the backward (P^T was stored by the read-out)
+      const float* tr = reinterpret_cast<const float*>(sm + R_TROW);
+      const float* ah = reinterpret_cast<const float*>(sm + R_AH);
+      for (int x = tid; x < C * C; x += NTH) {
+        const int o = (x >> 6) * 65 + (x & 63);
+        irec[INTER_T + x] = tr[o];
+        irec[INTER_AH + x] = ah[o];
+      }
+    }
     {
       const float* tr = reinterpret_cast<const float*>(sm + R_TROW);
       for (int x = tid; x < C * 16; x += NTH) {

@@ -14,6 +14,11 @@ constexpr int FWD_VBLOCK = 32;   // V columns per CTA in the chunked kernels
 // Ah [i][j] (row-major 64 x 64), [dP; dA] as [j][i'] (64 x 128, i' < 64 dP),
 // [dQE; dKE'] as [f][i'] (128 x 128, i' < 64 dQE), dKEd as [f][i] (128 x 64),
 // dbeta_R [64], dEl [128].
+// Per-(b, hv, 64-step chunk) interaction record that the tensor-core forward
+// stores with a workspace (floats): P^T row-major [j][i] at 0, T row-major at
+// INTER_T, Ah row-major at INTER_AH.  The backward reads it instead of
+// recomputing the interaction products and the inverse.
+constexpr int INTER_T = 4096, INTER_AH = 8192, INTER_REC = 12288;
 constexpr int G_AH = 0, G_PA = 4096, G_QK = 12288, G_KED = 28672, G_DBR = 36864, G_DEL = 36928,
               GREC = 37120;
 
@@ -23,6 +28,7 @@ struct FwdArgs {
   void* o;          // may be null (state pass only)
   float* S_T;       // may be null
   float* states;    // may be null; [B, HV, NT, K, V] state entering each chunk
+  float* inter;     // may be null; per-chunk interaction records (K = V = 128)
   float scale;
   int B, T, H, HV, K, V;
 };
@@ -31,6 +37,7 @@ struct BwdArgs {
   const void *q, *k, *v, *dO;
   const float *g, *beta, *dS_T;
   const float* states;   // [B, HV, NT, K, V]
+  const float* inter;    // per-chunk interaction records of the forward (K = V = 128), else null
   float* dstates;        // [B, HV, NT, K, V] gradient of the state leaving each chunk
   void *dq, *dk, *dv;    // dtype of q/k/v
   float *dg, *dbeta, *dS0;

@@ -235,7 +235,7 @@ __device__ __forceinline__ uint32_t p_off(int i, int j, bool transP) {
 // the two interaction products; the raw region must be free.  Ends with a
 // barrier.
 __device__ __forceinline__ void readout_ap(const Ctx& c, uint32_t tm_apa, uint32_t tm_apb, bool transP,
-                                           bool wide, const Pairwise& pw) {
+                                           bool wide, const Pairwise& pw, float* pt = nullptr) {
   using namespace tc;
   float* sAh = reinterpret_cast<float*>(c.sm + R_AH);
   {
@@ -249,8 +249,12 @@ __device__ __forceinline__ void readout_ap(const Ctx& c, uint32_t tm_apa, uint32
       const bool same = (i >> 5) == (j >> 5);
       if (!same && i >= 32) continue;  // lower-left block comes from product b
       const float val = (same && (isA ? j < i : j <= i)) ? v[jj] : 0.f;
-      if (isA) sAh[i * 65 + j] = val;
-      else st_tf32(c.sm, p_off(i, j, transP), val);
+      if (isA) {
+        sAh[i * 65 + j] = val;
+      } else {
+        st_tf32(c.sm, p_off(i, j, transP), val);
+        if (pt) pt[j * 64 + i] = val;
+      }
     }
   }
   {
@@ -261,8 +265,12 @@ __device__ __forceinline__ void readout_ap(const Ctx& c, uint32_t tm_apa, uint32
 #pragma unroll
       for (int jj = 0; jj < 16; ++jj) {
         const int j = c.hcol * 16 + jj;
-        if (r < 32) sAh[(32 + r) * 65 + j] = v[jj];
-        else st_tf32(c.sm, p_off(r, j, transP), v[jj]);
+        if (r < 32) {
+          sAh[(32 + r) * 65 + j] = v[jj];
+        } else {
+          st_tf32(c.sm, p_off(r, j, transP), v[jj]);
+          if (pt) pt[j * 64 + r] = v[jj];
+        }
       }
     }
   }
@@ -271,7 +279,10 @@ __device__ __forceinline__ void readout_ap(const Ctx& c, uint32_t tm_apa, uint32
     for (int jj = 0; jj < 16; ++jj) {
       const int j = pw.j0 + jj;
       if (pw.kind == 0 && j < pw.i) sAh[pw.i * 65 + j] = pw.v[jj];
-      if (pw.kind == 1 && j <= pw.i) st_tf32(c.sm, p_off(pw.i, j, transP), pw.v[jj]);
+      if (pw.kind == 1 && j <= pw.i) {
+        st_tf32(c.sm, p_off(pw.i, j, transP), pw.v[jj]);
+        if (pt) pt[j * 64 + pw.i] = pw.v[jj];
+      }
     }
     __syncthreads();
   }
