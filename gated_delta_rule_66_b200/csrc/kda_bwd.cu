@@ -472,6 +472,14 @@ __global__ void __launch_bounds__(NTHREADS, 2) kda_bwd_assemble_kernel(BwdArgs a
   const TIn* k = static_cast<const TIn*>(a.k);
   const int tid = threadIdx.x;
 
+  float4 qe[2], ke[2], kd[2];  // [dQE; dKE'] and dKEd of this quarter, consumed further down
+#pragma unroll
+  for (int m = 0; m < 2; ++m) {  // channel f of the quarter, four rows per item
+    const int idx = tid + m * NTHREADS, f = idx >> 4, i4 = (idx & 15) * 4;
+    qe[m] = *reinterpret_cast<const float4*>(rec + G_QK + (f0 + f) * 128 + i4);
+    ke[m] = *reinterpret_cast<const float4*>(rec + G_QK + (f0 + f) * 128 + 64 + i4);
+    kd[m] = *reinterpret_cast<const float4*>(rec + G_KED + (f0 + f) * 64 + i4);
+  }
   {  // inputs of this channel quarter (4 channels per item) and the C x C adjoints; loads first
     float4 gv[2], dp[4], da[4];
     float qv[2][4], kv[2][4];
@@ -527,6 +535,7 @@ __global__ void __launch_bounds__(NTHREADS, 2) kda_bwd_assemble_kernel(BwdArgs a
     const int i = tid;
     const float4* arow = reinterpret_cast<const float4*>(a.inter + (head * NT + ch) * INTER_REC + INTER_AH + i * 64);
     float s0 = rec[G_DBR + i], s1 = 0.f;
+#pragma unroll
     for (int j4 = 0; j4 < 16; ++j4) {
       const float4 ah = arow[j4];
       const float vah[4] = {ah.x, ah.y, ah.z, ah.w};
@@ -545,14 +554,6 @@ __global__ void __launch_bounds__(NTHREADS, 2) kda_bwd_assemble_kernel(BwdArgs a
     sdA[i * LDC + j] *= sBeta[i];
   }
   {  // element-wise terms; the chunk-end sum of dKEd o k o e^{c_last-c} goes through sE1
-    float4 qe[2], ke[2], kd[2];
-#pragma unroll
-    for (int m = 0; m < 2; ++m) {  // channel f of the quarter, four rows per item
-      const int idx = tid + m * NTHREADS, f = idx >> 4, i4 = (idx & 15) * 4;
-      qe[m] = *reinterpret_cast<const float4*>(rec + G_QK + (f0 + f) * 128 + i4);
-      ke[m] = *reinterpret_cast<const float4*>(rec + G_QK + (f0 + f) * 128 + 64 + i4);
-      kd[m] = *reinterpret_cast<const float4*>(rec + G_KED + (f0 + f) * 64 + i4);
-    }
 #pragma unroll
     for (int m = 0; m < 2; ++m) {
       const int idx = tid + m * NTHREADS, f = idx >> 4, i4 = (idx & 15) * 4;

@@ -425,91 +425,104 @@ __device__ void factored_block_mma(int J, const float* sK, const float* sQ, cons
 }
 
 // The interaction terms of factored_terms for C = 64 with 3xTF32 warp MMAs,
-// one pass, no shared scratch and no barriers: warp w owns the 16 x 8 output
-// tiles x = w and w + 8 (row block I = x / (K/8), channels 8 (x % (K/8))) and
+// one pass, no shared scratch and no barriers: warp w owns the 16 x 16 output
+// tile of row block I = w / 2 and channels 16 (w % 2) .. + 15 (K = 32) and
 // accumulates in registers, over every column block J <= I, the row terms of
-// its rows and, for J = I, the column terms of the same rows; the split
-// exponent factors are formed on the fly from c (natural units).  Requires
-// every 16-row block's decay span to be at most 80 (checked by the caller).
+// its rows and the column terms of the same rows (columns of block I); each
+// split A fragment feeds both 8-channel halves.  The split-exponent factors
+// are formed on the fly from c (natural units).  Requires every 16-row
+// block's decay span to be at most 80 (checked by the caller).
 template <int K>
 __device__ void factored_terms_fused(const float* sK, const float* sQ, const float* sC, const float* sdA,
                                      const float* sdP, float* sDq, float* sDk, float* sDc) {
-  constexpr int C = 64, LDK = K + 1, LDC = C + 1, NTL = K / 8;
-  static_assert(4 * NTL == 16, "two tiles per warp need 16 tiles");
+  constexpr int C = 64, LDK = K + 1, LDC = C + 1, NH = K / 16;
+  static_assert(4 * NH == NTHREADS / 32, "one 16 x 16 tile per warp");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  for (int x = warp; x < 4 * NTL; x += NTHREADS / 32) {
-    const int I = x / NTL, f0 = (x % NTL) * 8, i0 = I * BS;
-    const int fa = f0 + g;                      // channel of the B fragments
-    float totA[4] = {0.f, 0.f, 0.f, 0.f}, totP[4] = {0.f, 0.f, 0.f, 0.f};
-    // row terms: rows of block I against the columns of every block J <= I
-    for (int J = 0; J <= I; ++J) {
-      const int r0 = J * BS, ref = (I == J) ? r0 + BS / 2 - 1 : r0 + BS - 1;
-      float accA[4] = {0.f, 0.f, 0.f, 0.f}, accP[4] = {0.f, 0.f, 0.f, 0.f};
+  const int I = warp / NH, fb = (warp % NH) * 16, i0 = I * BS;
+  float totA[2][4] = {}, totP[2][4] = {};
+  // row terms: rows of block I against the columns of every block J <= I
+  for (int J = 0; J <= I; ++J) {
+    const int r0 = J * BS, ref = (I == J) ? r0 + BS / 2 - 1 : r0 + BS - 1;
+    float accA[2][4] = {}, accP[2][4] = {};
 #pragma unroll
-      for (int ks = 0; ks < 2; ++ks) {
-        const int j = r0 + ks * 8 + t;
-        Split aA[4], aP[4], bw[2];
-        aA[0] = split_tf32(sdA[(i0 + g) * LDC + j]);
-        aA[1] = split_tf32(sdA[(i0 + g + 8) * LDC + j]);
-        aA[2] = split_tf32(sdA[(i0 + g) * LDC + j + 4]);
-        aA[3] = split_tf32(sdA[(i0 + g + 8) * LDC + j + 4]);
-        aP[0] = split_tf32(sdP[(i0 + g) * LDC + j]);
-        aP[1] = split_tf32(sdP[(i0 + g + 8) * LDC + j]);
-        aP[2] = split_tf32(sdP[(i0 + g) * LDC + j + 4]);
-        aP[3] = split_tf32(sdP[(i0 + g + 8) * LDC + j + 4]);
+    for (int ks = 0; ks < 2; ++ks) {
+      const int j = r0 + ks * 8 + t;
+      Split aA[4], aP[4];
+      aA[0] = split_tf32(sdA[(i0 + g) * LDC + j]);
+      aA[1] = split_tf32(sdA[(i0 + g + 8) * LDC + j]);
+      aA[2] = split_tf32(sdA[(i0 + g) * LDC + j + 4]);
+      aA[3] = split_tf32(sdA[(i0 + g + 8) * LDC + j + 4]);
+      aP[0] = split_tf32(sdP[(i0 + g) * LDC + j]);
+      aP[1] = split_tf32(sdP[(i0 + g + 8) * LDC + j]);
+      aP[2] = split_tf32(sdP[(i0 + g) * LDC + j + 4]);
+      aP[3] = split_tf32(sdP[(i0 + g + 8) * LDC + j + 4]);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int fa = fb + 8 * h + g;
         const float cr = sC[ref * LDK + fa];
+        Split bw[2];
         bw[0] = split_tf32(sK[j * LDK + fa] * __expf(cr - sC[j * LDK + fa]));
         bw[1] = split_tf32(sK[(j + 4) * LDK + fa] * __expf(cr - sC[(j + 4) * LDK + fa]));
-        mma3(accA, aA, bw);
-        mma3(accP, aP, bw);
-      }
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int i = i0 + g + ((e & 2) ? 8 : 0), f = f0 + 2 * t + (e & 1);
-        const float e1 = __expf(sC[i * LDK + f] - sC[ref * LDK + f]);
-        totA[e] = fmaf(accA[e], e1, totA[e]);
-        totP[e] = fmaf(accP[e], e1, totP[e]);
+        mma3(accA[h], aA, bw);
+        mma3(accP[h], aP, bw);
       }
     }
-    // column terms: the columns of block I against its own rows and all rows below
-    float accD[4] = {0.f, 0.f, 0.f, 0.f}, accO[4] = {0.f, 0.f, 0.f, 0.f};
-    const int rd = i0 + BS / 2 - 1, ro = i0 + BS - 1;
-    for (int ks = 0; ks < (C - i0) / 8; ++ks) {
-      const int i = i0 + ks * 8 + t, ref = (ks < 2) ? rd : ro;
-      Split aA[4], aP[4], bk[2], bq[2];
-      aA[0] = split_tf32(sdA[i * LDC + i0 + g]);
-      aA[1] = split_tf32(sdA[i * LDC + i0 + g + 8]);
-      aA[2] = split_tf32(sdA[(i + 4) * LDC + i0 + g]);
-      aA[3] = split_tf32(sdA[(i + 4) * LDC + i0 + g + 8]);
-      aP[0] = split_tf32(sdP[i * LDC + i0 + g]);
-      aP[1] = split_tf32(sdP[i * LDC + i0 + g + 8]);
-      aP[2] = split_tf32(sdP[(i + 4) * LDC + i0 + g]);
-      aP[3] = split_tf32(sdP[(i + 4) * LDC + i0 + g + 8]);
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = i0 + g + ((e & 2) ? 8 : 0), f = fb + 8 * h + 2 * t + (e & 1);
+        const float e1 = __expf(sC[i * LDK + f] - sC[ref * LDK + f]);
+        totA[h][e] = fmaf(accA[h][e], e1, totA[h][e]);
+        totP[h][e] = fmaf(accP[h][e], e1, totP[h][e]);
+      }
+  }
+  // column terms: the columns of block I against its own rows and all rows below
+  float accD[2][4] = {}, accO[2][4] = {};
+  const int rd = i0 + BS / 2 - 1, ro = i0 + BS - 1;
+  for (int ks = 0; ks < (C - i0) / 8; ++ks) {
+    const int i = i0 + ks * 8 + t, ref = (ks < 2) ? rd : ro;
+    Split aA[4], aP[4];
+    aA[0] = split_tf32(sdA[i * LDC + i0 + g]);
+    aA[1] = split_tf32(sdA[i * LDC + i0 + g + 8]);
+    aA[2] = split_tf32(sdA[(i + 4) * LDC + i0 + g]);
+    aA[3] = split_tf32(sdA[(i + 4) * LDC + i0 + g + 8]);
+    aP[0] = split_tf32(sdP[i * LDC + i0 + g]);
+    aP[1] = split_tf32(sdP[i * LDC + i0 + g + 8]);
+    aP[2] = split_tf32(sdP[(i + 4) * LDC + i0 + g]);
+    aP[3] = split_tf32(sdP[(i + 4) * LDC + i0 + g + 8]);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int fa = fb + 8 * h + g;
       const float cr = sC[ref * LDK + fa];
       const float x0 = __expf(sC[i * LDK + fa] - cr), x1 = __expf(sC[(i + 4) * LDK + fa] - cr);
+      Split bk[2], bq[2];
       bk[0] = split_tf32(sK[i * LDK + fa] * x0);
       bk[1] = split_tf32(sK[(i + 4) * LDK + fa] * x1);
       bq[0] = split_tf32(sQ[i * LDK + fa] * x0);
       bq[1] = split_tf32(sQ[(i + 4) * LDK + fa] * x1);
       if (ks < 2) {
-        mma3(accD, aA, bk);
-        mma3(accD, aP, bq);
+        mma3(accD[h], aA, bk);
+        mma3(accD[h], aP, bq);
       } else {
-        mma3(accO, aA, bk);
-        mma3(accO, aP, bq);
+        mma3(accO[h], aA, bk);
+        mma3(accO[h], aP, bq);
       }
     }
+  }
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const int i = i0 + g + ((e & 2) ? 8 : 0), f = f0 + 2 * t + (e & 1), o = i * LDK + f;
+      const int i = i0 + g + ((e & 2) ? 8 : 0), f = fb + 8 * h + 2 * t + (e & 1), o = i * LDK + f;
       const float ci = sC[o];
-      const float col = accD[e] * __expf(sC[rd * LDK + f] - ci) + accO[e] * __expf(sC[ro * LDK + f] - ci);
+      const float col =
+          accD[h][e] * __expf(sC[rd * LDK + f] - ci) + accO[h][e] * __expf(sC[ro * LDK + f] - ci);
       const float kk = sK[o];
-      sDk[o] += totA[e] + col;
-      sDq[o] += totP[e];
-      sDc[o] += kk * (totA[e] - col) + sQ[o] * totP[e];
+      sDk[o] += totA[h][e] + col;
+      sDq[o] += totP[h][e];
+      sDc[o] += kk * (totA[h][e] - col) + sQ[o] * totP[h][e];
     }
-  }
   __syncthreads();
 }
 
