@@ -141,10 +141,21 @@ def _flush_l2(buf):
     buf.add_(1)
 
 
-def gpu_path(kda, name, steps, warmup, rank_barrier):
+_HOST_INPUTS = {}  # workload name -> its host inputs, shared with the oracle sampler
+
+
+def host_inputs(w):
+    if w.name not in _HOST_INPUTS:
+        _HOST_INPUTS[w.name] = make_inputs(w, with_do=(w.path == "fwdbwd"))
+    return _HOST_INPUTS[w.name]
+
+
+def gpu_path(kda, name, steps, warmup, rank_barrier, shrink=None):
     """Times one workload on this rank's GPU.  Returns a result dict."""
     w = BY_NAME[name]
-    inp = make_inputs(w, with_do=(w.path == "fwdbwd"))
+    if shrink:  # a smaller batch and length of the same workload (profiler captures only)
+        w = w.with_sizes(name=f"{name}_B{shrink[0]}_T{shrink[1]}", B=shrink[0], T=shrink[1])
+    inp = host_inputs(w)
     dev = torch.device("cuda")
     d = {n: (None if t is None else t.to(dev)) for n, t in inp.items()}
     flush = None
@@ -171,7 +182,8 @@ def gpu_path(kda, name, steps, warmup, rank_barrier):
                     workspace=ws)
             kda.bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["dO"], scale=w.scale,
                     initial_state=d["S0"], workspace=ws, states_from_fwd=True)
-        launches_per_step = 3 + (2 if w.HV > w.H else 0)
+        # kda_fwd: 1 launch; kda_bwd: state gradients, gradient products, assembly (+2 group sums)
+        launches_per_step = 4 + (2 if w.HV > w.H else 0)
         tokens = w.B * w.T
     else:
         S = d["S"]
@@ -221,6 +233,8 @@ def gpu_path(kda, name, steps, warmup, rank_barrier):
     pinned = {n: (None if t is None else t.pin_memory()) for n, t in inp.items()}
     h2d = sum(t.numel() * t.element_size() for t in pinned.values() if t is not None)
 
+    host_out = []  # pinned result buffers, allocated by the first (untimed) call
+
     def e2e_step():
         dd = {n: (None if t is None else t.to(dev, non_blocking=True)) for n, t in pinned.items()}
         if w.path == "fwd":
@@ -235,8 +249,12 @@ def gpu_path(kda, name, steps, warmup, rank_barrier):
         else:
             outs = (kda.decode_step(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["S"],
                                     scale=w.scale), dd["S"])
-        host = [t.to("cpu", non_blocking=True) for t in outs if t is not None]
-        return host
+        outs = [t for t in outs if t is not None]
+        if not host_out:
+            host_out.extend(torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs)
+        for hbuf, t in zip(host_out, outs):
+            hbuf.copy_(t, non_blocking=True)
+        return host_out
 
     e2e_steps = max(1, min(steps, 5))
     e2e_step()
@@ -255,6 +273,25 @@ def gpu_path(kda, name, steps, warmup, rank_barrier):
     return res, w
 
 
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch of ``kernel`` on ``workload`` from the ncu capture
+    recorded in profiles/dram_traffic.json, or None when there is none or the
+    kernel's sources changed since (their sha256 is stored beside the figure)."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "dram_traffic.json")) as f:
+            rec = json.load(f)[kernel]
+    except (OSError, KeyError, ValueError):
+        return None
+    h = hashlib.sha256()
+    for rel in rec["sources"]:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    if h.hexdigest() != rec["sources_sha256"]:
+        return None
+    return rec["bytes_per_launch"].get(workload)
+
+
 def roofline_for(res, w, peaks):
     hbm = peaks["hbm_gbs"]
     if w.path == "decode":
@@ -265,11 +302,12 @@ def roofline_for(res, w, peaks):
     if w.path == "fwd":
         byts = algorithmic_bytes(w, "fwd")
         t = res["calls"]["kernel_ms"] * 1e-3
-        return {"bound": "hbm", "kernel": "kda_fwd_chunk_kernel", "achieved": byts / t / 1e9,
+        return {"bound": "hbm", "kernel": "kda_fwd_tc_kernel" if w.K == 128 and w.dtype == "bf16"
+                else "kda_fwd_chunk_kernel", "achieved": byts / t / 1e9,
                 "peak": hbm, "unit": "GB/s", "frac": byts / t / 1e9 / hbm, "algorithmic_bytes": byts}
     byts = algorithmic_bytes(w, "fwd")
     t = res["calls"]["fwd_ms"] * 1e-3
-    return {"bound": "hbm", "kernel": "kda_fwd_chunk_kernel (state-storing forward of the step)",
+    return {"bound": "hbm", "kernel": "kda_fwd_tc_kernel (state-storing forward of the step)",
             "achieved": byts / t / 1e9, "peak": hbm, "unit": "GB/s", "frac": byts / t / 1e9 / hbm,
             "algorithmic_bytes": byts}
 
@@ -294,7 +332,7 @@ def run_gpu(args):
     for name in [HEADLINE] + [p for p in PATHS if p != HEADLINE and args.all_paths]:
         if name == HEADLINE:
             with Clocks(local) as clk:
-                res, w = gpu_path(kda, name, args.steps, args.warmup, barrier)
+                res, w = gpu_path(kda, name, args.steps, args.warmup, barrier, args.shrink)
             res["clocks"] = clk.summary()
         else:
             res, w = gpu_path(kda, name, args.steps, args.warmup, barrier)
@@ -324,11 +362,12 @@ def run_gpu(args):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded; q,k L2-normalised, g = -5 sigmoid(N(0,1)), beta = sigmoid(N(0,1)))",
-        "config": {"workload": "fwdbwd: B=2 H=HV=96 T=4096 K=V=128, bf16 q/k/v/dO, fp32 g/beta/state; "
-                               "step = kda_fwd (stores chunk states) + kda_bwd (reuses them)",
+        "config": {"workload": f"fwdbwd: B={w.B} H=HV={w.HV} T={w.T} K=V={w.K}, bf16 q/k/v/dO, fp32 g/beta/state; "
+                               "step = kda_fwd (stores chunk states and interaction records) + kda_bwd (reuses them)"
+                               + ("" if not args.shrink else " [reduced for a profiler capture]"),
                    "global_batch": w.B * world, "seq_len": w.T, "parallelism": f"replicas x{world}",
                    "l2": head["l2"]},
-        "roofline": dict(head["roofline"], traffic=None),
+        "roofline": dict(head["roofline"], traffic=recorded_traffic(head["roofline"]["kernel"].split()[0], HEADLINE)),
         "e2e": {"value": head["e2e_tokens_per_s"], "unit": "tokens/s",
                 "h2d_bytes_per_step": head["h2d_bytes"], "d2h_bytes_per_step": head["d2h_bytes"]},
         "gpu_launches": head["launches_per_step"] * args.steps,
@@ -350,14 +389,13 @@ def run_gpu(args):
 # ---------------------------------------------------------------------------- CPU oracle arm
 
 def _oracle_head(job):
-    """Runs the float64 oracle fwd (+bwd) on one value head of a sample."""
-    import numpy as np
+    """Runs the float64 oracle fwd (+bwd) on one (b, hv) head of a sample."""
     sys.path.insert(0, ROOT)
     import oracle
     path, arrays, scale = job
     q, k, v, g, beta, S0, dO = arrays
     t0 = time.perf_counter()
-    o, S = oracle.kda_forward(q, k, v, g, beta, scale, S0)
+    oracle.kda_forward(q, k, v, g, beta, scale, S0)
     if path == "fwdbwd":
         oracle.kda_backward(q, k, v, g, beta, scale, S0, dO)
     return time.perf_counter() - t0
@@ -369,51 +407,73 @@ def _warm(_):
     return 0
 
 
-def cpu_baseline(w, budget_s=20.0):
-    """Times the oracle on a bounded sample of workload ``w`` on the host's
-    cores: whole value heads (one per worker process) over the first T_s
-    tokens of batch row 0; tokens/s is scaled to all HV heads."""
-    import numpy as np
-    cores = len(os.sched_getaffinity(0))
-    Ts = {"fwdbwd": 256, "fwd": 512, "decode": 1}[w.path]
-    T_s = min(w.T, Ts)
-    sub = w.with_sizes(B=1, T=T_s) if w.path != "decode" else w
-    inp = make_inputs(sub, with_do=(w.path == "fwdbwd")) if w.path != "decode" else None
-    if w.path == "decode":
-        nheads = min(w.HV, cores * 4)
-        sub = w.with_sizes(B=1)
-        inp = make_inputs(sub)
-    f64 = lambda t: None if t is None else t.to(torch.float64).numpy()
-    G = w.HV // w.H
-    jobs = []
-    nheads = min(w.HV, max(cores, 1) * 2)
-    for hv in range(nheads):
-        h = hv // G
+class OracleSampler:
+    """The float64 oracle on the host's cores, on a bounded sample of a
+    workload: whole (b, hv) heads at the workload's full length (a GQA head
+    reads its own query/key head), one single-threaded worker process per
+    core, as many heads as fit the time budget.  tokens/s = sampled head-tokens
+    / HV / elapsed, i.e. scaled to all HV heads of a token."""
+
+    def __init__(self, w, budget_s):
+        for var in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS"):
+            os.environ[var] = "1"   # one thread per worker: `cores` threads in total
+        self.w = w
+        self.cores = len(os.sched_getaffinity(0))
+        inp = host_inputs(w)
+        f64 = lambda t: None if t is None else t.to(torch.float64).numpy()
+        G = w.HV // w.H
         if w.path == "decode":
-            arrays = (f64(inp["q"][:, None, h:h + 1]), f64(inp["k"][:, None, h:h + 1]),
-                      f64(inp["v"][:, None, hv:hv + 1]), f64(inp["g"][:, None, hv:hv + 1]),
-                      f64(inp["beta"][:, None, hv:hv + 1]), f64(inp["S"][:, hv:hv + 1]), None)
+            units = [(b, hv) for b in range(w.B) for hv in range(w.HV)]
+            T = 1
+            def arrays(b, hv):
+                h = hv // G
+                return (f64(inp["q"][b:b + 1, None, h:h + 1]), f64(inp["k"][b:b + 1, None, h:h + 1]),
+                        f64(inp["v"][b:b + 1, None, hv:hv + 1]), f64(inp["g"][b:b + 1, None, hv:hv + 1]),
+                        f64(inp["beta"][b:b + 1, None, hv:hv + 1]), f64(inp["S"][b:b + 1, hv:hv + 1]), None)
         else:
-            arrays = (f64(inp["q"][:, :, h:h + 1]), f64(inp["k"][:, :, h:h + 1]),
-                      f64(inp["v"][:, :, hv:hv + 1]), f64(inp["g"][:, :, hv:hv + 1]),
-                      f64(inp["beta"][:, :, hv:hv + 1]),
-                      None if inp["S0"] is None else f64(inp["S0"][:, hv:hv + 1]),
-                      None if inp.get("dO") is None else f64(inp["dO"][:, :, hv:hv + 1]))
-        jobs.append((w.path, arrays, w.scale))
-    for var in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS"):
-        os.environ[var] = "1"   # one thread per worker: `cores` threads in total
-    ctx = mp.get_context("spawn")
-    with ctx.Pool(processes=cores) as pool:
-        pool.map(_warm, range(cores))          # worker start-up stays outside the timing
+            units = [(b, hv) for b in range(w.B) for hv in range(w.HV)]
+            T = w.T
+            def arrays(b, hv):
+                h = hv // G
+                return (f64(inp["q"][b:b + 1, :, h:h + 1]), f64(inp["k"][b:b + 1, :, h:h + 1]),
+                        f64(inp["v"][b:b + 1, :, hv:hv + 1]), f64(inp["g"][b:b + 1, :, hv:hv + 1]),
+                        f64(inp["beta"][b:b + 1, :, hv:hv + 1]),
+                        None if inp["S0"] is None else f64(inp["S0"][b:b + 1, hv:hv + 1]),
+                        None if inp.get("dO") is None else f64(inp["dO"][b:b + 1, :, hv:hv + 1]))
+        # calibrate one head (in this process) on a short prefix, then size the sample
+        cal = min(T, 64)
+        q, k, v, g, beta, S0, dO = arrays(0, 0)
+        cut = lambda x: None if x is None or w.path == "decode" else x[:, :cal]
+        t_cal = _oracle_head((w.path, (cut(q), cut(k), cut(v), cut(g), cut(beta), S0, cut(dO)), w.scale))
+        t_head = max(t_cal * T / cal, 1e-4)
+        per_worker = max(1, int(budget_s / t_head))
+        n = min(len(units), self.cores * per_worker)
+        self.jobs = [(w.path, arrays(b, hv), w.scale) for (b, hv) in units[:n]]
+        self.head_tokens = n * T
+        self.desc = (f"{n} of {len(units)} (b, hv) heads, each the full {T} steps "
+                     f"({'fwd+bwd' if w.path == 'fwdbwd' else w.path}), float64 NumPy, one single-threaded "
+                     f"process per core; tokens/s = head-tokens / {w.HV} heads / elapsed")
+        self.pool = mp.get_context("spawn").Pool(processes=self.cores)
+        self.pool.map(_warm, range(self.cores))   # worker start-up stays outside the timing
+
+    def run(self):
         t0 = time.perf_counter()
-        pool.map(_oracle_head, jobs)
+        self.pool.map(_oracle_head, self.jobs, chunksize=1)
         elapsed = time.perf_counter() - t0
-    head_tokens = nheads * T_s
-    tokens_per_s = head_tokens / w.HV / elapsed
-    return {"value": tokens_per_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": f"{nheads} of {w.HV} value heads x {T_s} tokens of batch row 0 "
-                      f"({'fwd+bwd' if w.path == 'fwdbwd' else w.path}), float64 NumPy, one process per "
-                      f"core; tokens/s scaled to all {w.HV} heads", "seconds": elapsed}
+        return {"value": self.head_tokens / self.w.HV / elapsed, "unit": "tokens/s", "cores": self.cores,
+                "kind": "oracle", "sample": self.desc, "seconds": elapsed}
+
+    def close(self):
+        self.pool.close()
+        self.pool.join()
+
+
+def cpu_baseline(w, budget_s=20.0):
+    smp = OracleSampler(w, budget_s)
+    try:
+        return smp.run()
+    finally:
+        smp.close()
 
 
 def run_reference(args):
@@ -421,21 +481,22 @@ def run_reference(args):
     if rank != 0:
         return
     w = BY_NAME[HEADLINE]
-    times = []
-    cb = None
-    for _ in range(args.warmup + args.steps):
-        cb = cpu_baseline(w, budget_s=args.cpu_seconds)
-        times.append(cb)
-    timed = times[args.warmup:]
+    # each step is one bounded sample; the whole run stays within a few minutes
+    smp = OracleSampler(w, budget_s=max(2.0, 100.0 / (args.steps + args.warmup)))
+    try:
+        runs = [smp.run() for _ in range(args.warmup + args.steps)]
+    finally:
+        smp.close()
+    timed = runs[args.warmup:]
     val = statistics.median(c["value"] for c in timed)
     line = {"metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": BY_NAME[HEADLINE].B * BY_NAME[HEADLINE].T / val * 1e3,
+            "warmup": args.warmup, "ms_per_step": w.B * w.T / val * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": {"workload": "fwdbwd: B=2 H=HV=96 T=4096 K=V=128 (oracle on a bounded sample)",
+            "config": {"workload": "fwdbwd: B=2 H=HV=96 T=4096 K=V=128 (float64 oracle on a bounded sample)",
                        "global_batch": w.B, "seq_len": w.T, "parallelism": "none"},
-            "cpu_baseline": {"kind": "oracle", "cores": cb["cores"], "sample": cb["sample"], "value": val,
-                             "unit": "tokens/s"},
+            "cpu_baseline": {"kind": "oracle", "cores": timed[-1]["cores"], "sample": timed[-1]["sample"],
+                             "value": val, "unit": "tokens/s"},
             "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -449,6 +510,9 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--headline-only", dest="all_paths", action="store_false")
+    ap.add_argument("--shrink", type=lambda x: tuple(int(v) for v in x.split(",")), default=None,
+                    metavar="B,T", help="run the headline workload at batch B and length T (for ncu captures; "
+                                        "the printed line is not a headline number)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -5,19 +5,20 @@
 // From the chunk algebra (kda_tc_chunk.cuh) the gradient of the state entering
 // a chunk, given the gradient dM of the state leaving it, is
 //   dU  = P^T dO + (K o e^{c_last - c}) dM
-//   dX  = diag(beta) T^T dU
-//   dM_in = diag(e^{c_last}) dM + (Q~ o e^c)^T dO - (K o e^c)^T dX
+//   dR  = T^T dU
+//   dM_in = diag(e^{c_last}) dM + (Q~ o e^c)^T dO - (diag(beta) K o e^c)^T dR
 // ("recurrent.py", KDAFunction.backward, taken a chunk at a time; dM needs no
 // forward state).  One CTA per (b, hv) walks the chunks in reverse with dM^T
 // held in TMEM (lane = value column n, column = key channel f):
 //   dU^T  = dO^T P + dM^T (K o e^{c_last-c})^T      (A = dO^T or dM^T, both in TMEM)
-//   dX^T  = dU^T (diag(beta) T^T)^T
-//   dM_in^T = dM^T diag(e^{c_last}) + dO^T (Q~ o e^c) - dX^T (K o e^c)
+//   dR^T  = dU^T T
+//   dM_in^T = dM^T diag(e^{c_last}) + dO^T (Q~ o e^c) - dR^T (diag(beta) K o e^c)
+// P and T come from the forward's interaction record as ready operand images.
 // The state gradient at the chunk's midpoint (leaving step 31), needed for the
 // 32-step granularity of the per-chunk gradient kernel, is the same formula
 // over the second half alone:
 //   dM_mid^T = dM^T diag(e^{c_last - c_31}) + dO^T[:,32:] (Q~ o e^{c-c_31})[32:]
-//              - dX^T[:,32:] (K o e^{c-c_31})[32:].
+//              - dR^T[:,32:] (diag(beta) K o e^{c-c_31})[32:].
 #include <cuda_bf16.h>
 
 #include "kda_internal.h"
@@ -31,7 +32,7 @@ namespace tcb {
 using namespace tcc;
 constexpr uint32_t OP_KED = OP, OP_QET = OP + 32768, OP_NKET = OP + 65536, OP_Q2T = OP + 98304,
                    OP_NK2T = OP + 114688;
-constexpr uint32_t TM_S = 0, TM_DU = 128, TM_DX = 192, TM_DOT = 256, TM_APA = 320, TM_APB = 384,
+constexpr uint32_t TM_S = 0, TM_DU = 128, TM_DR = 192, TM_DOT = 256,
                    TM_MID = 384;  // mid-chunk gradient (the interaction tile is read by then)
 }  // namespace tcb
 
@@ -91,8 +92,14 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_dstate_tc_kernel(BwdArgs a) {
 
   for (int ch = NT - 1; ch >= 0; --ch) {
     const int t0 = ch * C, L = min(C, T - t0);
-    const float* irec = a.inter + (head * NT + ch) * INTER_REC;  // P^T, T of this chunk (forward)
-    load_raw(cx, qg, kg, dog, a.g, a.beta, b, T, t0, L, a.H, a.HV, h, hv);
+    const float* irec = a.inter + (head * NT + ch) * INTER_REC;  // P^T, T^T of this chunk (forward)
+    load_raw_issue(cx, qg, kg, dog, a.g, a.beta, b, T, t0, L, a.H, a.HV, h, hv);
+    if (ch > 0) {  // the next chunk down: raw rows and record images into L2
+      prefetch_chunk(cx, qg, kg, dog, a.g, b, T, t0 - C, C, a.H, a.HV, h, hv);
+      if (tid == 64) prefetch_l2(irec - INTER_REC, 16384);
+      if (tid == 192) prefetch_l2(irec - INTER_REC + INTER_TT, 16384);
+    }
+    load_raw_wait();
     cumsum_span(cx);
 
     // ---------------------------------------------------------------- operands of the gradient products
@@ -107,6 +114,7 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_dstate_tc_kernel(BwdArgs a) {
         float kf[4], qf[4];
         bf16x4(sm + RAW_K + i * 256 + fq * 2, kf);
         bf16x4(sm + RAW_Q + i * 256 + fq * 2, qf);
+        const float nb = -sBeta[i];
         float e[4], ed[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -118,14 +126,14 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_dstate_tc_kernel(BwdArgs a) {
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           st_tf32(sm, OP_QET + kmaj(fq + u, i, 64), qf[u] * e[u]);
-          st_tf32(sm, OP_NKET + kmaj(fq + u, i, 64), -kf[u] * e[u]);
+          st_tf32(sm, OP_NKET + kmaj(fq + u, i, 64), nb * kf[u] * e[u]);
         }
         if (i >= 32) {
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const float x2 = ex2(c[u] - c31[u]);
             st_tf32(sm, OP_Q2T + kmaj(fq + u, i - 32, 32), qf[u] * x2);
-            st_tf32(sm, OP_NK2T + kmaj(fq + u, i - 32, 32), -kf[u] * x2);
+            st_tf32(sm, OP_NK2T + kmaj(fq + u, i - 32, 32), nb * kf[u] * x2);
           }
         }
       }
@@ -147,18 +155,9 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_dstate_tc_kernel(BwdArgs a) {
     fence_async_smem();
     fence_before();
     __syncthreads();  // raw inputs consumed; the raw region is reused below
-    for (int x = tid; x < C * 16; x += NTH) {  // P^T (row i, K j) = P[j][i], from the record's P^T
-      const int i = x >> 4, j4 = (x & 15) * 4;
-      const float4 p = *reinterpret_cast<const float4*>(irec + i * 64 + j4);
-      st_tf32x4(sm, R_P + kmaj(i, j4, 64), p.x, p.y, p.z, p.w);
-    }
-    for (int x = tid; x < C * 16; x += NTH) {  // (diag(beta) T^T)^T: element (i, j) = beta_i T[j][i]
-      const int i = x & 63, j4 = (x >> 6) * 4;
-      const float bi = sBeta[i];
-      const float* tcol = irec + INTER_T + i;
-      st_tf32x4(sm, R_T + kmaj(i, j4, 64), bi * tcol[j4 * 64], bi * tcol[(j4 + 1) * 64], bi * tcol[(j4 + 2) * 64],
-                bi * tcol[(j4 + 3) * 64]);
-    }
+    copy_image(cx, R_P, irec);             // P^T: (row i, K j) = P[j][i]
+    copy_image(cx, R_T, irec + INTER_TT);  // T^T: (row i, K j) = T[j][i]
+    cp_async_wait_all();
     fence_async_smem();
     __syncthreads();
     if (tid == 0) {  // dU^T = dO^T P + dM^T (K o e^{c_last-c})^T
@@ -171,10 +170,10 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_dstate_tc_kernel(BwdArgs a) {
       commit(bar);
     }
     if (!wait_mma(bar, phase)) { failed = true; break; }
-    if (tid == 0) {  // dX^T = dU^T (diag(beta) T^T)^T
+    if (tid == 0) {  // dR^T = dU^T T
       const uint32_t id = idesc_tf32(128, 64);
       for (int ks = 0; ks < 8; ++ks)
-        mma_ts(tm + TM_DX, tm + TM_DU + ks * 8, desc(sb + R_T + ks * 256, 2048), id, ks > 0);
+        mma_ts(tm + TM_DR, tm + TM_DU + ks * 8, desc(sb + R_T + ks * 256, 2048), id, ks > 0);
       commit(bar);
     }
     if (!wait_mma(bar, phase)) { failed = true; break; }
@@ -207,11 +206,11 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_dstate_tc_kernel(BwdArgs a) {
       const uint32_t id = idesc_tf32(128, 128);
       for (int ks = 0; ks < 8; ++ks) {
         mma_ts(tm + TM_S, tm + TM_DOT + ks * 8, desc(sb + OP_QET + ks * 256, 2048), id, 1);
-        mma_ts(tm + TM_S, tm + TM_DX + ks * 8, desc(sb + OP_NKET + ks * 256, 2048), id, 1);
+        mma_ts(tm + TM_S, tm + TM_DR + ks * 8, desc(sb + OP_NKET + ks * 256, 2048), id, 1);
       }
       for (int ks = 0; ks < 4; ++ks) {
         mma_ts(tm + TM_MID, tm + TM_DOT + 32 + ks * 8, desc(sb + OP_Q2T + ks * 256, 1024), id, 1);
-        mma_ts(tm + TM_MID, tm + TM_DX + 32 + ks * 8, desc(sb + OP_NK2T + ks * 256, 1024), id, 1);
+        mma_ts(tm + TM_MID, tm + TM_DR + 32 + ks * 8, desc(sb + OP_NK2T + ks * 256, 1024), id, 1);
       }
       commit(bar);
     }
@@ -281,16 +280,35 @@ int launch_bwd_dstate_tc(const BwdArgs& a, cudaStream_t stream) {
 // ============================================================================
 namespace tcg {
 using namespace tcc;
-constexpr uint32_t OP_KE = OP, OP_U = OP, OP_KED = OP + 32768, OP_DO = OP + 65536, OP_TT = OP + 131072;
-constexpr uint32_t R_MB = 0;  // M or dM staged as [f][n] once the raw region is free
+// Shared memory: K o e^c and K o e^{c_last-c} until the first products, then U
+// over them; [dO; -dR] at the top of the operand region; the T^T, P^T and T
+// images in the raw region once the raw chunk is consumed; M or dM staged as
+// [f][n] over the raw region after the second products.  U, [dO; -dR], M and
+// dM use the padded layout (LBO 144), which their lane-per-column stores need.
+constexpr uint32_t OP_KE = OP, OP_KED = OP + 32768, OP_U = OP, OP_PBR = OP + 36864, OP_DO = OP + 73728;
+constexpr uint32_t R_TT = 16384, R_MB = 0;
+constexpr uint32_t PAD_SBO = 128 * 36;  // bytes per 8 rows of a padded 128-wide K tile
+static_assert(OP_DO + 2 * 64 * PAD_SBO / 8 <= SMALL && OP_PBR + 1024 <= OP_DO && R_MB + 16 * PAD_SBO <= OP &&
+                  R_TT + 16384 <= R_P,
+              "gradient-kernel shared-memory map");
 constexpr uint32_t TM_M = 0, TM_U = 0, TM_QK = 0, TM_DM = 128, TM_DR = 128, TM_KED = 128, TM_DOT = 256,
-                   TM_PA = 256, TM_APA = 320, TM_APB = 384, TM_X = 320, TM_DU = 384;
+                   TM_PA = 256, TM_X = 320, TM_DU = 384;
 }  // namespace tcg
 
-__device__ __forceinline__ float warp_sum(float x) {
+// Sums over the warp's 32 lanes of 32 values at once: lane l returns
+// sum over lanes of v[l] (31 shuffles instead of 32 x 5).  v is clobbered.
+__device__ __forceinline__ float warp_sum32(float (&v)[32], int lane) {
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
-  return x;
+  for (int off = 16; off > 0; off >>= 1) {
+    const bool up = (lane & off) != 0;
+#pragma unroll
+    for (int k = 0; k < off; ++k) {
+      const float send = up ? v[k] : v[k + off];
+      const float keep = up ? v[k + off] : v[k];
+      v[k] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+  return v[0];
 }
 
 __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
@@ -328,7 +346,7 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
   const float* sC = cx.c();
   // per-subpartition partial sums, added in a fixed order (deterministic)
   float* partEl = reinterpret_cast<float*>(sm + R_AH);   // [4][128], once Ah is in the record
-  float* partBr = reinterpret_cast<float*>(sm + OP_TT);  // [4][64], once T^T is consumed
+  float* partBr = reinterpret_cast<float*>(sm + OP_PBR);  // [4][64], once K o e^{c_last-c} is consumed
 
   if (cx.warp == 0) tmem_alloc(sTm, 512);
   if (tid == 0) mbar_init(bar, 1);
@@ -341,10 +359,19 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
   bool failed = false;
 
   do {
-    // ---------------------------------------------------------------- interaction products
-    load_raw(cx, qg, kg, dog, a.g, a.beta, b, T, t0, L, a.H, a.HV, h, hv);
+    // ---------------------------------------------------------------- loads
+    const float* irec = a.inter + (head * NT + ch) * INTER_REC;  // P^T, T, T^T images of this chunk (forward)
+    const int dm_idx = (2 * ch + 1 < NT32) ? 2 * ch + 1 : 2 * ch;
+    const float* mst = a.states + (head * NT32 + 2 * ch) * (size_t)(KD * VD);  // M: state entering the chunk
+    const float* dmst = a.dstates + (head * NT32 + dm_idx) * (size_t)(KD * VD);  // dM: gradient of the leaving state
+    load_raw_issue(cx, qg, kg, dog, a.g, a.beta, b, T, t0, L, a.H, a.HV, h, hv);
+    if (tid < 16) prefetch_l2(mst + tid * 1024, 4096);
+    else if (tid < 32) prefetch_l2(dmst + (tid - 16) * 1024, 4096);
+    else if (tid == 32) prefetch_l2(irec, 2 * 16384);
+    else if (tid == 33) prefetch_l2(irec + INTER_TT, 16384);
+    else if (tid >= 64 && tid < 64 + L) prefetch_l2(vg + (((size_t)b * T + t0 + tid - 64) * a.HV + hv) * VD, VD * 2);
+    load_raw_wait();
     cumsum_span(cx);
-    const float* irec = a.inter + (head * NT + ch) * INTER_REC;  // P^T, T of this chunk (forward)
 
     // ---------------------------------------------------------------- K o e^c, K o e^{c_last-c}, dO, dO^T
     {
@@ -366,7 +393,7 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
         }
         st_tf32x4(sm, OP_KE + kmaj(i, fq, 128), kf[0] * e[0], kf[1] * e[1], kf[2] * e[2], kf[3] * e[3]);
         st_tf32x4(sm, OP_KED + kmaj(i, fq, 128), kf[0] * ed[0], kf[1] * ed[1], kf[2] * ed[2], kf[3] * ed[3]);
-        st_tf32x4(sm, OP_DO + kmaj(i, fq, 128), df[0], df[1], df[2], df[3]);
+        st_tf32x4(sm, OP_DO + kmaj_pad(i, fq, 128), df[0], df[1], df[2], df[3]);
       }
       uint32_t r[32];
       const unsigned char* col = sm + RAW_X + Lr * 2;
@@ -379,39 +406,28 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
     fence_async_smem();
     fence_before();
     __syncthreads();  // raw inputs consumed
-    for (int x = tid; x < C * 16; x += NTH) {  // P^T and T diag(beta), (row i, K = j) operands
-      const int i = x >> 4, j4 = (x & 15) * 4;
-      const float4 p = *reinterpret_cast<const float4*>(irec + i * 64 + j4);
-      st_tf32x4(sm, R_P + kmaj(i, j4, 64), p.x, p.y, p.z, p.w);
-      const float4 t = *reinterpret_cast<const float4*>(irec + INTER_T + i * 64 + j4);
-      st_tf32x4(sm, R_T + kmaj(i, j4, 64), t.x * sBeta[j4], t.y * sBeta[j4 + 1], t.z * sBeta[j4 + 2],
-                t.w * sBeta[j4 + 3]);
-    }
-    for (int x = tid; x < C * 16; x += NTH) {  // T^T: element (i, j) = T[j][i]
-      const int i = x & 63, j4 = (x >> 6) * 4;
-      const float* tcol = irec + INTER_T + i;
-      st_tf32x4(sm, OP_TT + kmaj(i, j4, 64), tcol[j4 * 64], tcol[(j4 + 1) * 64], tcol[(j4 + 2) * 64],
-                tcol[(j4 + 3) * 64]);
-    }
+    copy_image(cx, R_P, irec);               // P^T: (row i, K j) = P[j][i]
+    copy_image(cx, R_T, irec + INTER_T);     // T:   (row i, K j) = T[i][j]
+    copy_image(cx, R_TT, irec + INTER_TT);   // T^T: (row i, K j) = T[j][i]
 
     // ---------------------------------------------------------------- M^T, dM^T into TMEM; dEl
     {
-      const int dm_idx = (2 * ch + 1 < NT32) ? 2 * ch + 1 : 2 * ch;
       for (int cb = 0; cb < 2; ++cb) {
         const int f0 = hcol * 64 + cb * 32;
         uint32_t rm[32], rd[32];
-        const float* ms = a.states + ((head * NT32 + 2 * ch) * KD + f0) * VD + Lr;
-        const float* ds = a.dstates + ((head * NT32 + dm_idx) * KD + f0) * VD + Lr;
+        float pr[32];
+        const float* ms = mst + f0 * VD + Lr;
+        const float* ds = dmst + f0 * VD + Lr;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           const float mv = ms[(size_t)j * VD], dv = ds[(size_t)j * VD];
           rm[j] = __float_as_uint(mv);
           rd[j] = __float_as_uint(dv);
-          const float s = warp_sum(mv * dv);
-          if (lane == 0) partEl[cx.sub * KD + f0 + j] = s;
+          pr[j] = mv * dv;
         }
         tmem_st32(tm + lo + TM_M + f0, rm);
         tmem_st32(tm + lo + TM_DM + f0, rd);
+        partEl[cx.sub * KD + f0 + lane] = warp_sum32(pr, lane);
       }
       tmem_wait_st();
     }
@@ -421,6 +437,7 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
       const int i = hcol * 32 + jj;
       vT[jj] = (i < L) ? __bfloat162float(vg[(((size_t)b * T + t0 + i) * a.HV + hv) * VD + Lr]) : 0.f;
     }
+    cp_async_wait_all();
     fence_async_smem();
     fence_before();
     __syncthreads();
@@ -437,23 +454,27 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
       commit(bar);
     }
     if (!wait_mma(bar, phase)) { failed = true; break; }
-    {  // X^T = V^T - X'^T
+    float xs[32];  // X^T = V^T - X'^T (lane n, rows i of this warp half), kept for dbeta_R
+    {
       float x[32];
       uint32_t r[32];
       tmem_ld32(tm + lo + TM_X + hcol * 32, x);
 #pragma unroll
-      for (int jj = 0; jj < 32; ++jj) r[jj] = tf32_rna(vT[jj] - x[jj]);
+      for (int jj = 0; jj < 32; ++jj) {
+        xs[jj] = vT[jj] - x[jj];
+        r[jj] = tf32_rna(sBeta[hcol * 32 + jj] * xs[jj]);
+      }
       tmem_st32(tm + lo + TM_X + hcol * 32, r);
       tmem_wait_st();
     }
     fence_before();
     __syncthreads();
-    if (tid == 0) {  // U^T = X^T (T diag(beta))^T ; dR^T = dU^T T
+    if (tid == 0) {  // U^T = (X^T diag(beta)) T^T ; dR^T = dU^T T
       fence_after();
       const uint32_t id = idesc_tf32(128, 64);
       for (int ks = 0; ks < 8; ++ks) {
         mma_ts(tm + TM_U, tm + TM_X + ks * 8, desc(sb + R_T + ks * 256, 2048), id, ks > 0);
-        mma_ts(tm + TM_DR, tm + TM_DU + ks * 8, desc(sb + OP_TT + ks * 256, 2048), id, ks > 0);
+        mma_ts(tm + TM_DR, tm + TM_DU + ks * 8, desc(sb + R_TT + ks * 256, 2048), id, ks > 0);
       }
       commit(bar);
     }
@@ -461,24 +482,23 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
 
     // ---------------------------------------------------------------- dv, dbeta_R; U and -dR as [i][n] operands
     {
-      float u[32], dr[32], x[32];
+      float u[32], dr[32];
       tmem_ld32(tm + lo + TM_U + hcol * 32, u);
       tmem_ld32(tm + lo + TM_DR + hcol * 32, dr);
-      tmem_ld32(tm + lo + TM_X + hcol * 32, x);
 #pragma unroll
       for (int jj = 0; jj < 32; ++jj) {
         const int i = hcol * 32 + jj;
         if (i < L) dvg[(((size_t)b * T + t0 + i) * a.HV + hv) * VD + Lr] = __float2bfloat16_rn(sBeta[i] * dr[jj]);
-        const float s = warp_sum(dr[jj] * x[jj]);
-        if (lane == 0) partBr[cx.sub * C + i] = s;
-        st_tf32(sm, OP_U + kmaj(i, Lr, 128), u[jj]);
-        st_tf32(sm, OP_DO + kmaj(64 + i, Lr, 128), -dr[jj]);
+        st_tf32(sm, OP_U + kmaj_pad(i, Lr, 128), u[jj]);
+        st_tf32(sm, OP_DO + kmaj_pad(64 + i, Lr, 128), -dr[jj]);
+        xs[jj] *= dr[jj];
       }
+      partBr[cx.sub * C + hcol * 32 + lane] = warp_sum32(xs, lane);
     }
     // M as [f][n] for the sums over n
     for (int e = tid; e < KD * 32; e += NTH) {
       const int f = e >> 5, n4 = (e & 31) * 4;
-      cp_async16(sb + R_MB + kmaj(f, n4, 128), a.states + ((head * NT32 + 2 * ch) * KD + f) * VD + n4, true);
+      cp_async16(sb + R_MB + kmaj_pad(f, n4, 128), mst + f * VD + n4, true);
     }
     cp_async_wait_all();
     fence_async_smem();
@@ -487,18 +507,17 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
     if (tid == 0) {  // [dP; dA] = [dO; -dR] U^T ; [dQE; dKE'] = [dO; -dR] M^T
       fence_after();
       for (int ks = 0; ks < 16; ++ks) {
-        const uint64_t aD = desc(sb + OP_DO + ks * 256, 4096);
-        mma_ss(tm + TM_PA, aD, desc(sb + OP_U + ks * 256, 4096), idesc_tf32(128, 64), ks > 0);
-        mma_ss(tm + TM_QK, aD, desc(sb + R_MB + ks * 256, 4096), idesc_tf32(128, 128), ks > 0);
+        const uint64_t aD = desc(sb + OP_DO + ks * 288, PAD_SBO, 144);
+        mma_ss(tm + TM_PA, aD, desc(sb + OP_U + ks * 288, PAD_SBO, 144), idesc_tf32(128, 64), ks > 0);
+        mma_ss(tm + TM_QK, aD, desc(sb + R_MB + ks * 288, PAD_SBO, 144), idesc_tf32(128, 128), ks > 0);
       }
       commit(bar);
     }
     if (!wait_mma(bar, phase)) { failed = true; break; }
     {  // dM as [f][n]
-      const int dm_idx = (2 * ch + 1 < NT32) ? 2 * ch + 1 : 2 * ch;
       for (int e = tid; e < KD * 32; e += NTH) {
         const int f = e >> 5, n4 = (e & 31) * 4;
-        cp_async16(sb + R_MB + kmaj(f, n4, 128), a.dstates + ((head * NT32 + dm_idx) * KD + f) * VD + n4, true);
+        cp_async16(sb + R_MB + kmaj_pad(f, n4, 128), dmst + f * VD + n4, true);
       }
       cp_async_wait_all();
     }
@@ -507,8 +526,8 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
     if (tid == 0) {  // dKEd = U dM^T
       fence_after();
       for (int ks = 0; ks < 16; ++ks)
-        mma_ss(tm + TM_KED, desc(sb + OP_U + ks * 256, 4096), desc(sb + R_MB + ks * 256, 4096), idesc_tf32(64, 128),
-               ks > 0);
+        mma_ss(tm + TM_KED, desc(sb + OP_U + ks * 288, PAD_SBO, 144), desc(sb + R_MB + ks * 288, PAD_SBO, 144),
+               idesc_tf32(64, 128), ks > 0);
       commit(bar);
     }
     if (!wait_mma(bar, phase)) { failed = true; break; }

@@ -99,7 +99,9 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_tc_kernel(FwdArgs a) {
 
   for (int ch = 0; ch < NT; ++ch) {
     const int t0 = ch * C, L = min(C, T - t0);
-    load_raw(cx, qg, kg, vg, a.g, a.beta, b, T, t0, L, a.H, a.HV, h, hv);
+    load_raw_issue(cx, qg, kg, vg, a.g, a.beta, b, T, t0, L, a.H, a.HV, h, hv);
+    if (ch + 1 < NT) prefetch_chunk(cx, qg, kg, vg, a.g, b, T, t0 + C, min(C, T - t0 - C), a.H, a.HV, h, hv);
+    load_raw_wait();
     const bool wide = cumsum_span(cx);
     build_op1_and_issue(cx, a.scale, tm + TM_APA, tm + TM_APB, bar);
     if (!wait_mma(bar, phase)) { failed = true; break; }
@@ -150,21 +152,23 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_tc_kernel(FwdArgs a) {
     float* irec = a.inter ? a.inter + (head * NT + ch) * INTER_REC : nullptr;
     readout_ap(cx, tm + TM_APA, tm + TM_APB, false, wide, pw, irec);
     invert(cx);
-    if (irec) {  // T and Ah for the backward (P^T was stored by the read-out)
+    {  // T as the operand image (rows i, K = j); with a record also its T, T^T images and Ah
       const float* tr = reinterpret_cast<const float*>(sm + R_TROW);
-      const float* ah = reinterpret_cast<const float*>(sm + R_AH);
-      for (int x = tid; x < C * C; x += NTH) {
-        const int o = (x >> 6) * 65 + (x & 63);
-        irec[INTER_T + x] = tr[o];
-        irec[INTER_AH + x] = ah[o];
-      }
-    }
-    {
-      const float* tr = reinterpret_cast<const float*>(sm + R_TROW);
-      for (int x = tid; x < C * 16; x += NTH) {
-        const int i = x >> 4, j4 = (x & 15) * 4;
+      for (int x = tid; x < C * 16; x += NTH) {  // 16-byte piece x of the image: x * 16 = kmaj(i, j4, 64)
+        const int i = ((x >> 7) << 3) | (x & 7), j4 = ((x >> 3) & 15) * 4;
         const float* p = tr + i * 65 + j4;
-        st_tf32x4(sm, R_T + kmaj(i, j4, 64), p[0], p[1], p[2], p[3]);
+        const uint4 t = make_uint4(tf32_rna(p[0]), tf32_rna(p[1]), tf32_rna(p[2]), tf32_rna(p[3]));
+        *reinterpret_cast<uint4*>(sm + R_T + x * 16) = t;
+        if (irec) {
+          const float* pc = tr + j4 * 65 + i;
+          *reinterpret_cast<uint4*>(irec + INTER_T + x * 4) = t;
+          *reinterpret_cast<uint4*>(irec + INTER_TT + x * 4) =
+              make_uint4(tf32_rna(pc[0]), tf32_rna(pc[65]), tf32_rna(pc[130]), tf32_rna(pc[195]));
+        }
+      }
+      if (irec) {
+        const float* ah = reinterpret_cast<const float*>(sm + R_AH);
+        for (int x = tid; x < C * C; x += NTH) irec[INTER_AH + x] = ah[(x >> 6) * 65 + (x & 63)];
       }
     }
     fence_async_smem();

@@ -15,10 +15,16 @@ constexpr int FWD_VBLOCK = 32;   // V columns per CTA in the chunked kernels
 // [dQE; dKE'] as [f][i'] (128 x 128, i' < 64 dQE), dKEd as [f][i] (128 x 64),
 // dbeta_R [64], dEl [128].
 // Per-(b, hv, 64-step chunk) interaction record that the tensor-core forward
-// stores with a workspace (floats): P^T row-major [j][i] at 0, T row-major at
-// INTER_T, Ah row-major at INTER_AH.  The backward reads it instead of
-// recomputing the interaction products and the inverse.
-constexpr int INTER_T = 4096, INTER_AH = 8192, INTER_REC = 12288;
+// stores with a workspace (floats).  Three 64 x 64 tf32 operand images in the
+// K-major canonical layout of the tensor-core kernels (element (r, k) at
+// float (r / 8) * 512 + (k / 4) * 32 + (r % 8) * 4 + k % 4), so that the
+// backward copies them into shared memory unchanged:
+//   [0, INTER_T)         P^T image:  (r, k) = P[k][r]
+//   [INTER_T, INTER_AH)  T image:    (r, k) = T[r][k]
+//   [INTER_TT, +4096)    T^T image:  (r, k) = T[k][r]
+// and Ah row-major at INTER_AH.  The backward reads it instead of recomputing
+// the interaction products and the inverse.
+constexpr int INTER_T = 4096, INTER_AH = 8192, INTER_TT = 12288, INTER_REC = 16384;
 constexpr int G_AH = 0, G_PA = 4096, G_QK = 12288, G_KED = 28672, G_DBR = 36864, G_DEL = 36928,
               GREC = 37120;
 

@@ -53,6 +53,12 @@ __device__ __forceinline__ uint32_t tf32_rna(float x) {
   return r;
 }
 
+// Hint: bring [p, p + bytes) into L2 (p 16-byte aligned, bytes a multiple of
+// 16, the whole range inside one allocation).
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

@@ -73,8 +73,8 @@ __device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast
 
 // Asynchronous load of one chunk: q, k rows of query/key head h, x rows of
 // value head hv (v or dO), g rows and beta; rows past the sequence end are
-// zero.  Completes (wait + barrier) before returning.
-__device__ __forceinline__ void load_raw(const Ctx& c, const __nv_bfloat16* q, const __nv_bfloat16* k,
+// zero.  Issues the copies only; load_raw_wait completes them.
+__device__ __forceinline__ void load_raw_issue(const Ctx& c, const __nv_bfloat16* q, const __nv_bfloat16* k,
                                          const __nv_bfloat16* x, const float* g, const float* beta,
                                          int b, int T, int t0, int L, int H, int HV, int h, int hv) {
   using namespace tc;
@@ -93,9 +93,35 @@ __device__ __forceinline__ void load_raw(const Ctx& c, const __nv_bfloat16* q, c
     cp_async16(c.sb + RAW_C + (i * LDCF + vec * 4) * 4, g + (t * HV + hv) * KD + vec * 4, ok);
   }
   if (c.tid < C) c.beta()[c.tid] = (c.tid < L) ? beta[((size_t)b * T + t0 + c.tid) * HV + hv] : 0.f;
-  cp_async_wait_all();
+}
+__device__ __forceinline__ void load_raw_wait() {
+  tc::cp_async_wait_all();
   __syncthreads();
 }
+
+// L2 prefetch of one chunk's q, k, x (v or dO) and g rows, for a chunk that a
+// later load_raw will read; one row of one tensor per thread.
+__device__ __forceinline__ void prefetch_chunk(const Ctx& c, const __nv_bfloat16* q, const __nv_bfloat16* k,
+                                               const __nv_bfloat16* x, const float* g, int b, int T, int t0,
+                                               int L, int H, int HV, int h, int hv) {
+  const int i = c.tid & 63, which = c.tid >> 6;
+  if (i >= L) return;
+  const size_t t = (size_t)b * T + t0 + i;
+  if (which == 0) tc::prefetch_l2(q + (t * H + h) * KD, KD * 2);
+  else if (which == 1) tc::prefetch_l2(k + (t * H + h) * KD, KD * 2);
+  else if (which == 2) tc::prefetch_l2(x + (t * HV + hv) * VD, VD * 2);
+  else tc::prefetch_l2(g + (t * HV + hv) * KD, KD * 4);
+}
+
+// Asynchronous copy of one 64 x 64 operand image of an interaction record
+// (16 KB) into shared memory at `dst`; completes with cp_async_wait_all.
+__device__ __forceinline__ void copy_image(const Ctx& c, uint32_t dst, const float* src) {
+#pragma unroll
+  for (int e = c.tid; e < 1024; e += NTH) tc::cp_async16(c.sb + dst + e * 16, src + e * 4, true);
+}
+
+// float index of element (r, k) in a 64 x 64 record image
+__device__ __forceinline__ int img(int r, int k) { return (int)(tc::kmaj(r, k, 64) >> 2); }
 
 // In-chunk cumulative decay (natural log summed, stored times log2(e)).
 // Returns, block-uniformly, whether some half's decay from its middle row to
@@ -232,8 +258,8 @@ __device__ __forceinline__ uint32_t p_off(int i, int j, bool transP) {
 }
 
 // Reads Ah (row-major, stride 65, at R_AH) and P (tf32 operand at R_P) out of
-// the two interaction products; the raw region must be free.  Ends with a
-// barrier.
+// the two interaction products; the raw region must be free.  With `pt` it
+// also stores the P^T image of the interaction record.  Ends with a barrier.
 __device__ __forceinline__ void readout_ap(const Ctx& c, uint32_t tm_apa, uint32_t tm_apb, bool transP,
                                            bool wide, const Pairwise& pw, float* pt = nullptr) {
   using namespace tc;
@@ -253,7 +279,7 @@ __device__ __forceinline__ void readout_ap(const Ctx& c, uint32_t tm_apa, uint32
         sAh[i * 65 + j] = val;
       } else {
         st_tf32(c.sm, p_off(i, j, transP), val);
-        if (pt) pt[j * 64 + i] = val;
+        if (pt) pt[img(j, i)] = __uint_as_float(tf32_rna(val));
       }
     }
   }
@@ -269,7 +295,7 @@ __device__ __forceinline__ void readout_ap(const Ctx& c, uint32_t tm_apa, uint32
           sAh[(32 + r) * 65 + j] = v[jj];
         } else {
           st_tf32(c.sm, p_off(r, j, transP), v[jj]);
-          if (pt) pt[j * 64 + r] = v[jj];
+          if (pt) pt[img(j, r)] = __uint_as_float(tf32_rna(v[jj]));
         }
       }
     }
@@ -281,7 +307,7 @@ __device__ __forceinline__ void readout_ap(const Ctx& c, uint32_t tm_apa, uint32
       if (pw.kind == 0 && j < pw.i) sAh[pw.i * 65 + j] = pw.v[jj];
       if (pw.kind == 1 && j <= pw.i) {
         st_tf32(c.sm, p_off(pw.i, j, transP), pw.v[jj]);
-        if (pt) pt[j * 64 + pw.i] = pw.v[jj];
+        if (pt) pt[img(j, pw.i)] = __uint_as_float(tf32_rna(pw.v[jj]));
       }
     }
     __syncthreads();
