@@ -69,8 +69,16 @@ static size_t inter_bytes(int B, int T, int HV, int K, int V) {
   return (size_t)B * HV * NT64 * INTER_REC * sizeof(float);
 }
 
+// per-chunk operand images of the two-kernel tensor-core forward (K = V = 128)
+static size_t img_bytes(int B, int T, int HV, int K, int V) {
+  if (K != 128 || V != 128) return 0;
+  const size_t NT64 = (size_t)(T + 63) / 64;
+  return (size_t)B * HV * NT64 * FWI_BYTES;
+}
+
+// training forward: [states | interaction records | chunk images]
 static size_t fwd_ws_bytes(int B, int T, int HV, int K, int V) {
-  return states_bytes(B, T, HV, K, V) + inter_bytes(B, T, HV, K, V);
+  return states_bytes(B, T, HV, K, V) + inter_bytes(B, T, HV, K, V) + img_bytes(B, T, HV, K, V);
 }
 
 }  // namespace kda
@@ -95,17 +103,30 @@ size_t kda_fwd_workspace_bytes(int B, int T, int HV, int K, int V) {
   return fwd_ws_bytes(B, T, HV, K, V);
 }
 
+size_t kda_fwd_scratch_bytes(int B, int T, int HV, int K, int V) {
+  if (B < 1 || T < 1 || HV < 1 || K < 1 || V < 1) return 0;
+  return img_bytes(B, T, HV, K, V);
+}
+
 static size_t grads_record_bytes(int B, int T, int HV, int K, int V) {
   if (K != 128 || V != 128) return 0;
   const size_t NT64 = (size_t)(T + 63) / 64;
   return (size_t)B * HV * NT64 * GREC * sizeof(float);
 }
 
-size_t kda_bwd_workspace_bytes(int B, int T, int H, int HV, int K, int V) {
-  if (B < 1 || T < 1 || H < 1 || HV < 1 || K < 1 || V < 1 || HV % H) return 0;
-  size_t bytes = fwd_ws_bytes(B, T, HV, K, V) + states_bytes(B, T, HV, K, V);
+// the part of the backward workspace after [states | interaction records]:
+// the forward's chunk images, which the backward then overwrites with
+// [state gradients | dq/dk partials | gradient records]
+static size_t bwd_tail_bytes(int B, int T, int H, int HV, int K, int V) {
+  size_t bytes = states_bytes(B, T, HV, K, V);
   if (HV > H) bytes += 2 * (size_t)B * T * HV * K * sizeof(float);
   return bytes + grads_record_bytes(B, T, HV, K, V);
+}
+
+size_t kda_bwd_workspace_bytes(int B, int T, int H, int HV, int K, int V) {
+  if (B < 1 || T < 1 || H < 1 || HV < 1 || K < 1 || V < 1 || HV % H) return 0;
+  const size_t tail = bwd_tail_bytes(B, T, H, HV, K, V), img = img_bytes(B, T, HV, K, V);
+  return states_bytes(B, T, HV, K, V) + inter_bytes(B, T, HV, K, V) + (tail > img ? tail : img);
 }
 
 int kda_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
@@ -116,15 +137,25 @@ int kda_fwd(const void* q, const void* k, const void* v, const float* g, const f
   if (rc) return rc;
   if (!q || !k || !v || !g || !beta || !o)
     return set_error(KDA_ERR_NULL, "kda_fwd: q, k, v, g, beta and o must be non-NULL");
+  float *states = nullptr, *inter = nullptr;
+  unsigned char* img = nullptr;
   if (workspace) {
-    if (workspace_bytes < fwd_ws_bytes(B, T, HV, K, V))
-      return set_error(KDA_ERR_WORKSPACE, "kda_fwd: workspace smaller than kda_fwd_workspace_bytes()");
     if (!aligned16(workspace)) return set_error(KDA_ERR_ARG, "kda_fwd: workspace must be 16-byte aligned");
+    char* ws = static_cast<char*>(workspace);
+    const size_t sb = states_bytes(B, T, HV, K, V), ib = inter_bytes(B, T, HV, K, V);
+    const size_t gb = img_bytes(B, T, HV, K, V);
+    if (workspace_bytes >= fwd_ws_bytes(B, T, HV, K, V)) {  // training: states for the backward
+      states = reinterpret_cast<float*>(ws);
+      inter = ib ? reinterpret_cast<float*>(ws + sb) : nullptr;
+      img = gb ? reinterpret_cast<unsigned char*>(ws + sb + ib) : nullptr;
+    } else if (gb && workspace_bytes >= gb) {  // scratch only
+      img = reinterpret_cast<unsigned char*>(ws);
+    } else {
+      return set_error(KDA_ERR_WORKSPACE,
+                       "kda_fwd: workspace smaller than kda_fwd_scratch_bytes() and kda_fwd_workspace_bytes()");
+    }
   }
-  float* inter = (workspace && inter_bytes(B, T, HV, K, V))
-                     ? reinterpret_cast<float*>(static_cast<char*>(workspace) + states_bytes(B, T, HV, K, V))
-                     : nullptr;
-  FwdArgs a{q, k, v, g, beta, S0, o, S_T, static_cast<float*>(workspace), inter, scale, B, T, H, HV, K, V};
+  FwdArgs a{q, k, v, g, beta, S0, o, S_T, states, inter, img, scale, B, T, H, HV, K, V};
   return launch_fwd(a, dtype, static_cast<cudaStream_t>(stream));
 }
 
@@ -161,24 +192,29 @@ int kda_bwd(const void* q, const void* k, const void* v, const float* g, const f
   const size_t sb = states_bytes(B, T, HV, K, V);
   char* ws = static_cast<char*>(workspace);
   float* states = reinterpret_cast<float*>(ws);
-  const size_t fb = fwd_ws_bytes(B, T, HV, K, V);
-  float* inter = inter_bytes(B, T, HV, K, V) ? reinterpret_cast<float*>(ws + sb) : nullptr;
-  float* dstates = reinterpret_cast<float*>(ws + fb);
+  const size_t ib = inter_bytes(B, T, HV, K, V);
+  float* inter = ib ? reinterpret_cast<float*>(ws + sb) : nullptr;
+  unsigned char* img = img_bytes(B, T, HV, K, V) ? reinterpret_cast<unsigned char*>(ws + sb + ib) : nullptr;
+  float* dstates = reinterpret_cast<float*>(ws + sb + ib);  // over the forward's chunk images
   float *dq_part = nullptr, *dk_part = nullptr;
-  size_t off = fb + sb;
+  size_t off = sb + ib + sb;
   if (HV > H) {
     dq_part = reinterpret_cast<float*>(ws + off);
     dk_part = dq_part + (size_t)B * T * HV * K;
     off += 2 * (size_t)B * T * HV * K * sizeof(float);
   }
   float* gws = grads_record_bytes(B, T, HV, K, V) ? reinterpret_cast<float*>(ws + off) : nullptr;
-  if (!(flags & KDA_BWD_STATES_FROM_FWD)) {
-    FwdArgs fa{q, k, v, g, beta, S0, nullptr, nullptr, states, inter, scale, B, T, H, HV, K, V};
-    rc = launch_fwd(fa, dtype, st);
-    if (rc) return rc;
-  }
   BwdArgs a{q, k, v, dO, g, beta, dS_T, states, inter, dstates, dq, dk, dv, dg, dbeta, dS0,
             dq_part, dk_part, gws, scale, B, T, H, HV, K, V};
+  FwdArgs fa{q, k, v, g, beta, S0, nullptr, nullptr, states, inter, img, scale, B, T, H, HV, K, V};
+  // The tensor-core forward keeps only the state entering each 64-step chunk,
+  // which is all the tensor-core backward reads; the CUDA-core backward needs
+  // every 32-step state, so it gets them from the CUDA-core forward.
+  const bool tc_bwd = bwd_tc_eligible(a, dtype);
+  if (!(flags & KDA_BWD_STATES_FROM_FWD) || (!tc_bwd && fwd_tc_eligible(fa, dtype))) {
+    rc = tc_bwd ? launch_fwd(fa, dtype, st) : launch_fwd_ffma(fa, dtype, st);
+    if (rc) return rc;
+  }
   return launch_bwd(a, dtype, st);
 }
 

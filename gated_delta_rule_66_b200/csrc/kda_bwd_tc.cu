@@ -1,6 +1,6 @@
 // Tensor-core (tcgen05) reverse pass of the KDA backward for K = V = 128,
-// bf16 q/k/dO, fp32 g/beta: the gradient of the state leaving every 32-step
-// block, and dS0.
+// bf16 q/k/dO, fp32 g/beta: the gradient of the state leaving every 64-step
+// chunk, and dS0.
 //
 // From the chunk algebra (kda_tc_chunk.cuh) the gradient of the state entering
 // a chunk, given the gradient dM of the state leaving it, is
@@ -14,11 +14,9 @@
 //   dR^T  = dU^T T
 //   dM_in^T = dM^T diag(e^{c_last}) + dO^T (Q~ o e^c) - dR^T (diag(beta) K o e^c)
 // P and T come from the forward's interaction record as ready operand images.
-// The state gradient at the chunk's midpoint (leaving step 31), needed for the
-// 32-step granularity of the per-chunk gradient kernel, is the same formula
-// over the second half alone:
-//   dM_mid^T = dM^T diag(e^{c_last - c_31}) + dO^T[:,32:] (Q~ o e^{c-c_31})[32:]
-//              - dR^T[:,32:] (diag(beta) K o e^{c-c_31})[32:].
+// The gradient of the state leaving every chunk is stored (at the chunk's odd
+// index of the 32-step state layout, or its even one when the sequence ends in
+// the chunk's first half); the per-chunk gradient kernel reads it there.
 #include <cuda_bf16.h>
 
 #include "kda_internal.h"
@@ -30,10 +28,8 @@ __device__ unsigned int g_kda_bwd_device_error;  // this file's kernels (one fla
 
 namespace tcb {
 using namespace tcc;
-constexpr uint32_t OP_KED = OP, OP_QET = OP + 32768, OP_NKET = OP + 65536, OP_Q2T = OP + 98304,
-                   OP_NK2T = OP + 114688;
-constexpr uint32_t TM_S = 0, TM_DU = 128, TM_DR = 192, TM_DOT = 256,
-                   TM_MID = 384;  // mid-chunk gradient (the interaction tile is read by then)
+constexpr uint32_t OP_KED = OP, OP_QET = OP + 32768, OP_NKET = OP + 65536;
+constexpr uint32_t TM_S = 0, TM_DU = 128, TM_DR = 192, TM_DOT = 256;
 }  // namespace tcb
 
 __global__ void __launch_bounds__(256, 1) kda_bwd_dstate_tc_kernel(BwdArgs a) {
@@ -61,7 +57,6 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_dstate_tc_kernel(BwdArgs a) {
   const __nv_bfloat16* dog = static_cast<const __nv_bfloat16*>(a.dO);
   float* sBeta = cx.beta();
   float* sEl = reinterpret_cast<float*>(sm + S_EL);
-  float* sEh = reinterpret_cast<float*>(sm + S_EMID);  // e^{c_last - c_31}
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + S_BAR);
   uint32_t* sTm = reinterpret_cast<uint32_t*>(sm + S_TMEM);
   const float* sC = cx.c();
@@ -103,44 +98,39 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_dstate_tc_kernel(BwdArgs a) {
     cumsum_span(cx);
 
     // ---------------------------------------------------------------- operands of the gradient products
-    const int fq = item_f(cx);
     {
-      const float4 c63v = ld4(sC + 63 * LDCF + fq), r31 = ld4(sC + 31 * LDCF + fq);
-      const float c63[4] = {c63v.x, c63v.y, c63v.z, c63v.w}, c31[4] = {r31.x, r31.y, r31.z, r31.w};
-      for (int m = 0; m < 8; ++m) {
-        const int i = item_row(cx, m);
-        const float4 c4 = ld4(sC + i * LDCF + fq);
-        const float c[4] = {c4.x, c4.y, c4.z, c4.w};
-        float kf[4], qf[4];
-        bf16x4(sm + RAW_K + i * 256 + fq * 2, kf);
-        bf16x4(sm + RAW_Q + i * 256 + fq * 2, qf);
-        const float nb = -sBeta[i];
-        float e[4], ed[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          qf[u] *= a.scale;
-          e[u] = ex2(c[u]);
-          ed[u] = ex2(c63[u] - c[u]);
+      {  // K o e^{c_last-c} as [i][f]: thread items of 4 channels, 16-byte stores
+        const int fq = item_f(cx);
+        const float4 c63v = ld4(sC + 63 * LDCF + fq);
+        const float c63[4] = {c63v.x, c63v.y, c63v.z, c63v.w};
+        for (int m = 0; m < 8; ++m) {
+          const int i = item_row(cx, m);
+          const float4 c4 = ld4(sC + i * LDCF + fq);
+          float kf[4];
+          bf16x4(sm + RAW_K + i * 256 + fq * 2, kf);
+          st_tf32x4(sm, OP_KED + kmaj(i, fq, 128), kf[0] * ex2(c63[0] - c4.x), kf[1] * ex2(c63[1] - c4.y),
+                    kf[2] * ex2(c63[2] - c4.z), kf[3] * ex2(c63[3] - c4.w));
         }
-        st_tf32x4(sm, OP_KED + kmaj(i, fq, 128), kf[0] * ed[0], kf[1] * ed[1], kf[2] * ed[2], kf[3] * ed[3]);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          st_tf32(sm, OP_QET + kmaj(fq + u, i, 64), qf[u] * e[u]);
-          st_tf32(sm, OP_NKET + kmaj(fq + u, i, 64), nb * kf[u] * e[u]);
-        }
-        if (i >= 32) {
+      }
+      {  // (Q~ o e^c)^T and -(diag(beta) K o e^c)^T as [f][i]: one channel x 4 rows, 16-byte stores
+        const int f = tid & 127;
+        const __nv_bfloat16* qcol = reinterpret_cast<const __nv_bfloat16*>(sm + RAW_Q) + f;
+        const __nv_bfloat16* kcol = reinterpret_cast<const __nv_bfloat16*>(sm + RAW_K) + f;
+        for (int m = 0; m < 8; ++m) {
+          const int i0 = ((tid >> 7) + 2 * m) * 4;
+          float qe[4], nke[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const float x2 = ex2(c[u] - c31[u]);
-            st_tf32(sm, OP_Q2T + kmaj(fq + u, i - 32, 32), qf[u] * x2);
-            st_tf32(sm, OP_NK2T + kmaj(fq + u, i - 32, 32), nb * kf[u] * x2);
+            const int i = i0 + u;
+            const float e = ex2(sC[i * LDCF + f]);
+            qe[u] = a.scale * __bfloat162float(qcol[i * 128]) * e;
+            nke[u] = -sBeta[i] * __bfloat162float(kcol[i * 128]) * e;
           }
+          st_tf32x4(sm, OP_QET + kmaj(f, i0, 64), qe[0], qe[1], qe[2], qe[3]);
+          st_tf32x4(sm, OP_NKET + kmaj(f, i0, 64), nke[0], nke[1], nke[2], nke[3]);
         }
       }
-      if (tid < KD) {
-        sEl[tid] = ex2(sC[63 * LDCF + tid]);
-        sEh[tid] = ex2(sC[63 * LDCF + tid] - sC[31 * LDCF + tid]);
-      }
+      if (tid < KD) sEl[tid] = ex2(sC[63 * LDCF + tid]);
       // dO^T into TMEM: lane n, columns j
       {
         uint32_t r[32];
@@ -178,21 +168,19 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_dstate_tc_kernel(BwdArgs a) {
     }
     if (!wait_mma(bar, phase)) { failed = true; break; }
 
-    // ---------------------------------------------------------------- store dM (leaving this chunk); start dM_in and dM_mid
+    // ---------------------------------------------------------------- store dM (leaving this chunk); start dM_in
     {
+      // index of the gradient of the state leaving this chunk in the 32-step
+      // layout (the last chunk may end inside its first half)
+      const int dm_idx = (2 * ch + 1 < NT32) ? 2 * ch + 1 : 2 * ch;
       uint32_t r[32];
       for (int cb = 0; cb < 2; ++cb) {
         const int f0 = hcol * 64 + cb * 32;
         float s[32];
         tmem_ld32(tm + lo + TM_S + f0, s);
-        if (2 * ch + 1 < NT32) {
-          float* dst = a.dstates + ((head * NT32 + 2 * ch + 1) * KD + f0) * VD + Lr;
+        float* dst = a.dstates + ((head * NT32 + dm_idx) * KD + f0) * VD + Lr;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) dst[(size_t)j * VD] = s[j];
-        }
-#pragma unroll
-        for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(s[j] * sEh[f0 + j]);
-        tmem_st32(tm + lo + TM_MID + f0, r);
+        for (int j = 0; j < 32; ++j) dst[(size_t)j * VD] = s[j];
 #pragma unroll
         for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(s[j] * sEl[f0 + j]);
         tmem_st32(tm + lo + TM_S + f0, r);
@@ -208,23 +196,9 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_dstate_tc_kernel(BwdArgs a) {
         mma_ts(tm + TM_S, tm + TM_DOT + ks * 8, desc(sb + OP_QET + ks * 256, 2048), id, 1);
         mma_ts(tm + TM_S, tm + TM_DR + ks * 8, desc(sb + OP_NKET + ks * 256, 2048), id, 1);
       }
-      for (int ks = 0; ks < 4; ++ks) {
-        mma_ts(tm + TM_MID, tm + TM_DOT + 32 + ks * 8, desc(sb + OP_Q2T + ks * 256, 1024), id, 1);
-        mma_ts(tm + TM_MID, tm + TM_DR + 32 + ks * 8, desc(sb + OP_NK2T + ks * 256, 1024), id, 1);
-      }
       commit(bar);
     }
     if (!wait_mma(bar, phase)) { failed = true; break; }
-    {  // gradient of the state leaving step 31 of this chunk
-      for (int cb = 0; cb < 2; ++cb) {
-        const int f0 = hcol * 64 + cb * 32;
-        float s[32];
-        tmem_ld32(tm + lo + TM_MID + f0, s);
-        float* dst = a.dstates + ((head * NT32 + 2 * ch) * KD + f0) * VD + Lr;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) dst[(size_t)j * VD] = s[j];
-      }
-    }
     fence_before();
     __syncthreads();
   }

@@ -171,6 +171,10 @@ static int launch_fwd_t(const FwdArgs& a, cudaStream_t stream) {
 
 int launch_fwd(const FwdArgs& a, int dtype, cudaStream_t stream) {
   if (fwd_tc_eligible(a, dtype)) return launch_fwd_tc(a, stream);
+  return launch_fwd_ffma(a, dtype, stream);
+}
+
+int launch_fwd_ffma(const FwdArgs& a, int dtype, cudaStream_t stream) {
   const bool bf = dtype == 1;
   switch (a.K) {
     case 32: return bf ? launch_fwd_t<32, __nv_bfloat16>(a, stream) : launch_fwd_t<32, float>(a, stream);

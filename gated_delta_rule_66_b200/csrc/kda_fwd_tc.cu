@@ -19,10 +19,9 @@
 // All products are tcgen05.mma kind::tf32 with fp32 accumulation in TMEM;
 // the CUDA cores write the operands into shared memory in the K-major
 // no-swizzle canonical layout (kda_tc.cuh), rounded to tf32.  With a state
-// workspace the kernel also stores the state entering every 32 steps (the
-// chunk start, and the mid-chunk state
-// M_mid^T = M^T diag(e^{c_31}) + U^T[:, :32] (K o e^{c_31 - c})[:32]) for the
-// backward.
+// workspace the kernel also stores the state entering every chunk (at even
+// indices of the 32-step state layout) and the chunk's interaction record for
+// the backward.
 #include <cuda_bf16.h>
 
 #include "kda_internal.h"
@@ -34,12 +33,123 @@ __device__ unsigned int g_kda_device_error;
 
 namespace tcf {
 using namespace tcc;
-constexpr uint32_t OP_BKET = OP, OP_BVT = OP + 32768, OP_QE = OP + 65536, OP_KEDT = OP + 98304,
-                   OP_KMID = OP + 131072;
+constexpr uint32_t OP_BKET = OP, OP_BVT = OP + 32768, OP_QE = OP + 65536, OP_KEDT = OP + 98304;
 // TMEM columns
-constexpr uint32_t TM_S = 0, TM_X = 128, TM_O = 192, TM_U = 256, TM_W = 320, TM_APA = 384, TM_APB = 448,
-                   TM_MID = 320;  // mid-chunk state (after the W and interaction tiles are read)
+constexpr uint32_t TM_S = 0, TM_X = 128, TM_O = 192, TM_U = 256, TM_W = 320, TM_APA = 384, TM_APB = 448;
 }  // namespace tcf
+
+// The state-independent part of one chunk: load, cumulative decay, the
+// interaction products and their read-out, the inverse T, the operands of the
+// state products (Q~ o e^c, (K o e^{c_last-c})^T in shared memory; e^{c_last}
+// per channel) and
+// W^T = (diag(beta) K o e^c)^T T^T, U0^T = (diag(beta) V)^T T^T in TMEM.  With
+// `irec` it stores the chunk's interaction record; with `img` it starts the
+// bulk stores of the chunk images of Q~ o e^c, (K o e^{c_last-c})^T and
+// e^{c_last} as soon as they are built.
+// Returns false, block-uniformly, if a tensor-core wait ran out.
+__device__ __forceinline__ bool fwd_chunk_head(const tcc::Ctx& cx, const FwdArgs& a, int b, int hv, int h,
+                                               int ch, bool prefetch_next, float* irec,
+                                               unsigned char* img, uint64_t* bar, uint32_t& phase) {
+  using namespace tcf;
+  using namespace tc;
+  unsigned char* sm = cx.sm;
+  const uint32_t sb = cx.sb, tm = cx.tm;
+  const int tid = cx.tid;
+  const int T = a.T, NT = (T + C - 1) / C, t0 = ch * C, L = min(C, T - t0);
+  const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(a.q);
+  const __nv_bfloat16* kg = static_cast<const __nv_bfloat16*>(a.k);
+  const __nv_bfloat16* vg = static_cast<const __nv_bfloat16*>(a.v);
+  const float* sBeta = cx.beta();
+  float* sEl = reinterpret_cast<float*>(sm + S_EL);
+  const float* sC = cx.c();
+  load_raw_issue(cx, qg, kg, vg, a.g, a.beta, b, T, t0, L, a.H, a.HV, h, hv);
+  if (prefetch_next && ch + 1 < NT)
+    prefetch_chunk(cx, qg, kg, vg, a.g, b, T, t0 + C, min(C, T - t0 - C), a.H, a.HV, h, hv);
+  load_raw_wait();
+  const bool wide = cumsum_span(cx);
+  build_op1_and_issue(cx, a.scale, tm + TM_APA, tm + TM_APB, bar);
+  if (!wait_mma(bar, phase)) return false;
+
+  // ---------------------------------------------------------------- state-product operands
+  {  // Q~ o e^c as [i][f]: thread items of 4 channels, 16-byte stores
+    const int fq = item_f(cx);
+    for (int m = 0; m < 8; ++m) {
+      const int i = item_row(cx, m);
+      const float4 c4 = ld4(sC + i * LDCF + fq);
+      float qf[4];
+      bf16x4(sm + RAW_Q + i * 256 + fq * 2, qf);
+      st_tf32x4(sm, OP_QE + kmaj(i, fq, 128), a.scale * qf[0] * ex2(c4.x), a.scale * qf[1] * ex2(c4.y),
+                a.scale * qf[2] * ex2(c4.z), a.scale * qf[3] * ex2(c4.w));
+    }
+  }
+  {  // transposed operands [f][i]: thread items of one channel x 4 rows, 16-byte stores
+    const int f = tid & 127;
+    const float c63 = sC[63 * LDCF + f];
+    const __nv_bfloat16* kcol = reinterpret_cast<const __nv_bfloat16*>(sm + RAW_K) + f;
+    const __nv_bfloat16* vcol = reinterpret_cast<const __nv_bfloat16*>(sm + RAW_X) + f;
+    for (int m = 0; m < 8; ++m) {
+      const int i0 = ((tid >> 7) + 2 * m) * 4;
+      float bke[4], ked[4], bv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u;
+        const float c = sC[i * LDCF + f], kk = __bfloat162float(kcol[i * 128]), bi = sBeta[i];
+        bke[u] = bi * kk * ex2(c);
+        ked[u] = kk * ex2(c63 - c);
+        bv[u] = bi * __bfloat162float(vcol[i * 128]);
+      }
+      st_tf32x4(sm, OP_BKET + kmaj(f, i0, 64), bke[0], bke[1], bke[2], bke[3]);
+      st_tf32x4(sm, OP_KEDT + kmaj(f, i0, 64), ked[0], ked[1], ked[2], ked[3]);
+      st_tf32x4(sm, OP_BVT + kmaj(f, i0, 64), bv[0], bv[1], bv[2], bv[3]);
+    }
+    if (tid < KD) sEl[tid] = ex2(c63);
+  }
+  Pairwise pw;
+  if (wide) pairwise_compute(cx, a.scale, pw);
+  if (img) fence_async_smem();
+  __syncthreads();  // raw inputs consumed; the raw region is reused below
+  if (img && tid == 0) {
+    bulk_s2g(img + FWI_QE, sb + OP_QE, FWI_KEDT - FWI_QE);
+    bulk_s2g(img + FWI_KEDT, sb + OP_KEDT, FWI_P - FWI_KEDT);
+    bulk_s2g(img + FWI_EL, sb + S_EL, FWI_U0 - FWI_EL);
+    bulk_commit();
+  }
+
+  readout_ap(cx, tm + TM_APA, tm + TM_APB, false, wide, pw, irec);
+  invert(cx);
+  {  // T as the operand image (rows i, K = j); with a record also its T, T^T images and Ah
+    const float* tr = reinterpret_cast<const float*>(sm + R_TROW);
+    for (int x = tid; x < C * 16; x += NTH) {  // 16-byte piece x of the image: x * 16 = kmaj(i, j4, 64)
+      const int i = ((x >> 7) << 3) | (x & 7), j4 = ((x >> 3) & 15) * 4;
+      const float* p = tr + i * 65 + j4;
+      const uint4 t = make_uint4(tf32_rna(p[0]), tf32_rna(p[1]), tf32_rna(p[2]), tf32_rna(p[3]));
+      *reinterpret_cast<uint4*>(sm + R_T + x * 16) = t;
+      if (irec) {
+        const float* pc = tr + j4 * 65 + i;
+        *reinterpret_cast<uint4*>(irec + INTER_T + x * 4) = t;
+        *reinterpret_cast<uint4*>(irec + INTER_TT + x * 4) =
+            make_uint4(tf32_rna(pc[0]), tf32_rna(pc[65]), tf32_rna(pc[130]), tf32_rna(pc[195]));
+      }
+    }
+    if (irec) {
+      const float* ah = reinterpret_cast<const float*>(sm + R_AH);
+      for (int x = tid; x < C * C; x += NTH) irec[INTER_AH + x] = ah[(x >> 6) * 65 + (x & 63)];
+    }
+  }
+  fence_async_smem();
+  __syncthreads();
+  if (tid == 0) {
+    fence_after();
+    const uint32_t id = idesc_tf32(128, 64);
+    for (int ks = 0; ks < 8; ++ks) {
+      const uint64_t bT = desc(sb + R_T + ks * 256, 2048);
+      mma_ss(tm + TM_W, desc(sb + OP_BKET + ks * 256, 2048), bT, id, ks > 0);
+      mma_ss(tm + TM_U, desc(sb + OP_BVT + ks * 256, 2048), bT, id, ks > 0);
+    }
+    commit(bar);
+  }
+  return wait_mma(bar, phase);
+}
 
 __global__ void __launch_bounds__(256, 1) kda_fwd_tc_kernel(FwdArgs a) {
   using namespace tcf;
@@ -68,7 +178,6 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_tc_kernel(FwdArgs a) {
   __nv_bfloat16* og = static_cast<__nv_bfloat16*>(a.o);
   float* sBeta = cx.beta();
   float* sEl = reinterpret_cast<float*>(sm + S_EL);
-  float* sE31 = reinterpret_cast<float*>(sm + S_EMID);
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + S_BAR);
   uint32_t* sTm = reinterpret_cast<uint32_t*>(sm + S_TMEM);
   const float* sC = cx.c();
@@ -99,91 +208,11 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_tc_kernel(FwdArgs a) {
 
   for (int ch = 0; ch < NT; ++ch) {
     const int t0 = ch * C, L = min(C, T - t0);
-    load_raw_issue(cx, qg, kg, vg, a.g, a.beta, b, T, t0, L, a.H, a.HV, h, hv);
-    if (ch + 1 < NT) prefetch_chunk(cx, qg, kg, vg, a.g, b, T, t0 + C, min(C, T - t0 - C), a.H, a.HV, h, hv);
-    load_raw_wait();
-    const bool wide = cumsum_span(cx);
-    build_op1_and_issue(cx, a.scale, tm + TM_APA, tm + TM_APB, bar);
-    if (!wait_mma(bar, phase)) { failed = true; break; }
-
-    // ---------------------------------------------------------------- state-product operands
-    {  // Q~ o e^c as [i][f]: thread items of 4 channels, 16-byte stores
-      const int fq = item_f(cx);
-      for (int m = 0; m < 8; ++m) {
-        const int i = item_row(cx, m);
-        const float4 c4 = ld4(sC + i * LDCF + fq);
-        float qf[4];
-        bf16x4(sm + RAW_Q + i * 256 + fq * 2, qf);
-        st_tf32x4(sm, OP_QE + kmaj(i, fq, 128), a.scale * qf[0] * ex2(c4.x), a.scale * qf[1] * ex2(c4.y),
-                  a.scale * qf[2] * ex2(c4.z), a.scale * qf[3] * ex2(c4.w));
-      }
-    }
-    {  // transposed operands [f][i]: thread items of one channel x 4 rows, 16-byte stores
-      const int f = tid & 127;
-      const float c63 = sC[63 * LDCF + f], c31 = sC[31 * LDCF + f];
-      const __nv_bfloat16* kcol = reinterpret_cast<const __nv_bfloat16*>(sm + RAW_K) + f;
-      const __nv_bfloat16* vcol = reinterpret_cast<const __nv_bfloat16*>(sm + RAW_X) + f;
-      for (int m = 0; m < 8; ++m) {
-        const int i0 = ((tid >> 7) + 2 * m) * 4;
-        float bke[4], ked[4], bv[4], kmid[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int i = i0 + u;
-          const float c = sC[i * LDCF + f], kk = __bfloat162float(kcol[i * 128]), bi = sBeta[i];
-          bke[u] = bi * kk * ex2(c);
-          ked[u] = kk * ex2(c63 - c);
-          bv[u] = bi * __bfloat162float(vcol[i * 128]);
-          if (a.states && i0 < 32) kmid[u] = kk * ex2(c31 - c);
-        }
-        st_tf32x4(sm, OP_BKET + kmaj(f, i0, 64), bke[0], bke[1], bke[2], bke[3]);
-        st_tf32x4(sm, OP_KEDT + kmaj(f, i0, 64), ked[0], ked[1], ked[2], ked[3]);
-        st_tf32x4(sm, OP_BVT + kmaj(f, i0, 64), bv[0], bv[1], bv[2], bv[3]);
-        if (a.states && i0 < 32) st_tf32x4(sm, OP_KMID + kmaj(f, i0, 32), kmid[0], kmid[1], kmid[2], kmid[3]);
-      }
-      if (tid < KD) {
-        sEl[tid] = ex2(c63);
-        sE31[tid] = ex2(c31);
-      }
-    }
-    Pairwise pw;
-    if (wide) pairwise_compute(cx, a.scale, pw);
-    __syncthreads();  // raw inputs consumed; the raw region is reused below
-
     float* irec = a.inter ? a.inter + (head * NT + ch) * INTER_REC : nullptr;
-    readout_ap(cx, tm + TM_APA, tm + TM_APB, false, wide, pw, irec);
-    invert(cx);
-    {  // T as the operand image (rows i, K = j); with a record also its T, T^T images and Ah
-      const float* tr = reinterpret_cast<const float*>(sm + R_TROW);
-      for (int x = tid; x < C * 16; x += NTH) {  // 16-byte piece x of the image: x * 16 = kmaj(i, j4, 64)
-        const int i = ((x >> 7) << 3) | (x & 7), j4 = ((x >> 3) & 15) * 4;
-        const float* p = tr + i * 65 + j4;
-        const uint4 t = make_uint4(tf32_rna(p[0]), tf32_rna(p[1]), tf32_rna(p[2]), tf32_rna(p[3]));
-        *reinterpret_cast<uint4*>(sm + R_T + x * 16) = t;
-        if (irec) {
-          const float* pc = tr + j4 * 65 + i;
-          *reinterpret_cast<uint4*>(irec + INTER_T + x * 4) = t;
-          *reinterpret_cast<uint4*>(irec + INTER_TT + x * 4) =
-              make_uint4(tf32_rna(pc[0]), tf32_rna(pc[65]), tf32_rna(pc[130]), tf32_rna(pc[195]));
-        }
-      }
-      if (irec) {
-        const float* ah = reinterpret_cast<const float*>(sm + R_AH);
-        for (int x = tid; x < C * C; x += NTH) irec[INTER_AH + x] = ah[(x >> 6) * 65 + (x & 63)];
-      }
+    if (!fwd_chunk_head(cx, a, b, hv, h, ch, true, irec, nullptr, bar, phase)) {
+      failed = true;
+      break;
     }
-    fence_async_smem();
-    __syncthreads();
-    if (tid == 0) {
-      fence_after();
-      const uint32_t id = idesc_tf32(128, 64);
-      for (int ks = 0; ks < 8; ++ks) {
-        const uint64_t bT = desc(sb + R_T + ks * 256, 2048);
-        mma_ss(tm + TM_W, desc(sb + OP_BKET + ks * 256, 2048), bT, id, ks > 0);
-        mma_ss(tm + TM_U, desc(sb + OP_BVT + ks * 256, 2048), bT, id, ks > 0);
-      }
-      commit(bar);
-    }
-    if (!wait_mma(bar, phase)) { failed = true; break; }
 
     // ---------------------------------------------------------------- W into shared memory
     {
@@ -218,13 +247,10 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_tc_kernel(FwdArgs a) {
         const int f0 = hcol * 64 + cb * 32;
         float s[32];
         tmem_ld32(tm + lo + TM_S + f0, s);
-        if (a.states) {  // the state entering this chunk, and e^{c_31} M^T to start the mid state
+        if (a.states) {  // the state entering this chunk
           float* dst = a.states + ((head * NT32 + 2 * ch) * KD + f0) * VD + Lr;
 #pragma unroll
           for (int j = 0; j < 32; ++j) dst[(size_t)j * VD] = s[j];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(s[j] * sE31[f0 + j]);
-          tmem_st32(tm + lo + TM_MID + f0, r);
         }
 #pragma unroll
         for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(s[j] * sEl[f0 + j]);
@@ -241,24 +267,11 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_tc_kernel(FwdArgs a) {
         mma_ts(tm + TM_S, tm + TM_U + ks * 8, desc(sb + OP_KEDT + ks * 256, 2048), idS, 1);
         mma_ts(tm + TM_O, tm + TM_U + ks * 8, desc(sb + R_P + ks * 256, 2048), idO, 1);
       }
-      if (a.states)
-        for (int ks = 0; ks < 4; ++ks)
-          mma_ts(tm + TM_MID, tm + TM_U + ks * 8, desc(sb + OP_KMID + ks * 256, 1024), idS, 1);
       commit(bar);
     }
     if (!wait_mma(bar, phase)) { failed = true; break; }
 
-    // ---------------------------------------------------------------- O out (and the mid-chunk state)
-    if (a.states && 2 * ch + 1 < NT32) {
-      for (int cb = 0; cb < 2; ++cb) {
-        const int f0 = hcol * 64 + cb * 32;
-        float s[32];
-        tmem_ld32(tm + lo + TM_MID + f0, s);
-        float* dst = a.states + ((head * NT32 + 2 * ch + 1) * KD + f0) * VD + Lr;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) dst[(size_t)j * VD] = s[j];
-      }
-    }
+    // ---------------------------------------------------------------- O out
     if (a.o) {
       float v[32];
       tmem_ld32(tm + lo + TM_O + hcol * 32, v);
@@ -290,10 +303,290 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_tc_kernel(FwdArgs a) {
 
 bool fwd_tc_eligible(const FwdArgs& a, int dtype) {
   auto al16 = [](const void* p) { return ((uintptr_t)p & 15u) == 0; };
-  return dtype == 1 && a.K == 128 && a.V == 128 && al16(a.q) && al16(a.k) && al16(a.v) && al16(a.g);
+  return dtype == 1 && a.K == 128 && a.V == 128 && al16(a.q) && al16(a.k) && al16(a.v) && al16(a.g) &&
+         al16(a.o);
+}
+
+// ============================================================================
+// Two-kernel forward (with a chunk-image workspace).  The state-independent
+// work of every chunk runs first, all chunks in parallel
+// (kda_fwd_prep_tc_kernel, one CTA per (b, hv, chunk)), and leaves the chunk's
+// operands of the state products in the workspace as ready shared-memory
+// images; kda_fwd_seq_tc_kernel then carries the state through the chunks of
+// one (b, hv) with only the state products per chunk:
+//   X^T = M^T W^T,  O^T = M^T (Q~ o e^c)^T,  U^T = U0^T - X^T,
+//   M'^T = M^T diag(e^{c_last}) + U^T (K o e^{c_last-c}),  O^T += U^T P^T.
+// ============================================================================
+__global__ void __launch_bounds__(256, 1) kda_fwd_prep_tc_kernel(FwdArgs a) {
+  using namespace tcf;
+  using namespace tc;
+  extern __shared__ __align__(1024) unsigned char sm[];
+  Ctx cx;
+  cx.sm = sm;
+  cx.sb = smem_u32(sm);
+  cx.tid = threadIdx.x;
+  cx.warp = cx.tid >> 5;
+  cx.lane = cx.tid & 31;
+  cx.sub = cx.warp & 3;
+  cx.hcol = cx.warp >> 2;
+  cx.Lr = cx.sub * 32 + cx.lane;
+  cx.lo = (uint32_t)(cx.sub * 32) << 16;
+  const int tid = cx.tid, hcol = cx.hcol, Lr = cx.Lr;
+  const uint32_t lo = cx.lo, sb = cx.sb;
+  const int G = a.HV / a.H, NT = (a.T + C - 1) / C;
+  const int items = NT * a.HV * a.B;  // item = (b * HV + hv) * NT + ch
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + S_BAR);
+  uint32_t* sTm = reinterpret_cast<uint32_t*>(sm + S_TMEM);
+
+  if (cx.warp == 0) tmem_alloc(sTm, 512);
+  if (tid == 0) mbar_init(bar, 1);
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tm = *sTm;
+  cx.tm = tm;
+  uint32_t phase = 0;
+  bool failed = false;
+  // persistent: this CTA takes items blockIdx.x, + gridDim.x, ...; each item's
+  // raw rows are brought into L2 while the previous item is processed
+  for (int item = blockIdx.x; item < items; item += gridDim.x) {
+    const int ch = item % NT, hv = (item / NT) % a.HV, b = item / (NT * a.HV), h = hv / G;
+    const size_t head = (size_t)b * a.HV + hv;
+    const int nxt = item + gridDim.x;
+    if (nxt < items) {
+      const int nch = nxt % NT, nhv = (nxt / NT) % a.HV, nb = nxt / (NT * a.HV);
+      prefetch_chunk(cx, static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),
+                     static_cast<const __nv_bfloat16*>(a.v), a.g, nb, a.T, nch * C, min(C, a.T - nch * C), a.H,
+                     a.HV, nhv / G, nhv);
+    }
+    if (tid == 0) bulk_wait_read();  // the previous item's image stores have left shared memory
+    __syncthreads();
+    float* irec = a.inter ? a.inter + (head * NT + ch) * INTER_REC : nullptr;
+    unsigned char* img = a.img + (head * NT + ch) * (size_t)FWI_BYTES;
+    if (!fwd_chunk_head(cx, a, b, hv, h, ch, false, irec, img, bar, phase)) {
+      failed = true;
+      break;
+    }
+    {  // W (rows i, K = f) padded, from W^T in TMEM (lane f)
+      float v[32];
+      tmem_ld32(tm + lo + TM_W + hcol * 32, v);
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) st_tf32(sm, R_WOP + kmaj_pad(hcol * 32 + jj, Lr, 128), v[jj]);
+    }
+    {  // U0^T (lane n) as [i][n]
+      float u[32];
+      tmem_ld32(tm + lo + TM_U + hcol * 32, u);
+      float* dst = reinterpret_cast<float*>(img + FWI_U0);
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) dst[(hcol * 32 + jj) * VD + Lr] = u[jj];
+    }
+    fence_async_smem();
+    fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      bulk_s2g(img + FWI_W, sb + R_WOP, FWI_QE - FWI_W);
+      bulk_s2g(img + FWI_P, sb + R_P, FWI_EL - FWI_P);
+      bulk_commit();
+    }
+  }
+  if (tid == 0) bulk_wait_read();
+  fence_before();
+  __syncthreads();
+  if (cx.warp == 0) tmem_dealloc(tm, 512);
+  if (failed && tid == 0) atomicOr(&g_kda_device_error, 1u);
+}
+
+namespace tcs {
+// shared memory of the sequential pass: two buffers for the first group of a
+// chunk's images (W, Q~ o e^c), one for the second ((K o e^{c_last-c})^T, P,
+// e^{c_last}), the bf16 output tile [i][n], then the barriers
+constexpr uint32_t SQ_A0 = 0, SQ_A1 = FWI_A_BYTES, SQ_B = 2 * FWI_A_BYTES, SQ_O = SQ_B + FWI_B_BYTES,
+                   SQ_BAR = SQ_O + 64 * 256, SQ_TMEM = SQ_BAR + 32, SQ_BYTES = SQ_TMEM + 16;
+constexpr uint32_t B_KEDT = 0, B_P = FWI_P - FWI_KEDT, B_EL = FWI_EL - FWI_KEDT;
+static_assert(SQ_BYTES <= 232448 && SQ_O % 16 == 0, "shared memory budget");
+constexpr uint32_t TM_S = 0, TM_X = 128, TM_O = 192, TM_U = 256;
+}  // namespace tcs
+
+// one thread: arm `bar` for `bytes` and fetch them from global to shared memory
+__device__ __forceinline__ void fetch_images(uint32_t sdst, const unsigned char* src, uint32_t bytes, uint64_t* bar) {
+  tc::mbar_expect_tx(bar, bytes);
+  for (uint32_t off = 0; off < bytes; off += 32768)
+    tc::bulk_g2s(sdst + off, src + off, min(32768u, bytes - off), bar);
+}
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity) {
+  const bool ok = tc::mbar_wait(bar, parity);
+  return !__syncthreads_or(!ok);
+}
+
+__global__ void __launch_bounds__(256, 1) kda_fwd_seq_tc_kernel(FwdArgs a) {
+  using namespace tcs;
+  using namespace tc;
+  extern __shared__ __align__(1024) unsigned char sm[];
+  const uint32_t sb = smem_u32(sm);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, hcol = warp >> 2;
+  const int Lr = (warp & 3) * 32 + lane;
+  const uint32_t lo = (uint32_t)((warp & 3) * 32) << 16;
+  const int hv = blockIdx.x, b = blockIdx.y;
+  const int T = a.T, NT = (T + tcc::C - 1) / tcc::C, NT32 = (T + 31) / 32;
+  constexpr int C = tcc::C, KD = tcc::KD, VD = tcc::VD;
+  const size_t head = (size_t)b * a.HV + hv;
+  const unsigned char* imgs = a.img + head * NT * (size_t)FWI_BYTES;
+  __nv_bfloat16* og = static_cast<__nv_bfloat16*>(a.o);
+  uint64_t* barA = reinterpret_cast<uint64_t*>(sm + SQ_BAR);  // [2]
+  uint64_t* barB = barA + 2;
+  uint64_t* bar = barA + 3;  // tensor-core completion
+  uint32_t* sTm = reinterpret_cast<uint32_t*>(sm + SQ_TMEM);
+  const float* sEl = reinterpret_cast<const float*>(sm + SQ_B + B_EL);
+
+  if (warp == 0) tmem_alloc(sTm, 512);
+  if (tid == 0) {
+    mbar_init(barA, 1);
+    mbar_init(barA + 1, 1);
+    mbar_init(barB, 1);
+    mbar_init(bar, 1);
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tm = *sTm;
+  if (tid == 0) {
+    fetch_images(sb + SQ_A0, imgs, FWI_A_BYTES, barA);
+    fetch_images(sb + SQ_B, imgs + FWI_KEDT, FWI_B_BYTES, barB);
+  }
+  {  // entering state, transposed: lane n, column f
+    for (int cb = 0; cb < 2; ++cb) {
+      const int f0 = hcol * 64 + cb * 32;
+      uint32_t r[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(a.S0 ? a.S0[(head * KD + f0 + j) * VD + Lr] : 0.f);
+      tmem_st32(tm + lo + TM_S + f0, r);
+    }
+    tmem_wait_st();
+  }
+  fence_before();
+  __syncthreads();
+  uint32_t phase = 0;
+  bool failed = false;
+
+  for (int ch = 0; ch < NT; ++ch) {
+    const int t0 = ch * C, L = min(C, T - t0);
+    const unsigned char* img = imgs + (size_t)ch * FWI_BYTES;
+    const uint32_t bufA = (ch & 1) ? SQ_A1 : SQ_A0;
+    if (tid == 32 && ch + 1 < NT) prefetch_l2(img + FWI_BYTES, FWI_BYTES);
+    float u0[32];
+    {
+      const float* src = reinterpret_cast<const float*>(img + FWI_U0);
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) u0[jj] = src[(hcol * 32 + jj) * VD + Lr];
+    }
+    if (!wait_bar(barA + (ch & 1), (ch >> 1) & 1)) { failed = true; break; }
+    if (tid == 0) {  // X^T = M^T W^T ; O^T = M^T (Q~ o e^c)^T ; then the next chunk's first images
+      fence_after();
+      const uint32_t id = idesc_tf32(128, 64);
+      for (int ks = 0; ks < 16; ++ks) {
+        mma_ts(tm + TM_X, tm + TM_S + ks * 8, desc(sb + bufA + FWI_W + ks * 288, 4608, 144), id, ks > 0);
+        mma_ts(tm + TM_O, tm + TM_S + ks * 8, desc(sb + bufA + FWI_QE + ks * 256, 4096), id, ks > 0);
+      }
+      commit(bar);
+      if (ch + 1 < NT) fetch_images(sb + ((ch & 1) ? SQ_A0 : SQ_A1), img + FWI_BYTES, FWI_A_BYTES, barA + ((ch + 1) & 1));
+    }
+    if (!tcc::wait_mma(bar, phase)) { failed = true; break; }
+    {  // U^T = U0^T - X^T
+      float x[32];
+      uint32_t r[32];
+      tmem_ld32(tm + lo + TM_X + hcol * 32, x);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) r[j] = tf32_rna(u0[j] - x[j]);
+      tmem_st32(tm + lo + TM_U + hcol * 32, r);
+    }
+    if (!wait_bar(barB, ch & 1)) { failed = true; break; }
+    {  // M^T <- M^T diag(e^{c_last}); the entering state for the backward
+      uint32_t r[32];
+      for (int cb = 0; cb < 2; ++cb) {
+        const int f0 = hcol * 64 + cb * 32;
+        float s[32];
+        tmem_ld32(tm + lo + TM_S + f0, s);
+        if (a.states) {
+          float* dst = a.states + ((head * NT32 + 2 * ch) * KD + f0) * VD + Lr;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) dst[(size_t)j * VD] = s[j];
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(s[j] * sEl[f0 + j]);
+        tmem_st32(tm + lo + TM_S + f0, r);
+      }
+      tmem_wait_st();
+    }
+    fence_before();
+    __syncthreads();
+    if (tid == 0) {  // M^T += U^T (K o e^{c_last-c}) ; O^T += U^T P^T
+      fence_after();
+      const uint32_t idS = idesc_tf32(128, 128), idO = idesc_tf32(128, 64);
+      for (int ks = 0; ks < 8; ++ks) {
+        mma_ts(tm + TM_S, tm + TM_U + ks * 8, desc(sb + SQ_B + B_KEDT + ks * 256, 2048), idS, 1);
+        mma_ts(tm + TM_O, tm + TM_U + ks * 8, desc(sb + SQ_B + B_P + ks * 256, 2048), idO, 1);
+      }
+      commit(bar);
+    }
+    if (!tcc::wait_mma(bar, phase)) { failed = true; break; }
+    if (tid == 0 && ch + 1 < NT) {  // the lanes' reads of e^{c_last} precede the overwrite
+      fence_async_smem();
+      fetch_images(sb + SQ_B, img + FWI_BYTES + FWI_KEDT, FWI_B_BYTES, barB);
+    }
+    if (a.o) {  // O^T (lane n) -> bf16 tile [i][n] -> 16-byte row pieces
+      __nv_bfloat16* so = reinterpret_cast<__nv_bfloat16*>(sm + SQ_O);
+      float v[32];
+      tmem_ld32(tm + lo + TM_O + hcol * 32, v);
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) so[(hcol * 32 + jj) * VD + Lr] = __float2bfloat16_rn(v[jj]);
+      __syncthreads();
+#pragma unroll
+      for (int x = tid; x < C * 16; x += 256) {
+        const int i = x >> 4, c16 = x & 15;
+        if (i < L)
+          *reinterpret_cast<uint4*>(og + (((size_t)b * T + t0 + i) * a.HV + hv) * VD + c16 * 8) =
+              *reinterpret_cast<const uint4*>(sm + SQ_O + i * 256 + c16 * 16);
+      }
+    }
+    fence_before();
+    __syncthreads();
+  }
+
+  if (!failed && a.S_T) {
+    fence_after();
+    for (int cb = 0; cb < 2; ++cb) {
+      const int f0 = hcol * 64 + cb * 32;
+      float s[32];
+      tmem_ld32(tm + lo + TM_S + f0, s);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) a.S_T[(head * KD + f0 + j) * VD + Lr] = s[j];
+    }
+  }
+  fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tm, 512);
+  if (failed && tid == 0) atomicOr(&g_kda_device_error, 1u);
 }
 
 int launch_fwd_tc(const FwdArgs& a, cudaStream_t stream) {
+  if (a.img) {  // two-kernel forward
+    cudaError_t e = cudaFuncSetAttribute(kda_fwd_prep_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)tcc::SMEM_BYTES);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(kda_fwd_seq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)tcs::SQ_BYTES);
+    if (e != cudaSuccess) return set_cuda_error("kda_fwd: cudaFuncSetAttribute", e);
+    const int items = (a.T + tcc::C - 1) / tcc::C * a.HV * a.B;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    kda_fwd_prep_tc_kernel<<<min(items, sms), tcc::NTH, tcc::SMEM_BYTES, stream>>>(a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return set_cuda_error("kda_fwd: tensor-core chunk launch", e);
+    kda_fwd_seq_tc_kernel<<<dim3(a.HV, a.B), tcc::NTH, tcs::SQ_BYTES, stream>>>(a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return set_cuda_error("kda_fwd: tensor-core state-pass launch", e);
+    return 0;
+  }
   cudaError_t e = cudaFuncSetAttribute(kda_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)tcc::SMEM_BYTES);
   if (e != cudaSuccess) return set_cuda_error("kda_fwd: cudaFuncSetAttribute", e);

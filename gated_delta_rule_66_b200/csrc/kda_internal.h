@@ -25,6 +25,19 @@ constexpr int FWD_VBLOCK = 32;   // V columns per CTA in the chunked kernels
 // and Ah row-major at INTER_AH.  The backward reads it instead of recomputing
 // the interaction products and the inverse.
 constexpr int INTER_T = 4096, INTER_AH = 8192, INTER_TT = 12288, INTER_REC = 16384;
+// Per-(b, hv, 64-step chunk) operand images of the two-kernel tensor-core
+// forward (bytes): everything the sequential state pass needs from a chunk,
+// laid out as its shared-memory operands so that it fetches them with two
+// bulk copies (W and Q~ o e^c; the rest) plus U0^T read by the lanes.
+//   FWI_W     W (rows i, K = f), padded K-major (LBO 144)     36864
+//   FWI_QE    Q~ o e^c (rows i, K = f)                        32768
+//   FWI_KEDT  (K o e^{c_last - c})^T (rows f, K = i)          32768
+//   FWI_P     P (rows i, K = j)                               16384
+//   FWI_EL    e^{c_last} [128]                                  512
+//   FWI_U0    U0^T = (T diag(beta) V)^T as [i][n] fp32        32768
+constexpr unsigned FWI_W = 0, FWI_QE = 36864, FWI_KEDT = 69632, FWI_P = 102400, FWI_EL = 118784,
+                   FWI_U0 = 119296, FWI_BYTES = 152064;
+constexpr unsigned FWI_A_BYTES = FWI_KEDT, FWI_B_BYTES = FWI_U0 - FWI_KEDT;
 constexpr int G_AH = 0, G_PA = 4096, G_QK = 12288, G_KED = 28672, G_DBR = 36864, G_DEL = 36928,
               GREC = 37120;
 
@@ -35,6 +48,7 @@ struct FwdArgs {
   float* S_T;       // may be null
   float* states;    // may be null; [B, HV, NT, K, V] state entering each chunk
   float* inter;     // may be null; per-chunk interaction records (K = V = 128)
+  unsigned char* img;  // may be null; per-chunk operand images of the two-kernel forward (K = V = 128)
   float scale;
   int B, T, H, HV, K, V;
 };
@@ -67,6 +81,8 @@ int set_error(int code, const char* msg);
 int set_cuda_error(const char* where, cudaError_t e);
 
 int launch_fwd(const FwdArgs& a, int dtype, cudaStream_t stream);
+// the CUDA-core forward whatever the shape (stores all 32-step states)
+int launch_fwd_ffma(const FwdArgs& a, int dtype, cudaStream_t stream);
 bool fwd_tc_eligible(const FwdArgs& a, int dtype);
 int launch_fwd_tc(const FwdArgs& a, cudaStream_t stream);
 int take_device_error(unsigned* out);

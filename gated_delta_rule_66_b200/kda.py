@@ -22,7 +22,7 @@ KDA_DTYPE_BF16 = 1
 KDA_BWD_STATES_FROM_FWD = 1
 CHUNK = 32  # chunk length of the library's chunked kernels (workspace layout)
 
-SYMBOLS = ("kda_last_error", "kda_device_status", "kda_fwd_workspace_bytes",
+SYMBOLS = ("kda_last_error", "kda_device_status", "kda_fwd_workspace_bytes", "kda_fwd_scratch_bytes",
            "kda_bwd_workspace_bytes", "kda_fwd", "kda_decode_step", "kda_bwd")
 
 
@@ -47,6 +47,8 @@ def _load():
     lib.kda_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint)]
     lib.kda_fwd_workspace_bytes.restype = sz
     lib.kda_fwd_workspace_bytes.argtypes = [i, i, i, i, i]
+    lib.kda_fwd_scratch_bytes.restype = sz
+    lib.kda_fwd_scratch_bytes.argtypes = [i, i, i, i, i]
     lib.kda_bwd_workspace_bytes.restype = sz
     lib.kda_bwd_workspace_bytes.argtypes = [i, i, i, i, i, i]
     lib.kda_fwd.restype = i
@@ -110,20 +112,26 @@ def device_status():
 
 
 def workspace_bytes(kind, B, T, H, HV, K, V):
-    """Workspace bytes of ``kind`` = "fwd" (chunk states) or "bwd"."""
+    """Workspace bytes of ``kind`` = "fwd" (training forward: chunk states and
+    records), "scratch" (forward scratch, no states) or "bwd"."""
     if kind == "fwd":
         return int(_lib.kda_fwd_workspace_bytes(B, T, HV, K, V))
+    if kind == "scratch":
+        return int(_lib.kda_fwd_scratch_bytes(B, T, HV, K, V))
     return int(_lib.kda_bwd_workspace_bytes(B, T, H, HV, K, V))
 
 
 def fwd(q, k, v, g, beta, scale=None, initial_state=None, output_final_state=True,
-        workspace=None, out=None):
+        workspace=None, out=None, scratch=True):
     """Prefill forward.  Returns (o [B,T,HV,V] in v's dtype, S_T or None).
 
     q, k [B,T,H,K]; v [B,T,HV,V] (same dtype); g [B,T,HV,K], beta [B,T,HV] and
     initial_state [B,HV,K,V] float32.  ``workspace`` (a uint8 CUDA tensor of
     at least workspace_bytes("fwd", ...)) receives the chunk states for a
-    later ``bwd(..., workspace=..., states_from_fwd=True)``.
+    later ``bwd(..., workspace=..., states_from_fwd=True)``.  Without one,
+    ``scratch`` lets the library use a fresh scratch allocation of
+    workspace_bytes("scratch", ...) (bf16 shapes that have a two-kernel
+    forward); ``scratch=False`` passes no workspace at all.
     """
     B, T, H, K = q.shape
     HV, V = v.shape[2], v.shape[3]
@@ -138,6 +146,10 @@ def fwd(q, k, v, g, beta, scale=None, initial_state=None, output_final_state=Tru
     o = torch.empty(B, T, HV, V, dtype=dt, device=q.device) if out is None else out
     _req("out", o, dt, 4)
     S_T = torch.empty(B, HV, K, V, dtype=torch.float32, device=q.device) if output_final_state else None
+    if workspace is None and scratch and dt == torch.bfloat16:
+        need = int(_lib.kda_fwd_scratch_bytes(B, T, HV, K, V))
+        if need:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     rc = _lib.kda_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state), scale,
                       B, T, H, HV, K, V, _dtype_code(q), _ptr(o), _ptr(S_T), _ptr(workspace),

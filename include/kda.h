@@ -60,9 +60,10 @@ enum { KDA_DTYPE_FP32 = 0, KDA_DTYPE_BF16 = 1 };
 
 /* Flags of kda_bwd. */
 enum {
-  /* The first kda_fwd_workspace_bytes() bytes of the workspace already hold
-   * the chunk states written by kda_fwd on the same inputs (same q, k, v, g,
-   * beta, S0, scale and sizes); kda_bwd then skips its own state pass. */
+  /* The workspace was given to a kda_fwd on the same inputs (same q, k, v,
+   * g, beta, S0, scale and sizes) with at least kda_fwd_workspace_bytes()
+   * bytes, and still holds the chunk states and interaction records that it
+   * stored at its start; kda_bwd then skips its own forward pass. */
   KDA_BWD_STATES_FROM_FWD = 1,
 };
 
@@ -77,13 +78,25 @@ const char* kda_last_error(void);
  * KDA_OK or KDA_ERR_CUDA; *flags receives the bits (0 = none). */
 int kda_device_status(unsigned* flags);
 
-/* Bytes of the optional kda_fwd workspace: the fp32 state entering every
- * chunk, laid out [B, HV, ceil(T / chunk), K, V]; 0 if a size is invalid. */
+/* Bytes of the training workspace of kda_fwd: the fp32 state entering every
+ * 32 steps [B, HV, ceil(T / 32), K, V], then (K = V = 128) the per-64-step
+ * interaction records (P^T, T, T^T operand images and Ah, 64 KB per chunk)
+ * and the scratch of kda_fwd_scratch_bytes(); 0 if a size is invalid. */
 size_t kda_fwd_workspace_bytes(int B, int T, int HV, int K, int V);
 
-/* Bytes kda_bwd needs: the chunk states, the gradients of the state leaving
- * every chunk (same layout), and, when HV > H, fp32 per-value-head partials
- * of dq and dk [B, T, HV, K] each; 0 if a size is invalid. */
+/* Bytes of the optional scratch that lets kda_fwd without stored states run
+ * as two kernels (K = V = 128, bf16): a chunk-parallel pass that leaves every
+ * 64-step chunk's operands of the state products there (165 KB per chunk),
+ * then the sequential state pass.  0 if the shape has no such path or a size
+ * is invalid. */
+size_t kda_fwd_scratch_bytes(int B, int T, int HV, int K, int V);
+
+/* Bytes kda_bwd needs: the chunk states and interaction records (as
+ * kda_fwd_workspace_bytes lays them out), then the larger of the forward's
+ * scratch and [gradients of the state leaving every 32 steps (state layout);
+ * when HV > H fp32 per-value-head partials of dq and dk [B, T, HV, K] each;
+ * per-chunk gradient records (K = V = 128)]; 0 if a size is invalid.  This is
+ * at least kda_fwd_workspace_bytes(), so one buffer serves both calls. */
 size_t kda_bwd_workspace_bytes(int B, int T, int H, int HV, int K, int V);
 
 /* Chunk-parallel prefill forward ("recurrent.py", naive_kda_fwd; the chunk
@@ -94,9 +107,11 @@ size_t kda_bwd_workspace_bytes(int B, int T, int H, int HV, int K, int V);
  *   S0    [B, HV, K, V]  float, or NULL for a zero initial state
  *   o     [B, T, HV, V]  dtype (output)
  *   S_T   [B, HV, K, V]  float (output), or NULL to skip the final state
- *   workspace: NULL, or at least kda_fwd_workspace_bytes(B, T, HV, K, V)
- *     bytes, 16-byte aligned; when given, the state entering every chunk is
- *     stored there for a later kda_bwd with KDA_BWD_STATES_FROM_FWD.
+ *   workspace: NULL; or, 16-byte aligned, at least
+ *     kda_fwd_workspace_bytes(B, T, HV, K, V) bytes: the states and records
+ *     for a later kda_bwd with KDA_BWD_STATES_FROM_FWD are stored there; or
+ *     at least kda_fwd_scratch_bytes() (but fewer than the former): used as
+ *     scratch only.  A workspace of neither size is KDA_ERR_WORKSPACE.
  * o and S_T must not alias any input.  S_T may alias S0 only if S0 is not
  * needed afterwards (S0 is read before S_T is written, per value column). */
 int kda_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,

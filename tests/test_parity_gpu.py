@@ -29,9 +29,10 @@ def kda():
     assert mod.device_status() == 0, "a kernel gave up on a bounded wait"
 
 
-def run_fwd(kda, inp, scale):
+def run_fwd(kda, inp, scale, scratch=True):
     d = to_cuda(inp)
-    o, S = kda.fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], scale=scale, initial_state=d["S0"])
+    o, S = kda.fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], scale=scale, initial_state=d["S0"],
+                   scratch=scratch)
     torch.cuda.synchronize()
     return o, S
 
@@ -41,8 +42,8 @@ def oracle_fwd(inp, scale):
                               f64(inp["beta"]), scale, f64(inp["S0"]))
 
 
-def check_fwd(kda, inp, scale, dtype, label):
-    o, S = run_fwd(kda, inp, scale)
+def check_fwd(kda, inp, scale, dtype, label, scratch=True):
+    o, S = run_fwd(kda, inp, scale, scratch)
     o_ref, S_ref = oracle_fwd(inp, scale)
     tol = tol_for(dtype)
     report(f"{label} o", f64(o), o_ref, tol, dtype)
@@ -87,6 +88,31 @@ def test_fwd_shapes(kda, name, base, over):
     check_fwd(kda, make_inputs(w), w.scale, w.torch_dtype, name)
 
 
+TC_CASES = [c for c in FWD_CASES if c[0].startswith("tc_")]
+
+
+@pytest.mark.parametrize("name,base,over", TC_CASES, ids=[c[0] for c in TC_CASES])
+def test_fwd_tc_single_kernel(kda, name, base, over):
+    """The tensor-core forward without a workspace (one kernel carrying the
+    whole chunk pipeline) on the same shapes as the two-kernel default."""
+    w = BY_NAME[base].with_sizes(**over)
+    check_fwd(kda, make_inputs(w), w.scale, w.torch_dtype, name + "_single", scratch=False)
+
+
+def test_fwd_tc_training_workspace_same_output(kda):
+    """With a training workspace (states and records stored) the two-kernel
+    forward gives bitwise the o and S_T of the scratch-only run."""
+    w = BY_NAME["prefill_gqa"].with_sizes(B=2, T=200, H=2, HV=4, s0_std=0.02)
+    d = to_cuda(make_inputs(w))
+    args = (d["q"], d["k"], d["v"], d["g"], d["beta"])
+    o1, S1 = kda.fwd(*args, scale=w.scale, initial_state=d["S0"])
+    ws = torch.empty(kda.workspace_bytes("fwd", w.B, w.T, w.H, w.HV, w.K, w.V), dtype=torch.uint8,
+                     device="cuda")
+    o2, S2 = kda.fwd(*args, scale=w.scale, initial_state=d["S0"], workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
+
+
 def test_fwd_strong_unbounded_decay(kda):
     """Very strong decays (|g| up to 40 per step) take the pair-by-pair path
     for diagonal blocks; results stay finite and match."""
@@ -104,6 +130,7 @@ def test_fwd_tc_strong_unbounded_decay(kda):
     inp = make_inputs(w)
     inp["g"] = inp["g"] * 8.0
     check_fwd(kda, inp, w.scale, w.torch_dtype, "tc_strong_decay")
+    check_fwd(kda, inp, w.scale, w.torch_dtype, "tc_strong_decay_single", scratch=False)
 
 
 def test_fwd_prefill_gqa_full_size(kda):
@@ -188,6 +215,7 @@ BWD_CASES = [
     ("fp32_K64_gqa", "twin", dict(B=2, T=64, H=1, HV=3, K=64, V=64)),
     ("bf16_K128_gqa_ragged", "prefill_gqa", dict(T=45, H=2, HV=4)),
     ("bf16_K128", "fwdbwd", dict(B=1, T=130, H=2, HV=2)),
+    ("bf16_K128_T96_half_chunk", "fwdbwd", dict(B=1, T=96, H=1, HV=2, s0_std=0.02)),
     ("fp32_K128V32", "fwdbwd", dict(B=1, T=40, H=1, HV=1, V=32, dtype="fp32", s0_std=0.05)),
 ]
 
@@ -200,6 +228,30 @@ def test_bwd_shapes(kda, name, base, over):
     if "dST" in name:
         dS_T = torch.randn(w.B, w.HV, w.K, w.V, generator=torch.Generator().manual_seed(5))
     check_bwd(kda, inp, w.scale, w.torch_dtype, name, dS_T)
+
+
+def test_bwd_misaligned_dO_after_tensor_core_forward(kda):
+    """A dO that is not 16-byte aligned keeps the backward off the tensor-core
+    path; with states_from_fwd it must then not rely on the tensor-core
+    forward's states (which keep only the chunk starts)."""
+    w = BY_NAME["fwdbwd"].with_sizes(B=1, T=100, H=2, HV=2)
+    inp = make_inputs(w, with_do=True)
+    d = to_cuda(inp)
+    buf = torch.empty(d["dO"].numel() + 1, dtype=d["dO"].dtype, device="cuda")
+    dO = buf[1:].view(d["dO"].shape)
+    dO.copy_(d["dO"])
+    assert dO.data_ptr() % 16 != 0
+    B, T, H, K = d["q"].shape
+    HV, V = d["v"].shape[2], d["v"].shape[3]
+    ws = torch.empty(kda.workspace_bytes("bwd", B, T, H, HV, K, V), dtype=torch.uint8, device="cuda")
+    kda.fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], scale=w.scale, workspace=ws)
+    got = kda.bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], dO, scale=w.scale, workspace=ws,
+                  states_from_fwd=True)
+    torch.cuda.synchronize()
+    ref = oracle_bwd(inp, w.scale)
+    for n, x, r in zip(GRAD_NAMES, got, ref):
+        out_dtype = w.torch_dtype if n in ("dq", "dk", "dv") else torch.float32
+        report(f"misaligned_dO {n}", f64(x), r, tol_for(w.torch_dtype), out_dtype)
 
 
 def test_bwd_reuses_forward_states(kda):
