@@ -417,8 +417,12 @@ __global__ void kda_group_sum_kernel(const float* __restrict__ part, TIn* __rest
 // then the interaction terms (factored_terms) and dg = reverse cumsum of dc.
 // Everything here is independent across key channels, so one CTA handles one
 // (b, hv, chunk, quarter of the 128 key channels); two CTAs fit on an SM.
+// Row strides (words): LDK = 40 (8 mod 32) puts the warp-MMA fragment loads of
+// K, Q and c (lanes: row t, channel g) in 32 distinct banks; LDC = 68 (4 mod
+// 32) does the same for the row-term fragments of dP and dA (lanes: row g,
+// column t).  Accesses with the lanes along a row are conflict-free anyway.
 struct AsmSmem {
-  static constexpr int C = 64, KQ = 32, LDK = KQ + 1, LDC = C + 1;
+  static constexpr int C = 64, KQ = 32, LDK = 40, LDC = 68;
   static constexpr int oK = 0, oQ = oK + C * LDK, oC = oQ + C * LDK, oDq = oC + C * LDK, oDk = oDq + C * LDK,
                        oDc = oDk + C * LDK, oE1 = oDc + C * LDK, oE2o = oE1 + C * LDK, oE2d = oE2o + BS * LDK,
                        odA = oE2d + BS * LDK, odP = odA + C * LDC, oBeta = odP + C * LDC, oSeg = oBeta + C,
@@ -472,13 +476,15 @@ __global__ void __launch_bounds__(NTHREADS, 2) kda_bwd_assemble_kernel(BwdArgs a
   const TIn* k = static_cast<const TIn*>(a.k);
   const int tid = threadIdx.x;
 
-  float4 qe[2], ke[2], kd[2];  // [dQE; dKE'] and dKEd of this quarter, consumed further down
+  // [dQE; dKE'] and dKEd of this quarter, consumed further down: lane = channel f,
+  // warp w = rows 8w .. 8w + 7 (each row a 128-byte run of the row-major record)
+  const int ef = tid & 31, ei = (tid >> 5) * 8;
+  float qe[8], ke[8], kd[8];
 #pragma unroll
-  for (int m = 0; m < 2; ++m) {  // channel f of the quarter, four rows per item
-    const int idx = tid + m * NTHREADS, f = idx >> 4, i4 = (idx & 15) * 4;
-    qe[m] = *reinterpret_cast<const float4*>(rec + G_QK + (f0 + f) * 128 + i4);
-    ke[m] = *reinterpret_cast<const float4*>(rec + G_QK + (f0 + f) * 128 + 64 + i4);
-    kd[m] = *reinterpret_cast<const float4*>(rec + G_KED + (f0 + f) * 64 + i4);
+  for (int u = 0; u < 8; ++u) {
+    qe[u] = rec[G_QK + (ei + u) * 128 + f0 + ef];
+    ke[u] = rec[G_QK + (64 + ei + u) * 128 + f0 + ef];
+    kd[u] = rec[G_KED + (ei + u) * 128 + f0 + ef];
   }
   {  // inputs of this channel quarter (4 channels per item) and the C x C adjoints; loads first
     float4 gv[2], dp[4], da[4];
@@ -500,10 +506,10 @@ __global__ void __launch_bounds__(NTHREADS, 2) kda_bwd_assemble_kernel(BwdArgs a
       }
     }
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {  // column j of [dP; dA], four rows per item
-      const int idx = tid + m * NTHREADS, j = idx >> 4, i4 = (idx & 15) * 4;
-      dp[m] = *reinterpret_cast<const float4*>(rec + G_PA + j * 128 + i4);
-      da[m] = *reinterpret_cast<const float4*>(rec + G_PA + j * 128 + 64 + i4);
+    for (int m = 0; m < 4; ++m) {  // row i of [dP; dA], four columns j per item
+      const int idx = tid + m * NTHREADS, i = idx >> 4, j4 = (idx & 15) * 4;
+      dp[m] = *reinterpret_cast<const float4*>(rec + G_PA + i * 64 + j4);
+      da[m] = *reinterpret_cast<const float4*>(rec + G_PA + (64 + i) * 64 + j4);
     }
     if (tid < C) sBeta[tid] = (tid < L) ? a.beta[((size_t)b * T + t0 + tid) * a.HV + hv] : 0.f;
 #pragma unroll
@@ -519,14 +525,19 @@ __global__ void __launch_bounds__(NTHREADS, 2) kda_bwd_assemble_kernel(BwdArgs a
     }
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
-      const int idx = tid + m * NTHREADS, j = idx >> 4, i4 = (idx & 15) * 4;
+      const int idx = tid + m * NTHREADS, i = idx >> 4, j4 = (idx & 15) * 4;
       const float vdp[4] = {dp[m].x, dp[m].y, dp[m].z, dp[m].w}, vda[4] = {da[m].x, da[m].y, da[m].z, da[m].w};
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int i = i4 + u;
-        sdP[i * LDC + j] = (j <= i) ? vdp[u] : 0.f;
-        sdA[i * LDC + j] = (j < i) ? vda[u] : 0.f;
-      }
+      float4 wp, wa;
+      wp.x = (j4 <= i) ? vdp[0] : 0.f;
+      wp.y = (j4 + 1 <= i) ? vdp[1] : 0.f;
+      wp.z = (j4 + 2 <= i) ? vdp[2] : 0.f;
+      wp.w = (j4 + 3 <= i) ? vdp[3] : 0.f;
+      wa.x = (j4 < i) ? vda[0] : 0.f;
+      wa.y = (j4 + 1 < i) ? vda[1] : 0.f;
+      wa.z = (j4 + 2 < i) ? vda[2] : 0.f;
+      wa.w = (j4 + 3 < i) ? vda[3] : 0.f;
+      *reinterpret_cast<float4*>(sdP + i * LDC + j4) = wp;  // LDC = 68: rows 16-byte aligned
+      *reinterpret_cast<float4*>(sdA + i * LDC + j4) = wa;
     }
   }
   __syncthreads();
@@ -556,9 +567,10 @@ __global__ void __launch_bounds__(NTHREADS, 2) kda_bwd_assemble_kernel(BwdArgs a
   {  // element-wise terms; the chunk-end sum of dKEd o k o e^{c_last-c} goes through sE1
 #pragma unroll
     for (int m = 0; m < 2; ++m) {
-      const int idx = tid + m * NTHREADS, f = idx >> 4, i4 = (idx & 15) * 4;
-      const float vq[4] = {qe[m].x, qe[m].y, qe[m].z, qe[m].w}, vk[4] = {ke[m].x, ke[m].y, ke[m].z, ke[m].w},
-                  vd[4] = {kd[m].x, kd[m].y, kd[m].z, kd[m].w};
+      const int f = ef, i4 = ei + 4 * m;
+      const float vq[4] = {qe[4 * m], qe[4 * m + 1], qe[4 * m + 2], qe[4 * m + 3]},
+                  vk[4] = {ke[4 * m], ke[4 * m + 1], ke[4 * m + 2], ke[4 * m + 3]},
+                  vd[4] = {kd[4 * m], kd[4 * m + 1], kd[4 * m + 2], kd[4 * m + 3]};
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int i = i4 + u, o = i * LDK + f;
@@ -594,9 +606,9 @@ __global__ void __launch_bounds__(NTHREADS, 2) kda_bwd_assemble_kernel(BwdArgs a
       wide = sC[(16 * J) * LDK + f] - sC[(16 * J + 15) * LDK + f] > DIAG_SPAN_MAX;
     }
     if (__syncthreads_or(wide))
-      factored_terms<KQ, C, false, false>(sK, sQ, sC, sdA, sdP, sE1, sE2o, sE2d, sFlag, sDq, sDk, sDc);
+      factored_terms<KQ, C, false, false, LDK, LDC>(sK, sQ, sC, sdA, sdP, sE1, sE2o, sE2d, sFlag, sDq, sDk, sDc);
     else
-      factored_terms_fused<KQ>(sK, sQ, sC, sdA, sdP, sDq, sDk, sDc);
+      factored_terms_fused<KQ, LDK, LDC>(sK, sQ, sC, sdA, sdP, sDq, sDk, sDc);
   }
   cumsum64<true>(sDc, sSeg, sLast);
   TIn* dq = static_cast<TIn*>(a.dq);

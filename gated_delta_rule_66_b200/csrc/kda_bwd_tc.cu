@@ -94,7 +94,7 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_dstate_tc_kernel(BwdArgs a) {
       if (tid == 64) prefetch_l2(irec - INTER_REC, 16384);
       if (tid == 192) prefetch_l2(irec - INTER_REC + INTER_TT, 16384);
     }
-    load_raw_wait();
+    if (!load_raw_wait(cx)) { failed = true; break; }
     cumsum_span(cx);
 
     // ---------------------------------------------------------------- operands of the gradient products
@@ -344,7 +344,7 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
     else if (tid == 32) prefetch_l2(irec, 2 * 16384);
     else if (tid == 33) prefetch_l2(irec + INTER_TT, 16384);
     else if (tid >= 64 && tid < 64 + L) prefetch_l2(vg + (((size_t)b * T + t0 + tid - 64) * a.HV + hv) * VD, VD * 2);
-    load_raw_wait();
+    if (!load_raw_wait(cx)) { failed = true; break; }
     cumsum_span(cx);
 
     // ---------------------------------------------------------------- K o e^c, K o e^{c_last-c}, dO, dO^T
@@ -507,21 +507,25 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
     if (!wait_mma(bar, phase)) { failed = true; break; }
 
     // ---------------------------------------------------------------- record
-    {
+    {  // rows (TMEM lanes) row-major: each lane stores its 32 consecutive columns as 16-byte pieces
       float v[32];
       tmem_ld32(tm + lo + TM_PA + hcol * 32, v);
+      float4* dst = reinterpret_cast<float4*>(rec + G_PA + Lr * 64 + hcol * 32);
 #pragma unroll
-      for (int jj = 0; jj < 32; ++jj) rec[G_PA + (hcol * 32 + jj) * 128 + Lr] = v[jj];
+      for (int q4 = 0; q4 < 8; ++q4) dst[q4] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
       for (int cb = 0; cb < 2; ++cb) {
         const int f0 = hcol * 64 + cb * 32;
         tmem_ld32(tm + lo + TM_QK + f0, v);
+        dst = reinterpret_cast<float4*>(rec + G_QK + Lr * 128 + f0);
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) rec[G_QK + (f0 + jj) * 128 + Lr] = v[jj];
+        for (int q4 = 0; q4 < 8; ++q4) dst[q4] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
         tmem_ld32(tm + lo + TM_KED + f0, v);
         if (lane < 16) {
           const int r = cx.sub * 16 + lane;  // M = 64 accumulator layout
+          dst = reinterpret_cast<float4*>(rec + G_KED + r * 128 + f0);
 #pragma unroll
-          for (int jj = 0; jj < 32; ++jj) rec[G_KED + (f0 + jj) * 64 + r] = v[jj];
+          for (int q4 = 0; q4 < 8; ++q4)
+            dst[q4] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
         }
       }
       if (tid < C) rec[G_DBR + tid] = sDbR[tid];

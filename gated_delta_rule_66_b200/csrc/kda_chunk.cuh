@@ -120,10 +120,10 @@ __device__ __forceinline__ void load_chunk_qkgb(const TIn* __restrict__ q, const
 //   sE2d[j][f] = exp(c_mid(J),f  - c_jf) for j in J (diagonal block columns)
 // Returns (block-uniformly) whether the diagonal block must be formed pair
 // by pair because its decay span exceeds DIAG_SPAN_MAX.
-template <int K, int C, bool PRECISE>
+template <int K, int C, bool PRECISE, int LDK_ = K + 1>
 __device__ __forceinline__ bool block_factors(int J, const float* sC, float* sE1, float* sE2o,
                                               float* sE2d, int* sFlag) {
-  constexpr int LDK = K + 1;
+  constexpr int LDK = LDK_;
   const int r0 = J * BS, rho_off = r0 + BS - 1, rho_diag = r0 + BS / 2 - 1;
   if (threadIdx.x == 0) *sFlag = 0;
   __syncthreads();
@@ -250,11 +250,11 @@ __device__ void invert_unit_lower(const float* sAh, const float* sBeta, float* s
 // are the scratch of block_factors.  One column block J at a time:
 // factored_block_scalar with fp32 FMA (any block), factored_block_mma with
 // 3xTF32 warp MMAs (blocks whose exponents split, K a multiple of 8).
-template <int K, int C, bool PRECISE>
+template <int K, int C, bool PRECISE, int LDK_ = K + 1, int LDC_ = C + 1>
 __device__ void factored_block_scalar(int J, bool pairwise, const float* sK, const float* sQ, const float* sC,
                                       const float* sdA, const float* sdP, const float* sE1, const float* sE2o,
                                       const float* sE2d, float* sDq, float* sDk, float* sDc) {
-  constexpr int LDK = K + 1, LDC = C + 1;
+  constexpr int LDK = LDK_, LDC = LDC_;
     const int r0 = J * BS;
     // row terms: rows i >= r0 against the columns of block J
     for (int idx = threadIdx.x; idx < (C - r0) * K; idx += NTHREADS) {
@@ -346,11 +346,11 @@ __device__ __forceinline__ void mma3(float (&d)[4], const Split (&a)[4], const S
   mma_16x8x8(d, ah, bh);
 }
 
-template <int K, int C>
+template <int K, int C, int LDK_ = K + 1, int LDC_ = C + 1>
 __device__ void factored_block_mma(int J, const float* sK, const float* sQ, const float* sdA, const float* sdP,
                                    const float* sE1, const float* sE2o, const float* sE2d, float* sDq, float* sDk,
                                    float* sDc) {
-  constexpr int LDK = K + 1, LDC = C + 1, NB = C / BS, NTL = K / 8;
+  constexpr int LDK = LDK_, LDC = LDC_, NB = C / BS, NTL = K / 8;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int r0 = J * BS;
   // row terms: row block I >= J, 8 key channels per tile
@@ -432,10 +432,10 @@ __device__ void factored_block_mma(int J, const float* sK, const float* sQ, cons
 // split A fragment feeds both 8-channel halves.  The split-exponent factors
 // are formed on the fly from c (natural units).  Requires every 16-row
 // block's decay span to be at most 80 (checked by the caller).
-template <int K>
+template <int K, int LDK_ = K + 1, int LDC_ = 65>
 __device__ void factored_terms_fused(const float* sK, const float* sQ, const float* sC, const float* sdA,
                                      const float* sdP, float* sDq, float* sDk, float* sDc) {
-  constexpr int C = 64, LDK = K + 1, LDC = C + 1, NH = K / 16;
+  constexpr int C = 64, LDK = LDK_, LDC = LDC_, NH = K / 16;
   static_assert(4 * NH == NTHREADS / 32, "one 16 x 16 tile per warp");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int I = warp / NH, fb = (warp % NH) * 16, i0 = I * BS;
@@ -526,17 +526,18 @@ __device__ void factored_terms_fused(const float* sK, const float* sQ, const flo
   __syncthreads();
 }
 
-template <int K, int C, bool PRECISE, bool USE_MMA>
+template <int K, int C, bool PRECISE, bool USE_MMA, int LDK_ = K + 1, int LDC_ = C + 1>
 __device__ void factored_terms(const float* sK, const float* sQ, const float* sC, const float* sdA,
                                const float* sdP, float* sE1, float* sE2o, float* sE2d, int* sFlag,
                                float* sDq, float* sDk, float* sDc) {
   constexpr int NB = C / BS;
   for (int J = 0; J < NB; ++J) {
-    const bool pairwise = block_factors<K, C, PRECISE>(J, sC, sE1, sE2o, sE2d, sFlag);
+    const bool pairwise = block_factors<K, C, PRECISE, LDK_>(J, sC, sE1, sE2o, sE2d, sFlag);
     if (USE_MMA && !pairwise)
-      factored_block_mma<K, C>(J, sK, sQ, sdA, sdP, sE1, sE2o, sE2d, sDq, sDk, sDc);
+      factored_block_mma<K, C, LDK_, LDC_>(J, sK, sQ, sdA, sdP, sE1, sE2o, sE2d, sDq, sDk, sDc);
     else
-      factored_block_scalar<K, C, PRECISE>(J, pairwise, sK, sQ, sC, sdA, sdP, sE1, sE2o, sE2d, sDq, sDk, sDc);
+      factored_block_scalar<K, C, PRECISE, LDK_, LDC_>(J, pairwise, sK, sQ, sC, sdA, sdP, sE1, sE2o, sE2d, sDq,
+                                                       sDk, sDc);
   }
 }
 

@@ -65,7 +65,7 @@ __device__ __forceinline__ bool fwd_chunk_head(const tcc::Ctx& cx, const FwdArgs
   load_raw_issue(cx, qg, kg, vg, a.g, a.beta, b, T, t0, L, a.H, a.HV, h, hv);
   if (prefetch_next && ch + 1 < NT)
     prefetch_chunk(cx, qg, kg, vg, a.g, b, T, t0 + C, min(C, T - t0 - C), a.H, a.HV, h, hv);
-  load_raw_wait();
+  if (!load_raw_wait(cx)) return false;
   const bool wide = cumsum_span(cx);
   build_op1_and_issue(cx, a.scale, tm + TM_APA, tm + TM_APB, bar);
   if (!wait_mma(bar, phase)) return false;
@@ -115,7 +115,7 @@ __device__ __forceinline__ bool fwd_chunk_head(const tcc::Ctx& cx, const FwdArgs
     bulk_commit();
   }
 
-  readout_ap(cx, tm + TM_APA, tm + TM_APB, false, wide, pw, irec);
+  readout_ap(cx, tm + TM_APA, tm + TM_APB, wide, pw, irec);
   invert(cx);
   {  // T as the operand image (rows i, K = j); with a record also its T, T^T images and Ah
     const float* tr = reinterpret_cast<const float*>(sm + R_TROW);

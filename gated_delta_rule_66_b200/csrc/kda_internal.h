@@ -10,10 +10,9 @@ constexpr int FWD_CHUNK = 32;    // chunk length of the chunked kernels
 constexpr int FWD_VBLOCK = 32;   // V columns per CTA in the chunked kernels
 
 // Per-(b, hv, 64-step chunk) record of the tensor-core backward (floats),
-// column-major so that the TMEM lanes (rows) are contiguous:
-// Ah [i][j] (row-major 64 x 64), [dP; dA] as [j][i'] (64 x 128, i' < 64 dP),
-// [dQE; dKE'] as [f][i'] (128 x 128, i' < 64 dQE), dKEd as [f][i] (128 x 64),
-// dbeta_R [64], dEl [128].
+// row-major: [dP; dA] as [i'][j] (128 x 64, i' < 64 dP), [dQE; dKE'] as
+// [i'][f] (128 x 128, i' < 64 dQE), dKEd as [i][f] (64 x 128), dbeta_R [64],
+// dEl [128] (G_AH unused).
 // Per-(b, hv, 64-step chunk) interaction record that the tensor-core forward
 // stores with a workspace (floats).  Three 64 x 64 tf32 operand images in the
 // K-major canonical layout of the tensor-core kernels (element (r, k) at

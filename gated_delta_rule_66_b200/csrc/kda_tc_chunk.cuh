@@ -73,10 +73,12 @@ __device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast
 
 // Asynchronous load of one chunk: q, k rows of query/key head h, x rows of
 // value head hv (v or dO), g rows and beta; rows past the sequence end are
-// zero.  Issues the copies only; load_raw_wait completes them.
+// zero.  Issues the copies only; load_raw_wait completes them.  (16-byte
+// cp.async per thread: measured faster here than per-row bulk copies issued
+// by one warp.)
 __device__ __forceinline__ void load_raw_issue(const Ctx& c, const __nv_bfloat16* q, const __nv_bfloat16* k,
-                                         const __nv_bfloat16* x, const float* g, const float* beta,
-                                         int b, int T, int t0, int L, int H, int HV, int h, int hv) {
+                                               const __nv_bfloat16* x, const float* g, const float* beta,
+                                               int b, int T, int t0, int L, int H, int HV, int h, int hv) {
   using namespace tc;
   for (int e = c.tid; e < C * 16; e += NTH) {
     const int i = e >> 4, vec = e & 15;
@@ -94,9 +96,12 @@ __device__ __forceinline__ void load_raw_issue(const Ctx& c, const __nv_bfloat16
   }
   if (c.tid < C) c.beta()[c.tid] = (c.tid < L) ? beta[((size_t)b * T + t0 + c.tid) * HV + hv] : 0.f;
 }
-__device__ __forceinline__ void load_raw_wait() {
+// Completes load_raw_issue (wait + barrier).  Returns true (the form of a
+// bounded wait, for the callers' uniform error path).
+__device__ __forceinline__ bool load_raw_wait(const Ctx&) {
   tc::cp_async_wait_all();
   __syncthreads();
+  return true;
 }
 
 // L2 prefetch of one chunk's q, k, x (v or dO) and g rows, for a chunk that a
@@ -251,17 +256,14 @@ __device__ __forceinline__ void pairwise_compute(const Ctx& c, float scale, Pair
   }
 }
 
-// byte offset of P[i][j] in its operand tile: P itself (rows i, K = j) for the
-// forward readout, P^T (rows j, K = i) for the backward
-__device__ __forceinline__ uint32_t p_off(int i, int j, bool transP) {
-  return R_P + (transP ? tc::kmaj(j, i, 64) : tc::kmaj(i, j, 64));
-}
+// byte offset of P[i][j] in its operand tile (rows i, K = j)
+__device__ __forceinline__ uint32_t p_off(int i, int j) { return R_P + tc::kmaj(i, j, 64); }
 
 // Reads Ah (row-major, stride 65, at R_AH) and P (tf32 operand at R_P) out of
 // the two interaction products; the raw region must be free.  With `pt` it
 // also stores the P^T image of the interaction record.  Ends with a barrier.
-__device__ __forceinline__ void readout_ap(const Ctx& c, uint32_t tm_apa, uint32_t tm_apb, bool transP,
-                                           bool wide, const Pairwise& pw, float* pt = nullptr) {
+__device__ __forceinline__ void readout_ap(const Ctx& c, uint32_t tm_apa, uint32_t tm_apb, bool wide,
+                                           const Pairwise& pw, float* pt = nullptr) {
   using namespace tc;
   float* sAh = reinterpret_cast<float*>(c.sm + R_AH);
   {
@@ -269,17 +271,25 @@ __device__ __forceinline__ void readout_ap(const Ctx& c, uint32_t tm_apa, uint32
     tmem_ld32(tm_apa + c.lo + c.hcol * 32, v);
     const bool isA = c.Lr < 64;
     const int i = isA ? c.Lr : c.Lr - 64;
+    if (isA) {
 #pragma unroll
-    for (int jj = 0; jj < 32; ++jj) {
-      const int j = c.hcol * 32 + jj;
-      const bool same = (i >> 5) == (j >> 5);
-      if (!same && i >= 32) continue;  // lower-left block comes from product b
-      const float val = (same && (isA ? j < i : j <= i)) ? v[jj] : 0.f;
-      if (isA) {
-        sAh[i * 65 + j] = val;
-      } else {
-        st_tf32(c.sm, p_off(i, j, transP), val);
-        if (pt) pt[img(j, i)] = __uint_as_float(tf32_rna(val));
+      for (int jj = 0; jj < 32; ++jj) {
+        const int j = c.hcol * 32 + jj;
+        const bool same = (i >> 5) == (j >> 5);
+        if (!same && i >= 32) continue;  // lower-left block comes from product b
+        sAh[i * 65 + j] = (same && j < i) ? v[jj] : 0.f;
+      }
+    } else if (!(i >= 32 && c.hcol == 0)) {  // P rows: four columns per 16-byte store
+#pragma unroll
+      for (int j4 = 0; j4 < 32; j4 += 4) {
+        float w[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int j = c.hcol * 32 + j4 + u;
+          w[u] = ((i >> 5) == (j >> 5) && j <= i) ? v[j4 + u] : 0.f;
+          if (pt) pt[img(j, i)] = __uint_as_float(tf32_rna(w[u]));
+        }
+        st_tf32x4(c.sm, p_off(i, c.hcol * 32 + j4), w[0], w[1], w[2], w[3]);
       }
     }
   }
@@ -288,14 +298,17 @@ __device__ __forceinline__ void readout_ap(const Ctx& c, uint32_t tm_apa, uint32
     tmem_ld16(tm_apb + c.lo + c.hcol * 16, v);
     if (c.lane < 16) {
       const int r = c.sub * 16 + c.lane;  // row of the 64-row product (M = 64 accumulator layout)
+      if (r < 32) {
 #pragma unroll
-      for (int jj = 0; jj < 16; ++jj) {
-        const int j = c.hcol * 16 + jj;
-        if (r < 32) {
-          sAh[(32 + r) * 65 + j] = v[jj];
-        } else {
-          st_tf32(c.sm, p_off(r, j, transP), v[jj]);
-          if (pt) pt[img(j, r)] = __uint_as_float(tf32_rna(v[jj]));
+        for (int jj = 0; jj < 16; ++jj) sAh[(32 + r) * 65 + c.hcol * 16 + jj] = v[jj];
+      } else {
+#pragma unroll
+        for (int j4 = 0; j4 < 16; j4 += 4) {
+          const int j = c.hcol * 16 + j4;
+          st_tf32x4(c.sm, p_off(r, j), v[j4], v[j4 + 1], v[j4 + 2], v[j4 + 3]);
+          if (pt)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) pt[img(j + u, r)] = __uint_as_float(tf32_rna(v[j4 + u]));
         }
       }
     }
@@ -306,7 +319,7 @@ __device__ __forceinline__ void readout_ap(const Ctx& c, uint32_t tm_apa, uint32
       const int j = pw.j0 + jj;
       if (pw.kind == 0 && j < pw.i) sAh[pw.i * 65 + j] = pw.v[jj];
       if (pw.kind == 1 && j <= pw.i) {
-        st_tf32(c.sm, p_off(pw.i, j, transP), pw.v[jj]);
+        st_tf32(c.sm, p_off(pw.i, j), pw.v[jj]);
         if (pt) pt[img(j, pw.i)] = __uint_as_float(tf32_rna(pw.v[jj]));
       }
     }
