@@ -107,15 +107,13 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_dstate_tc_kernel(BwdArgs a) {
           const int i = item_row(cx, m);
           const float4 c4 = ld4(sC + i * LDCF + fq);
           float kf[4];
-          bf16x4(sm + RAW_K + i * 256 + fq * 2, kf);
+          bf16x4(sm + RAW_K + raw_off(i, fq), kf);
           st_tf32x4(sm, OP_KED + kmaj(i, fq, 128), kf[0] * ex2(c63[0] - c4.x), kf[1] * ex2(c63[1] - c4.y),
                     kf[2] * ex2(c63[2] - c4.z), kf[3] * ex2(c63[3] - c4.w));
         }
       }
       {  // (Q~ o e^c)^T and -(diag(beta) K o e^c)^T as [f][i]: one channel x 4 rows, 16-byte stores
         const int f = tid & 127;
-        const __nv_bfloat16* qcol = reinterpret_cast<const __nv_bfloat16*>(sm + RAW_Q) + f;
-        const __nv_bfloat16* kcol = reinterpret_cast<const __nv_bfloat16*>(sm + RAW_K) + f;
         for (int m = 0; m < 8; ++m) {
           const int i0 = ((tid >> 7) + 2 * m) * 4;
           float qe[4], nke[4];
@@ -123,8 +121,9 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_dstate_tc_kernel(BwdArgs a) {
           for (int u = 0; u < 4; ++u) {
             const int i = i0 + u;
             const float e = ex2(sC[i * LDCF + f]);
-            qe[u] = a.scale * __bfloat162float(qcol[i * 128]) * e;
-            nke[u] = -sBeta[i] * __bfloat162float(kcol[i * 128]) * e;
+            const uint32_t o = raw_off(i, f);
+            qe[u] = a.scale * __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + RAW_Q + o)) * e;
+            nke[u] = -sBeta[i] * __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + RAW_K + o)) * e;
           }
           st_tf32x4(sm, OP_QET + kmaj(f, i0, 64), qe[0], qe[1], qe[2], qe[3]);
           st_tf32x4(sm, OP_NKET + kmaj(f, i0, 64), nke[0], nke[1], nke[2], nke[3]);
@@ -134,10 +133,10 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_dstate_tc_kernel(BwdArgs a) {
       // dO^T into TMEM: lane n, columns j
       {
         uint32_t r[32];
-        const unsigned char* col = sm + RAW_X + Lr * 2;
 #pragma unroll
         for (int jj = 0; jj < 32; ++jj)
-          r[jj] = tf32_rna(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(col + (hcol * 32 + jj) * 256)));
+          r[jj] = tf32_rna(__bfloat162float(
+              *reinterpret_cast<const __nv_bfloat16*>(sm + RAW_X + raw_off(hcol * 32 + jj, Lr))));
         tmem_st32(tm + lo + TM_DOT + hcol * 32, r);
         tmem_wait_st();
       }
@@ -357,8 +356,8 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
         const float4 c4 = ld4(sC + i * LDCF + fq);
         const float c[4] = {c4.x, c4.y, c4.z, c4.w};
         float kf[4], df[4];
-        bf16x4(sm + RAW_K + i * 256 + fq * 2, kf);
-        bf16x4(sm + RAW_X + i * 256 + fq * 2, df);
+        bf16x4(sm + RAW_K + raw_off(i, fq), kf);
+        bf16x4(sm + RAW_X + raw_off(i, fq), df);
         float e[4], ed[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -370,10 +369,10 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
         st_tf32x4(sm, OP_DO + kmaj_pad(i, fq, 128), df[0], df[1], df[2], df[3]);
       }
       uint32_t r[32];
-      const unsigned char* col = sm + RAW_X + Lr * 2;
 #pragma unroll
       for (int jj = 0; jj < 32; ++jj)
-        r[jj] = tf32_rna(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(col + (hcol * 32 + jj) * 256)));
+        r[jj] = tf32_rna(__bfloat162float(
+              *reinterpret_cast<const __nv_bfloat16*>(sm + RAW_X + raw_off(hcol * 32 + jj, Lr))));
       tmem_st32(tm + lo + TM_DOT + hcol * 32, r);
       tmem_wait_st();
     }

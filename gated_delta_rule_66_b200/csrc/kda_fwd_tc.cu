@@ -77,7 +77,7 @@ __device__ __forceinline__ bool fwd_chunk_head(const tcc::Ctx& cx, const FwdArgs
       const int i = item_row(cx, m);
       const float4 c4 = ld4(sC + i * LDCF + fq);
       float qf[4];
-      bf16x4(sm + RAW_Q + i * 256 + fq * 2, qf);
+      bf16x4(sm + RAW_Q + raw_off(i, fq), qf);
       st_tf32x4(sm, OP_QE + kmaj(i, fq, 128), a.scale * qf[0] * ex2(c4.x), a.scale * qf[1] * ex2(c4.y),
                 a.scale * qf[2] * ex2(c4.z), a.scale * qf[3] * ex2(c4.w));
     }
@@ -85,18 +85,18 @@ __device__ __forceinline__ bool fwd_chunk_head(const tcc::Ctx& cx, const FwdArgs
   {  // transposed operands [f][i]: thread items of one channel x 4 rows, 16-byte stores
     const int f = tid & 127;
     const float c63 = sC[63 * LDCF + f];
-    const __nv_bfloat16* kcol = reinterpret_cast<const __nv_bfloat16*>(sm + RAW_K) + f;
-    const __nv_bfloat16* vcol = reinterpret_cast<const __nv_bfloat16*>(sm + RAW_X) + f;
+
     for (int m = 0; m < 8; ++m) {
       const int i0 = ((tid >> 7) + 2 * m) * 4;
       float bke[4], ked[4], bv[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int i = i0 + u;
-        const float c = sC[i * LDCF + f], kk = __bfloat162float(kcol[i * 128]), bi = sBeta[i];
+        const float c = sC[i * LDCF + f], bi = sBeta[i];
+        const float kk = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + RAW_K + raw_off(i, f)));
         bke[u] = bi * kk * ex2(c);
         ked[u] = kk * ex2(c63 - c);
-        bv[u] = bi * __bfloat162float(vcol[i * 128]);
+        bv[u] = bi * __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + RAW_X + raw_off(i, f)));
       }
       st_tf32x4(sm, OP_BKET + kmaj(f, i0, 64), bke[0], bke[1], bke[2], bke[3]);
       st_tf32x4(sm, OP_KEDT + kmaj(f, i0, 64), ked[0], ked[1], ked[2], ked[3]);

@@ -46,6 +46,13 @@ static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 static_assert(R_T + 16384 <= OP && R_P + 16384 <= R_T && R_SW + 3072 <= R_P && R_WOP + 36864 <= R_P,
               "raw-region reuse (the padded W overlaps only the dead inverse scratch)");
 
+// byte offset of bf16 element (row i, channel f) in a raw q / k / x tile:
+// the 16-byte pieces of row i are stored XOR-swizzled by i % 8, so that one
+// piece of 8 consecutive rows lies in 8 different bank groups
+__device__ __forceinline__ uint32_t raw_off(int i, int f) {
+  return (uint32_t)(i * 256 + ((f >> 3) ^ (i & 7)) * 16 + (f & 7) * 2);
+}
+
 struct Ctx {
   unsigned char* sm;
   uint32_t sb;      // shared address of sm
@@ -84,9 +91,10 @@ __device__ __forceinline__ void load_raw_issue(const Ctx& c, const __nv_bfloat16
     const int i = e >> 4, vec = e & 15;
     const bool ok = i < L;
     const size_t t = (size_t)b * T + t0 + (ok ? i : 0);  // row 0 of the chunk is always valid
-    cp_async16(c.sb + RAW_Q + i * 256 + vec * 16, q + (t * H + h) * KD + vec * 8, ok);
-    cp_async16(c.sb + RAW_K + i * 256 + vec * 16, k + (t * H + h) * KD + vec * 8, ok);
-    cp_async16(c.sb + RAW_X + i * 256 + vec * 16, x + (t * HV + hv) * VD + vec * 8, ok);
+    const uint32_t d = raw_off(i, vec * 8);
+    cp_async16(c.sb + RAW_Q + d, q + (t * H + h) * KD + vec * 8, ok);
+    cp_async16(c.sb + RAW_K + d, k + (t * H + h) * KD + vec * 8, ok);
+    cp_async16(c.sb + RAW_X + d, x + (t * HV + hv) * VD + vec * 8, ok);
   }
   for (int e = c.tid; e < C * 32; e += NTH) {
     const int i = e >> 5, vec = e & 31;
@@ -178,8 +186,8 @@ __device__ __forceinline__ void build_op1_and_issue(const Ctx& c, float scale, u
     const float4 c4 = ld4(sC + i * LDCF + fq);
     const float cc[4] = {c4.x, c4.y, c4.z, c4.w};
     float kf[4], qf[4];
-    bf16x4(c.sm + RAW_K + i * 256 + fq * 2, kf);
-    bf16x4(c.sm + RAW_Q + i * 256 + fq * 2, qf);
+    bf16x4(c.sm + RAW_K + raw_off(i, fq), kf);
+    bf16x4(c.sm + RAW_Q + raw_off(i, fq), qf);
     const float4 rr = (i < 32) ? r15 : r47;
     const float cr[4] = {rr.x, rr.y, rr.z, rr.w};
     float xa[4], ya[4];
@@ -239,16 +247,15 @@ __device__ __forceinline__ void pairwise_compute(const Ctx& c, float scale, Pair
   pw.kind = c.tid >> 7;
   pw.i = (c.tid >> 1) & 63;
   pw.j0 = (pw.i & 32) + (c.tid & 1) * 16;
-  const unsigned char* rowi = c.sm + (pw.kind ? RAW_Q : RAW_K) + pw.i * 256;
+  const unsigned char* xi = c.sm + (pw.kind ? RAW_Q : RAW_K);
   for (int jj = 0; jj < 16; ++jj) {
     const int j = pw.j0 + jj;
     float acc = 0.f;
     if (pw.kind ? (j <= pw.i) : (j < pw.i)) {
-      const unsigned char* rowj = c.sm + RAW_K + j * 256;
       for (int f = 0; f < KD; ++f) {
-        const float xi = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(rowi + 2 * f));
-        const float kj = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(rowj + 2 * f));
-        acc = fmaf(xi * kj, tc::ex2(sC[pw.i * LDCF + f] - sC[j * LDCF + f]), acc);
+        const float xv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(xi + raw_off(pw.i, f)));
+        const float kj = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(c.sm + RAW_K + raw_off(j, f)));
+        acc = fmaf(xv * kj, tc::ex2(sC[pw.i * LDCF + f] - sC[j * LDCF + f]), acc);
       }
       if (pw.kind) acc *= scale;
     }
