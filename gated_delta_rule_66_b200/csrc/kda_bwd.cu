@@ -482,9 +482,9 @@ __global__ void __launch_bounds__(NTHREADS, 2) kda_bwd_assemble_kernel(BwdArgs a
   float qe[8], ke[8], kd[8];
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
-    qe[u] = rec[G_QK + (ei + u) * 128 + f0 + ef];
-    ke[u] = rec[G_QK + (64 + ei + u) * 128 + f0 + ef];
-    kd[u] = rec[G_KED + (ei + u) * 128 + f0 + ef];
+    qe[u] = rec[G_QK + rec_off(ei + u, f0 + ef, 128)];
+    ke[u] = rec[G_QK + rec_off(64 + ei + u, f0 + ef, 128)];
+    kd[u] = rec[G_KED + rec_off(ei + u, f0 + ef, 128)];
   }
   {  // inputs of this channel quarter (4 channels per item) and the C x C adjoints; loads first
     float4 gv[2], dp[4], da[4];
@@ -508,8 +508,8 @@ __global__ void __launch_bounds__(NTHREADS, 2) kda_bwd_assemble_kernel(BwdArgs a
 #pragma unroll
     for (int m = 0; m < 4; ++m) {  // row i of [dP; dA], four columns j per item
       const int idx = tid + m * NTHREADS, i = idx >> 4, j4 = (idx & 15) * 4;
-      dp[m] = *reinterpret_cast<const float4*>(rec + G_PA + i * 64 + j4);
-      da[m] = *reinterpret_cast<const float4*>(rec + G_PA + (64 + i) * 64 + j4);
+      dp[m] = *reinterpret_cast<const float4*>(rec + G_PA + rec_off(i, j4, 64));
+      da[m] = *reinterpret_cast<const float4*>(rec + G_PA + rec_off(64 + i, j4, 64));
     }
     if (tid < C) sBeta[tid] = (tid < L) ? a.beta[((size_t)b * T + t0 + tid) * a.HV + hv] : 0.f;
 #pragma unroll

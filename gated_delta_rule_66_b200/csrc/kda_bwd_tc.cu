@@ -506,29 +506,44 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
     if (!wait_mma(bar, phase)) { failed = true; break; }
 
     // ---------------------------------------------------------------- record
-    {  // rows (TMEM lanes) row-major: each lane stores its 32 consecutive columns as 16-byte pieces
+    {  // the record staged in shared memory (now free) in its global layout, then bulk-stored
+      float* st = reinterpret_cast<float*>(sm);  // [dP; dA] | [dQE; dKE'] | dKEd
+      constexpr int S_PA = 0, S_QK = 8192, S_KED = 24576;
+      static_assert(4 * (S_KED + 8192) <= OP_DO, "record staging below [dO; -dR]");
       float v[32];
       tmem_ld32(tm + lo + TM_PA + hcol * 32, v);
-      float4* dst = reinterpret_cast<float4*>(rec + G_PA + Lr * 64 + hcol * 32);
 #pragma unroll
-      for (int q4 = 0; q4 < 8; ++q4) dst[q4] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+      for (int q4 = 0; q4 < 8; ++q4)
+        *reinterpret_cast<float4*>(st + S_PA + rec_off(Lr, hcol * 32 + 4 * q4, 64)) =
+            make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
       for (int cb = 0; cb < 2; ++cb) {
         const int f0 = hcol * 64 + cb * 32;
         tmem_ld32(tm + lo + TM_QK + f0, v);
-        dst = reinterpret_cast<float4*>(rec + G_QK + Lr * 128 + f0);
 #pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) dst[q4] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+        for (int q4 = 0; q4 < 8; ++q4)
+          *reinterpret_cast<float4*>(st + S_QK + rec_off(Lr, f0 + 4 * q4, 128)) =
+              make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
         tmem_ld32(tm + lo + TM_KED + f0, v);
         if (lane < 16) {
           const int r = cx.sub * 16 + lane;  // M = 64 accumulator layout
-          dst = reinterpret_cast<float4*>(rec + G_KED + r * 128 + f0);
 #pragma unroll
           for (int q4 = 0; q4 < 8; ++q4)
-            dst[q4] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+            *reinterpret_cast<float4*>(st + S_KED + rec_off(r, f0 + 4 * q4, 128)) =
+                make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
         }
       }
-      if (tid < C) rec[G_DBR + tid] = sDbR[tid];
-      if (tid < KD) rec[G_DEL + tid] = sDEl[tid];
+      fence_async_smem();
+      __syncthreads();
+      if (tid == 0) {
+        bulk_s2g(rec + G_PA, sb + 4 * S_PA, 32768);
+        bulk_s2g(rec + G_QK, sb + 4 * S_QK, 32768);
+        bulk_s2g(rec + G_QK + 8192, sb + 4 * S_QK + 32768, 32768);
+        bulk_s2g(rec + G_KED, sb + 4 * S_KED, 32768);
+        bulk_s2g(rec + G_DBR, sb + S_EMID, 256);
+        bulk_s2g(rec + G_DEL, sb + S_EL, 512);
+        bulk_commit();
+        bulk_wait_read();
+      }
     }
   } while (false);
 

@@ -10,9 +10,10 @@ constexpr int FWD_CHUNK = 32;    // chunk length of the chunked kernels
 constexpr int FWD_VBLOCK = 32;   // V columns per CTA in the chunked kernels
 
 // Per-(b, hv, 64-step chunk) record of the tensor-core backward (floats),
-// row-major: [dP; dA] as [i'][j] (128 x 64, i' < 64 dP), [dQE; dKE'] as
-// [i'][f] (128 x 128, i' < 64 dQE), dKEd as [i][f] (64 x 128), dbeta_R [64],
-// dEl [128] (G_AH unused).
+// row-major with the 16-byte pieces of row r XOR-swizzled by r % 8 (element
+// (r, c) of a row of n floats at rec_off(r, c, n)): [dP; dA] as [i'][j]
+// (128 x 64, i' < 64 dP), [dQE; dKE'] as [i'][f] (128 x 128, i' < 64 dQE),
+// dKEd as [i][f] (64 x 128); then dbeta_R [64], dEl [128] (G_AH unused).
 // Per-(b, hv, 64-step chunk) interaction record that the tensor-core forward
 // stores with a workspace (floats).  Three 64 x 64 tf32 operand images in the
 // K-major canonical layout of the tensor-core kernels (element (r, k) at
@@ -39,6 +40,10 @@ constexpr unsigned FWI_W = 0, FWI_QE = 36864, FWI_KEDT = 69632, FWI_P = 102400, 
 constexpr unsigned FWI_A_BYTES = FWI_KEDT, FWI_B_BYTES = FWI_U0 - FWI_KEDT;
 constexpr int G_AH = 0, G_PA = 4096, G_QK = 12288, G_KED = 28672, G_DBR = 36864, G_DEL = 36928,
               GREC = 37120;
+
+__host__ __device__ constexpr int rec_off(int r, int c, int n) {
+  return r * n + ((((c >> 2) ^ (r & 7))) << 2) + (c & 3);
+}
 
 struct FwdArgs {
   const void *q, *k, *v;
