@@ -70,7 +70,9 @@ def algorithmic_bytes(w, kind):
     if kind == "fwd":
         return fwd_in + fwd_out + s0
     # backward: reads the forward inputs and dO, writes dq, dk, dv, dg, dbeta, dS0
-    bwd = fwd_in + B * T * HV * V * e + B * T * (2 * H * K * e + HV * V * e + HV * K * 4 + HV * 4) + state
+    bwd = fwd_in + s0 + B * T * HV * V * e + B * T * (2 * H * K * e + HV * V * e + HV * K * 4 + HV * 4) + state
+    if kind == "bwd":
+        return bwd
     return fwd_in + fwd_out + s0 + bwd
 
 
@@ -302,14 +304,21 @@ def roofline_for(res, w, peaks):
     if w.path == "fwd":
         byts = algorithmic_bytes(w, "fwd")
         t = res["calls"]["kernel_ms"] * 1e-3
-        return {"bound": "hbm", "kernel": "kda_fwd_tc_kernel" if w.K == 128 and w.dtype == "bf16"
-                else "kda_fwd_chunk_kernel", "achieved": byts / t / 1e9,
+        return {"bound": "hbm", "kernel": "kda_fwd (kda_fwd_prep_tc_kernel + kda_fwd_seq_tc_kernel)"
+                if w.K == 128 and w.dtype == "bf16" else "kda_fwd_chunk_kernel", "achieved": byts / t / 1e9,
                 "peak": hbm, "unit": "GB/s", "frac": byts / t / 1e9 / hbm, "algorithmic_bytes": byts}
-    byts = algorithmic_bytes(w, "fwd")
-    t = res["calls"]["fwd_ms"] * 1e-3
-    return {"bound": "hbm", "kernel": "kda_fwd_tc_kernel (state-storing forward of the step)",
+    # the step's dominant part is the backward call (three kernels: state gradients,
+    # gradient products, assembly); its algorithmic bytes are the backward's own I/O
+    byts = algorithmic_bytes(w, "bwd")
+    t = res["calls"]["bwd_ms"] * 1e-3
+    fb = algorithmic_bytes(w, "fwd")
+    tf = res["calls"]["fwd_ms"] * 1e-3
+    return {"bound": "hbm", "kernel": "kda_bwd (kda_bwd_dstate_tc_kernel + kda_bwd_grads_tc_kernel + "
+                                      "kda_bwd_assemble_kernel, one call)",
             "achieved": byts / t / 1e9, "peak": hbm, "unit": "GB/s", "frac": byts / t / 1e9 / hbm,
-            "algorithmic_bytes": byts}
+            "algorithmic_bytes": byts,
+            "fwd": {"kernel": "kda_fwd (kda_fwd_prep_tc_kernel + kda_fwd_seq_tc_kernel, one call)",
+                    "achieved": fb / tf / 1e9, "frac": fb / tf / 1e9 / hbm, "algorithmic_bytes": fb}}
 
 
 def run_gpu(args):
@@ -367,7 +376,8 @@ def run_gpu(args):
                                + ("" if not args.shrink else " [reduced for a profiler capture]"),
                    "global_batch": w.B * world, "seq_len": w.T, "parallelism": f"replicas x{world}",
                    "l2": head["l2"]},
-        "roofline": dict(head["roofline"], traffic=recorded_traffic(head["roofline"]["kernel"].split()[0], HEADLINE)),
+        "roofline": dict({k: v for k, v in head["roofline"].items() if k != "fwd"},
+                         traffic=recorded_traffic(head["roofline"]["kernel"].split()[0], HEADLINE)),
         "e2e": {"value": head["e2e_tokens_per_s"], "unit": "tokens/s",
                 "h2d_bytes_per_step": head["h2d_bytes"], "d2h_bytes_per_step": head["d2h_bytes"]},
         "gpu_launches": head["launches_per_step"] * args.steps,

@@ -373,10 +373,10 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_prep_tc_kernel(FwdArgs a) {
 #pragma unroll
       for (int jj = 0; jj < 32; ++jj) st_tf32(sm, R_WOP + kmaj_pad(hcol * 32 + jj, Lr, 128), v[jj]);
     }
-    {  // U0^T (lane n) as [i][n]
+    {  // U0^T (lane n) as [i][n], staged over (diag(beta) K o e^c)^T (consumed by the W product)
       float u[32];
       tmem_ld32(tm + lo + TM_U + hcol * 32, u);
-      float* dst = reinterpret_cast<float*>(img + FWI_U0);
+      float* dst = reinterpret_cast<float*>(sm + OP_BKET);
 #pragma unroll
       for (int jj = 0; jj < 32; ++jj) dst[(hcol * 32 + jj) * VD + Lr] = u[jj];
     }
@@ -386,6 +386,7 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_prep_tc_kernel(FwdArgs a) {
     if (tid == 0) {
       bulk_s2g(img + FWI_W, sb + R_WOP, FWI_QE - FWI_W);
       bulk_s2g(img + FWI_P, sb + R_P, FWI_EL - FWI_P);
+      bulk_s2g(img + FWI_U0, sb + OP_BKET, FWI_BYTES - FWI_U0);
       bulk_commit();
     }
   }
