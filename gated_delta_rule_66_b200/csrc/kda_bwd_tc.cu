@@ -89,11 +89,6 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_dstate_tc_kernel(BwdArgs a) {
     const int t0 = ch * C, L = min(C, T - t0);
     const float* irec = a.inter + (head * NT + ch) * INTER_REC;  // P^T, T^T of this chunk (forward)
     load_raw_issue(cx, qg, kg, dog, a.g, a.beta, b, T, t0, L, a.H, a.HV, h, hv);
-    if (ch > 0) {  // the next chunk down: raw rows and record images into L2
-      prefetch_chunk(cx, qg, kg, dog, a.g, b, T, t0 - C, C, a.H, a.HV, h, hv);
-      if (tid == 64) prefetch_l2(irec - INTER_REC, 16384);
-      if (tid == 192) prefetch_l2(irec - INTER_REC + INTER_TT, 16384);
-    }
     if (!load_raw_wait(cx)) { failed = true; break; }
     cumsum_span(cx);
 

@@ -47,6 +47,7 @@ constexpr uint32_t TM_S = 0, TM_X = 128, TM_O = 192, TM_U = 256, TM_W = 320, TM_
 // bulk stores of the chunk images of Q~ o e^c, (K o e^{c_last-c})^T and
 // e^{c_last} as soon as they are built.
 // Returns false, block-uniformly, if a tensor-core wait ran out.
+template <int NTHR>
 __device__ __forceinline__ bool fwd_chunk_head(const tcc::Ctx& cx, const FwdArgs& a, int b, int hv, int h,
                                                int ch, bool prefetch_next, float* irec,
                                                unsigned char* img, uint64_t* bar, uint32_t& phase) {
@@ -62,19 +63,19 @@ __device__ __forceinline__ bool fwd_chunk_head(const tcc::Ctx& cx, const FwdArgs
   const float* sBeta = cx.beta();
   float* sEl = reinterpret_cast<float*>(sm + S_EL);
   const float* sC = cx.c();
-  load_raw_issue(cx, qg, kg, vg, a.g, a.beta, b, T, t0, L, a.H, a.HV, h, hv);
+  load_raw_issue<NTHR>(cx, qg, kg, vg, a.g, a.beta, b, T, t0, L, a.H, a.HV, h, hv);
   if (prefetch_next && ch + 1 < NT)
     prefetch_chunk(cx, qg, kg, vg, a.g, b, T, t0 + C, min(C, T - t0 - C), a.H, a.HV, h, hv);
   if (!load_raw_wait(cx)) return false;
   const bool wide = cumsum_span(cx);
-  build_op1_and_issue(cx, a.scale, tm + TM_APA, tm + TM_APB, bar);
+  build_op1_and_issue<NTHR>(cx, a.scale, tm + TM_APA, tm + TM_APB, bar);
   if (!wait_mma(bar, phase)) return false;
 
   // ---------------------------------------------------------------- state-product operands
   {  // Q~ o e^c as [i][f]: thread items of 4 channels, 16-byte stores
-    const int fq = item_f(cx);
-    for (int m = 0; m < 8; ++m) {
-      const int i = item_row(cx, m);
+    const int fq = item_f<NTHR>(cx);
+    for (int m = 0; m < 2048 / NTHR; ++m) {
+      const int i = item_row<NTHR>(cx, m);
       const float4 c4 = ld4(sC + i * LDCF + fq);
       float qf[4];
       bf16x4(sm + RAW_Q + raw_off(i, fq), qf);
@@ -86,8 +87,8 @@ __device__ __forceinline__ bool fwd_chunk_head(const tcc::Ctx& cx, const FwdArgs
     const int f = tid & 127;
     const float c63 = sC[63 * LDCF + f];
 
-    for (int m = 0; m < 8; ++m) {
-      const int i0 = ((tid >> 7) + 2 * m) * 4;
+    for (int m = 0; m < 2048 / NTHR; ++m) {
+      const int i0 = ((tid >> 7) + (NTHR / 128) * m) * 4;
       float bke[4], ked[4], bv[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
@@ -108,18 +109,18 @@ __device__ __forceinline__ bool fwd_chunk_head(const tcc::Ctx& cx, const FwdArgs
   if (wide) pairwise_compute(cx, a.scale, pw);
   if (img) fence_async_smem();
   __syncthreads();  // raw inputs consumed; the raw region is reused below
-  if (img && tid == 0) {
-    bulk_s2g(img + FWI_QE, sb + OP_QE, FWI_KEDT - FWI_QE);
-    bulk_s2g(img + FWI_KEDT, sb + OP_KEDT, FWI_P - FWI_KEDT);
-    bulk_s2g(img + FWI_EL, sb + S_EL, FWI_U0 - FWI_EL);
+  if (img && (tid & 31) == 0 && tid < 96) {  // one bulk store per issuing warp
+    if (tid == 0) bulk_s2g(img + FWI_QE, sb + OP_QE, FWI_KEDT - FWI_QE);
+    if (tid == 32) bulk_s2g(img + FWI_KEDT, sb + OP_KEDT, FWI_P - FWI_KEDT);
+    if (tid == 64) bulk_s2g(img + FWI_EL, sb + S_EL, FWI_U0 - FWI_EL);
     bulk_commit();
   }
 
-  readout_ap(cx, tm + TM_APA, tm + TM_APB, wide, pw, irec);
-  invert(cx);
+  readout_ap<NTHR>(cx, tm + TM_APA, tm + TM_APB, wide, pw, irec);
+  invert<NTHR>(cx);
   {  // T as the operand image (rows i, K = j); with a record also its T, T^T images and Ah
     const float* tr = reinterpret_cast<const float*>(sm + R_TROW);
-    for (int x = tid; x < C * 16; x += NTH) {  // 16-byte piece x of the image: x * 16 = kmaj(i, j4, 64)
+    for (int x = tid; x < C * 16; x += NTHR) {  // 16-byte piece x of the image: x * 16 = kmaj(i, j4, 64)
       const int i = ((x >> 7) << 3) | (x & 7), j4 = ((x >> 3) & 15) * 4;
       const float* p = tr + i * 65 + j4;
       const uint4 t = make_uint4(tf32_rna(p[0]), tf32_rna(p[1]), tf32_rna(p[2]), tf32_rna(p[3]));
@@ -133,7 +134,7 @@ __device__ __forceinline__ bool fwd_chunk_head(const tcc::Ctx& cx, const FwdArgs
     }
     if (irec) {
       const float* ah = reinterpret_cast<const float*>(sm + R_AH);
-      for (int x = tid; x < C * C; x += NTH) irec[INTER_AH + x] = ah[(x >> 6) * 65 + (x & 63)];
+      for (int x = tid; x < C * C; x += NTHR) irec[INTER_AH + x] = ah[(x >> 6) * 65 + (x & 63)];
     }
   }
   fence_async_smem();
@@ -209,7 +210,7 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_tc_kernel(FwdArgs a) {
   for (int ch = 0; ch < NT; ++ch) {
     const int t0 = ch * C, L = min(C, T - t0);
     float* irec = a.inter ? a.inter + (head * NT + ch) * INTER_REC : nullptr;
-    if (!fwd_chunk_head(cx, a, b, hv, h, ch, true, irec, nullptr, bar, phase)) {
+    if (!fwd_chunk_head<NTH>(cx, a, b, hv, h, ch, true, irec, nullptr, bar, phase)) {
       failed = true;
       break;
     }
@@ -317,7 +318,9 @@ bool fwd_tc_eligible(const FwdArgs& a, int dtype) {
 //   X^T = M^T W^T,  O^T = M^T (Q~ o e^c)^T,  U^T = U0^T - X^T,
 //   M'^T = M^T diag(e^{c_last}) + U^T (K o e^{c_last-c}),  O^T += U^T P^T.
 // ============================================================================
-__global__ void __launch_bounds__(256, 1) kda_fwd_prep_tc_kernel(FwdArgs a) {
+constexpr int PREP_NT = 512;  // 16 warps: the chunk work is latency-bound, more warps hide it
+
+__global__ void __launch_bounds__(PREP_NT, 1) kda_fwd_prep_tc_kernel(FwdArgs a) {
   using namespace tcf;
   using namespace tc;
   extern __shared__ __align__(1024) unsigned char sm[];
@@ -347,50 +350,45 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_prep_tc_kernel(FwdArgs a) {
   cx.tm = tm;
   uint32_t phase = 0;
   bool failed = false;
-  // persistent: this CTA takes items blockIdx.x, + gridDim.x, ...; each item's
-  // raw rows are brought into L2 while the previous item is processed
+  // persistent: this CTA takes items blockIdx.x, + gridDim.x, ...  (An L2
+  // prefetch of the next item's rows measured slower: it queues behind the
+  // image stores.)
   for (int item = blockIdx.x; item < items; item += gridDim.x) {
     const int ch = item % NT, hv = (item / NT) % a.HV, b = item / (NT * a.HV), h = hv / G;
     const size_t head = (size_t)b * a.HV + hv;
-    const int nxt = item + gridDim.x;
-    if (nxt < items) {
-      const int nch = nxt % NT, nhv = (nxt / NT) % a.HV, nb = nxt / (NT * a.HV);
-      prefetch_chunk(cx, static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),
-                     static_cast<const __nv_bfloat16*>(a.v), a.g, nb, a.T, nch * C, min(C, a.T - nch * C), a.H,
-                     a.HV, nhv / G, nhv);
-    }
-    if (tid == 0) bulk_wait_read();  // the previous item's image stores have left shared memory
+    if ((tid & 31) == 0 && tid < 96) bulk_wait_read();  // the previous item's image stores have left smem
     __syncthreads();
     float* irec = a.inter ? a.inter + (head * NT + ch) * INTER_REC : nullptr;
     unsigned char* img = a.img + (head * NT + ch) * (size_t)FWI_BYTES;
-    if (!fwd_chunk_head(cx, a, b, hv, h, ch, false, irec, img, bar, phase)) {
+    if (!fwd_chunk_head<PREP_NT>(cx, a, b, hv, h, ch, false, irec, img, bar, phase)) {
       failed = true;
       break;
     }
+    constexpr int CW = 64 / (PREP_NT / 128);  // columns of W^T / U0^T per warp group
     {  // W (rows i, K = f) padded, from W^T in TMEM (lane f)
-      float v[32];
-      tmem_ld32(tm + lo + TM_W + hcol * 32, v);
+      float v[CW];
+      tmem_ldn<CW>(tm + lo + TM_W + hcol * CW, v);
 #pragma unroll
-      for (int jj = 0; jj < 32; ++jj) st_tf32(sm, R_WOP + kmaj_pad(hcol * 32 + jj, Lr, 128), v[jj]);
+      for (int jj = 0; jj < CW; ++jj) st_tf32(sm, R_WOP + kmaj_pad(hcol * CW + jj, Lr, 128), v[jj]);
     }
     {  // U0^T (lane n) as [i][n], staged over (diag(beta) K o e^c)^T (consumed by the W product)
-      float u[32];
-      tmem_ld32(tm + lo + TM_U + hcol * 32, u);
+      float u[CW];
+      tmem_ldn<CW>(tm + lo + TM_U + hcol * CW, u);
       float* dst = reinterpret_cast<float*>(sm + OP_BKET);
 #pragma unroll
-      for (int jj = 0; jj < 32; ++jj) dst[(hcol * 32 + jj) * VD + Lr] = u[jj];
+      for (int jj = 0; jj < CW; ++jj) dst[(hcol * CW + jj) * VD + Lr] = u[jj];
     }
     fence_async_smem();
     fence_before();
     __syncthreads();
-    if (tid == 0) {
-      bulk_s2g(img + FWI_W, sb + R_WOP, FWI_QE - FWI_W);
-      bulk_s2g(img + FWI_P, sb + R_P, FWI_EL - FWI_P);
-      bulk_s2g(img + FWI_U0, sb + OP_BKET, FWI_BYTES - FWI_U0);
+    if ((tid & 31) == 0 && tid < 96) {
+      if (tid == 0) bulk_s2g(img + FWI_W, sb + R_WOP, FWI_QE - FWI_W);
+      if (tid == 32) bulk_s2g(img + FWI_P, sb + R_P, FWI_EL - FWI_P);
+      if (tid == 64) bulk_s2g(img + FWI_U0, sb + OP_BKET, FWI_BYTES - FWI_U0);
       bulk_commit();
     }
   }
-  if (tid == 0) bulk_wait_read();
+  if ((tid & 31) == 0 && tid < 96) bulk_wait_read();
   fence_before();
   __syncthreads();
   if (cx.warp == 0) tmem_dealloc(tm, 512);
@@ -580,7 +578,7 @@ int launch_fwd_tc(const FwdArgs& a, cudaStream_t stream) {
     const int items = (a.T + tcc::C - 1) / tcc::C * a.HV * a.B;
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    kda_fwd_prep_tc_kernel<<<min(items, sms), tcc::NTH, tcc::SMEM_BYTES, stream>>>(a);
+    kda_fwd_prep_tc_kernel<<<min(items, sms), PREP_NT, tcc::SMEM_BYTES, stream>>>(a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return set_cuda_error("kda_fwd: tensor-core chunk launch", e);
     kda_fwd_seq_tc_kernel<<<dim3(a.HV, a.B), tcc::NTH, tcs::SQ_BYTES, stream>>>(a);

@@ -83,11 +83,12 @@ __device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast
 // zero.  Issues the copies only; load_raw_wait completes them.  (16-byte
 // cp.async per thread: measured faster here than per-row bulk copies issued
 // by one warp.)
+template <int NT = NTH>
 __device__ __forceinline__ void load_raw_issue(const Ctx& c, const __nv_bfloat16* q, const __nv_bfloat16* k,
                                                const __nv_bfloat16* x, const float* g, const float* beta,
                                                int b, int T, int t0, int L, int H, int HV, int h, int hv) {
   using namespace tc;
-  for (int e = c.tid; e < C * 16; e += NTH) {
+  for (int e = c.tid; e < C * 16; e += NT) {
     const int i = e >> 4, vec = e & 15;
     const bool ok = i < L;
     const size_t t = (size_t)b * T + t0 + (ok ? i : 0);  // row 0 of the chunk is always valid
@@ -96,7 +97,7 @@ __device__ __forceinline__ void load_raw_issue(const Ctx& c, const __nv_bfloat16
     cp_async16(c.sb + RAW_K + d, k + (t * H + h) * KD + vec * 8, ok);
     cp_async16(c.sb + RAW_X + d, x + (t * HV + hv) * VD + vec * 8, ok);
   }
-  for (int e = c.tid; e < C * 32; e += NTH) {
+  for (int e = c.tid; e < C * 32; e += NT) {
     const int i = e >> 5, vec = e & 31;
     const bool ok = i < L;
     const size_t t = (size_t)b * T + t0 + (ok ? i : 0);
@@ -118,7 +119,7 @@ __device__ __forceinline__ void prefetch_chunk(const Ctx& c, const __nv_bfloat16
                                                const __nv_bfloat16* x, const float* g, int b, int T, int t0,
                                                int L, int H, int HV, int h, int hv) {
   const int i = c.tid & 63, which = c.tid >> 6;
-  if (i >= L) return;
+  if (i >= L || which > 3) return;
   const size_t t = (size_t)b * T + t0 + i;
   if (which == 0) tc::prefetch_l2(q + (t * H + h) * KD, KD * 2);
   else if (which == 1) tc::prefetch_l2(k + (t * H + h) * KD, KD * 2);
@@ -128,9 +129,10 @@ __device__ __forceinline__ void prefetch_chunk(const Ctx& c, const __nv_bfloat16
 
 // Asynchronous copy of one 64 x 64 operand image of an interaction record
 // (16 KB) into shared memory at `dst`; completes with cp_async_wait_all.
+template <int NT = NTH>
 __device__ __forceinline__ void copy_image(const Ctx& c, uint32_t dst, const float* src) {
 #pragma unroll
-  for (int e = c.tid; e < 1024; e += NTH) tc::cp_async16(c.sb + dst + e * 16, src + e * 4, true);
+  for (int e = c.tid; e < 1024; e += NT) tc::cp_async16(c.sb + dst + e * 16, src + e * 4, true);
 }
 
 // float index of element (r, k) in a 64 x 64 record image
@@ -139,22 +141,27 @@ __device__ __forceinline__ int img(int r, int k) { return (int)(tc::kmaj(r, k, 6
 // In-chunk cumulative decay (natural log summed, stored times log2(e)).
 // Returns, block-uniformly, whether some half's decay from its middle row to
 // either end exceeds 80 (the split exponents would then leave fp32 range).
+// (The first 256 threads do the sums, two row halves per channel.)
 __device__ __forceinline__ bool cumsum_span(const Ctx& c) {
   float* sC = c.c();
   float* sCarry = reinterpret_cast<float*>(c.sm + S_CARRY);
   const int f = c.tid & 127, hh = c.tid >> 7;
   float v[32];
   float run = 0.f;
+  if (c.tid < 256) {
 #pragma unroll
-  for (int r = 0; r < 32; ++r) {
-    run += sC[(hh * 32 + r) * LDCF + f];
-    v[r] = run;
+    for (int r = 0; r < 32; ++r) {
+      run += sC[(hh * 32 + r) * LDCF + f];
+      v[r] = run;
+    }
+    if (hh == 0) sCarry[f] = run;
   }
-  if (hh == 0) sCarry[f] = run;
   __syncthreads();
-  const float carry = hh ? sCarry[f] : 0.f;
+  if (c.tid < 256) {
+    const float carry = hh ? sCarry[f] : 0.f;
 #pragma unroll
-  for (int r = 0; r < 32; ++r) sC[(hh * 32 + r) * LDCF + f] = (v[r] + carry) * LOG2E;
+    for (int r = 0; r < 32; ++r) sC[(hh * 32 + r) * LDCF + f] = (v[r] + carry) * LOG2E;
+  }
   __syncthreads();
   bool w = false;
   if (c.tid < KD) {
@@ -167,22 +174,26 @@ __device__ __forceinline__ bool cumsum_span(const Ctx& c) {
   return __syncthreads_or(w);
 }
 
-// Item mapping of the element-wise operand builders: thread t owns key
-// channels 4*((t>>3)&31) .. +3 and rows m*8 + (t&7), m = 0..7.
-__device__ __forceinline__ int item_f(const Ctx& c) { return ((c.tid >> 3) & 31) * 4; }
-__device__ __forceinline__ int item_row(const Ctx& c, int m) { return m * 8 + (c.tid & 7); }
+// Item mapping of the element-wise operand builders for NT threads (R = NT / 32
+// rows per round): thread t owns key channels 4*((t/R)&31) .. +3 and rows
+// m*R + t%R, m = 0 .. 64/R - 1 (eight consecutive lanes hold eight rows).
+template <int NT = NTH>
+__device__ __forceinline__ int item_f(const Ctx& c) { return ((c.tid / (NT / 32)) & 31) * 4; }
+template <int NT = NTH>
+__device__ __forceinline__ int item_row(const Ctx& c, int m) { return m * (NT / 32) + c.tid % (NT / 32); }
 
 // Interaction operands into the operand region, then the two products on
 // the tensor cores (issued by thread 0, completion on `bar`).
+template <int NT = NTH>
 __device__ __forceinline__ void build_op1_and_issue(const Ctx& c, float scale, uint32_t tm_apa,
                                                     uint32_t tm_apb, uint64_t* bar) {
   using namespace tc;
   const float* sC = c.c();
-  const int fq = item_f(c);
+  const int fq = item_f<NT>(c);
   const float4 r15 = ld4(sC + 15 * LDCF + fq), r47 = ld4(sC + 47 * LDCF + fq), r31 = ld4(sC + 31 * LDCF + fq);
   const float c31[4] = {r31.x, r31.y, r31.z, r31.w};
-  for (int m = 0; m < 8; ++m) {
-    const int i = item_row(c, m);
+  for (int m = 0; m < 2048 / NT; ++m) {
+    const int i = item_row<NT>(c, m);
     const float4 c4 = ld4(sC + i * LDCF + fq);
     const float cc[4] = {c4.x, c4.y, c4.z, c4.w};
     float kf[4], qf[4];
@@ -244,7 +255,11 @@ struct Pairwise {
 };
 __device__ __forceinline__ void pairwise_compute(const Ctx& c, float scale, Pairwise& pw) {
   const float* sC = c.c();
-  pw.kind = c.tid >> 7;
+  pw.kind = c.tid < 256 ? c.tid >> 7 : -1;  // the first 256 threads
+  if (pw.kind < 0) {
+    pw.i = pw.j0 = 0;
+    return;
+  }
   pw.i = (c.tid >> 1) & 63;
   pw.j0 = (pw.i & 32) + (c.tid & 1) * 16;
   const unsigned char* xi = c.sm + (pw.kind ? RAW_Q : RAW_K);
@@ -269,49 +284,53 @@ __device__ __forceinline__ uint32_t p_off(int i, int j) { return R_P + tc::kmaj(
 // Reads Ah (row-major, stride 65, at R_AH) and P (tf32 operand at R_P) out of
 // the two interaction products; the raw region must be free.  With `pt` it
 // also stores the P^T image of the interaction record.  Ends with a barrier.
+template <int NT = NTH>
 __device__ __forceinline__ void readout_ap(const Ctx& c, uint32_t tm_apa, uint32_t tm_apb, bool wide,
                                            const Pairwise& pw, float* pt = nullptr) {
   using namespace tc;
+  constexpr int CW = 64 / (NT / 128), CB = 32 / (NT / 128);  // columns per warp group of [Ah; P], of b
   float* sAh = reinterpret_cast<float*>(c.sm + R_AH);
   {
-    float v[32];
-    tmem_ld32(tm_apa + c.lo + c.hcol * 32, v);
+    float v[CW];
+    tmem_ldn<CW>(tm_apa + c.lo + c.hcol * CW, v);
     const bool isA = c.Lr < 64;
     const int i = isA ? c.Lr : c.Lr - 64;
     if (isA) {
 #pragma unroll
-      for (int jj = 0; jj < 32; ++jj) {
-        const int j = c.hcol * 32 + jj;
+      for (int jj = 0; jj < CW; ++jj) {
+        const int j = c.hcol * CW + jj;
         const bool same = (i >> 5) == (j >> 5);
         if (!same && i >= 32) continue;  // lower-left block comes from product b
         sAh[i * 65 + j] = (same && j < i) ? v[jj] : 0.f;
       }
-    } else if (!(i >= 32 && c.hcol == 0)) {  // P rows: four columns per 16-byte store
+    } else {  // P rows: four columns per 16-byte store
 #pragma unroll
-      for (int j4 = 0; j4 < 32; j4 += 4) {
+      for (int j4 = 0; j4 < CW; j4 += 4) {
+        const int jb = c.hcol * CW + j4;
+        if (i >= 32 && jb < 32) continue;  // lower-left block comes from product b
         float w[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const int j = c.hcol * 32 + j4 + u;
+          const int j = jb + u;
           w[u] = ((i >> 5) == (j >> 5) && j <= i) ? v[j4 + u] : 0.f;
           if (pt) pt[img(j, i)] = __uint_as_float(tf32_rna(w[u]));
         }
-        st_tf32x4(c.sm, p_off(i, c.hcol * 32 + j4), w[0], w[1], w[2], w[3]);
+        st_tf32x4(c.sm, p_off(i, jb), w[0], w[1], w[2], w[3]);
       }
     }
   }
   {
-    float v[16];
-    tmem_ld16(tm_apb + c.lo + c.hcol * 16, v);
+    float v[CB];
+    tmem_ldn<CB>(tm_apb + c.lo + c.hcol * CB, v);
     if (c.lane < 16) {
       const int r = c.sub * 16 + c.lane;  // row of the 64-row product (M = 64 accumulator layout)
       if (r < 32) {
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj) sAh[(32 + r) * 65 + c.hcol * 16 + jj] = v[jj];
+        for (int jj = 0; jj < CB; ++jj) sAh[(32 + r) * 65 + c.hcol * CB + jj] = v[jj];
       } else {
 #pragma unroll
-        for (int j4 = 0; j4 < 16; j4 += 4) {
-          const int j = c.hcol * 16 + j4;
+        for (int j4 = 0; j4 < CB; j4 += 4) {
+          const int j = c.hcol * CB + j4;
           st_tf32x4(c.sm, p_off(r, j), v[j4], v[j4 + 1], v[j4 + 2], v[j4 + 3]);
           if (pt)
 #pragma unroll
@@ -340,6 +359,7 @@ __device__ __forceinline__ void readout_ap(const Ctx& c, uint32_t tm_apa, uint32
 // registers; the blocks below follow in three levels of block substitution,
 // T_IJ = -T_II sum_{J<=L<I} A_IL T_LJ (level = block distance I - J), one
 // warp per block, as 3xTF32 warp MMAs (fp32-accurate).
+template <int NT = NTH>
 __device__ __forceinline__ void invert(const Ctx& c) {
   constexpr int LD = 65;
   const float* sAh = reinterpret_cast<const float*>(c.sm + R_AH);
@@ -347,7 +367,7 @@ __device__ __forceinline__ void invert(const Ctx& c) {
   float* sW = reinterpret_cast<float*>(c.sm + R_SW);  // one 16 x 16 scratch per warp (3 warps)
   const float* sB = c.beta();
   const int tid = c.tid;
-  for (int x = tid; x < 6 * 256; x += NTH) {  // strictly upper blocks
+  for (int x = tid; x < 6 * 256; x += NT) {  // strictly upper blocks
     const int blk = x >> 8, r = (x >> 4) & 15, col = x & 15;
     const int I = blk < 3 ? 0 : (blk < 5 ? 1 : 2), J = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
     sT[(16 * I + r) * LD + 16 * J + col] = 0.f;
