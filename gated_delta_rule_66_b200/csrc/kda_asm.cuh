@@ -1,0 +1,231 @@
+// Assembly of dq, dk, dg and dbeta for one quarter of the key channels of a
+// 64-step chunk from the per-chunk gradient record, with 3xTF32 warp MMAs for
+// the interaction terms (any decay span: pair by pair where the split
+// exponents would leave fp32 range).
+#pragma once
+
+#include "kda_chunk.cuh"
+#include "kda_internal.h"
+
+namespace kda {
+
+// Assembles dq, dk, dg and dbeta of one 64-step chunk from the record that
+// kda_bwd_grads_tc_kernel wrote (Ah, [dP; dA], [dQE; dKE'], dKEd, dbeta_R,
+// dEl): dbeta = dbeta_R + sum_j dA_ij Ah_ij; dq~ = dQE o e^c; dk = dKE o e^c +
+// dKEd o e^{c_last-c}; dc = (dQE o q~ + dKE o k) o e^c - dKEd o k o e^{c_last-c};
+// then the interaction terms (factored_terms) and dg = reverse cumsum of dc.
+// Everything here is independent across key channels, so one CTA handles one
+// (b, hv, chunk, quarter of the 128 key channels); two CTAs fit on an SM.
+// Row strides (words): LDK = 40 (8 mod 32) puts the warp-MMA fragment loads of
+// K, Q and c (lanes: row t, channel g) in 32 distinct banks; LDC = 68 (4 mod
+// 32) does the same for the row-term fragments of dP and dA (lanes: row g,
+// column t).  Accesses with the lanes along a row are conflict-free anyway.
+struct AsmSmem {
+  static constexpr int C = 64, KQ = 32, LDK = 40, LDC = 68;
+  static constexpr int oK = 0, oQ = oK + C * LDK, oC = oQ + C * LDK, oDq = oC + C * LDK, oDk = oDq + C * LDK,
+                       oDc = oDk + C * LDK, oE1 = oDc + C * LDK, oE2o = oE1 + C * LDK, oE2d = oE2o + BS * LDK,
+                       odA = oE2d + BS * LDK, odP = odA + C * LDC, oBeta = odP + C * LDC, oSeg = oBeta + C,
+                       oLast = oSeg + 8 * KQ, oFlag = oLast + KQ, total = oFlag + 4;
+  static constexpr size_t bytes = (size_t)total * sizeof(float);
+};
+
+// Inclusive (forward) or reverse cumulative sum over the C = 64 rows of each
+// of the KQ = 32 columns of a [64][LDK] array, by 8 segments of 8 rows
+// (256 threads; seg is 8 x KQ scratch; `base` is added to every element of a
+// reverse sum).  Ends with a barrier.
+template <bool REVERSE>
+__device__ __forceinline__ void cumsum64(float* a, float* seg, const float* base) {
+  constexpr int LDK = AsmSmem::LDK, KQ = AsmSmem::KQ;
+  const int f = threadIdx.x % KQ, sg = threadIdx.x / KQ;  // 8 segments
+  float v[8], run = 0.f;
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    const int i = REVERSE ? (63 - (sg * 8 + r)) : (sg * 8 + r);
+    run += a[i * LDK + f];
+    v[r] = run;
+  }
+  seg[sg * KQ + f] = run;
+  __syncthreads();
+  float carry = REVERSE && base ? base[f] : 0.f;
+  for (int s2 = 0; s2 < sg; ++s2) carry += seg[s2 * KQ + f];
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    const int i = REVERSE ? (63 - (sg * 8 + r)) : (sg * 8 + r);
+    a[i * LDK + f] = v[r] + carry;
+  }
+  __syncthreads();
+}
+
+// One (chunk, quarter) with the CTA's 256 threads, shared memory at `smem`
+// (AsmSmem::bytes).  Ends with a barrier.
+template <typename TIn>
+__device__ __forceinline__ void assemble_quarter(const BwdArgs& a, float* smem, int ch, int fq4, int hv, int b) {
+  using S = AsmSmem;
+  constexpr int C = S::C, KQ = S::KQ, LDK = S::LDK, LDC = S::LDC, KD = 128;
+  float *sK = smem + S::oK, *sQ = smem + S::oQ, *sC = smem + S::oC, *sDq = smem + S::oDq,
+        *sDk = smem + S::oDk, *sDc = smem + S::oDc, *sE1 = smem + S::oE1, *sE2o = smem + S::oE2o,
+        *sE2d = smem + S::oE2d, *sdA = smem + S::odA, *sdP = smem + S::odP, *sBeta = smem + S::oBeta,
+        *sSeg = smem + S::oSeg, *sLast = smem + S::oLast;
+  int* sFlag = reinterpret_cast<int*>(smem + S::oFlag);
+  const int G = a.HV / a.H, h = hv / G, T = a.T, NT = (T + C - 1) / C;
+  const int t0 = ch * C, L = min(C, T - t0), f0 = fq4 * KQ;
+  const size_t head = (size_t)b * a.HV + hv;
+  const float* rec = a.gws + (head * NT + ch) * GREC;
+  const TIn* q = static_cast<const TIn*>(a.q);
+  const TIn* k = static_cast<const TIn*>(a.k);
+  const int tid = threadIdx.x;
+
+  // [dQE; dKE'] and dKEd of this quarter, consumed further down: lane = channel f,
+  // warp w = rows 8w .. 8w + 7 (each row a 128-byte run of the row-major record)
+  const int ef = tid & 31, ei = (tid >> 5) * 8;
+  float qe[8], ke[8], kd[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    qe[u] = rec[G_QK + rec_off(ei + u, f0 + ef, 128)];
+    ke[u] = rec[G_QK + rec_off(64 + ei + u, f0 + ef, 128)];
+    kd[u] = rec[G_KED + rec_off(ei + u, f0 + ef, 128)];
+  }
+  {  // inputs of this channel quarter (4 channels per item) and the C x C adjoints; loads first
+    float4 gv[2], dp[4], da[4];
+    float qv[2][4], kv[2][4];
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+      const int idx = tid + m * NTHREADS, i = idx >> 3, f4 = (idx & 7) * 4;
+      gv[m] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) qv[m][u] = kv[m][u] = 0.f;
+      if (i < L) {
+        const size_t rq = (((size_t)b * T + t0 + i) * a.H + h) * KD + f0 + f4;
+        gv[m] = *reinterpret_cast<const float4*>(a.g + (((size_t)b * T + t0 + i) * a.HV + hv) * KD + f0 + f4);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          qv[m][u] = to_f(q[rq + u]);
+          kv[m][u] = to_f(k[rq + u]);
+        }
+      }
+    }
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {  // row i of [dP; dA], four columns j per item
+      const int idx = tid + m * NTHREADS, i = idx >> 4, j4 = (idx & 15) * 4;
+      dp[m] = *reinterpret_cast<const float4*>(rec + G_PA + rec_off(i, j4, 64));
+      da[m] = *reinterpret_cast<const float4*>(rec + G_PA + rec_off(64 + i, j4, 64));
+    }
+    if (tid < C) sBeta[tid] = (tid < L) ? a.beta[((size_t)b * T + t0 + tid) * a.HV + hv] : 0.f;
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+      const int idx = tid + m * NTHREADS, i = idx >> 3, f4 = (idx & 7) * 4;
+      const float gg[4] = {gv[m].x, gv[m].y, gv[m].z, gv[m].w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        sQ[i * LDK + f4 + u] = qv[m][u] * a.scale;
+        sK[i * LDK + f4 + u] = kv[m][u];
+        sC[i * LDK + f4 + u] = gg[u];
+      }
+    }
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int idx = tid + m * NTHREADS, i = idx >> 4, j4 = (idx & 15) * 4;
+      const float vdp[4] = {dp[m].x, dp[m].y, dp[m].z, dp[m].w}, vda[4] = {da[m].x, da[m].y, da[m].z, da[m].w};
+      float4 wp, wa;
+      wp.x = (j4 <= i) ? vdp[0] : 0.f;
+      wp.y = (j4 + 1 <= i) ? vdp[1] : 0.f;
+      wp.z = (j4 + 2 <= i) ? vdp[2] : 0.f;
+      wp.w = (j4 + 3 <= i) ? vdp[3] : 0.f;
+      wa.x = (j4 < i) ? vda[0] : 0.f;
+      wa.y = (j4 + 1 < i) ? vda[1] : 0.f;
+      wa.z = (j4 + 2 < i) ? vda[2] : 0.f;
+      wa.w = (j4 + 3 < i) ? vda[3] : 0.f;
+      *reinterpret_cast<float4*>(sdP + i * LDC + j4) = wp;  // LDC = 68: rows 16-byte aligned
+      *reinterpret_cast<float4*>(sdA + i * LDC + j4) = wa;
+    }
+  }
+  __syncthreads();
+  cumsum64<false>(sC, sSeg, nullptr);
+  if (fq4 == 0 && tid < L) {  // dbeta = dbeta_R + sum_{j<i} dA_ij Ah_ij (Ah read straight from the record)
+    const int i = tid;
+    const float4* arow = reinterpret_cast<const float4*>(a.inter + (head * NT + ch) * INTER_REC + INTER_AH + i * 64);
+    float s0 = rec[G_DBR + i], s1 = 0.f;
+#pragma unroll
+    for (int j4 = 0; j4 < 16; ++j4) {
+      const float4 ah = arow[j4];
+      const float vah[4] = {ah.x, ah.y, ah.z, ah.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = j4 * 4 + u;
+        if (u & 1) s1 = fmaf(sdA[i * LDC + j], vah[u], s1);
+        else s0 = fmaf(sdA[i * LDC + j], vah[u], s0);
+      }
+    }
+    a.dbeta[((size_t)b * T + t0 + i) * a.HV + hv] = s0 + s1;
+  }
+  __syncthreads();
+  for (int idx = tid; idx < C * C; idx += NTHREADS) {
+    const int i = idx >> 6, j = idx & 63;
+    sdA[i * LDC + j] *= sBeta[i];
+  }
+  {  // element-wise terms; the chunk-end sum of dKEd o k o e^{c_last-c} goes through sE1
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+      const int f = ef, i4 = ei + 4 * m;
+      const float vq[4] = {qe[4 * m], qe[4 * m + 1], qe[4 * m + 2], qe[4 * m + 3]},
+                  vk[4] = {ke[4 * m], ke[4 * m + 1], ke[4 * m + 2], ke[4 * m + 3]},
+                  vd[4] = {kd[4 * m], kd[4 * m + 1], kd[4 * m + 2], kd[4 * m + 3]};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i4 + u, o = i * LDK + f;
+        const float c = sC[o], e = __expf(c), ed = __expf(sC[(C - 1) * LDK + f] - c);
+        const float dqe = vq[u], dke = sBeta[i] * vk[u], dked = vd[u];
+        const float kk = sK[o], qq = sQ[o];
+        sDq[o] = dqe * e;
+        sDk[o] = dke * e + dked * ed;
+        sDc[o] = (dqe * qq + dke * kk) * e - dked * kk * ed;
+        sE1[o] = dked * kk * ed;
+      }
+    }
+  }
+  __syncthreads();
+  {  // chunk-end terms: dEl o e^{c_last} + sum_i dKEd o k o e^{c_last - c}
+    const int f = tid % KQ, sg = tid / KQ;
+    float s = 0.f;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) s += sE1[(sg * 8 + r) * LDK + f];
+    sSeg[sg * KQ + f] = s;
+    __syncthreads();
+    if (tid < KQ) {
+      float t = rec[G_DEL + f0 + tid] * __expf(sC[(C - 1) * LDK + tid]);
+      for (int s2 = 0; s2 < 8; ++s2) t += sSeg[s2 * KQ + tid];
+      sLast[tid] = t;
+    }
+    __syncthreads();
+  }
+  {  // split exponents hold when every 16-row block's decay span is at most 80
+    bool wide = false;
+    if (tid < 4 * KQ) {
+      const int J = tid / KQ, f = tid % KQ;
+      wide = sC[(16 * J) * LDK + f] - sC[(16 * J + 15) * LDK + f] > DIAG_SPAN_MAX;
+    }
+    if (__syncthreads_or(wide))
+      factored_terms<KQ, C, false, false, LDK, LDC>(sK, sQ, sC, sdA, sdP, sE1, sE2o, sE2d, sFlag, sDq, sDk, sDc);
+    else
+      factored_terms_fused<KQ, LDK, LDC>(sK, sQ, sC, sdA, sdP, sDq, sDk, sDc);
+  }
+  cumsum64<true>(sDc, sSeg, sLast);
+  TIn* dq = static_cast<TIn*>(a.dq);
+  TIn* dk = static_cast<TIn*>(a.dk);
+  for (int idx = tid; idx < L * KQ; idx += NTHREADS) {
+    const int i = idx / KQ, f = idx % KQ, o = i * LDK + f;
+    const size_t row_v = ((size_t)b * T + t0 + i) * a.HV + hv;
+    a.dg[row_v * KD + f0 + f] = sDc[o];
+    if (G == 1) {
+      const size_t row_h = ((size_t)b * T + t0 + i) * a.H + h;
+      dq[row_h * KD + f0 + f] = from_f<TIn>(a.scale * sDq[o]);
+      dk[row_h * KD + f0 + f] = from_f<TIn>(sDk[o]);
+    } else {
+      a.dq_part[row_v * KD + f0 + f] = a.scale * sDq[o];
+      a.dk_part[row_v * KD + f0 + f] = sDk[o];
+    }
+  }
+  __syncthreads();
+}
+
+}  // namespace kda

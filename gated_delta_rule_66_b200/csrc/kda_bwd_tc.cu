@@ -216,7 +216,7 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_dstate_tc_kernel(BwdArgs a) {
 bool bwd_tc_eligible(const BwdArgs& a, int dtype) {
   auto al16 = [](const void* p) { return ((uintptr_t)p & 15u) == 0; };
   return dtype == 1 && a.K == 128 && a.V == 128 && a.gws != nullptr && a.inter != nullptr && al16(a.q) &&
-         al16(a.k) && al16(a.v) && al16(a.dO) && al16(a.g);
+         al16(a.k) && al16(a.v) && al16(a.dO) && al16(a.g) && al16(a.dq);
 }
 
 int launch_bwd_dstate_tc(const BwdArgs& a, cudaStream_t stream) {
@@ -262,22 +262,6 @@ static_assert(OP_DO + 2 * 64 * PAD_SBO / 8 <= SMALL && OP_PBR + 1024 <= OP_DO &&
 constexpr uint32_t TM_M = 0, TM_U = 0, TM_QK = 0, TM_DM = 128, TM_DR = 128, TM_KED = 128, TM_DOT = 256,
                    TM_PA = 256, TM_X = 320, TM_DU = 384;
 }  // namespace tcg
-
-// Sums over the warp's 32 lanes of 32 values at once: lane l returns
-// sum over lanes of v[l] (31 shuffles instead of 32 x 5).  v is clobbered.
-__device__ __forceinline__ float warp_sum32(float (&v)[32], int lane) {
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    const bool up = (lane & off) != 0;
-#pragma unroll
-    for (int k = 0; k < off; ++k) {
-      const float send = up ? v[k] : v[k + off];
-      const float keep = up ? v[k + off] : v[k];
-      v[k] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-    }
-  }
-  return v[0];
-}
 
 __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
   using namespace tcg;

@@ -135,6 +135,22 @@ __device__ __forceinline__ void copy_image(const Ctx& c, uint32_t dst, const flo
   for (int e = c.tid; e < 1024; e += NT) tc::cp_async16(c.sb + dst + e * 16, src + e * 4, true);
 }
 
+// Sums over the warp's 32 lanes of 32 values at once: lane l returns
+// sum over lanes of v[l] (31 shuffles instead of 32 x 5).  v is clobbered.
+__device__ __forceinline__ float warp_sum32(float (&v)[32], int lane) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const bool up = (lane & off) != 0;
+#pragma unroll
+    for (int k = 0; k < off; ++k) {
+      const float send = up ? v[k] : v[k + off];
+      const float keep = up ? v[k + off] : v[k];
+      v[k] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+  return v[0];
+}
+
 // float index of element (r, k) in a 64 x 64 record image
 __device__ __forceinline__ int img(int r, int k) { return (int)(tc::kmaj(r, k, 64) >> 2); }
 

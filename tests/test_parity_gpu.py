@@ -230,6 +230,17 @@ def test_bwd_shapes(kda, name, base, over):
     check_bwd(kda, inp, w.scale, w.torch_dtype, name, dS_T)
 
 
+def test_bwd_tc_strong_unbounded_decay(kda):
+    """bf16 K = V = 128 with decays far beyond the -5 bound: chunks whose
+    decay span rules out the split-exponent factors of the tensor-core
+    assembly take the pair-by-pair route, the others the tensor cores."""
+    w = BY_NAME["fwdbwd"].with_sizes(B=1, T=192, H=1, HV=2)
+    inp = make_inputs(w, with_do=True)
+    inp["g"] = inp["g"] * 8.0
+    inp["g"][:, 64:128] = inp["g"][:, 64:128] / 8.0  # one chunk within range
+    check_bwd(kda, inp, w.scale, w.torch_dtype, "tc_strong_decay")
+
+
 def test_bwd_misaligned_dO_after_tensor_core_forward(kda):
     """A dO that is not 16-byte aligned keeps the backward off the tensor-core
     path; with states_from_fwd it must then not rely on the tensor-core
