@@ -5,6 +5,8 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <vector>
+
 #include "../../include/kda.h"
 #include "kda_internal.h"
 
@@ -79,6 +81,31 @@ static size_t img_bytes(int B, int T, int HV, int K, int V) {
 // training forward: [states | interaction records | chunk images]
 static size_t fwd_ws_bytes(int B, int T, int HV, int K, int V) {
   return states_bytes(B, T, HV, K, V) + inter_bytes(B, T, HV, K, V) + img_bytes(B, T, HV, K, V);
+}
+
+// Packed sequences: the chunk table (t0, L per chunk of at most 64 steps,
+// sequence by sequence) and each sequence's first chunk, from the host
+// cu_seqlens.  Returns the number of chunks, or -1 if cu_seqlens is invalid.
+static long varlen_chunks(const int* cu, int N, std::vector<int>* tab, std::vector<int>* seq0) {
+  if (!cu || N < 1 || cu[0] != 0) return -1;
+  long nc = 0;
+  for (int s = 0; s < N; ++s) {
+    if (cu[s + 1] < cu[s]) return -1;
+    if (seq0) seq0->push_back((int)nc);
+    for (int t0 = cu[s]; t0 < cu[s + 1]; t0 += 64, ++nc)
+      if (tab) {
+        tab->push_back(t0);
+        tab->push_back(cu[s + 1] - t0 < 64 ? cu[s + 1] - t0 : 64);
+      }
+  }
+  if (seq0) seq0->push_back((int)nc);
+  return nc;
+}
+
+// workspace of kda_fwd_varlen: [chunk table | sequence starts] (256-byte
+// aligned), then the chunk images of the two-kernel forward
+static size_t varlen_table_bytes(long nc, int N) {
+  return ((size_t)(2 * nc + N + 1) * sizeof(int) + 255) / 256 * 256;
 }
 
 }  // namespace kda
@@ -157,6 +184,46 @@ int kda_fwd(const void* q, const void* k, const void* v, const float* g, const f
   }
   FwdArgs a{q, k, v, g, beta, S0, o, S_T, states, inter, img, scale, B, T, H, HV, K, V};
   return launch_fwd(a, dtype, static_cast<cudaStream_t>(stream));
+}
+
+size_t kda_fwd_varlen_workspace_bytes(const int* cu_seqlens, int N, int HV, int K, int V) {
+  const long nc = varlen_chunks(cu_seqlens, N, nullptr, nullptr);
+  if (nc < 0 || HV < 1 || K != 128 || V != 128) return 0;
+  return varlen_table_bytes(nc, N) + (size_t)nc * HV * FWI_BYTES;
+}
+
+int kda_fwd_varlen(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                   const float* S0, float scale, const int* cu_seqlens, int N, int H, int HV, int K, int V,
+                   int dtype, void* o, float* S_T, void* workspace, size_t workspace_bytes, void* stream) {
+  g_err[0] = 0;
+  std::vector<int> tab, seq0;
+  const long nc = varlen_chunks(cu_seqlens, N, &tab, &seq0);
+  if (nc < 0)
+    return set_error(KDA_ERR_ARG, "kda_fwd_varlen: cu_seqlens must start at 0 and be non-decreasing (N >= 1)");
+  const int T = cu_seqlens[N];
+  int rc = check_common("kda_fwd_varlen", N, T > 0 ? T : 1, H, HV, K, V, dtype, scale);
+  if (rc) return rc;
+  if (T > 0 && (!q || !k || !v || !g || !beta || !o))
+    return set_error(KDA_ERR_NULL, "kda_fwd_varlen: q, k, v, g, beta and o must be non-NULL");
+  if (!workspace) return set_error(KDA_ERR_WORKSPACE, "kda_fwd_varlen: workspace is required");
+  if (!aligned16(workspace)) return set_error(KDA_ERR_ARG, "kda_fwd_varlen: workspace must be 16-byte aligned");
+  const size_t tb = varlen_table_bytes(nc, N), full = tb + (size_t)nc * HV * FWI_BYTES;
+  if (workspace_bytes < tb)
+    return set_error(KDA_ERR_WORKSPACE, "kda_fwd_varlen: workspace smaller than its chunk table");
+  char* ws = static_cast<char*>(workspace);
+  FwdArgs a{q, k, v, g, beta, S0, o, S_T, nullptr, nullptr,
+            workspace_bytes >= full ? reinterpret_cast<unsigned char*>(ws + tb) : nullptr, scale, N, T, H, HV, K,
+            V, reinterpret_cast<const int*>(ws), reinterpret_cast<const int*>(ws) + 2 * nc, (int)nc};
+  if (!fwd_tc_eligible(a, dtype))
+    return set_error(KDA_ERR_ARG,
+                     "kda_fwd_varlen: packed sequences run on the tensor-core path only (bf16, K = V = 128, "
+                     "16-byte aligned q, k, v, g, o)");
+  std::vector<int> host(tab);
+  host.insert(host.end(), seq0.begin(), seq0.end());
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(ws, host.data(), host.size() * sizeof(int), cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) return set_cuda_error("kda_fwd_varlen: chunk table upload", e);
+  return launch_fwd_tc(a, st);
 }
 
 int kda_decode_step(const void* q, const void* k, const void* v, const float* g,

@@ -38,6 +38,28 @@ constexpr uint32_t OP_BKET = OP, OP_BVT = OP + 32768, OP_QE = OP + 65536, OP_KED
 constexpr uint32_t TM_S = 0, TM_X = 128, TM_O = 192, TM_U = 256, TM_W = 320, TM_APA = 384, TM_APB = 448;
 }  // namespace tcf
 
+// The chunks of the sequence s that a CTA carries: [c0, c1), chunk c at steps
+// span(c).x .. + span(c).y - 1 of batch row `row` (uniform batches: sequence
+// = batch row, chunk c at 64 c; packed sequences: the chunk table, row 0).
+struct SeqChunks {
+  int c0, c1, row;
+  __device__ SeqChunks(const FwdArgs& a, int s) {
+    if (a.ctab) {
+      c0 = a.seq0[s];
+      c1 = a.seq0[s + 1];
+      row = 0;
+    } else {
+      c0 = 0;
+      c1 = (a.T + tcc::C - 1) / tcc::C;
+      row = s;
+    }
+  }
+  __device__ int2 span(const FwdArgs& a, int c) const {
+    if (a.ctab) return make_int2(a.ctab[2 * c], a.ctab[2 * c + 1]);
+    return make_int2(c * tcc::C, min(tcc::C, a.T - c * tcc::C));
+  }
+};
+
 // The state-independent part of one chunk: load, cumulative decay, the
 // interaction products and their read-out, the inverse T, the operands of the
 // state products (Q~ o e^c, (K o e^{c_last-c})^T in shared memory; e^{c_last}
@@ -46,17 +68,20 @@ constexpr uint32_t TM_S = 0, TM_X = 128, TM_O = 192, TM_U = 256, TM_W = 320, TM_
 // `irec` it stores the chunk's interaction record; with `img` it starts the
 // bulk stores of the chunk images of Q~ o e^c, (K o e^{c_last-c})^T and
 // e^{c_last} as soon as they are built.
+// The chunk covers steps t0 .. t0 + L - 1 of batch row b (packed sequences:
+// b = 0 and t0 on the packed axis); with Ln > 0 the next chunk of the same
+// sequence (Ln steps from t0 + 64) is prefetched into L2.
 // Returns false, block-uniformly, if a tensor-core wait ran out.
 template <int NTHR>
 __device__ __forceinline__ bool fwd_chunk_head(const tcc::Ctx& cx, const FwdArgs& a, int b, int hv, int h,
-                                               int ch, bool prefetch_next, float* irec,
+                                               int t0, int L, int Ln, float* irec,
                                                unsigned char* img, uint64_t* bar, uint32_t& phase) {
   using namespace tcf;
   using namespace tc;
   unsigned char* sm = cx.sm;
   const uint32_t sb = cx.sb, tm = cx.tm;
   const int tid = cx.tid;
-  const int T = a.T, NT = (T + C - 1) / C, t0 = ch * C, L = min(C, T - t0);
+  const int T = a.T;
   const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(a.q);
   const __nv_bfloat16* kg = static_cast<const __nv_bfloat16*>(a.k);
   const __nv_bfloat16* vg = static_cast<const __nv_bfloat16*>(a.v);
@@ -64,8 +89,7 @@ __device__ __forceinline__ bool fwd_chunk_head(const tcc::Ctx& cx, const FwdArgs
   float* sEl = reinterpret_cast<float*>(sm + S_EL);
   const float* sC = cx.c();
   load_raw_issue<NTHR>(cx, qg, kg, vg, a.g, a.beta, b, T, t0, L, a.H, a.HV, h, hv);
-  if (prefetch_next && ch + 1 < NT)
-    prefetch_chunk(cx, qg, kg, vg, a.g, b, T, t0 + C, min(C, T - t0 - C), a.H, a.HV, h, hv);
+  if (Ln > 0) prefetch_chunk(cx, qg, kg, vg, a.g, b, T, t0 + C, Ln, a.H, a.HV, h, hv);
   if (!load_raw_wait(cx)) return false;
   const bool wide = cumsum_span(cx);
   build_op1_and_issue<NTHR>(cx, a.scale, tm + TM_APA, tm + TM_APB, bar);
@@ -169,15 +193,13 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_tc_kernel(FwdArgs a) {
   const int tid = cx.tid, hcol = cx.hcol, Lr = cx.Lr;
   const uint32_t lo = cx.lo, sb = cx.sb;
 
-  const int hv = blockIdx.x, b = blockIdx.y;
+  const int hv = blockIdx.x, s = blockIdx.y;  // s: batch row, or sequence of a packed batch
+  const SeqChunks sc(a, s);
+  const int b = sc.row;
   const int G = a.HV / a.H, h = hv / G, T = a.T, NT = (T + C - 1) / C;
   const int NT32 = (T + 31) / 32;  // the state workspace holds the state entering every 32 steps
-  const size_t head = (size_t)b * a.HV + hv;
-  const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(a.q);
-  const __nv_bfloat16* kg = static_cast<const __nv_bfloat16*>(a.k);
-  const __nv_bfloat16* vg = static_cast<const __nv_bfloat16*>(a.v);
+  const size_t head = (size_t)s * a.HV + hv;
   __nv_bfloat16* og = static_cast<__nv_bfloat16*>(a.o);
-  float* sBeta = cx.beta();
   float* sEl = reinterpret_cast<float*>(sm + S_EL);
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + S_BAR);
   uint32_t* sTm = reinterpret_cast<uint32_t*>(sm + S_TMEM);
@@ -207,10 +229,12 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_tc_kernel(FwdArgs a) {
   fence_before();
   __syncthreads();
 
-  for (int ch = 0; ch < NT; ++ch) {
-    const int t0 = ch * C, L = min(C, T - t0);
+  for (int c = sc.c0; c < sc.c1; ++c) {
+    const int2 sp = sc.span(a, c);
+    const int t0 = sp.x, L = sp.y, ch = c - sc.c0;  // (records and states: uniform batches only)
+    const int Ln = c + 1 < sc.c1 ? sc.span(a, c + 1).y : 0;
     float* irec = a.inter ? a.inter + (head * NT + ch) * INTER_REC : nullptr;
-    if (!fwd_chunk_head<NTH>(cx, a, b, hv, h, ch, true, irec, nullptr, bar, phase)) {
+    if (!fwd_chunk_head<NTH>(cx, a, b, hv, h, t0, L, Ln, irec, nullptr, bar, phase)) {
       failed = true;
       break;
     }
@@ -337,7 +361,9 @@ __global__ void __launch_bounds__(PREP_NT, 1) kda_fwd_prep_tc_kernel(FwdArgs a) 
   const int tid = cx.tid, hcol = cx.hcol, Lr = cx.Lr;
   const uint32_t lo = cx.lo, sb = cx.sb;
   const int G = a.HV / a.H, NT = (a.T + C - 1) / C;
-  const int items = NT * a.HV * a.B;  // item = (b * HV + hv) * NT + ch
+  // item = (b * HV + hv) * NT + ch (uniform batches) or hv * NC + c (packed sequences);
+  // the item is also the index of the chunk's images
+  const int items = a.ctab ? a.NC * a.HV : NT * a.HV * a.B;
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + S_BAR);
   uint32_t* sTm = reinterpret_cast<uint32_t*>(sm + S_TMEM);
 
@@ -354,13 +380,26 @@ __global__ void __launch_bounds__(PREP_NT, 1) kda_fwd_prep_tc_kernel(FwdArgs a) 
   // prefetch of the next item's rows measured slower: it queues behind the
   // image stores.)
   for (int item = blockIdx.x; item < items; item += gridDim.x) {
-    const int ch = item % NT, hv = (item / NT) % a.HV, b = item / (NT * a.HV), h = hv / G;
-    const size_t head = (size_t)b * a.HV + hv;
+    int hv, b, t0, L;
+    if (a.ctab) {
+      const int c = item % a.NC;
+      hv = item / a.NC;
+      b = 0;
+      t0 = a.ctab[2 * c];
+      L = a.ctab[2 * c + 1];
+    } else {
+      const int ch = item % NT;
+      hv = (item / NT) % a.HV;
+      b = item / (NT * a.HV);
+      t0 = ch * C;
+      L = min(C, a.T - t0);
+    }
+    const int h = hv / G;
     if ((tid & 31) == 0 && tid < 96) bulk_wait_read();  // the previous item's image stores have left smem
     __syncthreads();
-    float* irec = a.inter ? a.inter + (head * NT + ch) * INTER_REC : nullptr;
-    unsigned char* img = a.img + (head * NT + ch) * (size_t)FWI_BYTES;
-    if (!fwd_chunk_head<PREP_NT>(cx, a, b, hv, h, ch, false, irec, img, bar, phase)) {
+    float* irec = a.inter ? a.inter + (size_t)item * INTER_REC : nullptr;  // (uniform batches only)
+    unsigned char* img = a.img + (size_t)item * FWI_BYTES;
+    if (!fwd_chunk_head<PREP_NT>(cx, a, b, hv, h, t0, L, 0, irec, img, bar, phase)) {
       failed = true;
       break;
     }
@@ -425,11 +464,14 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_seq_tc_kernel(FwdArgs a) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, hcol = warp >> 2;
   const int Lr = (warp & 3) * 32 + lane;
   const uint32_t lo = (uint32_t)((warp & 3) * 32) << 16;
-  const int hv = blockIdx.x, b = blockIdx.y;
+  const int hv = blockIdx.x, s = blockIdx.y;  // s: batch row, or sequence of a packed batch
+  const SeqChunks sc(a, s);
+  const int b = sc.row, nch = sc.c1 - sc.c0;
   const int T = a.T, NT = (T + tcc::C - 1) / tcc::C, NT32 = (T + 31) / 32;
   constexpr int C = tcc::C, KD = tcc::KD, VD = tcc::VD;
-  const size_t head = (size_t)b * a.HV + hv;
-  const unsigned char* imgs = a.img + head * NT * (size_t)FWI_BYTES;
+  const size_t head = (size_t)s * a.HV + hv;
+  // this sequence's chunk images, consecutive (the chunk kernel's item order)
+  const unsigned char* imgs = a.img + (a.ctab ? (size_t)hv * a.NC + sc.c0 : head * NT) * (size_t)FWI_BYTES;
   __nv_bfloat16* og = static_cast<__nv_bfloat16*>(a.o);
   uint64_t* barA = reinterpret_cast<uint64_t*>(sm + SQ_BAR);  // [2]
   uint64_t* barB = barA + 2;
@@ -448,7 +490,7 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_seq_tc_kernel(FwdArgs a) {
   __syncthreads();
   fence_after();
   const uint32_t tm = *sTm;
-  if (tid == 0) {
+  if (tid == 0 && nch > 0) {
     fetch_images(sb + SQ_A0, imgs, FWI_A_BYTES, barA);
     fetch_images(sb + SQ_B, imgs + FWI_KEDT, FWI_B_BYTES, barB);
   }
@@ -467,11 +509,12 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_seq_tc_kernel(FwdArgs a) {
   uint32_t phase = 0;
   bool failed = false;
 
-  for (int ch = 0; ch < NT; ++ch) {
-    const int t0 = ch * C, L = min(C, T - t0);
+  for (int ch = 0; ch < nch; ++ch) {
+    const int2 sp = sc.span(a, sc.c0 + ch);
+    const int t0 = sp.x, L = sp.y;
     const unsigned char* img = imgs + (size_t)ch * FWI_BYTES;
     const uint32_t bufA = (ch & 1) ? SQ_A1 : SQ_A0;
-    if (tid == 32 && ch + 1 < NT) prefetch_l2(img + FWI_BYTES, FWI_BYTES);
+    if (tid == 32 && ch + 1 < nch) prefetch_l2(img + FWI_BYTES, FWI_BYTES);
     float u0[32];
     {
       const float* src = reinterpret_cast<const float*>(img + FWI_U0);
@@ -487,7 +530,7 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_seq_tc_kernel(FwdArgs a) {
         mma_ts(tm + TM_O, tm + TM_S + ks * 8, desc(sb + bufA + FWI_QE + ks * 256, 4096), id, ks > 0);
       }
       commit(bar);
-      if (ch + 1 < NT) fetch_images(sb + ((ch & 1) ? SQ_A0 : SQ_A1), img + FWI_BYTES, FWI_A_BYTES, barA + ((ch + 1) & 1));
+      if (ch + 1 < nch) fetch_images(sb + ((ch & 1) ? SQ_A0 : SQ_A1), img + FWI_BYTES, FWI_A_BYTES, barA + ((ch + 1) & 1));
     }
     if (!tcc::wait_mma(bar, phase)) { failed = true; break; }
     {  // U^T = U0^T - X^T
@@ -528,7 +571,7 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_seq_tc_kernel(FwdArgs a) {
       commit(bar);
     }
     if (!tcc::wait_mma(bar, phase)) { failed = true; break; }
-    if (tid == 0 && ch + 1 < NT) {  // the lanes' reads of e^{c_last} precede the overwrite
+    if (tid == 0 && ch + 1 < nch) {  // the lanes' reads of e^{c_last} precede the overwrite
       fence_async_smem();
       fetch_images(sb + SQ_B, img + FWI_BYTES + FWI_KEDT, FWI_B_BYTES, barB);
     }
@@ -575,12 +618,14 @@ int launch_fwd_tc(const FwdArgs& a, cudaStream_t stream) {
       e = cudaFuncSetAttribute(kda_fwd_seq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)tcs::SQ_BYTES);
     if (e != cudaSuccess) return set_cuda_error("kda_fwd: cudaFuncSetAttribute", e);
-    const int items = (a.T + tcc::C - 1) / tcc::C * a.HV * a.B;
+    const int items = a.ctab ? a.NC * a.HV : (a.T + tcc::C - 1) / tcc::C * a.HV * a.B;
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    kda_fwd_prep_tc_kernel<<<min(items, sms), PREP_NT, tcc::SMEM_BYTES, stream>>>(a);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return set_cuda_error("kda_fwd: tensor-core chunk launch", e);
+    if (items > 0) {  // (packed batches of empty sequences have no chunks)
+      kda_fwd_prep_tc_kernel<<<min(items, sms), PREP_NT, tcc::SMEM_BYTES, stream>>>(a);
+      e = cudaGetLastError();
+      if (e != cudaSuccess) return set_cuda_error("kda_fwd: tensor-core chunk launch", e);
+    }
     kda_fwd_seq_tc_kernel<<<dim3(a.HV, a.B), tcc::NTH, tcs::SQ_BYTES, stream>>>(a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return set_cuda_error("kda_fwd: tensor-core state-pass launch", e);

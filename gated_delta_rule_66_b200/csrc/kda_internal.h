@@ -55,6 +55,13 @@ struct FwdArgs {
   unsigned char* img;  // may be null; per-chunk operand images of the two-kernel forward (K = V = 128)
   float scale;
   int B, T, H, HV, K, V;
+  // Packed sequences (null ctab: B uniform batch rows of T steps).  Then B is
+  // the number of sequences, T the packed length, rows index the packed axis;
+  // chunk c covers steps ctab[2c] .. ctab[2c] + ctab[2c+1] - 1, and sequence
+  // s owns chunks seq0[s] .. seq0[s+1] - 1 (NC chunks in all).
+  const int* ctab;
+  const int* seq0;
+  int NC;
 };
 
 struct BwdArgs {

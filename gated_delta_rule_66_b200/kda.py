@@ -23,7 +23,8 @@ KDA_BWD_STATES_FROM_FWD = 1
 CHUNK = 32  # chunk length of the library's chunked kernels (workspace layout)
 
 SYMBOLS = ("kda_last_error", "kda_device_status", "kda_fwd_workspace_bytes", "kda_fwd_scratch_bytes",
-           "kda_bwd_workspace_bytes", "kda_fwd", "kda_decode_step", "kda_bwd")
+           "kda_bwd_workspace_bytes", "kda_fwd", "kda_fwd_varlen_workspace_bytes", "kda_fwd_varlen",
+           "kda_decode_step", "kda_bwd")
 
 
 class KdaError(RuntimeError):
@@ -53,6 +54,11 @@ def _load():
     lib.kda_bwd_workspace_bytes.argtypes = [i, i, i, i, i, i]
     lib.kda_fwd.restype = i
     lib.kda_fwd.argtypes = [vp, vp, vp, vp, vp, vp, f, i, i, i, i, i, i, i, vp, vp, vp, sz, vp]
+    lib.kda_fwd_varlen_workspace_bytes.restype = sz
+    lib.kda_fwd_varlen_workspace_bytes.argtypes = [ctypes.POINTER(ctypes.c_int), i, i, i, i]
+    lib.kda_fwd_varlen.restype = i
+    lib.kda_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, f, ctypes.POINTER(ctypes.c_int), i, i, i, i, i, i,
+                                   vp, vp, vp, sz, vp]
     lib.kda_decode_step.restype = i
     lib.kda_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, f, i, i, i, i, i, i, vp, vp]
     lib.kda_bwd.restype = i
@@ -155,6 +161,43 @@ def fwd(q, k, v, g, beta, scale=None, initial_state=None, output_final_state=Tru
                       B, T, H, HV, K, V, _dtype_code(q), _ptr(o), _ptr(S_T), _ptr(workspace),
                       ws_bytes, _stream())
     _check("kda_fwd", rc)
+    return o, S_T
+
+
+def _cu_array(cu_seqlens):
+    cu = [int(x) for x in (cu_seqlens.tolist() if hasattr(cu_seqlens, "tolist") else cu_seqlens)]
+    return (ctypes.c_int * len(cu))(*cu), len(cu) - 1
+
+
+def fwd_varlen(q, k, v, g, beta, cu_seqlens, scale=None, initial_state=None, output_final_state=True,
+               workspace=None, out=None):
+    """Packed variable-length prefill.  q, k [T,H,K], v [T,HV,V] bf16, g [T,HV,K]
+    and beta [T,HV] float32 hold N sequences back to back; ``cu_seqlens`` (a
+    host list or CPU tensor of N + 1 offsets) marks them.  initial_state
+    [N,HV,K,V] float32.  Returns (o [T,HV,V], S_T [N,HV,K,V] or None).
+    ``workspace`` defaults to a fresh allocation of kda_fwd_varlen_workspace_bytes.
+    """
+    T, H, K = q.shape
+    HV, V = v.shape[1], v.shape[2]
+    cu, N = _cu_array(cu_seqlens)
+    scale = 1.0 / math.sqrt(K) if scale is None else float(scale)
+    dt = q.dtype
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _req(n, t, dt, 3)
+    _req("g", g, torch.float32, 3)
+    _req("beta", beta, torch.float32, 2)
+    _req("initial_state", initial_state, torch.float32, 4)
+    if workspace is None:
+        need = int(_lib.kda_fwd_varlen_workspace_bytes(cu, N, HV, K, V))
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _req("workspace", workspace)
+    o = torch.empty(T, HV, V, dtype=dt, device=q.device) if out is None else out
+    _req("out", o, dt, 3)
+    S_T = torch.empty(N, HV, K, V, dtype=torch.float32, device=q.device) if output_final_state else None
+    rc = _lib.kda_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state), scale, cu, N,
+                             H, HV, K, V, _dtype_code(q), _ptr(o), _ptr(S_T), _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), _stream())
+    _check("kda_fwd_varlen", rc)
     return o, S_T
 
 

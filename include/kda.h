@@ -118,6 +118,26 @@ int kda_fwd(const void* q, const void* k, const void* v, const float* g, const f
             const float* S0, float scale, int B, int T, int H, int HV, int K, int V, int dtype,
             void* o, float* S_T, void* workspace, size_t workspace_bytes, void* stream);
 
+/* Packed variable-length prefill: N sequences of lengths cu_seqlens[s+1] -
+ * cu_seqlens[s] laid back to back on one time axis of T = cu_seqlens[N] steps,
+ * each run as kda_fwd runs one batch row (its own initial and final state;
+ * the state passing of "recurrent.py", naive_kda_fwd, initial_state and
+ * output_final_state, per sequence).
+ *   q, k [T, H, K] dtype; v [T, HV, V] dtype; g [T, HV, K] float; beta [T, HV] float
+ *   cu_seqlens: HOST int32 [N + 1], cu_seqlens[0] = 0, non-decreasing (empty
+ *     sequences allowed: their final state is their initial state)
+ *   S0 [N, HV, K, V] float or NULL; o [T, HV, V] dtype; S_T [N, HV, K, V] float or NULL
+ *   workspace: required, 16-byte aligned; at least
+ *     kda_fwd_varlen_workspace_bytes() bytes for the two-kernel forward, else at
+ *     least its chunk table (then one kernel per (sequence, value head)).
+ * Runs on the tensor-core path only: bf16, K = V = 128, 16-byte aligned q, k,
+ * v, g and o (KDA_ERR_ARG otherwise).  The chunk table is uploaded from the
+ * host with one copy on `stream`. */
+size_t kda_fwd_varlen_workspace_bytes(const int* cu_seqlens, int N, int HV, int K, int V);
+int kda_fwd_varlen(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                   const float* S0, float scale, const int* cu_seqlens, int N, int H, int HV, int K, int V,
+                   int dtype, void* o, float* S_T, void* workspace, size_t workspace_bytes, void* stream);
+
 /* One decode token on a state updated IN PLACE ("kimi_k3_host/kda.rs",
  * kda_recurrent_step, with the q/k L2 normalisation and the sigmoid of beta
  * left to the caller).

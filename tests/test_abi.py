@@ -110,3 +110,42 @@ def test_last_error_clears_on_next_call(lib):
     assert lib.kda_last_error().decode() != ""
     fwd_call(lib, K=48)
     assert "K=48" in lib.kda_last_error().decode()
+
+
+def test_tensor_core_workspace_sizes(lib):
+    """K = V = 128: the training forward keeps the 32-step states, a 64 KB
+    interaction record and the 149 KB chunk images per 64-step chunk; the
+    backward overwrites the images with its own buffers; the scratch-only
+    forward needs the images alone."""
+    B, T, H, HV, K, V = 1, 130, 1, 2, 128, 128
+    nt32, nt64 = (T + 31) // 32, (T + 63) // 64
+    states = B * HV * nt32 * K * V * 4
+    inter = B * HV * nt64 * 16384 * 4
+    img = B * HV * nt64 * 152064
+    assert lib.kda_fwd_scratch_bytes(B, T, HV, K, V) == img
+    assert lib.kda_fwd_workspace_bytes(B, T, HV, K, V) == states + inter + img
+    tail = states + 2 * B * T * HV * K * 4 + B * HV * nt64 * 37120 * 4  # state grads, dq/dk partials, records
+    assert lib.kda_bwd_workspace_bytes(B, T, H, HV, K, V) == states + inter + max(tail, img)
+    assert lib.kda_bwd_workspace_bytes(B, T, H, HV, K, V) >= lib.kda_fwd_workspace_bytes(B, T, HV, K, V)
+    assert lib.kda_fwd_scratch_bytes(B, T, HV, 64, 64) == 0
+
+
+def _cu(vals):
+    return (ctypes.c_int * len(vals))(*vals)
+
+
+def test_varlen_workspace_and_validation(lib):
+    HV = 3
+    cu = _cu([0, 5, 5, 200])  # sequences of 5, 0 and 195 steps: 1 + 0 + 4 chunks
+    table = ((2 * 5 + 4) * 4 + 255) // 256 * 256
+    assert lib.kda_fwd_varlen_workspace_bytes(cu, 3, HV, 128, 128) == table + 5 * HV * 152064
+    assert lib.kda_fwd_varlen_workspace_bytes(_cu([1, 5]), 1, HV, 128, 128) == 0      # must start at 0
+    assert lib.kda_fwd_varlen_workspace_bytes(_cu([0, 9, 5]), 2, HV, 128, 128) == 0   # decreasing
+    assert lib.kda_fwd_varlen_workspace_bytes(cu, 3, HV, 64, 64) == 0                 # tensor-core shapes only
+    args = (FAKE, FAKE, FAKE, FAKE, FAKE, None, 0.5)
+    rc = lib.kda_fwd_varlen(*args, _cu([0, 9, 5]), 2, 1, HV, 128, 128, 1, FAKE, None, FAKE, 1 << 40, None)
+    assert rc == 7 and "cu_seqlens" in lib.kda_last_error().decode()
+    rc = lib.kda_fwd_varlen(*args, cu, 3, 1, HV, 128, 128, 1, FAKE, None, None, 0, None)
+    assert rc == 5 and "workspace" in lib.kda_last_error().decode()
+    rc = lib.kda_fwd_varlen(*args, cu, 3, 1, HV, 128, 128, 0, FAKE, None, FAKE, 1 << 40, None)  # fp32
+    assert rc == 7 and "tensor-core" in lib.kda_last_error().decode()

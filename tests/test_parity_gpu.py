@@ -351,3 +351,56 @@ def test_decode_sequence_equals_prefill(kda):
     torch.cuda.synchronize()
     assert rel_l2(f64(torch.stack(outs, 1)), f64(o)) < 1e-5
     assert rel_l2(f64(St), f64(S)) < 1e-5
+
+
+# ----------------------------------------------------------------------------- packed sequences
+
+VARLEN_CASES = [
+    # name, sequence lengths, H, HV
+    ("mixed", [5, 0, 195, 64, 1, 130], 2, 4),
+    ("one_long", [300], 1, 2),
+    ("all_short", [1, 2, 3, 63, 65], 1, 1),
+]
+
+
+def _varlen_inputs(lens, H, HV, seed=7):
+    T = sum(lens)
+    w = BY_NAME["prefill_gqa"].with_sizes(B=1, T=max(T, 1), H=H, HV=HV)
+    inp = make_inputs(w, seed=seed)
+    inp = {n: (t[0, :T] if t is not None and n != "S0" else t) for n, t in inp.items()}
+    gen = torch.Generator().manual_seed(seed + 1)
+    S0 = torch.randn(len(lens), HV, w.K, w.V, generator=gen) * 0.02
+    return w, inp, S0
+
+
+@pytest.mark.parametrize("scratch", [True, False], ids=["two_kernel", "single_kernel"])
+@pytest.mark.parametrize("name,lens,H,HV", VARLEN_CASES, ids=[c[0] for c in VARLEN_CASES])
+def test_fwd_varlen(kda, name, lens, H, HV, scratch):
+    """N packed sequences (empty, one-step, exact-chunk and ragged lengths)
+    against the oracle run on each sequence with its own initial state."""
+    w, inp, S0 = _varlen_inputs(lens, H, HV)
+    cu = [0]
+    for n in lens:
+        cu.append(cu[-1] + n)
+    d = {n: t.cuda() for n, t in inp.items() if t is not None}
+    ws = None
+    if not scratch:  # the chunk table only: one kernel per (sequence, value head)
+        nc = sum((n + 63) // 64 for n in lens)
+        ws = torch.empty(((2 * nc + len(lens) + 1) * 4 + 255) // 256 * 256, dtype=torch.uint8, device="cuda")
+    o, S = kda.fwd_varlen(d["q"], d["k"], d["v"], d["g"], d["beta"], cu, scale=w.scale,
+                          initial_state=S0.cuda(), workspace=ws)
+    torch.cuda.synchronize()
+    o_ref = np.zeros((cu[-1], HV, w.V))
+    S_ref = np.zeros((len(lens), HV, w.K, w.V))
+    for s, (a0, a1) in enumerate(zip(cu[:-1], cu[1:])):
+        if a1 == a0:
+            S_ref[s] = f64(S0[s])
+            continue
+        sl = lambda t: f64(t[a0:a1].unsqueeze(0))
+        os_, Ss = oracle.kda_forward(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]), sl(inp["g"]), sl(inp["beta"]),
+                                     w.scale, f64(S0[s:s + 1]))
+        o_ref[a0:a1] = os_[0]
+        S_ref[s] = Ss[0]
+    tol = tol_for(w.torch_dtype)
+    report(f"varlen_{name} o", f64(o), o_ref, tol, w.torch_dtype)
+    report(f"varlen_{name} S_T", f64(S), S_ref, tol, torch.float32)
