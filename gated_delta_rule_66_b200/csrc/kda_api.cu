@@ -108,6 +108,21 @@ static size_t varlen_table_bytes(long nc, int N) {
   return ((size_t)(2 * nc + N + 1) * sizeof(int) + 255) / 256 * 256;
 }
 
+// training workspace of packed sequences (K = V = 128): [table | states (one
+// per value head and chunk) | interaction records | the chunk images, which
+// the backward overwrites with [state gradients | dq/dk partials | records]]
+struct VarlenLayout {
+  size_t table, states, inter, img, tail, total;
+  VarlenLayout(long nc, int N, int T, int H, int HV) {
+    table = varlen_table_bytes(nc, N);
+    states = (size_t)HV * nc * 128 * 128 * sizeof(float);
+    inter = (size_t)HV * nc * INTER_REC * sizeof(float);
+    img = (size_t)HV * nc * FWI_BYTES;
+    tail = states + (HV > H ? 2 * (size_t)T * HV * 128 * sizeof(float) : 0) + (size_t)HV * nc * GREC * sizeof(float);
+    total = table + states + inter + (tail > img ? tail : img);
+  }
+};
+
 }  // namespace kda
 
 using namespace kda;
@@ -211,8 +226,15 @@ int kda_fwd_varlen(const void* q, const void* k, const void* v, const float* g, 
   if (workspace_bytes < tb)
     return set_error(KDA_ERR_WORKSPACE, "kda_fwd_varlen: workspace smaller than its chunk table");
   char* ws = static_cast<char*>(workspace);
-  FwdArgs a{q, k, v, g, beta, S0, o, S_T, nullptr, nullptr,
-            workspace_bytes >= full ? reinterpret_cast<unsigned char*>(ws + tb) : nullptr, scale, N, T, H, HV, K,
+  float *states = nullptr, *inter = nullptr;
+  unsigned char* img = workspace_bytes >= full ? reinterpret_cast<unsigned char*>(ws + tb) : nullptr;
+  const VarlenLayout lay(nc, N, T, H, HV);
+  if (K == 128 && V == 128 && workspace_bytes >= lay.total) {  // training: states and records for kda_bwd_varlen
+    states = reinterpret_cast<float*>(ws + tb);
+    inter = reinterpret_cast<float*>(ws + tb + lay.states);
+    img = reinterpret_cast<unsigned char*>(ws + tb + lay.states + lay.inter);
+  }
+  FwdArgs a{q, k, v, g, beta, S0, o, S_T, states, inter, img, scale, N, T, H, HV, K,
             V, reinterpret_cast<const int*>(ws), reinterpret_cast<const int*>(ws) + 2 * nc, (int)nc};
   if (!fwd_tc_eligible(a, dtype))
     return set_error(KDA_ERR_ARG,
@@ -224,6 +246,66 @@ int kda_fwd_varlen(const void* q, const void* k, const void* v, const float* g, 
   cudaError_t e = cudaMemcpyAsync(ws, host.data(), host.size() * sizeof(int), cudaMemcpyHostToDevice, st);
   if (e != cudaSuccess) return set_cuda_error("kda_fwd_varlen: chunk table upload", e);
   return launch_fwd_tc(a, st);
+}
+
+size_t kda_bwd_varlen_workspace_bytes(const int* cu_seqlens, int N, int H, int HV, int K, int V) {
+  const long nc = varlen_chunks(cu_seqlens, N, nullptr, nullptr);
+  if (nc < 0 || H < 1 || HV < 1 || HV % H || K != 128 || V != 128) return 0;
+  return VarlenLayout(nc, N, cu_seqlens[N], H, HV).total;
+}
+
+int kda_bwd_varlen(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                   const float* S0, const void* dO, const float* dS_T, float scale, const int* cu_seqlens, int N,
+                   int H, int HV, int K, int V, int dtype, void* dq, void* dk, void* dv, float* dg, float* dbeta,
+                   float* dS0, void* workspace, size_t workspace_bytes, int flags, void* stream) {
+  g_err[0] = 0;
+  std::vector<int> tab, seq0;
+  const long nc = varlen_chunks(cu_seqlens, N, &tab, &seq0);
+  if (nc < 0)
+    return set_error(KDA_ERR_ARG, "kda_bwd_varlen: cu_seqlens must start at 0 and be non-decreasing (N >= 1)");
+  const int T = cu_seqlens[N];
+  int rc = check_common("kda_bwd_varlen", N, T > 0 ? T : 1, H, HV, K, V, dtype, scale);
+  if (rc) return rc;
+  if (T > 0 && (!q || !k || !v || !g || !beta || !dO || !dq || !dk || !dv || !dg || !dbeta))
+    return set_error(KDA_ERR_NULL,
+                     "kda_bwd_varlen: q, k, v, g, beta, dO, dq, dk, dv, dg and dbeta must be non-NULL");
+  if (flags & ~KDA_BWD_STATES_FROM_FWD) return set_error(KDA_ERR_ARG, "kda_bwd_varlen: unknown flags");
+  if (K != 128 || V != 128 || dtype != KDA_DTYPE_BF16)
+    return set_error(KDA_ERR_ARG, "kda_bwd_varlen: packed sequences run on the tensor-core path only (bf16, K = V = 128)");
+  const VarlenLayout lay(nc, N, T, H, HV);
+  if (!workspace || workspace_bytes < lay.total)
+    return set_error(KDA_ERR_WORKSPACE, "kda_bwd_varlen: workspace smaller than kda_bwd_varlen_workspace_bytes()");
+  if (!aligned16(workspace)) return set_error(KDA_ERR_ARG, "kda_bwd_varlen: workspace must be 16-byte aligned");
+  char* ws = static_cast<char*>(workspace);
+  const int* ctab = reinterpret_cast<const int*>(ws);
+  float* states = reinterpret_cast<float*>(ws + lay.table);
+  float* inter = reinterpret_cast<float*>(ws + lay.table + lay.states);
+  char* x = ws + lay.table + lay.states + lay.inter;
+  float* dstates = reinterpret_cast<float*>(x);
+  float *dq_part = nullptr, *dk_part = nullptr;
+  size_t off = lay.states;
+  if (HV > H) {
+    dq_part = reinterpret_cast<float*>(x + off);
+    dk_part = dq_part + (size_t)T * HV * K;
+    off += 2 * (size_t)T * HV * K * sizeof(float);
+  }
+  float* gws = reinterpret_cast<float*>(x + off);
+  BwdArgs a{q, k, v, dO, g, beta, dS_T, states, inter, dstates, dq, dk, dv, dg, dbeta, dS0,
+            dq_part, dk_part, gws, scale, N, T, H, HV, K, V, ctab, ctab + 2 * nc, (int)nc};
+  FwdArgs fa{q, k, v, g, beta, S0, nullptr, nullptr, states, inter, reinterpret_cast<unsigned char*>(x), scale,
+             N, T, H, HV, K, V, ctab, ctab + 2 * nc, (int)nc};
+  if (!bwd_tc_eligible(a, dtype) || !fwd_tc_eligible(fa, dtype))
+    return set_error(KDA_ERR_ARG, "kda_bwd_varlen: the tensor-core path needs 16-byte aligned q, k, v, dO, g, dq");
+  std::vector<int> host(tab);
+  host.insert(host.end(), seq0.begin(), seq0.end());
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(ws, host.data(), host.size() * sizeof(int), cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) return set_cuda_error("kda_bwd_varlen: chunk table upload", e);
+  if (!(flags & KDA_BWD_STATES_FROM_FWD)) {
+    rc = launch_fwd_tc(fa, st);
+    if (rc) return rc;
+  }
+  return launch_bwd(a, dtype, st);
 }
 
 int kda_decode_step(const void* q, const void* k, const void* v, const float* g,

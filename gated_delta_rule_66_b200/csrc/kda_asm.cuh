@@ -57,9 +57,10 @@ __device__ __forceinline__ void cumsum64(float* a, float* seg, const float* base
 }
 
 // One (chunk, quarter) with the CTA's 256 threads, shared memory at `smem`
-// (AsmSmem::bytes).  Ends with a barrier.
+// (AsmSmem::bytes): chunk ch of batch row sq (packed sequences: chunk ch of
+// the table, sq = 0).  Ends with a barrier.
 template <typename TIn>
-__device__ __forceinline__ void assemble_quarter(const BwdArgs& a, float* smem, int ch, int fq4, int hv, int b) {
+__device__ __forceinline__ void assemble_quarter(const BwdArgs& a, float* smem, int ch, int fq4, int hv, int sq) {
   using S = AsmSmem;
   constexpr int C = S::C, KQ = S::KQ, LDK = S::LDK, LDC = S::LDC, KD = 128;
   float *sK = smem + S::oK, *sQ = smem + S::oQ, *sC = smem + S::oC, *sDq = smem + S::oDq,
@@ -67,10 +68,11 @@ __device__ __forceinline__ void assemble_quarter(const BwdArgs& a, float* smem, 
         *sE2d = smem + S::oE2d, *sdA = smem + S::odA, *sdP = smem + S::odP, *sBeta = smem + S::oBeta,
         *sSeg = smem + S::oSeg, *sLast = smem + S::oLast;
   int* sFlag = reinterpret_cast<int*>(smem + S::oFlag);
-  const int G = a.HV / a.H, h = hv / G, T = a.T, NT = (T + C - 1) / C;
-  const int t0 = ch * C, L = min(C, T - t0), f0 = fq4 * KQ;
-  const size_t head = (size_t)b * a.HV + hv;
-  const float* rec = a.gws + (head * NT + ch) * GREC;
+  const int G = a.HV / a.H, h = hv / G, T = a.T, b = row_of(a, sq);
+  const int2 sp = chunk_span(a, ch);
+  const int t0 = sp.x, L = sp.y, f0 = fq4 * KQ;
+  const size_t gc = chunk_gc(a, sq, hv, ch);
+  const float* rec = a.gws + gc * GREC;
   const TIn* q = static_cast<const TIn*>(a.q);
   const TIn* k = static_cast<const TIn*>(a.k);
   const int tid = threadIdx.x;
@@ -143,7 +145,7 @@ __device__ __forceinline__ void assemble_quarter(const BwdArgs& a, float* smem, 
   cumsum64<false>(sC, sSeg, nullptr);
   if (fq4 == 0 && tid < L) {  // dbeta = dbeta_R + sum_{j<i} dA_ij Ah_ij (Ah read straight from the record)
     const int i = tid;
-    const float4* arow = reinterpret_cast<const float4*>(a.inter + (head * NT + ch) * INTER_REC + INTER_AH + i * 64);
+    const float4* arow = reinterpret_cast<const float4*>(a.inter + gc * INTER_REC + INTER_AH + i * 64);
     float s0 = rec[G_DBR + i], s1 = 0.f;
 #pragma unroll
     for (int j4 = 0; j4 < 16; ++j4) {

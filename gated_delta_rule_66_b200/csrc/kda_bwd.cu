@@ -422,8 +422,9 @@ static int launch_assemble(const BwdArgs& a, cudaStream_t stream) {
   auto kern = kda_bwd_assemble_kernel<TIn>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)AsmSmem::bytes);
   if (e != cudaSuccess) return set_cuda_error("kda_bwd: cudaFuncSetAttribute", e);
-  const int NT = (a.T + 63) / 64;
-  kern<<<dim3(NT * 4, a.HV, a.B), NTHREADS, AsmSmem::bytes, stream>>>(a);
+  const int NT = a.ctab ? a.NC : (a.T + 63) / 64;
+  if (NT == 0) return 0;  // (packed batches of empty sequences)
+  kern<<<dim3(NT * 4, a.HV, a.ctab ? 1 : a.B), NTHREADS, AsmSmem::bytes, stream>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return set_cuda_error("kda_bwd: assemble launch", e);
   return 0;
@@ -457,8 +458,9 @@ static int launch_bwd_t(const BwdArgs& a, cudaStream_t stream) {
   }
   if (a.HV > a.H) {
     const int G = a.HV / a.H;
-    const size_t rows_h = (size_t)a.B * a.T * a.H;
+    const size_t rows_h = (size_t)(a.ctab ? 1 : a.B) * a.T * a.H;
     const size_t n = rows_h * a.K;
+    if (n == 0) return 0;
     const int blocks = (int)((n + 255) / 256 < 148 * 16 ? (n + 255) / 256 : 148 * 16);
     kda_group_sum_kernel<TIn><<<blocks, 256, 0, stream>>>(a.dq_part, static_cast<TIn*>(a.dq), rows_h, a.H, G, a.K);
     kda_group_sum_kernel<TIn><<<blocks, 256, 0, stream>>>(a.dk_part, static_cast<TIn*>(a.dk), rows_h, a.H, G, a.K);

@@ -49,9 +49,10 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_dstate_tc_kernel(BwdArgs a) {
   const int tid = cx.tid, hcol = cx.hcol, Lr = cx.Lr;
   const uint32_t lo = cx.lo, sb = cx.sb;
 
-  const int hv = blockIdx.x, b = blockIdx.y;
-  const int G = a.HV / a.H, h = hv / G, T = a.T, NT = (T + C - 1) / C, NT32 = (T + 31) / 32;
-  const size_t head = (size_t)b * a.HV + hv;
+  const int hv = blockIdx.x, sq = blockIdx.y;  // batch row, or sequence of a packed batch
+  const int b = row_of(a, sq), c0 = chunk_begin(a, sq), c1 = chunk_end(a, sq);
+  const int G = a.HV / a.H, h = hv / G, T = a.T;
+  const size_t head = (size_t)sq * a.HV + hv;
   const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(a.q);
   const __nv_bfloat16* kg = static_cast<const __nv_bfloat16*>(a.k);
   const __nv_bfloat16* dog = static_cast<const __nv_bfloat16*>(a.dO);
@@ -85,9 +86,10 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_dstate_tc_kernel(BwdArgs a) {
   fence_before();
   __syncthreads();
 
-  for (int ch = NT - 1; ch >= 0; --ch) {
-    const int t0 = ch * C, L = min(C, T - t0);
-    const float* irec = a.inter + (head * NT + ch) * INTER_REC;  // P^T, T^T of this chunk (forward)
+  for (int ch = c1 - 1; ch >= c0; --ch) {
+    const int2 sp = chunk_span(a, ch);
+    const int t0 = sp.x, L = sp.y;
+    const float* irec = a.inter + chunk_gc(a, sq, hv, ch) * INTER_REC;  // P^T, T^T of this chunk (forward)
     load_raw_issue(cx, qg, kg, dog, a.g, a.beta, b, T, t0, L, a.H, a.HV, h, hv);
     if (!load_raw_wait(cx)) { failed = true; break; }
     cumsum_span(cx);
@@ -164,15 +166,13 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_dstate_tc_kernel(BwdArgs a) {
 
     // ---------------------------------------------------------------- store dM (leaving this chunk); start dM_in
     {
-      // index of the gradient of the state leaving this chunk in the 32-step
-      // layout (the last chunk may end inside its first half)
-      const int dm_idx = (2 * ch + 1 < NT32) ? 2 * ch + 1 : 2 * ch;
+      const size_t dm_slot = dstate_slot(a, sq, hv, ch);
       uint32_t r[32];
       for (int cb = 0; cb < 2; ++cb) {
         const int f0 = hcol * 64 + cb * 32;
         float s[32];
         tmem_ld32(tm + lo + TM_S + f0, s);
-        float* dst = a.dstates + ((head * NT32 + dm_idx) * KD + f0) * VD + Lr;
+        float* dst = a.dstates + (dm_slot * KD + f0) * VD + Lr;
 #pragma unroll
         for (int j = 0; j < 32; ++j) dst[(size_t)j * VD] = s[j];
 #pragma unroll
@@ -280,11 +280,13 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
   const int tid = cx.tid, hcol = cx.hcol, Lr = cx.Lr, lane = cx.lane;
   const uint32_t lo = cx.lo, sb = cx.sb;
 
-  const int ch = blockIdx.x, hv = blockIdx.y, b = blockIdx.z;
-  const int G = a.HV / a.H, h = hv / G, T = a.T, NT = (T + C - 1) / C, NT32 = (T + 31) / 32;
-  const int t0 = ch * C, L = min(C, T - t0);
-  const size_t head = (size_t)b * a.HV + hv;
-  float* rec = a.gws + (head * NT + ch) * GREC;
+  // chunk ch of batch row sq (packed sequences: chunk ch of the table, sq = 0)
+  const int ch = blockIdx.x, hv = blockIdx.y, sq = blockIdx.z;
+  const int G = a.HV / a.H, h = hv / G, T = a.T, b = row_of(a, sq);
+  const int2 sp = chunk_span(a, ch);
+  const int t0 = sp.x, L = sp.y;
+  const size_t gc = chunk_gc(a, sq, hv, ch);
+  float* rec = a.gws + gc * GREC;
   const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(a.q);
   const __nv_bfloat16* kg = static_cast<const __nv_bfloat16*>(a.k);
   const __nv_bfloat16* vg = static_cast<const __nv_bfloat16*>(a.v);
@@ -312,10 +314,9 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
 
   do {
     // ---------------------------------------------------------------- loads
-    const float* irec = a.inter + (head * NT + ch) * INTER_REC;  // P^T, T, T^T images of this chunk (forward)
-    const int dm_idx = (2 * ch + 1 < NT32) ? 2 * ch + 1 : 2 * ch;
-    const float* mst = a.states + (head * NT32 + 2 * ch) * (size_t)(KD * VD);  // M: state entering the chunk
-    const float* dmst = a.dstates + (head * NT32 + dm_idx) * (size_t)(KD * VD);  // dM: gradient of the leaving state
+    const float* irec = a.inter + gc * INTER_REC;  // P^T, T, T^T images of this chunk (forward)
+    const float* mst = a.states + state_slot(a, sq, hv, ch) * (KD * VD);     // M: state entering the chunk
+    const float* dmst = a.dstates + dstate_slot(a, sq, hv, ch) * (KD * VD);  // dM: gradient of the leaving state
     load_raw_issue(cx, qg, kg, dog, a.g, a.beta, b, T, t0, L, a.H, a.HV, h, hv);
     if (tid < 16) prefetch_l2(mst + tid * 1024, 4096);
     else if (tid < 32) prefetch_l2(dmst + (tid - 16) * 1024, 4096);
@@ -536,8 +537,9 @@ int launch_bwd_grads_tc(const BwdArgs& a, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(kda_bwd_grads_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)tcc::SMEM_BYTES);
   if (e != cudaSuccess) return set_cuda_error("kda_bwd: cudaFuncSetAttribute", e);
-  const int NT = (a.T + tcc::C - 1) / tcc::C;
-  kda_bwd_grads_tc_kernel<<<dim3(NT, a.HV, a.B), tcc::NTH, tcc::SMEM_BYTES, stream>>>(a);
+  const int NT = a.ctab ? a.NC : (a.T + tcc::C - 1) / tcc::C;
+  if (NT == 0) return 0;  // (packed batches of empty sequences)
+  kda_bwd_grads_tc_kernel<<<dim3(NT, a.HV, a.ctab ? 1 : a.B), tcc::NTH, tcc::SMEM_BYTES, stream>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return set_cuda_error("kda_bwd: tensor-core gradient launch", e);
   return 0;

@@ -193,12 +193,11 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_tc_kernel(FwdArgs a) {
   const int tid = cx.tid, hcol = cx.hcol, Lr = cx.Lr;
   const uint32_t lo = cx.lo, sb = cx.sb;
 
-  const int hv = blockIdx.x, s = blockIdx.y;  // s: batch row, or sequence of a packed batch
-  const SeqChunks sc(a, s);
+  const int hv = blockIdx.x, sq = blockIdx.y;  // batch row, or sequence of a packed batch
+  const SeqChunks sc(a, sq);
   const int b = sc.row;
   const int G = a.HV / a.H, h = hv / G, T = a.T, NT = (T + C - 1) / C;
-  const int NT32 = (T + 31) / 32;  // the state workspace holds the state entering every 32 steps
-  const size_t head = (size_t)s * a.HV + hv;
+  const size_t head = (size_t)sq * a.HV + hv;
   __nv_bfloat16* og = static_cast<__nv_bfloat16*>(a.o);
   float* sEl = reinterpret_cast<float*>(sm + S_EL);
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + S_BAR);
@@ -231,9 +230,9 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_tc_kernel(FwdArgs a) {
 
   for (int c = sc.c0; c < sc.c1; ++c) {
     const int2 sp = sc.span(a, c);
-    const int t0 = sp.x, L = sp.y, ch = c - sc.c0;  // (records and states: uniform batches only)
+    const int t0 = sp.x, L = sp.y, ch = c - sc.c0;
     const int Ln = c + 1 < sc.c1 ? sc.span(a, c + 1).y : 0;
-    float* irec = a.inter ? a.inter + (head * NT + ch) * INTER_REC : nullptr;
+    float* irec = a.inter ? a.inter + chunk_gc(a, sq, hv, c) * INTER_REC : nullptr;
     if (!fwd_chunk_head<NTH>(cx, a, b, hv, h, t0, L, Ln, irec, nullptr, bar, phase)) {
       failed = true;
       break;
@@ -273,7 +272,7 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_tc_kernel(FwdArgs a) {
         float s[32];
         tmem_ld32(tm + lo + TM_S + f0, s);
         if (a.states) {  // the state entering this chunk
-          float* dst = a.states + ((head * NT32 + 2 * ch) * KD + f0) * VD + Lr;
+          float* dst = a.states + (state_slot(a, sq, hv, sc.c0 + ch) * KD + f0) * VD + Lr;
 #pragma unroll
           for (int j = 0; j < 32; ++j) dst[(size_t)j * VD] = s[j];
         }
@@ -397,7 +396,7 @@ __global__ void __launch_bounds__(PREP_NT, 1) kda_fwd_prep_tc_kernel(FwdArgs a) 
     const int h = hv / G;
     if ((tid & 31) == 0 && tid < 96) bulk_wait_read();  // the previous item's image stores have left smem
     __syncthreads();
-    float* irec = a.inter ? a.inter + (size_t)item * INTER_REC : nullptr;  // (uniform batches only)
+    float* irec = a.inter ? a.inter + (size_t)item * INTER_REC : nullptr;  // (item = chunk_gc)
     unsigned char* img = a.img + (size_t)item * FWI_BYTES;
     if (!fwd_chunk_head<PREP_NT>(cx, a, b, hv, h, t0, L, 0, irec, img, bar, phase)) {
       failed = true;
@@ -464,12 +463,12 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_seq_tc_kernel(FwdArgs a) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, hcol = warp >> 2;
   const int Lr = (warp & 3) * 32 + lane;
   const uint32_t lo = (uint32_t)((warp & 3) * 32) << 16;
-  const int hv = blockIdx.x, s = blockIdx.y;  // s: batch row, or sequence of a packed batch
-  const SeqChunks sc(a, s);
+  const int hv = blockIdx.x, sq = blockIdx.y;  // batch row, or sequence of a packed batch
+  const SeqChunks sc(a, sq);
   const int b = sc.row, nch = sc.c1 - sc.c0;
-  const int T = a.T, NT = (T + tcc::C - 1) / tcc::C, NT32 = (T + 31) / 32;
+  const int T = a.T, NT = (T + tcc::C - 1) / tcc::C;
   constexpr int C = tcc::C, KD = tcc::KD, VD = tcc::VD;
-  const size_t head = (size_t)s * a.HV + hv;
+  const size_t head = (size_t)sq * a.HV + hv;
   // this sequence's chunk images, consecutive (the chunk kernel's item order)
   const unsigned char* imgs = a.img + (a.ctab ? (size_t)hv * a.NC + sc.c0 : head * NT) * (size_t)FWI_BYTES;
   __nv_bfloat16* og = static_cast<__nv_bfloat16*>(a.o);
@@ -549,7 +548,7 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_seq_tc_kernel(FwdArgs a) {
         float s[32];
         tmem_ld32(tm + lo + TM_S + f0, s);
         if (a.states) {
-          float* dst = a.states + ((head * NT32 + 2 * ch) * KD + f0) * VD + Lr;
+          float* dst = a.states + (state_slot(a, sq, hv, sc.c0 + ch) * KD + f0) * VD + Lr;
 #pragma unroll
           for (int j = 0; j < 32; ++j) dst[(size_t)j * VD] = s[j];
         }

@@ -41,6 +41,38 @@ constexpr unsigned FWI_A_BYTES = FWI_KEDT, FWI_B_BYTES = FWI_U0 - FWI_KEDT;
 constexpr int G_AH = 0, G_PA = 4096, G_QK = 12288, G_KED = 28672, G_DBR = 36864, G_DEL = 36928,
               GREC = 37120;
 
+// Chunk geometry of the tensor-core kernels (Args: FwdArgs or BwdArgs).
+// Uniform batches: sequence s = batch row, NT = ceil(T / 64) chunks each, the
+// state workspace in the 32-step layout [B, HV, ceil(T / 32), K, V].  Packed
+// sequences: the chunk table; one state slot per (value head, chunk).  gc is
+// the global index of a (sequence, value head, chunk) for the per-chunk
+// records, images and buffers.
+template <class Args>
+__device__ __forceinline__ int chunk_begin(const Args& a, int s) { return a.ctab ? a.seq0[s] : 0; }
+template <class Args>
+__device__ __forceinline__ int chunk_end(const Args& a, int s) { return a.ctab ? a.seq0[s + 1] : (a.T + 63) / 64; }
+template <class Args>
+__device__ __forceinline__ int row_of(const Args& a, int s) { return a.ctab ? 0 : s; }  // batch row of the tokens
+template <class Args>
+__device__ __forceinline__ int2 chunk_span(const Args& a, int c) {  // (first step, steps)
+  if (a.ctab) return make_int2(a.ctab[2 * c], a.ctab[2 * c + 1]);
+  return make_int2(c * 64, min(64, a.T - c * 64));
+}
+template <class Args>
+__device__ __forceinline__ size_t chunk_gc(const Args& a, int s, int hv, int c) {
+  return a.ctab ? (size_t)hv * a.NC + c : ((size_t)s * a.HV + hv) * ((a.T + 63) / 64) + c;
+}
+template <class Args>  // slot of the state entering chunk c
+__device__ __forceinline__ size_t state_slot(const Args& a, int s, int hv, int c) {
+  return a.ctab ? (size_t)hv * a.NC + c : ((size_t)s * a.HV + hv) * ((a.T + 31) / 32) + 2 * c;
+}
+template <class Args>  // slot of the gradient of the state leaving chunk c
+__device__ __forceinline__ size_t dstate_slot(const Args& a, int s, int hv, int c) {
+  if (a.ctab) return (size_t)hv * a.NC + c;
+  const int nt32 = (a.T + 31) / 32;
+  return ((size_t)s * a.HV + hv) * nt32 + (2 * c + 1 < nt32 ? 2 * c + 1 : 2 * c);
+}
+
 __host__ __device__ constexpr int rec_off(int r, int c, int n) {
   return r * n + ((((c >> 2) ^ (r & 7))) << 2) + (c & 3);
 }
@@ -76,6 +108,9 @@ struct BwdArgs {
   float* gws;                // per-chunk records of the tensor-core backward (K = V = 128), else null
   float scale;
   int B, T, H, HV, K, V;
+  const int* ctab;  // packed sequences, as in FwdArgs (null: uniform batch rows)
+  const int* seq0;
+  int NC;
 };
 
 struct DecodeArgs {

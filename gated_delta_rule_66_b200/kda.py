@@ -24,7 +24,7 @@ CHUNK = 32  # chunk length of the library's chunked kernels (workspace layout)
 
 SYMBOLS = ("kda_last_error", "kda_device_status", "kda_fwd_workspace_bytes", "kda_fwd_scratch_bytes",
            "kda_bwd_workspace_bytes", "kda_fwd", "kda_fwd_varlen_workspace_bytes", "kda_fwd_varlen",
-           "kda_decode_step", "kda_bwd")
+           "kda_bwd_varlen_workspace_bytes", "kda_bwd_varlen", "kda_decode_step", "kda_bwd")
 
 
 class KdaError(RuntimeError):
@@ -59,6 +59,11 @@ def _load():
     lib.kda_fwd_varlen.restype = i
     lib.kda_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, f, ctypes.POINTER(ctypes.c_int), i, i, i, i, i, i,
                                    vp, vp, vp, sz, vp]
+    lib.kda_bwd_varlen_workspace_bytes.restype = sz
+    lib.kda_bwd_varlen_workspace_bytes.argtypes = [ctypes.POINTER(ctypes.c_int), i, i, i, i, i]
+    lib.kda_bwd_varlen.restype = i
+    lib.kda_bwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, f, ctypes.POINTER(ctypes.c_int), i, i, i, i, i,
+                                   i, vp, vp, vp, vp, vp, vp, vp, sz, i, vp]
     lib.kda_decode_step.restype = i
     lib.kda_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, f, i, i, i, i, i, i, vp, vp]
     lib.kda_bwd.restype = i
@@ -199,6 +204,52 @@ def fwd_varlen(q, k, v, g, beta, cu_seqlens, scale=None, initial_state=None, out
                              workspace.numel() * workspace.element_size(), _stream())
     _check("kda_fwd_varlen", rc)
     return o, S_T
+
+
+def varlen_workspace_bytes(kind, cu_seqlens, H, HV, K, V):
+    """Workspace bytes for packed sequences: "fwd" (two-kernel forward scratch)
+    or "bwd" (the training workspace shared by fwd_varlen and bwd_varlen)."""
+    cu, N = _cu_array(cu_seqlens)
+    if kind == "fwd":
+        return int(_lib.kda_fwd_varlen_workspace_bytes(cu, N, HV, K, V))
+    return int(_lib.kda_bwd_varlen_workspace_bytes(cu, N, H, HV, K, V))
+
+
+def bwd_varlen(q, k, v, g, beta, dO, cu_seqlens, scale=None, initial_state=None, dS_T=None, workspace=None,
+               states_from_fwd=False):
+    """Backward of fwd_varlen.  Returns (dq, dk, dv, dg, dbeta, dS0 [N,HV,K,V]).
+    With ``states_from_fwd`` the ``workspace`` (of varlen_workspace_bytes("bwd"))
+    must have gone through fwd_varlen on the same inputs."""
+    T, H, K = q.shape
+    HV, V = v.shape[1], v.shape[2]
+    cu, N = _cu_array(cu_seqlens)
+    scale = 1.0 / math.sqrt(K) if scale is None else float(scale)
+    dt = q.dtype
+    for n, t in (("q", q), ("k", k), ("v", v), ("dO", dO)):
+        _req(n, t, dt, 3)
+    _req("g", g, torch.float32, 3)
+    _req("beta", beta, torch.float32, 2)
+    _req("initial_state", initial_state, torch.float32, 4)
+    _req("dS_T", dS_T, torch.float32, 4)
+    need = int(_lib.kda_bwd_varlen_workspace_bytes(cu, N, H, HV, K, V))
+    if workspace is None:
+        if states_from_fwd:
+            raise ValueError("states_from_fwd needs the workspace given to fwd_varlen")
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _req("workspace", workspace)
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(k)
+    dv = torch.empty_like(v)
+    dg = torch.empty_like(g)
+    dbeta = torch.empty_like(beta)
+    dS0 = torch.empty(N, HV, K, V, dtype=torch.float32, device=q.device)
+    rc = _lib.kda_bwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state), _ptr(dO),
+                             _ptr(dS_T), scale, cu, N, H, HV, K, V, _dtype_code(q), _ptr(dq), _ptr(dk), _ptr(dv),
+                             _ptr(dg), _ptr(dbeta), _ptr(dS0), _ptr(workspace),
+                             workspace.numel() * workspace.element_size(),
+                             KDA_BWD_STATES_FROM_FWD if states_from_fwd else 0, _stream())
+    _check("kda_bwd_varlen", rc)
+    return dq, dk, dv, dg, dbeta, dS0
 
 
 def decode_step(q, k, v, g, beta, state, scale=None, out=None):

@@ -132,11 +132,29 @@ int kda_fwd(const void* q, const void* k, const void* v, const float* g, const f
  *     least its chunk table (then one kernel per (sequence, value head)).
  * Runs on the tensor-core path only: bf16, K = V = 128, 16-byte aligned q, k,
  * v, g and o (KDA_ERR_ARG otherwise).  The chunk table is uploaded from the
- * host with one copy on `stream`. */
+ * host with one copy on `stream`.  A workspace of at least
+ * kda_bwd_varlen_workspace_bytes() bytes also receives the states and
+ * interaction records for a later kda_bwd_varlen with KDA_BWD_STATES_FROM_FWD. */
 size_t kda_fwd_varlen_workspace_bytes(const int* cu_seqlens, int N, int HV, int K, int V);
 int kda_fwd_varlen(const void* q, const void* k, const void* v, const float* g, const float* beta,
                    const float* S0, float scale, const int* cu_seqlens, int N, int H, int HV, int K, int V,
                    int dtype, void* o, float* S_T, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Backward of kda_fwd_varlen (per sequence the backward of kda_bwd, from its
+ * own dS_T to its own dS0).
+ *   inputs and cu_seqlens as kda_fwd_varlen; dO [T, HV, V] dtype; dS_T
+ *   [N, HV, K, V] float or NULL
+ *   dq, dk [T, H, K] dtype; dv [T, HV, V] dtype; dg [T, HV, K] float;
+ *   dbeta [T, HV] float; dS0 [N, HV, K, V] float or NULL
+ *   workspace: at least kda_bwd_varlen_workspace_bytes() bytes, 16-byte aligned
+ *   flags: 0 (the forward pass runs first) or KDA_BWD_STATES_FROM_FWD (the
+ *     workspace went through kda_fwd_varlen on the same inputs)
+ * Tensor-core path only (bf16, K = V = 128, 16-byte aligned q, k, v, dO, g, dq). */
+size_t kda_bwd_varlen_workspace_bytes(const int* cu_seqlens, int N, int H, int HV, int K, int V);
+int kda_bwd_varlen(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                   const float* S0, const void* dO, const float* dS_T, float scale, const int* cu_seqlens, int N,
+                   int H, int HV, int K, int V, int dtype, void* dq, void* dk, void* dv, float* dg, float* dbeta,
+                   float* dS0, void* workspace, size_t workspace_bytes, int flags, void* stream);
 
 /* One decode token on a state updated IN PLACE ("kimi_k3_host/kda.rs",
  * kda_recurrent_step, with the q/k L2 normalisation and the sigmoid of beta

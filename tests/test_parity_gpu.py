@@ -404,3 +404,49 @@ def test_fwd_varlen(kda, name, lens, H, HV, scratch):
     tol = tol_for(w.torch_dtype)
     report(f"varlen_{name} o", f64(o), o_ref, tol, w.torch_dtype)
     report(f"varlen_{name} S_T", f64(S), S_ref, tol, torch.float32)
+
+
+VARLEN_BWD_CASES = [
+    ("mixed_gqa", [5, 0, 130, 64, 1], 1, 2),
+    ("mha", [200, 70], 2, 2),
+]
+
+
+@pytest.mark.parametrize("name,lens,H,HV", VARLEN_BWD_CASES, ids=[c[0] for c in VARLEN_BWD_CASES])
+def test_bwd_varlen(kda, name, lens, H, HV):
+    """Backward of packed sequences against the oracle's backward run per
+    sequence (its own S0, dO and dS_T); the result with the forward's stored
+    states is bitwise the result of the backward's own forward pass."""
+    w, inp, S0 = _varlen_inputs(lens, H, HV, seed=11)
+    T = sum(lens)
+    gen = torch.Generator().manual_seed(13)
+    dO = torch.randn(T, HV, w.V, generator=gen).to(torch.bfloat16)
+    dS_T = torch.randn(len(lens), HV, w.K, w.V, generator=gen)
+    cu = [0]
+    for n in lens:
+        cu.append(cu[-1] + n)
+    d = {n: t.cuda() for n, t in inp.items() if t is not None}
+    args = (d["q"], d["k"], d["v"], d["g"], d["beta"])
+    got = kda.bwd_varlen(*args, dO.cuda(), cu, scale=w.scale, initial_state=S0.cuda(), dS_T=dS_T.cuda())
+    ws = torch.empty(kda.varlen_workspace_bytes("bwd", cu, H, HV, w.K, w.V), dtype=torch.uint8, device="cuda")
+    kda.fwd_varlen(*args, cu, scale=w.scale, initial_state=S0.cuda(), workspace=ws)
+    again = kda.bwd_varlen(*args, dO.cuda(), cu, scale=w.scale, initial_state=S0.cuda(), dS_T=dS_T.cuda(),
+                           workspace=ws, states_from_fwd=True)
+    torch.cuda.synchronize()
+    for x, y in zip(got, again):
+        assert torch.equal(x, y)
+    ref = [np.zeros(tuple(t.shape)) for t in got]
+    for s, (a0, a1) in enumerate(zip(cu[:-1], cu[1:])):
+        if a1 == a0:
+            ref[5][s] = f64(dS_T[s])
+            continue
+        sl = lambda t: f64(t[a0:a1].unsqueeze(0))
+        r = oracle.kda_backward(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]), sl(inp["g"]), sl(inp["beta"]), w.scale,
+                                f64(S0[s:s + 1]), sl(dO), f64(dS_T[s:s + 1]))
+        for n in range(5):
+            ref[n][a0:a1] = r[n][0]
+        ref[5][s] = r[5][0]
+    tol = tol_for(w.torch_dtype)
+    for n, x, r in zip(GRAD_NAMES, got, ref):
+        out_dtype = w.torch_dtype if n in ("dq", "dk", "dv") else torch.float32
+        report(f"varlen_{name} {n}", f64(x), r, tol, out_dtype)
