@@ -450,3 +450,32 @@ def test_bwd_varlen(kda, name, lens, H, HV):
     for n, x, r in zip(GRAD_NAMES, got, ref):
         out_dtype = w.torch_dtype if n in ("dq", "dk", "dv") else torch.float32
         report(f"varlen_{name} {n}", f64(x), r, tol, out_dtype)
+
+
+def test_varlen_prefill_then_decode(kda):
+    """Packed prefill hands each sequence's final state to batched decode: the
+    decoded outputs equal the oracle run on each sequence's prompt followed by
+    its decoded tokens."""
+    lens, H, HV, steps = [70, 0, 1, 128, 33], 2, 4, 3
+    N = len(lens)
+    w, inp, S0 = _varlen_inputs(lens, H, HV, seed=21)
+    cu = [0]
+    for n in lens:
+        cu.append(cu[-1] + n)
+    d = {n: t.cuda() for n, t in inp.items() if t is not None}
+    _, S = kda.fwd_varlen(d["q"], d["k"], d["v"], d["g"], d["beta"], cu, scale=w.scale, initial_state=S0.cuda())
+    dec_w = BY_NAME["decode"].with_sizes(B=N, H=H, HV=HV)
+    dec = [make_inputs(dec_w, seed=40 + t) for t in range(steps)]
+    outs = []
+    for t in range(steps):
+        outs.append(kda.decode_step(*(dec[t][n].cuda() for n in ("q", "k", "v", "g", "beta")), S, scale=w.scale))
+    torch.cuda.synchronize()
+    tol = tol_for(w.torch_dtype)
+    for s, (a0, a1) in enumerate(zip(cu[:-1], cu[1:])):
+        cat = {n: torch.cat([inp[n][a0:a1]] + [dec[t][n][s:s + 1] for t in range(steps)]).unsqueeze(0)
+               for n in ("q", "k", "v", "g", "beta")}
+        o_ref, S_ref = oracle.kda_forward(*(f64(cat[n]) for n in ("q", "k", "v", "g", "beta")), w.scale,
+                                          f64(S0[s:s + 1]))
+        got = torch.stack([outs[t][s] for t in range(steps)])
+        report(f"prefill_then_decode seq{s} o", f64(got), o_ref[0, a1 - a0:], tol, w.torch_dtype)
+        report(f"prefill_then_decode seq{s} S", f64(S[s]), S_ref[0], tol, torch.float32)
