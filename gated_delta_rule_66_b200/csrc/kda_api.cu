@@ -321,6 +321,115 @@ int kda_decode_step(const void* q, const void* k, const void* v, const float* g,
   return launch_decode(a, K, V, dtype, static_cast<cudaStream_t>(stream));
 }
 
+static int check_gate(const char* fn, const void* z, const float* A_log, const float* dt_bias, float lb,
+                      const float* beta_logit) {
+  char buf[256];
+  if (!z || !A_log || !dt_bias || !beta_logit) {
+    snprintf(buf, sizeof(buf), "%s: z, A_log, dt_bias and beta_logit must be non-NULL", fn);
+    return set_error(KDA_ERR_NULL, buf);
+  }
+  if (!(lb <= 0.f) || !isfinite(lb)) {
+    snprintf(buf, sizeof(buf), "%s: gate_lower_bound=%g must be finite and <= 0 (0: no bound)", fn, (double)lb);
+    return set_error(KDA_ERR_ARG, buf);
+  }
+  return KDA_OK;
+}
+
+static bool ranges_overlap(const void* a, size_t an, const void* b, size_t bn) {
+  const uintptr_t x = (uintptr_t)a, y = (uintptr_t)b;
+  return a && b && x < y + bn && y < x + an;
+}
+
+size_t kda_fwd_prep_workspace_bytes(int B, int T, int H, int HV, int K, int V, int dtype) {
+  if (B < 1 || T < 1 || H < 1 || HV < 1 || K < 1 || V < 1 || HV % H) return 0;
+  const size_t img = img_bytes(B, T, HV, K, V);
+  const size_t o32 = dtype == KDA_DTYPE_BF16 ? (size_t)B * T * HV * V * sizeof(float) : 0;
+  return img > o32 ? img : o32;
+}
+
+int kda_fwd_prep(const void* q, const void* k, const void* v, const void* z, const float* A_log,
+                 const float* dt_bias, float gate_lower_bound, const float* beta_logit, const void* out_gate,
+                 float out_eps, const float* S0, float scale, int B, int T, int H, int HV, int K, int V, int dtype,
+                 void* o, float* S_T, void* workspace, size_t workspace_bytes, void* stream) {
+  g_err[0] = 0;
+  int rc = check_common("kda_fwd_prep", B, T, H, HV, K, V, dtype, scale);
+  if (rc) return rc;
+  if (!q || !k || !v || !o) return set_error(KDA_ERR_NULL, "kda_fwd_prep: q, k, v and o must be non-NULL");
+  if ((rc = check_gate("kda_fwd_prep", z, A_log, dt_bias, gate_lower_bound, beta_logit))) return rc;
+  if (out_gate && (!(out_eps >= 0.f) || !isfinite(out_eps)))
+    return set_error(KDA_ERR_ARG, "kda_fwd_prep: out_eps must be finite and >= 0");
+  if (workspace && !aligned16(workspace))
+    return set_error(KDA_ERR_ARG, "kda_fwd_prep: workspace must be 16-byte aligned");
+  FwdArgs a{q, k, v, nullptr, beta_logit, S0, o, S_T, nullptr, nullptr, nullptr, scale, B, T, H, HV, K, V};
+  a.prep = PrepArgs{z, A_log, dt_bias, gate_lower_bound};
+  a.og = out_gate;
+  a.og_eps = out_eps;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (fwd_tc_eligible(a, dtype)) {
+    if (workspace && workspace_bytes >= img_bytes(B, T, HV, K, V)) a.img = static_cast<unsigned char*>(workspace);
+    return launch_fwd_tc(a, st);
+  }
+  if (out_gate) {  // the CUDA-core forward stores fp32 o for the gate pass (in place for fp32)
+    if (dtype == KDA_DTYPE_FP32) {
+      a.o32 = static_cast<float*>(o);
+    } else {
+      if (!workspace || workspace_bytes < (size_t)B * T * HV * V * sizeof(float))
+        return set_error(KDA_ERR_WORKSPACE, "kda_fwd_prep: the output gate of this shape needs "
+                                            "kda_fwd_prep_workspace_bytes() of workspace");
+      a.o32 = static_cast<float*>(workspace);
+    }
+  }
+  return launch_fwd_ffma(a, dtype, st);
+}
+
+int kda_short_conv(const void* xq, const void* xk, const void* xv, const float* w, const float* state_in,
+                   float* state_out, int B, int T, int H, int HV, int K, int V, int W, int dtype, void* q,
+                   void* k, void* v, void* stream) {
+  g_err[0] = 0;
+  int rc = check_common("kda_short_conv", B, T, H, HV, K, V, dtype, 1.f);
+  if (rc) return rc;
+  if (!xq || !xk || !xv || !w || !q || !k || !v)
+    return set_error(KDA_ERR_NULL, "kda_short_conv: xq, xk, xv, w, q, k and v must be non-NULL");
+  if (W < 1 || W > 8) return set_error(KDA_ERR_ARG, "kda_short_conv: W must be in 1..8");
+  const size_t cn = (size_t)2 * H * K + (size_t)HV * V, win = (size_t)B * cn * W * sizeof(float);
+  if (ranges_overlap(state_in, win, state_out, win))
+    return set_error(KDA_ERR_ARG, "kda_short_conv: state_out must not overlap state_in");
+  const size_t es = dtype == KDA_DTYPE_BF16 ? 2 : 4, nqk = (size_t)B * T * H * K * es, nv = (size_t)B * T * HV * V * es;
+  const void* ins[3] = {xq, xk, xv};
+  const void* outs[3] = {q, k, v};
+  const size_t ns[3] = {nqk, nqk, nv};
+  for (int i = 0; i < 3; ++i)
+    for (int j = 0; j < 3; ++j)
+      if (ranges_overlap(ins[i], ns[i], outs[j], ns[j]))
+        return set_error(KDA_ERR_ARG, "kda_short_conv: the outputs must not alias the inputs");
+  ConvArgs a{xq, xk, xv, w, state_in, state_out, q, k, v, B, T, H, HV, K, V, W};
+  return launch_short_conv(a, dtype, static_cast<cudaStream_t>(stream));
+}
+
+int kda_decode_token(const void* xq, const void* xk, const void* xv, const float* conv_w, const float* conv_in,
+                     float* conv_out, int W, const void* z, const float* A_log, const float* dt_bias,
+                     float gate_lower_bound, const float* beta_logit, const void* out_gate, float out_eps, float* S,
+                     float scale, int B, int H, int HV, int K, int V, int dtype, void* o, void* stream) {
+  g_err[0] = 0;
+  int rc = check_common("kda_decode_token", B, 1, H, HV, K, V, dtype, scale);
+  if (rc) return rc;
+  if (!xq || !xk || !xv || !conv_w || !conv_out || !S || !o)
+    return set_error(KDA_ERR_NULL, "kda_decode_token: xq, xk, xv, conv_w, conv_out, S and o must be non-NULL");
+  if ((rc = check_gate("kda_decode_token", z, A_log, dt_bias, gate_lower_bound, beta_logit))) return rc;
+  if (W < 1 || W > 8) return set_error(KDA_ERR_ARG, "kda_decode_token: W must be in 1..8");
+  if (out_gate && (!(out_eps >= 0.f) || !isfinite(out_eps)))
+    return set_error(KDA_ERR_ARG, "kda_decode_token: out_eps must be finite and >= 0");
+  if (!aligned16(S)) return set_error(KDA_ERR_ARG, "kda_decode_token: S must be 16-byte aligned");
+  const size_t win = (size_t)B * (2 * (size_t)H * K + (size_t)HV * V) * W * sizeof(float);
+  if (H != HV && ranges_overlap(conv_in, win, conv_out, win))
+    return set_error(KDA_ERR_ARG, "kda_decode_token: conv_out may overlap conv_in only when H == HV");
+  if (conv_in && conv_in != conv_out && ranges_overlap(conv_in, win, conv_out, win))
+    return set_error(KDA_ERR_ARG, "kda_decode_token: conv_out must equal conv_in or not overlap it");
+  DecodeTokenArgs a{xq, xk, xv, conv_w, conv_in, conv_out, PrepArgs{z, A_log, dt_bias, gate_lower_bound},
+                    beta_logit, out_gate, out_eps, S, o, scale, B, H, HV, W};
+  return launch_decode_token(a, K, V, dtype, static_cast<cudaStream_t>(stream));
+}
+
 int kda_bwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
             const float* S0, const void* dO, const float* dS_T, float scale, int B, int T, int H,
             int HV, int K, int V, int dtype, void* dq, void* dk, void* dv, float* dg,

@@ -43,6 +43,15 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float
   return __float2bfloat16_rn(x);
 }
 
+// ---- preparation math ("kimi_k3_host/kda.rs")
+constexpr float KDA_L2_EPS_F = 1e-6f;  // l2norm_rows: eps added to the sum of squares
+__device__ __forceinline__ float prep_sigmoid(float x) { return 1.f / (1.f + expf(-x)); }
+// bounded_gate: lb sigmoid(dec x) (lb < 0) or -dec softplus(x) (lb = 0), x = z + dt_bias, dec = e^{A_log}
+__device__ __forceinline__ float prep_gate(float x, float dec, float lb) {
+  if (lb != 0.f) return lb * prep_sigmoid(dec * x);
+  return -dec * (fmaxf(x, 0.f) + log1pf(expf(-fabsf(x))));
+}
+
 template <bool PRECISE>
 __device__ __forceinline__ float kexp(float x) {
   if constexpr (PRECISE) return expf(x); else return __expf(x);
@@ -79,30 +88,56 @@ __device__ __forceinline__ void zero(float (&acc)[TM][TN]) {
 // shared memory as fp32; rows past the sequence end are zero (a zero row has
 // no decay, no write and no read, so it leaves the state untouched).
 // Then replaces g by its in-chunk cumulative sum c.
+// With z (fused preparation, "kimi_k3_host/kda.rs"): q and k rows are
+// L2-normalised (l2norm_rows), g = prep_gate(z + dt_bias) (bounded_gate) and
+// beta = sigmoid(beta) (kda_recurrent_step takes the logit).
 template <int K, int C, typename TIn>
 __device__ __forceinline__ void load_chunk_qkgb(const TIn* __restrict__ q, const TIn* __restrict__ k,
                                                 const float* __restrict__ g,
                                                 const float* __restrict__ beta, float scale, int b,
                                                 int t0, int L, int T, int H, int HV, int h, int hv,
-                                                float* sQ, float* sK, float* sC, float* sBeta) {
+                                                float* sQ, float* sK, float* sC, float* sBeta,
+                                                const TIn* __restrict__ z = nullptr,
+                                                const float* __restrict__ A_log = nullptr,
+                                                const float* __restrict__ dt_bias = nullptr, float lb = 0.f) {
   constexpr int LDK = K + 1;
+  const bool prep = z != nullptr;
+  const float dec = prep ? expf(A_log[hv]) : 0.f;
   for (int idx = threadIdx.x; idx < C * K; idx += NTHREADS) {
     const int i = idx / K, f = idx % K;
     float qv = 0.f, kv = 0.f, gv = 0.f;
     if (i < L) {
       const size_t rq = ((size_t)b * T + t0 + i) * H + h;
       const size_t rg = ((size_t)b * T + t0 + i) * HV + hv;
-      qv = to_f(q[rq * K + f]) * scale;
+      qv = to_f(q[rq * K + f]) * (prep ? 1.f : scale);
       kv = to_f(k[rq * K + f]);
-      gv = g[rg * K + f];
+      gv = prep ? prep_gate(to_f(z[rg * K + f]) + dt_bias[(size_t)hv * K + f], dec, lb) : g[rg * K + f];
     }
     sQ[i * LDK + f] = qv;
     sK[i * LDK + f] = kv;
     sC[i * LDK + f] = gv;
   }
-  for (int i = threadIdx.x; i < C; i += NTHREADS)
-    sBeta[i] = (i < L) ? beta[((size_t)b * T + t0 + i) * HV + hv] : 0.f;
+  for (int i = threadIdx.x; i < C; i += NTHREADS) {
+    float bv = 0.f;
+    if (i < L) {
+      bv = beta[((size_t)b * T + t0 + i) * HV + hv];
+      if (prep) bv = prep_sigmoid(bv);
+    }
+    sBeta[i] = bv;
+  }
   __syncthreads();
+  if (prep) {  // row norms: one warp per row at a time, then q~ = scale q_hat
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int r = warp; r < 2 * C; r += NTHREADS / 32) {
+      float* row = (r < C ? sQ : sK) + (r % C) * LDK;
+      float s = 0.f;
+      for (int f = lane; f < K; f += 32) s = fmaf(row[f], row[f], s);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+      const float mul = rsqrtf(s + KDA_L2_EPS_F) * (r < C ? scale : 1.f);
+      for (int f = lane; f < K; f += 32) row[f] *= mul;
+    }
+  }
   for (int f = threadIdx.x; f < K; f += NTHREADS) {
     float run = 0.f;
     for (int i = 0; i < C; ++i) {

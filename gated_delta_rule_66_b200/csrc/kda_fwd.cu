@@ -64,7 +64,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
     }
     load_chunk_qkgb<K, C, TIn>(q, k, a.g, a.beta, a.scale, b, t0, L, T, a.H, a.HV, h, hv, sQ, sK,
-                               sC, sBeta);
+                               sC, sBeta, static_cast<const TIn*>(a.prep.z), a.prep.A_log, a.prep.dt_bias,
+                               a.prep.gate_lb);
     for (int idx = threadIdx.x; idx < C * VB; idx += NTHREADS) {
       const int i = idx / VB, n = idx % VB;
       sV[i * LDV + n] = (i < L) ? to_f(v[(((size_t)b * T + t0 + i) * a.HV + hv) * V + v0 + n]) : 0.f;
@@ -125,7 +126,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
         for (int y = 0; y < TNV; ++y) {
           const int i = ty + 16 * x, n = tx + 16 * y;
-          if (i < L) o[(((size_t)b * T + t0 + i) * a.HV + hv) * V + v0 + n] = from_f<TIn>(acc[x][y]);
+          if (i < L) {
+            const size_t at = (((size_t)b * T + t0 + i) * a.HV + hv) * V + v0 + n;
+            if (a.o32) a.o32[at] = acc[x][y];  // fp32 for the output-gate pass
+            else o[at] = from_f<TIn>(acc[x][y]);
+          }
         }
     }
     {  // M' = diag(e^{c_last}) M + (K o e^{c_last - c})^T U
@@ -176,12 +181,58 @@ int launch_fwd(const FwdArgs& a, int dtype, cudaStream_t stream) {
 
 int launch_fwd_ffma(const FwdArgs& a, int dtype, cudaStream_t stream) {
   const bool bf = dtype == 1;
+  int rc = 4;
   switch (a.K) {
-    case 32: return bf ? launch_fwd_t<32, __nv_bfloat16>(a, stream) : launch_fwd_t<32, float>(a, stream);
-    case 64: return bf ? launch_fwd_t<64, __nv_bfloat16>(a, stream) : launch_fwd_t<64, float>(a, stream);
-    case 128: return bf ? launch_fwd_t<128, __nv_bfloat16>(a, stream) : launch_fwd_t<128, float>(a, stream);
+    case 32: rc = bf ? launch_fwd_t<32, __nv_bfloat16>(a, stream) : launch_fwd_t<32, float>(a, stream); break;
+    case 64: rc = bf ? launch_fwd_t<64, __nv_bfloat16>(a, stream) : launch_fwd_t<64, float>(a, stream); break;
+    case 128: rc = bf ? launch_fwd_t<128, __nv_bfloat16>(a, stream) : launch_fwd_t<128, float>(a, stream); break;
+    default: return set_error(4, "kda_fwd: unsupported K");
   }
-  return set_error(4, "kda_fwd: unsupported K");
+  if (rc || !a.o || !a.o32) return rc;
+  // the output gate needs whole rows of V; the chunk kernel's CTAs own V slices
+  return launch_out_gate(a.o32, a.og, a.og_eps, (size_t)a.B * a.T * a.HV, a.V, dtype, a.o, stream);
+}
+
+// "kimi_k3_host/kda.rs", full_rank_output_gate: one warp per (step, value
+// head) row of V values: o = sigmoid(og) o32 / sqrt(mean(o32^2) + eps).
+template <typename TIn>
+__global__ void __launch_bounds__(256) kda_out_gate_kernel(const float* __restrict__ o32,
+                                                           const TIn* __restrict__ og, float eps, size_t rows,
+                                                           int V, TIn* __restrict__ o) {
+  const size_t row = (size_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const float* src = o32 + row * V;
+  float x[4], s = 0.f;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int n = lane + 32 * u;
+    x[u] = n < V ? src[n] : 0.f;
+    s = fmaf(x[u], x[u], s);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+  const float inv = rsqrtf(s / (float)V + eps);
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int n = lane + 32 * u;
+    if (n < V) o[row * V + n] = from_f<TIn>(x[u] * inv * prep_sigmoid(to_f(og[row * V + n])));
+  }
+}
+
+int launch_out_gate(const float* o32, const void* og, float eps, size_t rows, int V, int dtype, void* o,
+                    cudaStream_t stream) {
+  if (rows == 0) return 0;
+  const unsigned blocks = (unsigned)((rows + 7) / 8);
+  if (dtype == 1)
+    kda_out_gate_kernel<__nv_bfloat16><<<blocks, 256, 0, stream>>>(
+        o32, static_cast<const __nv_bfloat16*>(og), eps, rows, V, static_cast<__nv_bfloat16*>(o));
+  else
+    kda_out_gate_kernel<float><<<blocks, 256, 0, stream>>>(o32, static_cast<const float*>(og), eps, rows, V,
+                                                           static_cast<float*>(o));
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_cuda_error("kda_fwd: output-gate launch", e);
+  return 0;
 }
 
 size_t fwd_smem_bytes(int K) {

@@ -60,6 +60,26 @@ struct SeqChunks {
   }
 };
 
+// Output gate ("kimi_k3_host/kda.rs", full_rank_output_gate) on an O^T tile
+// read out of TMEM: warp w holds rows 32 (w / 4) + jj, jj < 32, of the value
+// columns 32 (w % 4) + lane.  Scales v[jj] by 1 / sqrt(mean_n o^2 + eps) of
+// its row (the sigmoid factor is the caller's); `red` is 256 free floats.
+// Two block barriers (256 threads).
+__device__ __forceinline__ void out_gate_rows(float (&v)[32], float* red, int warp, int lane, float eps) {
+  float sq[32];
+#pragma unroll
+  for (int jj = 0; jj < 32; ++jj) sq[jj] = v[jj] * v[jj];
+  const float part = tcc::warp_sum32(sq, lane);  // row 32 (warp / 4) + lane, this warp's 32 columns
+  red[((warp >> 2) * 32 + lane) * 4 + (warp & 3)] = part;
+  __syncthreads();
+#pragma unroll
+  for (int jj = 0; jj < 32; ++jj) {
+    const float4 r = *reinterpret_cast<const float4*>(red + ((warp >> 2) * 32 + jj) * 4);
+    v[jj] *= rsqrtf((r.x + r.y + r.z + r.w) * (1.f / 128.f) + eps);
+  }
+  __syncthreads();
+}
+
 // The state-independent part of one chunk: load, cumulative decay, the
 // interaction products and their read-out, the inverse T, the operands of the
 // state products (Q~ o e^c, (K o e^{c_last-c})^T in shared memory; e^{c_last}
@@ -72,7 +92,9 @@ struct SeqChunks {
 // b = 0 and t0 on the packed axis); with Ln > 0 the next chunk of the same
 // sequence (Ln steps from t0 + 64) is prefetched into L2.
 // Returns false, block-uniformly, if a tensor-core wait ran out.
-template <int NTHR>
+// With PREP the fused input preparation runs on the loaded chunk (FwdArgs::prep):
+// q, k rows L2-normalised, g from z, beta from its logit.
+template <int NTHR, bool PREP = false>
 __device__ __forceinline__ bool fwd_chunk_head(const tcc::Ctx& cx, const FwdArgs& a, int b, int hv, int h,
                                                int t0, int L, int Ln, float* irec,
                                                unsigned char* img, uint64_t* bar, uint32_t& phase) {
@@ -88,11 +110,23 @@ __device__ __forceinline__ bool fwd_chunk_head(const tcc::Ctx& cx, const FwdArgs
   const float* sBeta = cx.beta();
   float* sEl = reinterpret_cast<float*>(sm + S_EL);
   const float* sC = cx.c();
-  load_raw_issue<NTHR>(cx, qg, kg, vg, a.g, a.beta, b, T, t0, L, a.H, a.HV, h, hv);
-  if (Ln > 0) prefetch_chunk(cx, qg, kg, vg, a.g, b, T, t0 + C, Ln, a.H, a.HV, h, hv);
+  const __nv_bfloat16* zg = static_cast<const __nv_bfloat16*>(a.prep.z);
+  if constexpr (PREP) {
+    load_raw_issue_prep<NTHR>(cx, qg, kg, vg, zg, a.beta, b, T, t0, L, a.H, a.HV, h, hv);
+    if (Ln > 0) prefetch_chunk(cx, qg, kg, vg, zg, b, T, t0 + C, Ln, a.H, a.HV, h, hv, 2);
+  } else {
+    load_raw_issue<NTHR>(cx, qg, kg, vg, a.g, a.beta, b, T, t0, L, a.H, a.HV, h, hv);
+    if (Ln > 0) prefetch_chunk(cx, qg, kg, vg, a.g, b, T, t0 + C, Ln, a.H, a.HV, h, hv);
+  }
   if (!load_raw_wait(cx)) return false;
-  const bool wide = cumsum_span(cx);
-  build_op1_and_issue<NTHR>(cx, a.scale, tm + TM_APA, tm + TM_APB, bar);
+  bool wide;
+  if constexpr (PREP) {
+    row_norms<NTHR>(cx, a.scale);
+    wide = cumsum_span<true>(cx, a.prep.dt_bias + (size_t)hv * KD, expf(a.prep.A_log[hv]), a.prep.gate_lb, L);
+  } else {
+    wide = cumsum_span(cx);
+  }
+  build_op1_and_issue<NTHR, PREP>(cx, a.scale, tm + TM_APA, tm + TM_APB, bar);
   if (!wait_mma(bar, phase)) return false;
 
   // ---------------------------------------------------------------- state-product operands
@@ -101,10 +135,11 @@ __device__ __forceinline__ bool fwd_chunk_head(const tcc::Ctx& cx, const FwdArgs
     for (int m = 0; m < 2048 / NTHR; ++m) {
       const int i = item_row<NTHR>(cx, m);
       const float4 c4 = ld4(sC + i * LDCF + fq);
+      const float qs = PREP ? sC[i * LDCF + NORM_Q] : a.scale;
       float qf[4];
       bf16x4(sm + RAW_Q + raw_off(i, fq), qf);
-      st_tf32x4(sm, OP_QE + kmaj(i, fq, 128), a.scale * qf[0] * ex2(c4.x), a.scale * qf[1] * ex2(c4.y),
-                a.scale * qf[2] * ex2(c4.z), a.scale * qf[3] * ex2(c4.w));
+      st_tf32x4(sm, OP_QE + kmaj(i, fq, 128), qs * qf[0] * ex2(c4.x), qs * qf[1] * ex2(c4.y),
+                qs * qf[2] * ex2(c4.z), qs * qf[3] * ex2(c4.w));
     }
   }
   {  // transposed operands [f][i]: thread items of one channel x 4 rows, 16-byte stores
@@ -118,7 +153,8 @@ __device__ __forceinline__ bool fwd_chunk_head(const tcc::Ctx& cx, const FwdArgs
       for (int u = 0; u < 4; ++u) {
         const int i = i0 + u;
         const float c = sC[i * LDCF + f], bi = sBeta[i];
-        const float kk = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + RAW_K + raw_off(i, f)));
+        float kk = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + RAW_K + raw_off(i, f)));
+        if (PREP) kk *= sC[i * LDCF + NORM_K];
         bke[u] = bi * kk * ex2(c);
         ked[u] = kk * ex2(c63 - c);
         bv[u] = bi * __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + RAW_X + raw_off(i, f)));
@@ -130,7 +166,7 @@ __device__ __forceinline__ bool fwd_chunk_head(const tcc::Ctx& cx, const FwdArgs
     if (tid < KD) sEl[tid] = ex2(c63);
   }
   Pairwise pw;
-  if (wide) pairwise_compute(cx, a.scale, pw);
+  if (wide) pairwise_compute<PREP>(cx, a.scale, pw);
   if (img) fence_async_smem();
   __syncthreads();  // raw inputs consumed; the raw region is reused below
   if (img && (tid & 31) == 0 && tid < 96) {  // one bulk store per issuing warp
@@ -176,6 +212,7 @@ __device__ __forceinline__ bool fwd_chunk_head(const tcc::Ctx& cx, const FwdArgs
   return wait_mma(bar, phase);
 }
 
+template <bool PREP>
 __global__ void __launch_bounds__(256, 1) kda_fwd_tc_kernel(FwdArgs a) {
   using namespace tcf;
   using namespace tc;
@@ -233,7 +270,7 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_tc_kernel(FwdArgs a) {
     const int t0 = sp.x, L = sp.y, ch = c - sc.c0;
     const int Ln = c + 1 < sc.c1 ? sc.span(a, c + 1).y : 0;
     float* irec = a.inter ? a.inter + chunk_gc(a, sq, hv, c) * INTER_REC : nullptr;
-    if (!fwd_chunk_head<NTH>(cx, a, b, hv, h, t0, L, Ln, irec, nullptr, bar, phase)) {
+    if (!fwd_chunk_head<NTH, PREP>(cx, a, b, hv, h, t0, L, Ln, irec, nullptr, bar, phase)) {
       failed = true;
       break;
     }
@@ -299,6 +336,15 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_tc_kernel(FwdArgs a) {
     if (a.o) {
       float v[32];
       tmem_ld32(tm + lo + TM_O + hcol * 32, v);
+      if (a.og) {  // output gate; the raw region is free here (W and P are consumed)
+        const __nv_bfloat16* gate = static_cast<const __nv_bfloat16*>(a.og);
+        out_gate_rows(v, reinterpret_cast<float*>(sm + R_AH), cx.warp, cx.lane, a.og_eps);
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) {
+          const int i = hcol * 32 + jj;
+          if (i < L) v[jj] *= prep_sigmoid(__bfloat162float(gate[(((size_t)b * T + t0 + i) * a.HV + hv) * VD + Lr]));
+        }
+      }
 #pragma unroll
       for (int jj = 0; jj < 32; ++jj) {
         const int i = hcol * 32 + jj;
@@ -328,7 +374,7 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_tc_kernel(FwdArgs a) {
 bool fwd_tc_eligible(const FwdArgs& a, int dtype) {
   auto al16 = [](const void* p) { return ((uintptr_t)p & 15u) == 0; };
   return dtype == 1 && a.K == 128 && a.V == 128 && al16(a.q) && al16(a.k) && al16(a.v) && al16(a.g) &&
-         al16(a.o);
+         al16(a.o) && al16(a.prep.z) && al16(a.og);
 }
 
 // ============================================================================
@@ -343,6 +389,7 @@ bool fwd_tc_eligible(const FwdArgs& a, int dtype) {
 // ============================================================================
 constexpr int PREP_NT = 512;  // 16 warps: the chunk work is latency-bound, more warps hide it
 
+template <bool PREP>
 __global__ void __launch_bounds__(PREP_NT, 1) kda_fwd_prep_tc_kernel(FwdArgs a) {
   using namespace tcf;
   using namespace tc;
@@ -398,7 +445,7 @@ __global__ void __launch_bounds__(PREP_NT, 1) kda_fwd_prep_tc_kernel(FwdArgs a) 
     __syncthreads();
     float* irec = a.inter ? a.inter + (size_t)item * INTER_REC : nullptr;  // (item = chunk_gc)
     unsigned char* img = a.img + (size_t)item * FWI_BYTES;
-    if (!fwd_chunk_head<PREP_NT>(cx, a, b, hv, h, t0, L, 0, irec, img, bar, phase)) {
+    if (!fwd_chunk_head<PREP_NT, PREP>(cx, a, b, hv, h, t0, L, 0, irec, img, bar, phase)) {
       failed = true;
       break;
     }
@@ -436,9 +483,11 @@ __global__ void __launch_bounds__(PREP_NT, 1) kda_fwd_prep_tc_kernel(FwdArgs a) 
 namespace tcs {
 // shared memory of the sequential pass: two buffers for the first group of a
 // chunk's images (W, Q~ o e^c), one for the second ((K o e^{c_last-c})^T, P,
-// e^{c_last}), the bf16 output tile [i][n], then the barriers
+// e^{c_last}), the bf16 output tile [i][n], the output-gate tile [i][n] and
+// its row sums, then the barriers
 constexpr uint32_t SQ_A0 = 0, SQ_A1 = FWI_A_BYTES, SQ_B = 2 * FWI_A_BYTES, SQ_O = SQ_B + FWI_B_BYTES,
-                   SQ_BAR = SQ_O + 64 * 256, SQ_TMEM = SQ_BAR + 32, SQ_BYTES = SQ_TMEM + 16;
+                   SQ_G = SQ_O + 64 * 256, SQ_RED = SQ_G + 64 * 256, SQ_BAR = SQ_RED + 1024,
+                   SQ_TMEM = SQ_BAR + 32, SQ_BYTES = SQ_TMEM + 16;
 constexpr uint32_t B_KEDT = 0, B_P = FWI_P - FWI_KEDT, B_EL = FWI_EL - FWI_KEDT;
 static_assert(SQ_BYTES <= 232448 && SQ_O % 16 == 0, "shared memory budget");
 constexpr uint32_t TM_S = 0, TM_X = 128, TM_O = 192, TM_U = 256;
@@ -513,6 +562,14 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_seq_tc_kernel(FwdArgs a) {
     const int t0 = sp.x, L = sp.y;
     const unsigned char* img = imgs + (size_t)ch * FWI_BYTES;
     const uint32_t bufA = (ch & 1) ? SQ_A1 : SQ_A0;
+    if (a.og && a.o) {  // this chunk's output-gate rows (bf16 [i][n]), completed before the epilogue
+      const __nv_bfloat16* gate = static_cast<const __nv_bfloat16*>(a.og);
+      for (int x = tid; x < C * 16; x += 256) {
+        const int i = x >> 4, c16 = x & 15;
+        cp_async16(sb + SQ_G + x * 16, gate + (((size_t)b * T + t0 + (i < L ? i : 0)) * a.HV + hv) * VD + c16 * 8,
+                   i < L);
+      }
+    }
     if (tid == 32 && ch + 1 < nch) prefetch_l2(img + FWI_BYTES, FWI_BYTES);
     float u0[32];
     {
@@ -578,6 +635,13 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_seq_tc_kernel(FwdArgs a) {
       __nv_bfloat16* so = reinterpret_cast<__nv_bfloat16*>(sm + SQ_O);
       float v[32];
       tmem_ld32(tm + lo + TM_O + hcol * 32, v);
+      if (a.og) {  // output gate
+        cp_async_wait_all();
+        out_gate_rows(v, reinterpret_cast<float*>(sm + SQ_RED), warp, lane, a.og_eps);
+        const __nv_bfloat16* sg = reinterpret_cast<const __nv_bfloat16*>(sm + SQ_G);
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) v[jj] *= prep_sigmoid(__bfloat162float(sg[(hcol * 32 + jj) * VD + Lr]));
+      }
 #pragma unroll
       for (int jj = 0; jj < 32; ++jj) so[(hcol * 32 + jj) * VD + Lr] = __float2bfloat16_rn(v[jj]);
       __syncthreads();
@@ -609,9 +673,10 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_seq_tc_kernel(FwdArgs a) {
   if (failed && tid == 0) atomicOr(&g_kda_device_error, 1u);
 }
 
-int launch_fwd_tc(const FwdArgs& a, cudaStream_t stream) {
+template <bool PREP>
+static int launch_fwd_tc_t(const FwdArgs& a, cudaStream_t stream) {
   if (a.img) {  // two-kernel forward
-    cudaError_t e = cudaFuncSetAttribute(kda_fwd_prep_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(kda_fwd_prep_tc_kernel<PREP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)tcc::SMEM_BYTES);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(kda_fwd_seq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -621,7 +686,7 @@ int launch_fwd_tc(const FwdArgs& a, cudaStream_t stream) {
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (items > 0) {  // (packed batches of empty sequences have no chunks)
-      kda_fwd_prep_tc_kernel<<<min(items, sms), PREP_NT, tcc::SMEM_BYTES, stream>>>(a);
+      kda_fwd_prep_tc_kernel<PREP><<<min(items, sms), PREP_NT, tcc::SMEM_BYTES, stream>>>(a);
       e = cudaGetLastError();
       if (e != cudaSuccess) return set_cuda_error("kda_fwd: tensor-core chunk launch", e);
     }
@@ -630,13 +695,17 @@ int launch_fwd_tc(const FwdArgs& a, cudaStream_t stream) {
     if (e != cudaSuccess) return set_cuda_error("kda_fwd: tensor-core state-pass launch", e);
     return 0;
   }
-  cudaError_t e = cudaFuncSetAttribute(kda_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(kda_fwd_tc_kernel<PREP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)tcc::SMEM_BYTES);
   if (e != cudaSuccess) return set_cuda_error("kda_fwd: cudaFuncSetAttribute", e);
-  kda_fwd_tc_kernel<<<dim3(a.HV, a.B), tcc::NTH, tcc::SMEM_BYTES, stream>>>(a);
+  kda_fwd_tc_kernel<PREP><<<dim3(a.HV, a.B), tcc::NTH, tcc::SMEM_BYTES, stream>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return set_cuda_error("kda_fwd: tensor-core launch", e);
   return 0;
+}
+
+int launch_fwd_tc(const FwdArgs& a, cudaStream_t stream) {
+  return a.prep.z ? launch_fwd_tc_t<true>(a, stream) : launch_fwd_tc_t<false>(a, stream);
 }
 
 int take_device_error(unsigned* out) {

@@ -77,6 +77,20 @@ __host__ __device__ constexpr int rec_off(int r, int c, int n) {
   return r * n + ((((c >> 2) ^ (r & 7))) << 2) + (c & 3);
 }
 
+// Fused input preparation ("kimi_k3_host/kda.rs": l2norm_rows, bounded_gate,
+// and the sigmoid kda_recurrent_step applies to its beta input).  With z set:
+// q and k rows are L2-normalised (eps KDA_L2_EPS inside the root), g is
+// computed from z (the gate pre-activation, [rows, HV, K] in the input dtype)
+// as gate_lb * sigmoid(e^{A_log[hv]} (z + dt_bias[hv])) for gate_lb < 0 or
+// -e^{A_log[hv]} softplus(z + dt_bias[hv]) for gate_lb = 0, and beta holds
+// logits.
+struct PrepArgs {
+  const void* z;
+  const float* A_log;    // [HV]
+  const float* dt_bias;  // [HV, K]
+  float gate_lb;
+};
+
 struct FwdArgs {
   const void *q, *k, *v;
   const float *g, *beta, *S0;
@@ -94,6 +108,10 @@ struct FwdArgs {
   const int* ctab;
   const int* seq0;
   int NC;
+  PrepArgs prep;      // fused input preparation (prep.z null: inputs used as given)
+  const void* og;     // output-gate pre-activation [rows, HV, V] in the input dtype, or null
+  float og_eps;
+  float* o32;         // CUDA-core path with og: fp32 output scratch [rows, HV, V] for the gate pass
 };
 
 struct BwdArgs {
@@ -122,6 +140,35 @@ struct DecodeArgs {
   int B, H, HV;
 };
 
+// One decode token from the raw projections ("kimi_k3_host/kda.rs",
+// kda_decode_token): the short-convolution step on the q | k | v channels,
+// then the prepared recurrence step and the optional output gate.
+struct DecodeTokenArgs {
+  const void *xq, *xk, *xv;     // [B, H, K], [B, H, K], [B, HV, V]
+  const float* conv_w;          // [Cn, W], Cn = 2 H K + HV V
+  const float* conv_in;         // [B, Cn, W]
+  float* conv_out;              // [B, Cn, W] (may equal conv_in when H == HV)
+  PrepArgs prep;                // z [B, HV, K]
+  const float* beta;            // logits [B, HV]
+  const void* og;               // [B, HV, V] or null
+  float og_eps;
+  float* S;                     // [B, HV, K, V] in place
+  void* o;                      // [B, HV, V]
+  float scale;
+  int B, H, HV, W;
+};
+
+// The short causal convolution with SiLU over whole sequences
+// ("kimi_k3_host/kda.rs", conv_update applied to every step in order).
+struct ConvArgs {
+  const void *xq, *xk, *xv;     // [B, T, H, K], [B, T, H, K], [B, T, HV, V]
+  const float* w;               // [Cn, W]
+  const float* state_in;        // [B, Cn, W] or null (zeros)
+  float* state_out;             // [B, Cn, W] or null
+  void *q, *k, *v;              // outputs, shapes of the inputs, input dtype
+  int B, T, H, HV, K, V, W;
+};
+
 // error reporting (thread-local message; returns the code)
 int set_error(int code, const char* msg);
 int set_cuda_error(const char* where, cudaError_t e);
@@ -139,5 +186,10 @@ bool bwd_tc_eligible(const BwdArgs& a, int dtype);
 int launch_bwd_dstate_tc(const BwdArgs& a, cudaStream_t stream);
 int launch_bwd_grads_tc(const BwdArgs& a, cudaStream_t stream);
 int launch_decode(const DecodeArgs& a, int K, int V, int dtype, cudaStream_t stream);
+int launch_decode_token(const DecodeTokenArgs& a, int K, int V, int dtype, cudaStream_t stream);
+int launch_short_conv(const ConvArgs& a, int dtype, cudaStream_t stream);
+// the output-gate pass of the CUDA-core forward: o = gate(o32, og)
+int launch_out_gate(const float* o32, const void* og, float eps, size_t rows, int V, int dtype, void* o,
+                    cudaStream_t stream);
 
 }  // namespace kda

@@ -105,6 +105,54 @@ __device__ __forceinline__ void load_raw_issue(const Ctx& c, const __nv_bfloat16
   }
   if (c.tid < C) c.beta()[c.tid] = (c.tid < L) ? beta[((size_t)b * T + t0 + c.tid) * HV + hv] : 0.f;
 }
+// The same load for the fused preparation: z (the gate pre-activation, bf16)
+// instead of g, as packed rows at the stride of the cumulative-decay rows
+// (row i at RAW_C + i * LDCF * 4, so that the per-row norms in the padding
+// floats LDCF-4 .. of every row survive), and beta from its logit.
+template <int NT = NTH>
+__device__ __forceinline__ void load_raw_issue_prep(const Ctx& c, const __nv_bfloat16* q, const __nv_bfloat16* k,
+                                                    const __nv_bfloat16* x, const __nv_bfloat16* z,
+                                                    const float* beta_logit, int b, int T, int t0, int L, int H,
+                                                    int HV, int h, int hv) {
+  using namespace tc;
+  for (int e = c.tid; e < C * 16; e += NT) {
+    const int i = e >> 4, vec = e & 15;
+    const bool ok = i < L;
+    const size_t t = (size_t)b * T + t0 + (ok ? i : 0);
+    const uint32_t d = raw_off(i, vec * 8);
+    cp_async16(c.sb + RAW_Q + d, q + (t * H + h) * KD + vec * 8, ok);
+    cp_async16(c.sb + RAW_K + d, k + (t * H + h) * KD + vec * 8, ok);
+    cp_async16(c.sb + RAW_X + d, x + (t * HV + hv) * VD + vec * 8, ok);
+    cp_async16(c.sb + RAW_C + i * LDCF * 4 + vec * 16, z + (t * HV + hv) * KD + vec * 8, ok);
+  }
+  if (c.tid < C) c.beta()[c.tid] = (c.tid < L) ? prep_sigmoid(beta_logit[((size_t)b * T + t0 + c.tid) * HV + hv]) : 0.f;
+}
+
+// Per-row factors of the fused preparation ("kimi_k3_host/kda.rs",
+// l2norm_rows): scale / sqrt(|q_i|^2 + eps) and 1 / sqrt(|k_i|^2 + eps),
+// kept in the padding floats 128 and 129 of row i of the cumulative-decay
+// rows.  Run after load_raw_wait; cumsum_span's barriers publish them.
+constexpr int NORM_Q = 128, NORM_K = 129;
+template <int NT = NTH>
+__device__ __forceinline__ void row_norms(const Ctx& c, float scale) {
+  constexpr int P = NT / 128, PC = 16 / P;  // threads per row, 16-byte pieces per thread
+  const int r = c.tid / P, part = c.tid % P, i = r & 63;
+  const unsigned char* base = c.sm + (r < 64 ? RAW_Q : RAW_K);
+  float s = 0.f;
+#pragma unroll
+  for (int pc = 0; pc < PC; ++pc) {
+    float x[4];
+    const int f = (part * PC + pc) * 8;
+    bf16x4(base + raw_off(i, f), x);
+    s = fmaf(x[0], x[0], fmaf(x[1], x[1], fmaf(x[2], x[2], fmaf(x[3], x[3], s))));
+    bf16x4(base + raw_off(i, f) + 8, x);
+    s = fmaf(x[0], x[0], fmaf(x[1], x[1], fmaf(x[2], x[2], fmaf(x[3], x[3], s))));
+  }
+#pragma unroll
+  for (int off = 1; off < P; off <<= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+  if (part == 0) c.c()[i * LDCF + (r < 64 ? NORM_Q : NORM_K)] = rsqrtf(s + KDA_L2_EPS_F) * (r < 64 ? scale : 1.f);
+}
+
 // Completes load_raw_issue (wait + barrier).  Returns true (the form of a
 // bounded wait, for the callers' uniform error path).
 __device__ __forceinline__ bool load_raw_wait(const Ctx&) {
@@ -115,16 +163,17 @@ __device__ __forceinline__ bool load_raw_wait(const Ctx&) {
 
 // L2 prefetch of one chunk's q, k, x (v or dO) and g rows, for a chunk that a
 // later load_raw will read; one row of one tensor per thread.
+// (g_elem: bytes per element of the gate rows, 4 for g or 2 for bf16 z)
 __device__ __forceinline__ void prefetch_chunk(const Ctx& c, const __nv_bfloat16* q, const __nv_bfloat16* k,
-                                               const __nv_bfloat16* x, const float* g, int b, int T, int t0,
-                                               int L, int H, int HV, int h, int hv) {
+                                               const __nv_bfloat16* x, const void* g, int b, int T, int t0,
+                                               int L, int H, int HV, int h, int hv, int g_elem = 4) {
   const int i = c.tid & 63, which = c.tid >> 6;
   if (i >= L || which > 3) return;
   const size_t t = (size_t)b * T + t0 + i;
   if (which == 0) tc::prefetch_l2(q + (t * H + h) * KD, KD * 2);
   else if (which == 1) tc::prefetch_l2(k + (t * H + h) * KD, KD * 2);
   else if (which == 2) tc::prefetch_l2(x + (t * HV + hv) * VD, VD * 2);
-  else tc::prefetch_l2(g + (t * HV + hv) * KD, KD * 4);
+  else tc::prefetch_l2(static_cast<const unsigned char*>(g) + (t * HV + hv) * KD * g_elem, KD * g_elem);
 }
 
 // Asynchronous copy of one 64 x 64 operand image of an interaction record
@@ -158,17 +207,33 @@ __device__ __forceinline__ int img(int r, int k) { return (int)(tc::kmaj(r, k, 6
 // Returns, block-uniformly, whether some half's decay from its middle row to
 // either end exceeds 80 (the split exponents would then leave fp32 range).
 // (The first 256 threads do the sums, two row halves per channel.)
-__device__ __forceinline__ bool cumsum_span(const Ctx& c) {
+// With GATE (fused preparation) the rows hold z (bf16, load_raw_issue_prep)
+// and g = prep_gate(z + dt_bias) is formed here ("kimi_k3_host/kda.rs",
+// bounded_gate); rows at or past L count as g = 0 as in the plain load.
+template <bool GATE = false>
+__device__ __forceinline__ bool cumsum_span(const Ctx& c, const float* dt_bias_row = nullptr, float dec = 0.f,
+                                            float lb = 0.f, int L = C) {
   float* sC = c.c();
   float* sCarry = reinterpret_cast<float*>(c.sm + S_CARRY);
   const int f = c.tid & 127, hh = c.tid >> 7;
   float v[32];
   float run = 0.f;
   if (c.tid < 256) {
+    if constexpr (GATE) {
+      const __nv_bfloat16* zr = reinterpret_cast<const __nv_bfloat16*>(c.sm + RAW_C);
+      const float dtb = dt_bias_row[f];
 #pragma unroll
-    for (int r = 0; r < 32; ++r) {
-      run += sC[(hh * 32 + r) * LDCF + f];
-      v[r] = run;
+      for (int r = 0; r < 32; ++r) {
+        const int i = hh * 32 + r;
+        run += i < L ? prep_gate(__bfloat162float(zr[i * 2 * LDCF + f]) + dtb, dec, lb) : 0.f;
+        v[r] = run;
+      }
+    } else {
+#pragma unroll
+      for (int r = 0; r < 32; ++r) {
+        run += sC[(hh * 32 + r) * LDCF + f];
+        v[r] = run;
+      }
     }
     if (hh == 0) sCarry[f] = run;
   }
@@ -200,7 +265,8 @@ __device__ __forceinline__ int item_row(const Ctx& c, int m) { return m * (NT / 
 
 // Interaction operands into the operand region, then the two products on
 // the tensor cores (issued by thread 0, completion on `bar`).
-template <int NT = NTH>
+// (NORM: q, k rows times their row_norms factors; the q factor includes scale)
+template <int NT = NTH, bool NORM = false>
 __device__ __forceinline__ void build_op1_and_issue(const Ctx& c, float scale, uint32_t tm_apa,
                                                     uint32_t tm_apb, uint64_t* bar) {
   using namespace tc;
@@ -217,10 +283,12 @@ __device__ __forceinline__ void build_op1_and_issue(const Ctx& c, float scale, u
     bf16x4(c.sm + RAW_Q + raw_off(i, fq), qf);
     const float4 rr = (i < 32) ? r15 : r47;
     const float cr[4] = {rr.x, rr.y, rr.z, rr.w};
+    const float qmul = NORM ? sC[i * LDCF + NORM_Q] : scale;
     float xa[4], ya[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      qf[u] *= scale;
+      qf[u] *= qmul;
+      if (NORM) kf[u] *= sC[i * LDCF + NORM_K];
       xa[u] = ex2(cc[u] - cr[u]);
       ya[u] = ex2(cr[u] - cc[u]);
     }
@@ -269,6 +337,7 @@ struct Pairwise {
   float v[16];
   int kind, i, j0;
 };
+template <bool NORM = false>
 __device__ __forceinline__ void pairwise_compute(const Ctx& c, float scale, Pairwise& pw) {
   const float* sC = c.c();
   pw.kind = c.tid < 256 ? c.tid >> 7 : -1;  // the first 256 threads
@@ -288,7 +357,10 @@ __device__ __forceinline__ void pairwise_compute(const Ctx& c, float scale, Pair
         const float kj = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(c.sm + RAW_K + raw_off(j, f)));
         acc = fmaf(xv * kj, tc::ex2(sC[pw.i * LDCF + f] - sC[j * LDCF + f]), acc);
       }
-      if (pw.kind) acc *= scale;
+      if (NORM)
+        acc *= sC[pw.i * LDCF + (pw.kind ? NORM_Q : NORM_K)] * sC[j * LDCF + NORM_K];
+      else if (pw.kind)
+        acc *= scale;
     }
     pw.v[jj] = acc;
   }

@@ -140,6 +140,44 @@ def make_inputs(w: Workload, seed: int | None = None, with_do: bool | None = Non
     return out
 
 
+def make_raw_inputs(w: Workload, seed: int | None = None, conv_width: int = 0, lower_bound: float = -5.0):
+    """Draw the RAW projections of workload ``w`` for the fused-preparation
+    entry points (nothing normalised, no gate or sigmoid applied).
+
+    One CPU generator (default seed 20261202 + 100 + workload index), draws in
+    this order: q, k [B,T,H,K] and v [B,T,HV,V] ~ N(0, 1); gate noise z
+    [B,T,HV,K] ~ N(0, 1); beta logit [B,T,HV] ~ N(0, 1); A_log [HV] ~ U(-2, 0);
+    dt_bias [HV,K] ~ N(0, 0.1^2); output-gate pre-activation [B,T,HV,V] ~
+    N(0, 1); S0 as in ``make_inputs``; with ``conv_width`` W > 0 the
+    convolution weights [2HK + HV V, W] ~ N(0, 0.5^2) and an initial window
+    [B, 2HK + HV V, W] ~ N(0, 1).  q, k, v, z and the output gate are rounded
+    to the workload dtype; the rest stays fp32.  ``lower_bound`` is the gate's
+    (-5 for the production geometry, 0 = the unbounded softplus form).
+    """
+    if seed is None:
+        seed = SEED_BASE + 100 + w.index
+    gen = torch.Generator().manual_seed(seed)
+    B, T, H, HV, K, V = w.B, w.T, w.H, w.HV, w.K, w.V
+
+    def randn(*shape):
+        return torch.randn(*shape, generator=gen, dtype=torch.float32)
+
+    dt = w.torch_dtype
+    out = {
+        "q": randn(B, T, H, K).to(dt), "k": randn(B, T, H, K).to(dt), "v": randn(B, T, HV, V).to(dt),
+        "z": randn(B, T, HV, K).to(dt), "beta_logit": randn(B, T, HV),
+        "A_log": torch.rand(HV, generator=gen, dtype=torch.float32) * 2.0 - 2.0,
+        "dt_bias": randn(HV, K) * 0.1, "og": randn(B, T, HV, V).to(dt),
+        "S0": randn(B, HV, K, V) * w.s0_std if w.s0_std > 0 else None,
+        "lower_bound": float(lower_bound),
+    }
+    if conv_width:
+        Cn = 2 * H * K + HV * V
+        out["conv_w"] = randn(Cn, conv_width) * 0.5
+        out["conv_state"] = randn(B, Cn, conv_width)
+    return out
+
+
 def head_subset(inputs: dict, H: int, HV: int, groups):
     """Slice whole grouped-query blocks out of forward/backward inputs.
 

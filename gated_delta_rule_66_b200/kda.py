@@ -24,7 +24,8 @@ CHUNK = 32  # chunk length of the library's chunked kernels (workspace layout)
 
 SYMBOLS = ("kda_last_error", "kda_device_status", "kda_fwd_workspace_bytes", "kda_fwd_scratch_bytes",
            "kda_bwd_workspace_bytes", "kda_fwd", "kda_fwd_varlen_workspace_bytes", "kda_fwd_varlen",
-           "kda_bwd_varlen_workspace_bytes", "kda_bwd_varlen", "kda_decode_step", "kda_bwd")
+           "kda_bwd_varlen_workspace_bytes", "kda_bwd_varlen", "kda_decode_step", "kda_bwd",
+           "kda_fwd_prep_workspace_bytes", "kda_fwd_prep", "kda_short_conv", "kda_decode_token")
 
 
 class KdaError(RuntimeError):
@@ -69,6 +70,16 @@ def _load():
     lib.kda_bwd.restype = i
     lib.kda_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, f, i, i, i, i, i, i, i,
                             vp, vp, vp, vp, vp, vp, vp, sz, i, vp]
+    lib.kda_fwd_prep_workspace_bytes.restype = sz
+    lib.kda_fwd_prep_workspace_bytes.argtypes = [i, i, i, i, i, i, i]
+    lib.kda_fwd_prep.restype = i
+    lib.kda_fwd_prep.argtypes = [vp, vp, vp, vp, vp, vp, f, vp, vp, f, vp, f, i, i, i, i, i, i, i, vp, vp, vp, sz,
+                                 vp]
+    lib.kda_short_conv.restype = i
+    lib.kda_short_conv.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, vp, vp, vp, vp]
+    lib.kda_decode_token.restype = i
+    lib.kda_decode_token.argtypes = [vp, vp, vp, vp, vp, vp, i, vp, vp, vp, f, vp, vp, f, vp, f, i, i, i, i, i, i,
+                                     vp, vp]
     return lib
 
 
@@ -312,3 +323,105 @@ def bwd(q, k, v, g, beta, dO, scale=None, initial_state=None, dS_T=None, workspa
                       KDA_BWD_STATES_FROM_FWD if states_from_fwd else 0, _stream())
     _check("kda_bwd", rc)
     return dq, dk, dv, dg, dbeta, dS0
+
+
+# ----------------------------------------------------------------------------- preparation
+L2_EPS = 1e-6  # KDA_L2_EPS: q/k row normalisation
+
+
+def prep_workspace_bytes(B, T, H, HV, K, V, dtype=torch.bfloat16):
+    """Scratch bytes with which ``fwd_prep`` runs its fastest path for every shape."""
+    code = KDA_DTYPE_BF16 if dtype == torch.bfloat16 else KDA_DTYPE_FP32
+    return int(_lib.kda_fwd_prep_workspace_bytes(B, T, H, HV, K, V, code))
+
+
+def fwd_prep(q, k, v, z, A_log, dt_bias, beta_logit, gate_lower_bound=-5.0, scale=None, initial_state=None,
+             out_gate=None, out_eps=L2_EPS, output_final_state=True, workspace=True):
+    """Prefill from the raw projections (the preparation fused into the forward).
+
+    q, k [B,T,H,K] (before L2 normalisation), v [B,T,HV,V], z [B,T,HV,K] (gate
+    pre-activation) and out_gate [B,T,HV,V] (or None) share one dtype;
+    A_log [HV], dt_bias [HV,K], beta_logit [B,T,HV] float32.
+    ``gate_lower_bound`` < 0 selects the bounded gate, 0 the softplus form.
+    ``workspace``: True allocates the scratch, None runs without, or a
+    uint8 tensor.  Returns (o [B,T,HV,V], S_T or None).
+    """
+    B, T, H, K = q.shape
+    HV, V = v.shape[2], v.shape[3]
+    scale = 1.0 / math.sqrt(K) if scale is None else float(scale)
+    dt = q.dtype
+    for n, t in (("q", q), ("k", k), ("v", v), ("z", z)):
+        _req(n, t, dt, 4)
+    _req("out_gate", out_gate, dt, 4)
+    _req("A_log", A_log, torch.float32, 1)
+    _req("dt_bias", dt_bias, torch.float32, 2)
+    _req("beta_logit", beta_logit, torch.float32, 3)
+    _req("initial_state", initial_state, torch.float32, 4)
+    o = torch.empty(B, T, HV, V, dtype=dt, device=q.device)
+    S_T = torch.empty(B, HV, K, V, dtype=torch.float32, device=q.device) if output_final_state else None
+    if workspace is True:
+        n = prep_workspace_bytes(B, T, H, HV, K, V, dt)
+        workspace = torch.empty(n, dtype=torch.uint8, device=q.device) if n else None
+    rc = _lib.kda_fwd_prep(_ptr(q), _ptr(k), _ptr(v), _ptr(z), _ptr(A_log), _ptr(dt_bias), float(gate_lower_bound),
+                           _ptr(beta_logit), _ptr(out_gate), float(out_eps), _ptr(initial_state), scale,
+                           B, T, H, HV, K, V, _dtype_code(q), _ptr(o), _ptr(S_T), _ptr(workspace),
+                           0 if workspace is None else workspace.numel(), _stream())
+    _check("kda_fwd_prep", rc)
+    return o, S_T
+
+
+def short_conv(xq, xk, xv, w, state_in=None, output_state=True):
+    """The short causal convolution with SiLU over whole sequences.
+
+    xq, xk [B,T,H,K], xv [B,T,HV,V] (one dtype); w [2HK + HV V, W] float32;
+    state_in [B, 2HK + HV V, W] float32 or None.  Returns (q, k, v, state_out
+    or None).
+    """
+    B, T, H, K = xq.shape
+    HV, V = xv.shape[2], xv.shape[3]
+    W = w.shape[1]
+    dt = xq.dtype
+    for n, t in (("xq", xq), ("xk", xk), ("xv", xv)):
+        _req(n, t, dt, 4)
+    _req("w", w, torch.float32, 2)
+    _req("state_in", state_in, torch.float32, 3)
+    q, k, v = torch.empty_like(xq), torch.empty_like(xk), torch.empty_like(xv)
+    st = torch.empty(B, w.shape[0], W, dtype=torch.float32, device=xq.device) if output_state else None
+    rc = _lib.kda_short_conv(_ptr(xq), _ptr(xk), _ptr(xv), _ptr(w), _ptr(state_in), _ptr(st), B, T, H, HV, K, V,
+                             W, _dtype_code(xq), _ptr(q), _ptr(k), _ptr(v), _stream())
+    _check("kda_short_conv", rc)
+    return q, k, v, st
+
+
+def decode_token(xq, xk, xv, conv_w, conv_state, z, A_log, dt_bias, beta_logit, state, gate_lower_bound=-5.0,
+                 scale=None, out_gate=None, out_eps=L2_EPS, conv_out=None):
+    """One decode token from the raw projections; ``state`` [B,HV,K,V] and
+    (unless ``conv_out`` is given) ``conv_state`` [B, 2HK + HV V, W] are
+    updated in place (in place needs H == HV; pass ``conv_out`` otherwise).
+
+    xq, xk [B,H,K], xv [B,HV,V], z [B,HV,K], out_gate [B,HV,V] or None (one
+    dtype); conv_w [2HK + HV V, W], A_log [HV], dt_bias [HV,K], beta_logit
+    [B,HV] float32.  Returns o [B,HV,V].
+    """
+    B, H, K = xq.shape
+    HV, V = xv.shape[1], xv.shape[2]
+    scale = 1.0 / math.sqrt(K) if scale is None else float(scale)
+    dt = xq.dtype
+    for n, t in (("xq", xq), ("xk", xk), ("xv", xv), ("z", z)):
+        _req(n, t, dt, 3)
+    _req("out_gate", out_gate, dt, 3)
+    _req("conv_w", conv_w, torch.float32, 2)
+    _req("conv_state", conv_state, torch.float32, 3)
+    _req("conv_out", conv_out, torch.float32, 3)
+    _req("A_log", A_log, torch.float32, 1)
+    _req("dt_bias", dt_bias, torch.float32, 2)
+    _req("beta_logit", beta_logit, torch.float32, 2)
+    _req("state", state, torch.float32, 4)
+    o = torch.empty(B, HV, V, dtype=dt, device=xq.device)
+    out_win = conv_state if conv_out is None else conv_out
+    rc = _lib.kda_decode_token(_ptr(xq), _ptr(xk), _ptr(xv), _ptr(conv_w), _ptr(conv_state), _ptr(out_win),
+                               conv_w.shape[1], _ptr(z), _ptr(A_log), _ptr(dt_bias), float(gate_lower_bound),
+                               _ptr(beta_logit), _ptr(out_gate), float(out_eps), _ptr(state), scale, B, H, HV, K, V,
+                               _dtype_code(xq), _ptr(o), _stream())
+    _check("kda_decode_token", rc)
+    return o

@@ -185,6 +185,73 @@ int kda_bwd(const void* q, const void* k, const void* v, const float* g, const f
             float* dbeta, float* dS0, void* workspace, size_t workspace_bytes, int flags,
             void* stream);
 
+/* ---- The preparation around the recurrence ("kimi_k3_host/kda.rs").
+ * L2 normalisation of a q or k row: x / sqrt(sum x^2 + KDA_L2_EPS)
+ * (l2norm_rows, KDA_L2_EPS).  Decay gate from its pre-activation z
+ * (bounded_gate), x = z + dt_bias[hv], d = exp(A_log[hv]):
+ *     g = gate_lower_bound * sigmoid(d x)      gate_lower_bound < 0
+ *     g = -d * softplus(x)                     gate_lower_bound = 0 (no bound)
+ * beta = sigmoid(beta_logit) (kda_recurrent_step).  Output gate
+ * (full_rank_output_gate), per (step, value head) row of V values:
+ *     o <- sigmoid(out_gate) * o / sqrt(mean(o^2) + out_eps).
+ * Short convolution (conv_update): depthwise over the channels q | k | v
+ * (2 H K + HV V channels: the H K query channels, the H K key channels, then
+ * the HV V value channels, each tensor's own row-major order), weights
+ * w [channels, W] and window [B, channels, W] (oldest input first, newest in
+ * slot W - 1), y = SiLU(sum_j w[c][j] window[j]) after the window takes the
+ * new input; 1 <= W <= 8. */
+#define KDA_L2_EPS 1e-6f
+
+/* Prefill from the raw projections: kda_fwd with the preparation fused into
+ * its kernels (q, k normalised per row, g from z, beta from its logit) and
+ * the optional output gate applied to o before it is stored.
+ *   q, k [B, T, H, K] dtype (before normalisation); v [B, T, HV, V] dtype
+ *   z [B, T, HV, K] dtype; A_log [HV] float; dt_bias [HV, K] float
+ *   beta_logit [B, T, HV] float
+ *   out_gate [B, T, HV, V] dtype, or NULL for no output gate; out_eps >= 0
+ *   S0, S_T, o as kda_fwd (o is gated when out_gate is given)
+ *   workspace: NULL, or 16-byte aligned scratch; with at least
+ *     kda_fwd_prep_workspace_bytes() bytes every path runs (the two-kernel
+ *     tensor-core forward, and the CUDA-core forward's fp32 output for the
+ *     gate pass); with NULL the tensor-core path runs as one kernel per
+ *     (b, hv), and a CUDA-core bf16 shape with an output gate returns
+ *     KDA_ERR_WORKSPACE.
+ * No chunk states are stored (there is no backward of the preparation). */
+size_t kda_fwd_prep_workspace_bytes(int B, int T, int H, int HV, int K, int V, int dtype);
+int kda_fwd_prep(const void* q, const void* k, const void* v, const void* z, const float* A_log,
+                 const float* dt_bias, float gate_lower_bound, const float* beta_logit, const void* out_gate,
+                 float out_eps, const float* S0, float scale, int B, int T, int H, int HV, int K, int V, int dtype,
+                 void* o, float* S_T, void* workspace, size_t workspace_bytes, void* stream);
+
+/* The short convolution with SiLU over whole sequences (the prefill form of
+ * conv_update, applied to every step in order).
+ *   xq, xk [B, T, H, K] dtype; xv [B, T, HV, V] dtype (the projections)
+ *   w [2 H K + HV V, W] float; state_in [B, 2 H K + HV V, W] float or NULL
+ *   (zero window); state_out the same shape (the window after the last step)
+ *   or NULL; state_out must not overlap state_in
+ *   q, k, v outputs in the shapes and dtype of xq, xk, xv (the convolved
+ *   activations, rounded to dtype); they must not alias the inputs. */
+int kda_short_conv(const void* xq, const void* xk, const void* xv, const float* w, const float* state_in,
+                   float* state_out, int B, int T, int H, int HV, int K, int V, int W, int dtype, void* q,
+                   void* k, void* v, void* stream);
+
+/* One decode token from the raw projections ("kimi_k3_host/kda.rs",
+ * kda_decode_token, with bounded_gate and full_rank_output_gate): the
+ * convolution step, the preparation, the recurrence step on S IN PLACE and
+ * the optional output gate, in one launch.
+ *   xq, xk [B, H, K] dtype; xv [B, HV, V] dtype
+ *   conv_w [2 H K + HV V, W] float; conv_in [B, 2 H K + HV V, W] float or NULL
+ *   (zero window); conv_out the same shape, receives the new window; it may
+ *   equal conv_in only when H == HV (grouped heads share the q/k windows)
+ *   z [B, HV, K] dtype; A_log, dt_bias, gate_lower_bound as kda_fwd_prep
+ *   beta_logit [B, HV] float; out_gate [B, HV, V] dtype or NULL
+ *   S [B, HV, K, V] float, 16-byte aligned, read and overwritten
+ *   o [B, HV, V] dtype (output) */
+int kda_decode_token(const void* xq, const void* xk, const void* xv, const float* conv_w, const float* conv_in,
+                     float* conv_out, int W, const void* z, const float* A_log, const float* dt_bias,
+                     float gate_lower_bound, const float* beta_logit, const void* out_gate, float out_eps, float* S,
+                     float scale, int B, int H, int HV, int K, int V, int dtype, void* o, void* stream);
+
 /* Size in bytes of the fixed device array that kda_bwd_noalloc uses as its
  * scratch (64 MiB, held on every GPU that loads the library until exit). */
 #define KDA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)

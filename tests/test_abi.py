@@ -149,3 +149,56 @@ def test_varlen_workspace_and_validation(lib):
     assert rc == 5 and "workspace" in lib.kda_last_error().decode()
     rc = lib.kda_fwd_varlen(*args, cu, 3, 1, HV, 128, 128, 0, FAKE, None, FAKE, 1 << 40, None)  # fp32
     assert rc == 7 and "tensor-core" in lib.kda_last_error().decode()
+
+
+def test_prep_workspace_and_validation(lib):
+    B, T, H, HV = 2, 100, 1, 2
+    # tensor-core shape: the chunk images; a CUDA-core bf16 shape: the fp32 output for the gate pass
+    assert lib.kda_fwd_prep_workspace_bytes(B, T, H, HV, 128, 128, 1) == B * HV * 2 * 152064
+    assert lib.kda_fwd_prep_workspace_bytes(B, T, H, HV, 64, 32, 1) == B * T * HV * 32 * 4
+    assert lib.kda_fwd_prep_workspace_bytes(B, T, H, HV, 64, 32, 0) == 0
+    assert lib.kda_fwd_prep_workspace_bytes(B, T, 2, 3, 64, 32, 0) == 0  # HV % H != 0
+
+    def fwd_prep(**over):
+        a = dict(q=FAKE, k=FAKE, v=FAKE, z=FAKE, A_log=FAKE, dt=FAKE, lb=-5.0, bl=FAKE, og=None, eps=1e-6,
+                 S0=None, scale=0.5, B=1, T=8, H=1, HV=2, K=64, V=32, dtype=1, o=FAKE, S_T=None, ws=None,
+                 ws_bytes=0)
+        a.update(over)
+        return lib.kda_fwd_prep(a["q"], a["k"], a["v"], a["z"], a["A_log"], a["dt"], a["lb"], a["bl"], a["og"],
+                                a["eps"], a["S0"], a["scale"], a["B"], a["T"], a["H"], a["HV"], a["K"], a["V"],
+                                a["dtype"], a["o"], a["S_T"], a["ws"], a["ws_bytes"], None)
+
+    assert fwd_prep(z=None) == 1 and "z, A_log" in lib.kda_last_error().decode()
+    assert fwd_prep(lb=0.5) == 7 and "gate_lower_bound" in lib.kda_last_error().decode()
+    assert fwd_prep(lb=float("nan")) == 7
+    assert fwd_prep(og=FAKE, eps=-1.0) == 7 and "out_eps" in lib.kda_last_error().decode()
+    assert fwd_prep(og=FAKE) == 5 and "workspace" in lib.kda_last_error().decode()  # bf16 gate pass, no scratch
+    assert fwd_prep(ws=ctypes.c_void_p(0x1004), ws_bytes=1 << 30) == 7
+    assert fwd_prep(K=48) == 4
+
+    def conv(**over):
+        a = dict(xq=FAKE, xk=FAKE, xv=FAKE, w=FAKE, si=None, so=None, B=1, T=8, H=1, HV=2, K=32, V=32, W=4,
+                 dtype=1, q=ctypes.c_void_p(0x100000), k=ctypes.c_void_p(0x200000), v=ctypes.c_void_p(0x300000))
+        a.update(over)
+        return lib.kda_short_conv(a["xq"], a["xk"], a["xv"], a["w"], a["si"], a["so"], a["B"], a["T"], a["H"],
+                                  a["HV"], a["K"], a["V"], a["W"], a["dtype"], a["q"], a["k"], a["v"], None)
+
+    assert conv(W=0) == 7 and conv(W=9) == 7
+    assert conv(si=ctypes.c_void_p(0x400000), so=ctypes.c_void_p(0x400040)) == 7
+    assert "overlap" in lib.kda_last_error().decode()
+    assert conv(q=FAKE) == 7 and "alias" in lib.kda_last_error().decode()
+    assert conv(w=None) == 1
+
+    def tok(**over):
+        a = dict(xq=FAKE, xk=FAKE, xv=FAKE, cw=FAKE, ci=ctypes.c_void_p(0x400000), co=ctypes.c_void_p(0x400000),
+                 W=4, z=FAKE, A_log=FAKE, dt=FAKE, lb=-5.0, bl=FAKE, og=None, eps=1e-6, S=FAKE, scale=0.5, B=1,
+                 H=1, HV=2, K=32, V=32, dtype=1, o=FAKE)
+        a.update(over)
+        return lib.kda_decode_token(a["xq"], a["xk"], a["xv"], a["cw"], a["ci"], a["co"], a["W"], a["z"],
+                                    a["A_log"], a["dt"], a["lb"], a["bl"], a["og"], a["eps"], a["S"], a["scale"],
+                                    a["B"], a["H"], a["HV"], a["K"], a["V"], a["dtype"], a["o"], None)
+
+    assert tok() == 7 and "H == HV" in lib.kda_last_error().decode()  # grouped heads share the q/k windows
+    assert tok(S=ctypes.c_void_p(0x1008), H=2) == 7 and "aligned" in lib.kda_last_error().decode()
+    assert tok(co=None) == 1
+    assert tok(W=12, H=2) == 7
