@@ -34,10 +34,13 @@ sys.path.insert(0, ROOT)
 
 import torch  # noqa: E402
 
-from gated_delta_rule_66_b200.inputs import BY_NAME, make_inputs  # noqa: E402
+from gated_delta_rule_66_b200.inputs import BY_NAME, make_inputs, make_raw_inputs  # noqa: E402
 
 HEADLINE = "fwdbwd"
-PATHS = ("twin", "prefill_gqa", "fwdbwd", "decode")
+PATHS = ("twin", "prefill_gqa", "fwdbwd", "decode", "prefill_prep", "decode_token")
+# paths from the raw projections (fused preparation): workload they take their sizes from
+PREP_PATHS = {"prefill_prep": "prefill_gqa", "decode_token": "decode"}
+CONV_W = 4  # the host model's short-convolution width
 METRIC = "KDA tokens/s at 1 B200 (prefill fwd, fwd+bwd, decode) + % of roofline"
 L2_BYTES = 126 * 2 ** 20
 
@@ -74,6 +77,21 @@ def algorithmic_bytes(w, kind):
     if kind == "bwd":
         return bwd
     return fwd_in + fwd_out + s0 + bwd
+
+
+def prep_algorithmic_bytes(w, kind):
+    """Bytes of the raw-projection paths: prefill_prep reads q, k, v, z, the
+    output gate (input dtype) and the beta logits, writes o and S_T;
+    decode_token also reads and writes the state and the convolution window
+    (fp32) and reads the convolution weights."""
+    B, T, H, HV, K, V, e = w.B, w.T, w.H, w.HV, w.K, w.V, esize(w)
+    state = B * HV * K * V * 4
+    per_tok = 2 * H * K * e + HV * V * e + HV * K * e + HV * V * e + HV * 4 + HV * V * e
+    small = HV * 4 + HV * K * 4  # A_log, dt_bias
+    if kind == "prefill_prep":
+        return B * T * per_tok + state + small
+    Cn = 2 * H * K + HV * V
+    return B * per_tok + 2 * state + 2 * B * Cn * CONV_W * 4 + Cn * CONV_W * 4 + small
 
 
 def chunk_flops_per_head_token(K, V, C):
@@ -152,8 +170,62 @@ def host_inputs(w):
     return _HOST_INPUTS[w.name]
 
 
+def gpu_prep_path(kda, name, steps, warmup, rank_barrier):
+    """Times a raw-projection path: the prefill with the preparation and
+    output gate fused (kda_fwd_prep, production prefill geometry) or the
+    decode token (kda_decode_token: convolution step, preparation,
+    recurrence, output gate; production decode geometry)."""
+    w = BY_NAME[PREP_PATHS[name]].with_sizes(name=name, s0_std=0.0)  # (decode_token draws its own state)
+    dev = torch.device("cuda")
+    stream = torch.cuda.current_stream()
+    if name == "prefill_prep":
+        r = make_raw_inputs(w)
+        d = {n: (t.to(dev) if isinstance(t, torch.Tensor) else t) for n, t in r.items()}
+        ws = torch.empty(kda.prep_workspace_bytes(w.B, w.T, w.H, w.HV, w.K, w.V, w.torch_dtype), dtype=torch.uint8,
+                         device=dev)
+
+        def step():
+            kda.fwd_prep(d["q"], d["k"], d["v"], d["z"], d["A_log"], d["dt_bias"], d["beta_logit"], scale=w.scale,
+                         out_gate=d["og"], workspace=ws)
+        tokens, launches = w.B * w.T, 2
+        kernel = "kda_fwd_prep (kda_fwd_prep_tc_kernel<true> + kda_fwd_seq_tc_kernel, one call)"
+        flush = None
+    else:
+        r = make_raw_inputs(w.with_sizes(T=1), conv_width=CONV_W)
+        d = {n: (t[:, 0].contiguous().to(dev) if isinstance(t, torch.Tensor) and t.dim() >= 3 and n != "conv_state"
+                 else (t.to(dev) if isinstance(t, torch.Tensor) else t)) for n, t in r.items()}
+        S = torch.randn(w.B, w.HV, w.K, w.V, generator=torch.Generator().manual_seed(3)).mul_(0.02).to(dev)
+        flush = None  # state and windows (1.8 GB) exceed L2
+
+        def step():
+            kda.decode_token(d["q"], d["k"], d["v"], d["conv_w"], d["conv_state"], d["z"], d["A_log"],
+                             d["dt_bias"], d["beta_logit"], S, scale=w.scale, out_gate=d["og"])
+        tokens, launches = w.B, 1
+        kernel = "kda_decode_token_kernel"
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    rank_barrier()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1) / steps
+    byts = prep_algorithmic_bytes(w, name)
+    hbm = load_peaks()["hbm_gbs"]
+    res = {"workload": name, "ms_per_step": ms, "tokens_per_step": tokens, "launches_per_step": launches,
+           "l2": "inputs > L2", "calls": {"kernel_ms": ms}, "e2e_ms": None,
+           "roofline": {"bound": "hbm", "kernel": kernel, "achieved": byts / (ms * 1e-3) / 1e9, "peak": hbm,
+                        "unit": "GB/s", "frac": byts / (ms * 1e-3) / 1e9 / hbm, "algorithmic_bytes": byts}}
+    return res, w
+
+
 def gpu_path(kda, name, steps, warmup, rank_barrier, shrink=None):
     """Times one workload on this rank's GPU.  Returns a result dict."""
+    if name in PREP_PATHS:
+        return gpu_prep_path(kda, name, steps, warmup, rank_barrier)
     w = BY_NAME[name]
     if shrink:  # a smaller batch and length of the same workload (profiler captures only)
         w = w.with_sizes(name=f"{name}_B{shrink[0]}_T{shrink[1]}", B=shrink[0], T=shrink[1])
@@ -345,7 +417,8 @@ def run_gpu(args):
             res["clocks"] = clk.summary()
         else:
             res, w = gpu_path(kda, name, args.steps, args.warmup, barrier)
-        res["roofline"] = roofline_for(res, w, peaks)
+        if "roofline" not in res:
+            res["roofline"] = roofline_for(res, w, peaks)
         ms = res["ms_per_step"]
         if world > 1:
             t = torch.tensor([ms], device="cuda")
@@ -353,7 +426,8 @@ def run_gpu(args):
             ms = float(t.item())
             res["ms_per_step"] = ms
         res["tokens_per_s"] = res["tokens_per_step"] * world / (ms * 1e-3)
-        res["e2e_tokens_per_s"] = res["tokens_per_step"] * world / (res["e2e_ms"] * 1e-3)
+        res["e2e_tokens_per_s"] = (res["tokens_per_step"] * world / (res["e2e_ms"] * 1e-3)
+                                   if res["e2e_ms"] else None)
         results[name] = (res, w)
         torch.cuda.empty_cache()
 

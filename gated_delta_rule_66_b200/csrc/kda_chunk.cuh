@@ -52,6 +52,19 @@ __device__ __forceinline__ float prep_gate(float x, float dec, float lb) {
   return -dec * (fmaxf(x, 0.f) + log1pf(expf(-fabsf(x))));
 }
 
+// The same with the fast exp / reciprocal / log (absolute error of g ~1e-7;
+// the bf16 tensor-core paths, whose bar is 2e-3)
+__device__ __forceinline__ float rcp_approx(float x) {  // hardware reciprocal; rcp(+inf) = +0
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ float prep_sigmoid_fast(float x) { return rcp_approx(1.f + __expf(-x)); }
+__device__ __forceinline__ float prep_gate_fast(float x, float dec, float lb) {
+  if (lb != 0.f) return lb * prep_sigmoid_fast(dec * x);
+  return -dec * (fmaxf(x, 0.f) + __logf(1.f + __expf(-fabsf(x))));
+}
+
 template <bool PRECISE>
 __device__ __forceinline__ float kexp(float x) {
   if constexpr (PRECISE) return expf(x); else return __expf(x);

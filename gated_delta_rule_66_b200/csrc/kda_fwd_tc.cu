@@ -63,8 +63,9 @@ struct SeqChunks {
 // Output gate ("kimi_k3_host/kda.rs", full_rank_output_gate) on an O^T tile
 // read out of TMEM: warp w holds rows 32 (w / 4) + jj, jj < 32, of the value
 // columns 32 (w % 4) + lane.  Scales v[jj] by 1 / sqrt(mean_n o^2 + eps) of
-// its row (the sigmoid factor is the caller's); `red` is 256 free floats.
-// Two block barriers (256 threads).
+// its row (the sigmoid factor is the caller's); `red` is 256 floats that
+// nothing else touches until a later block barrier.  One block barrier
+// (256 threads).
 __device__ __forceinline__ void out_gate_rows(float (&v)[32], float* red, int warp, int lane, float eps) {
   float sq[32];
 #pragma unroll
@@ -77,7 +78,6 @@ __device__ __forceinline__ void out_gate_rows(float (&v)[32], float* red, int wa
     const float4 r = *reinterpret_cast<const float4*>(red + ((warp >> 2) * 32 + jj) * 4);
     v[jj] *= rsqrtf((r.x + r.y + r.z + r.w) * (1.f / 128.f) + eps);
   }
-  __syncthreads();
 }
 
 // The state-independent part of one chunk: load, cumulative decay, the
@@ -111,8 +111,11 @@ __device__ __forceinline__ bool fwd_chunk_head(const tcc::Ctx& cx, const FwdArgs
   float* sEl = reinterpret_cast<float*>(sm + S_EL);
   const float* sC = cx.c();
   const __nv_bfloat16* zg = static_cast<const __nv_bfloat16*>(a.prep.z);
+  float dtb = 0.f, dec = 0.f;  // gate constants, loaded while the chunk's copies are in flight
   if constexpr (PREP) {
     load_raw_issue_prep<NTHR>(cx, qg, kg, vg, zg, a.beta, b, T, t0, L, a.H, a.HV, h, hv);
+    dtb = a.prep.dt_bias[(size_t)hv * KD + (tid & 127)];
+    dec = a.prep.A_log[hv];
     if (Ln > 0) prefetch_chunk(cx, qg, kg, vg, zg, b, T, t0 + C, Ln, a.H, a.HV, h, hv, 2);
   } else {
     load_raw_issue<NTHR>(cx, qg, kg, vg, a.g, a.beta, b, T, t0, L, a.H, a.HV, h, hv);
@@ -122,7 +125,7 @@ __device__ __forceinline__ bool fwd_chunk_head(const tcc::Ctx& cx, const FwdArgs
   bool wide;
   if constexpr (PREP) {
     row_norms<NTHR>(cx, a.scale);
-    wide = cumsum_span<true>(cx, a.prep.dt_bias + (size_t)hv * KD, expf(a.prep.A_log[hv]), a.prep.gate_lb, L);
+    wide = cumsum_span<true, NTHR>(cx, dtb, expf(dec), a.prep.gate_lb, L);
   } else {
     wide = cumsum_span(cx);
   }
@@ -342,7 +345,7 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_tc_kernel(FwdArgs a) {
 #pragma unroll
         for (int jj = 0; jj < 32; ++jj) {
           const int i = hcol * 32 + jj;
-          if (i < L) v[jj] *= prep_sigmoid(__bfloat162float(gate[(((size_t)b * T + t0 + i) * a.HV + hv) * VD + Lr]));
+          if (i < L) v[jj] *= prep_sigmoid_fast(__bfloat162float(gate[(((size_t)b * T + t0 + i) * a.HV + hv) * VD + Lr]));
         }
       }
 #pragma unroll
@@ -615,6 +618,8 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_seq_tc_kernel(FwdArgs a) {
       }
       tmem_wait_st();
     }
+    const bool gated = a.og && a.o;
+    if (gated) cp_async_wait_all();  // this thread's pieces of the gate tile; the barrier publishes them
     fence_before();
     __syncthreads();
     if (tid == 0) {  // M^T += U^T (K o e^{c_last-c}) ; O^T += U^T P^T
@@ -626,6 +631,12 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_seq_tc_kernel(FwdArgs a) {
       }
       commit(bar);
     }
+    float sig[32];  // sigmoid of the output gate, formed while the products run
+    if (gated) {
+      const __nv_bfloat16* sg = reinterpret_cast<const __nv_bfloat16*>(sm + SQ_G);
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) sig[jj] = prep_sigmoid_fast(__bfloat162float(sg[(hcol * 32 + jj) * VD + Lr]));
+    }
     if (!tcc::wait_mma(bar, phase)) { failed = true; break; }
     if (tid == 0 && ch + 1 < nch) {  // the lanes' reads of e^{c_last} precede the overwrite
       fence_async_smem();
@@ -635,12 +646,10 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_seq_tc_kernel(FwdArgs a) {
       __nv_bfloat16* so = reinterpret_cast<__nv_bfloat16*>(sm + SQ_O);
       float v[32];
       tmem_ld32(tm + lo + TM_O + hcol * 32, v);
-      if (a.og) {  // output gate
-        cp_async_wait_all();
+      if (gated) {  // output gate
         out_gate_rows(v, reinterpret_cast<float*>(sm + SQ_RED), warp, lane, a.og_eps);
-        const __nv_bfloat16* sg = reinterpret_cast<const __nv_bfloat16*>(sm + SQ_G);
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) v[jj] *= prep_sigmoid(__bfloat162float(sg[(hcol * 32 + jj) * VD + Lr]));
+        for (int jj = 0; jj < 32; ++jj) v[jj] *= sig[jj];
       }
 #pragma unroll
       for (int jj = 0; jj < 32; ++jj) so[(hcol * 32 + jj) * VD + Lr] = __float2bfloat16_rn(v[jj]);

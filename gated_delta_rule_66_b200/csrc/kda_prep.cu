@@ -21,15 +21,18 @@ namespace kda {
 
 constexpr int CONV_MAX_W = 8;
 
-// One channel's convolution step: shift the window (in[0..W-1], oldest
-// first) by x, store the new window to out[0..W-1] and return
-// SiLU(sum_j w[j] window[j]).
-__device__ __forceinline__ float conv_step(const float* in, const float* w, float x, float* out, int W) {
+// One channel's convolution step on a window of W <= CONV_MAX_W inputs held
+// in registers (oldest first): shift in x, return SiLU(sum_j w[j] win[j]).
+// The loops are unrolled over CONV_MAX_W with predicates, so the window
+// never goes to local memory.
+__device__ __forceinline__ float conv_step(float (&win)[CONV_MAX_W], const float (&w)[CONV_MAX_W], float x, int W) {
   float acc = 0.f;
-  for (int j = 0; j < W; ++j) {
-    const float u = j + 1 < W ? in[j + 1] : x;
-    acc = fmaf(w[j], u, acc);
-    out[j] = u;
+#pragma unroll
+  for (int j = 0; j < CONV_MAX_W; ++j) {
+    if (j < W) {
+      win[j] = j + 1 < W ? win[j + 1] : x;
+      acc = fmaf(w[j], win[j], acc);
+    }
   }
   return acc * prep_sigmoid(acc);
 }
@@ -54,39 +57,64 @@ __global__ void __launch_bounds__(256) kda_decode_token_kernel(DecodeTokenArgs a
     s[it] = __ldcs(S4 + row * LPR + c4);
   }
 
-  // ---- convolution step of this head's channels: q (K), k (K), v (V)
+  // ---- every other global load of the CTA is issued here, next to the state
+  // loads, so that their latencies overlap: this thread's (at most two)
+  // channels of the convolution (input, window, weights), its gate channel,
+  // the beta logit and its output-gate column.
+  constexpr int NCH = 2 * K + V, PER = (NCH + 255) / 256;
   const size_t Cn = (size_t)2 * a.H * K + (size_t)a.HV * V;
   const float* win_in = a.conv_in ? a.conv_in + (size_t)b * Cn * a.W : nullptr;  // null: zero window
   float* win_out = a.conv_out + (size_t)b * Cn * a.W;
-  const bool own_qk = hv % G == 0;  // one value head of the group writes the shared q/k windows
-  for (int e = threadIdx.x; e < 2 * K + V; e += 256) {
-    size_t ch;
-    float x;
+  float xin[PER], win[PER][CONV_MAX_W], wt[PER][CONV_MAX_W];
+  size_t chan[PER];
+#pragma unroll
+  for (int p = 0; p < PER; ++p) {
+    const int e = threadIdx.x + 256 * p;
+    size_t ch = 0;
+    float x = 0.f;
     if (e < K) {
       ch = (size_t)h * K + e;
       x = to_f(static_cast<const TIn*>(a.xq)[((size_t)b * a.H + h) * K + e]);
     } else if (e < 2 * K) {
       ch = (size_t)a.H * K + (size_t)h * K + (e - K);
       x = to_f(static_cast<const TIn*>(a.xk)[((size_t)b * a.H + h) * K + e - K]);
-    } else {
+    } else if (e < NCH) {
       ch = (size_t)2 * a.H * K + (size_t)hv * V + (e - 2 * K);
       x = to_f(static_cast<const TIn*>(a.xv)[((size_t)b * a.HV + hv) * V + e - 2 * K]);
     }
-    float in[CONV_MAX_W], out[CONV_MAX_W];
-    for (int j = 0; j < a.W; ++j) in[j] = win_in ? win_in[ch * a.W + j] : 0.f;
-    const float y = conv_step(in, a.conv_w + ch * a.W, x, out, a.W);
+    chan[p] = ch;
+    xin[p] = x;
+#pragma unroll
+    for (int j = 0; j < CONV_MAX_W; ++j) {
+      const bool ok = e < NCH && j < a.W;
+      win[p][j] = (ok && win_in) ? win_in[ch * a.W + j] : 0.f;
+      wt[p][j] = ok ? a.conv_w[ch * a.W + j] : 0.f;
+    }
+  }
+  const int fz = threadIdx.x < K ? threadIdx.x : 0;
+  const float zf = to_f(static_cast<const TIn*>(a.prep.z)[((size_t)b * a.HV + hv) * K + fz]);
+  const float dtb = a.prep.dt_bias[(size_t)hv * K + fz];
+  const float alog = a.prep.A_log[hv];
+  const float blog = a.beta[(size_t)b * a.HV + hv];
+  const int nog = threadIdx.x < V ? threadIdx.x : 0;
+  const float ogv = a.og ? to_f(static_cast<const TIn*>(a.og)[((size_t)b * a.HV + hv) * V + nog]) : 0.f;
+
+  // ---- convolution step of this head's channels: q (K), k (K), v (V)
+  const bool own_qk = hv % G == 0;  // one value head of the group writes the shared q/k windows
+#pragma unroll
+  for (int p = 0; p < PER; ++p) {
+    const int e = threadIdx.x + 256 * p;
+    if (e >= NCH) continue;
+    const float y = conv_step(win[p], wt[p], xin[p], a.W);
     if (e >= 2 * K || own_qk)
-      for (int j = 0; j < a.W; ++j) win_out[ch * a.W + j] = out[j];
+#pragma unroll
+      for (int j = 0; j < CONV_MAX_W; ++j)
+        if (j < a.W) win_out[chan[p] * a.W + j] = win[p][j];
     if (e < K) sQ[e] = y;
     else if (e < 2 * K) sK[e - K] = y;
     else sV[e - 2 * K] = y;
   }
-  {  // decay from the gate pre-activation
-    const float dec = expf(a.prep.A_log[hv]);
-    const TIn* z = static_cast<const TIn*>(a.prep.z) + ((size_t)b * a.HV + hv) * K;
-    for (int f = threadIdx.x; f < K; f += 256)
-      sDec[f] = expf(prep_gate(to_f(z[f]) + a.prep.dt_bias[(size_t)hv * K + f], dec, a.prep.gate_lb));
-  }
+  if (threadIdx.x < K) sDec[threadIdx.x] = expf(prep_gate(zf + dtb, expf(alog), a.prep.gate_lb));
   __syncthreads();
   if (warp < 2) {  // L2 norms of q (warp 0) and k (warp 1)
     const float* x = warp ? sK : sQ;
@@ -136,7 +164,7 @@ __global__ void __launch_bounds__(256) kda_decode_token_kernel(DecodeTokenArgs a
     sRq[warp][4 * c4 + 2] = pq.z; sRq[warp][4 * c4 + 3] = pq.w;
   }
   __syncthreads();
-  const float beta = prep_sigmoid(a.beta[(size_t)b * a.HV + hv]);
+  const float beta = prep_sigmoid(blog);
   for (int n = threadIdx.x; n < V; n += 256) {
     float p = 0.f, qs = 0.f;
 #pragma unroll
@@ -156,8 +184,7 @@ __global__ void __launch_bounds__(256) kda_decode_token_kernel(DecodeTokenArgs a
       if (lane == 0) sRms = rsqrtf(ss / (float)V + a.og_eps);
     }
     __syncthreads();
-    const TIn* gate = static_cast<const TIn*>(a.og) + ((size_t)b * a.HV + hv) * V;
-    for (int n = threadIdx.x; n < V; n += 256) o[n] = from_f<TIn>(sO[n] * sRms * prep_sigmoid(to_f(gate[n])));
+    if (threadIdx.x < V) o[threadIdx.x] = from_f<TIn>(sO[threadIdx.x] * sRms * prep_sigmoid(ogv));
   } else {
     for (int n = threadIdx.x; n < V; n += 256) o[n] = from_f<TIn>(sO[n]);
   }
@@ -226,19 +253,26 @@ __global__ void __launch_bounds__(CONV_NT) kda_short_conv_kernel(ConvArgs a) {
   const float* st = a.state_in ? a.state_in + ((size_t)b * Cn + c) * W : nullptr;
   const float* w = a.w + (size_t)c * W;
   float wr[CONV_MAX_W], win[CONV_MAX_W];
-  for (int j = 0; j < W; ++j) wr[j] = w[j];
   // window before step t0: slot j holds step t0 - W + j (slot 0 drops out first);
-  // a step tau < 0 lives in the state's slot tau + W
-  for (int j = 1; j < W; ++j) {
+  // a step tau < 0 lives in the state's slot tau + W.  (Loops unrolled over
+  // CONV_MAX_W with predicates: the window stays in registers.)
+#pragma unroll
+  for (int j = 0; j < CONV_MAX_W; ++j) {
+    wr[j] = j < W ? w[j] : 0.f;
     const int tau = t0 - W + j;
-    win[j] = tau >= 0 ? to_f(x[base + (size_t)tau * stride]) : (st ? st[tau + W] : 0.f);
+    win[j] = (j < 1 || j >= W) ? 0.f : (tau >= 0 ? to_f(x[base + (size_t)tau * stride]) : (st ? st[tau + W] : 0.f));
   }
   const int t1 = min(t0 + CONV_TB, a.T);
   for (int t = t0; t < t1; ++t) {
-    for (int j = 0; j + 1 < W; ++j) win[j] = win[j + 1];
-    win[W - 1] = to_f(x[base + (size_t)t * stride]);
+    const float xt = to_f(x[base + (size_t)t * stride]);
     float acc = 0.f;
-    for (int j = 0; j < W; ++j) acc = fmaf(wr[j], win[j], acc);
+#pragma unroll
+    for (int j = 0; j < CONV_MAX_W; ++j) {
+      if (j < W) {
+        win[j] = j + 1 < W ? win[j + 1] : xt;
+        acc = fmaf(wr[j], win[j], acc);
+      }
+    }
     y[base + (size_t)t * stride] = from_f<TIn>(acc * prep_sigmoid(acc));
   }
   if (a.state_out && t1 == a.T) {  // the window after the last step

@@ -125,7 +125,8 @@ __device__ __forceinline__ void load_raw_issue_prep(const Ctx& c, const __nv_bfl
     cp_async16(c.sb + RAW_X + d, x + (t * HV + hv) * VD + vec * 8, ok);
     cp_async16(c.sb + RAW_C + i * LDCF * 4 + vec * 16, z + (t * HV + hv) * KD + vec * 8, ok);
   }
-  if (c.tid < C) c.beta()[c.tid] = (c.tid < L) ? prep_sigmoid(beta_logit[((size_t)b * T + t0 + c.tid) * HV + hv]) : 0.f;
+  if (c.tid < C)
+    c.beta()[c.tid] = (c.tid < L) ? prep_sigmoid_fast(beta_logit[((size_t)b * T + t0 + c.tid) * HV + hv]) : 0.f;
 }
 
 // Per-row factors of the fused preparation ("kimi_k3_host/kda.rs",
@@ -210,30 +211,36 @@ __device__ __forceinline__ int img(int r, int k) { return (int)(tc::kmaj(r, k, 6
 // With GATE (fused preparation) the rows hold z (bf16, load_raw_issue_prep)
 // and g = prep_gate(z + dt_bias) is formed here ("kimi_k3_host/kda.rs",
 // bounded_gate); rows at or past L count as g = 0 as in the plain load.
-template <bool GATE = false>
-__device__ __forceinline__ bool cumsum_span(const Ctx& c, const float* dt_bias_row = nullptr, float dec = 0.f,
-                                            float lb = 0.f, int L = C) {
+// (GATE: dtb = dt_bias[hv][tid % 128], dec = e^{A_log[hv]}, both loaded by
+// the caller ahead of the chunk's load wait, so that no global load sits on
+// this critical path)
+template <bool GATE = false, int NT = NTH>
+__device__ __forceinline__ bool cumsum_span(const Ctx& c, float dtb = 0.f, float dec = 0.f, float lb = 0.f,
+                                            int L = C) {
   float* sC = c.c();
   float* sCarry = reinterpret_cast<float*>(c.sm + S_CARRY);
   const int f = c.tid & 127, hh = c.tid >> 7;
+  if constexpr (GATE) {  // all threads: z -> g in registers, then over z in place (fp32 rows)
+    constexpr int PER = C * KD / NT;
+    const __nv_bfloat16* zr = reinterpret_cast<const __nv_bfloat16*>(c.sm + RAW_C);
+    float gv[PER];  // element e = tid + m NT has channel e % 128 = f
+#pragma unroll
+    for (int m = 0; m < PER; ++m) {
+      const int i = (c.tid + m * NT) >> 7;
+      gv[m] = i < L ? prep_gate_fast(__bfloat162float(zr[i * 2 * LDCF + f]) + dtb, dec, lb) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int m = 0; m < PER; ++m) sC[((c.tid + m * NT) >> 7) * LDCF + f] = gv[m];
+    __syncthreads();
+  }
   float v[32];
   float run = 0.f;
   if (c.tid < 256) {
-    if constexpr (GATE) {
-      const __nv_bfloat16* zr = reinterpret_cast<const __nv_bfloat16*>(c.sm + RAW_C);
-      const float dtb = dt_bias_row[f];
 #pragma unroll
-      for (int r = 0; r < 32; ++r) {
-        const int i = hh * 32 + r;
-        run += i < L ? prep_gate(__bfloat162float(zr[i * 2 * LDCF + f]) + dtb, dec, lb) : 0.f;
-        v[r] = run;
-      }
-    } else {
-#pragma unroll
-      for (int r = 0; r < 32; ++r) {
-        run += sC[(hh * 32 + r) * LDCF + f];
-        v[r] = run;
-      }
+    for (int r = 0; r < 32; ++r) {
+      run += sC[(hh * 32 + r) * LDCF + f];
+      v[r] = run;
     }
     if (hh == 0) sCarry[f] = run;
   }
