@@ -34,10 +34,10 @@ sys.path.insert(0, ROOT)
 
 import torch  # noqa: E402
 
-from gated_delta_rule_66_b200.inputs import BY_NAME, make_inputs, make_raw_inputs  # noqa: E402
+from gated_delta_rule_66_b200.inputs import BY_NAME, make_erase_inputs, make_inputs, make_raw_inputs  # noqa: E402
 
 HEADLINE = "fwdbwd"
-PATHS = ("twin", "prefill_gqa", "fwdbwd", "decode", "prefill_prep", "decode_token")
+PATHS = ("twin", "prefill_gqa", "fwdbwd", "decode", "prefill_prep", "decode_token", "erase")
 # paths from the raw projections (fused preparation): workload they take their sizes from
 PREP_PATHS = {"prefill_prep": "prefill_gqa", "decode_token": "decode"}
 CONV_W = 4  # the host model's short-convolution width
@@ -222,10 +222,44 @@ def gpu_prep_path(kda, name, steps, warmup, rank_barrier):
     return res, w
 
 
+def gpu_erase_path(kda, steps, warmup, rank_barrier):
+    """Times the asymmetric erase/write variant (kda_fwd_erase) on its
+    workload: B=1, T=8192, 32 query heads over 8 state heads, K=64, V=128."""
+    w = BY_NAME["erase"]
+    d = {n: (None if t is None else t.cuda()) for n, t in make_erase_inputs(w).items()}
+    stream = torch.cuda.current_stream()
+
+    def step():
+        kda.fwd_erase(d["q"], d["k"], d["e"], d["z"], d["g"], scale=w.scale)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    rank_barrier()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1) / steps
+    e = esize(w)
+    byts = (w.B * w.T * (w.H * w.K * e + 2 * w.HV * w.K * e + w.HV * w.V * e + w.HV * w.K * 4 + w.H * w.V * e)
+            + w.B * w.HV * w.K * w.V * 4)
+    hbm = load_peaks()["hbm_gbs"]
+    res = {"workload": "erase", "ms_per_step": ms, "tokens_per_step": w.B * w.T, "launches_per_step": 1,
+           "l2": "inputs > L2", "calls": {"kernel_ms": ms}, "e2e_ms": None,
+           "roofline": {"bound": "hbm", "kernel": "kda_fwd_chunk_kernel<ERASE> (CUDA-core path)",
+                        "achieved": byts / (ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
+                        "frac": byts / (ms * 1e-3) / 1e9 / hbm, "algorithmic_bytes": byts}}
+    return res, w
+
+
 def gpu_path(kda, name, steps, warmup, rank_barrier, shrink=None):
     """Times one workload on this rank's GPU.  Returns a result dict."""
     if name in PREP_PATHS:
         return gpu_prep_path(kda, name, steps, warmup, rank_barrier)
+    if name == "erase":
+        return gpu_erase_path(kda, steps, warmup, rank_barrier)
     w = BY_NAME[name]
     if shrink:  # a smaller batch and length of the same workload (profiler captures only)
         w = w.with_sizes(name=f"{name}_B{shrink[0]}_T{shrink[1]}", B=shrink[0], T=shrink[1])

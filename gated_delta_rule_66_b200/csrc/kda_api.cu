@@ -321,6 +321,24 @@ int kda_decode_step(const void* q, const void* k, const void* v, const float* g,
   return launch_decode(a, K, V, dtype, static_cast<cudaStream_t>(stream));
 }
 
+int kda_fwd_erase(const void* q, const void* k, const void* e, const void* z, const float* g, const float* S0,
+                  float scale, int B, int T, int HQ, int HV, int K, int V, int dtype, void* o, float* S_T,
+                  void* stream) {
+  g_err[0] = 0;
+  char buf[256];
+  int rc = check_common("kda_fwd_erase", B, T, 1, 1, K, V, dtype, scale);
+  if (rc) return rc;
+  if (HQ < 1 || HV < 1 || HQ % HV || HQ > 65535) {
+    snprintf(buf, sizeof(buf), "kda_fwd_erase: HQ=%d must be a positive multiple of HV=%d (<= 65535)", HQ, HV);
+    return set_error(KDA_ERR_SHAPE, buf);
+  }
+  if (!q || !k || !e || !z || !g || !o)
+    return set_error(KDA_ERR_NULL, "kda_fwd_erase: q, k, e, z, g and o must be non-NULL");
+  FwdArgs a{q, k, z, g, nullptr, S0, o, S_T, nullptr, nullptr, nullptr, scale, B, T, HQ, HV, K, V};
+  a.erase = e;
+  return launch_fwd_erase(a, dtype, static_cast<cudaStream_t>(stream));
+}
+
 static int check_gate(const char* fn, const void* z, const float* A_log, const float* dt_bias, float lb,
                       const float* beta_logit) {
   char buf[256];

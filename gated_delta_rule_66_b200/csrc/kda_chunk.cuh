@@ -193,10 +193,15 @@ __device__ __forceinline__ bool block_factors(int J, const float* sC, float* sE1
 }
 
 // Builds Ah (strict lower) and P (lower incl. diagonal), C x C, row stride C+1.
+// With sR (the erase rows of the asymmetric variant, "research_layers.py",
+// delta_recurrence: read = erase * decay) Ah[i][j] = sum_f r_if k_jf e^{c_i - c_j}
+// instead of k_if.
 template <int K, int C, bool PRECISE>
 __device__ void build_interaction(const float* sK, const float* sQ, const float* sC, float* sE1,
-                                  float* sE2o, float* sE2d, int* sFlag, float* sAh, float* sP) {
+                                  float* sE2o, float* sE2d, int* sFlag, float* sAh, float* sP,
+                                  const float* sR = nullptr) {
   constexpr int LDK = K + 1, LDC = C + 1, NB = C / BS;
+  if (!sR) sR = sK;
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
   for (int J = 0; J < NB; ++J) {
     const bool pairwise = block_factors<K, C, PRECISE>(J, sC, sE1, sE2o, sE2d, sFlag);
@@ -214,7 +219,7 @@ __device__ void build_interaction(const float* sK, const float* sQ, const float*
         for (int f = 0; f < K; ++f) {
           const float e = kexp<PRECISE>(sC[i * LDK + f] - sC[j * LDK + f]);
           const float kj = sK[j * LDK + f] * e;
-          accA = fmaf(sK[i * LDK + f], kj, accA);
+          accA = fmaf(sR[i * LDK + f], kj, accA);
           accP = fmaf(sQ[i * LDK + f], kj, accP);
         }
       } else {
@@ -223,7 +228,7 @@ __device__ void build_interaction(const float* sK, const float* sQ, const float*
         for (int f = 0; f < K; ++f) {
           const float kj = sK[j * LDK + f] * e2[tx * LDK + f];
           const float e1 = sE1[i * LDK + f];
-          accA = fmaf(sK[i * LDK + f] * e1, kj, accA);
+          accA = fmaf(sR[i * LDK + f] * e1, kj, accA);
           accP = fmaf(sQ[i * LDK + f] * e1, kj, accP);
         }
       }

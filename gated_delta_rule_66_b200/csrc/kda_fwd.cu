@@ -14,38 +14,82 @@
 
 namespace kda {
 
-template <int K, int C, int VB>
+template <int K, int C, int VB, bool ERASE = false>
 struct FwdSmem {
   static constexpr int LDK = K + 1, LDC = C + 1, LDV = VB + 1;
   static constexpr int oK = 0, oQ = oK + C * LDK, oC = oQ + C * LDK, oE1 = oC + C * LDK,
                        oE2o = oE1 + C * LDK, oE2d = oE2o + BS * LDK, oAh = oE2d + BS * LDK,
                        oT = oAh + C * LDC, oP = oT + C * LDC, oW = oP + C * LDC, oV = oW + BS * LDC,
                        oM = oV + C * LDV, oBeta = oM + K * LDV, oEl = oBeta + C, oFlag = oEl + K,
-                       total = oFlag + 4;
+                       oR = oFlag + 4, total = oR + (ERASE ? C * LDK : 0);
   static constexpr size_t bytes = (size_t)total * sizeof(float);
 };
 
-template <int K, int C, int VB, typename TIn>
+// The chunk of the asymmetric erase/write variant: q~ = scale q of query head
+// hq, the write keys k, erase rows e and decay g of state head hv (rows past
+// the sequence end zero), beta = 1; then g is replaced by its cumulative sum.
+template <int K, int C, typename TIn>
+__device__ __forceinline__ void load_chunk_erase(const FwdArgs& a, int b, int t0, int L, int hq, int hv, float* sQ,
+                                                 float* sK, float* sR, float* sC, float* sBeta) {
+  constexpr int LDK = K + 1;
+  const TIn* q = static_cast<const TIn*>(a.q);
+  const TIn* k = static_cast<const TIn*>(a.k);
+  const TIn* e = static_cast<const TIn*>(a.erase);
+  for (int idx = threadIdx.x; idx < C * K; idx += NTHREADS) {
+    const int i = idx / K, f = idx % K;
+    float qv = 0.f, kv = 0.f, ev = 0.f, gv = 0.f;
+    if (i < L) {
+      const size_t t = (size_t)b * a.T + t0 + i;
+      qv = to_f(q[(t * a.H + hq) * K + f]) * a.scale;
+      kv = to_f(k[(t * a.HV + hv) * K + f]);
+      ev = to_f(e[(t * a.HV + hv) * K + f]);
+      gv = a.g[(t * a.HV + hv) * K + f];
+    }
+    sQ[i * LDK + f] = qv;
+    sK[i * LDK + f] = kv;
+    sR[i * LDK + f] = ev;
+    sC[i * LDK + f] = gv;
+  }
+  for (int i = threadIdx.x; i < C; i += NTHREADS) sBeta[i] = 1.f;
+  __syncthreads();
+  for (int f = threadIdx.x; f < K; f += NTHREADS) {
+    float run = 0.f;
+    for (int i = 0; i < C; ++i) {
+      run += sC[i * LDK + f];
+      sC[i * LDK + f] = run;
+    }
+  }
+  __syncthreads();
+}
+
+// ERASE: the asymmetric erase/write variant ("research_layers.py",
+// delta_recurrence): blockIdx.y is the query head hq, which carries (a copy
+// of) the recurrence of state head hv = hq / (H / HV) and reads it out; the
+// erase rows take k's place in the interaction Ah and in the residual.
+template <int K, int C, int VB, typename TIn, bool ERASE = false>
 __global__ void __launch_bounds__(NTHREADS, 1)
     kda_fwd_chunk_kernel(FwdArgs a) {
-  using S = FwdSmem<K, C, VB>;
+  using S = FwdSmem<K, C, VB, ERASE>;
   constexpr bool PRECISE = sizeof(TIn) == 4;
   constexpr int LDK = S::LDK, LDC = S::LDC, LDV = S::LDV;
   extern __shared__ float smem[];
   float *sK = smem + S::oK, *sQ = smem + S::oQ, *sC = smem + S::oC, *sE1 = smem + S::oE1,
         *sE2o = smem + S::oE2o, *sE2d = smem + S::oE2d, *sAh = smem + S::oAh, *sT = smem + S::oT,
         *sP = smem + S::oP, *sW = smem + S::oW, *sV = smem + S::oV, *sM = smem + S::oM,
-        *sBeta = smem + S::oBeta, *sEl = smem + S::oEl;
+        *sBeta = smem + S::oBeta, *sEl = smem + S::oEl, *sR = ERASE ? smem + S::oR : nullptr;
   int* sFlag = reinterpret_cast<int*>(smem + S::oFlag);
 
   const TIn* __restrict__ q = static_cast<const TIn*>(a.q);
   const TIn* __restrict__ k = static_cast<const TIn*>(a.k);
   const TIn* __restrict__ v = static_cast<const TIn*>(a.v);
   TIn* __restrict__ o = static_cast<TIn*>(a.o);
-  const int v0 = blockIdx.x * VB, hv = blockIdx.y, b = blockIdx.z;
-  const int h = hv / (a.HV / a.H);
+  const int v0 = blockIdx.x * VB, b = blockIdx.z;
+  const int hq = blockIdx.y, hv = ERASE ? hq / (a.H / a.HV) : hq;  // (query head = value head for KDA)
+  const int h = ERASE ? 0 : hv / (a.HV / a.H);
   const int T = a.T, V = a.V, NT = (T + C - 1) / C;
   const size_t head = (size_t)b * a.HV + hv;
+  const int HO = ERASE ? a.H : a.HV, ho = hq;  // heads of o, this CTA's head in o
+  const bool writes_state = !ERASE || hq % (a.H / a.HV) == 0;
 
   // entering state
   for (int idx = threadIdx.x; idx < K * VB; idx += NTHREADS) {
@@ -63,14 +107,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         dst[(size_t)f * V + v0 + n] = sM[f * LDV + n];
       }
     }
-    load_chunk_qkgb<K, C, TIn>(q, k, a.g, a.beta, a.scale, b, t0, L, T, a.H, a.HV, h, hv, sQ, sK,
-                               sC, sBeta, static_cast<const TIn*>(a.prep.z), a.prep.A_log, a.prep.dt_bias,
-                               a.prep.gate_lb);
+    if constexpr (ERASE)
+      load_chunk_erase<K, C, TIn>(a, b, t0, L, hq, hv, sQ, sK, sR, sC, sBeta);
+    else
+      load_chunk_qkgb<K, C, TIn>(q, k, a.g, a.beta, a.scale, b, t0, L, T, a.H, a.HV, h, hv, sQ, sK,
+                                 sC, sBeta, static_cast<const TIn*>(a.prep.z), a.prep.A_log, a.prep.dt_bias,
+                                 a.prep.gate_lb);
     for (int idx = threadIdx.x; idx < C * VB; idx += NTHREADS) {
       const int i = idx / VB, n = idx % VB;
       sV[i * LDV + n] = (i < L) ? to_f(v[(((size_t)b * T + t0 + i) * a.HV + hv) * V + v0 + n]) : 0.f;
     }
-    build_interaction<K, C, PRECISE>(sK, sQ, sC, sE1, sE2o, sE2d, sFlag, sAh, sP);
+    build_interaction<K, C, PRECISE>(sK, sQ, sC, sE1, sE2o, sE2d, sFlag, sAh, sP, sR);
     invert_unit_lower<C>(sAh, sBeta, sT, sW);
 
     // decayed operands: sE1 <- k o e^{c_last - c}, sK <- k o e^c, sQ <- q~ o e^c
@@ -80,7 +127,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const float e = kexp<PRECISE>(c), ed = kexp<PRECISE>(cl - c);
       const float kk = sK[i * LDK + f];
       sE1[i * LDK + f] = kk * ed;
-      sK[i * LDK + f] = kk * e;
+      if constexpr (ERASE) sR[i * LDK + f] *= e;  // the residual reads the erase rows
+      else sK[i * LDK + f] = kk * e;
       sQ[i * LDK + f] *= e;
     }
     for (int f = threadIdx.x; f < K; f += NTHREADS) sEl[f] = kexp<PRECISE>(sC[(C - 1) * LDK + f]);
@@ -91,7 +139,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     {  // R = diag(beta) (V - (K o e^c) M), in place in sV
       float acc[TMC][TNV];
       zero(acc);
-      mm(acc, K, [&](int i, int f) { return sK[i * LDK + f]; },
+      const float* sRes = ERASE ? sR : sK;
+      mm(acc, K, [&](int i, int f) { return sRes[i * LDK + f]; },
          [&](int f, int n) { return sM[f * LDV + n]; });
 #pragma unroll
       for (int x = 0; x < TMC; ++x)
@@ -127,7 +176,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int y = 0; y < TNV; ++y) {
           const int i = ty + 16 * x, n = tx + 16 * y;
           if (i < L) {
-            const size_t at = (((size_t)b * T + t0 + i) * a.HV + hv) * V + v0 + n;
+            const size_t at = (((size_t)b * T + t0 + i) * HO + ho) * V + v0 + n;
             if (a.o32) a.o32[at] = acc[x][y];  // fp32 for the output-gate pass
             else o[at] = from_f<TIn>(acc[x][y]);
           }
@@ -152,7 +201,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
   }
   __syncthreads();
-  if (a.S_T) {
+  if (a.S_T && writes_state) {
     for (int idx = threadIdx.x; idx < K * VB; idx += NTHREADS) {
       const int f = idx / VB, n = idx % VB;
       a.S_T[(head * K + f) * V + v0 + n] = sM[f * LDV + n];
@@ -172,6 +221,29 @@ static int launch_fwd_t(const FwdArgs& a, cudaStream_t stream) {
   e = cudaGetLastError();
   if (e != cudaSuccess) return set_cuda_error("kda_fwd: launch", e);
   return 0;
+}
+
+template <int K, typename TIn>
+static int launch_fwd_erase_t(const FwdArgs& a, cudaStream_t stream) {
+  constexpr int C = FWD_CHUNK, VB = FWD_VBLOCK;
+  using S = FwdSmem<K, C, VB, true>;
+  auto kern = kda_fwd_chunk_kernel<K, C, VB, TIn, true>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::bytes);
+  if (e != cudaSuccess) return set_cuda_error("kda_fwd_erase: cudaFuncSetAttribute", e);
+  kern<<<dim3(a.V / VB, a.H, a.B), NTHREADS, S::bytes, stream>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return set_cuda_error("kda_fwd_erase: launch", e);
+  return 0;
+}
+
+int launch_fwd_erase(const FwdArgs& a, int dtype, cudaStream_t stream) {
+  const bool bf = dtype == 1;
+  switch (a.K) {
+    case 32: return bf ? launch_fwd_erase_t<32, __nv_bfloat16>(a, stream) : launch_fwd_erase_t<32, float>(a, stream);
+    case 64: return bf ? launch_fwd_erase_t<64, __nv_bfloat16>(a, stream) : launch_fwd_erase_t<64, float>(a, stream);
+    case 128: return bf ? launch_fwd_erase_t<128, __nv_bfloat16>(a, stream) : launch_fwd_erase_t<128, float>(a, stream);
+  }
+  return set_error(4, "kda_fwd_erase: unsupported K");
 }
 
 int launch_fwd(const FwdArgs& a, int dtype, cudaStream_t stream) {

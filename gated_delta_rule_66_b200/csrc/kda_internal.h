@@ -112,6 +112,12 @@ struct FwdArgs {
   const void* og;     // output-gate pre-activation [rows, HV, V] in the input dtype, or null
   float og_eps;
   float* o32;         // CUDA-core path with og: fp32 output scratch [rows, HV, V] for the gate pass
+  // Asymmetric erase/write variant ("research_layers.py", delta_recurrence):
+  // erase [rows, HV, K] in the input dtype; then H counts QUERY heads (a
+  // multiple of HV: query head hq reads state head hq / (H / HV)), k, g and
+  // erase have HV heads, v holds z [rows, HV, V], beta is unused and o is
+  // [rows, H, V].
+  const void* erase;
 };
 
 struct BwdArgs {
@@ -177,6 +183,7 @@ int launch_fwd(const FwdArgs& a, int dtype, cudaStream_t stream);
 // the CUDA-core forward whatever the shape (stores all 32-step states)
 int launch_fwd_ffma(const FwdArgs& a, int dtype, cudaStream_t stream);
 bool fwd_tc_eligible(const FwdArgs& a, int dtype);
+int launch_fwd_erase(const FwdArgs& a, int dtype, cudaStream_t stream);
 int launch_fwd_tc(const FwdArgs& a, cudaStream_t stream);
 int take_device_error(unsigned* out);
 int take_bwd_device_error(unsigned* out);

@@ -75,6 +75,12 @@ WORKLOADS = [
              gate="bounded", s0_std=0.02, path="decode", chunk=64),
 ]
 BY_NAME = {w.name: w for w in WORKLOADS}
+# The asymmetric erase/write variant ("research_layers.py"): H counts query
+# heads (32), HV state heads (8, groups of 4 query heads), K the feature
+# dimension (the layer's default 64), V the head dimension.
+ERASE = Workload("erase", 5, B=1, T=8192, H=32, HV=8, K=64, V=128, dtype="bf16",
+                 gate="erase", s0_std=0.0, path="erase", chunk=32)
+BY_NAME[ERASE.name] = ERASE
 
 
 def _l2norm_rows(x):
@@ -176,6 +182,37 @@ def make_raw_inputs(w: Workload, seed: int | None = None, conv_width: int = 0, l
         out["conv_w"] = randn(Cn, conv_width) * 0.5
         out["conv_state"] = randn(B, Cn, conv_width)
     return out
+
+
+def make_erase_inputs(w: Workload, seed: int | None = None):
+    """Draw the inputs of the erase/write variant with the value ranges of the
+    research layer's feature maps ("research_layers.py", features): q, k rows
+    L2-normalised; erase = k * sigmoid(N(-1, 1)) (gate bias -1); z = v *
+    sigmoid(N(-1, 1)) with v ~ N(0, 1); g = -0.25 sigmoid(N(log(0.04/0.96), 1))
+    (the layer's bounded forget gate).  One CPU generator (default seed
+    20261202 + 200 + workload index), draws in the order q, k, v, erase noise,
+    write noise, forget noise, S0.  q, k, erase and z are rounded to the
+    dtype; g and S0 stay fp32.  Shapes: q [B,T,H,K] (H query heads), k,
+    erase, g [B,T,HV,K], z [B,T,HV,V], S0 [B,HV,K,V] or None.
+    """
+    if seed is None:
+        seed = SEED_BASE + 200 + w.index
+    gen = torch.Generator().manual_seed(seed)
+    B, T, H, HV, K, V = w.B, w.T, w.H, w.HV, w.K, w.V
+
+    def randn(*shape):
+        return torch.randn(*shape, generator=gen, dtype=torch.float32)
+
+    dt = w.torch_dtype
+    q = _l2norm_rows(randn(B, T, H, K))
+    k = _l2norm_rows(randn(B, T, HV, K))
+    v = randn(B, T, HV, V)
+    erase = k * torch.sigmoid(randn(B, T, HV, K) - 1.0)
+    z = v * torch.sigmoid(randn(B, T, HV, V) - 1.0)
+    g = -0.25 * torch.sigmoid(randn(B, T, HV, K) + math.log(0.04 / 0.96))
+    S0 = randn(B, HV, K, V) * w.s0_std if w.s0_std > 0 else None
+    return {"q": q.to(dt).contiguous(), "k": k.to(dt).contiguous(), "e": erase.to(dt).contiguous(),
+            "z": z.to(dt).contiguous(), "g": g.contiguous(), "S0": S0}
 
 
 def head_subset(inputs: dict, H: int, HV: int, groups):

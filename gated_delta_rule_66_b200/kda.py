@@ -25,7 +25,8 @@ CHUNK = 32  # chunk length of the library's chunked kernels (workspace layout)
 SYMBOLS = ("kda_last_error", "kda_device_status", "kda_fwd_workspace_bytes", "kda_fwd_scratch_bytes",
            "kda_bwd_workspace_bytes", "kda_fwd", "kda_fwd_varlen_workspace_bytes", "kda_fwd_varlen",
            "kda_bwd_varlen_workspace_bytes", "kda_bwd_varlen", "kda_decode_step", "kda_bwd",
-           "kda_fwd_prep_workspace_bytes", "kda_fwd_prep", "kda_short_conv", "kda_decode_token")
+           "kda_fwd_prep_workspace_bytes", "kda_fwd_prep", "kda_short_conv", "kda_decode_token",
+           "kda_fwd_erase")
 
 
 class KdaError(RuntimeError):
@@ -80,6 +81,8 @@ def _load():
     lib.kda_decode_token.restype = i
     lib.kda_decode_token.argtypes = [vp, vp, vp, vp, vp, vp, i, vp, vp, vp, f, vp, vp, f, vp, f, i, i, i, i, i, i,
                                      vp, vp]
+    lib.kda_fwd_erase.restype = i
+    lib.kda_fwd_erase.argtypes = [vp, vp, vp, vp, vp, vp, f, i, i, i, i, i, i, i, vp, vp, vp]
     return lib
 
 
@@ -425,3 +428,27 @@ def decode_token(xq, xk, xv, conv_w, conv_state, z, A_log, dt_bias, beta_logit, 
                                _dtype_code(xq), _ptr(o), _stream())
     _check("kda_decode_token", rc)
     return o
+
+
+# ----------------------------------------------------------------------------- erase/write variant
+def fwd_erase(q, k, e, z, g, scale=None, initial_state=None, output_final_state=True):
+    """Prefill of the asymmetric erase/write delta recurrence.
+
+    q [B,T,HQ,K]; k (write), e (erase) [B,T,HV,K]; z [B,T,HV,V] (one dtype);
+    g [B,T,HV,K] float32; HQ a multiple of HV (query head hq reads state head
+    hq // (HQ // HV)).  Returns (o [B,T,HQ,V], S_T [B,HV,K,V] or None).
+    """
+    B, T, HQ, K = q.shape
+    HV, V = k.shape[2], z.shape[3]
+    scale = 1.0 / math.sqrt(K) if scale is None else float(scale)
+    dt = q.dtype
+    for n, t in (("q", q), ("k", k), ("e", e), ("z", z)):
+        _req(n, t, dt, 4)
+    _req("g", g, torch.float32, 4)
+    _req("initial_state", initial_state, torch.float32, 4)
+    o = torch.empty(B, T, HQ, V, dtype=dt, device=q.device)
+    S_T = torch.empty(B, HV, K, V, dtype=torch.float32, device=q.device) if output_final_state else None
+    rc = _lib.kda_fwd_erase(_ptr(q), _ptr(k), _ptr(e), _ptr(z), _ptr(g), _ptr(initial_state), scale, B, T, HQ, HV,
+                            K, V, _dtype_code(q), _ptr(o), _ptr(S_T), _stream())
+    _check("kda_fwd_erase", rc)
+    return o, S_T

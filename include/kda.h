@@ -252,6 +252,22 @@ int kda_decode_token(const void* xq, const void* xk, const void* xv, const float
                      float gate_lower_bound, const float* beta_logit, const void* out_gate, float out_eps, float* S,
                      float scale, int B, int H, int HV, int K, int V, int dtype, void* o, void* stream);
 
+/* Prefill of the asymmetric erase/write delta recurrence ("research_layers.py",
+ * delta_recurrence and delta_token_reference), per state head hv:
+ *     S_bar = exp(g_t) (.) S_{t-1}
+ *     S_t   = S_bar + k_t (z_t - e_t^T S_bar)^T     (erase along e, write along k)
+ *     o_t   = (scale q_t)^T S_t                     per query head, after the write
+ * KDA is the case e = beta k, z = beta v.  Heads follow the page's layer:
+ * query head hq reads state head hq / (HQ / HV).
+ *   q [B, T, HQ, K] dtype; k, e [B, T, HV, K] dtype; z [B, T, HV, V] dtype;
+ *   g [B, T, HV, K] float; S0 [B, HV, K, V] float or NULL
+ *   o [B, T, HQ, V] dtype (output); S_T [B, HV, K, V] float or NULL
+ * HQ must be a multiple of HV.  Runs on the CUDA-core chunk kernels (one CTA
+ * per query head and 32 value columns, each carrying its state head). */
+int kda_fwd_erase(const void* q, const void* k, const void* e, const void* z, const float* g, const float* S0,
+                  float scale, int B, int T, int HQ, int HV, int K, int V, int dtype, void* o, float* S_T,
+                  void* stream);
+
 /* Size in bytes of the fixed device array that kda_bwd_noalloc uses as its
  * scratch (64 MiB, held on every GPU that loads the library until exit). */
 #define KDA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)

@@ -202,3 +202,18 @@ def test_prep_workspace_and_validation(lib):
     assert tok(S=ctypes.c_void_p(0x1008), H=2) == 7 and "aligned" in lib.kda_last_error().decode()
     assert tok(co=None) == 1
     assert tok(W=12, H=2) == 7
+
+
+def test_erase_validation(lib):
+    def call(**over):
+        a = dict(q=FAKE, k=FAKE, e=FAKE, z=FAKE, g=FAKE, S0=None, scale=0.5, B=1, T=8, HQ=4, HV=2, K=64, V=128,
+                 dtype=1, o=FAKE, S_T=None)
+        a.update(over)
+        return lib.kda_fwd_erase(a["q"], a["k"], a["e"], a["z"], a["g"], a["S0"], a["scale"], a["B"], a["T"],
+                                 a["HQ"], a["HV"], a["K"], a["V"], a["dtype"], a["o"], a["S_T"], None)
+
+    assert call(HQ=3) == 2 and "multiple of HV" in lib.kda_last_error().decode()
+    assert call(e=None) == 1
+    assert call(K=48) == 4
+    assert call(scale=-1.0) == 7
+    assert call(T=0) == 2

@@ -213,3 +213,69 @@ def test_raw_prefill_then_decode(kda):
         report(f"pipeline decode step{t} o", f64(outs[t]), o_t, tol, w.torch_dtype)
     report("pipeline final S", f64(S), S_ref, tol, torch.float32)
     assert np.array_equal(f64(win), win_ref)
+
+
+# ----------------------------------------------------------------------------- erase/write variant
+from gated_delta_rule_66_b200.inputs import make_erase_inputs  # noqa: E402
+
+ERASE_CASES = [
+    # name, size overrides of the erase workload
+    ("fp32_k32_ragged", dict(B=2, T=77, H=4, HV=2, K=32, V=32, dtype="fp32", s0_std=0.05)),
+    ("bf16_k64_v128", dict(B=1, T=100, H=8, HV=2, K=64, V=128)),
+    ("bf16_k128_mha", dict(B=2, T=65, H=2, HV=2, K=128, V=64, s0_std=0.05)),
+]
+
+
+def _erase_oracle(r, scale):
+    return oracle.erase_forward(f64(r["q"]), f64(r["k"]), f64(r["e"]), f64(r["z"]), f64(r["g"]), scale,
+                                f64(r["S0"]))
+
+
+@pytest.mark.parametrize("name,over", ERASE_CASES, ids=[c[0] for c in ERASE_CASES])
+def test_fwd_erase(kda, name, over):
+    """The asymmetric erase/write recurrence (separate erase and write
+    vectors, query heads grouped over state heads) against the token loop."""
+    w = BY_NAME["erase"].with_sizes(**over)
+    r = make_erase_inputs(w)
+    d = {n: (None if t is None else t.cuda()) for n, t in r.items()}
+    o, S = kda.fwd_erase(d["q"], d["k"], d["e"], d["z"], d["g"], scale=w.scale, initial_state=d["S0"])
+    torch.cuda.synchronize()
+    o_ref, S_ref = _erase_oracle(r, w.scale)
+    tol = tol_for(w.torch_dtype)
+    report(f"erase_{name} o", f64(o), o_ref, tol, w.torch_dtype)
+    report(f"erase_{name} S_T", f64(S), S_ref, tol, torch.float32)
+
+
+def test_fwd_erase_kda_special_case(kda):
+    """e = beta k and z = beta v make the variant KDA: its output equals the
+    KDA forward's on the same GPU (fp32, within the fp32 bar of each other)."""
+    from gated_delta_rule_66_b200.inputs import make_inputs
+    w = BY_NAME["twin"].with_sizes(B=1, T=96, H=2, HV=2)
+    inp = make_inputs(w)
+    d = {n: (None if t is None else t.cuda()) for n, t in inp.items()}
+    o_k, S_k = kda.fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], scale=w.scale, initial_state=d["S0"])
+    e = (d["beta"][..., None] * d["k"]).contiguous()
+    z = (d["beta"][..., None] * d["v"]).contiguous()
+    o_e, S_e = kda.fwd_erase(d["q"], d["k"], e, z, d["g"], scale=w.scale, initial_state=d["S0"])
+    torch.cuda.synchronize()
+    report("erase_as_kda o", f64(o_e), f64(o_k), 1e-5, torch.float32)
+    report("erase_as_kda S_T", f64(S_e), f64(S_k), 1e-5, torch.float32)
+
+
+def test_fwd_erase_full_size(kda):
+    """The erase workload (B=1, T=8192, 32 query heads over 8 state heads,
+    K=64, V=128, bf16) in full on the GPU; the oracle checks state head 3 and
+    its four query heads."""
+    w = BY_NAME["erase"]
+    r = make_erase_inputs(w)
+    d = {n: (None if t is None else t.cuda()) for n, t in r.items()}
+    o, S = kda.fwd_erase(d["q"], d["k"], d["e"], d["z"], d["g"], scale=w.scale)
+    torch.cuda.synchronize()
+    QG = w.H // w.HV
+    hq = list(range(3 * QG, 4 * QG))
+    sub = {"q": r["q"][:, :, hq], "k": r["k"][:, :, [3]], "e": r["e"][:, :, [3]], "z": r["z"][:, :, [3]],
+           "g": r["g"][:, :, [3]], "S0": None}
+    o_ref, S_ref = _erase_oracle(sub, w.scale)
+    report("erase_full o[state head 3]", f64(o[:, :, hq]), o_ref, tol_for(w.torch_dtype), w.torch_dtype)
+    report("erase_full S_T[state head 3]", f64(S[:, [3]]), S_ref, tol_for(w.torch_dtype), torch.float32)
+    assert torch.isfinite(o.float()).all()
