@@ -427,6 +427,14 @@ def roofline_for(res, w, peaks):
                     "achieved": fb / tf / 1e9, "frac": fb / tf / 1e9 / hbm, "algorithmic_bytes": fb}}
 
 
+def job_throughput(ms_local, tokens_per_step, world, all_reduce_max):
+    """Whole-job throughput of replicas: the slowest rank's step time (the
+    all-reduce MAX of every rank's device time) and the tokens all ranks
+    processed per step.  Returns (ms_per_step, tokens/s)."""
+    ms = all_reduce_max(ms_local) if world > 1 else ms_local
+    return ms, tokens_per_step * world / (ms * 1e-3)
+
+
 def run_gpu(args):
     import torch.distributed as dist
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -453,13 +461,12 @@ def run_gpu(args):
             res, w = gpu_path(kda, name, args.steps, args.warmup, barrier)
         if "roofline" not in res:
             res["roofline"] = roofline_for(res, w, peaks)
-        ms = res["ms_per_step"]
-        if world > 1:
-            t = torch.tensor([ms], device="cuda")
+        def reduce_max(x):
+            t = torch.tensor([x], device="cuda")
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = float(t.item())
-            res["ms_per_step"] = ms
-        res["tokens_per_s"] = res["tokens_per_step"] * world / (ms * 1e-3)
+            return float(t.item())
+        ms, res["tokens_per_s"] = job_throughput(res["ms_per_step"], res["tokens_per_step"], world, reduce_max)
+        res["ms_per_step"] = ms
         res["e2e_tokens_per_s"] = (res["tokens_per_step"] * world / (res["e2e_ms"] * 1e-3)
                                    if res["e2e_ms"] else None)
         results[name] = (res, w)
