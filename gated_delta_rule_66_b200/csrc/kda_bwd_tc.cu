@@ -29,6 +29,10 @@ __device__ unsigned int g_kda_bwd_device_error;  // this file's kernels (one fla
 namespace tcb {
 using namespace tcc;
 constexpr uint32_t OP_KED = OP, OP_QET = OP + 32768, OP_NKET = OP + 65536;
+// the chunk's P^T and T^T images, above the operands (the raw region then
+// takes the next chunk's rows while this chunk's products run)
+constexpr uint32_t IMG_PT = OP + 98304, IMG_TT = OP + 114688;
+static_assert(IMG_TT + 16384 <= SMALL, "state-gradient shared-memory map");
 constexpr uint32_t TM_S = 0, TM_DU = 128, TM_DR = 192, TM_DOT = 256;
 }  // namespace tcb
 
@@ -86,12 +90,22 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_dstate_tc_kernel(BwdArgs a) {
   fence_before();
   __syncthreads();
 
+  // Copies run one chunk ahead, in cp.async groups committed in the order
+  // raw(c1-1), images(c1-1), raw(c1-2), images(c1-2), ...: a chunk's raw rows
+  // are requested once the previous chunk's rows are consumed, its images
+  // once the previous chunk's products have read theirs.
+  if (c1 > c0) {
+    const int2 sp = chunk_span(a, c1 - 1);
+    load_raw_issue<NTH, true>(cx, qg, kg, dog, a.g, a.beta, b, T, sp.x, sp.y, a.H, a.HV, h, hv);
+    cp_async_commit();
+    const float* irec = a.inter + chunk_gc(a, sq, hv, c1 - 1) * INTER_REC;
+    copy_image(cx, IMG_PT, irec);             // P^T: (row i, K j) = P[j][i]
+    copy_image(cx, IMG_TT, irec + INTER_TT);  // T^T: (row i, K j) = T[j][i]
+    cp_async_commit();
+  }
   for (int ch = c1 - 1; ch >= c0; --ch) {
-    const int2 sp = chunk_span(a, ch);
-    const int t0 = sp.x, L = sp.y;
-    const float* irec = a.inter + chunk_gc(a, sq, hv, ch) * INTER_REC;  // P^T, T^T of this chunk (forward)
-    load_raw_issue(cx, qg, kg, dog, a.g, a.beta, b, T, t0, L, a.H, a.HV, h, hv);
-    if (!load_raw_wait(cx)) { failed = true; break; }
+    cp_async_wait_group<1>();  // this chunk's raw rows (its images may still be in flight)
+    __syncthreads();
     cumsum_span(cx);
 
     // ---------------------------------------------------------------- operands of the gradient products
@@ -138,19 +152,21 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_dstate_tc_kernel(BwdArgs a) {
         tmem_wait_st();
       }
     }
-    fence_async_smem();
     fence_before();
-    __syncthreads();  // raw inputs consumed; the raw region is reused below
-    copy_image(cx, R_P, irec);             // P^T: (row i, K j) = P[j][i]
-    copy_image(cx, R_T, irec + INTER_TT);  // T^T: (row i, K j) = T[j][i]
-    cp_async_wait_all();
+    __syncthreads();  // this chunk's raw rows are consumed: the next chunk's may come in
+    if (ch > c0) {
+      const int2 sp = chunk_span(a, ch - 1);
+      load_raw_issue<NTH, true>(cx, qg, kg, dog, a.g, a.beta, b, T, sp.x, sp.y, a.H, a.HV, h, hv);
+    }
+    cp_async_commit();           // (an empty group on the last chunk keeps the count uniform)
+    cp_async_wait_group<1>();    // this chunk's images
     fence_async_smem();
     __syncthreads();
     if (tid == 0) {  // dU^T = dO^T P + dM^T (K o e^{c_last-c})^T
       fence_after();
       const uint32_t id = idesc_tf32(128, 64);
       for (int ks = 0; ks < 8; ++ks)
-        mma_ts(tm + TM_DU, tm + TM_DOT + ks * 8, desc(sb + R_P + ks * 256, 2048), id, ks > 0);
+        mma_ts(tm + TM_DU, tm + TM_DOT + ks * 8, desc(sb + IMG_PT + ks * 256, 2048), id, ks > 0);
       for (int ks = 0; ks < 16; ++ks)
         mma_ts(tm + TM_DU, tm + TM_S + ks * 8, desc(sb + OP_KED + ks * 256, 4096), id, 1);
       commit(bar);
@@ -159,10 +175,16 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_dstate_tc_kernel(BwdArgs a) {
     if (tid == 0) {  // dR^T = dU^T T
       const uint32_t id = idesc_tf32(128, 64);
       for (int ks = 0; ks < 8; ++ks)
-        mma_ts(tm + TM_DR, tm + TM_DU + ks * 8, desc(sb + R_T + ks * 256, 2048), id, ks > 0);
+        mma_ts(tm + TM_DR, tm + TM_DU + ks * 8, desc(sb + IMG_TT + ks * 256, 2048), id, ks > 0);
       commit(bar);
     }
     if (!wait_mma(bar, phase)) { failed = true; break; }
+    if (ch > c0) {  // the products have read this chunk's images: the next chunk's may come in
+      const float* irec = a.inter + chunk_gc(a, sq, hv, ch - 1) * INTER_REC;
+      copy_image(cx, IMG_PT, irec);
+      copy_image(cx, IMG_TT, irec + INTER_TT);
+    }
+    cp_async_commit();
 
     // ---------------------------------------------------------------- store dM (leaving this chunk); start dM_in
     {
@@ -197,6 +219,7 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_dstate_tc_kernel(BwdArgs a) {
     __syncthreads();
   }
 
+  cp_async_wait_all();  // (copies still in flight after an early exit)
   if (!failed && a.dS0) {
     fence_after();
     for (int cb = 0; cb < 2; ++cb) {

@@ -83,7 +83,8 @@ __device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast
 // zero.  Issues the copies only; load_raw_wait completes them.  (16-byte
 // cp.async per thread: measured faster here than per-row bulk copies issued
 // by one warp.)
-template <int NT = NTH>
+// (ASYNC_BETA: beta also by cp.async, so that issuing the load never waits)
+template <int NT = NTH, bool ASYNC_BETA = false>
 __device__ __forceinline__ void load_raw_issue(const Ctx& c, const __nv_bfloat16* q, const __nv_bfloat16* k,
                                                const __nv_bfloat16* x, const float* g, const float* beta,
                                                int b, int T, int t0, int L, int H, int HV, int h, int hv) {
@@ -103,7 +104,12 @@ __device__ __forceinline__ void load_raw_issue(const Ctx& c, const __nv_bfloat16
     const size_t t = (size_t)b * T + t0 + (ok ? i : 0);
     cp_async16(c.sb + RAW_C + (i * LDCF + vec * 4) * 4, g + (t * HV + hv) * KD + vec * 4, ok);
   }
-  if (c.tid < C) c.beta()[c.tid] = (c.tid < L) ? beta[((size_t)b * T + t0 + c.tid) * HV + hv] : 0.f;
+  if (c.tid < C) {
+    const bool ok = c.tid < L;
+    const float* src = beta + ((size_t)b * T + t0 + (ok ? c.tid : 0)) * HV + hv;
+    if constexpr (ASYNC_BETA) tc::cp_async4(c.sb + S_BETA + c.tid * 4, src, ok);
+    else c.beta()[c.tid] = ok ? *src : 0.f;
+  }
 }
 // The same load for the fused preparation: z (the gate pre-activation, bf16)
 // instead of g, as packed rows at the stride of the cumulative-decay rows
