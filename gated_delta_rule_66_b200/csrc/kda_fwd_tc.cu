@@ -93,8 +93,11 @@ __device__ __forceinline__ void out_gate_rows(float (&v)[32], float* red, int wa
 // sequence (Ln steps from t0 + 64) is prefetched into L2.
 // Returns false, block-uniformly, if a tensor-core wait ran out.
 // With PREP the fused input preparation runs on the loaded chunk (FwdArgs::prep):
-// q, k rows L2-normalised, g from z, beta from its logit.
-template <int NTHR, bool PREP = false>
+// q, k rows L2-normalised, g from z, beta from its logit.  With PRELOADED
+// the caller has already issued the chunk's raw loads (issue_chunk_loads).
+// With `img` the P image is bulk-stored as soon as it is read out (thread 32's
+// bulk group), so that the raw region it sits in is free again at the end.
+template <int NTHR, bool PREP = false, bool PRELOADED = false>
 __device__ __forceinline__ bool fwd_chunk_head(const tcc::Ctx& cx, const FwdArgs& a, int b, int hv, int h,
                                                int t0, int L, int Ln, float* irec,
                                                unsigned char* img, uint64_t* bar, uint32_t& phase) {
@@ -113,12 +116,12 @@ __device__ __forceinline__ bool fwd_chunk_head(const tcc::Ctx& cx, const FwdArgs
   const __nv_bfloat16* zg = static_cast<const __nv_bfloat16*>(a.prep.z);
   float dtb = 0.f, dec = 0.f;  // gate constants, loaded while the chunk's copies are in flight
   if constexpr (PREP) {
-    load_raw_issue_prep<NTHR>(cx, qg, kg, vg, zg, a.beta, b, T, t0, L, a.H, a.HV, h, hv);
+    if (!PRELOADED) load_raw_issue_prep<NTHR>(cx, qg, kg, vg, zg, a.beta, b, T, t0, L, a.H, a.HV, h, hv);
     dtb = a.prep.dt_bias[(size_t)hv * KD + (tid & 127)];
     dec = a.prep.A_log[hv];
     if (Ln > 0) prefetch_chunk(cx, qg, kg, vg, zg, b, T, t0 + C, Ln, a.H, a.HV, h, hv, 2);
   } else {
-    load_raw_issue<NTHR>(cx, qg, kg, vg, a.g, a.beta, b, T, t0, L, a.H, a.HV, h, hv);
+    if (!PRELOADED) load_raw_issue<NTHR>(cx, qg, kg, vg, a.g, a.beta, b, T, t0, L, a.H, a.HV, h, hv);
     if (Ln > 0) prefetch_chunk(cx, qg, kg, vg, a.g, b, T, t0 + C, Ln, a.H, a.HV, h, hv);
   }
   if (!load_raw_wait(cx)) return false;
@@ -180,6 +183,14 @@ __device__ __forceinline__ bool fwd_chunk_head(const tcc::Ctx& cx, const FwdArgs
   }
 
   readout_ap<NTHR>(cx, tm + TM_APA, tm + TM_APB, wide, pw, irec);
+  if (img) {  // P is final: store its image now (R_P is not touched again in this chunk)
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 32) {
+      bulk_s2g(img + FWI_P, sb + R_P, FWI_EL - FWI_P);
+      bulk_commit();
+    }
+  }
   invert<NTHR>(cx);
   {  // T as the operand image (rows i, K = j); with a record also its T, T^T images and Ah
     const float* tr = reinterpret_cast<const float*>(sm + R_TROW);
@@ -425,11 +436,11 @@ __global__ void __launch_bounds__(PREP_NT, 1) kda_fwd_prep_tc_kernel(FwdArgs a) 
   cx.tm = tm;
   uint32_t phase = 0;
   bool failed = false;
-  // persistent: this CTA takes items blockIdx.x, + gridDim.x, ...  (An L2
-  // prefetch of the next item's rows measured slower: it queues behind the
-  // image stores.)
-  for (int item = blockIdx.x; item < items; item += gridDim.x) {
-    int hv, b, t0, L;
+  // persistent: this CTA takes items blockIdx.x, + gridDim.x, ...; the raw
+  // rows of the next item are requested as soon as the current item's
+  // products have consumed the raw region (its tail stages W and U0^T in the
+  // operand region instead), so their latency hides behind the tail.
+  const auto span_of = [&](int item, int& hv, int& b, int& t0, int& L) {
     if (a.ctab) {
       const int c = item % a.NC;
       hv = item / a.NC;
@@ -443,26 +454,49 @@ __global__ void __launch_bounds__(PREP_NT, 1) kda_fwd_prep_tc_kernel(FwdArgs a) 
       t0 = ch * C;
       L = min(C, a.T - t0);
     }
+  };
+  const auto issue = [&](int item) {
+    int hv, b, t0, L;
+    span_of(item, hv, b, t0, L);
+    const __nv_bfloat16 *qg = static_cast<const __nv_bfloat16*>(a.q), *kg = static_cast<const __nv_bfloat16*>(a.k),
+                        *vg = static_cast<const __nv_bfloat16*>(a.v);
+    if constexpr (PREP)
+      load_raw_issue_prep<PREP_NT>(cx, qg, kg, vg, static_cast<const __nv_bfloat16*>(a.prep.z), a.beta, b, a.T, t0,
+                                   L, a.H, a.HV, hv / G, hv);
+    else
+      load_raw_issue<PREP_NT, true>(cx, qg, kg, vg, a.g, a.beta, b, a.T, t0, L, a.H, a.HV, hv / G, hv);
+  };
+  constexpr uint32_t ST_W = OP, ST_U0 = OP + (FWI_QE - FWI_W);  // tail staging of W and U0^T
+  static_assert(ST_U0 + (FWI_BYTES - FWI_U0) <= OP_QE + 32768, "staging stays inside the operand region");
+  if (blockIdx.x < items) issue(blockIdx.x);
+  for (int item = blockIdx.x; item < items; item += gridDim.x) {
+    int hv, b, t0, L;
+    span_of(item, hv, b, t0, L);
     const int h = hv / G;
-    if ((tid & 31) == 0 && tid < 96) bulk_wait_read();  // the previous item's image stores have left smem
+    if ((tid & 31) == 0 && tid < 96) bulk_wait_read();  // the previous item's W and U0^T have left smem
     __syncthreads();
     float* irec = a.inter ? a.inter + (size_t)item * INTER_REC : nullptr;  // (item = chunk_gc)
     unsigned char* img = a.img + (size_t)item * FWI_BYTES;
-    if (!fwd_chunk_head<PREP_NT, PREP>(cx, a, b, hv, h, t0, L, 0, irec, img, bar, phase)) {
+    if (!fwd_chunk_head<PREP_NT, PREP, true>(cx, a, b, hv, h, t0, L, 0, irec, img, bar, phase)) {
       failed = true;
       break;
     }
+    // the products have read the raw region (T image) and the operands; P, Q~ o e^c,
+    // (K o e^{c_last-c})^T and e^{c_last} must have left smem before the region is reused
+    if ((tid & 31) == 0 && tid < 96) bulk_wait_read();
+    __syncthreads();
+    if (item + (int)gridDim.x < items) issue(item + gridDim.x);
     constexpr int CW = 64 / (PREP_NT / 128);  // columns of W^T / U0^T per warp group
     {  // W (rows i, K = f) padded, from W^T in TMEM (lane f)
       float v[CW];
       tmem_ldn<CW>(tm + lo + TM_W + hcol * CW, v);
 #pragma unroll
-      for (int jj = 0; jj < CW; ++jj) st_tf32(sm, R_WOP + kmaj_pad(hcol * CW + jj, Lr, 128), v[jj]);
+      for (int jj = 0; jj < CW; ++jj) st_tf32(sm, ST_W + kmaj_pad(hcol * CW + jj, Lr, 128), v[jj]);
     }
-    {  // U0^T (lane n) as [i][n], staged over (diag(beta) K o e^c)^T (consumed by the W product)
+    {  // U0^T (lane n) as [i][n]
       float u[CW];
       tmem_ldn<CW>(tm + lo + TM_U + hcol * CW, u);
-      float* dst = reinterpret_cast<float*>(sm + OP_BKET);
+      float* dst = reinterpret_cast<float*>(sm + ST_U0);
 #pragma unroll
       for (int jj = 0; jj < CW; ++jj) dst[(hcol * CW + jj) * VD + Lr] = u[jj];
     }
@@ -470,12 +504,12 @@ __global__ void __launch_bounds__(PREP_NT, 1) kda_fwd_prep_tc_kernel(FwdArgs a) 
     fence_before();
     __syncthreads();
     if ((tid & 31) == 0 && tid < 96) {
-      if (tid == 0) bulk_s2g(img + FWI_W, sb + R_WOP, FWI_QE - FWI_W);
-      if (tid == 32) bulk_s2g(img + FWI_P, sb + R_P, FWI_EL - FWI_P);
-      if (tid == 64) bulk_s2g(img + FWI_U0, sb + OP_BKET, FWI_BYTES - FWI_U0);
+      if (tid == 0) bulk_s2g(img + FWI_W, sb + ST_W, FWI_QE - FWI_W);
+      if (tid == 64) bulk_s2g(img + FWI_U0, sb + ST_U0, FWI_BYTES - FWI_U0);
       bulk_commit();
     }
   }
+  cp_async_wait_all();  // (a prefetch still in flight after an early exit)
   if ((tid & 31) == 0 && tid < 96) bulk_wait_read();
   fence_before();
   __syncthreads();
