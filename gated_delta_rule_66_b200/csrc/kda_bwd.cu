@@ -436,8 +436,7 @@ static int launch_bwd_t(const BwdArgs& a, cudaStream_t stream) {
   const int NT = (a.T + C - 1) / C;
   const bool tc = bwd_tc_eligible(a, sizeof(TIn) == 2 ? 1 : 0);
   if (tc) {
-    int rc = launch_bwd_dstate_tc(a, stream);
-    if (!rc) rc = launch_bwd_grads_tc(a, stream);
+    int rc = launch_bwd_tc_passes(a, stream);
     if (!rc) rc = launch_assemble<TIn>(a, stream);
     if (rc) return rc;
   } else {

@@ -19,6 +19,8 @@
 // the chunk's first half); the per-chunk gradient kernel reads it there.
 #include <cuda_bf16.h>
 
+#include <mutex>
+
 #include "kda_internal.h"
 #include "kda_tc_chunk.cuh"
 
@@ -53,7 +55,8 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_dstate_tc_kernel(BwdArgs a) {
   const int tid = cx.tid, hcol = cx.hcol, Lr = cx.Lr;
   const uint32_t lo = cx.lo, sb = cx.sb;
 
-  const int hv = blockIdx.x, sq = blockIdx.y;  // batch row, or sequence of a packed batch
+  const int head_ = a.head0 + blockIdx.x;
+  const int hv = head_ % a.HV, sq = head_ / a.HV;  // batch row, or sequence of a packed batch
   const int b = row_of(a, sq), c0 = chunk_begin(a, sq), c1 = chunk_end(a, sq);
   const int G = a.HV / a.H, h = hv / G, T = a.T;
   const size_t head = (size_t)sq * a.HV + hv;
@@ -242,11 +245,11 @@ bool bwd_tc_eligible(const BwdArgs& a, int dtype) {
          al16(a.k) && al16(a.v) && al16(a.dO) && al16(a.g) && al16(a.dq);
 }
 
-int launch_bwd_dstate_tc(const BwdArgs& a, cudaStream_t stream) {
+static int launch_bwd_dstate_tc(const BwdArgs& a, int nheads, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(kda_bwd_dstate_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)tcc::SMEM_BYTES);
   if (e != cudaSuccess) return set_cuda_error("kda_bwd: cudaFuncSetAttribute", e);
-  kda_bwd_dstate_tc_kernel<<<dim3(a.HV, a.B), tcc::NTH, tcc::SMEM_BYTES, stream>>>(a);
+  kda_bwd_dstate_tc_kernel<<<nheads, tcc::NTH, tcc::SMEM_BYTES, stream>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return set_cuda_error("kda_bwd: tensor-core state-gradient launch", e);
   return 0;
@@ -303,13 +306,9 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
   const int tid = cx.tid, hcol = cx.hcol, Lr = cx.Lr, lane = cx.lane;
   const uint32_t lo = cx.lo, sb = cx.sb;
 
-  // chunk ch of batch row sq (packed sequences: chunk ch of the table, sq = 0)
-  const int ch = blockIdx.x, hv = blockIdx.y, sq = blockIdx.z;
-  const int G = a.HV / a.H, h = hv / G, T = a.T, b = row_of(a, sq);
-  const int2 sp = chunk_span(a, ch);
-  const int t0 = sp.x, L = sp.y;
-  const size_t gc = chunk_gc(a, sq, hv, ch);
-  float* rec = a.gws + gc * GREC;
+  const int G = a.HV / a.H, T = a.T;
+  const int NT = a.ctab ? a.NC : (T + C - 1) / C;
+  const int items = a.item1 > 0 ? a.item1 : NT * a.HV * (a.ctab ? 1 : a.B);
   const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(a.q);
   const __nv_bfloat16* kg = static_cast<const __nv_bfloat16*>(a.k);
   const __nv_bfloat16* vg = static_cast<const __nv_bfloat16*>(a.v);
@@ -335,7 +334,15 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
   uint32_t phase = 0;
   bool failed = false;
 
-  do {
+  // one item per CTA: chunk ch of batch row sq (packed sequences: chunk ch of
+  // the table, sq = 0); items run chunk fastest, then value head, then batch row
+  for (int item = a.item0 + blockIdx.x; item < items && !failed; item += gridDim.x) {
+    const int ch = item % NT, hv = (item / NT) % a.HV, sq = item / (NT * a.HV);
+    const int h = hv / G, b = row_of(a, sq);
+    const int2 sp = chunk_span(a, ch);
+    const int t0 = sp.x, L = sp.y;
+    const size_t gc = chunk_gc(a, sq, hv, ch);
+    float* rec = a.gws + gc * GREC;
     // ---------------------------------------------------------------- loads
     const float* irec = a.inter + gc * INTER_REC;  // P^T, T, T^T images of this chunk (forward)
     const float* mst = a.states + state_slot(a, sq, hv, ch) * (KD * VD);     // M: state entering the chunk
@@ -548,7 +555,11 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
         bulk_wait_read();
       }
     }
-  } while (false);
+    // the record's shared-memory sources are read and every TMEM read-out is
+    // complete before the next item overwrites them
+    fence_before();
+    __syncthreads();
+  }
 
   fence_before();
   __syncthreads();
@@ -556,16 +567,81 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
   if (failed && tid == 0) atomicOr(&g_kda_bwd_device_error, 1u);
 }
 
-int launch_bwd_grads_tc(const BwdArgs& a, cudaStream_t stream) {
+static int launch_bwd_grads_tc(const BwdArgs& a, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(kda_bwd_grads_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)tcc::SMEM_BYTES);
   if (e != cudaSuccess) return set_cuda_error("kda_bwd: cudaFuncSetAttribute", e);
   const int NT = a.ctab ? a.NC : (a.T + tcc::C - 1) / tcc::C;
   if (NT == 0) return 0;  // (packed batches of empty sequences)
-  kda_bwd_grads_tc_kernel<<<dim3(NT, a.HV, a.ctab ? 1 : a.B), tcc::NTH, tcc::SMEM_BYTES, stream>>>(a);
+  const long long items = (a.item1 > 0 ? a.item1 : (long long)NT * a.HV * (a.ctab ? 1 : a.B)) - a.item0;
+  if (items <= 0) return 0;
+  // one CTA per item (not persistent): when the kernel shares the GPU with the
+  // state-gradient pass, the SMs that pass frees take the remaining items
+  kda_bwd_grads_tc_kernel<<<(int)items, tcc::NTH, tcc::SMEM_BYTES, stream>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return set_cuda_error("kda_bwd: tensor-core gradient launch", e);
   return 0;
+}
+
+// A non-blocking stream of the highest priority on the current device, made
+// on first use and kept until exit (null if it cannot be made).
+static cudaStream_t side_stream() {
+  static std::mutex mu;
+  static cudaStream_t streams[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!streams[dev]) {
+    int lo = 0, hi = 0;
+    cudaStream_t s = nullptr;
+    if (cudaDeviceGetStreamPriorityRange(&lo, &hi) == cudaSuccess &&
+        cudaStreamCreateWithPriority(&s, cudaStreamNonBlocking, hi) == cudaSuccess)
+      streams[dev] = s;
+    else
+      cudaGetLastError();
+  }
+  return streams[dev];
+}
+
+// The reverse state-gradient pass and the per-chunk gradient products.  The
+// pass has one CTA per (sequence, value head) and one CTA per SM; when the
+// heads fill some waves of SMs and leave a partial last wave, that last wave
+// runs on a high-priority side stream, and the gradient products of the heads
+// already finished start on the caller's stream in the SMs it leaves idle.
+int launch_bwd_tc_passes(const BwdArgs& a, cudaStream_t stream) {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int nheads = a.B * a.HV, NT = (a.T + tcc::C - 1) / tcc::C;
+  const int nA = (nheads / sms) * sms;
+  cudaStream_t side = (!a.ctab && nA > 0 && nA < nheads) ? side_stream() : nullptr;
+  if (!side) {
+    int rc = launch_bwd_dstate_tc(a, nheads, stream);
+    return rc ? rc : launch_bwd_grads_tc(a, stream);
+  }
+  cudaEvent_t evA = nullptr, evB = nullptr;
+  cudaError_t e = cudaEventCreateWithFlags(&evA, cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&evB, cudaEventDisableTiming);
+  int rc = 0;
+  BwdArgs aA = a, aB = a;
+  aA.item0 = 0;
+  aA.item1 = nA * NT;
+  aB.head0 = nA;
+  aB.item0 = nA * NT;
+  aB.item1 = nheads * NT;
+  if (e == cudaSuccess) rc = launch_bwd_dstate_tc(aA, nA, stream);
+  if (e == cudaSuccess && !rc) e = cudaEventRecord(evA, stream);
+  if (e == cudaSuccess && !rc) e = cudaStreamWaitEvent(side, evA, 0);
+  if (e == cudaSuccess && !rc) {  // the side stream's work, joined back into the caller's stream
+    rc = launch_bwd_dstate_tc(aB, nheads - nA, side);
+    e = cudaEventRecord(evB, side);
+    if (e == cudaSuccess && !rc) rc = launch_bwd_grads_tc(aA, stream);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, evB, 0);
+  }
+  if (e == cudaSuccess && !rc) rc = launch_bwd_grads_tc(aB, stream);
+  if (evA) cudaEventDestroy(evA);
+  if (evB) cudaEventDestroy(evB);
+  if (e != cudaSuccess) return set_cuda_error("kda_bwd: side-stream ordering", e);
+  return rc;
 }
 
 }  // namespace kda

@@ -135,6 +135,10 @@ struct BwdArgs {
   const int* ctab;  // packed sequences, as in FwdArgs (null: uniform batch rows)
   const int* seq0;
   int NC;
+  // tensor-core launches over part of the problem: the state-gradient pass
+  // covers heads (sequence * HV + hv) head0 .. head0 + its grid - 1, the
+  // gradient kernel items item0 .. item1 - 1 (item1 <= 0: all)
+  int head0, item0, item1;
 };
 
 struct DecodeArgs {
@@ -190,8 +194,7 @@ int take_bwd_device_error(unsigned* out);
 size_t fwd_smem_bytes(int K);
 int launch_bwd(const BwdArgs& a, int dtype, cudaStream_t stream);
 bool bwd_tc_eligible(const BwdArgs& a, int dtype);
-int launch_bwd_dstate_tc(const BwdArgs& a, cudaStream_t stream);
-int launch_bwd_grads_tc(const BwdArgs& a, cudaStream_t stream);
+int launch_bwd_tc_passes(const BwdArgs& a, cudaStream_t stream);
 int launch_decode(const DecodeArgs& a, int K, int V, int dtype, cudaStream_t stream);
 int launch_decode_token(const DecodeTokenArgs& a, int K, int V, int dtype, cudaStream_t stream);
 int launch_short_conv(const ConvArgs& a, int dtype, cudaStream_t stream);
