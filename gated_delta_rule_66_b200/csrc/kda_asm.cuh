@@ -1,7 +1,7 @@
 // Assembly of dq, dk, dg and dbeta for one quarter of the key channels of a
-// 64-step chunk from the per-chunk gradient record, with 3xTF32 warp MMAs for
-// the interaction terms (any decay span: pair by pair where the split
-// exponents would leave fp32 range).
+// 64-step chunk from the per-chunk gradient record, with tf32 warp MMAs for
+// the interaction terms (any decay span: pair by pair, with 3xTF32 products,
+// where the split exponents would leave fp32 range).
 #pragma once
 
 #include "kda_chunk.cuh"
@@ -209,7 +209,7 @@ __device__ __forceinline__ void assemble_quarter(const BwdArgs& a, float* smem, 
     if (__syncthreads_or(wide))
       factored_terms<KQ, C, false, false, LDK, LDC>(sK, sQ, sC, sdA, sdP, sE1, sE2o, sE2d, sFlag, sDq, sDk, sDc);
     else
-      factored_terms_fused<KQ, LDK, LDC>(sK, sQ, sC, sdA, sdP, sDq, sDk, sDc);
+      factored_terms_tf32<KQ, LDK, LDC>(sK, sQ, sC, sdA, sdP, sDq, sDk, sDc);
   }
   cumsum64<true>(sDc, sSeg, sLast);
   TIn* dq = static_cast<TIn*>(a.dq);

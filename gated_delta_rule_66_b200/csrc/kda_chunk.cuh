@@ -484,22 +484,33 @@ __device__ void factored_block_mma(int J, const float* sK, const float* sQ, cons
   __syncthreads();
 }
 
-// The interaction terms of factored_terms for C = 64 with 3xTF32 warp MMAs,
-// one pass, no shared scratch and no barriers: warp w owns the 16 x 16 output
+// The interaction terms of factored_terms for C = 64 on tf32 warp MMAs, one
+// pass, no shared scratch and no barriers: warp w owns the 16 x 16 output
 // tile of row block I = w / 2 and channels 16 (w % 2) .. + 15 (K = 32) and
 // accumulates in registers, over every column block J <= I, the row terms of
 // its rows and the column terms of the same rows (columns of block I); each
-// split A fragment feeds both 8-channel halves.  The split-exponent factors
-// are formed on the fly from c (natural units).  Requires every 16-row
-// block's decay span to be at most 80 (checked by the caller).
+// A fragment feeds both 8-channel halves.  The split-exponent factors are
+// formed on the fly from c (natural units).  Requires every 16-row block's
+// decay span to be at most 80 (checked by the caller).
+// Each product rounds its operands to tf32 once.  Every pair (i, j) enters
+// dc twice, as a row term of i and as a column term of j, and the reverse
+// cumulative sum of dc cancels the pairs that do not straddle the row; so
+// that this cancellation is exact, both entries of a pair are formed from
+// the same rounded factors: the row term multiplies its product by the
+// rounded operand that the column term of the pair feeds to the MMA (and the
+// other way round), and both use the same reference row of the split
+// exponent.  dq and dk keep the fp32 factors.  (Splitting the operands into
+// tf32 hi/lo pairs instead, with three products each, costs twice the time.)
+__device__ __forceinline__ float tf32f(float x) { return __uint_as_float(to_tf32(x)); }
+
 template <int K, int LDK_ = K + 1, int LDC_ = 65>
-__device__ void factored_terms_fused(const float* sK, const float* sQ, const float* sC, const float* sdA,
-                                     const float* sdP, float* sDq, float* sDk, float* sDc) {
+__device__ void factored_terms_tf32(const float* sK, const float* sQ, const float* sC, const float* sdA,
+                                    const float* sdP, float* sDq, float* sDk, float* sDc) {
   constexpr int C = 64, LDK = LDK_, LDC = LDC_, NH = K / 16;
   static_assert(4 * NH == NTHREADS / 32, "one 16 x 16 tile per warp");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int I = warp / NH, fb = (warp % NH) * 16, i0 = I * BS;
-  float totA[2][4] = {}, totP[2][4] = {};
+  float totA[2][4] = {}, totP[2][4] = {}, dcr[2][4] = {};
   // row terms: rows of block I against the columns of every block J <= I
   for (int J = 0; J <= I; ++J) {
     const int r0 = J * BS, ref = (I == J) ? r0 + BS / 2 - 1 : r0 + BS - 1;
@@ -507,24 +518,18 @@ __device__ void factored_terms_fused(const float* sK, const float* sQ, const flo
 #pragma unroll
     for (int ks = 0; ks < 2; ++ks) {
       const int j = r0 + ks * 8 + t;
-      Split aA[4], aP[4];
-      aA[0] = split_tf32(sdA[(i0 + g) * LDC + j]);
-      aA[1] = split_tf32(sdA[(i0 + g + 8) * LDC + j]);
-      aA[2] = split_tf32(sdA[(i0 + g) * LDC + j + 4]);
-      aA[3] = split_tf32(sdA[(i0 + g + 8) * LDC + j + 4]);
-      aP[0] = split_tf32(sdP[(i0 + g) * LDC + j]);
-      aP[1] = split_tf32(sdP[(i0 + g + 8) * LDC + j]);
-      aP[2] = split_tf32(sdP[(i0 + g) * LDC + j + 4]);
-      aP[3] = split_tf32(sdP[(i0 + g + 8) * LDC + j + 4]);
+      const uint32_t aA[4] = {to_tf32(sdA[(i0 + g) * LDC + j]), to_tf32(sdA[(i0 + g + 8) * LDC + j]),
+                              to_tf32(sdA[(i0 + g) * LDC + j + 4]), to_tf32(sdA[(i0 + g + 8) * LDC + j + 4])};
+      const uint32_t aP[4] = {to_tf32(sdP[(i0 + g) * LDC + j]), to_tf32(sdP[(i0 + g + 8) * LDC + j]),
+                              to_tf32(sdP[(i0 + g) * LDC + j + 4]), to_tf32(sdP[(i0 + g + 8) * LDC + j + 4])};
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int fa = fb + 8 * h + g;
         const float cr = sC[ref * LDK + fa];
-        Split bw[2];
-        bw[0] = split_tf32(sK[j * LDK + fa] * __expf(cr - sC[j * LDK + fa]));
-        bw[1] = split_tf32(sK[(j + 4) * LDK + fa] * __expf(cr - sC[(j + 4) * LDK + fa]));
-        mma3(accA[h], aA, bw);
-        mma3(accP[h], aP, bw);
+        const uint32_t bw[2] = {to_tf32(sK[j * LDK + fa] * __expf(cr - sC[j * LDK + fa])),
+                                to_tf32(sK[(j + 4) * LDK + fa] * __expf(cr - sC[(j + 4) * LDK + fa]))};
+        mma_16x8x8(accA[h], aA, bw);
+        mma_16x8x8(accP[h], aP, bw);
       }
     }
 #pragma unroll
@@ -535,6 +540,8 @@ __device__ void factored_terms_fused(const float* sK, const float* sQ, const flo
         const float e1 = __expf(sC[i * LDK + f] - sC[ref * LDK + f]);
         totA[h][e] = fmaf(accA[h][e], e1, totA[h][e]);
         totP[h][e] = fmaf(accP[h][e], e1, totP[h][e]);
+        const float ak = tf32f(sK[i * LDK + f] * e1), aq = tf32f(sQ[i * LDK + f] * e1);
+        dcr[h][e] = fmaf(accA[h][e], ak, fmaf(accP[h][e], aq, dcr[h][e]));
       }
   }
   // column terms: the columns of block I against its own rows and all rows below
@@ -542,31 +549,23 @@ __device__ void factored_terms_fused(const float* sK, const float* sQ, const flo
   const int rd = i0 + BS / 2 - 1, ro = i0 + BS - 1;
   for (int ks = 0; ks < (C - i0) / 8; ++ks) {
     const int i = i0 + ks * 8 + t, ref = (ks < 2) ? rd : ro;
-    Split aA[4], aP[4];
-    aA[0] = split_tf32(sdA[i * LDC + i0 + g]);
-    aA[1] = split_tf32(sdA[i * LDC + i0 + g + 8]);
-    aA[2] = split_tf32(sdA[(i + 4) * LDC + i0 + g]);
-    aA[3] = split_tf32(sdA[(i + 4) * LDC + i0 + g + 8]);
-    aP[0] = split_tf32(sdP[i * LDC + i0 + g]);
-    aP[1] = split_tf32(sdP[i * LDC + i0 + g + 8]);
-    aP[2] = split_tf32(sdP[(i + 4) * LDC + i0 + g]);
-    aP[3] = split_tf32(sdP[(i + 4) * LDC + i0 + g + 8]);
+    const uint32_t aA[4] = {to_tf32(sdA[i * LDC + i0 + g]), to_tf32(sdA[i * LDC + i0 + g + 8]),
+                            to_tf32(sdA[(i + 4) * LDC + i0 + g]), to_tf32(sdA[(i + 4) * LDC + i0 + g + 8])};
+    const uint32_t aP[4] = {to_tf32(sdP[i * LDC + i0 + g]), to_tf32(sdP[i * LDC + i0 + g + 8]),
+                            to_tf32(sdP[(i + 4) * LDC + i0 + g]), to_tf32(sdP[(i + 4) * LDC + i0 + g + 8])};
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int fa = fb + 8 * h + g;
       const float cr = sC[ref * LDK + fa];
       const float x0 = __expf(sC[i * LDK + fa] - cr), x1 = __expf(sC[(i + 4) * LDK + fa] - cr);
-      Split bk[2], bq[2];
-      bk[0] = split_tf32(sK[i * LDK + fa] * x0);
-      bk[1] = split_tf32(sK[(i + 4) * LDK + fa] * x1);
-      bq[0] = split_tf32(sQ[i * LDK + fa] * x0);
-      bq[1] = split_tf32(sQ[(i + 4) * LDK + fa] * x1);
+      const uint32_t bk[2] = {to_tf32(sK[i * LDK + fa] * x0), to_tf32(sK[(i + 4) * LDK + fa] * x1)};
+      const uint32_t bq[2] = {to_tf32(sQ[i * LDK + fa] * x0), to_tf32(sQ[(i + 4) * LDK + fa] * x1)};
       if (ks < 2) {
-        mma3(accD[h], aA, bk);
-        mma3(accD[h], aP, bq);
+        mma_16x8x8(accD[h], aA, bk);
+        mma_16x8x8(accD[h], aP, bq);
       } else {
-        mma3(accO[h], aA, bk);
-        mma3(accO[h], aP, bq);
+        mma_16x8x8(accO[h], aA, bk);
+        mma_16x8x8(accO[h], aP, bq);
       }
     }
   }
@@ -575,13 +574,13 @@ __device__ void factored_terms_fused(const float* sK, const float* sQ, const flo
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const int i = i0 + g + ((e & 2) ? 8 : 0), f = fb + 8 * h + 2 * t + (e & 1), o = i * LDK + f;
-      const float ci = sC[o];
-      const float col =
-          accD[h][e] * __expf(sC[rd * LDK + f] - ci) + accO[h][e] * __expf(sC[ro * LDK + f] - ci);
-      const float kk = sK[o];
+      const float ci = sC[o], kk = sK[o];
+      const float yd = __expf(sC[rd * LDK + f] - ci), yo = __expf(sC[ro * LDK + f] - ci);
+      const float col = accD[h][e] * yd + accO[h][e] * yo;
+      const float dcc = accD[h][e] * tf32f(kk * yd) + accO[h][e] * tf32f(kk * yo);
       sDk[o] += totA[h][e] + col;
       sDq[o] += totP[h][e];
-      sDc[o] += kk * (totA[h][e] - col) + sQ[o] * totP[h][e];
+      sDc[o] += dcr[h][e] - dcc;
     }
   __syncthreads();
 }
