@@ -459,7 +459,9 @@ __device__ __forceinline__ void readout_ap(const Ctx& c, uint32_t tm_apa, uint32
 // solved by forward substitution with a whole column per thread in
 // registers; the blocks below follow in three levels of block substitution,
 // T_IJ = -T_II sum_{J<=L<I} A_IL T_LJ (level = block distance I - J), one
-// warp per block, as 3xTF32 warp MMAs (fp32-accurate).
+// warp per block, as tf32 warp MMAs.  (T enters the state products as a tf32
+// operand anyway; hi/lo-split products here measured no better in o and cost
+// 0.06 ms per forward on the fwd+bwd workload.)
 template <int NT = NTH>
 __device__ __forceinline__ void invert(const Ctx& c) {
   constexpr int LD = 65;
@@ -499,17 +501,14 @@ __device__ __forceinline__ void invert(const Ctx& c) {
       const float bg = sB[ri + g], bg8 = sB[ri + g + 8];
       for (int ks = 0; ks < 2 * d; ++ks) {
         const int l = 16 * J + 8 * ks + t4;
-        Split a[4];
-        a[0] = split_tf32(bg * sAh[(ri + g) * LD + l]);
-        a[1] = split_tf32(bg8 * sAh[(ri + g + 8) * LD + l]);
-        a[2] = split_tf32(bg * sAh[(ri + g) * LD + l + 4]);
-        a[3] = split_tf32(bg8 * sAh[(ri + g + 8) * LD + l + 4]);
+        const uint32_t a[4] = {to_tf32(bg * sAh[(ri + g) * LD + l]), to_tf32(bg8 * sAh[(ri + g + 8) * LD + l]),
+                               to_tf32(bg * sAh[(ri + g) * LD + l + 4]),
+                               to_tf32(bg8 * sAh[(ri + g + 8) * LD + l + 4])};
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
-          Split bb[2];
-          bb[0] = split_tf32(sT[l * LD + 16 * J + nt * 8 + g]);
-          bb[1] = split_tf32(sT[(l + 4) * LD + 16 * J + nt * 8 + g]);
-          mma3(acc[nt], a, bb);
+          const uint32_t bb[2] = {to_tf32(sT[l * LD + 16 * J + nt * 8 + g]),
+                                  to_tf32(sT[(l + 4) * LD + 16 * J + nt * 8 + g])};
+          mma_16x8x8(acc[nt], a, bb);
         }
       }
       float* w = sW + warp * 256;
@@ -523,17 +522,13 @@ __device__ __forceinline__ void invert(const Ctx& c) {
 #pragma unroll
       for (int ks = 0; ks < 2; ++ks) {
         const int m = 8 * ks + t4;
-        Split a[4];
-        a[0] = split_tf32(sT[(ri + g) * LD + ri + m]);
-        a[1] = split_tf32(sT[(ri + g + 8) * LD + ri + m]);
-        a[2] = split_tf32(sT[(ri + g) * LD + ri + m + 4]);
-        a[3] = split_tf32(sT[(ri + g + 8) * LD + ri + m + 4]);
+        const uint32_t a[4] = {to_tf32(sT[(ri + g) * LD + ri + m]), to_tf32(sT[(ri + g + 8) * LD + ri + m]),
+                               to_tf32(sT[(ri + g) * LD + ri + m + 4]),
+                               to_tf32(sT[(ri + g + 8) * LD + ri + m + 4])};
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
-          Split bb[2];
-          bb[0] = split_tf32(w[m * 16 + nt * 8 + g]);
-          bb[1] = split_tf32(w[(m + 4) * 16 + nt * 8 + g]);
-          mma3(tt[nt], a, bb);
+          const uint32_t bb[2] = {to_tf32(w[m * 16 + nt * 8 + g]), to_tf32(w[(m + 4) * 16 + nt * 8 + g])};
+          mma_16x8x8(tt[nt], a, bb);
         }
       }
 #pragma unroll
