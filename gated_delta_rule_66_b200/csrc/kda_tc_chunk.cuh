@@ -460,8 +460,9 @@ __device__ __forceinline__ void readout_ap(const Ctx& c, uint32_t tm_apa, uint32
 // registers; the blocks below follow in three levels of block substitution,
 // T_IJ = -T_II sum_{J<=L<I} A_IL T_LJ (level = block distance I - J), one
 // warp per block, as tf32 warp MMAs.  (T enters the state products as a tf32
-// operand anyway; hi/lo-split products here measured no better in o and cost
-// 0.06 ms per forward on the fwd+bwd workload.)
+// operand anyway; with single products here the o error stays ~0.5e-3 above
+// the bf16 rounding floor, and hi/lo-split products cost 0.06 ms more per
+// forward on the fwd+bwd workload.)
 template <int NT = NTH>
 __device__ __forceinline__ void invert(const Ctx& c) {
   constexpr int LD = 65;
