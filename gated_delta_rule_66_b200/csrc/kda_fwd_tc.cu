@@ -132,6 +132,10 @@ __device__ __forceinline__ bool fwd_chunk_head(const tcc::Ctx& cx, const FwdArgs
   } else {
     wide = cumsum_span(cx);
   }
+  if constexpr (PRELOADED) {  // the previous item's W and U0^T bulk stores have read the operand region
+    if ((tid & 31) == 0 && tid < 96) bulk_wait_read();
+    __syncthreads();
+  }
   build_op1_and_issue<NTHR, PREP>(cx, a.scale, tm + TM_APA, tm + TM_APB, bar);
   if (!wait_mma(bar, phase)) return false;
 
@@ -473,8 +477,9 @@ __global__ void __launch_bounds__(PREP_NT, 1) kda_fwd_prep_tc_kernel(FwdArgs a) 
     int hv, b, t0, L;
     span_of(item, hv, b, t0, L);
     const int h = hv / G;
-    if ((tid & 31) == 0 && tid < 96) bulk_wait_read();  // the previous item's W and U0^T have left smem
-    __syncthreads();
+    // (the previous item's W and U0^T leave the operand region while this
+    // item's raw rows are waited for and its decay is summed: fwd_chunk_head
+    // waits for them just before it builds its first operands)
     float* irec = a.inter ? a.inter + (size_t)item * INTER_REC : nullptr;  // (item = chunk_gc)
     unsigned char* img = a.img + (size_t)item * FWI_BYTES;
     if (!fwd_chunk_head<PREP_NT, PREP, true>(cx, a, b, hv, h, t0, L, 0, irec, img, bar, phase)) {
