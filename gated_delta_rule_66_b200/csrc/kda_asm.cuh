@@ -80,6 +80,11 @@ __device__ __forceinline__ void assemble_quarter(const BwdArgs& a, float* smem, 
   // [dQE; dKE'] and dKEd of this quarter, consumed further down: lane = channel f,
   // warp w = rows 8w .. 8w + 7 (each row a 128-byte run of the row-major record)
   const int ef = tid & 31, ei = (tid >> 5) * 8;
+  // Ah of row 16 fq4 + tid / 16, columns 4 (tid % 16) .. + 3 (for dbeta; rows past L are zero)
+  const float4 ah4 = (16 * fq4 + (tid >> 4) < L)
+                         ? *reinterpret_cast<const float4*>(a.inter + gc * INTER_REC + INTER_AH +
+                                                            (16 * fq4 + (tid >> 4)) * 64 + (tid & 15) * 4)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
   float qe[8], ke[8], kd[8];
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
@@ -112,6 +117,12 @@ __device__ __forceinline__ void assemble_quarter(const BwdArgs& a, float* smem, 
       dp[m] = *reinterpret_cast<const float4*>(rec + G_PA + rec_off(i, j4, 64));
       da[m] = *reinterpret_cast<const float4*>(rec + G_PA + rec_off(64 + i, j4, 64));
     }
+    float bt[4];  // beta of the rows of the [dA] items
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int i = (tid >> 4) + 16 * m;
+      bt[m] = (i < L) ? a.beta[((size_t)b * T + t0 + i) * a.HV + hv] : 0.f;
+    }
     if (tid < C) sBeta[tid] = (tid < L) ? a.beta[((size_t)b * T + t0 + tid) * a.HV + hv] : 0.f;
 #pragma unroll
     for (int m = 0; m < 2; ++m) {
@@ -137,34 +148,22 @@ __device__ __forceinline__ void assemble_quarter(const BwdArgs& a, float* smem, 
       wa.y = (j4 + 1 < i) ? vda[1] : 0.f;
       wa.z = (j4 + 2 < i) ? vda[2] : 0.f;
       wa.w = (j4 + 3 < i) ? vda[3] : 0.f;
+      if (m == fq4) {  // dbeta = dbeta_R + sum_{j<i} dA_ij Ah_ij for this quarter's 16 rows (16 threads per row)
+        float sb = fmaf(wa.x, ah4.x, fmaf(wa.y, ah4.y, fmaf(wa.z, ah4.z, wa.w * ah4.w)));
+#pragma unroll
+        for (int off = 8; off > 0; off >>= 1) sb += __shfl_xor_sync(0xffffffffu, sb, off);
+        if ((tid & 15) == 0 && i < L) a.dbeta[((size_t)b * T + t0 + i) * a.HV + hv] = rec[G_DBR + i] + sb;
+      }
+      wa.x *= bt[m];  // the interaction terms take diag(beta) dA
+      wa.y *= bt[m];
+      wa.z *= bt[m];
+      wa.w *= bt[m];
       *reinterpret_cast<float4*>(sdP + i * LDC + j4) = wp;  // LDC = 68: rows 16-byte aligned
       *reinterpret_cast<float4*>(sdA + i * LDC + j4) = wa;
     }
   }
   __syncthreads();
   cumsum64<false>(sC, sSeg, nullptr);
-  if (fq4 == 0 && tid < L) {  // dbeta = dbeta_R + sum_{j<i} dA_ij Ah_ij (Ah read straight from the record)
-    const int i = tid;
-    const float4* arow = reinterpret_cast<const float4*>(a.inter + gc * INTER_REC + INTER_AH + i * 64);
-    float s0 = rec[G_DBR + i], s1 = 0.f;
-#pragma unroll
-    for (int j4 = 0; j4 < 16; ++j4) {
-      const float4 ah = arow[j4];
-      const float vah[4] = {ah.x, ah.y, ah.z, ah.w};
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int j = j4 * 4 + u;
-        if (u & 1) s1 = fmaf(sdA[i * LDC + j], vah[u], s1);
-        else s0 = fmaf(sdA[i * LDC + j], vah[u], s0);
-      }
-    }
-    a.dbeta[((size_t)b * T + t0 + i) * a.HV + hv] = s0 + s1;
-  }
-  __syncthreads();
-  for (int idx = tid; idx < C * C; idx += NTHREADS) {
-    const int i = idx >> 6, j = idx & 63;
-    sdA[i * LDC + j] *= sBeta[i];
-  }
   {  // element-wise terms; the chunk-end sum of dKEd o k o e^{c_last-c} goes through sE1
 #pragma unroll
     for (int m = 0; m < 2; ++m) {
