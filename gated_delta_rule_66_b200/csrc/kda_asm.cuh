@@ -29,6 +29,29 @@ struct AsmSmem {
   static constexpr size_t bytes = (size_t)total * sizeof(float);
 };
 
+// Four consecutive q or k values (16-byte aligned fp32 or 8-byte aligned bf16)
+__device__ __forceinline__ void load4(const float* p, float (&o)[4]) {
+  const float4 v = *reinterpret_cast<const float4*>(p);
+  o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+}
+__device__ __forceinline__ void load4(const __nv_bfloat16* p, float (&o)[4]) {
+  const uint2 r = *reinterpret_cast<const uint2*>(p);
+  const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&r.x);
+  const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&r.y);
+  o[0] = __low2float(lo); o[1] = __high2float(lo); o[2] = __low2float(hi); o[3] = __high2float(hi);
+}
+
+__device__ __forceinline__ void store4(float* p, float x, float y, float z, float w) {
+  *reinterpret_cast<float4*>(p) = make_float4(x, y, z, w);
+}
+__device__ __forceinline__ void store4(__nv_bfloat16* p, float x, float y, float z, float w) {
+  const __nv_bfloat162 lo = __floats2bfloat162_rn(x, y), hi = __floats2bfloat162_rn(z, w);
+  uint2 r;
+  r.x = *reinterpret_cast<const uint32_t*>(&lo);
+  r.y = *reinterpret_cast<const uint32_t*>(&hi);
+  *reinterpret_cast<uint2*>(p) = r;
+}
+
 // Inclusive (forward) or reverse cumulative sum over the C = 64 rows of each
 // of the KQ = 32 columns of a [64][LDK] array, by 8 segments of 8 rows
 // (256 threads; seg is 8 x KQ scratch; `base` is added to every element of a
@@ -104,11 +127,8 @@ __device__ __forceinline__ void assemble_quarter(const BwdArgs& a, float* smem, 
       if (i < L) {
         const size_t rq = (((size_t)b * T + t0 + i) * a.H + h) * KD + f0 + f4;
         gv[m] = *reinterpret_cast<const float4*>(a.g + (((size_t)b * T + t0 + i) * a.HV + hv) * KD + f0 + f4);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          qv[m][u] = to_f(q[rq + u]);
-          kv[m][u] = to_f(k[rq + u]);
-        }
+        load4(q + rq, qv[m]);
+        load4(k + rq, kv[m]);
       }
     }
 #pragma unroll
@@ -128,12 +148,11 @@ __device__ __forceinline__ void assemble_quarter(const BwdArgs& a, float* smem, 
     for (int m = 0; m < 2; ++m) {
       const int idx = tid + m * NTHREADS, i = idx >> 3, f4 = (idx & 7) * 4;
       const float gg[4] = {gv[m].x, gv[m].y, gv[m].z, gv[m].w};
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        sQ[i * LDK + f4 + u] = qv[m][u] * a.scale;
-        sK[i * LDK + f4 + u] = kv[m][u];
-        sC[i * LDK + f4 + u] = gg[u];
-      }
+      // (LDK = 40: rows 16-byte aligned)
+      *reinterpret_cast<float4*>(sQ + i * LDK + f4) =
+          make_float4(qv[m][0] * a.scale, qv[m][1] * a.scale, qv[m][2] * a.scale, qv[m][3] * a.scale);
+      *reinterpret_cast<float4*>(sK + i * LDK + f4) = make_float4(kv[m][0], kv[m][1], kv[m][2], kv[m][3]);
+      *reinterpret_cast<float4*>(sC + i * LDK + f4) = make_float4(gg[0], gg[1], gg[2], gg[3]);
     }
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
@@ -213,6 +232,28 @@ __device__ __forceinline__ void assemble_quarter(const BwdArgs& a, float* smem, 
   cumsum64<true>(sDc, sSeg, sLast);
   TIn* dq = static_cast<TIn*>(a.dq);
   TIn* dk = static_cast<TIn*>(a.dk);
+  const uintptr_t al = (uintptr_t)a.dg | (G == 1 ? ((uintptr_t)dq | (uintptr_t)dk)
+                                                 : ((uintptr_t)a.dq_part | (uintptr_t)a.dk_part));
+  if ((al & 15u) == 0) {  // four channels per item, 16-byte (fp32) and 8-byte (bf16) stores
+    for (int idx = tid; idx < L * (KQ / 4); idx += NTHREADS) {
+      const int i = idx / (KQ / 4), f = (idx % (KQ / 4)) * 4, o = i * LDK + f;
+      const size_t row_v = ((size_t)b * T + t0 + i) * a.HV + hv;
+      const float4 c4 = *reinterpret_cast<const float4*>(sDc + o), q4 = *reinterpret_cast<const float4*>(sDq + o),
+                   k4 = *reinterpret_cast<const float4*>(sDk + o);
+      *reinterpret_cast<float4*>(a.dg + row_v * KD + f0 + f) = c4;
+      const float sc = a.scale;
+      if (G == 1) {
+        const size_t row_h = ((size_t)b * T + t0 + i) * a.H + h;
+        store4(dq + row_h * KD + f0 + f, sc * q4.x, sc * q4.y, sc * q4.z, sc * q4.w);
+        store4(dk + row_h * KD + f0 + f, k4.x, k4.y, k4.z, k4.w);
+      } else {
+        *reinterpret_cast<float4*>(a.dq_part + row_v * KD + f0 + f) = make_float4(sc * q4.x, sc * q4.y, sc * q4.z, sc * q4.w);
+        *reinterpret_cast<float4*>(a.dk_part + row_v * KD + f0 + f) = k4;
+      }
+    }
+    __syncthreads();
+    return;
+  }
   for (int idx = tid; idx < L * KQ; idx += NTHREADS) {
     const int i = idx / KQ, f = idx % KQ, o = i * LDK + f;
     const size_t row_v = ((size_t)b * T + t0 + i) * a.HV + hv;
