@@ -414,17 +414,21 @@ __global__ void kda_group_sum_kernel(const float* __restrict__ part, TIn* __rest
 template <typename TIn>
 __global__ void __launch_bounds__(NTHREADS, 2) kda_bwd_assemble_kernel(BwdArgs a) {
   extern __shared__ float smem[];
-  assemble_quarter<TIn>(a, smem, blockIdx.x >> 2, blockIdx.x & 3, blockIdx.y, blockIdx.z);
+  const int head = a.head0 + blockIdx.y;  // (sequence or batch row) * HV + hv
+  assemble_quarter<TIn>(a, smem, blockIdx.x >> 2, blockIdx.x & 3, head % a.HV, head / a.HV);
 }
 
+// The assembly of heads (sequence * HV + hv) head0 .. head0 + nheads - 1.
 template <typename TIn>
-static int launch_assemble(const BwdArgs& a, cudaStream_t stream) {
+static int launch_assemble(const BwdArgs& a0, int head0, int nheads, cudaStream_t stream) {
   auto kern = kda_bwd_assemble_kernel<TIn>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)AsmSmem::bytes);
   if (e != cudaSuccess) return set_cuda_error("kda_bwd: cudaFuncSetAttribute", e);
-  const int NT = a.ctab ? a.NC : (a.T + 63) / 64;
-  if (NT == 0) return 0;  // (packed batches of empty sequences)
-  kern<<<dim3(NT * 4, a.HV, a.ctab ? 1 : a.B), NTHREADS, AsmSmem::bytes, stream>>>(a);
+  const int NT = a0.ctab ? a0.NC : (a0.T + 63) / 64;
+  if (NT == 0 || nheads <= 0) return 0;  // (packed batches of empty sequences)
+  BwdArgs a = a0;
+  a.head0 = head0;
+  kern<<<dim3(NT * 4, nheads), NTHREADS, AsmSmem::bytes, stream>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return set_cuda_error("kda_bwd: assemble launch", e);
   return 0;
@@ -436,8 +440,7 @@ static int launch_bwd_t(const BwdArgs& a, cudaStream_t stream) {
   const int NT = (a.T + C - 1) / C;
   const bool tc = bwd_tc_eligible(a, sizeof(TIn) == 2 ? 1 : 0);
   if (tc) {
-    int rc = launch_bwd_tc_passes(a, stream);
-    if (!rc) rc = launch_assemble<TIn>(a, stream);
+    int rc = launch_bwd_tc_passes(a, stream, launch_assemble<TIn>);
     if (rc) return rc;
   } else {
     using S = DstSmem<K, C, VB>;

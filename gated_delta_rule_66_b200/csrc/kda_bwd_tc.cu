@@ -603,12 +603,15 @@ static cudaStream_t side_stream() {
   return streams[dev];
 }
 
-// The reverse state-gradient pass and the per-chunk gradient products.  The
-// pass has one CTA per (sequence, value head) and one CTA per SM; when the
-// heads fill some waves of SMs and leave a partial last wave, that last wave
-// runs on a high-priority side stream, and the gradient products of the heads
-// already finished start on the caller's stream in the SMs it leaves idle.
-int launch_bwd_tc_passes(const BwdArgs& a, cudaStream_t stream) {
+// The reverse state-gradient pass, the per-chunk gradient products and the
+// assembly.  The pass has one CTA per (sequence, value head) and one CTA per
+// SM; when the heads fill some waves of SMs and leave a partial last wave
+// (heads A, then B), that wave runs on a high-priority side stream while the
+// gradient products of heads A start in the SMs it leaves idle; then the
+// assembly of heads A follows on the side stream while the gradient products
+// of heads B run on the caller's stream (the two kernels load and compute in
+// different phases), and the assembly of heads B ends the call.
+int launch_bwd_tc_passes(const BwdArgs& a, cudaStream_t stream, AssembleLaunch assemble) {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int nheads = a.B * a.HV, NT = (a.T + tcc::C - 1) / tcc::C;
@@ -616,11 +619,12 @@ int launch_bwd_tc_passes(const BwdArgs& a, cudaStream_t stream) {
   cudaStream_t side = (!a.ctab && nA > 0 && nA < nheads) ? side_stream() : nullptr;
   if (!side) {
     int rc = launch_bwd_dstate_tc(a, nheads, stream);
-    return rc ? rc : launch_bwd_grads_tc(a, stream);
+    if (!rc) rc = launch_bwd_grads_tc(a, stream);
+    return rc ? rc : assemble(a, 0, nheads, stream);
   }
-  cudaEvent_t evA = nullptr, evB = nullptr;
-  cudaError_t e = cudaEventCreateWithFlags(&evA, cudaEventDisableTiming);
-  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&evB, cudaEventDisableTiming);
+  cudaEvent_t ev[3] = {nullptr, nullptr, nullptr};  // dstate(A) done, grads(A) done, side work done
+  cudaError_t e = cudaSuccess;
+  for (int i = 0; i < 3 && e == cudaSuccess; ++i) e = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming);
   int rc = 0;
   BwdArgs aA = a, aB = a;
   aA.item0 = 0;
@@ -629,17 +633,27 @@ int launch_bwd_tc_passes(const BwdArgs& a, cudaStream_t stream) {
   aB.item0 = nA * NT;
   aB.item1 = nheads * NT;
   if (e == cudaSuccess) rc = launch_bwd_dstate_tc(aA, nA, stream);
-  if (e == cudaSuccess && !rc) e = cudaEventRecord(evA, stream);
-  if (e == cudaSuccess && !rc) e = cudaStreamWaitEvent(side, evA, 0);
+  if (e == cudaSuccess && !rc) e = cudaEventRecord(ev[0], stream);
+  if (e == cudaSuccess && !rc) e = cudaStreamWaitEvent(side, ev[0], 0);
   if (e == cudaSuccess && !rc) {  // the side stream's work, joined back into the caller's stream
     rc = launch_bwd_dstate_tc(aB, nheads - nA, side);
-    e = cudaEventRecord(evB, side);
+    cudaEvent_t evB = nullptr;
+    if (!rc) e = cudaEventCreateWithFlags(&evB, cudaEventDisableTiming);
+    if (e == cudaSuccess && !rc) e = cudaEventRecord(evB, side);
     if (e == cudaSuccess && !rc) rc = launch_bwd_grads_tc(aA, stream);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, evB, 0);
+    if (e == cudaSuccess && !rc) e = cudaEventRecord(ev[1], stream);
+    if (e == cudaSuccess && !rc) e = cudaStreamWaitEvent(side, ev[1], 0);
+    if (e == cudaSuccess && !rc) rc = assemble(a, 0, nA, side);
+    const cudaError_t e2 = cudaEventRecord(ev[2], side);
+    if (e == cudaSuccess) e = e2;
+    if (e == cudaSuccess && !rc) e = cudaStreamWaitEvent(stream, evB, 0);
+    if (e == cudaSuccess && !rc) rc = launch_bwd_grads_tc(aB, stream);
+    if (e == cudaSuccess && !rc) rc = assemble(a, nA, nheads - nA, stream);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, ev[2], 0);
+    if (evB) cudaEventDestroy(evB);
   }
-  if (e == cudaSuccess && !rc) rc = launch_bwd_grads_tc(aB, stream);
-  if (evA) cudaEventDestroy(evA);
-  if (evB) cudaEventDestroy(evB);
+  for (int i = 0; i < 3; ++i)
+    if (ev[i]) cudaEventDestroy(ev[i]);
   if (e != cudaSuccess) return set_cuda_error("kda_bwd: side-stream ordering", e);
   return rc;
 }

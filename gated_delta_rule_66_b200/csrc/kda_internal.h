@@ -194,7 +194,10 @@ int take_bwd_device_error(unsigned* out);
 size_t fwd_smem_bytes(int K);
 int launch_bwd(const BwdArgs& a, int dtype, cudaStream_t stream);
 bool bwd_tc_eligible(const BwdArgs& a, int dtype);
-int launch_bwd_tc_passes(const BwdArgs& a, cudaStream_t stream);
+// the tensor-core backward: state-gradient pass, gradient products and the
+// assembly (launched through `assemble` for a range of heads)
+typedef int (*AssembleLaunch)(const BwdArgs& a, int head0, int nheads, cudaStream_t stream);
+int launch_bwd_tc_passes(const BwdArgs& a, cudaStream_t stream, AssembleLaunch assemble);
 int launch_decode(const DecodeArgs& a, int K, int V, int dtype, cudaStream_t stream);
 int launch_decode_token(const DecodeTokenArgs& a, int K, int V, int dtype, cudaStream_t stream);
 int launch_short_conv(const ConvArgs& a, int dtype, cudaStream_t stream);
