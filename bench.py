@@ -279,8 +279,8 @@ def gpu_path(kda, name, steps, warmup, rank_barrier, shrink=None):
             if flush is not None:
                 _flush_l2(flush)
             kda.fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], scale=w.scale, initial_state=d["S0"])
-        # tensor-core shapes: chunk-parallel kernel + state pass; else one chunk kernel
-        launches_per_step = 2 if (w.dtype == "bf16" and w.K == w.V == 128) else 1
+        # chunk-parallel kernel + state pass (tensor-core or CUDA-core path, with scratch)
+        launches_per_step = 2
         tokens = w.B * w.T
     elif w.path == "fwdbwd":
         ws = torch.empty(kda.workspace_bytes("bwd", w.B, w.T, w.H, w.HV, w.K, w.V), dtype=torch.uint8,

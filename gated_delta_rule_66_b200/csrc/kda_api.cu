@@ -78,9 +78,18 @@ static size_t img_bytes(int B, int T, int HV, int K, int V) {
   return (size_t)B * HV * NT64 * FWI_BYTES;
 }
 
-// training forward: [states | interaction records | chunk images]
+// scratch of the two-kernel forwards: the chunk images of the tensor-core
+// path (K = V = 128) or the chunk records of the CUDA-core path (fp32, or
+// other K and V), whichever is larger (the dtype is not an argument here)
+static size_t scratch_bytes(int B, int T, int HV, int K, int V) {
+  if (K != 32 && K != 64 && K != 128) return 0;
+  const size_t img = img_bytes(B, T, HV, K, V), prep = fma_prep_bytes(B, T, HV, K, 1);
+  return img > prep ? img : prep;
+}
+
+// training forward: [states | interaction records | scratch]
 static size_t fwd_ws_bytes(int B, int T, int HV, int K, int V) {
-  return states_bytes(B, T, HV, K, V) + inter_bytes(B, T, HV, K, V) + img_bytes(B, T, HV, K, V);
+  return states_bytes(B, T, HV, K, V) + inter_bytes(B, T, HV, K, V) + scratch_bytes(B, T, HV, K, V);
 }
 
 // Packed sequences: the chunk table (t0, L per chunk of at most 64 steps,
@@ -147,7 +156,7 @@ size_t kda_fwd_workspace_bytes(int B, int T, int HV, int K, int V) {
 
 size_t kda_fwd_scratch_bytes(int B, int T, int HV, int K, int V) {
   if (B < 1 || T < 1 || HV < 1 || K < 1 || V < 1) return 0;
-  return img_bytes(B, T, HV, K, V);
+  return scratch_bytes(B, T, HV, K, V);
 }
 
 static size_t grads_record_bytes(int B, int T, int HV, int K, int V) {
@@ -167,7 +176,7 @@ static size_t bwd_tail_bytes(int B, int T, int H, int HV, int K, int V) {
 
 size_t kda_bwd_workspace_bytes(int B, int T, int H, int HV, int K, int V) {
   if (B < 1 || T < 1 || H < 1 || HV < 1 || K < 1 || V < 1 || HV % H) return 0;
-  const size_t tail = bwd_tail_bytes(B, T, H, HV, K, V), img = img_bytes(B, T, HV, K, V);
+  const size_t tail = bwd_tail_bytes(B, T, H, HV, K, V), img = scratch_bytes(B, T, HV, K, V);
   return states_bytes(B, T, HV, K, V) + inter_bytes(B, T, HV, K, V) + (tail > img ? tail : img);
 }
 
@@ -185,7 +194,7 @@ int kda_fwd(const void* q, const void* k, const void* v, const float* g, const f
     if (!aligned16(workspace)) return set_error(KDA_ERR_ARG, "kda_fwd: workspace must be 16-byte aligned");
     char* ws = static_cast<char*>(workspace);
     const size_t sb = states_bytes(B, T, HV, K, V), ib = inter_bytes(B, T, HV, K, V);
-    const size_t gb = img_bytes(B, T, HV, K, V);
+    const size_t gb = scratch_bytes(B, T, HV, K, V);
     if (workspace_bytes >= fwd_ws_bytes(B, T, HV, K, V)) {  // training: states for the backward
       states = reinterpret_cast<float*>(ws);
       inter = ib ? reinterpret_cast<float*>(ws + sb) : nullptr;
@@ -198,7 +207,14 @@ int kda_fwd(const void* q, const void* k, const void* v, const float* g, const f
     }
   }
   FwdArgs a{q, k, v, g, beta, S0, o, S_T, states, inter, img, scale, B, T, H, HV, K, V};
-  return launch_fwd(a, dtype, static_cast<cudaStream_t>(stream));
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (fwd_tc_eligible(a, dtype)) return launch_fwd_tc(a, st);
+  if (img && fwd_fma2_eligible(a, img)) {  // the scratch holds the CUDA-core path's chunk records
+    a.img = nullptr;
+    return launch_fwd_fma2(a, dtype, false, reinterpret_cast<float*>(img), st);
+  }
+  a.img = nullptr;
+  return launch_fwd_ffma(a, dtype, st);
 }
 
 size_t kda_fwd_varlen_workspace_bytes(const int* cu_seqlens, int N, int HV, int K, int V) {
@@ -321,9 +337,14 @@ int kda_decode_step(const void* q, const void* k, const void* v, const float* g,
   return launch_decode(a, K, V, dtype, static_cast<cudaStream_t>(stream));
 }
 
+size_t kda_fwd_erase_workspace_bytes(int B, int T, int HQ, int HV, int K, int V) {
+  if (B < 1 || T < 1 || HQ < 1 || HV < 1 || HQ % HV || V < 1 || (K != 32 && K != 64 && K != 128)) return 0;
+  return fma_prep_bytes(B, T, HV, K, HQ / HV);
+}
+
 int kda_fwd_erase(const void* q, const void* k, const void* e, const void* z, const float* g, const float* S0,
                   float scale, int B, int T, int HQ, int HV, int K, int V, int dtype, void* o, float* S_T,
-                  void* stream) {
+                  void* workspace, size_t workspace_bytes, void* stream) {
   g_err[0] = 0;
   char buf[256];
   int rc = check_common("kda_fwd_erase", B, T, 1, 1, K, V, dtype, scale);
@@ -336,7 +357,13 @@ int kda_fwd_erase(const void* q, const void* k, const void* e, const void* z, co
     return set_error(KDA_ERR_NULL, "kda_fwd_erase: q, k, e, z, g and o must be non-NULL");
   FwdArgs a{q, k, z, g, nullptr, S0, o, S_T, nullptr, nullptr, nullptr, scale, B, T, HQ, HV, K, V};
   a.erase = e;
-  return launch_fwd_erase(a, dtype, static_cast<cudaStream_t>(stream));
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (workspace) {
+    if (workspace_bytes < kda_fwd_erase_workspace_bytes(B, T, HQ, HV, K, V))
+      return set_error(KDA_ERR_WORKSPACE, "kda_fwd_erase: workspace smaller than kda_fwd_erase_workspace_bytes()");
+    if (fwd_fma2_eligible(a, workspace)) return launch_fwd_fma2(a, dtype, true, static_cast<float*>(workspace), st);
+  }
+  return launch_fwd_erase(a, dtype, st);
 }
 
 static int check_gate(const char* fn, const void* z, const float* A_log, const float* dt_bias, float lb,

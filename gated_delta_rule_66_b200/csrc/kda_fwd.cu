@@ -11,6 +11,7 @@
 // state carry) with fp32 FMA on a 16 x 16 thread grid.
 #include "kda_chunk.cuh"
 #include "kda_internal.h"
+#include "kda_tc.cuh"
 
 namespace kda {
 
@@ -207,6 +208,310 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       a.S_T[(head * K + f) * V + v0 + n] = sM[f * LDV + n];
     }
   }
+}
+
+// ============================================================================
+// Two-kernel CUDA-core forward (chunk-parallel preparation + sequential state
+// pass), used when the caller gives a workspace of kda_fwd_scratch_bytes()
+// (or kda_fwd_erase_workspace_bytes()).
+//
+// The state-independent part of every chunk (interactions, inverse, decayed
+// operands) runs first for all chunks at once, one CTA per (b, state head,
+// chunk), and leaves per chunk in the workspace (FmaRec):
+//   Tb   = T diag(beta)                  C x C
+//   Rt   = Tb (R o e^c)                  C x K  (R = k; the erase rows e)
+//   KEd  = k o e^{c_last - c}            C x K
+//   El   = e^{c_last}                    K
+//   per query head: P (C x C) and Q~ o e^c (C x K)
+// so that the state pass only applies, per chunk and V slice,
+//   U = Tb V - Rt M,   O = (Q~ o e^c) M + P U,   M' = diag(El) M + KEd^T U
+// (the same chunk algebra as the single-kernel path, with the residual's two
+// terms multiplied through by Tb ahead of time).  For the erase/write variant
+// one state pass carries a state head once and reads it out for all its
+// query heads.
+// ============================================================================
+__host__ __device__ constexpr int fma_rec_floats(int K, int C, int QG) {
+  return C * C + 2 * C * K + K + QG * (C * C + C * K);
+}
+
+template <int K, int C, bool ERASE>
+struct PrepSmem {
+  static constexpr int LDK = K + 1, LDC = C + 1;
+  static constexpr int oK = 0, oQ = oK + C * LDK, oC = oQ + C * LDK, oE1 = oC + C * LDK,
+                       oE2o = oE1 + C * LDK, oE2d = oE2o + BS * LDK, oAh = oE2d + BS * LDK,
+                       oT = oAh + C * LDC, oP = oT + C * LDC, oW = oP + C * LDC, oBeta = oW + BS * LDC,
+                       oFlag = oBeta + C, oR = oFlag + 4, total = oR + (ERASE ? C * LDK : 0);
+  static constexpr size_t bytes = (size_t)total * sizeof(float);
+};
+
+// q~ = scale q of query head hq for one chunk (rows past the end zero)
+template <int K, int C, typename TIn>
+__device__ __forceinline__ void load_chunk_q(const FwdArgs& a, int b, int t0, int L, int hq, float* sQ) {
+  constexpr int LDK = K + 1;
+  const TIn* q = static_cast<const TIn*>(a.q);
+  for (int idx = threadIdx.x; idx < C * K; idx += NTHREADS) {
+    const int i = idx / K, f = idx % K;
+    sQ[i * LDK + f] = (i < L) ? to_f(q[(((size_t)b * a.T + t0 + i) * a.H + hq) * K + f]) * a.scale : 0.f;
+  }
+  __syncthreads();
+}
+
+template <int K, int C, typename TIn, bool ERASE>
+__global__ void __launch_bounds__(NTHREADS) kda_fwd_chunkprep_kernel(FwdArgs a, float* __restrict__ prep) {
+  using S = PrepSmem<K, C, ERASE>;
+  constexpr bool PRECISE = sizeof(TIn) == 4;
+  constexpr int LDK = S::LDK, LDC = S::LDC;
+  extern __shared__ float smem[];
+  float *sK = smem + S::oK, *sQ = smem + S::oQ, *sC = smem + S::oC, *sE1 = smem + S::oE1,
+        *sE2o = smem + S::oE2o, *sE2d = smem + S::oE2d, *sAh = smem + S::oAh, *sT = smem + S::oT,
+        *sP = smem + S::oP, *sW = smem + S::oW, *sBeta = smem + S::oBeta, *sR = ERASE ? smem + S::oR : nullptr;
+  int* sFlag = reinterpret_cast<int*>(smem + S::oFlag);
+  const int ch = blockIdx.x, hv = blockIdx.y, b = blockIdx.z;
+  const int T = a.T, NT = (T + C - 1) / C, t0 = ch * C, L = min(C, T - t0);
+  const int QG = ERASE ? a.H / a.HV : 1;
+  float* rec = prep + (((size_t)b * a.HV + hv) * NT + ch) * fma_rec_floats(K, C, QG);
+  float *gTb = rec, *gRt = gTb + C * C, *gKEd = gRt + C * K, *gEl = gKEd + C * K, *gQ0 = gEl + K;
+
+  if constexpr (ERASE)
+    load_chunk_erase<K, C, TIn>(a, b, t0, L, hv * QG, hv, sQ, sK, sR, sC, sBeta);
+  else
+    load_chunk_qkgb<K, C, TIn>(static_cast<const TIn*>(a.q), static_cast<const TIn*>(a.k), a.g, a.beta, a.scale,
+                               b, t0, L, T, a.H, a.HV, hv / (a.HV / a.H), hv, sQ, sK, sC, sBeta);
+  for (int qi = 0; qi < QG; ++qi) {
+    if (qi > 0) load_chunk_q<K, C, TIn>(a, b, t0, L, hv * QG + qi, sQ);
+    // Ah (erase or key rows against keys) and P (queries against keys); the
+    // inverse below needs the first Ah only (later query heads overwrite it)
+    build_interaction<K, C, PRECISE>(sK, sQ, sC, sE1, sE2o, sE2d, sFlag, sAh, sP, sR);
+    float* gP = gQ0 + (size_t)qi * (C * C + C * K);
+    float* gQE = gP + C * C;
+    for (int idx = threadIdx.x; idx < C * C; idx += NTHREADS) gP[idx] = sP[(idx / C) * LDC + idx % C];
+    for (int idx = threadIdx.x; idx < C * K; idx += NTHREADS) {
+      const int i = idx / K, f = idx % K;
+      gQE[idx] = sQ[i * LDK + f] * kexp<PRECISE>(sC[i * LDK + f]);
+    }
+    if (qi == 0) invert_unit_lower<C>(sAh, sBeta, sT, sW);
+    __syncthreads();
+  }
+  // decayed operands: KEd (global), R o e^c (in place), e^{c_last}; Tb = T diag(beta)
+  float* sRe = ERASE ? sR : sK;
+  for (int idx = threadIdx.x; idx < C * K; idx += NTHREADS) {
+    const int i = idx / K, f = idx % K;
+    const float c = sC[i * LDK + f], cl = sC[(C - 1) * LDK + f];
+    gKEd[idx] = sK[i * LDK + f] * kexp<PRECISE>(cl - c);
+    if constexpr (ERASE) sRe[i * LDK + f] *= kexp<PRECISE>(c);
+  }
+  __syncthreads();
+  if constexpr (!ERASE) {  // (k's rows are read above before they are scaled)
+    for (int idx = threadIdx.x; idx < C * K; idx += NTHREADS) {
+      const int i = idx / K, f = idx % K;
+      sRe[i * LDK + f] *= kexp<PRECISE>(sC[i * LDK + f]);
+    }
+  }
+  for (int f = threadIdx.x; f < K; f += NTHREADS) gEl[f] = kexp<PRECISE>(sC[(C - 1) * LDK + f]);
+  for (int idx = threadIdx.x; idx < C * C; idx += NTHREADS) {
+    const int i = idx / C, j = idx % C;
+    const float v = sT[i * LDC + j] * sBeta[j];
+    sT[i * LDC + j] = v;
+    gTb[idx] = v;
+  }
+  __syncthreads();
+  {  // Rt = Tb (R o e^c)
+    constexpr int TMC = C / 16, TNK = K / 16;
+    float acc[TMC][TNK];
+    zero(acc);
+    mm(acc, C, [&](int i, int j) { return sT[i * LDC + j]; }, [&](int j, int f) { return sRe[j * LDK + f]; });
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+#pragma unroll
+    for (int x = 0; x < TMC; ++x)
+#pragma unroll
+      for (int y = 0; y < TNK; ++y) gRt[(ty + 16 * x) * K + tx + 16 * y] = acc[x][y];
+  }
+}
+
+// The state pass: one CTA per (b, state head, V slice of VB columns) carries
+// the K x VB state through the chunks; each chunk's operands (FmaRec) and V
+// rows come in by 16-byte cp.async, one chunk ahead when two buffers fit.
+template <int K, int C, int VB, typename TIn>
+struct StateSmem {
+  static constexpr int LDV = VB + 1;
+  static constexpr int oM = 0, oU = oM + K * LDV, oBuf = oU + C * LDV;
+  // a buffer: the chunk's record, then its V rows (TIn, C x VB)
+  static constexpr int vfloats(int) { return (C * VB * (int)sizeof(TIn) + 15) / 16 * 4; }
+  static int buf_floats(int QG) { return fma_rec_floats(K, C, QG) + vfloats(0); }
+  static size_t bytes(int QG, int nbuf) { return (size_t)(oBuf + nbuf * buf_floats(QG)) * sizeof(float); }
+};
+
+template <int K, int C, int VB, typename TIn, bool ERASE>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    kda_fwd_statepass_kernel(FwdArgs a, const float* __restrict__ prep, int nbuf) {
+  using S = StateSmem<K, C, VB, TIn>;
+  constexpr int LDV = S::LDV, TMC = C / 16, TNV = VB / 16, TMK = K / 16;
+  extern __shared__ __align__(16) float smem[];
+  float *sM = smem + S::oM, *sU = smem + S::oU;
+  const int QG = ERASE ? a.H / a.HV : 1, REC = fma_rec_floats(K, C, QG), BUF = REC + S::vfloats(0);
+  const int v0 = blockIdx.x * VB, hv = blockIdx.y, b = blockIdx.z;
+  const int T = a.T, V = a.V, NT = (T + C - 1) / C;
+  const size_t head = (size_t)b * a.HV + hv;
+  const int HO = ERASE ? a.H : a.HV;
+  const TIn* __restrict__ v = static_cast<const TIn*>(a.v);
+  TIn* __restrict__ o = static_cast<TIn*>(a.o);
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const float* recs = prep + head * NT * (size_t)REC;
+
+  const auto issue = [&](int ch, float* buf) {  // the chunk's record and V rows into buf
+    const float* src = recs + (size_t)ch * REC;
+    const uint32_t sb = (uint32_t)__cvta_generic_to_shared(buf);
+    for (int x = threadIdx.x; x < REC / 4; x += NTHREADS) tc::cp_async16(sb + x * 16, src + x * 4, true);
+    constexpr int PR = VB * (int)sizeof(TIn) / 16;  // 16-byte pieces per V row
+    const int t0 = ch * C, L = min(C, T - t0);
+    const uint32_t vb = sb + REC * 4;
+    for (int x = threadIdx.x; x < C * PR; x += NTHREADS) {
+      const int i = x / PR, pc = x % PR;
+      const bool ok = i < L;
+      const TIn* row = v + (((size_t)b * T + t0 + (ok ? i : 0)) * a.HV + hv) * V + v0;
+      tc::cp_async16(vb + x * 16, reinterpret_cast<const unsigned char*>(row) + pc * 16, ok);
+    }
+    tc::cp_async_commit();
+  };
+
+  for (int idx = threadIdx.x; idx < K * VB; idx += NTHREADS) {
+    const int f = idx / VB, n = idx % VB;
+    sM[f * LDV + n] = a.S0 ? a.S0[(head * K + f) * V + v0 + n] : 0.f;
+  }
+  float* buf0 = smem + S::oBuf;
+  issue(0, buf0);
+  for (int ch = 0; ch < NT; ++ch) {
+    const int t0 = ch * C, L = min(C, T - t0);
+    float* cur = buf0 + (nbuf == 2 ? (ch & 1) * BUF : 0);
+    if (nbuf == 2 && ch + 1 < NT) {  // (the other buffer's last readers passed the previous chunk's end barrier)
+      issue(ch + 1, buf0 + ((ch + 1) & 1) * BUF);
+      tc::cp_async_wait_group<1>();
+    } else {
+      tc::cp_async_wait_group<0>();
+    }
+    __syncthreads();
+    const float *cTb = cur, *cRt = cTb + C * C, *cKEd = cRt + C * K, *cEl = cKEd + C * K, *cQ0 = cEl + K;
+    const TIn* cV = reinterpret_cast<const TIn*>(cur + REC);
+    if (a.states) {
+      float* dst = a.states + ((head * NT + ch) * K) * V;
+      for (int idx = threadIdx.x; idx < K * VB; idx += NTHREADS) {
+        const int f = idx / VB, n = idx % VB;
+        dst[(size_t)f * V + v0 + n] = sM[f * LDV + n];
+      }
+    }
+    {  // U = Tb V - Rt M
+      float acc[TMC][TNV], neg[TMC][TNV];
+      zero(acc);
+      zero(neg);
+      mm(acc, C, [&](int i, int j) { return cTb[i * C + j]; }, [&](int j, int n) { return to_f(cV[j * VB + n]); });
+      mm(neg, K, [&](int i, int f) { return cRt[i * K + f]; }, [&](int f, int n) { return sM[f * LDV + n]; });
+#pragma unroll
+      for (int x = 0; x < TMC; ++x)
+#pragma unroll
+        for (int y = 0; y < TNV; ++y) sU[(ty + 16 * x) * LDV + tx + 16 * y] = acc[x][y] - neg[x][y];
+    }
+    __syncthreads();
+    if (a.o) {
+      for (int qi = 0; qi < QG; ++qi) {  // O = (Q~ o e^c) M + P U for each query head of this state head
+        const float* cP = cQ0 + (size_t)qi * (C * C + C * K);
+        const float* cQE = cP + C * C;
+        float acc[TMC][TNV];
+        zero(acc);
+        mm(acc, K, [&](int i, int f) { return cQE[i * K + f]; }, [&](int f, int n) { return sM[f * LDV + n]; });
+        mm(acc, C, [&](int i, int j) { return cP[i * C + j]; }, [&](int j, int n) { return sU[j * LDV + n]; });
+        const int ho = ERASE ? hv * QG + qi : hv;
+#pragma unroll
+        for (int x = 0; x < TMC; ++x)
+#pragma unroll
+          for (int y = 0; y < TNV; ++y) {
+            const int i = ty + 16 * x, n = tx + 16 * y;
+            if (i < L) o[(((size_t)b * T + t0 + i) * HO + ho) * V + v0 + n] = from_f<TIn>(acc[x][y]);
+          }
+      }
+    }
+    {  // M' = diag(El) M + KEd^T U
+      float acc[TMK][TNV];
+#pragma unroll
+      for (int x = 0; x < TMK; ++x)
+#pragma unroll
+        for (int y = 0; y < TNV; ++y) {
+          const int f = ty + 16 * x, n = tx + 16 * y;
+          acc[x][y] = cEl[f] * sM[f * LDV + n];
+        }
+      mm(acc, C, [&](int f, int i) { return cKEd[i * K + f]; }, [&](int i, int n) { return sU[i * LDV + n]; });
+      __syncthreads();
+#pragma unroll
+      for (int x = 0; x < TMK; ++x)
+#pragma unroll
+        for (int y = 0; y < TNV; ++y) sM[(ty + 16 * x) * LDV + tx + 16 * y] = acc[x][y];
+    }
+    if (nbuf == 1 && ch + 1 < NT) {
+      __syncthreads();  // every read of this chunk's buffer is done
+      issue(ch + 1, buf0);
+    }
+    __syncthreads();
+  }
+  if (a.S_T) {
+    for (int idx = threadIdx.x; idx < K * VB; idx += NTHREADS) {
+      const int f = idx / VB, n = idx % VB;
+      a.S_T[(head * K + f) * V + v0 + n] = sM[f * LDV + n];
+    }
+  }
+}
+
+size_t fma_prep_bytes(int B, int T, int HV, int K, int QG) {
+  const size_t NT = (size_t)(T + FWD_CHUNK - 1) / FWD_CHUNK;
+  return (size_t)B * HV * NT * fma_rec_floats(K, FWD_CHUNK, QG) * sizeof(float);
+}
+
+// Whether the two-kernel CUDA-core forward takes this call: plain inputs (no
+// fused preparation or output gate), 16-byte aligned v (its rows come in by
+// 16-byte copies) and workspace.
+bool fwd_fma2_eligible(const FwdArgs& a, const void* workspace) {
+  auto al16 = [](const void* p) { return ((uintptr_t)p & 15u) == 0; };
+  return !a.ctab && !a.prep.z && !a.og && workspace && al16(workspace) && al16(a.v) && a.V % FWD_VBLOCK == 0;
+}
+
+template <int K, typename TIn, bool ERASE>
+static int launch_fwd_fma2_t(const FwdArgs& a, float* prep, cudaStream_t stream) {
+  constexpr int C = FWD_CHUNK, VB = FWD_VBLOCK;
+  const char* who = ERASE ? "kda_fwd_erase" : "kda_fwd";
+  const int NT = (a.T + C - 1) / C, QG = ERASE ? a.H / a.HV : 1;
+  auto k1 = kda_fwd_chunkprep_kernel<K, C, TIn, ERASE>;
+  cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)PrepSmem<K, C, ERASE>::bytes);
+  if (e != cudaSuccess) return set_cuda_error(who, e);
+  k1<<<dim3(NT, a.HV, a.B), NTHREADS, PrepSmem<K, C, ERASE>::bytes, stream>>>(a, prep);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return set_cuda_error(who, e);
+  using SS = StateSmem<K, C, VB, TIn>;
+  const int nbuf = SS::bytes(QG, 2) <= 200 * 1024 ? 2 : 1;
+  if (SS::bytes(QG, nbuf) > 227 * 1024) return set_error(4, "two-kernel CUDA-core forward: too many query heads per state head");
+  auto k2 = kda_fwd_statepass_kernel<K, C, VB, TIn, ERASE>;
+  e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SS::bytes(QG, nbuf));
+  if (e != cudaSuccess) return set_cuda_error(who, e);
+  k2<<<dim3(a.V / VB, a.HV, a.B), NTHREADS, SS::bytes(QG, nbuf), stream>>>(a, prep, nbuf);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return set_cuda_error(who, e);
+  return 0;
+}
+
+int launch_fwd_fma2(const FwdArgs& a, int dtype, bool erase, float* prep, cudaStream_t stream) {
+  const bool bf = dtype == 1;
+#define KDA_FMA2(KK)                                                                                     \
+  case KK:                                                                                               \
+    if (erase)                                                                                           \
+      return bf ? launch_fwd_fma2_t<KK, __nv_bfloat16, true>(a, prep, stream)                           \
+                : launch_fwd_fma2_t<KK, float, true>(a, prep, stream);                                   \
+    return bf ? launch_fwd_fma2_t<KK, __nv_bfloat16, false>(a, prep, stream)                            \
+              : launch_fwd_fma2_t<KK, float, false>(a, prep, stream);
+  switch (a.K) {
+    KDA_FMA2(32)
+    KDA_FMA2(64)
+    KDA_FMA2(128)
+  }
+#undef KDA_FMA2
+  return set_error(4, "kda_fwd: unsupported K");
 }
 
 template <int K, typename TIn>

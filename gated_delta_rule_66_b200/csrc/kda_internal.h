@@ -188,6 +188,11 @@ int launch_fwd(const FwdArgs& a, int dtype, cudaStream_t stream);
 int launch_fwd_ffma(const FwdArgs& a, int dtype, cudaStream_t stream);
 bool fwd_tc_eligible(const FwdArgs& a, int dtype);
 int launch_fwd_erase(const FwdArgs& a, int dtype, cudaStream_t stream);
+// two-kernel CUDA-core forward (chunk preparation into `prep`, then the state
+// pass); erase: the asymmetric erase/write variant
+bool fwd_fma2_eligible(const FwdArgs& a, const void* workspace);
+size_t fma_prep_bytes(int B, int T, int HV, int K, int QG);
+int launch_fwd_fma2(const FwdArgs& a, int dtype, bool erase, float* prep, cudaStream_t stream);
 int launch_fwd_tc(const FwdArgs& a, cudaStream_t stream);
 int take_device_error(unsigned* out);
 int take_bwd_device_error(unsigned* out);

@@ -26,7 +26,7 @@ SYMBOLS = ("kda_last_error", "kda_device_status", "kda_fwd_workspace_bytes", "kd
            "kda_bwd_workspace_bytes", "kda_fwd", "kda_fwd_varlen_workspace_bytes", "kda_fwd_varlen",
            "kda_bwd_varlen_workspace_bytes", "kda_bwd_varlen", "kda_decode_step", "kda_bwd",
            "kda_fwd_prep_workspace_bytes", "kda_fwd_prep", "kda_short_conv", "kda_decode_token",
-           "kda_fwd_erase")
+           "kda_fwd_erase", "kda_fwd_erase_workspace_bytes")
 
 
 class KdaError(RuntimeError):
@@ -82,7 +82,9 @@ def _load():
     lib.kda_decode_token.argtypes = [vp, vp, vp, vp, vp, vp, i, vp, vp, vp, f, vp, vp, f, vp, f, i, i, i, i, i, i,
                                      vp, vp]
     lib.kda_fwd_erase.restype = i
-    lib.kda_fwd_erase.argtypes = [vp, vp, vp, vp, vp, vp, f, i, i, i, i, i, i, i, vp, vp, vp]
+    lib.kda_fwd_erase.argtypes = [vp, vp, vp, vp, vp, vp, f, i, i, i, i, i, i, i, vp, vp, vp, sz, vp]
+    lib.kda_fwd_erase_workspace_bytes.restype = sz
+    lib.kda_fwd_erase_workspace_bytes.argtypes = [i, i, i, i, i, i]
     return lib
 
 
@@ -171,7 +173,7 @@ def fwd(q, k, v, g, beta, scale=None, initial_state=None, output_final_state=Tru
     o = torch.empty(B, T, HV, V, dtype=dt, device=q.device) if out is None else out
     _req("out", o, dt, 4)
     S_T = torch.empty(B, HV, K, V, dtype=torch.float32, device=q.device) if output_final_state else None
-    if workspace is None and scratch and dt == torch.bfloat16:
+    if workspace is None and scratch:
         need = int(_lib.kda_fwd_scratch_bytes(B, T, HV, K, V))
         if need:
             workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
@@ -431,12 +433,15 @@ def decode_token(xq, xk, xv, conv_w, conv_state, z, A_log, dt_bias, beta_logit, 
 
 
 # ----------------------------------------------------------------------------- erase/write variant
-def fwd_erase(q, k, e, z, g, scale=None, initial_state=None, output_final_state=True):
+def fwd_erase(q, k, e, z, g, scale=None, initial_state=None, output_final_state=True, scratch=True):
     """Prefill of the asymmetric erase/write delta recurrence.
 
     q [B,T,HQ,K]; k (write), e (erase) [B,T,HV,K]; z [B,T,HV,V] (one dtype);
     g [B,T,HV,K] float32; HQ a multiple of HV (query head hq reads state head
     hq // (HQ // HV)).  Returns (o [B,T,HQ,V], S_T [B,HV,K,V] or None).
+    ``scratch`` gives the library a fresh workspace of
+    kda_fwd_erase_workspace_bytes (the two-kernel path); ``scratch=False``
+    runs the single-kernel path.
     """
     B, T, HQ, K = q.shape
     HV, V = k.shape[2], z.shape[3]
@@ -448,7 +453,13 @@ def fwd_erase(q, k, e, z, g, scale=None, initial_state=None, output_final_state=
     _req("initial_state", initial_state, torch.float32, 4)
     o = torch.empty(B, T, HQ, V, dtype=dt, device=q.device)
     S_T = torch.empty(B, HV, K, V, dtype=torch.float32, device=q.device) if output_final_state else None
+    ws = None
+    if scratch:
+        need = int(_lib.kda_fwd_erase_workspace_bytes(B, T, HQ, HV, K, V))
+        if need:
+            ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if ws is None else ws.numel()
     rc = _lib.kda_fwd_erase(_ptr(q), _ptr(k), _ptr(e), _ptr(z), _ptr(g), _ptr(initial_state), scale, B, T, HQ, HV,
-                            K, V, _dtype_code(q), _ptr(o), _ptr(S_T), _stream())
+                            K, V, _dtype_code(q), _ptr(o), _ptr(S_T), _ptr(ws), ws_bytes, _stream())
     _check("kda_fwd_erase", rc)
     return o, S_T

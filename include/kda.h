@@ -84,11 +84,13 @@ int kda_device_status(unsigned* flags);
  * and the scratch of kda_fwd_scratch_bytes(); 0 if a size is invalid. */
 size_t kda_fwd_workspace_bytes(int B, int T, int HV, int K, int V);
 
-/* Bytes of the optional scratch that lets kda_fwd without stored states run
- * as two kernels (K = V = 128, bf16): a chunk-parallel pass that leaves every
- * 64-step chunk's operands of the state products there (165 KB per chunk),
- * then the sequential state pass.  0 if the shape has no such path or a size
- * is invalid. */
+/* Bytes of the optional scratch that lets kda_fwd run as two kernels: a
+ * chunk-parallel pass that leaves every chunk's operands of the state
+ * products there, then the sequential state pass.  On the tensor-core path
+ * (K = V = 128, bf16) the chunk images take 152,064 bytes per 64-step chunk;
+ * on the CUDA-core path (fp32 inputs, or other K and V) the chunk records take
+ * 4 (2 C^2 + 3 C K + K) bytes per 32-step chunk (C = 32); the larger of the
+ * two, as the dtype is not an argument.  0 if a size is invalid. */
 size_t kda_fwd_scratch_bytes(int B, int T, int HV, int K, int V);
 
 /* Bytes kda_bwd needs: the chunk states and interaction records (as
@@ -111,7 +113,11 @@ size_t kda_bwd_workspace_bytes(int B, int T, int H, int HV, int K, int V);
  *     kda_fwd_workspace_bytes(B, T, HV, K, V) bytes: the states and records
  *     for a later kda_bwd with KDA_BWD_STATES_FROM_FWD are stored there; or
  *     at least kda_fwd_scratch_bytes() (but fewer than the former): used as
- *     scratch only.  A workspace of neither size is KDA_ERR_WORKSPACE.
+ *     scratch only.  A workspace of neither size is KDA_ERR_WORKSPACE.  With
+ *     either, the forward runs as two kernels (chunk-parallel pass, then the
+ *     state pass: tensor-core shapes; CUDA-core shapes when v is 16-byte
+ *     aligned); without one, one kernel carries each state slice through
+ *     its chunks.
  * o and S_T must not alias any input.  S_T may alias S0 only if S0 is not
  * needed afterwards (S0 is read before S_T is written, per value column). */
 int kda_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
@@ -262,11 +268,23 @@ int kda_decode_token(const void* xq, const void* xk, const void* xv, const float
  *   q [B, T, HQ, K] dtype; k, e [B, T, HV, K] dtype; z [B, T, HV, V] dtype;
  *   g [B, T, HV, K] float; S0 [B, HV, K, V] float or NULL
  *   o [B, T, HQ, V] dtype (output); S_T [B, HV, K, V] float or NULL
- * HQ must be a multiple of HV.  Runs on the CUDA-core chunk kernels (one CTA
- * per query head and 32 value columns, each carrying its state head). */
+ * HQ must be a multiple of HV.  Runs on the CUDA-core chunk kernels; see
+ * kda_fwd_erase_workspace_bytes for the workspace. */
 int kda_fwd_erase(const void* q, const void* k, const void* e, const void* z, const float* g, const float* S0,
                   float scale, int B, int T, int HQ, int HV, int K, int V, int dtype, void* o, float* S_T,
-                  void* stream);
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of the optional workspace of kda_fwd_erase (16-byte aligned, with a
+ * 16-byte aligned z): with it the variant runs as two kernels, a
+ * chunk-parallel pass that leaves every 32-step chunk's operands there
+ * (4 (2 C^2 + 3 C K + K + (HQ / HV - 1)(C^2 + C K)) bytes per chunk and state
+ * head, C = 32: the inverse times diag(beta), the residual and carry
+ * operands, and P and the decayed queries of every query head), then a state
+ * pass per state head and 32 value columns that reads the state out for all
+ * its query heads.  Without a workspace (NULL) one kernel per query head
+ * carries a copy of its state head.  A non-NULL workspace smaller than this
+ * is KDA_ERR_WORKSPACE.  0 if a size is invalid. */
+size_t kda_fwd_erase_workspace_bytes(int B, int T, int HQ, int HV, int K, int V);
 
 /* Size in bytes of the fixed device array that kda_bwd_noalloc uses as its
  * scratch (64 MiB, held on every GPU that loads the library until exit). */

@@ -40,13 +40,26 @@ def test_library_exports_every_declared_symbol(lib):
         assert hasattr(lib, n), n
 
 
+def fma_rec_bytes(K, QG=1, C=32):
+    """One 32-step chunk record of the two-kernel CUDA-core forward: T diag(beta)
+    and P (C x C per query head), the residual and carry operands and Q~ o e^c
+    (C x K, the last per query head), e^{c_last} (K); fp32."""
+    return 4 * (C * C + 2 * C * K + K + QG * (C * C + C * K))
+
+
 def test_workspace_sizes(lib):
+    """CUDA-core shapes: the training forward keeps the 32-step states and the
+    scratch of the two-kernel forward (its chunk records); the backward
+    overwrites the records with the state gradients (and dq/dk partials)."""
     B, T, H, HV, K, V = 2, 100, 2, 6, 64, 32
     NT = (T + 31) // 32
     states = B * HV * NT * K * V * 4
-    assert lib.kda_fwd_workspace_bytes(B, T, HV, K, V) == states
-    assert lib.kda_bwd_workspace_bytes(B, T, H, HV, K, V) == 2 * states + 2 * B * T * HV * K * 4
-    assert lib.kda_bwd_workspace_bytes(B, T, HV, HV, K, V) == 2 * states
+    prep = B * HV * NT * fma_rec_bytes(K)
+    assert lib.kda_fwd_scratch_bytes(B, T, HV, K, V) == prep
+    assert lib.kda_fwd_workspace_bytes(B, T, HV, K, V) == states + prep
+    assert lib.kda_bwd_workspace_bytes(B, T, H, HV, K, V) == states + max(states + 2 * B * T * HV * K * 4, prep)
+    assert lib.kda_bwd_workspace_bytes(B, T, HV, HV, K, V) == states + max(states, prep)
+    assert lib.kda_bwd_workspace_bytes(B, T, H, HV, K, V) >= lib.kda_fwd_workspace_bytes(B, T, HV, K, V)
     assert lib.kda_fwd_workspace_bytes(0, T, HV, K, V) == 0
     assert lib.kda_bwd_workspace_bytes(B, T, 4, HV, K, V) == 0   # HV % H != 0
 
@@ -121,13 +134,15 @@ def test_tensor_core_workspace_sizes(lib):
     nt32, nt64 = (T + 31) // 32, (T + 63) // 64
     states = B * HV * nt32 * K * V * 4
     inter = B * HV * nt64 * 16384 * 4
-    img = B * HV * nt64 * 152064
+    img = B * HV * nt64 * 152064  # (larger than the CUDA-core records of the same shape)
+    assert img >= B * HV * nt32 * fma_rec_bytes(K)
     assert lib.kda_fwd_scratch_bytes(B, T, HV, K, V) == img
     assert lib.kda_fwd_workspace_bytes(B, T, HV, K, V) == states + inter + img
     tail = states + 2 * B * T * HV * K * 4 + B * HV * nt64 * 37120 * 4  # state grads, dq/dk partials, records
     assert lib.kda_bwd_workspace_bytes(B, T, H, HV, K, V) == states + inter + max(tail, img)
     assert lib.kda_bwd_workspace_bytes(B, T, H, HV, K, V) >= lib.kda_fwd_workspace_bytes(B, T, HV, K, V)
-    assert lib.kda_fwd_scratch_bytes(B, T, HV, 64, 64) == 0
+    assert lib.kda_fwd_scratch_bytes(B, T, HV, 64, 64) == B * HV * nt32 * fma_rec_bytes(64)  # CUDA-core records
+    assert lib.kda_fwd_scratch_bytes(B, T, HV, 48, 64) == 0  # unsupported K
 
 
 def _cu(vals):
@@ -210,10 +225,15 @@ def test_erase_validation(lib):
                  dtype=1, o=FAKE, S_T=None)
         a.update(over)
         return lib.kda_fwd_erase(a["q"], a["k"], a["e"], a["z"], a["g"], a["S0"], a["scale"], a["B"], a["T"],
-                                 a["HQ"], a["HV"], a["K"], a["V"], a["dtype"], a["o"], a["S_T"], None)
+                                 a["HQ"], a["HV"], a["K"], a["V"], a["dtype"], a["o"], a["S_T"],
+                                 a.get("ws"), a.get("ws_bytes", 0), None)
 
     assert call(HQ=3) == 2 and "multiple of HV" in lib.kda_last_error().decode()
     assert call(e=None) == 1
     assert call(K=48) == 4
     assert call(scale=-1.0) == 7
     assert call(T=0) == 2
+    # the two-kernel path's workspace: one record per 32-step chunk and state head
+    assert lib.kda_fwd_erase_workspace_bytes(1, 8, 4, 2, 64, 128) == 1 * 2 * 1 * fma_rec_bytes(64, QG=2)
+    assert lib.kda_fwd_erase_workspace_bytes(1, 8, 3, 2, 64, 128) == 0  # HQ % HV != 0
+    assert call(ws=FAKE, ws_bytes=16) == 5 and "workspace" in lib.kda_last_error().decode()

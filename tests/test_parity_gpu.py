@@ -89,6 +89,16 @@ def test_fwd_shapes(kda, name, base, over):
 
 
 TC_CASES = [c for c in FWD_CASES if c[0].startswith("tc_")]
+FMA_CASES = [c for c in FWD_CASES if not c[0].startswith("tc_")]
+
+
+@pytest.mark.parametrize("name,base,over", FMA_CASES, ids=[c[0] for c in FMA_CASES])
+def test_fwd_single_kernel(kda, name, base, over):
+    """Without a workspace the CUDA-core shapes run one kernel per state slice
+    (the default is the two-kernel path: chunk preparation, then the state
+    pass); the same shapes against the oracle."""
+    w = BY_NAME[base].with_sizes(**over)
+    check_fwd(kda, make_inputs(w), w.scale, w.torch_dtype, name + "_single", scratch=False)
 
 
 @pytest.mark.parametrize("name,base,over", TC_CASES, ids=[c[0] for c in TC_CASES])
@@ -272,6 +282,17 @@ def test_bwd_reuses_forward_states(kda):
     b = run_bwd(kda, inp, w.scale, reuse=True)
     for x, y in zip(a, b):
         assert torch.equal(x, y)
+
+
+def test_bwd_reuses_two_kernel_cuda_core_states(kda):
+    """CUDA-core shapes: the training forward runs as two kernels and stores
+    every 32-step state; the backward that reuses them meets the fp32 bar
+    (its own forward recomputation takes the single-kernel path)."""
+    w = BY_NAME["twin"].with_sizes(B=1, T=100, H=2, HV=4, K=64, V=32)
+    inp = make_inputs(w, with_do=True)
+    grads = run_bwd(kda, inp, w.scale, reuse=True)
+    for n, x, r in zip(GRAD_NAMES, grads, oracle_bwd(inp, w.scale)):
+        report(f"fma_reuse {n}", f64(x), r, tol_for(w.torch_dtype), torch.float32)
 
 
 def test_fwdbwd_full_size(kda):

@@ -231,19 +231,24 @@ def _erase_oracle(r, scale):
                                 f64(r["S0"]))
 
 
+@pytest.mark.parametrize("scratch", [True, False], ids=["two_kernel", "single_kernel"])
 @pytest.mark.parametrize("name,over", ERASE_CASES, ids=[c[0] for c in ERASE_CASES])
-def test_fwd_erase(kda, name, over):
+def test_fwd_erase(kda, name, over, scratch):
     """The asymmetric erase/write recurrence (separate erase and write
-    vectors, query heads grouped over state heads) against the token loop."""
+    vectors, query heads grouped over state heads) against the token loop, on
+    the two-kernel path (chunk preparation, then one state pass per state
+    head for all its query heads) and on the single-kernel path."""
     w = BY_NAME["erase"].with_sizes(**over)
     r = make_erase_inputs(w)
     d = {n: (None if t is None else t.cuda()) for n, t in r.items()}
-    o, S = kda.fwd_erase(d["q"], d["k"], d["e"], d["z"], d["g"], scale=w.scale, initial_state=d["S0"])
+    o, S = kda.fwd_erase(d["q"], d["k"], d["e"], d["z"], d["g"], scale=w.scale, initial_state=d["S0"],
+                         scratch=scratch)
     torch.cuda.synchronize()
     o_ref, S_ref = _erase_oracle(r, w.scale)
     tol = tol_for(w.torch_dtype)
-    report(f"erase_{name} o", f64(o), o_ref, tol, w.torch_dtype)
-    report(f"erase_{name} S_T", f64(S), S_ref, tol, torch.float32)
+    tag = f"erase_{name}" + ("" if scratch else "_single")
+    report(f"{tag} o", f64(o), o_ref, tol, w.torch_dtype)
+    report(f"{tag} S_T", f64(S), S_ref, tol, torch.float32)
 
 
 def test_fwd_erase_kda_special_case(kda):
