@@ -339,7 +339,7 @@ int kda_decode_step(const void* q, const void* k, const void* v, const float* g,
 
 size_t kda_fwd_erase_workspace_bytes(int B, int T, int HQ, int HV, int K, int V) {
   if (B < 1 || T < 1 || HQ < 1 || HV < 1 || HQ % HV || V < 1 || (K != 32 && K != 64 && K != 128)) return 0;
-  return fma_prep_bytes(B, T, HV, K, HQ / HV);
+  return fma_erase_bytes(B, T, HQ, HV, K, V);
 }
 
 int kda_fwd_erase(const void* q, const void* k, const void* e, const void* z, const float* g, const float* S0,

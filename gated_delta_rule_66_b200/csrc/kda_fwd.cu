@@ -341,9 +341,13 @@ struct StateSmem {
   static size_t bytes(int QG, int nbuf) { return (size_t)(oBuf + nbuf * buf_floats(QG)) * sizeof(float); }
 };
 
+// (ERASE: the read-out of the query heads is left to kda_fwd_readout_kernel;
+// the pass stores the state entering every chunk into mst [B, HV, NT, K, V]
+// and U into ust [B, HV, NT, C, V] instead.)
 template <int K, int C, int VB, typename TIn, bool ERASE>
 __global__ void __launch_bounds__(NTHREADS, 1)
-    kda_fwd_statepass_kernel(FwdArgs a, const float* __restrict__ prep, int nbuf) {
+    kda_fwd_statepass_kernel(FwdArgs a, const float* __restrict__ prep, int nbuf, float* __restrict__ mst,
+                             float* __restrict__ ust) {
   using S = StateSmem<K, C, VB, TIn>;
   constexpr int LDV = S::LDV, TMC = C / 16, TNV = VB / 16, TMK = K / 16;
   extern __shared__ __align__(16) float smem[];
@@ -392,8 +396,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     __syncthreads();
     const float *cTb = cur, *cRt = cTb + C * C, *cKEd = cRt + C * K, *cEl = cKEd + C * K, *cQ0 = cEl + K;
     const TIn* cV = reinterpret_cast<const TIn*>(cur + REC);
-    if (a.states) {
-      float* dst = a.states + ((head * NT + ch) * K) * V;
+    float* const mdst = ERASE ? mst : a.states;
+    if (mdst) {
+      float* dst = mdst + ((head * NT + ch) * K) * V;
       for (int idx = threadIdx.x; idx < K * VB; idx += NTHREADS) {
         const int f = idx / VB, n = idx % VB;
         dst[(size_t)f * V + v0 + n] = sM[f * LDV + n];
@@ -408,10 +413,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
       for (int x = 0; x < TMC; ++x)
 #pragma unroll
-        for (int y = 0; y < TNV; ++y) sU[(ty + 16 * x) * LDV + tx + 16 * y] = acc[x][y] - neg[x][y];
+        for (int y = 0; y < TNV; ++y) {
+          const float u = acc[x][y] - neg[x][y];
+          sU[(ty + 16 * x) * LDV + tx + 16 * y] = u;
+          if constexpr (ERASE) ust[((head * NT + ch) * C + ty + 16 * x) * V + v0 + tx + 16 * y] = u;
+        }
     }
     __syncthreads();
-    if (a.o) {
+    if (!ERASE && a.o) {
       for (int qi = 0; qi < QG; ++qi) {  // O = (Q~ o e^c) M + P U for each query head of this state head
         const float* cP = cQ0 + (size_t)qi * (C * C + C * K);
         const float* cQE = cP + C * C;
@@ -459,9 +468,63 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
 }
 
+// Read-out of the erase/write variant, one CTA per (b, query head, chunk):
+// O = (Q~ o e^c) M + P U over all V columns, from the chunk record and the
+// state and U the state pass stored.
+template <int K, int C, int V, typename TIn>
+__global__ void __launch_bounds__(NTHREADS) kda_fwd_readout_kernel(FwdArgs a, const float* __restrict__ prep,
+                                                                    const float* __restrict__ mst,
+                                                                    const float* __restrict__ ust) {
+  constexpr int TMC = C / 16, TNV = V / 16, LDV = V + 4;
+  extern __shared__ __align__(16) float smem[];
+  float *sQE = smem, *sP = sQE + C * K, *sM = sP + C * C, *sU = sM + K * LDV;
+  const int ch = blockIdx.x, hq = blockIdx.y, b = blockIdx.z;
+  const int QG = a.H / a.HV, hv = hq / QG, qi = hq % QG;
+  const int T = a.T, NT = (T + C - 1) / C, t0 = ch * C, L = min(C, T - t0);
+  const size_t hc = ((size_t)b * a.HV + hv) * NT + ch;
+  const float* rec = prep + hc * fma_rec_floats(K, C, QG);
+  const float* gP = rec + C * C + 2 * C * K + K + (size_t)qi * (C * C + C * K);
+  const float* gQE = gP + C * C;
+  const uint32_t s0 = (uint32_t)__cvta_generic_to_shared(smem);
+  for (int x = threadIdx.x; x < C * K / 4; x += NTHREADS) tc::cp_async16(s0 + x * 16, gQE + x * 4, true);
+  for (int x = threadIdx.x; x < C * C / 4; x += NTHREADS) tc::cp_async16(s0 + (C * K + x * 4) * 4, gP + x * 4, true);
+  const float* gM = mst + hc * K * V;
+  const float* gU = ust + hc * C * V;
+  for (int x = threadIdx.x; x < K * V / 4; x += NTHREADS) {
+    const int f = x / (V / 4), n4 = (x % (V / 4)) * 4;
+    tc::cp_async16(s0 + (uint32_t)(sM - smem + f * LDV + n4) * 4, gM + f * V + n4, true);
+  }
+  for (int x = threadIdx.x; x < C * V / 4; x += NTHREADS) {
+    const int i = x / (V / 4), n4 = (x % (V / 4)) * 4;
+    tc::cp_async16(s0 + (uint32_t)(sU - smem + i * LDV + n4) * 4, gU + i * V + n4, true);
+  }
+  tc::cp_async_wait_all();
+  __syncthreads();
+  float acc[TMC][TNV];
+  zero(acc);
+  mm(acc, K, [&](int i, int f) { return sQE[i * K + f]; }, [&](int f, int n) { return sM[f * LDV + n]; });
+  mm(acc, C, [&](int i, int j) { return sP[i * C + j]; }, [&](int j, int n) { return sU[j * LDV + n]; });
+  TIn* o = static_cast<TIn*>(a.o);
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+#pragma unroll
+  for (int x = 0; x < TMC; ++x)
+#pragma unroll
+    for (int y = 0; y < TNV; ++y) {
+      const int i = ty + 16 * x, n = tx + 16 * y;
+      if (i < L) o[(((size_t)b * T + t0 + i) * a.H + hq) * V + n] = from_f<TIn>(acc[x][y]);
+    }
+}
+
 size_t fma_prep_bytes(int B, int T, int HV, int K, int QG) {
   const size_t NT = (size_t)(T + FWD_CHUNK - 1) / FWD_CHUNK;
   return (size_t)B * HV * NT * fma_rec_floats(K, FWD_CHUNK, QG) * sizeof(float);
+}
+
+// The erase/write variant's workspace: the chunk records, then the state
+// entering every chunk and U of every chunk for its read-out kernel.
+size_t fma_erase_bytes(int B, int T, int HQ, int HV, int K, int V) {
+  const size_t NT = (size_t)(T + FWD_CHUNK - 1) / FWD_CHUNK;
+  return fma_prep_bytes(B, T, HV, K, HQ / HV) + (size_t)B * HV * NT * ((size_t)K * V + (size_t)FWD_CHUNK * V) * 4;
 }
 
 // Whether the two-kernel CUDA-core forward takes this call: plain inputs (no
@@ -490,9 +553,26 @@ static int launch_fwd_fma2_t(const FwdArgs& a, float* prep, cudaStream_t stream)
   auto k2 = kda_fwd_statepass_kernel<K, C, VB, TIn, ERASE>;
   e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SS::bytes(QG, nbuf));
   if (e != cudaSuccess) return set_cuda_error(who, e);
-  k2<<<dim3(a.V / VB, a.HV, a.B), NTHREADS, SS::bytes(QG, nbuf), stream>>>(a, prep, nbuf);
+  float* mst = nullptr;
+  float* ust = nullptr;
+  if constexpr (ERASE) {
+    mst = prep + fma_prep_bytes(a.B, a.T, a.HV, K, QG) / sizeof(float);
+    ust = mst + (size_t)a.B * a.HV * NT * K * a.V;
+  }
+  k2<<<dim3(a.V / VB, a.HV, a.B), NTHREADS, SS::bytes(QG, nbuf), stream>>>(a, prep, nbuf, mst, ust);
   e = cudaGetLastError();
   if (e != cudaSuccess) return set_cuda_error(who, e);
+  if constexpr (ERASE) {
+    if (!a.o) return 0;
+    const size_t sb = (size_t)(C * K + C * C + (K + C) * (a.V + 4)) * sizeof(float);
+    const auto k3 = a.V == 32 ? kda_fwd_readout_kernel<K, C, 32, TIn>
+                  : a.V == 64 ? kda_fwd_readout_kernel<K, C, 64, TIn> : kda_fwd_readout_kernel<K, C, 128, TIn>;
+    e = cudaFuncSetAttribute(k3, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sb);
+    if (e != cudaSuccess) return set_cuda_error(who, e);
+    k3<<<dim3(NT, a.H, a.B), NTHREADS, sb, stream>>>(a, prep, mst, ust);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return set_cuda_error(who, e);
+  }
   return 0;
 }
 

@@ -275,15 +275,17 @@ int kda_fwd_erase(const void* q, const void* k, const void* e, const void* z, co
                   void* workspace, size_t workspace_bytes, void* stream);
 
 /* Bytes of the optional workspace of kda_fwd_erase (16-byte aligned, with a
- * 16-byte aligned z): with it the variant runs as two kernels, a
+ * 16-byte aligned z): with it the variant runs as three kernels, a
  * chunk-parallel pass that leaves every 32-step chunk's operands there
  * (4 (2 C^2 + 3 C K + K + (HQ / HV - 1)(C^2 + C K)) bytes per chunk and state
  * head, C = 32: the inverse times diag(beta), the residual and carry
- * operands, and P and the decayed queries of every query head), then a state
- * pass per state head and 32 value columns that reads the state out for all
- * its query heads.  Without a workspace (NULL) one kernel per query head
- * carries a copy of its state head.  A non-NULL workspace smaller than this
- * is KDA_ERR_WORKSPACE.  0 if a size is invalid. */
+ * operands, and P and the decayed queries of every query head), a state pass
+ * per state head and 32 value columns that carries the state once and stores
+ * the state entering every chunk and the chunk's residual solution U
+ * (4 (K V + C V) bytes per chunk and state head), and a chunk-parallel
+ * read-out of every query head.  Without a workspace (NULL) one kernel per
+ * query head carries a copy of its state head.  A non-NULL workspace smaller
+ * than this is KDA_ERR_WORKSPACE.  0 if a size is invalid. */
 size_t kda_fwd_erase_workspace_bytes(int B, int T, int HQ, int HV, int K, int V);
 
 /* Size in bytes of the fixed device array that kda_bwd_noalloc uses as its

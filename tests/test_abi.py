@@ -234,6 +234,8 @@ def test_erase_validation(lib):
     assert call(scale=-1.0) == 7
     assert call(T=0) == 2
     # the two-kernel path's workspace: one record per 32-step chunk and state head
-    assert lib.kda_fwd_erase_workspace_bytes(1, 8, 4, 2, 64, 128) == 1 * 2 * 1 * fma_rec_bytes(64, QG=2)
+    # (then the state entering each chunk and its U, for the read-out kernel)
+    assert lib.kda_fwd_erase_workspace_bytes(1, 8, 4, 2, 64, 128) == 1 * 2 * 1 * (fma_rec_bytes(64, QG=2) +
+                                                                                 4 * (64 * 128 + 32 * 128))
     assert lib.kda_fwd_erase_workspace_bytes(1, 8, 3, 2, 64, 128) == 0  # HQ % HV != 0
     assert call(ws=FAKE, ws_bytes=16) == 5 and "workspace" in lib.kda_last_error().decode()
