@@ -78,11 +78,14 @@ static size_t img_bytes(int B, int T, int HV, int K, int V) {
   return (size_t)B * HV * NT64 * FWI_BYTES;
 }
 
-// scratch of the two-kernel forwards: the chunk images of the tensor-core
-// path (K = V = 128) or the chunk records of the CUDA-core path (fp32, or
-// other K and V), whichever is larger (the dtype is not an argument here)
+// scratch of the two-kernel forwards: for K = V = 128 the chunk images of the
+// tensor-core path or the CUDA-core path's chunk records (fp32 inputs),
+// whichever is larger (the dtype is not an argument here); for other K and V
+// the CUDA-core records, then the state entering and U of every chunk for the
+// separate read-out kernel
 static size_t scratch_bytes(int B, int T, int HV, int K, int V) {
   if (K != 32 && K != 64 && K != 128) return 0;
+  if (fma_kda_split(K, V)) return fma_split_bytes(B, T, HV, HV, K, V);
   const size_t img = img_bytes(B, T, HV, K, V), prep = fma_prep_bytes(B, T, HV, K, 1);
   return img > prep ? img : prep;
 }
@@ -339,7 +342,7 @@ int kda_decode_step(const void* q, const void* k, const void* v, const float* g,
 
 size_t kda_fwd_erase_workspace_bytes(int B, int T, int HQ, int HV, int K, int V) {
   if (B < 1 || T < 1 || HQ < 1 || HV < 1 || HQ % HV || V < 1 || (K != 32 && K != 64 && K != 128)) return 0;
-  return fma_erase_bytes(B, T, HQ, HV, K, V);
+  return fma_split_bytes(B, T, HQ, HV, K, V);
 }
 
 int kda_fwd_erase(const void* q, const void* k, const void* e, const void* z, const float* g, const float* S0,

@@ -336,23 +336,32 @@ struct StateSmem {
   static constexpr int LDV = VB + 1;
   static constexpr int oM = 0, oU = oM + K * LDV, oBuf = oU + C * LDV;
   // a buffer: the chunk's record, then its V rows (TIn, C x VB)
-  static constexpr int vfloats(int) { return (C * VB * (int)sizeof(TIn) + 15) / 16 * 4; }
-  static int buf_floats(int QG) { return fma_rec_floats(K, C, QG) + vfloats(0); }
-  static size_t bytes(int QG, int nbuf) { return (size_t)(oBuf + nbuf * buf_floats(QG)) * sizeof(float); }
+  __host__ __device__ static constexpr int vfloats(int) { return (C * VB * (int)sizeof(TIn) + 15) / 16 * 4; }
+  // (with the read-out split the pass reads only the first part of a record:
+  // T diag(beta), Rt, KEd, e^{c_last})
+  __host__ __device__ static int rec_load(int QG, bool split) {
+    return split ? C * C + 2 * C * K + K : fma_rec_floats(K, C, QG);
+  }
+  __host__ __device__ static int buf_floats(int QG, bool split) { return rec_load(QG, split) + vfloats(0); }
+  static size_t bytes(int QG, bool split, int nbuf) {
+    return (size_t)(oBuf + nbuf * buf_floats(QG, split)) * sizeof(float);
+  }
 };
 
-// (ERASE: the read-out of the query heads is left to kda_fwd_readout_kernel;
-// the pass stores the state entering every chunk into mst [B, HV, NT, K, V]
-// and U into ust [B, HV, NT, C, V] instead.)
+// (With mst and ust (always for ERASE) the read-out is left to
+// kda_fwd_readout_kernel: the pass stores the state entering every chunk into
+// mst [B, HV, NT, K, V] and U into ust [B, HV, NT, C, V] instead.)
 template <int K, int C, int VB, typename TIn, bool ERASE>
 __global__ void __launch_bounds__(NTHREADS, 1)
     kda_fwd_statepass_kernel(FwdArgs a, const float* __restrict__ prep, int nbuf, float* __restrict__ mst,
                              float* __restrict__ ust) {
+  const bool split = ust != nullptr;
   using S = StateSmem<K, C, VB, TIn>;
   constexpr int LDV = S::LDV, TMC = C / 16, TNV = VB / 16, TMK = K / 16;
   extern __shared__ __align__(16) float smem[];
   float *sM = smem + S::oM, *sU = smem + S::oU;
-  const int QG = ERASE ? a.H / a.HV : 1, REC = fma_rec_floats(K, C, QG), BUF = REC + S::vfloats(0);
+  const int QG = ERASE ? a.H / a.HV : 1, REC = fma_rec_floats(K, C, QG), LREC = S::rec_load(QG, split),
+            BUF = S::buf_floats(QG, split);
   const int v0 = blockIdx.x * VB, hv = blockIdx.y, b = blockIdx.z;
   const int T = a.T, V = a.V, NT = (T + C - 1) / C;
   const size_t head = (size_t)b * a.HV + hv;
@@ -365,10 +374,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const auto issue = [&](int ch, float* buf) {  // the chunk's record and V rows into buf
     const float* src = recs + (size_t)ch * REC;
     const uint32_t sb = (uint32_t)__cvta_generic_to_shared(buf);
-    for (int x = threadIdx.x; x < REC / 4; x += NTHREADS) tc::cp_async16(sb + x * 16, src + x * 4, true);
+    for (int x = threadIdx.x; x < LREC / 4; x += NTHREADS) tc::cp_async16(sb + x * 16, src + x * 4, true);
     constexpr int PR = VB * (int)sizeof(TIn) / 16;  // 16-byte pieces per V row
     const int t0 = ch * C, L = min(C, T - t0);
-    const uint32_t vb = sb + REC * 4;
+    const uint32_t vb = sb + LREC * 4;
     for (int x = threadIdx.x; x < C * PR; x += NTHREADS) {
       const int i = x / PR, pc = x % PR;
       const bool ok = i < L;
@@ -395,8 +404,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     __syncthreads();
     const float *cTb = cur, *cRt = cTb + C * C, *cKEd = cRt + C * K, *cEl = cKEd + C * K, *cQ0 = cEl + K;
-    const TIn* cV = reinterpret_cast<const TIn*>(cur + REC);
-    float* const mdst = ERASE ? mst : a.states;
+    const TIn* cV = reinterpret_cast<const TIn*>(cur + LREC);
+    float* const mdst = split ? mst : a.states;  // (mst is the state store when the call keeps states)
     if (mdst) {
       float* dst = mdst + ((head * NT + ch) * K) * V;
       for (int idx = threadIdx.x; idx < K * VB; idx += NTHREADS) {
@@ -416,11 +425,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int y = 0; y < TNV; ++y) {
           const float u = acc[x][y] - neg[x][y];
           sU[(ty + 16 * x) * LDV + tx + 16 * y] = u;
-          if constexpr (ERASE) ust[((head * NT + ch) * C + ty + 16 * x) * V + v0 + tx + 16 * y] = u;
+          if (split) ust[((head * NT + ch) * C + ty + 16 * x) * V + v0 + tx + 16 * y] = u;
         }
     }
     __syncthreads();
-    if (!ERASE && a.o) {
+    if (!split && a.o) {
       for (int qi = 0; qi < QG; ++qi) {  // O = (Q~ o e^c) M + P U for each query head of this state head
         const float* cP = cQ0 + (size_t)qi * (C * C + C * K);
         const float* cQE = cP + C * C;
@@ -468,10 +477,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
 }
 
-// Read-out of the erase/write variant, one CTA per (b, query head, chunk):
-// O = (Q~ o e^c) M + P U over all V columns, from the chunk record and the
-// state and U the state pass stored.
-template <int K, int C, int V, typename TIn>
+// Read-out, one CTA per (b, query head, chunk): O = (Q~ o e^c) M + P U over
+// all V columns, from the chunk record and the state and U the state pass
+// stored (KDA: the query head is the value head).
+template <int K, int C, int V, typename TIn, bool ERASE>
 __global__ void __launch_bounds__(NTHREADS) kda_fwd_readout_kernel(FwdArgs a, const float* __restrict__ prep,
                                                                     const float* __restrict__ mst,
                                                                     const float* __restrict__ ust) {
@@ -479,7 +488,7 @@ __global__ void __launch_bounds__(NTHREADS) kda_fwd_readout_kernel(FwdArgs a, co
   extern __shared__ __align__(16) float smem[];
   float *sQE = smem, *sP = sQE + C * K, *sM = sP + C * C, *sU = sM + K * LDV;
   const int ch = blockIdx.x, hq = blockIdx.y, b = blockIdx.z;
-  const int QG = a.H / a.HV, hv = hq / QG, qi = hq % QG;
+  const int QG = ERASE ? a.H / a.HV : 1, hv = hq / QG, qi = hq % QG, HO = ERASE ? a.H : a.HV;
   const int T = a.T, NT = (T + C - 1) / C, t0 = ch * C, L = min(C, T - t0);
   const size_t hc = ((size_t)b * a.HV + hv) * NT + ch;
   const float* rec = prep + hc * fma_rec_floats(K, C, QG);
@@ -511,7 +520,7 @@ __global__ void __launch_bounds__(NTHREADS) kda_fwd_readout_kernel(FwdArgs a, co
 #pragma unroll
     for (int y = 0; y < TNV; ++y) {
       const int i = ty + 16 * x, n = tx + 16 * y;
-      if (i < L) o[(((size_t)b * T + t0 + i) * a.H + hq) * V + n] = from_f<TIn>(acc[x][y]);
+      if (i < L) o[(((size_t)b * T + t0 + i) * HO + hq) * V + n] = from_f<TIn>(acc[x][y]);
     }
 }
 
@@ -520,24 +529,32 @@ size_t fma_prep_bytes(int B, int T, int HV, int K, int QG) {
   return (size_t)B * HV * NT * fma_rec_floats(K, FWD_CHUNK, QG) * sizeof(float);
 }
 
-// The erase/write variant's workspace: the chunk records, then the state
-// entering every chunk and U of every chunk for its read-out kernel.
-size_t fma_erase_bytes(int B, int T, int HQ, int HV, int K, int V) {
+// The workspace of the read-out split: the chunk records, then the state
+// entering every chunk and U of every chunk for the read-out kernel.
+size_t fma_split_bytes(int B, int T, int HQ, int HV, int K, int V) {
   const size_t NT = (size_t)(T + FWD_CHUNK - 1) / FWD_CHUNK;
   return fma_prep_bytes(B, T, HV, K, HQ / HV) + (size_t)B * HV * NT * ((size_t)K * V + (size_t)FWD_CHUNK * V) * 4;
 }
+// KDA shapes other than K = V = 128 run the read-out split (their scratch is
+// sized for it); K = V = 128 keeps the read-out in the state pass, so that
+// its scratch stays within the tensor-core path's chunk images.
+bool fma_kda_split(int K, int V) { return !(K == 128 && V == 128); }
 
 // Whether the two-kernel CUDA-core forward takes this call: plain inputs (no
 // fused preparation or output gate), 16-byte aligned v (its rows come in by
 // 16-byte copies) and workspace.
 bool fwd_fma2_eligible(const FwdArgs& a, const void* workspace) {
   auto al16 = [](const void* p) { return ((uintptr_t)p & 15u) == 0; };
-  return !a.ctab && !a.prep.z && !a.og && workspace && al16(workspace) && al16(a.v) && a.V % FWD_VBLOCK == 0;
+  return !a.ctab && !a.prep.z && !a.og && workspace && al16(workspace) && al16(a.v) && a.V % 16 == 0;
 }
+
+// state slices of 16 value columns (twice the CTAs of 32-column slices: the
+// pass is latency-bound, measured 0.134 vs 0.147 ms on the fp32 twin workload)
+constexpr int FMA2_VB = 16;
 
 template <int K, typename TIn, bool ERASE>
 static int launch_fwd_fma2_t(const FwdArgs& a, float* prep, cudaStream_t stream) {
-  constexpr int C = FWD_CHUNK, VB = FWD_VBLOCK;
+  constexpr int C = FWD_CHUNK, VB = FMA2_VB;
   const char* who = ERASE ? "kda_fwd_erase" : "kda_fwd";
   const int NT = (a.T + C - 1) / C, QG = ERASE ? a.H / a.HV : 1;
   auto k1 = kda_fwd_chunkprep_kernel<K, C, TIn, ERASE>;
@@ -548,28 +565,32 @@ static int launch_fwd_fma2_t(const FwdArgs& a, float* prep, cudaStream_t stream)
   e = cudaGetLastError();
   if (e != cudaSuccess) return set_cuda_error(who, e);
   using SS = StateSmem<K, C, VB, TIn>;
-  const int nbuf = SS::bytes(QG, 2) <= 200 * 1024 ? 2 : 1;
-  if (SS::bytes(QG, nbuf) > 227 * 1024) return set_error(4, "two-kernel CUDA-core forward: too many query heads per state head");
+  const bool split = ERASE || fma_kda_split(K, a.V);
+  const int nbuf = SS::bytes(QG, split, 2) <= 200 * 1024 ? 2 : 1;
+  if (SS::bytes(QG, split, nbuf) > 227 * 1024)
+    return set_error(4, "two-kernel CUDA-core forward: too many query heads per state head");
   auto k2 = kda_fwd_statepass_kernel<K, C, VB, TIn, ERASE>;
-  e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SS::bytes(QG, nbuf));
+  e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SS::bytes(QG, split, nbuf));
   if (e != cudaSuccess) return set_cuda_error(who, e);
   float* mst = nullptr;
   float* ust = nullptr;
-  if constexpr (ERASE) {
-    mst = prep + fma_prep_bytes(a.B, a.T, a.HV, K, QG) / sizeof(float);
-    ust = mst + (size_t)a.B * a.HV * NT * K * a.V;
+  if (split) {  // (a kept state store doubles as the read-out's state)
+    float* region = prep + fma_prep_bytes(a.B, a.T, a.HV, K, QG) / sizeof(float);
+    mst = (!ERASE && a.states) ? a.states : region;
+    ust = region + (size_t)a.B * a.HV * NT * K * a.V;
   }
-  k2<<<dim3(a.V / VB, a.HV, a.B), NTHREADS, SS::bytes(QG, nbuf), stream>>>(a, prep, nbuf, mst, ust);
+  k2<<<dim3(a.V / VB, a.HV, a.B), NTHREADS, SS::bytes(QG, split, nbuf), stream>>>(a, prep, nbuf, mst, ust);
   e = cudaGetLastError();
   if (e != cudaSuccess) return set_cuda_error(who, e);
-  if constexpr (ERASE) {
+  if (split) {
     if (!a.o) return 0;
     const size_t sb = (size_t)(C * K + C * C + (K + C) * (a.V + 4)) * sizeof(float);
-    const auto k3 = a.V == 32 ? kda_fwd_readout_kernel<K, C, 32, TIn>
-                  : a.V == 64 ? kda_fwd_readout_kernel<K, C, 64, TIn> : kda_fwd_readout_kernel<K, C, 128, TIn>;
+    const auto k3 = a.V == 32 ? kda_fwd_readout_kernel<K, C, 32, TIn, ERASE>
+                  : a.V == 64 ? kda_fwd_readout_kernel<K, C, 64, TIn, ERASE>
+                              : kda_fwd_readout_kernel<K, C, 128, TIn, ERASE>;
     e = cudaFuncSetAttribute(k3, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sb);
     if (e != cudaSuccess) return set_cuda_error(who, e);
-    k3<<<dim3(NT, a.H, a.B), NTHREADS, sb, stream>>>(a, prep, mst, ust);
+    k3<<<dim3(NT, ERASE ? a.H : a.HV, a.B), NTHREADS, sb, stream>>>(a, prep, mst, ust);
     e = cudaGetLastError();
     if (e != cudaSuccess) return set_cuda_error(who, e);
   }

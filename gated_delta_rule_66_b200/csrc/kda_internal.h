@@ -192,7 +192,8 @@ int launch_fwd_erase(const FwdArgs& a, int dtype, cudaStream_t stream);
 // pass); erase: the asymmetric erase/write variant
 bool fwd_fma2_eligible(const FwdArgs& a, const void* workspace);
 size_t fma_prep_bytes(int B, int T, int HV, int K, int QG);
-size_t fma_erase_bytes(int B, int T, int HQ, int HV, int K, int V);
+size_t fma_split_bytes(int B, int T, int HQ, int HV, int K, int V);
+bool fma_kda_split(int K, int V);
 int launch_fwd_fma2(const FwdArgs& a, int dtype, bool erase, float* prep, cudaStream_t stream);
 int launch_fwd_tc(const FwdArgs& a, cudaStream_t stream);
 int take_device_error(unsigned* out);

@@ -89,8 +89,11 @@ size_t kda_fwd_workspace_bytes(int B, int T, int HV, int K, int V);
  * products there, then the sequential state pass.  On the tensor-core path
  * (K = V = 128, bf16) the chunk images take 152,064 bytes per 64-step chunk;
  * on the CUDA-core path (fp32 inputs, or other K and V) the chunk records take
- * 4 (2 C^2 + 3 C K + K) bytes per 32-step chunk (C = 32); the larger of the
- * two, as the dtype is not an argument.  0 if a size is invalid. */
+ * 4 (2 C^2 + 3 C K + K) bytes per 32-step chunk (C = 32); for K = V = 128 the
+ * larger of the two, as the dtype is not an argument.  For other K and V the
+ * CUDA-core path also keeps the state entering every chunk and its residual
+ * solution U (4 (K V + C V) bytes per chunk), and a third, chunk-parallel
+ * kernel forms the outputs.  0 if a size is invalid. */
 size_t kda_fwd_scratch_bytes(int B, int T, int HV, int K, int V);
 
 /* Bytes kda_bwd needs: the chunk states and interaction records (as

@@ -54,7 +54,7 @@ def test_workspace_sizes(lib):
     B, T, H, HV, K, V = 2, 100, 2, 6, 64, 32
     NT = (T + 31) // 32
     states = B * HV * NT * K * V * 4
-    prep = B * HV * NT * fma_rec_bytes(K)
+    prep = B * HV * NT * (fma_rec_bytes(K) + 4 * (K * V + 32 * V))  # records, then M and U per chunk
     assert lib.kda_fwd_scratch_bytes(B, T, HV, K, V) == prep
     assert lib.kda_fwd_workspace_bytes(B, T, HV, K, V) == states + prep
     assert lib.kda_bwd_workspace_bytes(B, T, H, HV, K, V) == states + max(states + 2 * B * T * HV * K * 4, prep)
@@ -141,7 +141,7 @@ def test_tensor_core_workspace_sizes(lib):
     tail = states + 2 * B * T * HV * K * 4 + B * HV * nt64 * 37120 * 4  # state grads, dq/dk partials, records
     assert lib.kda_bwd_workspace_bytes(B, T, H, HV, K, V) == states + inter + max(tail, img)
     assert lib.kda_bwd_workspace_bytes(B, T, H, HV, K, V) >= lib.kda_fwd_workspace_bytes(B, T, HV, K, V)
-    assert lib.kda_fwd_scratch_bytes(B, T, HV, 64, 64) == B * HV * nt32 * fma_rec_bytes(64)  # CUDA-core records
+    assert lib.kda_fwd_scratch_bytes(B, T, HV, 64, 64) == B * HV * nt32 * (fma_rec_bytes(64) + 4 * (64 * 64 + 32 * 64))
     assert lib.kda_fwd_scratch_bytes(B, T, HV, 48, 64) == 0  # unsupported K
 
 
