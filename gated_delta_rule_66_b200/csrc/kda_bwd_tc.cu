@@ -190,18 +190,16 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_dstate_tc_kernel(BwdArgs a) {
     cp_async_commit();
 
     // ---------------------------------------------------------------- store dM (leaving this chunk); start dM_in
+    float sv[2][32];  // dM leaving this chunk (this thread's lane, 64 channels), stored once
+                      // the products below are under way
     {
-      const size_t dm_slot = dstate_slot(a, sq, hv, ch);
       uint32_t r[32];
+#pragma unroll
       for (int cb = 0; cb < 2; ++cb) {
         const int f0 = hcol * 64 + cb * 32;
-        float s[32];
-        tmem_ld32(tm + lo + TM_S + f0, s);
-        float* dst = a.dstates + (dm_slot * KD + f0) * VD + Lr;
+        tmem_ld32(tm + lo + TM_S + f0, sv[cb]);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) dst[(size_t)j * VD] = s[j];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(s[j] * sEl[f0 + j]);
+        for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(sv[cb][j] * sEl[f0 + j]);
         tmem_st32(tm + lo + TM_S + f0, r);
       }
       tmem_wait_st();
@@ -216,6 +214,13 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_dstate_tc_kernel(BwdArgs a) {
         mma_ts(tm + TM_S, tm + TM_DR + ks * 8, desc(sb + OP_NKET + ks * 256, 2048), id, 1);
       }
       commit(bar);
+    }
+    {
+      float* dst = a.dstates + (dstate_slot(a, sq, hv, ch) * KD + hcol * 64) * VD + Lr;
+#pragma unroll
+      for (int cb = 0; cb < 2; ++cb)
+#pragma unroll
+        for (int j = 0; j < 32; ++j) dst[(size_t)(cb * 32 + j) * VD] = sv[cb][j];
     }
     if (!wait_mma(bar, phase)) { failed = true; break; }
     fence_before();
@@ -280,6 +285,8 @@ using namespace tcc;
 // [f][n] over the raw region after the second products.  U, [dO; -dR], M and
 // dM use the padded layout (LBO 144), which their lane-per-column stores need.
 constexpr uint32_t OP_KE = OP, OP_KED = OP + 32768, OP_U = OP, OP_PBR = OP + 36864, OP_DO = OP + 73728;
+// the V rows (bf16 [i][n], 16 KB) wait in the -dR half of [dO; -dR] until X is formed
+constexpr uint32_t OP_V = OP_DO + 64 * 128 * 36 / 8;
 constexpr uint32_t R_TT = 16384, R_MB = 0;
 constexpr uint32_t PAD_SBO = 128 * 36;  // bytes per 8 rows of a padded 128-wide K tile
 static_assert(OP_DO + 2 * 64 * PAD_SBO / 8 <= SMALL && OP_PBR + 1024 <= OP_DO && R_MB + 16 * PAD_SBO <= OP &&
@@ -348,11 +355,14 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
     const float* mst = a.states + state_slot(a, sq, hv, ch) * (KD * VD);     // M: state entering the chunk
     const float* dmst = a.dstates + dstate_slot(a, sq, hv, ch) * (KD * VD);  // dM: gradient of the leaving state
     load_raw_issue(cx, qg, kg, dog, a.g, a.beta, b, T, t0, L, a.H, a.HV, h, hv);
+    for (int x = tid; x < C * 16; x += NTH) {  // V rows [i][n] (bf16) into the -dR half of [dO; -dR]
+      const int i = x >> 4, c16 = x & 15;
+      cp_async16(sb + OP_V + x * 16, vg + (((size_t)b * T + t0 + (i < L ? i : 0)) * a.HV + hv) * VD + c16 * 8, i < L);
+    }
     if (tid < 16) prefetch_l2(mst + tid * 1024, 4096);
     else if (tid < 32) prefetch_l2(dmst + (tid - 16) * 1024, 4096);
     else if (tid == 32) prefetch_l2(irec, 2 * 16384);
     else if (tid == 33) prefetch_l2(irec + INTER_TT, 16384);
-    else if (tid >= 64 && tid < 64 + L) prefetch_l2(vg + (((size_t)b * T + t0 + tid - 64) * a.HV + hv) * VD, VD * 2);
     if (!load_raw_wait(cx)) { failed = true; break; }
     cumsum_span(cx);
 
@@ -414,12 +424,6 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
       }
       tmem_wait_st();
     }
-    float vT[32];  // V^T: lane n, rows i of this warp half
-#pragma unroll
-    for (int jj = 0; jj < 32; ++jj) {
-      const int i = hcol * 32 + jj;
-      vT[jj] = (i < L) ? __bfloat162float(vg[(((size_t)b * T + t0 + i) * a.HV + hv) * VD + Lr]) : 0.f;
-    }
     cp_async_wait_all();
     fence_async_smem();
     fence_before();
@@ -443,8 +447,9 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
       uint32_t r[32];
       tmem_ld32(tm + lo + TM_X + hcol * 32, x);
 #pragma unroll
+      const __nv_bfloat16* sV = reinterpret_cast<const __nv_bfloat16*>(sm + OP_V);
       for (int jj = 0; jj < 32; ++jj) {
-        xs[jj] = vT[jj] - x[jj];
+        xs[jj] = __bfloat162float(sV[(hcol * 32 + jj) * VD + Lr]) - x[jj];
         r[jj] = tf32_rna(sBeta[hcol * 32 + jj] * xs[jj]);
       }
       tmem_st32(tm + lo + TM_X + hcol * 32, r);

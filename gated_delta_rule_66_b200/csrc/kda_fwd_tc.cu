@@ -640,19 +640,16 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_seq_tc_kernel(FwdArgs a) {
       tmem_st32(tm + lo + TM_U + hcol * 32, r);
     }
     if (!wait_bar(barB, ch & 1)) { failed = true; break; }
-    {  // M^T <- M^T diag(e^{c_last}); the entering state for the backward
+    float sv[2][32];  // the entering state (this thread's lane, 64 channels), stored for the
+                      // backward once the state products are under way
+    {  // M^T <- M^T diag(e^{c_last})
       uint32_t r[32];
+#pragma unroll
       for (int cb = 0; cb < 2; ++cb) {
         const int f0 = hcol * 64 + cb * 32;
-        float s[32];
-        tmem_ld32(tm + lo + TM_S + f0, s);
-        if (a.states) {
-          float* dst = a.states + (state_slot(a, sq, hv, sc.c0 + ch) * KD + f0) * VD + Lr;
+        tmem_ld32(tm + lo + TM_S + f0, sv[cb]);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) dst[(size_t)j * VD] = s[j];
-        }
-#pragma unroll
-        for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(s[j] * sEl[f0 + j]);
+        for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(sv[cb][j] * sEl[f0 + j]);
         tmem_st32(tm + lo + TM_S + f0, r);
       }
       tmem_wait_st();
@@ -669,6 +666,13 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_seq_tc_kernel(FwdArgs a) {
         mma_ts(tm + TM_O, tm + TM_U + ks * 8, desc(sb + SQ_B + B_P + ks * 256, 2048), idO, 1);
       }
       commit(bar);
+    }
+    if (a.states) {  // (off the critical path: the products above do not wait for these stores)
+      float* dst = a.states + (state_slot(a, sq, hv, sc.c0 + ch) * KD + hcol * 64) * VD + Lr;
+#pragma unroll
+      for (int cb = 0; cb < 2; ++cb)
+#pragma unroll
+        for (int j = 0; j < 32; ++j) dst[(size_t)(cb * 32 + j) * VD] = sv[cb][j];
     }
     float sig[32];  // sigmoid of the output gate, formed while the products run
     if (gated) {
