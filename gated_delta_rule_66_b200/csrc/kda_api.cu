@@ -314,7 +314,7 @@ int kda_bwd_varlen(const void* q, const void* k, const void* v, const float* g, 
   FwdArgs fa{q, k, v, g, beta, S0, nullptr, nullptr, states, inter, reinterpret_cast<unsigned char*>(x), scale,
              N, T, H, HV, K, V, ctab, ctab + 2 * nc, (int)nc};
   if (!bwd_tc_eligible(a, dtype) || !fwd_tc_eligible(fa, dtype))
-    return set_error(KDA_ERR_ARG, "kda_bwd_varlen: the tensor-core path needs 16-byte aligned q, k, v, dO, g, dq");
+    return set_error(KDA_ERR_ARG, "kda_bwd_varlen: the tensor-core path needs 16-byte aligned q, k, v, dO, g, dq, dv");
   std::vector<int> host(tab);
   host.insert(host.end(), seq0.begin(), seq0.end());
   cudaStream_t st = static_cast<cudaStream_t>(stream);

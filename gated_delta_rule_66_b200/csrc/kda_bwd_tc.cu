@@ -247,7 +247,7 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_dstate_tc_kernel(BwdArgs a) {
 bool bwd_tc_eligible(const BwdArgs& a, int dtype) {
   auto al16 = [](const void* p) { return ((uintptr_t)p & 15u) == 0; };
   return dtype == 1 && a.K == 128 && a.V == 128 && a.gws != nullptr && a.inter != nullptr && al16(a.q) &&
-         al16(a.k) && al16(a.v) && al16(a.dO) && al16(a.g) && al16(a.dq);
+         al16(a.k) && al16(a.v) && al16(a.dO) && al16(a.g) && al16(a.dq) && al16(a.dv);
 }
 
 static int launch_bwd_dstate_tc(const BwdArgs& a, int nheads, cudaStream_t stream) {
@@ -287,6 +287,11 @@ using namespace tcc;
 constexpr uint32_t OP_KE = OP, OP_KED = OP + 32768, OP_U = OP, OP_PBR = OP + 36864, OP_DO = OP + 73728;
 // the V rows (bf16 [i][n], 16 KB) wait in the -dR half of [dO; -dR] until X is formed
 constexpr uint32_t OP_V = OP_DO + 64 * 128 * 36 / 8;
+// dv rows (bf16 [i][n], 16 KB) are staged in the dead K o e^{c_last-c} operand
+// (after the first products, clear of U, the dbeta_R partials and the record)
+constexpr uint32_t OP_DV = OP + 48128;
+static_assert(OP_DV >= OP_PBR + 1024 && OP_DV + 16384 <= OP_KED + 32768 && OP_DV >= 4 * 32768,
+              "dv staging");
 constexpr uint32_t R_TT = 16384, R_MB = 0;
 constexpr uint32_t PAD_SBO = 128 * 36;  // bytes per 8 rows of a padded 128-wide K tile
 static_assert(OP_DO + 2 * 64 * PAD_SBO / 8 <= SMALL && OP_PBR + 1024 <= OP_DO && R_MB + 16 * PAD_SBO <= OP &&
@@ -476,7 +481,7 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
 #pragma unroll
       for (int jj = 0; jj < 32; ++jj) {
         const int i = hcol * 32 + jj;
-        if (i < L) dvg[(((size_t)b * T + t0 + i) * a.HV + hv) * VD + Lr] = __float2bfloat16_rn(sBeta[i] * dr[jj]);
+        reinterpret_cast<__nv_bfloat16*>(sm + OP_DV)[i * VD + Lr] = __float2bfloat16_rn(sBeta[i] * dr[jj]);
         st_tf32(sm, OP_U + kmaj_pad(i, Lr, 128), u[jj]);
         st_tf32(sm, OP_DO + kmaj_pad(64 + i, Lr, 128), -dr[jj]);
         xs[jj] *= dr[jj];
@@ -491,6 +496,11 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
     cp_async_wait_all();
     fence_async_smem();
     __syncthreads();
+    for (int x = tid; x < L * 16; x += NTH) {  // dv rows as 16-byte pieces
+      const int i = x >> 4, c16 = x & 15;
+      *reinterpret_cast<uint4*>(dvg + (((size_t)b * T + t0 + i) * a.HV + hv) * VD + c16 * 8) =
+          *reinterpret_cast<const uint4*>(sm + OP_DV + x * 16);
+    }
     if (tid < C) sDbR[tid] = ((partBr[tid] + partBr[C + tid]) + partBr[2 * C + tid]) + partBr[3 * C + tid];
     if (tid == 0) {  // [dP; dA] = [dO; -dR] U^T ; [dQE; dKE'] = [dO; -dR] M^T
       fence_after();

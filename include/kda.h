@@ -158,7 +158,7 @@ int kda_fwd_varlen(const void* q, const void* k, const void* v, const float* g, 
  *   workspace: at least kda_bwd_varlen_workspace_bytes() bytes, 16-byte aligned
  *   flags: 0 (the forward pass runs first) or KDA_BWD_STATES_FROM_FWD (the
  *     workspace went through kda_fwd_varlen on the same inputs)
- * Tensor-core path only (bf16, K = V = 128, 16-byte aligned q, k, v, dO, g, dq). */
+ * Tensor-core path only (bf16, K = V = 128, 16-byte aligned q, k, v, dO, g, dq, dv). */
 size_t kda_bwd_varlen_workspace_bytes(const int* cu_seqlens, int N, int H, int HV, int K, int V);
 int kda_bwd_varlen(const void* q, const void* k, const void* v, const float* g, const float* beta,
                    const float* S0, const void* dO, const float* dS_T, float scale, const int* cu_seqlens, int N,
