@@ -186,7 +186,19 @@ __device__ __forceinline__ bool fwd_chunk_head(const tcc::Ctx& cx, const FwdArgs
     bulk_commit();
   }
 
-  readout_ap<NTHR>(cx, tm + TM_APA, tm + TM_APB, wide, pw, irec);
+  readout_ap<NTHR>(cx, tm + TM_APA, tm + TM_APB, wide, pw, nullptr);
+  if (irec) {  // the P^T image of the record from the P image (16-byte pieces; piece x holds
+               // P^T(r, k .. k + 3) = P[k .. k + 3][r], r = 8 (x / 128) + x % 8, k = 4 ((x % 128) / 8))
+    for (int x = tid; x < C * C / 4; x += NTHR) {
+      const int r = (x >> 7) * 8 + (x & 7), k = ((x & 127) >> 3) * 4;
+      uint4 w;
+      w.x = *reinterpret_cast<const uint32_t*>(sm + p_off(k, r));
+      w.y = *reinterpret_cast<const uint32_t*>(sm + p_off(k + 1, r));
+      w.z = *reinterpret_cast<const uint32_t*>(sm + p_off(k + 2, r));
+      w.w = *reinterpret_cast<const uint32_t*>(sm + p_off(k + 3, r));
+      *reinterpret_cast<uint4*>(irec + x * 4) = w;
+    }
+  }
   if (img) {  // P is final: store its image now (R_P is not touched again in this chunk)
     fence_async_smem();
     __syncthreads();
