@@ -297,9 +297,26 @@ constexpr uint32_t PAD_SBO = 128 * 36;  // bytes per 8 rows of a padded 128-wide
 static_assert(OP_DO + 2 * 64 * PAD_SBO / 8 <= SMALL && OP_PBR + 1024 <= OP_DO && R_MB + 16 * PAD_SBO <= OP &&
                   R_TT + 16384 <= R_P,
               "gradient-kernel shared-memory map");
-constexpr uint32_t TM_M = 0, TM_U = 0, TM_QK = 0, TM_DM = 128, TM_DR = 128, TM_KED = 128, TM_DOT = 256,
+// TMEM columns: M^T and dM^T stay until they are staged as [f][n] operands
+// for the third and fourth products (U at 448, dR over the spent dO^T)
+constexpr uint32_t TM_M = 0, TM_U = 448, TM_QK = 0, TM_DM = 128, TM_DR = 256, TM_KED = 128, TM_DOT = 256,
                    TM_PA = 256, TM_X = 320, TM_DU = 384;
 }  // namespace tcg
+
+// A K x V state held transposed in TMEM (lane n, column f; columns tmc ..
+// tmc + 127) written to R_MB as the [f][n] operand (padded K-major layout):
+// each thread its lane n and the 64 channels of its column half.
+__device__ __forceinline__ void stage_fn(const tcc::Ctx& cx, uint32_t tmc) {
+  using namespace tcg;
+#pragma unroll
+  for (int cb = 0; cb < 2; ++cb) {
+    const int f0 = cx.hcol * 64 + cb * 32;
+    float v[32];
+    tc::tmem_ld32(cx.tm + cx.lo + tmc + f0, v);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) *reinterpret_cast<float*>(cx.sm + R_MB + tc::kmaj_pad(f0 + j, cx.Lr, 128)) = v[j];
+  }
+}
 
 __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
   using namespace tcg;
@@ -488,12 +505,8 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
       }
       partBr[cx.sub * C + hcol * 32 + lane] = warp_sum32(xs, lane);
     }
-    // M as [f][n] for the sums over n
-    for (int e = tid; e < KD * 32; e += NTH) {
-      const int f = e >> 5, n4 = (e & 31) * 4;
-      cp_async16(sb + R_MB + kmaj_pad(f, n4, 128), mst + f * VD + n4, true);
-    }
-    cp_async_wait_all();
+    stage_fn(cx, TM_M);  // M as [f][n] for the sums over n (from M^T in TMEM)
+    fence_before();
     fence_async_smem();
     __syncthreads();
     for (int x = tid; x < L * 16; x += NTH) {  // dv rows as 16-byte pieces
@@ -512,13 +525,8 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
       commit(bar);
     }
     if (!wait_mma(bar, phase)) { failed = true; break; }
-    {  // dM as [f][n]
-      for (int e = tid; e < KD * 32; e += NTH) {
-        const int f = e >> 5, n4 = (e & 31) * 4;
-        cp_async16(sb + R_MB + kmaj_pad(f, n4, 128), dmst + f * VD + n4, true);
-      }
-      cp_async_wait_all();
-    }
+    stage_fn(cx, TM_DM);  // dM as [f][n] (from dM^T in TMEM)
+    fence_before();
     fence_async_smem();
     __syncthreads();
     if (tid == 0) {  // dKEd = U dM^T
