@@ -211,6 +211,9 @@ int kda_fwd(const void* q, const void* k, const void* v, const float* g, const f
   }
   FwdArgs a{q, k, v, g, beta, S0, o, S_T, states, inter, img, scale, B, T, H, HV, K, V};
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (states && dtype == KDA_DTYPE_BF16 && K == 128 && V == 128 && aligned16(q) && aligned16(k) && aligned16(v) &&
+      aligned16(g) && !aligned16(o))  // (a tensor-core backward on these inputs reads tensor-core records)
+    return set_error(KDA_ERR_ARG, "kda_fwd: the training forward of this shape needs a 16-byte aligned o");
   if (fwd_tc_eligible(a, dtype)) return launch_fwd_tc(a, st);
   if (img && fwd_fma2_eligible(a, img)) {  // the scratch holds the CUDA-core path's chunk records
     a.img = nullptr;

@@ -121,6 +121,10 @@ size_t kda_bwd_workspace_bytes(int B, int T, int H, int HV, int K, int V);
  *     state pass: tensor-core shapes; CUDA-core shapes when v is 16-byte
  *     aligned); without one, one kernel carries each state slice through
  *     its chunks.
+ * With a training workspace, bf16 K = V = 128 and 16-byte aligned q, k, v, g
+ * (the inputs of the tensor-core backward), o must be 16-byte aligned too
+ * (KDA_ERR_ARG otherwise), so that the stored states and records are the
+ * tensor-core path's.
  * o and S_T must not alias any input.  S_T may alias S0 only if S0 is not
  * needed afterwards (S0 is read before S_T is written, per value column). */
 int kda_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,

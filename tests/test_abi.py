@@ -239,3 +239,15 @@ def test_erase_validation(lib):
                                                                                  4 * (64 * 128 + 32 * 128))
     assert lib.kda_fwd_erase_workspace_bytes(1, 8, 3, 2, 64, 128) == 0  # HQ % HV != 0
     assert call(ws=FAKE, ws_bytes=16) == 5 and "workspace" in lib.kda_last_error().decode()
+
+
+def test_training_forward_wants_aligned_o(lib):
+    """bf16 K = V = 128 with aligned inputs and a training workspace: a
+    misaligned o would send the forward down the CUDA-core path while a later
+    tensor-core backward reads tensor-core records, so it is rejected before
+    anything is enqueued."""
+    B, T, H, HV, K, V = 1, 64, 1, 1, 128, 128
+    ws_bytes = lib.kda_fwd_workspace_bytes(B, T, HV, K, V)
+    rc = lib.kda_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, None, 0.1, B, T, H, HV, K, V, 1, ctypes.c_void_p(0x1008), None,
+                     FAKE, ws_bytes, None)
+    assert rc == 7 and "aligned o" in lib.kda_last_error().decode()
