@@ -89,6 +89,25 @@ __device__ __forceinline__ void mm(float (&acc)[TM][TN], int kd, FA fa, FB fb) {
   }
 }
 
+// The same with a compile-time depth, fully unrolled (the loads of later
+// steps are issued ahead: for short, latency-bound products).
+template <int KD, int TM, int TN, typename FA, typename FB>
+__device__ __forceinline__ void mmk(float (&acc)[TM][TN], FA fa, FB fb) {
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+#pragma unroll
+  for (int kk = 0; kk < KD; ++kk) {
+    float a[TM], b[TN];
+#pragma unroll
+    for (int i = 0; i < TM; ++i) a[i] = fa(ty + 16 * i, kk);
+#pragma unroll
+    for (int j = 0; j < TN; ++j) b[j] = fb(kk, tx + 16 * j);
+#pragma unroll
+    for (int i = 0; i < TM; ++i)
+#pragma unroll
+      for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+  }
+}
+
 template <int TM, int TN>
 __device__ __forceinline__ void zero(float (&acc)[TM][TN]) {
 #pragma unroll

@@ -417,8 +417,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       float acc[TMC][TNV], neg[TMC][TNV];
       zero(acc);
       zero(neg);
-      mm(acc, C, [&](int i, int j) { return cTb[i * C + j]; }, [&](int j, int n) { return to_f(cV[j * VB + n]); });
-      mm(neg, K, [&](int i, int f) { return cRt[i * K + f]; }, [&](int f, int n) { return sM[f * LDV + n]; });
+      mmk<C>(acc, [&](int i, int j) { return cTb[i * C + j]; }, [&](int j, int n) { return to_f(cV[j * VB + n]); });
+      mmk<K>(neg, [&](int i, int f) { return cRt[i * K + f]; }, [&](int f, int n) { return sM[f * LDV + n]; });
 #pragma unroll
       for (int x = 0; x < TMC; ++x)
 #pragma unroll
@@ -435,8 +435,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const float* cQE = cP + C * C;
         float acc[TMC][TNV];
         zero(acc);
-        mm(acc, K, [&](int i, int f) { return cQE[i * K + f]; }, [&](int f, int n) { return sM[f * LDV + n]; });
-        mm(acc, C, [&](int i, int j) { return cP[i * C + j]; }, [&](int j, int n) { return sU[j * LDV + n]; });
+        mmk<K>(acc, [&](int i, int f) { return cQE[i * K + f]; }, [&](int f, int n) { return sM[f * LDV + n]; });
+        mmk<C>(acc, [&](int i, int j) { return cP[i * C + j]; }, [&](int j, int n) { return sU[j * LDV + n]; });
         const int ho = ERASE ? hv * QG + qi : hv;
 #pragma unroll
         for (int x = 0; x < TMC; ++x)
@@ -456,7 +456,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           const int f = ty + 16 * x, n = tx + 16 * y;
           acc[x][y] = cEl[f] * sM[f * LDV + n];
         }
-      mm(acc, C, [&](int f, int i) { return cKEd[i * K + f]; }, [&](int i, int n) { return sU[i * LDV + n]; });
+      mmk<C>(acc, [&](int f, int i) { return cKEd[i * K + f]; }, [&](int i, int n) { return sU[i * LDV + n]; });
       __syncthreads();
 #pragma unroll
       for (int x = 0; x < TMK; ++x)

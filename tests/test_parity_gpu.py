@@ -284,15 +284,16 @@ def test_bwd_reuses_forward_states(kda):
         assert torch.equal(x, y)
 
 
-def test_bwd_reuses_two_kernel_cuda_core_states(kda):
-    """CUDA-core shapes: the training forward runs as two kernels and stores
-    every 32-step state; the backward that reuses them meets the fp32 bar
-    (its own forward recomputation takes the single-kernel path)."""
-    w = BY_NAME["twin"].with_sizes(B=1, T=100, H=2, HV=4, K=64, V=32)
+@pytest.mark.parametrize("K,V", [(64, 32), (128, 128)], ids=["K64V32_split_readout", "K128V128_fp32"])
+def test_bwd_reuses_two_kernel_cuda_core_states(kda, K, V):
+    """CUDA-core shapes: the training forward runs as two (or three) kernels
+    and stores every 32-step state; the backward that reuses them meets the
+    fp32 bar (its own forward recomputation takes the single-kernel path)."""
+    w = BY_NAME["twin"].with_sizes(B=1, T=100, H=2, HV=4, K=K, V=V)
     inp = make_inputs(w, with_do=True)
     grads = run_bwd(kda, inp, w.scale, reuse=True)
     for n, x, r in zip(GRAD_NAMES, grads, oracle_bwd(inp, w.scale)):
-        report(f"fma_reuse {n}", f64(x), r, tol_for(w.torch_dtype), torch.float32)
+        report(f"fma_reuse_K{K}V{V} {n}", f64(x), r, tol_for(w.torch_dtype), torch.float32)
 
 
 def test_fwdbwd_full_size(kda):
