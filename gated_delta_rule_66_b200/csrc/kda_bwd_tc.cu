@@ -282,8 +282,9 @@ using namespace tcc;
 // Shared memory: K o e^c and K o e^{c_last-c} until the first products, then U
 // over them; [dO; -dR] at the top of the operand region; the T^T, P^T and T
 // images in the raw region once the raw chunk is consumed; M or dM staged as
-// [f][n] over the raw region after the second products.  U, [dO; -dR], M and
-// dM use the padded layout (LBO 144), which their lane-per-column stores need.
+// [f][n] over the raw region after the second products (written from their
+// transposed TMEM copies).  U, [dO; -dR], M and dM use the padded layout
+// (LBO 144), which their lane-per-column stores need.
 constexpr uint32_t OP_KE = OP, OP_KED = OP + 32768, OP_U = OP, OP_PBR = OP + 36864, OP_DO = OP + 73728;
 // the V rows (bf16 [i][n], 16 KB) wait in the -dR half of [dO; -dR] until X is formed
 constexpr uint32_t OP_V = OP_DO + 64 * 128 * 36 / 8;
