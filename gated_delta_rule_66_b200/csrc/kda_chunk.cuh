@@ -418,13 +418,6 @@ __device__ __forceinline__ void mma3(float (&d)[4], const Split (&a)[4], const S
   mma_16x8x8(d, ah, bh);
 }
 
-// One tf32 product (operands rounded to tf32 once: relative error ~2^-11 per
-// product), for sums whose result is rounded to bf16 anyway.
-__device__ __forceinline__ void mma1(float (&d)[4], const Split (&a)[4], const Split (&b)[2]) {
-  const uint32_t ah[4] = {a[0].hi, a[1].hi, a[2].hi, a[3].hi}, bh[2] = {b[0].hi, b[1].hi};
-  mma_16x8x8(d, ah, bh);
-}
-
 template <int K, int C, int LDK_ = K + 1, int LDC_ = C + 1>
 __device__ void factored_block_mma(int J, const float* sK, const float* sQ, const float* sdA, const float* sdP,
                                    const float* sE1, const float* sE2o, const float* sE2d, float* sDq, float* sDk,

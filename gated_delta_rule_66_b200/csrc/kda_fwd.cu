@@ -713,13 +713,4 @@ int launch_out_gate(const float* o32, const void* og, float eps, size_t rows, in
   return 0;
 }
 
-size_t fwd_smem_bytes(int K) {
-  switch (K) {
-    case 32: return FwdSmem<32, FWD_CHUNK, FWD_VBLOCK>::bytes;
-    case 64: return FwdSmem<64, FWD_CHUNK, FWD_VBLOCK>::bytes;
-    case 128: return FwdSmem<128, FWD_CHUNK, FWD_VBLOCK>::bytes;
-  }
-  return 0;
-}
-
 }  // namespace kda

@@ -198,7 +198,6 @@ int launch_fwd_fma2(const FwdArgs& a, int dtype, bool erase, float* prep, cudaSt
 int launch_fwd_tc(const FwdArgs& a, cudaStream_t stream);
 int take_device_error(unsigned* out);
 int take_bwd_device_error(unsigned* out);
-size_t fwd_smem_bytes(int K);
 int launch_bwd(const BwdArgs& a, int dtype, cudaStream_t stream);
 bool bwd_tc_eligible(const BwdArgs& a, int dtype);
 // the tensor-core backward: state-gradient pass, gradient products and the
