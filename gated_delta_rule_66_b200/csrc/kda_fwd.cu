@@ -511,8 +511,8 @@ __global__ void __launch_bounds__(NTHREADS) kda_fwd_readout_kernel(FwdArgs a, co
   __syncthreads();
   float acc[TMC][TNV];
   zero(acc);
-  mm(acc, K, [&](int i, int f) { return sQE[i * K + f]; }, [&](int f, int n) { return sM[f * LDV + n]; });
-  mm(acc, C, [&](int i, int j) { return sP[i * C + j]; }, [&](int j, int n) { return sU[j * LDV + n]; });
+  mmk<K>(acc, [&](int i, int f) { return sQE[i * K + f]; }, [&](int f, int n) { return sM[f * LDV + n]; });
+  mmk<C>(acc, [&](int i, int j) { return sP[i * C + j]; }, [&](int j, int n) { return sU[j * LDV + n]; });
   TIn* o = static_cast<TIn*>(a.o);
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
 #pragma unroll
