@@ -315,11 +315,11 @@ def gpu_path(kda, name, steps, warmup, rank_barrier, shrink=None):
             kda.bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["dO"], scale=w.scale,
                     initial_state=d["S0"], workspace=ws, states_from_fwd=True)
         # kda_fwd: chunk-parallel kernel + state pass; kda_bwd: state gradients,
-        # gradient products, assembly (the first two launched twice when the
-        # heads leave a partial last wave of SMs), +2 group sums when HV > H
+        # gradient products, assembly (each launched twice when the heads leave
+        # a partial last wave of SMs), +2 group sums when HV > H
         sms = torch.cuda.get_device_properties(dev).multi_processor_count
         heads = w.B * w.HV
-        launches_per_step = 2 + (5 if heads > sms and heads % sms else 3) + (2 if w.HV > w.H else 0)
+        launches_per_step = 2 + (6 if heads > sms and heads % sms else 3) + (2 if w.HV > w.H else 0)
         tokens = w.B * w.T
     else:
         S = d["S"]
