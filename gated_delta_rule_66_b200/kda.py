@@ -118,6 +118,11 @@ def _req(name, t, dtype=None, ndim=None):
         return
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
+    if t.get_device() != torch.cuda.current_device():
+        # the library launches on the calling thread's current device and on
+        # its stream; a buffer of another GPU would be read across devices
+        raise ValueError(f"{name} is on cuda:{t.get_device()} but the current CUDA device is "
+                         f"cuda:{torch.cuda.current_device()} (use torch.cuda.device / set_device)")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if dtype is not None and t.dtype != dtype:

@@ -17,7 +17,9 @@
  *
  * Conventions shared by every entry point
  *   - All tensor pointers are caller-owned DEVICE pointers to dense row-major
- *     arrays with the stated shapes.  The library never frees or retains them.
+ *     arrays with the stated shapes, in the memory of the calling thread's
+ *     current CUDA device (the one the kernels launch on; stream must belong
+ *     to it too).  The library never frees or retains them.
  *   - dtype selects the element type of q, k, v, o, dO, dq, dk, dv:
  *     KDA_DTYPE_FP32 (float) or KDA_DTYPE_BF16 (bfloat16).  g, beta, states
  *     and their gradients are always float.
