@@ -427,10 +427,12 @@ static int launch_assemble(const BwdArgs& a0, int head0, int nheads, cudaStream_
   const int NT = a0.ctab ? a0.NC : (a0.T + 63) / 64;
   if (NT == 0 || nheads <= 0) return 0;  // (packed batches of empty sequences)
   BwdArgs a = a0;
-  a.head0 = head0;
-  kern<<<dim3(NT * 4, nheads), NTHREADS, AsmSmem::bytes, stream>>>(a);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return set_cuda_error("kda_bwd: assemble launch", e);
+  for (int done = 0; done < nheads; done += 65535) {  // gridDim.y is at most 65535
+    a.head0 = head0 + done;
+    kern<<<dim3(NT * 4, min(nheads - done, 65535)), NTHREADS, AsmSmem::bytes, stream>>>(a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return set_cuda_error("kda_bwd: assemble launch", e);
+  }
   return 0;
 }
 
