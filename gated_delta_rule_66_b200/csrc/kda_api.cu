@@ -442,6 +442,8 @@ int kda_short_conv(const void* xq, const void* xk, const void* xv, const float* 
   if (!xq || !xk || !xv || !w || !q || !k || !v)
     return set_error(KDA_ERR_NULL, "kda_short_conv: xq, xk, xv, w, q, k and v must be non-NULL");
   if (W < 1 || W > 8) return set_error(KDA_ERR_ARG, "kda_short_conv: W must be in 1..8");
+  if ((long long)T > 65535LL * 32)  // blocks of 32 steps on gridDim.y
+    return set_error(KDA_ERR_SHAPE, "kda_short_conv: T above 2097120 steps exceeds the launch grid");
   const size_t cn = (size_t)2 * H * K + (size_t)HV * V, win = (size_t)B * cn * W * sizeof(float);
   if (ranges_overlap(state_in, win, state_out, win))
     return set_error(KDA_ERR_ARG, "kda_short_conv: state_out must not overlap state_in");

@@ -245,7 +245,8 @@ int kda_fwd_prep(const void* q, const void* k, const void* v, const void* z, con
  *   (zero window); state_out the same shape (the window after the last step)
  *   or NULL; state_out must not overlap state_in
  *   q, k, v outputs in the shapes and dtype of xq, xk, xv (the convolved
- *   activations, rounded to dtype); they must not alias the inputs. */
+ *   activations, rounded to dtype); they must not alias the inputs.
+ *   T <= 2097120 (65535 blocks of 32 steps; KDA_ERR_SHAPE above). */
 int kda_short_conv(const void* xq, const void* xk, const void* xv, const float* w, const float* state_in,
                    float* state_out, int B, int T, int H, int HV, int K, int V, int W, int dtype, void* q,
                    void* k, void* v, void* stream);

@@ -203,6 +203,7 @@ def test_prep_workspace_and_validation(lib):
     assert "overlap" in lib.kda_last_error().decode()
     assert conv(q=FAKE) == 7 and "alias" in lib.kda_last_error().decode()
     assert conv(w=None) == 1
+    assert conv(T=65535 * 32 + 1) == 2 and "launch grid" in lib.kda_last_error().decode()
 
     def tok(**over):
         a = dict(xq=FAKE, xk=FAKE, xv=FAKE, cw=FAKE, ci=ctypes.c_void_p(0x400000), co=ctypes.c_void_p(0x400000),
