@@ -638,11 +638,20 @@ class OracleSampler:
                         f64(inp["beta"][b:b + 1, :, hv:hv + 1]),
                         None if inp["S0"] is None else f64(inp["S0"][b:b + 1, hv:hv + 1]),
                         None if inp.get("dO") is None else f64(inp["dO"][b:b + 1, :, hv:hv + 1]))
-        # calibrate one head (in this process) on a short prefix, then size the sample
+        self.pool = mp.get_context("spawn").Pool(processes=self.cores)
+        self.pool.map(_warm, range(self.cores))   # worker start-up stays outside the timing
+        # calibrate on a short prefix of one head with every worker busy at once
+        # (as in the timed run: shared cores and memory bandwidth), then size the sample
         cal = min(T, 64)
         q, k, v, g, beta, S0, dO = arrays(0, 0)
         cut = lambda x: None if x is None or w.path == "decode" else x[:, :cal]
-        t_cal = _oracle_head((w.path, (cut(q), cut(k), cut(v), cut(g), cut(beta), S0, cut(dO)), w.scale))
+        cal_job = (w.path, (cut(q), cut(k), cut(v), cut(g), cut(beta), S0, cut(dO)), w.scale)
+        try:  # the first pass warms every worker's NumPy; the second is timed
+            self.pool.map(_oracle_head, [cal_job] * self.cores, chunksize=1)
+            t_cal = statistics.median(self.pool.map(_oracle_head, [cal_job] * self.cores, chunksize=1))
+        except BaseException:
+            self.pool.terminate()
+            raise
         t_head = max(t_cal * T / cal, 1e-4)
         per_worker = max(1, int(budget_s / t_head))
         n = min(len(units), self.cores * per_worker)
@@ -651,8 +660,6 @@ class OracleSampler:
         self.desc = (f"{n} of {len(units)} (b, hv) heads, each the full {T} steps "
                      f"({'fwd+bwd' if w.path == 'fwdbwd' else w.path}), float64 NumPy, one single-threaded "
                      f"process per core; tokens/s = head-tokens / {w.HV} heads / elapsed")
-        self.pool = mp.get_context("spawn").Pool(processes=self.cores)
-        self.pool.map(_warm, range(self.cores))   # worker start-up stays outside the timing
 
     def run(self):
         t0 = time.perf_counter()
