@@ -557,11 +557,13 @@ def run_gpu(args):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": "tf32",  # arithmetic: tf32 tensor-core products, fp32 accumulation and CUDA-core steps
         "data": "synthetic (seeded; q,k L2-normalised, g = -5 sigmoid(N(0,1)), beta = sigmoid(N(0,1)))",
         "config": {"workload": f"fwdbwd: B={w.B} H=HV={w.HV} T={w.T} K=V={w.K}, bf16 q/k/v/dO, fp32 g/beta/state; "
                                "step = kda_fwd (stores chunk states and interaction records) + kda_bwd (reuses them)"
                                + ("" if not args.shrink else " [reduced for a profiler capture]"),
+                   "arithmetic": "tf32 tensor-core products with fp32 accumulation, fp32 CUDA-core steps; "
+                                 "bf16 q/k/v/o/dO storage",
                    "global_batch": w.B * world, "seq_len": w.T, "parallelism": f"replicas x{world}",
                    "l2": head["l2"]},
         "roofline": dict({k: v for k, v in head["roofline"].items() if k != "fwd"},
