@@ -76,3 +76,28 @@ def test_raw_and_erase_inputs_are_seeded():
         if isinstance(t, torch.Tensor):
             assert torch.equal(t, e2[n]), n
     assert (e1["g"] < 0).all() and (e1["g"] > -0.25).all()       # -0.25 sigmoid(.)
+
+
+def test_head_subset_keeps_whole_query_groups():
+    """The full-size parity tests check a subset of query/key heads with all
+    their value heads; on the oracle, the subset's results must equal the
+    full problem's results at those heads (heads are independent, and dq/dk
+    sum whole groups)."""
+    import numpy as np
+
+    import oracle
+    from gated_delta_rule_66_b200.inputs import head_subset
+
+    w = BY_NAME["prefill_gqa"].with_sizes(B=1, T=9, H=3, HV=6, K=32, V=32, dtype="fp32")
+    full = make_inputs(w, with_do=True)
+    sub, hv_idx = head_subset(full, w.H, w.HV, [2, 0])
+    assert hv_idx == [4, 5, 0, 1]
+    f64 = lambda d: [None if d[n] is None else d[n].double().numpy() for n in ("q", "k", "v", "g", "beta")]
+    o_full, S_full = oracle.kda_forward(*f64(full), w.scale, None)
+    o_sub, S_sub = oracle.kda_forward(*f64(sub), w.scale, None)
+    assert np.allclose(o_sub, o_full[:, :, hv_idx], rtol=0, atol=1e-14)
+    assert np.allclose(S_sub, S_full[:, hv_idx], rtol=0, atol=1e-14)
+    g_full = oracle.kda_backward(*f64(full), w.scale, None, full["dO"].double().numpy())
+    g_sub = oracle.kda_backward(*f64(sub), w.scale, None, sub["dO"].double().numpy())
+    assert np.allclose(g_sub[0], g_full[0][:, :, [2, 0]], rtol=0, atol=1e-13)   # dq over whole groups
+    assert np.allclose(g_sub[2], g_full[2][:, :, hv_idx], rtol=0, atol=1e-13)   # dv per value head
