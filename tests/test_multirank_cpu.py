@@ -39,7 +39,7 @@ def _rank_main(rank, world, port, out):
 
 def test_job_throughput_two_gloo_ranks():
     world, port = 2, _free_port()
-    out = tmp.Manager().dict()
+    out = tmp.get_context("spawn").Manager().dict()  # no fork of this (threaded) process
     tmp.spawn(_rank_main, args=(world, port, out), nprocs=world, join=True)
     for r in range(world):
         ms, tps = out[r]
