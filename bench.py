@@ -101,6 +101,35 @@ def chunk_flops_per_head_token(K, V, C):
     return 2 * (3 * K * V + 2 * C * K + 2 * C * V)
 
 
+# The chunked backward's contractions per (head, token), as a multiple of the
+# forward's: the state-gradient products, the recomputed residuals, the
+# gradient products summed over the value columns and the interaction terms
+# (dense tiles) come to about 2.5 times the forward's.
+BWD_FLOPS_RATIO = 2.5
+NOMINAL_HBM_GBS = 7700.0  # B200 HGX nominal HBM3e bandwidth, for context beside the measured copy peak
+
+
+def tf32_peak_tflops(peaks):
+    """Dense tf32 tensor peak: the measured dense bf16 peak times the nominal
+    tf32 : bf16 ratio (1.1 : 2.25 PFLOP/s, i.e. one half)."""
+    return peaks["bf16_tflops"] * 0.5
+
+
+def two_rooflines(byts, flops, seconds, peaks):
+    """Both fractions of a chunked call (HBM bytes and tf32 tensor flops) and
+    the binding one (the bound whose ideal time is longer)."""
+    hbm, tpk = peaks["hbm_gbs"], tf32_peak_tflops(peaks)
+    gbs, tfs = byts / seconds / 1e9, flops / seconds / 1e12
+    t_hbm, t_tc = byts / (hbm * 1e9), flops / (tpk * 1e12)
+    hbm_part = {"achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm, "algorithmic_bytes": byts,
+                "peak_source": f"{peaks['source']} copy bandwidth"}
+    tc_part = {"achieved": tfs, "peak": tpk, "unit": "TFLOP/s", "frac": tfs / tpk, "algorithmic_flops": flops,
+               "peak_source": f"{peaks['source']} dense bf16 x 1/2 (nominal tf32 : bf16 ratio)"}
+    top = dict(tc_part, bound="tensor") if t_tc > t_hbm else dict(hbm_part, bound="hbm")
+    top["hbm"], top["tensor"] = hbm_part, tc_part
+    return top
+
+
 # ---------------------------------------------------------------------------- GPU arm
 
 class Clocks:
@@ -479,25 +508,27 @@ def roofline_for(res, w, peaks):
         byts = algorithmic_bytes(w, "decode")
         t = res["calls"]["kernel_ms"] * 1e-3
         return {"bound": "hbm", "kernel": "kda_decode_kernel", "achieved": byts / t / 1e9,
-                "peak": hbm, "unit": "GB/s", "frac": byts / t / 1e9 / hbm, "algorithmic_bytes": byts}
+                "peak": hbm, "unit": "GB/s", "frac": byts / t / 1e9 / hbm, "algorithmic_bytes": byts,
+                "frac_of_nominal": byts / t / 1e9 / NOMINAL_HBM_GBS, "nominal_peak": NOMINAL_HBM_GBS}
+    C = 64 if w.K == 128 else 32
+    head_tokens = w.B * w.T * w.HV
+    fwd_flops = chunk_flops_per_head_token(w.K, w.V, C) * head_tokens
     if w.path == "fwd":
-        byts = algorithmic_bytes(w, "fwd")
-        t = res["calls"]["kernel_ms"] * 1e-3
-        return {"bound": "hbm", "kernel": "kda_fwd (kda_fwd_prep_tc_kernel + kda_fwd_seq_tc_kernel)"
-                if w.K == 128 and w.dtype == "bf16" else "kda_fwd_chunk_kernel", "achieved": byts / t / 1e9,
-                "peak": hbm, "unit": "GB/s", "frac": byts / t / 1e9 / hbm, "algorithmic_bytes": byts}
-    # the step's dominant part is the backward call (three kernels: state gradients,
-    # gradient products, assembly); its algorithmic bytes are the backward's own I/O
-    byts = algorithmic_bytes(w, "bwd")
-    t = res["calls"]["bwd_ms"] * 1e-3
-    fb = algorithmic_bytes(w, "fwd")
-    tf = res["calls"]["fwd_ms"] * 1e-3
-    return {"bound": "hbm", "kernel": "kda_bwd (kda_bwd_dstate_tc_kernel + kda_bwd_grads_tc_kernel + "
-                                      "kda_bwd_assemble_kernel, one call)",
-            "achieved": byts / t / 1e9, "peak": hbm, "unit": "GB/s", "frac": byts / t / 1e9 / hbm,
-            "algorithmic_bytes": byts,
-            "fwd": {"kernel": "kda_fwd (kda_fwd_prep_tc_kernel + kda_fwd_seq_tc_kernel, one call)",
-                    "achieved": fb / tf / 1e9, "frac": fb / tf / 1e9 / hbm, "algorithmic_bytes": fb}}
+        r = two_rooflines(algorithmic_bytes(w, "fwd"), fwd_flops, res["calls"]["kernel_ms"] * 1e-3, peaks)
+        r["kernel"] = ("kda_fwd (tensor-core chunk kernels, one call)"
+                       if w.K == 128 and w.dtype == "bf16" else "kda_fwd (CUDA-core chunk kernels)")
+        return r
+    # the step's dominant part is the backward call (state gradients, gradient
+    # products, assembly); its algorithmic bytes are the backward's own I/O
+    r = two_rooflines(algorithmic_bytes(w, "bwd"), BWD_FLOPS_RATIO * fwd_flops, res["calls"]["bwd_ms"] * 1e-3,
+                      peaks)
+    r["kernel"] = ("kda_bwd (kda_bwd_dstate_tc_kernel + kda_bwd_grads_tc_kernel + kda_bwd_assemble_kernel, "
+                   "one call)")
+    r["fwd"] = dict(two_rooflines(algorithmic_bytes(w, "fwd"), fwd_flops, res["calls"]["fwd_ms"] * 1e-3, peaks),
+                    kernel="kda_fwd (tensor-core chunk kernels, one call)")
+    r["step"] = two_rooflines(algorithmic_bytes(w, "fwdbwd"), (1 + BWD_FLOPS_RATIO) * fwd_flops,
+                              res["ms_per_step"] * 1e-3, peaks)
+    return r
 
 
 def job_throughput(ms_local, tokens_per_step, world, all_reduce_max):
@@ -684,6 +715,13 @@ def cpu_baseline(w, budget_s=20.0):
 
 
 def run_reference(args):
+    """The reference arm: the float64 oracle on the host cores.  One step is
+    one bounded sample of the headline workload (whole (b, hv) heads at the
+    full length, as many as fit the step's time budget), so ms_per_step is the
+    time the sample actually took and steps x ms_per_step is the time this
+    run spent in timed steps.  The throughput scales the sample's head-tokens
+    to all value heads of a token; the time a whole step (every head) would
+    take at that rate is reported beside it, labelled as an extrapolation."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
@@ -696,12 +734,16 @@ def run_reference(args):
         smp.close()
     timed = runs[args.warmup:]
     val = statistics.median(c["value"] for c in timed)
-    line = {"metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": w.B * w.T / val * 1e3,
+    sample_ms = statistics.median(c["seconds"] for c in timed) * 1e3
+    line = {"metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": 1, "steps": len(timed),
+            "warmup": len(runs) - len(timed), "ms_per_step": sample_ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": {"workload": "fwdbwd: B=2 H=HV=96 T=4096 K=V=128 (float64 oracle on a bounded sample)",
-                       "global_batch": w.B, "seq_len": w.T, "parallelism": "none"},
+            "config": {"workload": "fwdbwd: B=2 H=HV=96 T=4096 K=V=128 (float64 oracle); one step = one bounded "
+                                   "sample of whole heads, tokens/s scaled to all value heads",
+                       "global_batch": w.B, "seq_len": w.T, "parallelism": "none",
+                       "step": timed[-1]["sample"],
+                       "extrapolated_full_step_ms": w.B * w.T / val * 1e3},
             "cpu_baseline": {"kind": "oracle", "cores": timed[-1]["cores"], "sample": timed[-1]["sample"],
                              "value": val, "unit": "tokens/s"},
             "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

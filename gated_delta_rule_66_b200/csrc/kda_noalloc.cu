@@ -33,7 +33,10 @@ void* g_scratch_ptr[kMaxDevices] = {};
 
 // Device address of g_kda_scratch on the current device (looked up once per
 // device; the host-side name g_kda_scratch is only a stand-in and must never
-// be handed to a kernel).
+// be handed to a kernel).  The cached address belongs to the device's primary
+// context: a cudaDeviceReset() destroys that context, and the address is not
+// looked up again afterwards, so such a process must not call
+// kda_bwd_noalloc again.
 int scratch_for_current_device(void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);

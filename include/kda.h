@@ -35,8 +35,10 @@
  *     arguments are validated before anything is enqueued, so a non-zero
  *     return from validation leaves all buffers untouched.  kda_last_error()
  *     returns a message for the calling thread's most recent failure.
- *   - The library allocates no device memory; the backward takes its scratch
- *     from the caller's workspace.
+ *   - The library makes no device allocation when it is called: scratch
+ *     comes from the caller's workspace.  Its module does hold one fixed
+ *     array of KDA_NOALLOC_SCRATCH_BYTES on every GPU that loads it (the
+ *     scratch of kda_bwd_noalloc), from load until the process exits.
  */
 #ifndef KDA_H_
 #define KDA_H_
@@ -305,8 +307,9 @@ size_t kda_fwd_erase_workspace_bytes(int B, int T, int HQ, int HV, int K, int V)
 /* kda_bwd for callers that cannot allocate device memory: a plugin whose host
  * framework owns all device memory and gives it no workspace, or a running
  * loop that forbids allocator calls (cudaMalloc/cudaFree synchronise the
- * device and fail once another allocator has reserved the memory).  The paper
- * has no counterpart to this entry point; it is a deployment convenience.
+ * device and fail once another allocator has reserved the memory).  Nothing
+ * in the method's definition corresponds to this entry point; it is a
+ * deployment convenience.
  *   Arguments, layouts and results are those of kda_bwd (flags = 0); the
  *   caller still owns every input and output.  The scratch is a file-scope
  *   __device__ array of KDA_NOALLOC_SCRATCH_BYTES; a problem whose
@@ -314,7 +317,8 @@ size_t kda_fwd_erase_workspace_bytes(int B, int T, int HQ, int HV, int K, int V)
  *   message and enqueues nothing.  Nothing is allocated: the first call on a
  *   device looks up the array's device address (cudaGetSymbolAddress) with
  *   that device current and caches it, so make that first call before any
- *   stream capture.  All calls share the one array: calls whose work overlaps
+ *   stream capture.  A cudaDeviceReset() on that device invalidates the
+ *   cached address: do not call kda_bwd_noalloc again in such a process.  All calls share the one array: calls whose work overlaps
  *   on the GPU (other streams or threads on the same device) race and must be
  *   ordered by the caller.  Each call writes every scratch byte it reads, so
  *   stale contents from an earlier call are never used. */

@@ -298,13 +298,20 @@ def test_bwd_reuses_two_kernel_cuda_core_states(kda, K, V):
 
 def test_fwdbwd_full_size(kda):
     """Production fwd+bwd (B=2, H=HV=96, T=4096, K=V=128, bf16) on the GPU in
-    full; the oracle checks value heads 17 and 60 of both batch rows."""
+    full, run exactly as the benchmark step runs it: the training forward
+    stores its chunk states and records in the workspace and the backward
+    reuses them (B * HV = 192 heads also exercise the backward's split of the
+    partial last wave onto its side stream).  The oracle checks value heads 17
+    and 60 of both batch rows."""
     w = BY_NAME["fwdbwd"]
     inp = make_inputs(w)
     d = to_cuda(inp)
-    o, S = kda.fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], scale=w.scale, initial_state=d["S0"])
+    ws = torch.empty(kda.workspace_bytes("bwd", w.B, w.T, w.H, w.HV, w.K, w.V), dtype=torch.uint8,
+                     device="cuda")
+    o, S = kda.fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], scale=w.scale, initial_state=d["S0"],
+                   workspace=ws)
     grads = kda.bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["dO"], scale=w.scale,
-                    initial_state=d["S0"])
+                    initial_state=d["S0"], workspace=ws, states_from_fwd=True)
     torch.cuda.synchronize()
     sub, hv_idx = head_subset(inp, w.H, w.HV, [17, 60])
     o_ref, S_ref = oracle_fwd(sub, w.scale)

@@ -3,10 +3,11 @@
 Such callers (a plugin whose host framework owns all device memory, a
 running loop that forbids allocator calls) cannot hand kda_bwd a workspace;
 kda_bwd_noalloc takes its scratch from a fixed device array inside the
-library instead.  These tests call it through the C ABI and check that two
-calls in a row (the second reusing the array the first left behind) match
-kda_bwd with a caller workspace.  The file is named so that pytest collects
-it last.
+library instead.  These tests call it through the C ABI twice in a row on each
+problem (the second call reuses the array exactly as the first left it) and
+check both results bit for bit against kda_bwd with a caller workspace (the
+kernels are deterministic) and against the float64 oracle.  The file is named
+so that pytest collects it last.
 """
 from __future__ import annotations
 
@@ -15,6 +16,7 @@ import ctypes
 import pytest
 import torch
 
+import oracle
 from gated_delta_rule_66_b200.inputs import BY_NAME, make_inputs
 from kda_testlib import f64, rel_l2, tol_for
 
@@ -69,14 +71,21 @@ def test_noalloc_matches_workspace_backward_twice():
     kda, lib = _lib()
     cases = [BY_NAME["prefill_gqa"].with_sizes(T=200, H=2, HV=4),          # bf16, grouped heads
              BY_NAME["twin"].with_sizes(B=2, T=150, H=2, HV=2, K=64, V=64)]  # fp32, S0 != 0
-    for w in cases:  # two calls in a row; the second reuses what the first left in the array
+    names = ("dq", "dk", "dv", "dg", "dbeta", "dS0")
+    for w in cases:
         assert kda.workspace_bytes("bwd", w.B, w.T, w.H, w.HV, w.K, w.V) <= NOALLOC_BYTES
         inp = make_inputs(w, with_do=True)
         d = {n: (None if t is None else t.cuda()) for n, t in inp.items()}
         ref = kda.bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["dO"], scale=w.scale,
                       initial_state=d["S0"])
-        got = _noalloc_grads(kda, lib, d, w)
-        torch.cuda.synchronize()
-        for name, x, r in zip(("dq", "dk", "dv", "dg", "dbeta", "dS0"), got, ref):
-            err = rel_l2(f64(x), f64(r))
-            assert err <= tol_for(w.torch_dtype), f"{w.name} {name}: {err:.3e}"
+        exact = oracle.kda_backward(f64(inp["q"]), f64(inp["k"]), f64(inp["v"]), f64(inp["g"]),
+                                    f64(inp["beta"]), w.scale, f64(inp["S0"]), f64(inp["dO"]))
+        for call in range(2):  # the second call starts from what the first left in the array
+            got = _noalloc_grads(kda, lib, d, w)
+            torch.cuda.synchronize()
+            for name, x, r, e in zip(names, got, ref, exact):
+                assert torch.equal(x, r), (
+                    f"{w.name} call {call} {name}: differs from kda_bwd "
+                    f"(rel_l2 {rel_l2(f64(x), f64(r)):.3e})")
+                err = rel_l2(f64(x), e)
+                assert err <= tol_for(w.torch_dtype), f"{w.name} call {call} {name}: {err:.3e} vs oracle"
