@@ -71,7 +71,7 @@ static size_t inter_bytes(int B, int T, int HV, int K, int V) {
   return (size_t)B * HV * NT64 * INTER_REC * sizeof(float);
 }
 
-// per-chunk operand images of the two-kernel tensor-core forward (K = V = 128)
+// per-chunk T and P images of the chunked tensor-core forward (K = V = 128)
 static size_t img_bytes(int B, int T, int HV, int K, int V) {
   if (K != 128 || V != 128) return 0;
   const size_t NT64 = (size_t)(T + 63) / 64;
@@ -145,11 +145,17 @@ const char* kda_last_error(void) { return g_err; }
 
 int kda_device_status(unsigned* flags) {
   if (!flags) return set_error(KDA_ERR_NULL, "kda_device_status: flags must be non-NULL");
-  unsigned f1 = 0, f2 = 0;
+  unsigned f1 = 0, f2 = 0, f3 = 0;
   int rc = take_device_error(&f1);
   if (!rc) rc = take_bwd_device_error(&f2);
-  *flags = f1 | f2;
+  if (!rc) rc = take_fwd_chunked_error(&f3);
+  *flags = f1 | f2 | f3;
   return rc;
+}
+
+int kda_set_wait_polls(unsigned polls) {
+  g_err[0] = 0;
+  return set_wait_polls(polls);
 }
 
 size_t kda_fwd_workspace_bytes(int B, int T, int HV, int K, int V) {

@@ -60,47 +60,22 @@ struct SeqChunks {
   }
 };
 
-// Output gate ("kimi_k3_host/kda.rs", full_rank_output_gate) on an O^T tile
-// read out of TMEM: warp w holds rows 32 (w / 4) + jj, jj < 32, of the value
-// columns 32 (w % 4) + lane.  Scales v[jj] by 1 / sqrt(mean_n o^2 + eps) of
-// its row (the sigmoid factor is the caller's); `red` is 256 floats that
-// nothing else touches until a later block barrier.  One block barrier
-// (256 threads).
-__device__ __forceinline__ void out_gate_rows(float (&v)[32], float* red, int warp, int lane, float eps) {
-  float sq[32];
-#pragma unroll
-  for (int jj = 0; jj < 32; ++jj) sq[jj] = v[jj] * v[jj];
-  const float part = tcc::warp_sum32(sq, lane);  // row 32 (warp / 4) + lane, this warp's 32 columns
-  red[((warp >> 2) * 32 + lane) * 4 + (warp & 3)] = part;
-  __syncthreads();
-#pragma unroll
-  for (int jj = 0; jj < 32; ++jj) {
-    const float4 r = *reinterpret_cast<const float4*>(red + ((warp >> 2) * 32 + jj) * 4);
-    v[jj] *= rsqrtf((r.x + r.y + r.z + r.w) * (1.f / 128.f) + eps);
-  }
-}
-
 // The state-independent part of one chunk: load, cumulative decay, the
 // interaction products and their read-out, the inverse T, the operands of the
 // state products (Q~ o e^c, (K o e^{c_last-c})^T in shared memory; e^{c_last}
 // per channel) and
 // W^T = (diag(beta) K o e^c)^T T^T, U0^T = (diag(beta) V)^T T^T in TMEM.  With
-// `irec` it stores the chunk's interaction record; with `img` it starts the
-// bulk stores of the chunk images of Q~ o e^c, (K o e^{c_last-c})^T and
-// e^{c_last} as soon as they are built.
+// `irec` it stores the chunk's interaction record.
 // The chunk covers steps t0 .. t0 + L - 1 of batch row b (packed sequences:
 // b = 0 and t0 on the packed axis); with Ln > 0 the next chunk of the same
 // sequence (Ln steps from t0 + 64) is prefetched into L2.
 // Returns false, block-uniformly, if a tensor-core wait ran out.
 // With PREP the fused input preparation runs on the loaded chunk (FwdArgs::prep):
-// q, k rows L2-normalised, g from z, beta from its logit.  With PRELOADED
-// the caller has already issued the chunk's raw loads (issue_chunk_loads).
-// With `img` the P image is bulk-stored as soon as it is read out (thread 32's
-// bulk group), so that the raw region it sits in is free again at the end.
-template <int NTHR, bool PREP = false, bool PRELOADED = false>
+// q, k rows L2-normalised, g from z, beta from its logit.
+template <int NTHR, bool PREP = false>
 __device__ __forceinline__ bool fwd_chunk_head(const tcc::Ctx& cx, const FwdArgs& a, int b, int hv, int h,
-                                               int t0, int L, int Ln, float* irec,
-                                               unsigned char* img, uint64_t* bar, uint32_t& phase) {
+                                               int t0, int L, int Ln, float* irec, uint64_t* bar,
+                                               uint32_t& phase) {
   using namespace tcf;
   using namespace tc;
   unsigned char* sm = cx.sm;
@@ -116,12 +91,12 @@ __device__ __forceinline__ bool fwd_chunk_head(const tcc::Ctx& cx, const FwdArgs
   const __nv_bfloat16* zg = static_cast<const __nv_bfloat16*>(a.prep.z);
   float dtb = 0.f, dec = 0.f;  // gate constants, loaded while the chunk's copies are in flight
   if constexpr (PREP) {
-    if (!PRELOADED) load_raw_issue_prep<NTHR>(cx, qg, kg, vg, zg, a.beta, b, T, t0, L, a.H, a.HV, h, hv);
+    load_raw_issue_prep<NTHR>(cx, qg, kg, vg, zg, a.beta, b, T, t0, L, a.H, a.HV, h, hv);
     dtb = a.prep.dt_bias[(size_t)hv * KD + (tid & 127)];
     dec = a.prep.A_log[hv];
     if (Ln > 0) prefetch_chunk(cx, qg, kg, vg, zg, b, T, t0 + C, Ln, a.H, a.HV, h, hv, 2);
   } else {
-    if (!PRELOADED) load_raw_issue<NTHR>(cx, qg, kg, vg, a.g, a.beta, b, T, t0, L, a.H, a.HV, h, hv);
+    load_raw_issue<NTHR>(cx, qg, kg, vg, a.g, a.beta, b, T, t0, L, a.H, a.HV, h, hv);
     if (Ln > 0) prefetch_chunk(cx, qg, kg, vg, a.g, b, T, t0 + C, Ln, a.H, a.HV, h, hv);
   }
   if (!load_raw_wait(cx)) return false;
@@ -131,10 +106,6 @@ __device__ __forceinline__ bool fwd_chunk_head(const tcc::Ctx& cx, const FwdArgs
     wide = cumsum_span<true, NTHR>(cx, dtb, expf(dec), a.prep.gate_lb, L);
   } else {
     wide = cumsum_span(cx);
-  }
-  if constexpr (PRELOADED) {  // the previous item's W and U0^T bulk stores have read the operand region
-    if ((tid & 31) == 0 && tid < 96) bulk_wait_read();
-    __syncthreads();
   }
   build_op1_and_issue<NTHR, PREP>(cx, a.scale, tm + TM_APA, tm + TM_APB, bar);
   if (!wait_mma(bar, phase)) return false;
@@ -177,14 +148,7 @@ __device__ __forceinline__ bool fwd_chunk_head(const tcc::Ctx& cx, const FwdArgs
   }
   Pairwise pw;
   if (wide) pairwise_compute<PREP>(cx, a.scale, pw);
-  if (img) fence_async_smem();
   __syncthreads();  // raw inputs consumed; the raw region is reused below
-  if (img && (tid & 31) == 0 && tid < 96) {  // one bulk store per issuing warp
-    if (tid == 0) bulk_s2g(img + FWI_QE, sb + OP_QE, FWI_KEDT - FWI_QE);
-    if (tid == 32) bulk_s2g(img + FWI_KEDT, sb + OP_KEDT, FWI_P - FWI_KEDT);
-    if (tid == 64) bulk_s2g(img + FWI_EL, sb + S_EL, FWI_U0 - FWI_EL);
-    bulk_commit();
-  }
 
   readout_ap<NTHR>(cx, tm + TM_APA, tm + TM_APB, wide, pw, nullptr);
   if (irec) {  // the P^T image of the record from the P image (16-byte pieces; piece x holds
@@ -197,14 +161,6 @@ __device__ __forceinline__ bool fwd_chunk_head(const tcc::Ctx& cx, const FwdArgs
       w.z = *reinterpret_cast<const uint32_t*>(sm + p_off(k + 2, r));
       w.w = *reinterpret_cast<const uint32_t*>(sm + p_off(k + 3, r));
       *reinterpret_cast<uint4*>(irec + x * 4) = w;
-    }
-  }
-  if (img) {  // P is final: store its image now (R_P is not touched again in this chunk)
-    fence_async_smem();
-    __syncthreads();
-    if (tid == 32) {
-      bulk_s2g(img + FWI_P, sb + R_P, FWI_EL - FWI_P);
-      bulk_commit();
     }
   }
   invert<NTHR>(cx);
@@ -300,7 +256,7 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_tc_kernel(FwdArgs a) {
     const int t0 = sp.x, L = sp.y, ch = c - sc.c0;
     const int Ln = c + 1 < sc.c1 ? sc.span(a, c + 1).y : 0;
     float* irec = a.inter ? a.inter + chunk_gc(a, sq, hv, c) * INTER_REC : nullptr;
-    if (!fwd_chunk_head<NTH, PREP>(cx, a, b, hv, h, t0, L, Ln, irec, nullptr, bar, phase)) {
+    if (!fwd_chunk_head<NTH, PREP>(cx, a, b, hv, h, t0, L, Ln, irec, bar, phase)) {
       failed = true;
       break;
     }
@@ -407,358 +363,9 @@ bool fwd_tc_eligible(const FwdArgs& a, int dtype) {
          al16(a.o) && al16(a.prep.z) && al16(a.og);
 }
 
-// ============================================================================
-// Two-kernel forward (with a chunk-image workspace).  The state-independent
-// work of every chunk runs first, all chunks in parallel
-// (kda_fwd_prep_tc_kernel, one CTA per (b, hv, chunk)), and leaves the chunk's
-// operands of the state products in the workspace as ready shared-memory
-// images; kda_fwd_seq_tc_kernel then carries the state through the chunks of
-// one (b, hv) with only the state products per chunk:
-//   X^T = M^T W^T,  O^T = M^T (Q~ o e^c)^T,  U^T = U0^T - X^T,
-//   M'^T = M^T diag(e^{c_last}) + U^T (K o e^{c_last-c}),  O^T += U^T P^T.
-// ============================================================================
-constexpr int PREP_NT = 512;  // 16 warps: the chunk work is latency-bound, more warps hide it
-
-template <bool PREP>
-__global__ void __launch_bounds__(PREP_NT, 1) kda_fwd_prep_tc_kernel(FwdArgs a) {
-  using namespace tcf;
-  using namespace tc;
-  extern __shared__ __align__(1024) unsigned char sm[];
-  Ctx cx;
-  cx.sm = sm;
-  cx.sb = smem_u32(sm);
-  cx.tid = threadIdx.x;
-  cx.warp = cx.tid >> 5;
-  cx.lane = cx.tid & 31;
-  cx.sub = cx.warp & 3;
-  cx.hcol = cx.warp >> 2;
-  cx.Lr = cx.sub * 32 + cx.lane;
-  cx.lo = (uint32_t)(cx.sub * 32) << 16;
-  const int tid = cx.tid, hcol = cx.hcol, Lr = cx.Lr;
-  const uint32_t lo = cx.lo, sb = cx.sb;
-  const int G = a.HV / a.H, NT = (a.T + C - 1) / C;
-  // item = (b * HV + hv) * NT + ch (uniform batches) or hv * NC + c (packed sequences);
-  // the item is also the index of the chunk's images
-  const int items = a.ctab ? a.NC * a.HV : NT * a.HV * a.B;
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + S_BAR);
-  uint32_t* sTm = reinterpret_cast<uint32_t*>(sm + S_TMEM);
-
-  if (cx.warp == 0) tmem_alloc(sTm, 512);
-  if (tid == 0) mbar_init(bar, 1);
-  fence_before();
-  __syncthreads();
-  fence_after();
-  const uint32_t tm = *sTm;
-  cx.tm = tm;
-  uint32_t phase = 0;
-  bool failed = false;
-  // persistent: this CTA takes items blockIdx.x, + gridDim.x, ...; the raw
-  // rows of the next item are requested as soon as the current item's
-  // products have consumed the raw region (its tail stages W and U0^T in the
-  // operand region instead), so their latency hides behind the tail.
-  const auto span_of = [&](int item, int& hv, int& b, int& t0, int& L) {
-    if (a.ctab) {
-      const int c = item % a.NC;
-      hv = item / a.NC;
-      b = 0;
-      t0 = a.ctab[2 * c];
-      L = a.ctab[2 * c + 1];
-    } else {
-      const int ch = item % NT;
-      hv = (item / NT) % a.HV;
-      b = item / (NT * a.HV);
-      t0 = ch * C;
-      L = min(C, a.T - t0);
-    }
-  };
-  const auto issue = [&](int item) {
-    int hv, b, t0, L;
-    span_of(item, hv, b, t0, L);
-    const __nv_bfloat16 *qg = static_cast<const __nv_bfloat16*>(a.q), *kg = static_cast<const __nv_bfloat16*>(a.k),
-                        *vg = static_cast<const __nv_bfloat16*>(a.v);
-    if constexpr (PREP)
-      load_raw_issue_prep<PREP_NT>(cx, qg, kg, vg, static_cast<const __nv_bfloat16*>(a.prep.z), a.beta, b, a.T, t0,
-                                   L, a.H, a.HV, hv / G, hv);
-    else
-      load_raw_issue<PREP_NT, true>(cx, qg, kg, vg, a.g, a.beta, b, a.T, t0, L, a.H, a.HV, hv / G, hv);
-  };
-  constexpr uint32_t ST_W = OP, ST_U0 = OP + (FWI_QE - FWI_W);  // tail staging of W and U0^T
-  static_assert(ST_U0 + (FWI_BYTES - FWI_U0) <= OP_QE + 32768, "staging stays inside the operand region");
-  if (blockIdx.x < items) issue(blockIdx.x);
-  for (int item = blockIdx.x; item < items; item += gridDim.x) {
-    int hv, b, t0, L;
-    span_of(item, hv, b, t0, L);
-    const int h = hv / G;
-    // (the previous item's W and U0^T leave the operand region while this
-    // item's raw rows are waited for and its decay is summed: fwd_chunk_head
-    // waits for them just before it builds its first operands)
-    float* irec = a.inter ? a.inter + (size_t)item * INTER_REC : nullptr;  // (item = chunk_gc)
-    unsigned char* img = a.img + (size_t)item * FWI_BYTES;
-    if (!fwd_chunk_head<PREP_NT, PREP, true>(cx, a, b, hv, h, t0, L, 0, irec, img, bar, phase)) {
-      failed = true;
-      break;
-    }
-    // the products have read the raw region (T image) and the operands; P, Q~ o e^c,
-    // (K o e^{c_last-c})^T and e^{c_last} must have left smem before the region is reused
-    if ((tid & 31) == 0 && tid < 96) bulk_wait_read();
-    __syncthreads();
-    if (item + (int)gridDim.x < items) issue(item + gridDim.x);
-    constexpr int CW = 64 / (PREP_NT / 128);  // columns of W^T / U0^T per warp group
-    {  // W (rows i, K = f) padded, from W^T in TMEM (lane f)
-      float v[CW];
-      tmem_ldn<CW>(tm + lo + TM_W + hcol * CW, v);
-#pragma unroll
-      for (int jj = 0; jj < CW; ++jj) st_tf32(sm, ST_W + kmaj_pad(hcol * CW + jj, Lr, 128), v[jj]);
-    }
-    {  // U0^T (lane n) as [i][n]
-      float u[CW];
-      tmem_ldn<CW>(tm + lo + TM_U + hcol * CW, u);
-      float* dst = reinterpret_cast<float*>(sm + ST_U0);
-#pragma unroll
-      for (int jj = 0; jj < CW; ++jj) dst[(hcol * CW + jj) * VD + Lr] = u[jj];
-    }
-    fence_async_smem();
-    fence_before();
-    __syncthreads();
-    if ((tid & 31) == 0 && tid < 96) {
-      if (tid == 0) bulk_s2g(img + FWI_W, sb + ST_W, FWI_QE - FWI_W);
-      if (tid == 64) bulk_s2g(img + FWI_U0, sb + ST_U0, FWI_BYTES - FWI_U0);
-      bulk_commit();
-    }
-  }
-  cp_async_wait_all();  // (a prefetch still in flight after an early exit)
-  if ((tid & 31) == 0 && tid < 96) bulk_wait_read();
-  fence_before();
-  __syncthreads();
-  if (cx.warp == 0) tmem_dealloc(tm, 512);
-  if (failed && tid == 0) atomicOr(&g_kda_device_error, 1u);
-}
-
-namespace tcs {
-// shared memory of the sequential pass: two buffers for the first group of a
-// chunk's images (W, Q~ o e^c), one for the second ((K o e^{c_last-c})^T, P,
-// e^{c_last}), the bf16 output tile [i][n], the output-gate tile [i][n] and
-// its row sums, then the barriers
-constexpr uint32_t SQ_A0 = 0, SQ_A1 = FWI_A_BYTES, SQ_B = 2 * FWI_A_BYTES, SQ_O = SQ_B + FWI_B_BYTES,
-                   SQ_G = SQ_O + 64 * 256, SQ_RED = SQ_G + 64 * 256, SQ_BAR = SQ_RED + 1024,
-                   SQ_TMEM = SQ_BAR + 32, SQ_BYTES = SQ_TMEM + 16;
-constexpr uint32_t B_KEDT = 0, B_P = FWI_P - FWI_KEDT, B_EL = FWI_EL - FWI_KEDT;
-static_assert(SQ_BYTES <= 232448 && SQ_O % 16 == 0, "shared memory budget");
-constexpr uint32_t TM_S = 0, TM_X = 128, TM_O = 192, TM_U = 256;
-}  // namespace tcs
-
-// one thread: arm `bar` for `bytes` and fetch them from global to shared memory
-__device__ __forceinline__ void fetch_images(uint32_t sdst, const unsigned char* src, uint32_t bytes, uint64_t* bar) {
-  tc::mbar_expect_tx(bar, bytes);
-  for (uint32_t off = 0; off < bytes; off += 32768)
-    tc::bulk_g2s(sdst + off, src + off, min(32768u, bytes - off), bar);
-}
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity) {
-  const bool ok = tc::mbar_wait(bar, parity);
-  return !__syncthreads_or(!ok);
-}
-
-__global__ void __launch_bounds__(256, 1) kda_fwd_seq_tc_kernel(FwdArgs a) {
-  using namespace tcs;
-  using namespace tc;
-  extern __shared__ __align__(1024) unsigned char sm[];
-  const uint32_t sb = smem_u32(sm);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, hcol = warp >> 2;
-  const int Lr = (warp & 3) * 32 + lane;
-  const uint32_t lo = (uint32_t)((warp & 3) * 32) << 16;
-  const int hv = blockIdx.x, sq = blockIdx.y;  // batch row, or sequence of a packed batch
-  const SeqChunks sc(a, sq);
-  const int b = sc.row, nch = sc.c1 - sc.c0;
-  const int T = a.T, NT = (T + tcc::C - 1) / tcc::C;
-  constexpr int C = tcc::C, KD = tcc::KD, VD = tcc::VD;
-  const size_t head = (size_t)sq * a.HV + hv;
-  // this sequence's chunk images, consecutive (the chunk kernel's item order)
-  const unsigned char* imgs = a.img + (a.ctab ? (size_t)hv * a.NC + sc.c0 : head * NT) * (size_t)FWI_BYTES;
-  __nv_bfloat16* og = static_cast<__nv_bfloat16*>(a.o);
-  uint64_t* barA = reinterpret_cast<uint64_t*>(sm + SQ_BAR);  // [2]
-  uint64_t* barB = barA + 2;
-  uint64_t* bar = barA + 3;  // tensor-core completion
-  uint32_t* sTm = reinterpret_cast<uint32_t*>(sm + SQ_TMEM);
-  const float* sEl = reinterpret_cast<const float*>(sm + SQ_B + B_EL);
-
-  if (warp == 0) tmem_alloc(sTm, 512);
-  if (tid == 0) {
-    mbar_init(barA, 1);
-    mbar_init(barA + 1, 1);
-    mbar_init(barB, 1);
-    mbar_init(bar, 1);
-  }
-  fence_before();
-  __syncthreads();
-  fence_after();
-  const uint32_t tm = *sTm;
-  if (tid == 0 && nch > 0) {
-    fetch_images(sb + SQ_A0, imgs, FWI_A_BYTES, barA);
-    fetch_images(sb + SQ_B, imgs + FWI_KEDT, FWI_B_BYTES, barB);
-  }
-  {  // entering state, transposed: lane n, column f
-    for (int cb = 0; cb < 2; ++cb) {
-      const int f0 = hcol * 64 + cb * 32;
-      uint32_t r[32];
-#pragma unroll
-      for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(a.S0 ? a.S0[(head * KD + f0 + j) * VD + Lr] : 0.f);
-      tmem_st32(tm + lo + TM_S + f0, r);
-    }
-    tmem_wait_st();
-  }
-  fence_before();
-  __syncthreads();
-  uint32_t phase = 0;
-  bool failed = false;
-
-  for (int ch = 0; ch < nch; ++ch) {
-    const int2 sp = sc.span(a, sc.c0 + ch);
-    const int t0 = sp.x, L = sp.y;
-    const unsigned char* img = imgs + (size_t)ch * FWI_BYTES;
-    const uint32_t bufA = (ch & 1) ? SQ_A1 : SQ_A0;
-    if (a.og && a.o) {  // this chunk's output-gate rows (bf16 [i][n]), completed before the epilogue
-      const __nv_bfloat16* gate = static_cast<const __nv_bfloat16*>(a.og);
-      for (int x = tid; x < C * 16; x += 256) {
-        const int i = x >> 4, c16 = x & 15;
-        cp_async16(sb + SQ_G + x * 16, gate + (((size_t)b * T + t0 + (i < L ? i : 0)) * a.HV + hv) * VD + c16 * 8,
-                   i < L);
-      }
-    }
-    if (tid == 32 && ch + 1 < nch) prefetch_l2(img + FWI_BYTES, FWI_BYTES);
-    float u0[32];
-    {
-      const float* src = reinterpret_cast<const float*>(img + FWI_U0);
-#pragma unroll
-      for (int jj = 0; jj < 32; ++jj) u0[jj] = src[(hcol * 32 + jj) * VD + Lr];
-    }
-    if (!wait_bar(barA + (ch & 1), (ch >> 1) & 1)) { failed = true; break; }
-    if (tid == 0) {  // X^T = M^T W^T ; O^T = M^T (Q~ o e^c)^T ; then the next chunk's first images
-      fence_after();
-      const uint32_t id = idesc_tf32(128, 64);
-      for (int ks = 0; ks < 16; ++ks) {
-        mma_ts(tm + TM_X, tm + TM_S + ks * 8, desc(sb + bufA + FWI_W + ks * 288, 4608, 144), id, ks > 0);
-        mma_ts(tm + TM_O, tm + TM_S + ks * 8, desc(sb + bufA + FWI_QE + ks * 256, 4096), id, ks > 0);
-      }
-      commit(bar);
-      if (ch + 1 < nch) fetch_images(sb + ((ch & 1) ? SQ_A0 : SQ_A1), img + FWI_BYTES, FWI_A_BYTES, barA + ((ch + 1) & 1));
-    }
-    if (!tcc::wait_mma(bar, phase)) { failed = true; break; }
-    {  // U^T = U0^T - X^T
-      float x[32];
-      uint32_t r[32];
-      tmem_ld32(tm + lo + TM_X + hcol * 32, x);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) r[j] = tf32_rna(u0[j] - x[j]);
-      tmem_st32(tm + lo + TM_U + hcol * 32, r);
-    }
-    if (!wait_bar(barB, ch & 1)) { failed = true; break; }
-    float sv[2][32];  // the entering state (this thread's lane, 64 channels), stored for the
-                      // backward once the state products are under way
-    {  // M^T <- M^T diag(e^{c_last})
-      uint32_t r[32];
-#pragma unroll
-      for (int cb = 0; cb < 2; ++cb) {
-        const int f0 = hcol * 64 + cb * 32;
-        tmem_ld32(tm + lo + TM_S + f0, sv[cb]);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(sv[cb][j] * sEl[f0 + j]);
-        tmem_st32(tm + lo + TM_S + f0, r);
-      }
-      tmem_wait_st();
-    }
-    const bool gated = a.og && a.o;
-    if (gated) cp_async_wait_all();  // this thread's pieces of the gate tile; the barrier publishes them
-    fence_before();
-    __syncthreads();
-    if (tid == 0) {  // M^T += U^T (K o e^{c_last-c}) ; O^T += U^T P^T
-      fence_after();
-      const uint32_t idS = idesc_tf32(128, 128), idO = idesc_tf32(128, 64);
-      for (int ks = 0; ks < 8; ++ks) {
-        mma_ts(tm + TM_S, tm + TM_U + ks * 8, desc(sb + SQ_B + B_KEDT + ks * 256, 2048), idS, 1);
-        mma_ts(tm + TM_O, tm + TM_U + ks * 8, desc(sb + SQ_B + B_P + ks * 256, 2048), idO, 1);
-      }
-      commit(bar);
-    }
-    if (a.states) {  // (off the critical path: the products above do not wait for these stores)
-      float* dst = a.states + (state_slot(a, sq, hv, sc.c0 + ch) * KD + hcol * 64) * VD + Lr;
-#pragma unroll
-      for (int cb = 0; cb < 2; ++cb)
-#pragma unroll
-        for (int j = 0; j < 32; ++j) dst[(size_t)(cb * 32 + j) * VD] = sv[cb][j];
-    }
-    float sig[32];  // sigmoid of the output gate, formed while the products run
-    if (gated) {
-      const __nv_bfloat16* sg = reinterpret_cast<const __nv_bfloat16*>(sm + SQ_G);
-#pragma unroll
-      for (int jj = 0; jj < 32; ++jj) sig[jj] = prep_sigmoid_fast(__bfloat162float(sg[(hcol * 32 + jj) * VD + Lr]));
-    }
-    if (!tcc::wait_mma(bar, phase)) { failed = true; break; }
-    if (tid == 0 && ch + 1 < nch) {  // the lanes' reads of e^{c_last} precede the overwrite
-      fence_async_smem();
-      fetch_images(sb + SQ_B, img + FWI_BYTES + FWI_KEDT, FWI_B_BYTES, barB);
-    }
-    if (a.o) {  // O^T (lane n) -> bf16 tile [i][n] -> 16-byte row pieces
-      __nv_bfloat16* so = reinterpret_cast<__nv_bfloat16*>(sm + SQ_O);
-      float v[32];
-      tmem_ld32(tm + lo + TM_O + hcol * 32, v);
-      if (gated) {  // output gate
-        out_gate_rows(v, reinterpret_cast<float*>(sm + SQ_RED), warp, lane, a.og_eps);
-#pragma unroll
-        for (int jj = 0; jj < 32; ++jj) v[jj] *= sig[jj];
-      }
-#pragma unroll
-      for (int jj = 0; jj < 32; ++jj) so[(hcol * 32 + jj) * VD + Lr] = __float2bfloat16_rn(v[jj]);
-      __syncthreads();
-#pragma unroll
-      for (int x = tid; x < C * 16; x += 256) {
-        const int i = x >> 4, c16 = x & 15;
-        if (i < L)
-          *reinterpret_cast<uint4*>(og + (((size_t)b * T + t0 + i) * a.HV + hv) * VD + c16 * 8) =
-              *reinterpret_cast<const uint4*>(sm + SQ_O + i * 256 + c16 * 16);
-      }
-    }
-    fence_before();
-    __syncthreads();
-  }
-
-  if (!failed && a.S_T) {
-    fence_after();
-    for (int cb = 0; cb < 2; ++cb) {
-      const int f0 = hcol * 64 + cb * 32;
-      float s[32];
-      tmem_ld32(tm + lo + TM_S + f0, s);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) a.S_T[(head * KD + f0 + j) * VD + Lr] = s[j];
-    }
-  }
-  fence_before();
-  __syncthreads();
-  if (warp == 0) tmem_dealloc(tm, 512);
-  if (failed && tid == 0) atomicOr(&g_kda_device_error, 1u);
-}
-
 template <bool PREP>
 static int launch_fwd_tc_t(const FwdArgs& a, cudaStream_t stream) {
-  if (a.img) {  // two-kernel forward
-    cudaError_t e = cudaFuncSetAttribute(kda_fwd_prep_tc_kernel<PREP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)tcc::SMEM_BYTES);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(kda_fwd_seq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)tcs::SQ_BYTES);
-    if (e != cudaSuccess) return set_cuda_error("kda_fwd: cudaFuncSetAttribute", e);
-    const int items = a.ctab ? a.NC * a.HV : (a.T + tcc::C - 1) / tcc::C * a.HV * a.B;
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (items > 0) {  // (packed batches of empty sequences have no chunks)
-      kda_fwd_prep_tc_kernel<PREP><<<min(items, sms), PREP_NT, tcc::SMEM_BYTES, stream>>>(a);
-      e = cudaGetLastError();
-      if (e != cudaSuccess) return set_cuda_error("kda_fwd: tensor-core chunk launch", e);
-    }
-    kda_fwd_seq_tc_kernel<<<dim3(a.HV, a.B), tcc::NTH, tcs::SQ_BYTES, stream>>>(a);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return set_cuda_error("kda_fwd: tensor-core state-pass launch", e);
-    return 0;
-  }
+  if (a.img) return launch_fwd_chunked(a, stream);  // chunk-parallel kernel + state pass
   cudaError_t e = cudaFuncSetAttribute(kda_fwd_tc_kernel<PREP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)tcc::SMEM_BYTES);
   if (e != cudaSuccess) return set_cuda_error("kda_fwd: cudaFuncSetAttribute", e);

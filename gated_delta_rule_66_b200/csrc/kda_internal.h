@@ -25,19 +25,11 @@ constexpr int FWD_VBLOCK = 32;   // V columns per CTA in the chunked kernels
 // and Ah row-major at INTER_AH.  The backward reads it instead of recomputing
 // the interaction products and the inverse.
 constexpr int INTER_T = 4096, INTER_AH = 8192, INTER_TT = 12288, INTER_REC = 16384;
-// Per-(b, hv, 64-step chunk) operand images of the two-kernel tensor-core
-// forward (bytes): everything the sequential state pass needs from a chunk,
-// laid out as its shared-memory operands so that it fetches them with two
-// bulk copies (W and Q~ o e^c; the rest) plus U0^T read by the lanes.
-//   FWI_W     W (rows i, K = f), padded K-major (LBO 144)     36864
-//   FWI_QE    Q~ o e^c (rows i, K = f)                        32768
-//   FWI_KEDT  (K o e^{c_last - c})^T (rows f, K = i)          32768
-//   FWI_P     P (rows i, K = j)                               16384
-//   FWI_EL    e^{c_last} [128]                                  512
-//   FWI_U0    U0^T = (T diag(beta) V)^T as [i][n] fp32        32768
-constexpr unsigned FWI_W = 0, FWI_QE = 36864, FWI_KEDT = 69632, FWI_P = 102400, FWI_EL = 118784,
-                   FWI_U0 = 119296, FWI_BYTES = 152064;
-constexpr unsigned FWI_A_BYTES = FWI_KEDT, FWI_B_BYTES = FWI_U0 - FWI_KEDT;
+// Per-(b, hv, 64-step chunk) record of the chunked tensor-core forward
+// (bytes): the T and P operand images that the chunk-parallel kernel leaves
+// for the state pass (64 x 64 tf32 each, K-major canonical layout,
+// (r, k) = T[r][k] and P[r][k]).
+constexpr unsigned FWR_T = 0, FWR_P = 16384, FWI_BYTES = 32768;
 constexpr int G_AH = 0, G_PA = 4096, G_QK = 12288, G_KED = 28672, G_DBR = 36864, G_DEL = 36928,
               GREC = 37120;
 
@@ -196,6 +188,12 @@ size_t fma_split_bytes(int B, int T, int HQ, int HV, int K, int V);
 bool fma_kda_split(int K, int V);
 int launch_fwd_fma2(const FwdArgs& a, int dtype, bool erase, float* prep, cudaStream_t stream);
 int launch_fwd_tc(const FwdArgs& a, cudaStream_t stream);
+// the chunked tensor-core forward (a.img: FWI_BYTES per chunk): chunk-parallel
+// interaction and inverse, then the state pass
+int launch_fwd_chunked(const FwdArgs& a, cudaStream_t stream);
+int take_fwd_chunked_error(unsigned* out);
+// probes of every bounded wait in the chunked forward (0: the default)
+int set_wait_polls(unsigned polls);
 int take_device_error(unsigned* out);
 int take_bwd_device_error(unsigned* out);
 int launch_bwd(const BwdArgs& a, int dtype, cudaStream_t stream);

@@ -210,6 +210,34 @@ __device__ __forceinline__ float warp_sum32(float (&v)[32], int lane) {
 // float index of element (r, k) in a 64 x 64 record image
 __device__ __forceinline__ int img(int r, int k) { return (int)(tc::kmaj(r, k, 64) >> 2); }
 
+// Output gate ("kimi_k3_host/kda.rs", full_rank_output_gate) on an O^T tile
+// read out of TMEM: warp w holds rows 32 (w / 4) + jj, jj < 32, of the value
+// columns 32 (w % 4) + lane.  Scales v[jj] by 1 / sqrt(mean_n o^2 + eps) of
+// its row (the sigmoid factor is the caller's); `red` is 256 floats that
+// nothing else touches until a later block barrier.  One block barrier
+// (256 threads).
+// (sync: the barrier of the 256 threads taking part)
+template <class Sync>
+__device__ __forceinline__ void out_gate_rows(float (&v)[32], float* red, int warp, int lane, float eps, Sync sync) {
+  float sq[32];
+#pragma unroll
+  for (int jj = 0; jj < 32; ++jj) sq[jj] = v[jj] * v[jj];
+  const float part = warp_sum32(sq, lane);  // row 32 (warp / 4) + lane, this warp's 32 columns
+  red[((warp >> 2) * 32 + lane) * 4 + (warp & 3)] = part;
+  sync();
+#pragma unroll
+  for (int jj = 0; jj < 32; ++jj) {
+    const float4 r = *reinterpret_cast<const float4*>(red + ((warp >> 2) * 32 + jj) * 4);
+    v[jj] *= rsqrtf((r.x + r.y + r.z + r.w) * (1.f / 128.f) + eps);
+  }
+}
+__device__ __forceinline__ void out_gate_rows(float (&v)[32], float* red, int warp, int lane, float eps) {
+  struct All {
+    __device__ void operator()() const { __syncthreads(); }
+  };
+  out_gate_rows(v, red, warp, lane, eps, All());
+}
+
 // In-chunk cumulative decay (natural log summed, stored times log2(e)).
 // Returns, block-uniformly, whether some half's decay from its middle row to
 // either end exceeds 80 (the split exponents would then leave fp32 range).
@@ -380,14 +408,15 @@ __device__ __forceinline__ void pairwise_compute(const Ctx& c, float scale, Pair
 }
 
 // byte offset of P[i][j] in its operand tile (rows i, K = j)
-__device__ __forceinline__ uint32_t p_off(int i, int j) { return R_P + tc::kmaj(i, j, 64); }
+__device__ __forceinline__ uint32_t p_off(int i, int j, uint32_t base = R_P) { return base + tc::kmaj(i, j, 64); }
 
 // Reads Ah (row-major, stride 65, at R_AH) and P (tf32 operand at R_P) out of
 // the two interaction products; the raw region must be free.  With `pt` it
 // also stores the P^T image of the interaction record.  Ends with a barrier.
+// (p_base: shared-memory byte offset of the P image, R_P by default)
 template <int NT = NTH>
 __device__ __forceinline__ void readout_ap(const Ctx& c, uint32_t tm_apa, uint32_t tm_apb, bool wide,
-                                           const Pairwise& pw, float* pt = nullptr) {
+                                           const Pairwise& pw, float* pt = nullptr, uint32_t p_base = R_P) {
   using namespace tc;
   constexpr int CW = 64 / (NT / 128), CB = 32 / (NT / 128);  // columns per warp group of [Ah; P], of b
   float* sAh = reinterpret_cast<float*>(c.sm + R_AH);
@@ -416,7 +445,7 @@ __device__ __forceinline__ void readout_ap(const Ctx& c, uint32_t tm_apa, uint32
           w[u] = ((i >> 5) == (j >> 5) && j <= i) ? v[j4 + u] : 0.f;
           if (pt) pt[img(j, i)] = __uint_as_float(tf32_rna(w[u]));
         }
-        st_tf32x4(c.sm, p_off(i, jb), w[0], w[1], w[2], w[3]);
+        st_tf32x4(c.sm, p_off(i, jb, p_base), w[0], w[1], w[2], w[3]);
       }
     }
   }
@@ -432,7 +461,7 @@ __device__ __forceinline__ void readout_ap(const Ctx& c, uint32_t tm_apa, uint32
 #pragma unroll
         for (int j4 = 0; j4 < CB; j4 += 4) {
           const int j = c.hcol * CB + j4;
-          st_tf32x4(c.sm, p_off(r, j), v[j4], v[j4 + 1], v[j4 + 2], v[j4 + 3]);
+          st_tf32x4(c.sm, p_off(r, j, p_base), v[j4], v[j4 + 1], v[j4 + 2], v[j4 + 3]);
           if (pt)
 #pragma unroll
             for (int u = 0; u < 4; ++u) pt[img(j + u, r)] = __uint_as_float(tf32_rna(v[j4 + u]));
@@ -446,7 +475,7 @@ __device__ __forceinline__ void readout_ap(const Ctx& c, uint32_t tm_apa, uint32
       const int j = pw.j0 + jj;
       if (pw.kind == 0 && j < pw.i) sAh[pw.i * 65 + j] = pw.v[jj];
       if (pw.kind == 1 && j <= pw.i) {
-        st_tf32(c.sm, p_off(pw.i, j), pw.v[jj]);
+        st_tf32(c.sm, p_off(pw.i, j, p_base), pw.v[jj]);
         if (pt) pt[img(j, pw.i)] = __uint_as_float(tf32_rna(pw.v[jj]));
       }
     }
@@ -463,13 +492,14 @@ __device__ __forceinline__ void readout_ap(const Ctx& c, uint32_t tm_apa, uint32
 // operand anyway; with single products here the o error stays ~0.5e-3 above
 // the bf16 rounding floor, and hi/lo-split products cost 0.06 ms more per
 // forward on the fwd+bwd workload.)
+// (beta: the chunk's 64 beta values in shared memory, c.beta() by default)
 template <int NT = NTH>
-__device__ __forceinline__ void invert(const Ctx& c) {
+__device__ __forceinline__ void invert(const Ctx& c, const float* beta = nullptr) {
   constexpr int LD = 65;
   const float* sAh = reinterpret_cast<const float*>(c.sm + R_AH);
   float* sT = reinterpret_cast<float*>(c.sm + R_TROW);
   float* sW = reinterpret_cast<float*>(c.sm + R_SW);  // one 16 x 16 scratch per warp (3 warps)
-  const float* sB = c.beta();
+  const float* sB = beta ? beta : c.beta();
   const int tid = c.tid;
   for (int x = tid; x < 6 * 256; x += NT) {  // strictly upper blocks
     const int blk = x >> 8, r = (x >> 4) & 15, col = x & 15;

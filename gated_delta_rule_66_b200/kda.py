@@ -26,7 +26,7 @@ SYMBOLS = ("kda_last_error", "kda_device_status", "kda_fwd_workspace_bytes", "kd
            "kda_bwd_workspace_bytes", "kda_fwd", "kda_fwd_varlen_workspace_bytes", "kda_fwd_varlen",
            "kda_bwd_varlen_workspace_bytes", "kda_bwd_varlen", "kda_decode_step", "kda_bwd",
            "kda_fwd_prep_workspace_bytes", "kda_fwd_prep", "kda_short_conv", "kda_decode_token",
-           "kda_fwd_erase", "kda_fwd_erase_workspace_bytes")
+           "kda_fwd_erase", "kda_fwd_erase_workspace_bytes", "kda_set_wait_polls")
 
 
 class KdaError(RuntimeError):
@@ -48,6 +48,8 @@ def _load():
     lib.kda_last_error.argtypes = []
     lib.kda_device_status.restype = i
     lib.kda_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint)]
+    lib.kda_set_wait_polls.restype = i
+    lib.kda_set_wait_polls.argtypes = [ctypes.c_uint]
     lib.kda_fwd_workspace_bytes.restype = sz
     lib.kda_fwd_workspace_bytes.argtypes = [i, i, i, i, i]
     lib.kda_fwd_scratch_bytes.restype = sz
@@ -141,6 +143,14 @@ def device_status():
     flags = ctypes.c_uint(0)
     _check("kda_device_status", _lib.kda_device_status(ctypes.byref(flags)))
     return int(flags.value)
+
+
+def set_wait_polls(polls):
+    """Test hook: probes of every bounded wait of the chunked tensor-core
+    forward on the current device (0 restores the default).  A kernel whose
+    wait runs out drains its own issued work, frees its tensor memory and sets
+    bit 0 of device_status()."""
+    _check("kda_set_wait_polls", _lib.kda_set_wait_polls(int(polls)))
 
 
 def workspace_bytes(kind, B, T, H, HV, K, V):

@@ -78,9 +78,23 @@ const char* kda_last_error(void);
 /* Reads and clears the device-side error bits of the library's kernels on the
  * current device, synchronising it first.  Bit 0: a tensor-core kernel gave
  * up waiting for its own tensor-core work (a bounded wait ran out) and
- * skipped the rest of its launch; its outputs are then undefined.  Returns
+ * skipped the rest of its launch; its outputs are then undefined.  Bit 1: a
+ * kernel of the chunked tensor-core forward found its shared memory not
+ * 1024-byte aligned (its TMA tiles need it) and skipped its launch.  Returns
  * KDA_OK or KDA_ERR_CUDA; *flags receives the bits (0 = none). */
 int kda_device_status(unsigned* flags);
+
+/* Test hook for the failure path of the bounded waits.  Every wait of the
+ * chunked tensor-core forward (the two kernels that kda_fwd, kda_fwd_varlen
+ * and kda_fwd_prep run when given their workspace) probes its mbarrier at
+ * most `polls` times (0 restores the default, 2^24) before it gives up.  A
+ * kernel that gives up first waits, under the default bound, for every copy
+ * and tensor-core product it has already issued, then frees its tensor
+ * memory, sets bit 0 of kda_device_status() and returns; its outputs are
+ * undefined.  With polls = 1 the first wait of each such kernel gives up.
+ * The value is per device (the current one) and persists until changed.
+ * Returns KDA_OK or KDA_ERR_CUDA. */
+int kda_set_wait_polls(unsigned polls);
 
 /* Bytes of the training workspace of kda_fwd: the fp32 state entering every
  * 32 steps [B, HV, ceil(T / 32), K, V], then (K = V = 128) the per-64-step
@@ -91,7 +105,9 @@ size_t kda_fwd_workspace_bytes(int B, int T, int HV, int K, int V);
 /* Bytes of the optional scratch that lets kda_fwd run as two kernels: a
  * chunk-parallel pass that leaves every chunk's operands of the state
  * products there, then the sequential state pass.  On the tensor-core path
- * (K = V = 128, bf16) the chunk images take 152,064 bytes per 64-step chunk;
+ * (K = V = 128, bf16) the chunk-parallel pass leaves the T and P operand
+ * images (32,768 bytes per 64-step chunk) and the state pass rebuilds the
+ * other operands from the inputs;
  * on the CUDA-core path (fp32 inputs, or other K and V) the chunk records take
  * 4 (2 C^2 + 3 C K + K) bytes per 32-step chunk (C = 32); for K = V = 128 the
  * larger of the two, as the dtype is not an argument.  For other K and V the

@@ -127,15 +127,15 @@ def test_last_error_clears_on_next_call(lib):
 
 def test_tensor_core_workspace_sizes(lib):
     """K = V = 128: the training forward keeps the 32-step states, a 64 KB
-    interaction record and the 149 KB chunk images per 64-step chunk; the
-    backward overwrites the images with its own buffers; the scratch-only
-    forward needs the images alone."""
+    interaction record and the scratch per 64-step chunk; the scratch holds the
+    32 KB T and P images of the tensor-core path or the CUDA-core path's
+    records (fp32 inputs), whichever is larger, since the dtype is not an
+    argument; the backward overwrites it with its own buffers."""
     B, T, H, HV, K, V = 1, 130, 1, 2, 128, 128
     nt32, nt64 = (T + 31) // 32, (T + 63) // 64
     states = B * HV * nt32 * K * V * 4
     inter = B * HV * nt64 * 16384 * 4
-    img = B * HV * nt64 * 152064  # (larger than the CUDA-core records of the same shape)
-    assert img >= B * HV * nt32 * fma_rec_bytes(K)
+    img = max(B * HV * nt64 * 32768, B * HV * nt32 * fma_rec_bytes(K))
     assert lib.kda_fwd_scratch_bytes(B, T, HV, K, V) == img
     assert lib.kda_fwd_workspace_bytes(B, T, HV, K, V) == states + inter + img
     tail = states + 2 * B * T * HV * K * 4 + B * HV * nt64 * 37120 * 4  # state grads, dq/dk partials, records
@@ -153,7 +153,7 @@ def test_varlen_workspace_and_validation(lib):
     HV = 3
     cu = _cu([0, 5, 5, 200])  # sequences of 5, 0 and 195 steps: 1 + 0 + 4 chunks
     table = ((2 * 5 + 4) * 4 + 255) // 256 * 256
-    assert lib.kda_fwd_varlen_workspace_bytes(cu, 3, HV, 128, 128) == table + 5 * HV * 152064
+    assert lib.kda_fwd_varlen_workspace_bytes(cu, 3, HV, 128, 128) == table + 5 * HV * 32768
     assert lib.kda_fwd_varlen_workspace_bytes(_cu([1, 5]), 1, HV, 128, 128) == 0      # must start at 0
     assert lib.kda_fwd_varlen_workspace_bytes(_cu([0, 9, 5]), 2, HV, 128, 128) == 0   # decreasing
     assert lib.kda_fwd_varlen_workspace_bytes(cu, 3, HV, 64, 64) == 0                 # tensor-core shapes only
@@ -168,8 +168,8 @@ def test_varlen_workspace_and_validation(lib):
 
 def test_prep_workspace_and_validation(lib):
     B, T, H, HV = 2, 100, 1, 2
-    # tensor-core shape: the chunk images; a CUDA-core bf16 shape: the fp32 output for the gate pass
-    assert lib.kda_fwd_prep_workspace_bytes(B, T, H, HV, 128, 128, 1) == B * HV * 2 * 152064
+    # tensor-core shape: the T and P images; a CUDA-core bf16 shape: the fp32 output for the gate pass
+    assert lib.kda_fwd_prep_workspace_bytes(B, T, H, HV, 128, 128, 1) == B * HV * 2 * 32768
     assert lib.kda_fwd_prep_workspace_bytes(B, T, H, HV, 64, 32, 1) == B * T * HV * 32 * 4
     assert lib.kda_fwd_prep_workspace_bytes(B, T, H, HV, 64, 32, 0) == 0
     assert lib.kda_fwd_prep_workspace_bytes(B, T, 2, 3, 64, 32, 0) == 0  # HV % H != 0

@@ -123,6 +123,30 @@ def test_fwd_tc_training_workspace_same_output(kda):
     assert torch.equal(o1, o2) and torch.equal(S1, S2)
 
 
+def test_bounded_wait_gives_up_then_recovers(kda):
+    """The failure path of the bounded waits, without any fault: with one
+    probe per wait the chunked forward's kernels give up at their first wait
+    (the copy they just issued cannot have landed), drain the copies and
+    products they issued, free their tensor memory and report bit 0; after
+    the default is restored the same call on the same context matches the
+    oracle."""
+    w = BY_NAME["prefill_gqa"].with_sizes(T=130, H=1, HV=2)
+    inp = make_inputs(w)
+    d = to_cuda(inp)
+    assert kda.device_status() == 0
+    kda.set_wait_polls(1)
+    try:
+        kda.fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], scale=w.scale, initial_state=d["S0"])
+        torch.cuda.synchronize()
+        flags = kda.device_status()
+    finally:
+        kda.set_wait_polls(0)
+    assert flags & 1, f"no kernel reported giving up (flags {flags})"
+    assert not flags & 2
+    check_fwd(kda, inp, w.scale, w.torch_dtype, "after_give_up")
+    assert kda.device_status() == 0
+
+
 def test_fwd_strong_unbounded_decay(kda):
     """Very strong decays (|g| up to 40 per step) take the pair-by-pair path
     for diagonal blocks; results stay finite and match."""
