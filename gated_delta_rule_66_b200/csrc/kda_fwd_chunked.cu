@@ -509,8 +509,11 @@ __global__ void __launch_bounds__(NTH, 2) kda_fwd_intra_tc_kernel(const __grid_c
 // tcgen05.commit.  A wait that gives up sets the shared abort word, which
 // ends the other roles' waits too.
 //
-// Shared memory (bytes): raw q, k, g / decay, v tiles (TMA; the v tile also
-// stages the previous chunk's bf16 output for its TMA store); the
+// Per chunk the products run in the order [Y^T | O^T] (m1), the previous
+// chunk's O^T += U^T P^T (m4, deferred so that it is off the state's path),
+// U^T (m2), M^T += U^T (K o e^{c_last-c}) (m3).
+//
+// Shared memory (bytes): raw q, k, g / decay, v tiles (TMA); the
 // [K o e^c ; Q~ o e^c] operand (rows 0..63 and 64..127, K = key channel,
 // K extent 128); (K o e^{c_last - c})^T (rows = key channel, K = step,
 // extent 64); the T diag(beta) and P images; then e^{c_last}, the output gate's row sums, the row factors, the
@@ -526,7 +529,7 @@ constexpr int K2_THREADS = 544, CH0 = 32, CH_THREADS = 256, BU0 = 288, BU_THREAD
 // U^T
 constexpr uint32_t TM_S = 0, TM_D0 = 128, TM_U = 384;
 // barriers: async copies and products (counted in S2_CNT for the drain), then the roles' arrivals
-enum { B_RAW, B_V, B_T, B_P, B_M1, B_M2, B_M3, NB_ASYNC, B_KQ = NB_ASYNC, B_KD, B_Z, B_O, B_UR, NB_ALL };
+enum { B_RAW, B_V, B_T, B_P, B_M1, B_M2, B_M3, B_M4, NB_ASYNC, B_KQ = NB_ASYNC, B_KD, B_Z, B_O, B_UR, NB_ALL };
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(tc::smem_u32(bar)) : "memory");
@@ -612,6 +615,24 @@ __global__ void __launch_bounds__(K2_THREADS, 1) kda_fwd_state_tc_kernel(const _
         commit(bars + which);
         ++cnt[which];
       };
+      const auto o_part = [&](int ch) {  // O^T += U^T P^T of chunk ch
+        for (int ks = 0; ks < 8; ++ks)
+          mma_ts(tm + TM_D0 + (ch & 1) * 128 + 64, tm + TM_U + ks * 8, desc(sb + S2_P + ks * 256, 2048),
+                 idesc_tf32(128, 64), 1);
+        commit_to(B_M4);
+      };
+      // the output rows of chunk ch, staged over the T slot, leave by TMA store
+      const auto store_o = [&](int ch) {
+        if (!wait_one(bars + B_O, ch & 1, polls, abort)) return false;
+        if (a.o && tma_out(ch)) {
+          const int t0 = span(ch).x;
+          tma_store_4d(&maps.o, 0, hv, t0, b, sb + S2_T);
+          tma_store_4d(&maps.o, 64, hv, t0, b, sb + S2_T + 8192);
+          bulk_commit();
+          bulk_wait_read();
+        }
+        return true;
+      };
       issue_v(0);
       issue_img(B_T, sb + S2_T, 0, FWR_T);
       issue_img(B_P, sb + S2_P, 0, FWR_P);
@@ -624,7 +645,10 @@ __global__ void __launch_bounds__(K2_THREADS, 1) kda_fwd_state_tc_kernel(const _
         for (int ks = 0; ks < 16; ++ks)
           mma_ts(tm + D, tm + TM_S + ks * 8, desc(sb + S2_KQ + ks * 256, 4096), idesc_tf32(128, 128), ks > 0);
         commit_to(B_M1);
-        if (ch > 0) issue_img(B_P, sb + S2_P, ch, FWR_P);  // the previous chunk's P is consumed
+        if (ch > 0) {  // (U^T and P of the previous chunk are still resident)
+          if (!wait_one(bars + B_P, par ^ 1, polls, abort)) break;
+          o_part(ch - 1);
+        }
         // U^T = Z^T (T diag(beta))^T
         if (!wait_one(bars + B_Z, par, polls, abort)) break;
         if (!wait_one(bars + B_T, par, polls, abort)) break;
@@ -632,37 +656,27 @@ __global__ void __launch_bounds__(K2_THREADS, 1) kda_fwd_state_tc_kernel(const _
         for (int ks = 0; ks < 8; ++ks)
           mma_ts(tm + TM_U, tm + D + ks * 8, desc(sb + S2_T + ks * 256, 2048), idesc_tf32(128, 64), ks > 0);
         commit_to(B_M2);
-        // the previous chunk's output (staged over v) leaves; then the next chunk's v comes in
-        if (ch > 0 && a.o && tma_out(ch - 1)) {
-          if (!wait_one(bars + B_O, (ch - 1) & 1, polls, abort)) break;
-          const int t0 = span(ch - 1).x;
-          tma_store_4d(&maps.o, 0, hv, t0, b, sb + S2_V);
-          tma_store_4d(&maps.o, 64, hv, t0, b, sb + S2_V + 8192);
-          bulk_commit();
-          bulk_wait_read();
-        } else if (ch > 0 && a.o) {
-          if (!wait_one(bars + B_O, (ch - 1) & 1, polls, abort)) break;
+        if (ch + 1 < nch) issue_v(ch + 1);  // this chunk's v is consumed
+        if (ch > 0) {  // the previous chunk's P is consumed once its output products are done
+          if (!wait_one(bars + B_M4, par ^ 1, polls, abort)) break;
+          issue_img(B_P, sb + S2_P, ch, FWR_P);
         }
-        if (ch + 1 < nch) issue_v(ch + 1);
-        if (!wait_one(bars + B_M2, par, polls, abort)) break;
-        if (ch + 1 < nch) issue_img(B_T, sb + S2_T, ch + 1, FWR_T);  // this chunk's T is consumed
-        // M^T += U^T (K o e^{c_last-c}), O^T += U^T P^T once U^T is rounded and the state decayed
+        // M^T += U^T (K o e^{c_last-c}) once U^T is rounded and the state decayed
         if (!wait_one(bars + B_UR, par, polls, abort)) break;
         if (!wait_one(bars + B_KD, par, polls, abort)) break;
-        if (!wait_one(bars + B_P, par, polls, abort)) break;
         fence_after();
-        for (int ks = 0; ks < 8; ++ks) {
+        for (int ks = 0; ks < 8; ++ks)
           mma_ts(tm + TM_S, tm + TM_U + ks * 8, desc(sb + S2_KD + ks * 256, 2048), idesc_tf32(128, 128), 1);
-          mma_ts(tm + D + 64, tm + TM_U + ks * 8, desc(sb + S2_P + ks * 256, 2048), idesc_tf32(128, 64), 1);
-        }
         commit_to(B_M3);
+        // the previous chunk's output (staged over T, free since m2) leaves; then the next T
+        if (ch > 0 && !store_o(ch - 1)) break;
+        if (ch + 1 < nch) issue_img(B_T, sb + S2_T, ch + 1, FWR_T);
       }
-      if (!*abort && a.o && tma_out(nch - 1)) {  // the last chunk's output
-        if (wait_one(bars + B_O, (nch - 1) & 1, polls, abort)) {
-          const int t0 = span(nch - 1).x;
-          tma_store_4d(&maps.o, 0, hv, t0, b, sb + S2_V);
-          tma_store_4d(&maps.o, 64, hv, t0, b, sb + S2_V + 8192);
-          bulk_commit();
+      if (!*abort) {  // the last chunk's output products and rows
+        if (wait_one(bars + B_P, (nch - 1) & 1, polls, abort)) {
+          fence_after();
+          o_part(nch - 1);
+          store_o(nch - 1);
         }
       }
       asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
@@ -695,7 +709,7 @@ __global__ void __launch_bounds__(K2_THREADS, 1) kda_fwd_state_tc_kernel(const _
       if (tma_out(ch)) {
 #pragma unroll
         for (int j = 0; j < 32; ++j)
-          *reinterpret_cast<__nv_bfloat16*>(sm + S2_V + bt_off(hc * 32 + j, n)) = __float2bfloat16_rn(v[j]);
+          *reinterpret_cast<__nv_bfloat16*>(sm + S2_T + bt_off(hc * 32 + j, n)) = __float2bfloat16_rn(v[j]);
         fence_async_smem();
       } else {
         __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.o) + (((size_t)b * T + s.x + hc * 32) * a.HV + hv) * VD + n;
@@ -705,7 +719,6 @@ __global__ void __launch_bounds__(K2_THREADS, 1) kda_fwd_state_tc_kernel(const _
         for (int j = 0; j < 32; ++j)
           if (j < rows) dst[j * step] = __float2bfloat16_rn(v[j]);
       }
-      mbar_arrive(bars + B_O);
     };
     {  // entering state, transposed: lane n, columns hc * 64 .. + 63
       for (int cb = 0; cb < 2; ++cb) {
@@ -742,11 +755,6 @@ __global__ void __launch_bounds__(K2_THREADS, 1) kda_fwd_state_tc_kernel(const _
       tmem_wait_st();
       fence_before();
       mbar_arrive(bars + B_Z);
-      // the previous chunk's o, staged over the v tile (every chain thread is done reading v)
-      if (ch > 0 && a.o) {
-        csync();
-        out_rows(ch - 1, Dp);
-      }
       // M^T <- M^T diag(e^{c_last}), storing the entering state for the backward
       if (!(ok = role_wait(bars + B_KD, par, polls, abort, 1, CH_THREADS))) break;
       {
@@ -783,13 +791,22 @@ __global__ void __launch_bounds__(K2_THREADS, 1) kda_fwd_state_tc_kernel(const _
       tmem_wait_st();
       fence_before();
       mbar_arrive(bars + B_UR);
-      // this chunk's state products done (its O^T is final)
-      if (!(ok = role_wait(bars + B_M3, par, polls, abort, 1, CH_THREADS))) break;
-      fence_after();
+      // the previous chunk's output rows (its products ended before this chunk's U^T was formed)
+      if (ch > 0) {
+        if (!(ok = role_wait(bars + B_M4, par ^ 1, polls, abort, 1, CH_THREADS))) break;
+        fence_after();
+        if (a.o) out_rows(ch - 1, Dp);
+        fence_before();
+        mbar_arrive(bars + B_O);
+      }
     }
-    if (ok && nch > 0 && a.o) {
-      csync();  // (the previous output's store has read the v tile: the issuer waited before loading v)
-      out_rows(nch - 1, TM_D0 + ((nch - 1) & 1) * 128);
+    if (ok && nch > 0) {  // the last chunk: its output products, then its rows and the final state
+      if ((ok = role_wait(bars + B_M4, (nch - 1) & 1, polls, abort, 1, CH_THREADS))) {
+        fence_after();
+        if (a.o) out_rows(nch - 1, TM_D0 + ((nch - 1) & 1) * 128);
+        fence_before();
+        mbar_arrive(bars + B_O);
+      }
     }
     if (ok && a.S_T) {
       fence_after();
