@@ -216,8 +216,8 @@ def gpu_prep_path(kda, name, steps, warmup, rank_barrier):
         def step():
             kda.fwd_prep(d["q"], d["k"], d["v"], d["z"], d["A_log"], d["dt_bias"], d["beta_logit"], scale=w.scale,
                          out_gate=d["og"], workspace=ws)
-        tokens, launches = w.B * w.T, 2
-        kernel = "kda_fwd_prep (kda_fwd_prep_tc_kernel<true> + kda_fwd_seq_tc_kernel, one call)"
+        tokens, launches = w.B * w.T, 4
+        kernel = "kda_fwd_prep (kda_prep_gate_kernel + kda_fwd_intra_tc_kernel<1> + kda_fwd_state_tc_kernel<1> + kda_out_gate_kernel, one call)"
         flush = None
     else:
         r = make_raw_inputs(w.with_sizes(T=1), conv_width=CONV_W)
@@ -515,7 +515,7 @@ def roofline_for(res, w, peaks):
     fwd_flops = chunk_flops_per_head_token(w.K, w.V, C) * head_tokens
     if w.path == "fwd":
         r = two_rooflines(algorithmic_bytes(w, "fwd"), fwd_flops, res["calls"]["kernel_ms"] * 1e-3, peaks)
-        r["kernel"] = ("kda_fwd (tensor-core chunk kernels, one call)"
+        r["kernel"] = ("kda_fwd (kda_fwd_intra_tc_kernel + kda_fwd_state_tc_kernel, one call)"
                        if w.K == 128 and w.dtype == "bf16" else "kda_fwd (CUDA-core chunk kernels)")
         return r
     # the step's dominant part is the backward call (state gradients, gradient
@@ -525,7 +525,7 @@ def roofline_for(res, w, peaks):
     r["kernel"] = ("kda_bwd (kda_bwd_dstate_tc_kernel + kda_bwd_grads_tc_kernel + kda_bwd_assemble_kernel, "
                    "one call)")
     r["fwd"] = dict(two_rooflines(algorithmic_bytes(w, "fwd"), fwd_flops, res["calls"]["fwd_ms"] * 1e-3, peaks),
-                    kernel="kda_fwd (tensor-core chunk kernels, one call)")
+                    kernel="kda_fwd (kda_fwd_intra_tc_kernel + kda_fwd_state_tc_kernel, one call)")
     r["step"] = two_rooflines(algorithmic_bytes(w, "fwdbwd"), (1 + BWD_FLOPS_RATIO) * fwd_flops,
                               res["ms_per_step"] * 1e-3, peaks)
     return r

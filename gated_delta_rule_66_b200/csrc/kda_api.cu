@@ -397,11 +397,16 @@ static bool ranges_overlap(const void* a, size_t an, const void* b, size_t bn) {
   return a && b && x < y + bn && y < x + an;
 }
 
+// the tensor-core path of kda_fwd_prep: [T and P images | g (fp32) | fp32 rows for the output gate]
+static size_t prep_tc_bytes(int B, int T, int HV, int K, int V) {
+  return img_bytes(B, T, HV, K, V) + (size_t)B * T * HV * K * sizeof(float) + (size_t)B * T * HV * V * sizeof(float);
+}
+
 size_t kda_fwd_prep_workspace_bytes(int B, int T, int H, int HV, int K, int V, int dtype) {
   if (B < 1 || T < 1 || H < 1 || HV < 1 || K < 1 || V < 1 || HV % H) return 0;
-  const size_t img = img_bytes(B, T, HV, K, V);
+  const size_t tc = (dtype == KDA_DTYPE_BF16 && K == 128 && V == 128) ? prep_tc_bytes(B, T, HV, K, V) : 0;
   const size_t o32 = dtype == KDA_DTYPE_BF16 ? (size_t)B * T * HV * V * sizeof(float) : 0;
-  return img > o32 ? img : o32;
+  return tc > o32 ? tc : o32;
 }
 
 int kda_fwd_prep(const void* q, const void* k, const void* v, const void* z, const float* A_log,
@@ -423,8 +428,20 @@ int kda_fwd_prep(const void* q, const void* k, const void* v, const void* z, con
   a.og_eps = out_eps;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (fwd_tc_eligible(a, dtype)) {
-    if (workspace && workspace_bytes >= img_bytes(B, T, HV, K, V)) a.img = static_cast<unsigned char*>(workspace);
-    return launch_fwd_tc(a, st);
+    if (!workspace || workspace_bytes < prep_tc_bytes(B, T, HV, K, V))
+      return launch_fwd_tc(a, st);  // one kernel per (b, hv) carrying the whole pipeline
+    // chunk-parallel kernel and state pass: the gate first (element-wise), then the
+    // two kernels on g, then the output gate over the fp32 rows
+    char* ws = static_cast<char*>(workspace);
+    const size_t ib = img_bytes(B, T, HV, K, V), gb = (size_t)B * T * HV * K * sizeof(float);
+    float* gbuf = reinterpret_cast<float*>(ws + ib);
+    a.img = reinterpret_cast<unsigned char*>(ws);
+    a.g = gbuf;
+    if (out_gate) a.o32 = reinterpret_cast<float*>(ws + ib + gb);
+    rc = launch_prep_gate(z, A_log, dt_bias, gate_lower_bound, gbuf, (size_t)B * T, HV, st);
+    if (!rc) rc = launch_fwd_tc(a, st);
+    if (!rc && out_gate) rc = launch_out_gate(a.o32, out_gate, out_eps, (size_t)B * T * HV, V, dtype, o, st);
+    return rc;
   }
   if (out_gate) {  // the CUDA-core forward stores fp32 o for the gate pass (in place for fp32)
     if (dtype == KDA_DTYPE_FP32) {

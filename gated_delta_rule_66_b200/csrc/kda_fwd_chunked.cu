@@ -23,8 +23,13 @@
 //       last state products run, and the previous chunk's output leaves while
 //       the next chunk's first products run.
 //
-// q, k, v and g (or the bf16 gate pre-activation z of the fused preparation)
-// are staged by TMA (cp.async.bulk.tensor, 128-byte swizzle, no multicast)
+// With the fused preparation (PREP) the gate g = gate(z + dt_bias) comes from
+// kda_prep_gate_kernel (an element-wise pass over z), the kernels form the
+// q and k row factors scale / |q_i| and 1 / |k_i| from the raw rows and the
+// beta sigmoid themselves, and with an output gate the state pass writes fp32
+// rows that the row kernel of the output gate finishes.
+//
+// q, k, v and g are staged by TMA (cp.async.bulk.tensor, 128-byte swizzle, no multicast)
 // from 4-D tensor maps [B, T, heads, 128]; the T and P images by 1-D bulk
 // copies.  beta is HV floats apart per step, which no tensor map can address
 // (its row stride need not be a multiple of 16 bytes): 64 threads load it.
@@ -55,8 +60,7 @@ using namespace tcc;
 // 4-D tensor maps [rows, T, heads, 128] of the raw inputs (rows = B, or 1 for
 // packed sequences); box 64 steps x one head x one 128-byte column block.
 struct FwdMaps {
-  CUtensorMap q, k, v, g;  // g: fp32 g, or the bf16 gate pre-activation z (fused preparation)
-  CUtensorMap o;           // the output (shape of v), written by TMA stores
+  CUtensorMap q, k, v, g;
 };
 
 // Byte offsets inside a raw tile of 64 rows x 128 channels as the 128-byte
@@ -89,84 +93,56 @@ struct SyncNamed {
 };
 
 // One thread issues the TMA loads of a chunk's q, k rows (query/key head h)
-// and g rows (value head hv; with PREP the bf16 z rows into the upper half of
-// the fp32 tile) on `bar`.
-template <bool PREP>
+// and g rows (value head hv) on `bar`.
 __device__ __forceinline__ void issue_qkg(const FwdMaps& m, uint32_t sQ, uint32_t sK, uint32_t sG, uint64_t* bar,
                                           int b, int t0, int h, int hv) {
   using namespace tc;
-  mbar_expect_tx(bar, 2 * TILE_BF16 + (PREP ? TILE_BF16 : TILE_F32));
+  mbar_expect_tx(bar, 2 * TILE_BF16 + TILE_F32);
   tma_load_4d(sQ, &m.q, 0, h, t0, b, bar);
   tma_load_4d(sQ + 8192, &m.q, 64, h, t0, b, bar);
   tma_load_4d(sK, &m.k, 0, h, t0, b, bar);
   tma_load_4d(sK + 8192, &m.k, 64, h, t0, b, bar);
-  if constexpr (PREP) {
-    tma_load_4d(sG + TILE_BF16, &m.g, 0, hv, t0, b, bar);
-    tma_load_4d(sG + TILE_BF16 + 8192, &m.g, 64, hv, t0, b, bar);
-  } else {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) tma_load_4d(sG + j * 8192, &m.g, 32 * j, hv, t0, b, bar);
-  }
+  for (int j = 0; j < 4; ++j) tma_load_4d(sG + j * 8192, &m.g, 32 * j, hv, t0, b, bar);
 }
-template <bool PREP>
 __device__ __forceinline__ void prefetch_qkg(const FwdMaps& m, int b, int t0, int h, int hv) {
   using namespace tc;
   tma_prefetch_4d(&m.q, 0, h, t0, b);
   tma_prefetch_4d(&m.q, 64, h, t0, b);
   tma_prefetch_4d(&m.k, 0, h, t0, b);
   tma_prefetch_4d(&m.k, 64, h, t0, b);
-  if constexpr (PREP) {
-    tma_prefetch_4d(&m.g, 0, hv, t0, b);
-    tma_prefetch_4d(&m.g, 64, hv, t0, b);
-  } else {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) tma_prefetch_4d(&m.g, 32 * j, hv, t0, b);
-  }
+  for (int j = 0; j < 4; ++j) tma_prefetch_4d(&m.g, 32 * j, hv, t0, b);
 }
 
-// Per-chunk input preparation on the landed raw tiles (256 threads): with
-// PREP the gate g = prep_gate(z + dt_bias) ("kimi_k3_host/kda.rs",
-// bounded_gate) replaces z, and the row factors scale / |q_i| and 1 / |k_i|
-// (l2norm_rows) go to sNq, sNk; without it the g rows at or past L are
-// cleared (packed sequences: they belong to the next sequence).  Rows at or
-// past L count as g = 0 either way, so that c_63 = c_{L-1}.  Ends with a
-// barrier of the 256 threads that run it (`sync`; tid counts from 0 among them).
+// Per-chunk input preparation on the landed raw tiles (256 threads): the g
+// rows at or past L are cleared (packed sequences: they belong to the next
+// sequence), so that c_63 = c_{L-1}; with PREP the row factors scale / |q_i|
+// and 1 / |k_i| ("kimi_k3_host/kda.rs", l2norm_rows) go to sNq, sNk.  Ends
+// with a barrier of the 256 threads that run it (`sync`; tid counts from 0
+// among them).
 template <bool PREP, class Sync>
 __device__ __forceinline__ void prep_tile(unsigned char* sQ, unsigned char* sK, unsigned char* sG, float* sNq,
-                                          float* sNk, int tid, int L, float scale, float dtb, float dec, float lb,
-                                          Sync sync) {
-  if constexpr (PREP) {
-    const int f = tid & 127, r0 = tid >> 7;
-    float gv[32];
+                                          float* sNk, int tid, int L, float scale, Sync sync) {
+  if constexpr (PREP) {  // 2 threads per row, rows 0..63 of q then of k
+    const int r = tid >> 1, part = tid & 1, i = r & 63;
+    const unsigned char* t = r < 64 ? sQ : sK;
+    float s = 0.f;
 #pragma unroll
-    for (int m = 0; m < 32; ++m) {
-      const int i = r0 + 2 * m;
-      gv[m] = i < L ? prep_gate_fast(ldb(sG + TILE_BF16, i, f) + dtb, dec, lb) : 0.f;
+    for (int u = 0; u < 16; ++u) {
+      float x[4];
+      bf16x4(t + bt_off(i, part * 64 + 4 * u), x);
+      s = fmaf(x[0], x[0], fmaf(x[1], x[1], fmaf(x[2], x[2], fmaf(x[3], x[3], s))));
     }
-    {  // row norms: 2 threads per row, rows 0..63 of q then of k
-      const int r = tid >> 1, part = tid & 1, i = r & 63;
-      const unsigned char* t = r < 64 ? sQ : sK;
-      float s = 0.f;
-#pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        float x[4];
-        bf16x4(t + bt_off(i, part * 64 + 4 * u), x);
-        s = fmaf(x[0], x[0], fmaf(x[1], x[1], fmaf(x[2], x[2], fmaf(x[3], x[3], s))));
-      }
-      s += __shfl_xor_sync(0xffffffffu, s, 1);
-      if (part == 0) {
-        const float n = rsqrtf(s + KDA_L2_EPS_F);
-        if (r < 64) sNq[i] = n * scale;
-        else sNk[i] = n;
-      }
+    s += __shfl_xor_sync(0xffffffffu, s, 1);
+    if (part == 0) {
+      const float nrm = rsqrtf(s + KDA_L2_EPS_F);
+      if (r < 64) sNq[i] = nrm * scale;
+      else sNk[i] = nrm;
     }
-    sync();
-#pragma unroll
-    for (int m = 0; m < 32; ++m) *reinterpret_cast<float*>(sG + ft_off(r0 + 2 * m, f)) = gv[m];
-  } else {
-    if (L < C)
-      for (int x = tid; x < (C - L) * KD; x += NTH) *reinterpret_cast<float*>(sG + ft_off(L + x / KD, x % KD)) = 0.f;
   }
+  if (L < C)
+    for (int x = tid; x < (C - L) * KD; x += NTH) *reinterpret_cast<float*>(sG + ft_off(L + x / KD, x % KD)) = 0.f;
   sync();
 }
 
@@ -366,7 +342,7 @@ __global__ void __launch_bounds__(NTH, 2) kda_fwd_intra_tc_kernel(const __grid_c
   const auto issue = [&](int item) {
     int hv, b, t0, L;
     span_of(item, hv, b, t0, L);
-    issue_qkg<PREP>(maps, sb + K1_Q, sb + K1_K, sb + K1_C, bar_raw, b, t0, hv / G, hv);
+    issue_qkg(maps, sb + K1_Q, sb + K1_K, sb + K1_C, bar_raw, b, t0, hv / G, hv);
   };
   if (blockIdx.x < items) {
     if (tid == 0) issue(blockIdx.x);
@@ -376,14 +352,10 @@ __global__ void __launch_bounds__(NTH, 2) kda_fwd_intra_tc_kernel(const __grid_c
   for (int item = blockIdx.x; item < items; item += gridDim.x) {
     int hv, b, t0, L;
     span_of(item, hv, b, t0, L);
-    float bval = 0.f, dtb = 0.f, dec = 0.f;
+    float bval = 0.f;
     if (tid < C && tid < L) {
       bval = a.beta[((size_t)b * a.T + t0 + tid) * a.HV + hv];
       if (PREP) bval = prep_sigmoid_fast(bval);
-    }
-    if constexpr (PREP) {
-      dtb = a.prep.dt_bias[(size_t)hv * KD + (tid & 127)];
-      dec = expf(a.prep.A_log[hv]);
     }
     if (!wait_all(bar_raw, w_raw & 1, polls)) { failed = true; break; }
     ++w_raw;
@@ -391,10 +363,10 @@ __global__ void __launch_bounds__(NTH, 2) kda_fwd_intra_tc_kernel(const __grid_c
     if (tid == 0 && item + 2 * (int)gridDim.x < items) {  // the item after next into L2
       int hv2, b2, t2, L2;
       span_of(item + 2 * gridDim.x, hv2, b2, t2, L2);
-      prefetch_qkg<PREP>(maps, b2, t2, hv2 / G, hv2);
+      prefetch_qkg(maps, b2, t2, hv2 / G, hv2);
     }
     prep_tile<PREP>(sm + K1_Q, sm + K1_K, sm + K1_C, reinterpret_cast<float*>(sm + K1_NQ),
-                    reinterpret_cast<float*>(sm + K1_NK), tid, L, a.scale, dtb, dec, a.prep.gate_lb, SyncAll());
+                    reinterpret_cast<float*>(sm + K1_NK), tid, L, a.scale, SyncAll());
     const bool wide = cumsum_tile<true>(sm + K1_C, reinterpret_cast<float*>(sm + K1_CARRY), tid, SyncAll());
 
     for (int p = 0; p < 4; ++p) {
@@ -495,8 +467,8 @@ __global__ void __launch_bounds__(NTH, 2) kda_fwd_intra_tc_kernel(const __grid_c
 // ============================================================================
 // Warp-specialised, 544 threads (17 warps):
 //   issuer warp 0 (lane 0): every tensor-core product and the v, T, P copies
-//     and the output's TMA stores (a tcgen05.mma issue can block its thread
-//     for about the product's duration, so this warp does nothing else);
+//     (a tcgen05.mma issue can block its thread for about the product's
+//     duration, so this warp does nothing else);
 //   chain warps 1-8 (warp w: TMEM lanes 32 (w % 4) .. + 31, lane = value
 //     column n; column half (w - 1) / 4 of every accumulator): the residual
 //     Z^T = V^T - Y^T, the tf32 rounding of U^T, the state's decay (storing
@@ -504,6 +476,8 @@ __global__ void __launch_bounds__(NTH, 2) kda_fwd_intra_tc_kernel(const __grid_c
 //   builder warps 9-16: the next chunk's decay, [K o e^c ; Q~ o e^c] and
 //     (K o e^{c_last-c})^T operands and e^{c_last}; builder thread 0 issues the
 //     raw q / k / g copies.
+// The output rows of a chunk leave from the chain's registers: the chain reads
+// O^T out of TMEM, releases the accumulator (B_O) and then stores.
 // The roles meet on mbarriers only: builders and chain threads arrive when an
 // operand or a step is done, tensor-core completions arrive through
 // tcgen05.commit.  A wait that gives up sets the shared abort word, which
@@ -593,9 +567,6 @@ __global__ void __launch_bounds__(K2_THREADS, 1) kda_fwd_state_tc_kernel(const _
 
   const auto span = [&](int ch) { return chunk_span(a, c0 + ch); };
   const auto rec = [&](int ch) { return a.img + chunk_gc(a, sq, hv, c0 + ch) * (size_t)FWI_BYTES; };
-  // the output of chunk ch goes out by TMA store unless it is a short chunk of
-  // a packed batch (its box would reach into the next sequence)
-  const auto tma_out = [&](int ch) { return !a.ctab || span(ch).y == C; };
 
   if (warp == 0) {
     // ======================================================================== issuer warp
@@ -621,26 +592,16 @@ __global__ void __launch_bounds__(K2_THREADS, 1) kda_fwd_state_tc_kernel(const _
                  idesc_tf32(128, 64), 1);
         commit_to(B_M4);
       };
-      // the output rows of chunk ch, staged over the T slot, leave by TMA store
-      const auto store_o = [&](int ch) {
-        if (!wait_one(bars + B_O, ch & 1, polls, abort)) return false;
-        if (a.o && tma_out(ch)) {
-          const int t0 = span(ch).x;
-          tma_store_4d(&maps.o, 0, hv, t0, b, sb + S2_T);
-          tma_store_4d(&maps.o, 64, hv, t0, b, sb + S2_T + 8192);
-          bulk_commit();
-          bulk_wait_read();
-        }
-        return true;
-      };
       issue_v(0);
       issue_img(B_T, sb + S2_T, 0, FWR_T);
       issue_img(B_P, sb + S2_P, 0, FWR_P);
       for (int ch = 0; ch < nch; ++ch) {
         const uint32_t par = ch & 1, D = TM_D0 + (ch & 1) * 128;
-        // [Y^T | O^T] = M^T [K o e^c ; Q~ o e^c]^T once the operand is built and the state updated
+        // [Y^T | O^T] = M^T [K o e^c ; Q~ o e^c]^T once the operand is built, the state updated
+        // and the output of two chunks back (same accumulator) read out
         if (!wait_one(bars + B_KQ, par, polls, abort)) break;
         if (ch > 0 && !wait_one(bars + B_M3, par ^ 1, polls, abort)) break;
+        if (ch > 1 && !wait_one(bars + B_O, par, polls, abort)) break;
         fence_after();
         for (int ks = 0; ks < 16; ++ks)
           mma_ts(tm + D, tm + TM_S + ks * 8, desc(sb + S2_KQ + ks * 256, 4096), idesc_tf32(128, 128), ks > 0);
@@ -661,6 +622,8 @@ __global__ void __launch_bounds__(K2_THREADS, 1) kda_fwd_state_tc_kernel(const _
           if (!wait_one(bars + B_M4, par ^ 1, polls, abort)) break;
           issue_img(B_P, sb + S2_P, ch, FWR_P);
         }
+        if (!wait_one(bars + B_M2, par, polls, abort)) break;
+        if (ch + 1 < nch) issue_img(B_T, sb + S2_T, ch + 1, FWR_T);  // this chunk's T is consumed
         // M^T += U^T (K o e^{c_last-c}) once U^T is rounded and the state decayed
         if (!wait_one(bars + B_UR, par, polls, abort)) break;
         if (!wait_one(bars + B_KD, par, polls, abort)) break;
@@ -668,53 +631,35 @@ __global__ void __launch_bounds__(K2_THREADS, 1) kda_fwd_state_tc_kernel(const _
         for (int ks = 0; ks < 8; ++ks)
           mma_ts(tm + TM_S, tm + TM_U + ks * 8, desc(sb + S2_KD + ks * 256, 2048), idesc_tf32(128, 128), 1);
         commit_to(B_M3);
-        // the previous chunk's output (staged over T, free since m2) leaves; then the next T
-        if (ch > 0 && !store_o(ch - 1)) break;
-        if (ch + 1 < nch) issue_img(B_T, sb + S2_T, ch + 1, FWR_T);
       }
-      if (!*abort) {  // the last chunk's output products and rows
-        if (wait_one(bars + B_P, (nch - 1) & 1, polls, abort)) {
-          fence_after();
-          o_part(nch - 1);
-          store_o(nch - 1);
-        }
+      if (!*abort && wait_one(bars + B_P, (nch - 1) & 1, polls, abort)) {  // the last chunk's output products
+        fence_after();
+        o_part(nch - 1);
       }
-      asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
     }
     __syncwarp();
   } else if (warp <= 8) {
     // ======================================================================== chain warps
     const int n = (warp & 3) * 32 + lane, hc = (warp - 1) >> 2;  // TMEM lane (value column), column half
     const uint32_t lo = (uint32_t)((warp & 3) * 32) << 16;
-    const __nv_bfloat16* gate = static_cast<const __nv_bfloat16*>(a.og);
-    float* red = reinterpret_cast<float*>(sm + S2_RED);
     const SyncNamed csync{1, CH_THREADS};
-    // o rows hc * 32 .. + 31 of chunk ch (value column n) from O^T in accumulator d: staged
-    // over the v tile for the issuer's TMA store, or stored directly (short chunks of a packed batch)
+    // o rows hc * 32 .. + 31 of chunk ch (value column n) from O^T in accumulator d: read
+    // out, released to the issuer (B_O), then stored from registers (fp32 into o32 when
+    // an output gate follows, else in the output dtype)
     const auto out_rows = [&](int ch, uint32_t d) {
       const int2 s = span(ch);
       float v[32];
       tmem_ld32(tm + lo + d + 64 + hc * 32, v);
-      if (gate) {  // "kimi_k3_host/kda.rs", full_rank_output_gate: o / rms(o) * sigmoid(gate), rows over n
-        float gv[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int i = hc * 32 + j;
-          gv[j] = i < s.y ? __bfloat162float(gate[(((size_t)b * T + s.x + i) * a.HV + hv) * VD + n]) : 0.f;
-        }
-        out_gate_rows(v, red, warp - 1, lane, a.og_eps, csync);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] *= prep_sigmoid_fast(gv[j]);
-      }
-      if (tma_out(ch)) {
+      fence_before();
+      mbar_arrive(bars + B_O);
+      const size_t row0 = (((size_t)b * T + s.x + hc * 32) * a.HV + hv) * VD + n, step = (size_t)a.HV * VD;
+      const int rows = min(32, s.y - hc * 32);
+      if (a.o32) {
 #pragma unroll
         for (int j = 0; j < 32; ++j)
-          *reinterpret_cast<__nv_bfloat16*>(sm + S2_T + bt_off(hc * 32 + j, n)) = __float2bfloat16_rn(v[j]);
-        fence_async_smem();
-      } else {
-        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.o) + (((size_t)b * T + s.x + hc * 32) * a.HV + hv) * VD + n;
-        const size_t step = (size_t)a.HV * VD;
-        const int rows = min(32, s.y - hc * 32);
+          if (j < rows) a.o32[row0 + j * step] = v[j];
+      } else if (a.o) {
+        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.o) + row0;
 #pragma unroll
         for (int j = 0; j < 32; ++j)
           if (j < rows) dst[j * step] = __float2bfloat16_rn(v[j]);
@@ -741,16 +686,12 @@ __global__ void __launch_bounds__(K2_THREADS, 1) kda_fwd_state_tc_kernel(const _
       if (!(ok = role_wait(bars + B_M1, par, polls, abort, 1, CH_THREADS))) break;
       fence_after();
       {
-        uint32_t y[32];
-        tmem_ld32_nw(tm + lo + D + hc * 32, y);
-        float vv[32];
+        float y[32];
+        uint32_t z[32];
+        tmem_ld32(tm + lo + D + hc * 32, y);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) vv[j] = ldb(sm + S2_V, hc * 32 + j, n);
-        tmem_wait_ld();
-        tmem_regs_ready(y);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) y[j] = tf32_rna(vv[j] - __uint_as_float(y[j]));
-        tmem_st32(tm + lo + D + hc * 32, y);
+        for (int j = 0; j < 32; ++j) z[j] = tf32_rna(ldb(sm + S2_V, hc * 32 + j, n) - y[j]);
+        tmem_st32(tm + lo + D + hc * 32, z);
       }
       tmem_wait_st();
       fence_before();
@@ -763,30 +704,28 @@ __global__ void __launch_bounds__(K2_THREADS, 1) kda_fwd_state_tc_kernel(const _
         const float* el = sEl + hc * 64;
 #pragma unroll 1
         for (int cb = 0; cb < 2; ++cb) {
-          uint32_t sv[32];
-          tmem_ld32_nw(tm + lo + TM_S + hc * 64 + cb * 32, sv);
-          tmem_wait_ld();
-          tmem_regs_ready(sv);
+          float sv[32];
+          uint32_t r[32];
+          tmem_ld32(tm + lo + TM_S + hc * 64 + cb * 32, sv);
           if (dst) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) dst[(size_t)(cb * 32 + j) * VD] = __uint_as_float(sv[j]);
+            for (int j = 0; j < 32; ++j) dst[(size_t)(cb * 32 + j) * VD] = sv[j];
           }
 #pragma unroll
-          for (int j = 0; j < 32; ++j) sv[j] = __float_as_uint(__uint_as_float(sv[j]) * el[cb * 32 + j]);
-          tmem_st32(tm + lo + TM_S + hc * 64 + cb * 32, sv);
+          for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(sv[j] * el[cb * 32 + j]);
+          tmem_st32(tm + lo + TM_S + hc * 64 + cb * 32, r);
         }
       }
       // U^T rounded to tf32
       if (!(ok = role_wait(bars + B_M2, par, polls, abort, 1, CH_THREADS))) break;
       fence_after();
       {
-        uint32_t u[32];
-        tmem_ld32_nw(tm + lo + TM_U + hc * 32, u);
-        tmem_wait_ld();
-        tmem_regs_ready(u);
+        float u[32];
+        uint32_t r[32];
+        tmem_ld32(tm + lo + TM_U + hc * 32, u);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) u[j] = tf32_rna(__uint_as_float(u[j]));
-        tmem_st32(tm + lo + TM_U + hc * 32, u);
+        for (int j = 0; j < 32; ++j) r[j] = tf32_rna(u[j]);
+        tmem_st32(tm + lo + TM_U + hc * 32, r);
       }
       tmem_wait_st();
       fence_before();
@@ -795,17 +734,13 @@ __global__ void __launch_bounds__(K2_THREADS, 1) kda_fwd_state_tc_kernel(const _
       if (ch > 0) {
         if (!(ok = role_wait(bars + B_M4, par ^ 1, polls, abort, 1, CH_THREADS))) break;
         fence_after();
-        if (a.o) out_rows(ch - 1, Dp);
-        fence_before();
-        mbar_arrive(bars + B_O);
+        out_rows(ch - 1, Dp);
       }
     }
     if (ok && nch > 0) {  // the last chunk: its output products, then its rows and the final state
       if ((ok = role_wait(bars + B_M4, (nch - 1) & 1, polls, abort, 1, CH_THREADS))) {
         fence_after();
-        if (a.o) out_rows(nch - 1, TM_D0 + ((nch - 1) & 1) * 128);
-        fence_before();
-        mbar_arrive(bars + B_O);
+        out_rows(nch - 1, TM_D0 + ((nch - 1) & 1) * 128);
       }
     }
     if (ok && a.S_T) {
@@ -824,19 +759,14 @@ __global__ void __launch_bounds__(K2_THREADS, 1) kda_fwd_state_tc_kernel(const _
     const SyncNamed bsync{2, BU_THREADS};
     float* sNq = reinterpret_cast<float*>(sm + S2_NQ);
     float* sNk = reinterpret_cast<float*>(sm + S2_NK);
-    float dtb = 0.f, dec = 0.f;
-    if constexpr (PREP) {
-      dtb = a.prep.dt_bias[(size_t)hv * KD + (bt & 127)];
-      dec = expf(a.prep.A_log[hv]);
-    }
     const auto issue_raw = [&](int ch) {
-      issue_qkg<PREP>(maps, sb + S2_Q, sb + S2_K, sb + S2_C, bars + B_RAW, b, span(ch).x, h, hv);
+      issue_qkg(maps, sb + S2_Q, sb + S2_K, sb + S2_C, bars + B_RAW, b, span(ch).x, h, hv);
       ++cnt[B_RAW];
     };
     if (nch > 0 && bt == 0) {
       issue_raw(0);
       if (nch > 1) {
-        prefetch_qkg<PREP>(maps, b, span(1).x, h, hv);
+        prefetch_qkg(maps, b, span(1).x, h, hv);
         tma_prefetch_4d(&maps.v, 0, hv, span(1).x, b);
         tma_prefetch_4d(&maps.v, 64, hv, span(1).x, b);
       }
@@ -845,8 +775,7 @@ __global__ void __launch_bounds__(K2_THREADS, 1) kda_fwd_state_tc_kernel(const _
     for (int ch = 0; ch < nch; ++ch) {
       const int2 sp = span(ch);
       if (!role_wait(bars + B_RAW, ch & 1, polls, abort, 2, BU_THREADS)) break;
-      prep_tile<PREP>(sm + S2_Q, sm + S2_K, sm + S2_C, sNq, sNk, bt, sp.y, a.scale, dtb, dec, a.prep.gate_lb,
-                      bsync);
+      prep_tile<PREP>(sm + S2_Q, sm + S2_K, sm + S2_C, sNq, sNk, bt, sp.y, a.scale, bsync);
       cumsum_tile<false>(sm + S2_C, reinterpret_cast<float*>(sm + S2_CARRY), bt, bsync);
       // [K o e^c ; Q~ o e^c]: its slot is free once the previous chunk's first products are done
       if (ch > 0 && !role_wait(bars + B_M1, (ch - 1) & 1, polls, abort, 2, BU_THREADS)) break;
@@ -891,7 +820,7 @@ __global__ void __launch_bounds__(K2_THREADS, 1) kda_fwd_state_tc_kernel(const _
       if (bt == 0 && ch + 1 < nch) {
         issue_raw(ch + 1);
         if (ch + 2 < nch) {
-          prefetch_qkg<PREP>(maps, b, span(ch + 2).x, h, hv);
+          prefetch_qkg(maps, b, span(ch + 2).x, h, hv);
           tma_prefetch_4d(&maps.v, 0, hv, span(ch + 2).x, b);
           tma_prefetch_4d(&maps.v, 64, hv, span(ch + 2).x, b);
           prefetch_l2(rec(ch + 2), FWI_BYTES);
@@ -960,8 +889,7 @@ int launch_t(const FwdArgs& a, cudaStream_t stream) {
   int rc = head_map(&m.q, a.q, true, rows, a.T, a.H, 64);
   if (!rc) rc = head_map(&m.k, a.k, true, rows, a.T, a.H, 64);
   if (!rc) rc = head_map(&m.v, a.v, true, rows, a.T, a.HV, 64);
-  if (!rc) rc = PREP ? head_map(&m.g, a.prep.z, true, rows, a.T, a.HV, 64) : head_map(&m.g, a.g, false, rows, a.T, a.HV, 32);
-  if (!rc) rc = head_map(&m.o, a.o ? a.o : a.v, true, rows, a.T, a.HV, 64);  // (no o: never used)
+  if (!rc) rc = head_map(&m.g, a.g, false, rows, a.T, a.HV, 32);
   if (rc) return rc;
   cudaError_t e = cudaFuncSetAttribute(kda_fwd_intra_tc_kernel<PREP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)K1_BYTES);
@@ -983,6 +911,38 @@ int launch_t(const FwdArgs& a, cudaStream_t stream) {
   return 0;
 }
 }  // namespace
+
+// The gate of the fused preparation ("kimi_k3_host/kda.rs", bounded_gate):
+// g[r][hv][f] = gate(z[r][hv][f] + dt_bias[hv][f]) with e^{A_log[hv]}, eight
+// channels (one 16-byte piece of z) per thread.
+__global__ void __launch_bounds__(256) kda_prep_gate_kernel(const __nv_bfloat16* __restrict__ z,
+                                                             const float* __restrict__ A_log,
+                                                             const float* __restrict__ dt_bias, float lb,
+                                                             float* __restrict__ g, size_t pieces, int HV) {
+  const size_t x = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (x >= pieces) return;
+  const int hv = (int)((x >> 4) % HV), f0 = (int)(x & 15) * 8;  // 16 pieces of 8 channels per (row, hv)
+  const uint4 zr = reinterpret_cast<const uint4*>(z)[x];
+  const __nv_bfloat16* zb = reinterpret_cast<const __nv_bfloat16*>(&zr);
+  const float dec = expf(A_log[hv]);
+  float o[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) o[u] = prep_gate_fast(__bfloat162float(zb[u]) + dt_bias[hv * 128 + f0 + u], dec, lb);
+  float4* dst = reinterpret_cast<float4*>(g + x * 8);
+  dst[0] = make_float4(o[0], o[1], o[2], o[3]);
+  dst[1] = make_float4(o[4], o[5], o[6], o[7]);
+}
+
+int launch_prep_gate(const void* z, const float* A_log, const float* dt_bias, float lb, float* g, size_t rows, int HV,
+                     cudaStream_t stream) {
+  const size_t pieces = rows * (size_t)HV * 16;  // K = 128
+  if (pieces == 0) return 0;
+  kda_prep_gate_kernel<<<(unsigned)((pieces + 255) / 256), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(z), A_log, dt_bias, lb, g, pieces, HV);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_cuda_error("kda_fwd_prep: gate launch", e);
+  return 0;
+}
 
 int launch_fwd_chunked(const FwdArgs& a, cudaStream_t stream) {
   return a.prep.z ? launch_t<true>(a, stream) : launch_t<false>(a, stream);

@@ -192,6 +192,9 @@ int launch_fwd_tc(const FwdArgs& a, cudaStream_t stream);
 // interaction and inverse, then the state pass
 int launch_fwd_chunked(const FwdArgs& a, cudaStream_t stream);
 int take_fwd_chunked_error(unsigned* out);
+// the gate of the fused preparation into g (fp32 [rows, HV, 128]) from the bf16 z
+int launch_prep_gate(const void* z, const float* A_log, const float* dt_bias, float lb, float* g, size_t rows, int HV,
+                     cudaStream_t stream);
 // probes of every bounded wait in the chunked forward (0: the default)
 int set_wait_polls(unsigned polls);
 int take_device_error(unsigned* out);

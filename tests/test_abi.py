@@ -168,8 +168,10 @@ def test_varlen_workspace_and_validation(lib):
 
 def test_prep_workspace_and_validation(lib):
     B, T, H, HV = 2, 100, 1, 2
-    # tensor-core shape: the T and P images; a CUDA-core bf16 shape: the fp32 output for the gate pass
-    assert lib.kda_fwd_prep_workspace_bytes(B, T, H, HV, 128, 128, 1) == B * HV * 2 * 32768
+    # tensor-core shape: see below; a CUDA-core bf16 shape: the fp32 output for the gate pass
+    # (the T and P images, fp32 g and the fp32 rows of the output gate)
+    assert lib.kda_fwd_prep_workspace_bytes(B, T, H, HV, 128, 128, 1) == (B * HV * 2 * 32768 + B * T * HV * 128 * 4
+                                                                         + B * T * HV * 128 * 4)
     assert lib.kda_fwd_prep_workspace_bytes(B, T, H, HV, 64, 32, 1) == B * T * HV * 32 * 4
     assert lib.kda_fwd_prep_workspace_bytes(B, T, H, HV, 64, 32, 0) == 0
     assert lib.kda_fwd_prep_workspace_bytes(B, T, 2, 3, 64, 32, 0) == 0  # HV % H != 0

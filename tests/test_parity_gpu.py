@@ -336,7 +336,12 @@ def test_fwdbwd_full_size(kda):
                    workspace=ws)
     grads = kda.bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["dO"], scale=w.scale,
                     initial_state=d["S0"], workspace=ws, states_from_fwd=True)
+    # the same forward again gives the same bits (no data race in the pipelined kernels)
+    o2, S2 = kda.fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], scale=w.scale, initial_state=d["S0"],
+                     workspace=ws)
     torch.cuda.synchronize()
+    assert torch.equal(o, o2) and torch.equal(S, S2), "two identical forwards differ"
+    del o2, S2
     sub, hv_idx = head_subset(inp, w.H, w.HV, [17, 60])
     o_ref, S_ref = oracle_fwd(sub, w.scale)
     tol = tol_for(w.torch_dtype)
