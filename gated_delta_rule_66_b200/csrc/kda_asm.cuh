@@ -4,6 +4,8 @@
 // where the split exponents would leave fp32 range).
 #pragma once
 
+#include <cuda_fp16.h>
+
 #include "kda_chunk.cuh"
 #include "kda_internal.h"
 
@@ -56,6 +58,14 @@ __device__ __forceinline__ void store4(__nv_bfloat16* p, float x, float y, float
 // of the KQ = 32 columns of a [64][LDK] array, by 8 segments of 8 rows
 // (256 threads; seg is 8 x KQ scratch; `base` is added to every element of a
 // reverse sum).  Ends with a barrier.
+
+// four consecutive fp16 record elements (8-byte aligned) as floats
+__device__ __forceinline__ float4 ld4h(const __half* p) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
+  const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&u.y));
+  return make_float4(lo.x, lo.y, hi.x, hi.y);
+}
 template <bool REVERSE>
 __device__ __forceinline__ void cumsum64(float* a, float* seg, const float* base) {
   constexpr int LDK = AsmSmem::LDK, KQ = AsmSmem::KQ;
@@ -96,6 +106,7 @@ __device__ __forceinline__ void assemble_quarter(const BwdArgs& a, float* smem, 
   const int t0 = sp.x, L = sp.y, f0 = fq4 * KQ;
   const size_t gc = chunk_gc(a, sq, hv, ch);
   const float* rec = a.gws + gc * GREC;
+  const __half* rech = reinterpret_cast<const __half*>(rec);
   const TIn* q = static_cast<const TIn*>(a.q);
   const TIn* k = static_cast<const TIn*>(a.k);
   const int tid = threadIdx.x;
@@ -111,9 +122,9 @@ __device__ __forceinline__ void assemble_quarter(const BwdArgs& a, float* smem, 
   float qe[8], ke[8], kd[8];
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
-    qe[u] = rec[G_QK + rec_off(ei + u, f0 + ef, 128)];
-    ke[u] = rec[G_QK + rec_off(64 + ei + u, f0 + ef, 128)];
-    kd[u] = rec[G_KED + rec_off(ei + u, f0 + ef, 128)];
+    qe[u] = __half2float(rech[GH_QK + rec_off(ei + u, f0 + ef, 128)]);
+    ke[u] = __half2float(rech[GH_QK + rec_off(64 + ei + u, f0 + ef, 128)]);
+    kd[u] = __half2float(rech[GH_KED + rec_off(ei + u, f0 + ef, 128)]);
   }
   {  // inputs of this channel quarter (4 channels per item) and the C x C adjoints; loads first
     float4 gv[2], dp[4], da[4];
@@ -134,8 +145,8 @@ __device__ __forceinline__ void assemble_quarter(const BwdArgs& a, float* smem, 
 #pragma unroll
     for (int m = 0; m < 4; ++m) {  // row i of [dP; dA], four columns j per item
       const int idx = tid + m * NTHREADS, i = idx >> 4, j4 = (idx & 15) * 4;
-      dp[m] = *reinterpret_cast<const float4*>(rec + G_PA + rec_off(i, j4, 64));
-      da[m] = *reinterpret_cast<const float4*>(rec + G_PA + rec_off(64 + i, j4, 64));
+      dp[m] = ld4h(rech + GH_PA + rec_off(i, j4, 64));
+      da[m] = ld4h(rech + GH_PA + rec_off(64 + i, j4, 64));
     }
     float bt[4];  // beta of the rows of the [dA] items
 #pragma unroll

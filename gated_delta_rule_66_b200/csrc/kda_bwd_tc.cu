@@ -18,6 +18,7 @@
 // index of the 32-step state layout, or its even one when the sequence ends in
 // the chunk's first half); the per-chunk gradient kernel reads it there.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include <mutex>
 
@@ -38,6 +39,14 @@ static_assert(IMG_TT + 16384 <= SMALL, "state-gradient shared-memory map");
 constexpr uint32_t TM_S = 0, TM_DU = 128, TM_DR = 192, TM_DOT = 256;
 }  // namespace tcb
 
+// four fp32 values rounded to fp16 into 8 bytes of shared memory
+__device__ __forceinline__ void st4h(__half* p, const float* v) {
+  const __half2 lo = __floats2half2_rn(v[0], v[1]), hi = __floats2half2_rn(v[2], v[3]);
+  uint2 u;
+  u.x = *reinterpret_cast<const unsigned*>(&lo);
+  u.y = *reinterpret_cast<const unsigned*>(&hi);
+  *reinterpret_cast<uint2*>(p) = u;
+}
 __global__ void __launch_bounds__(256, 1) kda_bwd_dstate_tc_kernel(BwdArgs a) {
   using namespace tcb;
   using namespace tc;
@@ -541,38 +550,30 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
 
     // ---------------------------------------------------------------- record
     {  // the record staged in shared memory (now free) in its global layout, then bulk-stored
-      float* st = reinterpret_cast<float*>(sm);  // [dP; dA] | [dQE; dKE'] | dKEd
-      constexpr int S_PA = 0, S_QK = 8192, S_KED = 24576;
-      static_assert(4 * (S_KED + 8192) <= OP_DO, "record staging below [dO; -dR]");
+      __half* st = reinterpret_cast<__half*>(sm);  // fp16 [dP; dA] | [dQE; dKE'] | dKEd, as in the record
+      static_assert(2 * (GH_KED + 8192) <= OP_DO, "record staging below [dO; -dR]");
+      static_assert(2 * (GH_KED + 8192) == 4 * G_DBR, "fp32 tail follows the fp16 matrices");
       float v[32];
       tmem_ld32(tm + lo + TM_PA + hcol * 32, v);
 #pragma unroll
-      for (int q4 = 0; q4 < 8; ++q4)
-        *reinterpret_cast<float4*>(st + S_PA + rec_off(Lr, hcol * 32 + 4 * q4, 64)) =
-            make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+      for (int q4 = 0; q4 < 8; ++q4) st4h(st + GH_PA + rec_off(Lr, hcol * 32 + 4 * q4, 64), v + 4 * q4);
       for (int cb = 0; cb < 2; ++cb) {
         const int f0 = hcol * 64 + cb * 32;
         tmem_ld32(tm + lo + TM_QK + f0, v);
 #pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4)
-          *reinterpret_cast<float4*>(st + S_QK + rec_off(Lr, f0 + 4 * q4, 128)) =
-              make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+        for (int q4 = 0; q4 < 8; ++q4) st4h(st + GH_QK + rec_off(Lr, f0 + 4 * q4, 128), v + 4 * q4);
         tmem_ld32(tm + lo + TM_KED + f0, v);
         if (lane < 16) {
           const int r = cx.sub * 16 + lane;  // M = 64 accumulator layout
 #pragma unroll
-          for (int q4 = 0; q4 < 8; ++q4)
-            *reinterpret_cast<float4*>(st + S_KED + rec_off(r, f0 + 4 * q4, 128)) =
-                make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+          for (int q4 = 0; q4 < 8; ++q4) st4h(st + GH_KED + rec_off(r, f0 + 4 * q4, 128), v + 4 * q4);
         }
       }
       fence_async_smem();
       __syncthreads();
       if (tid == 0) {
-        bulk_s2g(rec + G_PA, sb + 4 * S_PA, 32768);
-        bulk_s2g(rec + G_QK, sb + 4 * S_QK, 32768);
-        bulk_s2g(rec + G_QK + 8192, sb + 4 * S_QK + 32768, 32768);
-        bulk_s2g(rec + G_KED, sb + 4 * S_KED, 32768);
+        bulk_s2g(rec, sb, 32768);
+        bulk_s2g(rec + 8192, sb + 32768, 32768);
         bulk_s2g(rec + G_DBR, sb + S_EMID, 256);
         bulk_s2g(rec + G_DEL, sb + S_EL, 512);
         bulk_commit();

@@ -9,11 +9,14 @@ namespace kda {
 constexpr int FWD_CHUNK = 32;    // chunk length of the chunked kernels
 constexpr int FWD_VBLOCK = 32;   // V columns per CTA in the chunked kernels
 
-// Per-(b, hv, 64-step chunk) record of the tensor-core backward (floats),
-// row-major with the 16-byte pieces of row r XOR-swizzled by r % 8 (element
-// (r, c) of a row of n floats at rec_off(r, c, n)): [dP; dA] as [i'][j]
-// (128 x 64, i' < 64 dP), [dQE; dKE'] as [i'][f] (128 x 128, i' < 64 dQE),
-// dKEd as [i][f] (64 x 128); then dbeta_R [64], dEl [128] (G_AH unused).
+// Per-(b, hv, 64-step chunk) record of the tensor-core backward: three fp16
+// matrices, row-major with the 4-element groups of row r XOR-swizzled by
+// r % 8 (element (r, c) of a row of n at rec_off(r, c, n)): [dP; dA] as [i'][j]
+// (128 x 64, i' < 64 dP) at half offset GH_PA, [dQE; dKE'] as [i'][f] (128 x
+// 128, i' < 64 dQE) at GH_QK, dKEd as [i][f] (64 x 128) at GH_KED; then fp32
+// dbeta_R [64] and dEl [128] at float offsets G_DBR, G_DEL; GREC floats per
+// chunk.  (fp16 keeps 11 significant bits: about 3e-4 relative RMS added to
+// the gradients, against their 2e-3 bar; the range covers these sums.)
 // Per-(b, hv, 64-step chunk) interaction record that the tensor-core forward
 // stores with a workspace (floats).  Three 64 x 64 tf32 operand images in the
 // K-major canonical layout of the tensor-core kernels (element (r, k) at
@@ -30,8 +33,7 @@ constexpr int INTER_T = 4096, INTER_AH = 8192, INTER_TT = 12288, INTER_REC = 163
 // for the state pass (64 x 64 tf32 each, K-major canonical layout,
 // (r, k) = T[r][k] and P[r][k]).
 constexpr unsigned FWR_T = 0, FWR_P = 16384, FWI_BYTES = 32768;
-constexpr int G_AH = 0, G_PA = 4096, G_QK = 12288, G_KED = 28672, G_DBR = 36864, G_DEL = 36928,
-              GREC = 37120;
+constexpr int GH_PA = 0, GH_QK = 8192, GH_KED = 24576, G_DBR = 16384, G_DEL = 16448, GREC = 16576;
 
 // Chunk geometry of the tensor-core kernels (Args: FwdArgs or BwdArgs).
 // Uniform batches: sequence s = batch row, NT = ceil(T / 64) chunks each, the
