@@ -498,6 +498,11 @@ constexpr uint32_t S2_Q = 0, S2_K = 16384, S2_C = 32768, S2_V = 65536, S2_KQ = 8
                    S2_TMEM = S2_CNT + 64, S2_BYTES = S2_TMEM + 16;
 static_assert(S2_BYTES + 1024 <= 233472, "one CTA per SM");
 constexpr int K2_THREADS = 544, CH0 = 32, CH_THREADS = 256, BU0 = 288, BU_THREADS = 256;
+// named barriers: 1 the chain warps, 2 the builder warps, 3 the issuer warp with the chain warps
+constexpr int BAR_STATE0 = 3;
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
 // TMEM columns: the state M^T (lane = value column n, column = key channel);
 // two [Y^T | O^T] accumulators (chunks alternate; Z^T is written over Y^T);
 // U^T
@@ -570,6 +575,8 @@ __global__ void __launch_bounds__(K2_THREADS, 1) kda_fwd_state_tc_kernel(const _
 
   if (warp == 0) {
     // ======================================================================== issuer warp
+    // no product before the chain has written the entering state into TMEM
+    named_sync(BAR_STATE0, 32 + CH_THREADS);
     if (lane == 0 && nch > 0) {
       const auto issue_v = [&](int ch) {
         mbar_expect_tx(bars + B_V, TILE_BF16);
@@ -642,7 +649,6 @@ __global__ void __launch_bounds__(K2_THREADS, 1) kda_fwd_state_tc_kernel(const _
     // ======================================================================== chain warps
     const int n = (warp & 3) * 32 + lane, hc = (warp - 1) >> 2;  // TMEM lane (value column), column half
     const uint32_t lo = (uint32_t)((warp & 3) * 32) << 16;
-    const SyncNamed csync{1, CH_THREADS};
     // o rows hc * 32 .. + 31 of chunk ch (value column n) from O^T in accumulator d: read
     // out, released to the issuer (B_O), then stored from registers (fp32 into o32 when
     // an output gate follows, else in the output dtype)
@@ -676,7 +682,7 @@ __global__ void __launch_bounds__(K2_THREADS, 1) kda_fwd_state_tc_kernel(const _
       tmem_wait_st();
     }
     fence_before();
-    csync();  // the state is in TMEM before anyone can arrive for the first products
+    named_sync(BAR_STATE0, 32 + CH_THREADS);  // the state is in TMEM before the issuer starts any product
     bool ok = true;
     for (int ch = 0; ch < nch; ++ch) {
       const uint32_t D = TM_D0 + (ch & 1) * 128, Dp = TM_D0 + ((ch + 1) & 1) * 128;
