@@ -92,6 +92,37 @@ __device__ __forceinline__ void cumsum64(float* a, float* seg, const float* base
 // One (chunk, quarter) with the CTA's 256 threads, shared memory at `smem`
 // (AsmSmem::bytes): chunk ch of batch row sq (packed sequences: chunk ch of
 // the table, sq = 0).  Ends with a barrier.
+// L2 prefetch of everything the four quarters of chunk ch of (sq, hv) read:
+// its gradient record, q and k rows of its key head, g rows, and Ah.
+template <typename TIn>
+__device__ __forceinline__ void prefetch_assembly(const BwdArgs& a, int ch, int hv, int sq) {
+  constexpr int KD = 128;
+  const int tid = threadIdx.x, G = a.HV / a.H, h = hv / G, b = row_of(a, sq);
+  const int2 sp = chunk_span(a, ch);
+  const size_t gc = chunk_gc(a, sq, hv, ch);
+  if (tid < 17) {  // GREC floats = 16 pieces of 4096 bytes + 768
+    const uint32_t bytes = tid < 16 ? 4096u : (uint32_t)(GREC * 4 - 16 * 4096);
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a.gws + gc * GREC + tid * 1024), "r"(bytes)
+                 : "memory");
+    return;
+  }
+  if (tid >= 20 && tid < 24) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a.inter + gc * INTER_REC + INTER_AH +
+                                                                    (tid - 20) * 1024),
+                 "r"(4096u)
+                 : "memory");
+    return;
+  }
+  const int i = tid & 63, which = tid >> 6;  // which 1: q, 2: k, 3: g
+  if (which == 0 || i >= sp.y) return;
+  const size_t t = (size_t)b * a.T + sp.x + i;
+  const void* p = which == 1   ? static_cast<const void*>(static_cast<const TIn*>(a.q) + (t * a.H + h) * KD)
+                  : which == 2 ? static_cast<const void*>(static_cast<const TIn*>(a.k) + (t * a.H + h) * KD)
+                               : static_cast<const void*>(a.g + (t * a.HV + hv) * KD);
+  const uint32_t bytes = which == 3 ? KD * 4 : KD * (uint32_t)sizeof(TIn);
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 template <typename TIn>
 __device__ __forceinline__ void assemble_quarter(const BwdArgs& a, float* smem, int ch, int fq4, int hv, int sq) {
   using S = AsmSmem;
@@ -145,8 +176,10 @@ __device__ __forceinline__ void assemble_quarter(const BwdArgs& a, float* smem, 
 #pragma unroll
     for (int m = 0; m < 4; ++m) {  // row i of [dP; dA], four columns j per item
       const int idx = tid + m * NTHREADS, i = idx >> 4, j4 = (idx & 15) * 4;
-      dp[m] = ld4h(rech + GH_PA + rec_off(i, j4, 64));
-      da[m] = ld4h(rech + GH_PA + rec_off(64 + i, j4, 64));
+      // only the lower triangle is used (dP: j <= i, dA: j < i): wholly upper pieces are not read
+      const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+      dp[m] = (j4 <= i) ? ld4h(rech + GH_PA + rec_off(i, j4, 64)) : z4;
+      da[m] = (j4 <= i) ? ld4h(rech + GH_PA + rec_off(64 + i, j4, 64)) : z4;
     }
     float bt[4];  // beta of the rows of the [dA] items
 #pragma unroll
@@ -194,7 +227,9 @@ __device__ __forceinline__ void assemble_quarter(const BwdArgs& a, float* smem, 
   }
   __syncthreads();
   cumsum64<false>(sC, sSeg, nullptr);
-  {  // element-wise terms; the chunk-end sum of dKEd o k o e^{c_last-c} goes through sE1
+  {  // element-wise terms; the chunk-end sum of dKEd o k o e^{c_last-c} over this warp's
+     // 8 rows goes to sSeg (warp w = rows 8w .. 8w + 7, lane = channel)
+    float send = 0.f;
 #pragma unroll
     for (int m = 0; m < 2; ++m) {
       const int f = ef, i4 = ei + 4 * m;
@@ -210,18 +245,13 @@ __device__ __forceinline__ void assemble_quarter(const BwdArgs& a, float* smem, 
         sDq[o] = dqe * e;
         sDk[o] = dke * e + dked * ed;
         sDc[o] = (dqe * qq + dke * kk) * e - dked * kk * ed;
-        sE1[o] = dked * kk * ed;
+        send += dked * kk * ed;
       }
     }
+    sSeg[(ei >> 3) * KQ + ef] = send;
   }
   __syncthreads();
   {  // chunk-end terms: dEl o e^{c_last} + sum_i dKEd o k o e^{c_last - c}
-    const int f = tid % KQ, sg = tid / KQ;
-    float s = 0.f;
-#pragma unroll
-    for (int r = 0; r < 8; ++r) s += sE1[(sg * 8 + r) * LDK + f];
-    sSeg[sg * KQ + f] = s;
-    __syncthreads();
     if (tid < KQ) {
       float t = rec[G_DEL + f0 + tid] * __expf(sC[(C - 1) * LDK + tid]);
       for (int s2 = 0; s2 < 8; ++s2) t += sSeg[s2 * KQ + tid];

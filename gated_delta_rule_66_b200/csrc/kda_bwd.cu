@@ -415,6 +415,16 @@ template <typename TIn>
 __global__ void __launch_bounds__(NTHREADS, 2) kda_bwd_assemble_kernel(BwdArgs a) {
   extern __shared__ float smem[];
   const int head = a.head0 + blockIdx.y;  // (sequence or batch row) * HV + hv
+  if (a.pf_items > 0 && (blockIdx.x & 3) == 0) {
+    // CTAs start in linear order, so the CTA that follows this one on its SM is
+    // about pf_items (a multiple of 4: all CTAs resident at once) further on:
+    // the chunk it and its three neighbours assemble goes into L2 now
+    const long long nx = (long long)blockIdx.y * gridDim.x + blockIdx.x + a.pf_items;
+    if (nx < (long long)gridDim.x * gridDim.y) {
+      const int hn = a.head0 + (int)(nx / gridDim.x);
+      prefetch_assembly<TIn>(a, (int)(nx % gridDim.x) >> 2, hn % a.HV, hn / a.HV);
+    }
+  }
   assemble_quarter<TIn>(a, smem, blockIdx.x >> 2, blockIdx.x & 3, head % a.HV, head / a.HV);
 }
 
@@ -427,6 +437,11 @@ static int launch_assemble(const BwdArgs& a0, int head0, int nheads, cudaStream_
   const int NT = a0.ctab ? a0.NC : (a0.T + 63) / 64;
   if (NT == 0 || nheads <= 0) return 0;  // (packed batches of empty sequences)
   BwdArgs a = a0;
+  int dev = 0, sms = 148, per_sm = 1;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, NTHREADS, AsmSmem::bytes) != cudaSuccess)
+    per_sm = 1;
+  a.pf_items = (sms * (per_sm > 0 ? per_sm : 1)) & ~3;
   for (int done = 0; done < nheads; done += 65535) {  // gridDim.y is at most 65535
     a.head0 = head0 + done;
     kern<<<dim3(NT * 4, min(nheads - done, 65535)), NTHREADS, AsmSmem::bytes, stream>>>(a);

@@ -601,7 +601,10 @@ static int launch_bwd_grads_tc(const BwdArgs& a, cudaStream_t stream) {
   const long long items = (a.item1 > 0 ? a.item1 : (long long)NT * a.HV * (a.ctab ? 1 : a.B)) - a.item0;
   if (items <= 0) return 0;
   // one CTA per item (not persistent): when the kernel shares the GPU with the
-  // state-gradient pass, the SMs that pass frees take the remaining items
+  // state-gradient pass, the SMs that pass frees take the remaining items.
+  // (An L2 prefetch of the inputs of the item one SM count further on, as
+  // the assembly does, measured 0.36 ms slower per fwd+bwd step at B = 2,
+  // H = 96, T = 4096.)
   kda_bwd_grads_tc_kernel<<<(int)items, tcc::NTH, tcc::SMEM_BYTES, stream>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return set_cuda_error("kda_bwd: tensor-core gradient launch", e);

@@ -133,6 +133,10 @@ struct BwdArgs {
   // covers heads (sequence * HV + hv) head0 .. head0 + its grid - 1, the
   // gradient kernel items item0 .. item1 - 1 (item1 <= 0: all)
   int head0, item0, item1;
+  // assembly: CTA i prefetches to L2 what CTA i + pf_items (a multiple of 4,
+  // the CTAs resident at once: most likely its successor on the SM) reads
+  // (0: none)
+  int pf_items;
 };
 
 struct DecodeArgs {
