@@ -556,13 +556,16 @@ def run_gpu(args):
     from gated_delta_rule_66_b200 import kda
     peaks = load_peaks()
     results = {}
-    for name in [HEADLINE] + [p for p in PATHS if p != HEADLINE and args.all_paths]:
+    chosen = None if args.paths is None else set(args.paths.split(","))
+    others = [p for p in PATHS if p != HEADLINE and args.all_paths and (chosen is None or p in chosen)]
+    for name in [HEADLINE] + others:
         if name == HEADLINE:
             with Clocks(local) as clk:
                 res, w = gpu_path(kda, name, args.steps, args.warmup, barrier, args.shrink)
             res["clocks"] = clk.summary()
-        else:
-            res, w = gpu_path(kda, name, args.steps, args.warmup, barrier)
+        else:  # (--shrink B,T reduces the decode batch to B as well)
+            small = (args.shrink[0], 1) if args.shrink and name == "decode" else None
+            res, w = gpu_path(kda, name, args.steps, args.warmup, barrier, small)
         if "roofline" not in res:
             res["roofline"] = roofline_for(res, w, peaks)
         def reduce_max(x):
@@ -762,6 +765,8 @@ def main():
     ap.add_argument("--shrink", type=lambda x: tuple(int(v) for v in x.split(",")), default=None,
                     metavar="B,T", help="run the headline workload at batch B and length T (for ncu captures; "
                                         "the printed line is not a headline number)")
+    ap.add_argument("--paths", default=None, metavar="NAME,...",
+                    help="the other paths to run after the headline (default: all of them)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
