@@ -563,8 +563,9 @@ def run_gpu(args):
             with Clocks(local) as clk:
                 res, w = gpu_path(kda, name, args.steps, args.warmup, barrier, args.shrink)
             res["clocks"] = clk.summary()
-        else:  # (--shrink B,T reduces the decode batch to B as well)
-            small = (args.shrink[0], 1) if args.shrink and name == "decode" else None
+        else:  # (--shrink B,T[,BD] reduces the decode batch to BD, else B, as well)
+            small = (args.shrink[-1] if len(args.shrink) > 2 else args.shrink[0], 1) \
+                if args.shrink and name == "decode" else None
             res, w = gpu_path(kda, name, args.steps, args.warmup, barrier, small)
         if "roofline" not in res:
             res["roofline"] = roofline_for(res, w, peaks)
@@ -763,8 +764,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--headline-only", dest="all_paths", action="store_false")
     ap.add_argument("--shrink", type=lambda x: tuple(int(v) for v in x.split(",")), default=None,
-                    metavar="B,T", help="run the headline workload at batch B and length T (for ncu captures; "
-                                        "the printed line is not a headline number)")
+                    metavar="B,T[,BD]", help="run the headline workload at batch B and length T and the decode "
+                                             "path at batch BD (default B) (for ncu captures; the printed line "
+                                             "is not a headline number)")
     ap.add_argument("--paths", default=None, metavar="NAME,...",
                     help="the other paths to run after the headline (default: all of them)")
     args = ap.parse_args()
