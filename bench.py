@@ -217,7 +217,7 @@ def gpu_prep_path(kda, name, steps, warmup, rank_barrier):
             kda.fwd_prep(d["q"], d["k"], d["v"], d["z"], d["A_log"], d["dt_bias"], d["beta_logit"], scale=w.scale,
                          out_gate=d["og"], workspace=ws)
         tokens, launches = w.B * w.T, 4
-        kernel = "kda_fwd_prep (kda_prep_gate_kernel + kda_fwd_intra_tc_kernel<1> + kda_fwd_state_tc_kernel<1> + kda_out_gate_kernel, one call)"
+        kernel = "kda_fwd_prep (kda_prep_gate_kernel + kda_fwd_intra_tc_kernel<1> + kda_fwd_state_tc_kernel<1> + kda_out_gate4_kernel, one call)"
         flush = None
     else:
         r = make_raw_inputs(w.with_sizes(T=1), conv_width=CONV_W)

@@ -225,11 +225,9 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_dstate_tc_kernel(BwdArgs a) {
       commit(bar);
     }
     {
-      float* dst = a.dstates + (dstate_slot(a, sq, hv, ch) * KD + hcol * 64) * VD + Lr;
-#pragma unroll
-      for (int cb = 0; cb < 2; ++cb)
-#pragma unroll
-        for (int j = 0; j < 32; ++j) dst[(size_t)(cb * 32 + j) * VD] = sv[cb][j];
+      float* slot = a.dstates + dstate_slot(a, sq, hv, ch) * (KD * VD);
+      store_slot32(slot, hcol * 2, Lr, sv[0]);
+      store_slot32(slot, hcol * 2 + 1, Lr, sv[1]);
     }
     if (!wait_mma(bar, phase)) { failed = true; break; }
     fence_before();
@@ -391,8 +389,8 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
       const int i = x >> 4, c16 = x & 15;
       cp_async16(sb + OP_V + x * 16, vg + (((size_t)b * T + t0 + (i < L ? i : 0)) * a.HV + hv) * VD + c16 * 8, i < L);
     }
-    if (tid < 16) prefetch_l2(mst + tid * 1024, 4096);
-    else if (tid < 32) prefetch_l2(dmst + (tid - 16) * 1024, 4096);
+    if (tid < 9) prefetch_l2(mst + tid * 1024, tid < 8 ? 4096 : 2048);  // (fp16 values and their scales)
+    else if (tid >= 16 && tid < 25) prefetch_l2(dmst + (tid - 16) * 1024, tid < 24 ? 4096 : 2048);
     else if (tid == 32) prefetch_l2(irec, 2 * 16384);
     else if (tid == 33) prefetch_l2(irec + INTER_TT, 16384);
     if (!load_raw_wait(cx)) { failed = true; break; }
@@ -440,15 +438,14 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
       for (int cb = 0; cb < 2; ++cb) {
         const int f0 = hcol * 64 + cb * 32;
         uint32_t rm[32], rd[32];
-        float pr[32];
-        const float* ms = mst + f0 * VD + Lr;
-        const float* ds = dmst + f0 * VD + Lr;
+        float pr[32], mv[32], dv[32];
+        load_slot32(mst, f0 / 32, Lr, mv);
+        load_slot32(dmst, f0 / 32, Lr, dv);
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          const float mv = ms[(size_t)j * VD], dv = ds[(size_t)j * VD];
-          rm[j] = __float_as_uint(mv);
-          rd[j] = __float_as_uint(dv);
-          pr[j] = mv * dv;
+          rm[j] = __float_as_uint(mv[j]);
+          rd[j] = __float_as_uint(dv[j]);
+          pr[j] = mv[j] * dv[j];
         }
         tmem_st32(tm + lo + TM_M + f0, rm);
         tmem_st32(tm + lo + TM_DM + f0, rd);

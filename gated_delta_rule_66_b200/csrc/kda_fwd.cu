@@ -698,10 +698,61 @@ __global__ void __launch_bounds__(256) kda_out_gate_kernel(const float* __restri
   }
 }
 
+// The same for V = 128 with four consecutive values per lane: one 16-byte
+// load of o32 and one 8-byte (bf16) or 16-byte (fp32) load of og and store
+// of o per lane and row.
+template <typename TIn>
+__global__ void __launch_bounds__(256) kda_out_gate4_kernel(const float* __restrict__ o32,
+                                                            const TIn* __restrict__ og, float eps, size_t rows,
+                                                            TIn* __restrict__ o) {
+  const size_t row = (size_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const size_t e0 = row * 128 + 4 * lane;
+  const float4 x = *reinterpret_cast<const float4*>(o32 + e0);
+  float gv[4];
+  if constexpr (sizeof(TIn) == 2) {
+    const uint2 r = *reinterpret_cast<const uint2*>(og + e0);
+    const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&r.x);
+    const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&r.y);
+    gv[0] = __low2float(lo); gv[1] = __high2float(lo); gv[2] = __low2float(hi); gv[3] = __high2float(hi);
+  } else {
+    const float4 r = *reinterpret_cast<const float4*>(og + e0);
+    gv[0] = r.x; gv[1] = r.y; gv[2] = r.z; gv[3] = r.w;
+  }
+  float s = fmaf(x.x, x.x, fmaf(x.y, x.y, fmaf(x.z, x.z, x.w * x.w)));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+  const float inv = rsqrtf(s / 128.f + eps);
+  const float y[4] = {x.x * inv * prep_sigmoid(gv[0]), x.y * inv * prep_sigmoid(gv[1]),
+                      x.z * inv * prep_sigmoid(gv[2]), x.w * inv * prep_sigmoid(gv[3])};
+  if constexpr (sizeof(TIn) == 2) {
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(y[0], y[1]), hi = __floats2bfloat162_rn(y[2], y[3]);
+    uint2 r;
+    r.x = *reinterpret_cast<const uint32_t*>(&lo);
+    r.y = *reinterpret_cast<const uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(o + e0) = r;
+  } else {
+    *reinterpret_cast<float4*>(o + e0) = make_float4(y[0], y[1], y[2], y[3]);
+  }
+}
+
 int launch_out_gate(const float* o32, const void* og, float eps, size_t rows, int V, int dtype, void* o,
                     cudaStream_t stream) {
   if (rows == 0) return 0;
   const unsigned blocks = (unsigned)((rows + 7) / 8);
+  const size_t al = (size_t)o32 | (size_t)og | (size_t)o;
+  if (V == 128 && (al & 15) == 0) {
+    if (dtype == 1)
+      kda_out_gate4_kernel<__nv_bfloat16><<<blocks, 256, 0, stream>>>(
+          o32, static_cast<const __nv_bfloat16*>(og), eps, rows, static_cast<__nv_bfloat16*>(o));
+    else
+      kda_out_gate4_kernel<float><<<blocks, 256, 0, stream>>>(o32, static_cast<const float*>(og), eps, rows,
+                                                              static_cast<float*>(o));
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return set_cuda_error("kda_fwd: output-gate launch", e);
+    return 0;
+  }
   if (dtype == 1)
     kda_out_gate_kernel<__nv_bfloat16><<<blocks, 256, 0, stream>>>(
         o32, static_cast<const __nv_bfloat16*>(og), eps, rows, V, static_cast<__nv_bfloat16*>(o));

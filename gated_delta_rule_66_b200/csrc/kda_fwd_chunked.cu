@@ -705,18 +705,14 @@ __global__ void __launch_bounds__(K2_THREADS, 1) kda_fwd_state_tc_kernel(const _
       // M^T <- M^T diag(e^{c_last}), storing the entering state for the backward
       if (!(ok = role_wait(bars + B_KD, par, polls, abort, 1, CH_THREADS))) break;
       {
-        float* dst = a.states ? a.states + state_slot(a, sq, hv, c0 + ch) * (KD * VD) + (size_t)(hc * 64) * VD + n
-                              : nullptr;
+        float* slot = a.states ? a.states + state_slot(a, sq, hv, c0 + ch) * (KD * VD) : nullptr;
         const float* el = sEl + hc * 64;
 #pragma unroll 1
         for (int cb = 0; cb < 2; ++cb) {
           float sv[32];
           uint32_t r[32];
           tmem_ld32(tm + lo + TM_S + hc * 64 + cb * 32, sv);
-          if (dst) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) dst[(size_t)(cb * 32 + j) * VD] = sv[j];
-          }
+          if (slot) store_slot32(slot, hc * 2 + cb, n, sv);
 #pragma unroll
           for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(sv[j] * el[cb * 32 + j]);
           tmem_st32(tm + lo + TM_S + hc * 64 + cb * 32, r);

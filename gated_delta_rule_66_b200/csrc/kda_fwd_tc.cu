@@ -294,11 +294,8 @@ __global__ void __launch_bounds__(256, 1) kda_fwd_tc_kernel(FwdArgs a) {
         const int f0 = hcol * 64 + cb * 32;
         float s[32];
         tmem_ld32(tm + lo + TM_S + f0, s);
-        if (a.states) {  // the state entering this chunk
-          float* dst = a.states + (state_slot(a, sq, hv, sc.c0 + ch) * KD + f0) * VD + Lr;
-#pragma unroll
-          for (int j = 0; j < 32; ++j) dst[(size_t)j * VD] = s[j];
-        }
+        if (a.states)  // the state entering this chunk
+          store_slot32(a.states + state_slot(a, sq, hv, sc.c0 + ch) * (KD * VD), f0 / 32, Lr, s);
 #pragma unroll
         for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(s[j] * sEl[f0 + j]);
         tmem_st32(tm + lo + TM_S + f0, r);

@@ -25,6 +25,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "kda_chunk.cuh"
 #include "kda_tc.cuh"
@@ -45,6 +46,36 @@ constexpr float LOG2E = 1.4426950408889634f;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 static_assert(R_T + 16384 <= OP && R_P + 16384 <= R_T && R_SW + 3072 <= R_P && R_WOP + 36864 <= R_P,
               "raw-region reuse (the padded W overlaps only the dead inverse scratch)");
+
+// A K x V state (or state gradient) slot of the tensor-core path, in its 64 KB
+// fp32 slot of the state layout: the values [f][n] as fp16 (32 KB), then one
+// power-of-two scale per value column n and group of 32 key channels
+// ([4][128] floats at float offset SLOT_SCALES): x = half(x / s) * s.  The
+// scale puts the group's largest magnitude in [2^14, 2^15), so every value
+// keeps fp16's 11 significant bits (what the tf32 products read anyway:
+// 10 stored mantissa bits) whatever the state's range; values below 2^-29 of
+// the group's largest lose bits.  Half the bytes of the fp32 slot.
+constexpr int SLOT_SCALES = KD * VD / 2;
+// one thread's 32 values of column n, channels 32 grp .. 32 grp + 31
+__device__ __forceinline__ void store_slot32(float* slot, int grp, int n, const float (&v)[32]) {
+  float m = 0.f;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) m = fmaxf(m, fabsf(v[j]));
+  // m < 2^ex (ex from the exponent field; 0 and subnormal m give the clamp)
+  const int ex = ((__float_as_int(m) >> 23) & 0xff) - 126;
+  const int e = min(126, max(-126, 15 - ex));
+  const float up = __int_as_float((127 + e) << 23);
+  __half* h = reinterpret_cast<__half*>(slot) + (size_t)(32 * grp) * VD + n;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) h[(size_t)j * VD] = __float2half_rn(v[j] * up);
+  slot[SLOT_SCALES + grp * VD + n] = __int_as_float((127 - e) << 23);
+}
+__device__ __forceinline__ void load_slot32(const float* slot, int grp, int n, float (&v)[32]) {
+  const __half* h = reinterpret_cast<const __half*>(slot) + (size_t)(32 * grp) * VD + n;
+  const float s = slot[SLOT_SCALES + grp * VD + n];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = __half2float(h[(size_t)j * VD]) * s;
+}
 
 // byte offset of bf16 element (row i, channel f) in a raw q / k / x tile:
 // the 16-byte pieces of row i are stored XOR-swizzled by i % 8, so that one
