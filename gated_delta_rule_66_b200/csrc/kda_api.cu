@@ -155,7 +155,8 @@ int kda_device_status(unsigned* flags) {
 
 int kda_set_wait_polls(unsigned polls) {
   g_err[0] = 0;
-  return set_wait_polls(polls);
+  const int rc = set_wait_polls(polls);
+  return rc ? rc : set_bwd_wait_polls(polls);
 }
 
 size_t kda_fwd_workspace_bytes(int B, int T, int HV, int K, int V) {

@@ -29,16 +29,6 @@ namespace kda {
 
 __device__ unsigned int g_kda_bwd_device_error;  // this file's kernels (one flag per translation unit)
 
-namespace tcb {
-using namespace tcc;
-constexpr uint32_t OP_KED = OP, OP_QET = OP + 32768, OP_NKET = OP + 65536;
-// the chunk's P^T and T^T images, above the operands (the raw region then
-// takes the next chunk's rows while this chunk's products run)
-constexpr uint32_t IMG_PT = OP + 98304, IMG_TT = OP + 114688;
-static_assert(IMG_TT + 16384 <= SMALL, "state-gradient shared-memory map");
-constexpr uint32_t TM_S = 0, TM_DU = 128, TM_DR = 192, TM_DOT = 256;
-}  // namespace tcb
-
 // four fp32 values rounded to fp16 into 8 bytes of shared memory
 __device__ __forceinline__ void st4h(__half* p, const float* v) {
   const __half2 lo = __floats2half2_rn(v[0], v[1]), hi = __floats2half2_rn(v[2], v[3]);
@@ -47,208 +37,329 @@ __device__ __forceinline__ void st4h(__half* p, const float* v) {
   u.y = *reinterpret_cast<const unsigned*>(&hi);
   *reinterpret_cast<uint2*>(p) = u;
 }
-__global__ void __launch_bounds__(256, 1) kda_bwd_dstate_tc_kernel(BwdArgs a) {
-  using namespace tcb;
+// Warp-specialised, 544 threads (17 warps), one CTA per (sequence, value head):
+//   issuer warp 0 (lane 0): the three products of every chunk and the P^T,
+//     T^T image copies (a tcgen05.mma issue holds its thread for about the
+//     product's duration, so this warp does nothing else);
+//   chain warps 1-8 (TMEM lanes 32 (w % 4) .., lane = value column n; column
+//     half (w - 1) / 4): the state gradient's decay in TMEM, storing the
+//     gradient leaving every chunk on the way;
+//   builder warps 9-16: the decay and the chunk's operands K o e^{c_last-c}
+//     as [i][f], (Q~ o e^c)^T and -(diag(beta) K o e^c)^T as [f][i],
+//     e^{c_last}, and dO^T into one of two TMEM buffers, the next chunk's
+//     while this chunk's products run;
+//   loader warp 17 (lane 0): the next chunk's q, k, dO and g tiles by TMA
+//     once the builders are done with the current ones, and the chunk after
+//     next into L2 (a TMA issue can hold its thread for a while).
+// Per chunk (in reverse): dU^T (waits for the previous chunk's state
+// product), dR^T = dU^T T, then dM^T <- dM^T diag(e^{c_last}) + dO^T (Q~ o
+// e^c) - dR^T (diag(beta) K o e^c) once the chain has decayed dM^T.  Every wait
+// is bounded (g_kda_bwd_wait_polls probes); one that gives up sets the
+// shared abort word, which ends the other roles' waits too.
+namespace tcd {
+using namespace tcc;
+constexpr int D_THREADS = 576, D_CH = 256, D_BU0 = 288, D_BU = 256, D_LD0 = 544;
+constexpr uint32_t D_KED = OP, D_QET = OP + 32768, D_NKET = OP + 65536, D_PT = OP + 98304, D_TT = OP + 114688,
+                   D_BAR = OP + 131072, D_CNT = D_BAR + 128;
+static_assert(D_CNT + 64 <= SMALL, "state-gradient shared-memory map");
+// TMEM columns: dM^T, dU^T, dR^T, two dO^T buffers (chunks alternate), and the
+// chain's copy of the gradient leaving the chunk (stored after the decay is released)
+constexpr uint32_t DT_S = 0, DT_DU = 128, DT_DR = 192, DT_DOT = 256, DT_COPY = 384;
+enum { DB_RAW, DB_P, DB_T, DB_DU, DB_DR, DB_S, DNB_ASYNC, DB_KED = DNB_ASYNC, DB_QN, DB_RS, DNB_ALL };
+// named barriers: 1 the chain warps, 2 the builder warps, 3 the issuer warp with the chain warps
+constexpr int DBAR_CH = 1, DBAR_BU = 2, DBAR_S0 = 3;
+}  // namespace tcd
+
+__device__ unsigned int g_kda_bwd_wait_polls = 1u << 24;
+
+__global__ void __launch_bounds__(tcd::D_THREADS, 1) kda_bwd_dstate_tc_kernel(const __grid_constant__ RawMaps4 maps,
+                                                                              BwdArgs a) {
+  using namespace tcd;
   using namespace tc;
   extern __shared__ __align__(1024) unsigned char sm[];
-  Ctx cx;
-  cx.sm = sm;
-  cx.sb = smem_u32(sm);
-  cx.tid = threadIdx.x;
-  cx.warp = cx.tid >> 5;
-  cx.lane = cx.tid & 31;
-  cx.sub = cx.warp & 3;
-  cx.hcol = cx.warp >> 2;
-  cx.Lr = cx.sub * 32 + cx.lane;
-  cx.lo = (uint32_t)(cx.sub * 32) << 16;
-  const int tid = cx.tid, hcol = cx.hcol, Lr = cx.Lr;
-  const uint32_t lo = cx.lo, sb = cx.sb;
-
+  const uint32_t sb = smem_u32(sm);
+  if (sb & 1023u) {  // the 128-byte swizzle of the TMA tiles needs a 1024-byte aligned base
+    if (threadIdx.x == 0) atomicOr(&g_kda_bwd_device_error, 2u);
+    return;
+  }
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int head_ = a.head0 + blockIdx.x;
   const int hv = head_ % a.HV, sq = head_ / a.HV;  // batch row, or sequence of a packed batch
-  const int b = row_of(a, sq), c0 = chunk_begin(a, sq), c1 = chunk_end(a, sq);
+  const int b = row_of(a, sq), c0 = chunk_begin(a, sq), c1 = chunk_end(a, sq), nch = c1 - c0;
   const int G = a.HV / a.H, h = hv / G, T = a.T;
   const size_t head = (size_t)sq * a.HV + hv;
-  const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(a.q);
-  const __nv_bfloat16* kg = static_cast<const __nv_bfloat16*>(a.k);
-  const __nv_bfloat16* dog = static_cast<const __nv_bfloat16*>(a.dO);
-  float* sBeta = cx.beta();
-  float* sEl = reinterpret_cast<float*>(sm + S_EL);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + S_BAR);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + D_BAR);
+  int* cnt = reinterpret_cast<int*>(sm + D_CNT);  // issued phases per async barrier; [15]: abort
+  volatile int* abort = cnt + 15;
   uint32_t* sTm = reinterpret_cast<uint32_t*>(sm + S_TMEM);
-  const float* sC = cx.c();
+  float* sEl = reinterpret_cast<float*>(sm + S_EL);
+  unsigned char* tC = sm + RAW_C;  // g, then the cumulative decay (fp32 TMA tile)
+  const uint32_t polls = g_kda_bwd_wait_polls;
 
-  if (cx.warp == 0) tmem_alloc(sTm, 512);
-  if (tid == 0) mbar_init(bar, 1);
+  if (warp == 0) tmem_alloc(sTm, 512);
+  if (tid == 0) {
+    for (int i = 0; i < DNB_ALL; ++i) mbar_init(bars + i, i < DNB_ASYNC ? 1 : (i == DB_RS ? D_CH : D_BU));
+    for (int i = 0; i < 16; ++i) cnt[i] = 0;
+  }
   fence_before();
   __syncthreads();
   fence_after();
   const uint32_t tm = *sTm;
-  cx.tm = tm;
-  uint32_t phase = 0;
-  bool failed = false;
+  const auto irec = [&](int ch) { return a.inter + chunk_gc(a, sq, hv, ch) * INTER_REC; };
 
-  {  // gradient of the final state, transposed
-    for (int cb = 0; cb < 2; ++cb) {
-      const int f0 = hcol * 64 + cb * 32;
+  if (warp == 0) {
+    // ======================================================================== issuer warp
+    named_sync(DBAR_S0, 32 + D_CH);  // the final state's gradient is in TMEM
+    if (lane == 0 && nch > 0) {
+      const auto issue_img = [&](int which, uint32_t dst, const float* src) {
+        mbar_expect_tx(bars + which, 16384);
+        bulk_g2s(dst, src, 16384, bars + which);
+        ++cnt[which];
+      };
+      const auto commit_to = [&](int which) {
+        commit(bars + which);
+        ++cnt[which];
+      };
+      issue_img(DB_P, sb + D_PT, irec(c1 - 1));             // P^T: (row i, K j) = P[j][i]
+      issue_img(DB_T, sb + D_TT, irec(c1 - 1) + INTER_TT);  // T^T: (row i, K j) = T[j][i]
+      for (int k = 0; k < nch; ++k) {
+        const int ch = c1 - 1 - k;
+        const uint32_t par = k & 1, dot = DT_DOT + (k & 1) * 64;
+        // dU^T = dO^T P + dM^T (K o e^{c_last-c})^T, dM^T the gradient leaving this chunk
+        if (!wait_one(bars + DB_KED, par, polls, abort)) break;
+        if (!wait_one(bars + DB_P, par, polls, abort)) break;
+        if (k > 0 && !wait_one(bars + DB_S, par ^ 1, polls, abort)) break;
+        fence_after();
+        for (int ks = 0; ks < 8; ++ks)
+          mma_ts(tm + DT_DU, tm + dot + ks * 8, desc(sb + D_PT + ks * 256, 2048), idesc_tf32(128, 64), ks > 0);
+        for (int ks = 0; ks < 16; ++ks)
+          mma_ts(tm + DT_DU, tm + DT_S + ks * 8, desc(sb + D_KED + ks * 256, 4096), idesc_tf32(128, 64), 1);
+        commit_to(DB_DU);
+        if (!wait_one(bars + DB_DU, par, polls, abort)) break;
+        if (k + 1 < nch) issue_img(DB_P, sb + D_PT, irec(ch - 1));  // this chunk's P^T is consumed
+        // dR^T = dU^T T
+        if (!wait_one(bars + DB_T, par, polls, abort)) break;
+        fence_after();
+        for (int ks = 0; ks < 8; ++ks)
+          mma_ts(tm + DT_DR, tm + DT_DU + ks * 8, desc(sb + D_TT + ks * 256, 2048), idesc_tf32(128, 64), ks > 0);
+        commit_to(DB_DR);
+        if (!wait_one(bars + DB_DR, par, polls, abort)) break;
+        if (k + 1 < nch) issue_img(DB_T, sb + D_TT, irec(ch - 1) + INTER_TT);
+        // dM^T += dO^T (Q~ o e^c) - dR^T (diag(beta) K o e^c) once the chain has decayed dM^T
+        if (!wait_one(bars + DB_QN, par, polls, abort)) break;
+        if (!wait_one(bars + DB_RS, par, polls, abort)) break;
+        fence_after();
+        for (int ks = 0; ks < 8; ++ks) {
+          mma_ts(tm + DT_S, tm + dot + ks * 8, desc(sb + D_QET + ks * 256, 2048), idesc_tf32(128, 128), 1);
+          mma_ts(tm + DT_S, tm + DT_DR + ks * 8, desc(sb + D_NKET + ks * 256, 2048), idesc_tf32(128, 128), 1);
+        }
+        commit_to(DB_S);
+      }
+    }
+    __syncwarp();
+  } else if (warp <= 8) {
+    // ======================================================================== chain warps
+    const int n = (warp & 3) * 32 + lane, hc = (warp - 1) >> 2;  // TMEM lane (value column), column half
+    const uint32_t lo = (uint32_t)((warp & 3) * 32) << 16;
+    for (int cb = 0; cb < 2; ++cb) {  // gradient of the final state, transposed
+      const int f0 = hc * 64 + cb * 32;
       uint32_t r[32];
 #pragma unroll
-      for (int j = 0; j < 32; ++j)
-        r[j] = __float_as_uint(a.dS_T ? a.dS_T[(head * KD + f0 + j) * VD + Lr] : 0.f);
-      tmem_st32(tm + lo + TM_S + f0, r);
+      for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(a.dS_T ? a.dS_T[(head * KD + f0 + j) * VD + n] : 0.f);
+      tmem_st32(tm + lo + DT_S + f0, r);
     }
     tmem_wait_st();
-  }
-  fence_before();
-  __syncthreads();
-
-  // Copies run one chunk ahead, in cp.async groups committed in the order
-  // raw(c1-1), images(c1-1), raw(c1-2), images(c1-2), ...: a chunk's raw rows
-  // are requested once the previous chunk's rows are consumed, its images
-  // once the previous chunk's products have read theirs.
-  if (c1 > c0) {
-    const int2 sp = chunk_span(a, c1 - 1);
-    load_raw_issue<NTH, true>(cx, qg, kg, dog, a.g, a.beta, b, T, sp.x, sp.y, a.H, a.HV, h, hv);
-    cp_async_commit();
-    const float* irec = a.inter + chunk_gc(a, sq, hv, c1 - 1) * INTER_REC;
-    copy_image(cx, IMG_PT, irec);             // P^T: (row i, K j) = P[j][i]
-    copy_image(cx, IMG_TT, irec + INTER_TT);  // T^T: (row i, K j) = T[j][i]
-    cp_async_commit();
-  }
-  for (int ch = c1 - 1; ch >= c0; --ch) {
-    cp_async_wait_group<1>();  // this chunk's raw rows (its images may still be in flight)
-    __syncthreads();
-    cumsum_span(cx);
-
-    // ---------------------------------------------------------------- operands of the gradient products
-    {
-      {  // K o e^{c_last-c} as [i][f]: thread items of 4 channels, 16-byte stores
-        const int fq = item_f(cx);
-        const float4 c63v = ld4(sC + 63 * LDCF + fq);
-        const float c63[4] = {c63v.x, c63v.y, c63v.z, c63v.w};
-        for (int m = 0; m < 8; ++m) {
-          const int i = item_row(cx, m);
-          const float4 c4 = ld4(sC + i * LDCF + fq);
-          float kf[4];
-          bf16x4(sm + RAW_K + raw_off(i, fq), kf);
-          st_tf32x4(sm, OP_KED + kmaj(i, fq, 128), kf[0] * ex2(c63[0] - c4.x), kf[1] * ex2(c63[1] - c4.y),
-                    kf[2] * ex2(c63[2] - c4.z), kf[3] * ex2(c63[3] - c4.w));
+    fence_before();
+    named_sync(DBAR_S0, 32 + D_CH);
+    bool ok = true;
+    for (int k = 0; k < nch; ++k) {
+      const int ch = c1 - 1 - k;
+      const uint32_t par = k & 1;
+      // the gradient leaving this chunk: stored, then decayed by e^{c_last} once dU^T has read it
+      if (!(ok = role_wait(bars + DB_DU, par, polls, abort, DBAR_CH, D_CH))) break;
+      if (!(ok = role_wait(bars + DB_QN, par, polls, abort, DBAR_CH, D_CH))) break;
+      fence_after();
+#pragma unroll 1
+      for (int cb = 0; cb < 2; ++cb) {
+        const int f0 = hc * 64 + cb * 32;
+        float sv[32];
+        uint32_t r[32];
+        tmem_ld32(tm + lo + DT_S + f0, sv);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(sv[j]);
+        tmem_st32(tm + lo + DT_COPY + f0, r);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(sv[j] * sEl[f0 + j]);
+        tmem_st32(tm + lo + DT_S + f0, r);
+      }
+      tmem_wait_st();
+      fence_before();
+      mbar_arrive(bars + DB_RS);
+      // the gradient leaving this chunk to the workspace, while the state product runs
+      float* slot = a.dstates + dstate_slot(a, sq, hv, ch) * (KD * VD);
+#pragma unroll 1
+      for (int cb = 0; cb < 2; ++cb) {
+        float sv[32];
+        tmem_ld32(tm + lo + DT_COPY + hc * 64 + cb * 32, sv);
+        store_slot32(slot, hc * 2 + cb, n, sv);
+      }
+    }
+    if (ok && a.dS0 && (nch == 0 || role_wait(bars + DB_S, (nch - 1) & 1, polls, abort, DBAR_CH, D_CH))) {
+      fence_after();
+      for (int cb = 0; cb < 2; ++cb) {
+        const int f0 = hc * 64 + cb * 32;
+        float sv[32];
+        tmem_ld32(tm + lo + DT_S + f0, sv);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) a.dS0[(head * KD + f0 + j) * VD + n] = sv[j];
+      }
+    }
+  } else if (warp < D_LD0 / 32) {
+    // ======================================================================== builder warps
+    const int bt = tid - D_BU0;  // 0 .. 255
+    Ctx cx;  // the builders' view: thread index bt
+    cx.sm = sm;
+    cx.sb = sb;
+    cx.tid = bt;
+    float* sBeta = cx.beta();
+    float* sCarry = reinterpret_cast<float*>(sm + S_CARRY);
+    const int n = (warp & 3) * 32 + lane, hb = (warp - 9) >> 2;  // dO^T: TMEM lane n, columns 32 hb ..
+    const uint32_t lo = (uint32_t)((warp & 3) * 32) << 16;
+    // beta (HV floats apart per step, which no tensor map addresses) goes through the
+    // registers of 64 threads
+    const auto beta_of = [&](int ch) {
+      const int2 sp = chunk_span(a, ch);
+      return bt < sp.y ? a.beta[((size_t)b * T + sp.x + bt) * a.HV + hv] : 0.f;
+    };
+    float bval = 0.f;
+    if (nch > 0 && bt < C) bval = beta_of(c1 - 1);
+    for (int k = 0; k < nch; ++k) {
+      const int ch = c1 - 1 - k, L = chunk_span(a, ch).y;
+      const uint32_t par = k & 1, dot = DT_DOT + (k & 1) * 64;
+      if (!role_wait(bars + DB_RAW, par, polls, abort, DBAR_BU, D_BU)) break;
+      if (bt < C) sBeta[bt] = bval;
+      if (L < C) {  // rows past the sequence (a packed batch's next sequence) count as zero
+        for (int x = bt; x < (C - L) * 16; x += D_BU) {  // 16-byte pieces of the bf16 rows
+          const int i = L + (x >> 4), p = x & 15;
+          const uint32_t o = (uint32_t)((p >> 3) * 8192 + i * 128 + (((p & 7) ^ (i & 7)) << 4));
+          const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+          *reinterpret_cast<uint4*>(sm + RAW_Q + o) = z;
+          *reinterpret_cast<uint4*>(sm + RAW_K + o) = z;
+          *reinterpret_cast<uint4*>(sm + RAW_X + o) = z;
+        }
+        for (int x = bt; x < (C - L) * 32; x += D_BU) {  // and of the fp32 g rows
+          const int i = L + (x >> 5), p = x & 31;
+          *reinterpret_cast<uint4*>(tC + (p >> 3) * 8192 + i * 128 + (((p & 7) ^ (i & 7)) << 4)) =
+              make_uint4(0u, 0u, 0u, 0u);
         }
       }
-      {  // (Q~ o e^c)^T and -(diag(beta) K o e^c)^T as [f][i]: one channel x 4 rows, 16-byte stores
-        const int f = tid & 127;
+      named_sync(DBAR_BU, D_BU);
+      {  // cumulative decay (times log2 e) in place: channel bt % 128, rows 32 (bt / 128) ..
+        const int f = bt & 127, hh = bt >> 7;
+        float v[32], run = 0.f;
+#pragma unroll
+        for (int r = 0; r < 32; ++r) {
+          run += ldf(tC, hh * 32 + r, f);
+          v[r] = run;
+        }
+        if (hh == 0) sCarry[f] = run;
+        named_sync(DBAR_BU, D_BU);
+        const float carry = hh ? sCarry[f] : 0.f;
+#pragma unroll
+        for (int r = 0; r < 32; ++r) *reinterpret_cast<float*>(tC + ft_off(hh * 32 + r, f)) = (v[r] + carry) * LOG2E;
+        named_sync(DBAR_BU, D_BU);
+      }
+      // K o e^{c_last-c} as [i][f] and dO^T: free once the previous chunk's dU^T is done
+      if (k > 0 && !role_wait(bars + DB_DU, par ^ 1, polls, abort, DBAR_BU, D_BU)) break;
+      {
+        const int fq = item_f<D_BU>(cx);
+        const float4 c63v = *reinterpret_cast<const float4*>(tC + ft_off(63, fq));
+        const float c63[4] = {c63v.x, c63v.y, c63v.z, c63v.w};
         for (int m = 0; m < 8; ++m) {
-          const int i0 = ((tid >> 7) + 2 * m) * 4;
+          const int i = item_row<D_BU>(cx, m);
+          const float4 c4 = *reinterpret_cast<const float4*>(tC + ft_off(i, fq));
+          float kf[4];
+          bf16x4(sm + RAW_K + bt_off(i, fq), kf);
+          st_tf32x4(sm, D_KED + kmaj(i, fq, 128), kf[0] * ex2(c63[0] - c4.x), kf[1] * ex2(c63[1] - c4.y),
+                    kf[2] * ex2(c63[2] - c4.z), kf[3] * ex2(c63[3] - c4.w));
+        }
+        uint32_t r[32];  // dO^T: lane n, columns j = 32 hb ..
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) r[jj] = tf32_rna(ldb(sm + RAW_X, hb * 32 + jj, n));
+        tmem_st32(tm + lo + dot + hb * 32, r);
+        tmem_wait_st();
+      }
+      fence_async_smem();
+      fence_before();
+      mbar_arrive(bars + DB_KED);
+      // (Q~ o e^c)^T, -(diag(beta) K o e^c)^T as [f][i] and e^{c_last}: free once the previous
+      // chunk's state product is done (it follows the chain's use of e^{c_last})
+      if (k > 0 && !role_wait(bars + DB_S, par ^ 1, polls, abort, DBAR_BU, D_BU)) break;
+      {
+        const int f = bt & 127;
+        for (int m = 0; m < 8; ++m) {
+          const int i0 = ((bt >> 7) + 2 * m) * 4;
           float qe[4], nke[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const int i = i0 + u;
-            const float e = ex2(sC[i * LDCF + f]);
-            const uint32_t o = raw_off(i, f);
-            qe[u] = a.scale * __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + RAW_Q + o)) * e;
-            nke[u] = -sBeta[i] * __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + RAW_K + o)) * e;
+            const float e = ex2(ldf(tC, i, f));
+            qe[u] = a.scale * ldb(sm + RAW_Q, i, f) * e;
+            nke[u] = -sBeta[i] * ldb(sm + RAW_K, i, f) * e;
           }
-          st_tf32x4(sm, OP_QET + kmaj(f, i0, 64), qe[0], qe[1], qe[2], qe[3]);
-          st_tf32x4(sm, OP_NKET + kmaj(f, i0, 64), nke[0], nke[1], nke[2], nke[3]);
+          st_tf32x4(sm, D_QET + kmaj(f, i0, 64), qe[0], qe[1], qe[2], qe[3]);
+          st_tf32x4(sm, D_NKET + kmaj(f, i0, 64), nke[0], nke[1], nke[2], nke[3]);
         }
+        if (bt < KD) sEl[bt] = ex2(ldf(tC, 63, bt));
       }
-      if (tid < KD) sEl[tid] = ex2(sC[63 * LDCF + tid]);
-      // dO^T into TMEM: lane n, columns j
-      {
-        uint32_t r[32];
-#pragma unroll
-        for (int jj = 0; jj < 32; ++jj)
-          r[jj] = tf32_rna(__bfloat162float(
-              *reinterpret_cast<const __nv_bfloat16*>(sm + RAW_X + raw_off(hcol * 32 + jj, Lr))));
-        tmem_st32(tm + lo + TM_DOT + hcol * 32, r);
-        tmem_wait_st();
+      fence_async_smem();
+      mbar_arrive(bars + DB_QN);  // (also: this chunk's raw rows are consumed)
+      if (k + 1 < nch && bt < C) bval = beta_of(ch - 1);
+    }
+  } else {
+    // ======================================================================== loader warp
+    if (lane == 0 && nch > 0) {
+      const auto raw = [&](int ch) {
+        const int t0 = chunk_span(a, ch).x;
+        mbar_expect_tx(bars + DB_RAW, 3 * TILE_BF16 + TILE_F32);
+        for (int j = 0; j < 2; ++j) {
+          tma_load_4d(sb + RAW_Q + j * 8192, maps.q, 64 * j, h, t0, b, bars + DB_RAW);
+          tma_load_4d(sb + RAW_K + j * 8192, maps.k, 64 * j, h, t0, b, bars + DB_RAW);
+          tma_load_4d(sb + RAW_X + j * 8192, maps.x, 64 * j, hv, t0, b, bars + DB_RAW);
+        }
+        for (int j = 0; j < 4; ++j) tma_load_4d(sb + RAW_C + j * 8192, maps.g, 32 * j, hv, t0, b, bars + DB_RAW);
+        ++cnt[DB_RAW];
+      };
+      const auto prefetch = [&](int ch) {
+        const int t2 = chunk_span(a, ch).x;
+        for (int j = 0; j < 2; ++j) {
+          tma_prefetch_4d(maps.q, 64 * j, h, t2, b);
+          tma_prefetch_4d(maps.k, 64 * j, h, t2, b);
+          tma_prefetch_4d(maps.x, 64 * j, hv, t2, b);
+        }
+        for (int j = 0; j < 4; ++j) tma_prefetch_4d(maps.g, 32 * j, hv, t2, b);
+      };
+      raw(c1 - 1);
+      if (nch > 1) prefetch(c1 - 2);
+      for (int k = 0; k + 1 < nch; ++k) {  // chunk k + 1's tiles once the builders are done with chunk k's
+        if (!wait_one(bars + DB_QN, k & 1, polls, abort)) break;
+        raw(c1 - 2 - k);
+        if (k + 2 < nch) prefetch(c1 - 3 - k);
       }
     }
-    fence_before();
-    __syncthreads();  // this chunk's raw rows are consumed: the next chunk's may come in
-    if (ch > c0) {
-      const int2 sp = chunk_span(a, ch - 1);
-      load_raw_issue<NTH, true>(cx, qg, kg, dog, a.g, a.beta, b, T, sp.x, sp.y, a.H, a.HV, h, hv);
-    }
-    cp_async_commit();           // (an empty group on the last chunk keeps the count uniform)
-    cp_async_wait_group<1>();    // this chunk's images
-    fence_async_smem();
-    __syncthreads();
-    if (tid == 0) {  // dU^T = dO^T P + dM^T (K o e^{c_last-c})^T
-      fence_after();
-      const uint32_t id = idesc_tf32(128, 64);
-      for (int ks = 0; ks < 8; ++ks)
-        mma_ts(tm + TM_DU, tm + TM_DOT + ks * 8, desc(sb + IMG_PT + ks * 256, 2048), id, ks > 0);
-      for (int ks = 0; ks < 16; ++ks)
-        mma_ts(tm + TM_DU, tm + TM_S + ks * 8, desc(sb + OP_KED + ks * 256, 4096), id, 1);
-      commit(bar);
-    }
-    if (!wait_mma(bar, phase)) { failed = true; break; }
-    if (tid == 0) {  // dR^T = dU^T T
-      const uint32_t id = idesc_tf32(128, 64);
-      for (int ks = 0; ks < 8; ++ks)
-        mma_ts(tm + TM_DR, tm + TM_DU + ks * 8, desc(sb + IMG_TT + ks * 256, 2048), id, ks > 0);
-      commit(bar);
-    }
-    if (!wait_mma(bar, phase)) { failed = true; break; }
-    if (ch > c0) {  // the products have read this chunk's images: the next chunk's may come in
-      const float* irec = a.inter + chunk_gc(a, sq, hv, ch - 1) * INTER_REC;
-      copy_image(cx, IMG_PT, irec);
-      copy_image(cx, IMG_TT, irec + INTER_TT);
-    }
-    cp_async_commit();
-
-    // ---------------------------------------------------------------- store dM (leaving this chunk); start dM_in
-    float sv[2][32];  // dM leaving this chunk (this thread's lane, 64 channels), stored once
-                      // the products below are under way
-    {
-      uint32_t r[32];
-#pragma unroll
-      for (int cb = 0; cb < 2; ++cb) {
-        const int f0 = hcol * 64 + cb * 32;
-        tmem_ld32(tm + lo + TM_S + f0, sv[cb]);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(sv[cb][j] * sEl[f0 + j]);
-        tmem_st32(tm + lo + TM_S + f0, r);
-      }
-      tmem_wait_st();
-    }
-    fence_before();
-    __syncthreads();
-    if (tid == 0) {
-      fence_after();
-      const uint32_t id = idesc_tf32(128, 128);
-      for (int ks = 0; ks < 8; ++ks) {
-        mma_ts(tm + TM_S, tm + TM_DOT + ks * 8, desc(sb + OP_QET + ks * 256, 2048), id, 1);
-        mma_ts(tm + TM_S, tm + TM_DR + ks * 8, desc(sb + OP_NKET + ks * 256, 2048), id, 1);
-      }
-      commit(bar);
-    }
-    {
-      float* slot = a.dstates + dstate_slot(a, sq, hv, ch) * (KD * VD);
-      store_slot32(slot, hcol * 2, Lr, sv[0]);
-      store_slot32(slot, hcol * 2 + 1, Lr, sv[1]);
-    }
-    if (!wait_mma(bar, phase)) { failed = true; break; }
-    fence_before();
-    __syncthreads();
+    __syncwarp();
   }
 
-  cp_async_wait_all();  // (copies still in flight after an early exit)
-  if (!failed && a.dS0) {
-    fence_after();
-    for (int cb = 0; cb < 2; ++cb) {
-      const int f0 = hcol * 64 + cb * 32;
-      float s[32];
-      tmem_ld32(tm + lo + TM_S + f0, s);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) a.dS0[(head * KD + f0 + j) * VD + Lr] = s[j];
-    }
+  cp_async_wait_all();  // (the builders' copies still in flight after an early exit)
+  __syncthreads();
+  if (tid == 0) {  // every issued copy and product (the last state product too) ends before the memory goes
+    for (int i = 0; i < DNB_ASYNC; ++i)
+      if (cnt[i] > 0) mbar_wait_lim(bars + i, (cnt[i] - 1) & 1, 1u << 24);
   }
   fence_before();
   __syncthreads();
-  if (cx.warp == 0) tmem_dealloc(tm, 512);
-  if (failed && tid == 0) atomicOr(&g_kda_bwd_device_error, 1u);
+  if (warp == 0) tmem_dealloc(tm, 512);
+  if (*abort && tid == 0) atomicOr(&g_kda_bwd_device_error, 1u);
 }
 
 bool bwd_tc_eligible(const BwdArgs& a, int dtype) {
@@ -258,10 +369,13 @@ bool bwd_tc_eligible(const BwdArgs& a, int dtype) {
 }
 
 static int launch_bwd_dstate_tc(const BwdArgs& a, int nheads, cudaStream_t stream) {
+  RawMaps4 maps;
+  const int rc = make_raw_maps(&maps, a.q, a.k, a.dO, a.g, a.ctab ? 1 : a.B, a.T, a.H, a.HV);
+  if (rc) return rc;
   cudaError_t e = cudaFuncSetAttribute(kda_bwd_dstate_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)tcc::SMEM_BYTES);
   if (e != cudaSuccess) return set_cuda_error("kda_bwd: cudaFuncSetAttribute", e);
-  kda_bwd_dstate_tc_kernel<<<nheads, tcc::NTH, tcc::SMEM_BYTES, stream>>>(a);
+  kda_bwd_dstate_tc_kernel<<<nheads, tcd::D_THREADS, tcc::SMEM_BYTES, stream>>>(maps, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return set_cuda_error("kda_bwd: tensor-core state-gradient launch", e);
   return 0;
@@ -686,6 +800,13 @@ int launch_bwd_tc_passes(const BwdArgs& a, cudaStream_t stream, AssembleLaunch a
 }  // namespace kda
 
 namespace kda {
+int set_bwd_wait_polls(unsigned polls) {
+  const unsigned v = polls ? polls : (1u << 24);
+  const cudaError_t e = cudaMemcpyToSymbol(g_kda_bwd_wait_polls, &v, sizeof(v));
+  if (e != cudaSuccess) return set_cuda_error("kda_set_wait_polls", e);
+  return 0;
+}
+
 int take_bwd_device_error(unsigned* out) {
   unsigned v = 0, zero = 0;
   cudaError_t e = cudaMemcpyFromSymbol(&v, g_kda_bwd_device_error, sizeof(v));

@@ -63,24 +63,6 @@ struct FwdMaps {
   CUtensorMap q, k, v, g;
 };
 
-// Byte offsets inside a raw tile of 64 rows x 128 channels as the 128-byte
-// swizzle of TMA leaves it: bf16 as two 8 KB boxes of 64 channels, fp32 as
-// four 8 KB boxes of 32 channels; the 16-byte pieces of row i are permuted
-// by i % 8 (each box base 1024-byte aligned).
-__device__ __forceinline__ uint32_t bt_off(int i, int f) {
-  return (uint32_t)((f >> 6) * 8192 + i * 128 + ((((f & 63) >> 3) ^ (i & 7)) << 4) + (f & 7) * 2);
-}
-__device__ __forceinline__ uint32_t ft_off(int i, int f) {
-  return (uint32_t)((f >> 5) * 8192 + i * 128 + ((((f & 31) >> 2) ^ (i & 7)) << 4) + (f & 3) * 4);
-}
-__device__ __forceinline__ float ldf(const unsigned char* t, int i, int f) {
-  return *reinterpret_cast<const float*>(t + ft_off(i, f));
-}
-__device__ __forceinline__ float ldb(const unsigned char* t, int i, int f) {
-  return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(t + bt_off(i, f)));
-}
-
-constexpr uint32_t TILE_BF16 = 16384, TILE_F32 = 32768;
 
 // Barrier of the threads that run a per-chunk preparation: the whole CTA, or
 // one role of a warp-specialised kernel (named barrier `id` over `n` threads).
@@ -500,42 +482,12 @@ static_assert(S2_BYTES + 1024 <= 233472, "one CTA per SM");
 constexpr int K2_THREADS = 544, CH0 = 32, CH_THREADS = 256, BU0 = 288, BU_THREADS = 256;
 // named barriers: 1 the chain warps, 2 the builder warps, 3 the issuer warp with the chain warps
 constexpr int BAR_STATE0 = 3;
-__device__ __forceinline__ void named_sync(int id, int n) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
 // TMEM columns: the state M^T (lane = value column n, column = key channel);
 // two [Y^T | O^T] accumulators (chunks alternate; Z^T is written over Y^T);
 // U^T
 constexpr uint32_t TM_S = 0, TM_D0 = 128, TM_U = 384;
 // barriers: async copies and products (counted in S2_CNT for the drain), then the roles' arrivals
 enum { B_RAW, B_V, B_T, B_P, B_M1, B_M2, B_M3, B_M4, NB_ASYNC, B_KQ = NB_ASYNC, B_KD, B_Z, B_O, B_UR, NB_ALL };
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(tc::smem_u32(bar)) : "memory");
-}
-// Bounded wait, also giving up when another role has set *abort.
-__device__ __forceinline__ bool wait_one(uint64_t* bar, uint32_t parity, uint32_t polls, volatile int* abort) {
-  bool ok = tc::mbar_wait_lim(bar, parity, 1);
-  for (uint32_t it = 1; !ok && it < polls; it += 64) {
-    if (*abort) break;
-    ok = tc::mbar_wait_lim(bar, parity, 64);
-  }
-  return ok;
-}
-// The same for every thread of a role (named barrier `id`, `n` threads): the
-// role's common verdict (true: the phase completed for every thread).
-__device__ __forceinline__ bool role_wait(uint64_t* bar, uint32_t parity, uint32_t polls, volatile int* abort,
-                                          int id, int n) {
-  const bool ok = wait_one(bar, parity, polls, abort);
-  uint32_t bad;
-  asm volatile(
-      "{\n.reg .pred p, q;\nsetp.eq.u32 p, %1, 0;\nbar.red.or.pred q, %2, %3, p;\nselp.u32 %0, 1, 0, q;\n}\n"
-      : "=r"(bad)
-      : "r"((uint32_t)ok), "r"(id), "r"(n)
-      : "memory");
-  if (bad) *abort = 1;
-  return !bad;
-}
 
 template <bool PREP>
 __global__ void __launch_bounds__(K2_THREADS, 1) kda_fwd_state_tc_kernel(const __grid_constant__ FwdMaps maps,
@@ -913,6 +865,16 @@ int launch_t(const FwdArgs& a, cudaStream_t stream) {
   return 0;
 }
 }  // namespace
+
+int make_raw_maps(RawMaps4* m, const void* q, const void* k, const void* x, const float* g, int rows, int T, int H,
+                  int HV) {
+  static_assert(sizeof(CUtensorMap) == 128 && alignof(CUtensorMap) <= 64, "tensor map size");
+  int rc = head_map(reinterpret_cast<CUtensorMap*>(m->q), q, true, rows, T, H, 64);
+  if (!rc) rc = head_map(reinterpret_cast<CUtensorMap*>(m->k), k, true, rows, T, H, 64);
+  if (!rc) rc = head_map(reinterpret_cast<CUtensorMap*>(m->x), x, true, rows, T, HV, 64);
+  if (!rc) rc = head_map(reinterpret_cast<CUtensorMap*>(m->g), g, false, rows, T, HV, 32);
+  return rc;
+}
 
 // The gate of the fused preparation ("kimi_k3_host/kda.rs", bounded_gate):
 // g[r][hv][f] = gate(z[r][hv][f] + dt_bias[hv][f]) with e^{A_log[hv]}, eight

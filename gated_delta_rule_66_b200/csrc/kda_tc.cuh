@@ -200,6 +200,37 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols));
 }
 
+// ---- warp-specialised kernels: roles meet on mbarriers and named barriers
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// Bounded wait, also giving up when another role has set *abort.
+__device__ __forceinline__ bool wait_one(uint64_t* bar, uint32_t parity, uint32_t polls, volatile int* abort) {
+  bool ok = mbar_wait_lim(bar, parity, 1);
+  for (uint32_t it = 1; !ok && it < polls; it += 64) {
+    if (*abort) break;
+    ok = mbar_wait_lim(bar, parity, 64);
+  }
+  return ok;
+}
+// The same for every thread of a role (named barrier `id`, `n` threads): the
+// role's common verdict (true: the phase completed for every thread).
+__device__ __forceinline__ bool role_wait(uint64_t* bar, uint32_t parity, uint32_t polls, volatile int* abort,
+                                          int id, int n) {
+  const bool ok = wait_one(bar, parity, polls, abort);
+  uint32_t bad;
+  asm volatile(
+      "{\n.reg .pred p, q;\nsetp.eq.u32 p, %1, 0;\nbar.red.or.pred q, %2, %3, p;\nselp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(bad)
+      : "r"((uint32_t)ok), "r"(id), "r"(n)
+      : "memory");
+  if (bad) *abort = 1;
+  return !bad;
+}
+
 // 32 lanes x 32 consecutive 32-bit columns: thread i of the warp gets lane
 // (subpartition base + i), columns [col, col + 32).  The load and its wait
 // are one statement, so that no use of the registers can be scheduled

@@ -77,6 +77,25 @@ __device__ __forceinline__ void load_slot32(const float* slot, int grp, int n, f
   for (int j = 0; j < 32; ++j) v[j] = __half2float(h[(size_t)j * VD]) * s;
 }
 
+// Byte offsets inside a raw tile of 64 rows x 128 channels as the 128-byte
+// swizzle of TMA leaves it: bf16 as two 8 KB boxes of 64 channels, fp32 as
+// four 8 KB boxes of 32 channels; the 16-byte pieces of row i are permuted
+// by i % 8 (each box base 1024-byte aligned).
+__device__ __forceinline__ uint32_t bt_off(int i, int f) {
+  return (uint32_t)((f >> 6) * 8192 + i * 128 + ((((f & 63) >> 3) ^ (i & 7)) << 4) + (f & 7) * 2);
+}
+__device__ __forceinline__ uint32_t ft_off(int i, int f) {
+  return (uint32_t)((f >> 5) * 8192 + i * 128 + ((((f & 31) >> 2) ^ (i & 7)) << 4) + (f & 3) * 4);
+}
+__device__ __forceinline__ float ldf(const unsigned char* t, int i, int f) {
+  return *reinterpret_cast<const float*>(t + ft_off(i, f));
+}
+__device__ __forceinline__ float ldb(const unsigned char* t, int i, int f) {
+  return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(t + bt_off(i, f)));
+}
+
+constexpr uint32_t TILE_BF16 = 16384, TILE_F32 = 32768;
+
 // byte offset of bf16 element (row i, channel f) in a raw q / k / x tile:
 // the 16-byte pieces of row i are stored XOR-swizzled by i % 8, so that one
 // piece of 8 consecutive rows lies in 8 different bank groups

@@ -86,8 +86,9 @@ int kda_device_status(unsigned* flags);
 
 /* Test hook for the failure path of the bounded waits.  Every wait of the
  * chunked tensor-core forward (the two kernels that kda_fwd, kda_fwd_varlen
- * and kda_fwd_prep run when given their workspace) probes its mbarrier at
- * most `polls` times (0 restores the default, 2^24) before it gives up.  A
+ * and kda_fwd_prep run when given their workspace) and of the tensor-core
+ * backward's state-gradient pass probes its mbarrier at most `polls` times
+ * (0 restores the default, 2^24) before it gives up.  A
  * kernel that gives up first waits, under the default bound, for every copy
  * and tensor-core product it has already issued, then frees its tensor
  * memory, sets bit 0 of kda_device_status() and returns; its outputs are

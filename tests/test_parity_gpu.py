@@ -147,6 +147,35 @@ def test_bounded_wait_gives_up_then_recovers(kda):
     assert kda.device_status() == 0
 
 
+def test_bounded_wait_backward_gives_up_then_recovers(kda):
+    """The same for the tensor-core backward's warp-specialised state-gradient
+    pass: with one probe per wait its issuer gives up at its first wait (the
+    builders cannot have formed the first operand yet), every role leaves,
+    the issued copies drain and bit 0 is reported (the later kernels of the
+    call run on undefined state gradients, which is no fault); with the
+    default restored the backward matches the oracle."""
+    w = BY_NAME["fwdbwd"].with_sizes(B=1, T=130, H=2, HV=2)
+    inp = make_inputs(w, with_do=True)
+    d = to_cuda(inp)
+    B, T, H, K = d["q"].shape
+    HV, V = d["v"].shape[2], d["v"].shape[3]
+    ws = torch.empty(kda.workspace_bytes("bwd", B, T, H, HV, K, V), dtype=torch.uint8, device="cuda")
+    kda.fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], scale=w.scale, initial_state=d["S0"], workspace=ws)
+    torch.cuda.synchronize()
+    assert kda.device_status() == 0
+    kda.set_wait_polls(1)
+    try:
+        kda.bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["dO"], scale=w.scale, initial_state=d["S0"],
+                workspace=ws, states_from_fwd=True)
+        torch.cuda.synchronize()
+        flags = kda.device_status()
+    finally:
+        kda.set_wait_polls(0)
+    assert flags & 1, f"no kernel reported giving up (flags {flags})"
+    check_bwd(kda, inp, w.scale, w.torch_dtype, "bwd_after_give_up", reuse=True)
+    assert kda.device_status() == 0
+
+
 def test_fwd_strong_unbounded_decay(kda):
     """Very strong decays (|g| up to 40 per step) take the pair-by-pair path
     for diagonal blocks; results stay finite and match."""
