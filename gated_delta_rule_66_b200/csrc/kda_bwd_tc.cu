@@ -42,12 +42,12 @@ __device__ __forceinline__ void st4h(__half* p, const float* v) {
 //     T^T image copies (a tcgen05.mma issue holds its thread for about the
 //     product's duration, so this warp does nothing else);
 //   chain warps 1-8 (TMEM lanes 32 (w % 4) .., lane = value column n; column
-//     half (w - 1) / 4): the state gradient's decay in TMEM, storing the
-//     gradient leaving every chunk on the way;
-//   builder warps 9-16: the decay and the chunk's operands K o e^{c_last-c}
-//     as [i][f], (Q~ o e^c)^T and -(diag(beta) K o e^c)^T as [f][i],
-//     e^{c_last}, and dO^T into one of two TMEM buffers, the next chunk's
-//     while this chunk's products run;
+//     half (w - 1) / 4): the operands of the state product, (Q~ o e^c)^T and
+//     -(diag(beta) K o e^c)^T as [f][i], and e^{c_last}; the state gradient's
+//     decay in TMEM, storing the gradient leaving every chunk on the way;
+//   builder warps 9-16: the decay and the operands K o e^{c_last-c} as
+//     [i][f] and dO^T (into one of two TMEM buffers), the next chunk's while
+//     this chunk's products run;
 //   loader warp 17 (lane 0): the next chunk's q, k, dO and g tiles by TMA
 //     once the builders are done with the current ones, and the chunk after
 //     next into L2 (a TMA issue can hold its thread for a while).
@@ -65,7 +65,7 @@ static_assert(D_CNT + 64 <= SMALL, "state-gradient shared-memory map");
 // TMEM columns: dM^T, dU^T, dR^T, two dO^T buffers (chunks alternate), and the
 // chain's copy of the gradient leaving the chunk (stored after the decay is released)
 constexpr uint32_t DT_S = 0, DT_DU = 128, DT_DR = 192, DT_DOT = 256, DT_COPY = 384;
-enum { DB_RAW, DB_P, DB_T, DB_DU, DB_DR, DB_S, DNB_ASYNC, DB_KED = DNB_ASYNC, DB_QN, DB_RS, DNB_ALL };
+enum { DB_RAW, DB_P, DB_T, DB_DU, DB_DR, DB_S, DNB_ASYNC, DB_KED = DNB_ASYNC, DB_C, DB_QN, DB_RS, DNB_ALL };
 // named barriers: 1 the chain warps, 2 the builder warps, 3 the issuer warp with the chain warps
 constexpr int DBAR_CH = 1, DBAR_BU = 2, DBAR_S0 = 3;
 }  // namespace tcd
@@ -93,12 +93,14 @@ __global__ void __launch_bounds__(tcd::D_THREADS, 1) kda_bwd_dstate_tc_kernel(co
   volatile int* abort = cnt + 15;
   uint32_t* sTm = reinterpret_cast<uint32_t*>(sm + S_TMEM);
   float* sEl = reinterpret_cast<float*>(sm + S_EL);
+  float* sBeta = reinterpret_cast<float*>(sm + S_BETA);
   unsigned char* tC = sm + RAW_C;  // g, then the cumulative decay (fp32 TMA tile)
   const uint32_t polls = g_kda_bwd_wait_polls;
 
   if (warp == 0) tmem_alloc(sTm, 512);
   if (tid == 0) {
-    for (int i = 0; i < DNB_ALL; ++i) mbar_init(bars + i, i < DNB_ASYNC ? 1 : (i == DB_RS ? D_CH : D_BU));
+    for (int i = 0; i < DNB_ALL; ++i)
+      mbar_init(bars + i, i < DNB_ASYNC ? 1 : (i == DB_RS || i == DB_QN ? D_CH : D_BU));
     for (int i = 0; i < 16; ++i) cnt[i] = 0;
   }
   fence_before();
@@ -172,12 +174,36 @@ __global__ void __launch_bounds__(tcd::D_THREADS, 1) kda_bwd_dstate_tc_kernel(co
     fence_before();
     named_sync(DBAR_S0, 32 + D_CH);
     bool ok = true;
+    const int ct = tid - 32;  // 0 .. 255
     for (int k = 0; k < nch; ++k) {
       const int ch = c1 - 1 - k;
       const uint32_t par = k & 1;
+      // (Q~ o e^c)^T, -(diag(beta) K o e^c)^T as [f][i] and e^{c_last}: once this chunk's decay is
+      // formed and the previous chunk's state product (which read them) is done
+      if (!(ok = role_wait(bars + DB_C, par, polls, abort, DBAR_CH, D_CH))) break;
+      if (k > 0 && !(ok = role_wait(bars + DB_S, par ^ 1, polls, abort, DBAR_CH, D_CH))) break;
+      {
+        const int f = ct & 127;
+        for (int m = 0; m < 8; ++m) {
+          const int i0 = ((ct >> 7) + 2 * m) * 4;
+          float qe[4], nke[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int i = i0 + u;
+            const float e = ex2(ldf(tC, i, f));
+            qe[u] = a.scale * ldb(sm + RAW_Q, i, f) * e;
+            nke[u] = -sBeta[i] * ldb(sm + RAW_K, i, f) * e;
+          }
+          st_tf32x4(sm, D_QET + kmaj(f, i0, 64), qe[0], qe[1], qe[2], qe[3]);
+          st_tf32x4(sm, D_NKET + kmaj(f, i0, 64), nke[0], nke[1], nke[2], nke[3]);
+        }
+        if (ct < KD) sEl[ct] = ex2(ldf(tC, 63, ct));
+      }
+      fence_async_smem();
+      mbar_arrive(bars + DB_QN);  // (also: the chain is done with this chunk's raw rows)
       // the gradient leaving this chunk: stored, then decayed by e^{c_last} once dU^T has read it
+      // (the wait is also the chain's barrier for e^{c_last})
       if (!(ok = role_wait(bars + DB_DU, par, polls, abort, DBAR_CH, D_CH))) break;
-      if (!(ok = role_wait(bars + DB_QN, par, polls, abort, DBAR_CH, D_CH))) break;
       fence_after();
 #pragma unroll 1
       for (int cb = 0; cb < 2; ++cb) {
@@ -221,7 +247,6 @@ __global__ void __launch_bounds__(tcd::D_THREADS, 1) kda_bwd_dstate_tc_kernel(co
     cx.sm = sm;
     cx.sb = sb;
     cx.tid = bt;
-    float* sBeta = cx.beta();
     float* sCarry = reinterpret_cast<float*>(sm + S_CARRY);
     const int n = (warp & 3) * 32 + lane, hb = (warp - 9) >> 2;  // dO^T: TMEM lane n, columns 32 hb ..
     const uint32_t lo = (uint32_t)((warp & 3) * 32) << 16;
@@ -269,6 +294,7 @@ __global__ void __launch_bounds__(tcd::D_THREADS, 1) kda_bwd_dstate_tc_kernel(co
         for (int r = 0; r < 32; ++r) *reinterpret_cast<float*>(tC + ft_off(hh * 32 + r, f)) = (v[r] + carry) * LOG2E;
         named_sync(DBAR_BU, D_BU);
       }
+      mbar_arrive(bars + DB_C);  // the decay (and beta) of this chunk for the chain's operands
       // K o e^{c_last-c} as [i][f] and dO^T: free once the previous chunk's dU^T is done
       if (k > 0 && !role_wait(bars + DB_DU, par ^ 1, polls, abort, DBAR_BU, D_BU)) break;
       {
@@ -291,29 +317,7 @@ __global__ void __launch_bounds__(tcd::D_THREADS, 1) kda_bwd_dstate_tc_kernel(co
       }
       fence_async_smem();
       fence_before();
-      mbar_arrive(bars + DB_KED);
-      // (Q~ o e^c)^T, -(diag(beta) K o e^c)^T as [f][i] and e^{c_last}: free once the previous
-      // chunk's state product is done (it follows the chain's use of e^{c_last})
-      if (k > 0 && !role_wait(bars + DB_S, par ^ 1, polls, abort, DBAR_BU, D_BU)) break;
-      {
-        const int f = bt & 127;
-        for (int m = 0; m < 8; ++m) {
-          const int i0 = ((bt >> 7) + 2 * m) * 4;
-          float qe[4], nke[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int i = i0 + u;
-            const float e = ex2(ldf(tC, i, f));
-            qe[u] = a.scale * ldb(sm + RAW_Q, i, f) * e;
-            nke[u] = -sBeta[i] * ldb(sm + RAW_K, i, f) * e;
-          }
-          st_tf32x4(sm, D_QET + kmaj(f, i0, 64), qe[0], qe[1], qe[2], qe[3]);
-          st_tf32x4(sm, D_NKET + kmaj(f, i0, 64), nke[0], nke[1], nke[2], nke[3]);
-        }
-        if (bt < KD) sEl[bt] = ex2(ldf(tC, 63, bt));
-      }
-      fence_async_smem();
-      mbar_arrive(bars + DB_QN);  // (also: this chunk's raw rows are consumed)
+      mbar_arrive(bars + DB_KED);  // (also: the builders are done with this chunk's raw rows)
       if (k + 1 < nch && bt < C) bval = beta_of(ch - 1);
     }
   } else {
@@ -341,7 +345,8 @@ __global__ void __launch_bounds__(tcd::D_THREADS, 1) kda_bwd_dstate_tc_kernel(co
       };
       raw(c1 - 1);
       if (nch > 1) prefetch(c1 - 2);
-      for (int k = 0; k + 1 < nch; ++k) {  // chunk k + 1's tiles once the builders are done with chunk k's
+      for (int k = 0; k + 1 < nch; ++k) {  // chunk k + 1's tiles once builders and chain are done with chunk k's
+        if (!wait_one(bars + DB_KED, k & 1, polls, abort)) break;
         if (!wait_one(bars + DB_QN, k & 1, polls, abort)) break;
         raw(c1 - 2 - k);
         if (k + 2 < nch) prefetch(c1 - 3 - k);
