@@ -72,7 +72,7 @@ constexpr int DBAR_CH = 1, DBAR_BU = 2, DBAR_S0 = 3;
 
 __device__ unsigned int g_kda_bwd_wait_polls = 1u << 24;
 
-__global__ void __launch_bounds__(tcd::D_THREADS, 1) kda_bwd_dstate_tc_kernel(const __grid_constant__ RawMaps4 maps,
+__global__ void __launch_bounds__(tcd::D_THREADS, 1) kda_bwd_dstate_tc_kernel(const __grid_constant__ RawMaps maps,
                                                                               BwdArgs a) {
   using namespace tcd;
   using namespace tc;
@@ -374,8 +374,8 @@ bool bwd_tc_eligible(const BwdArgs& a, int dtype) {
 }
 
 static int launch_bwd_dstate_tc(const BwdArgs& a, int nheads, cudaStream_t stream) {
-  RawMaps4 maps;
-  const int rc = make_raw_maps(&maps, a.q, a.k, a.dO, a.g, a.ctab ? 1 : a.B, a.T, a.H, a.HV);
+  RawMaps maps;
+  const int rc = make_raw_maps(&maps, a.q, a.k, a.dO, a.g, nullptr, a.ctab ? 1 : a.B, a.T, a.H, a.HV);
   if (rc) return rc;
   cudaError_t e = cudaFuncSetAttribute(kda_bwd_dstate_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)tcc::SMEM_BYTES);
@@ -445,10 +445,15 @@ __device__ __forceinline__ void stage_fn(const tcc::Ctx& cx, uint32_t tmc) {
   }
 }
 
-__global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
+__global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(const __grid_constant__ RawMaps maps,
+                                                                   BwdArgs a) {
   using namespace tcg;
   using namespace tc;
   extern __shared__ __align__(1024) unsigned char sm[];
+  if (smem_u32(sm) & 1023u) {  // the 128-byte swizzle of the TMA tiles needs a 1024-byte aligned base
+    if (threadIdx.x == 0) atomicOr(&g_kda_bwd_device_error, 2u);
+    return;
+  }
   Ctx cx;
   cx.sm = sm;
   cx.sb = smem_u32(sm);
@@ -465,23 +470,26 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
   const int G = a.HV / a.H, T = a.T;
   const int NT = a.ctab ? a.NC : (T + C - 1) / C;
   const int items = a.item1 > 0 ? a.item1 : NT * a.HV * (a.ctab ? 1 : a.B);
-  const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(a.q);
-  const __nv_bfloat16* kg = static_cast<const __nv_bfloat16*>(a.k);
-  const __nv_bfloat16* vg = static_cast<const __nv_bfloat16*>(a.v);
-  const __nv_bfloat16* dog = static_cast<const __nv_bfloat16*>(a.dO);
   __nv_bfloat16* dvg = static_cast<__nv_bfloat16*>(a.dv);
   float* sBeta = cx.beta();
   float* sDEl = reinterpret_cast<float*>(sm + S_EL);    // 128 floats
   float* sDbR = reinterpret_cast<float*>(sm + S_EMID);  // 64 floats
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + S_BAR);
+  uint64_t* bar_raw = reinterpret_cast<uint64_t*>(sm + S_TMEM + 8);  // the raw tiles' TMA
   uint32_t* sTm = reinterpret_cast<uint32_t*>(sm + S_TMEM);
-  const float* sC = cx.c();
+  unsigned char* tC = sm + RAW_C;  // g, then the cumulative decay (fp32 TMA tile)
+  float* sCarry = reinterpret_cast<float*>(sm + S_CARRY);
+  const uint32_t polls = g_kda_bwd_wait_polls;
+  uint32_t n_raw = 0, w_raw = 0;
   // per-subpartition partial sums, added in a fixed order (deterministic)
   float* partEl = reinterpret_cast<float*>(sm + R_AH);   // [4][128], once Ah is in the record
   float* partBr = reinterpret_cast<float*>(sm + OP_PBR);  // [4][64], once K o e^{c_last-c} is consumed
 
   if (cx.warp == 0) tmem_alloc(sTm, 512);
-  if (tid == 0) mbar_init(bar, 1);
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    mbar_init(bar_raw, 1);
+  }
   fence_before();
   __syncthreads();
   fence_after();
@@ -503,30 +511,71 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
     const float* irec = a.inter + gc * INTER_REC;  // P^T, T, T^T images of this chunk (forward)
     const float* mst = a.states + state_slot(a, sq, hv, ch) * (KD * VD);     // M: state entering the chunk
     const float* dmst = a.dstates + dstate_slot(a, sq, hv, ch) * (KD * VD);  // dM: gradient of the leaving state
-    load_raw_issue(cx, qg, kg, dog, a.g, a.beta, b, T, t0, L, a.H, a.HV, h, hv);
-    for (int x = tid; x < C * 16; x += NTH) {  // V rows [i][n] (bf16) into the -dR half of [dO; -dR]
-      const int i = x >> 4, c16 = x & 15;
-      cp_async16(sb + OP_V + x * 16, vg + (((size_t)b * T + t0 + (i < L ? i : 0)) * a.HV + hv) * VD + c16 * 8, i < L);
+    // q, k, dO, g tiles into the raw region and the v tile into the -dR half of [dO; -dR], by
+    // TMA from one thread; beta (HV floats apart per step) by 64 threads
+    if (tid == 0) {
+      mbar_expect_tx(bar_raw, 4 * TILE_BF16 + TILE_F32);
+      for (int j = 0; j < 2; ++j) {
+        tma_load_4d(sb + RAW_Q + j * 8192, maps.q, 64 * j, h, t0, b, bar_raw);
+        tma_load_4d(sb + RAW_K + j * 8192, maps.k, 64 * j, h, t0, b, bar_raw);
+        tma_load_4d(sb + RAW_X + j * 8192, maps.x, 64 * j, hv, t0, b, bar_raw);
+        tma_load_4d(sb + OP_V + j * 8192, maps.v, 64 * j, hv, t0, b, bar_raw);
+      }
+      for (int j = 0; j < 4; ++j) tma_load_4d(sb + RAW_C + j * 8192, maps.g, 32 * j, hv, t0, b, bar_raw);
     }
+    ++n_raw;
+    if (tid < C) sBeta[tid] = tid < L ? a.beta[((size_t)b * T + t0 + tid) * a.HV + hv] : 0.f;
     if (tid < 9) prefetch_l2(mst + tid * 1024, tid < 8 ? 4096 : 2048);  // (fp16 values and their scales)
     else if (tid >= 16 && tid < 25) prefetch_l2(dmst + (tid - 16) * 1024, tid < 24 ? 4096 : 2048);
     else if (tid == 32) prefetch_l2(irec, 2 * 16384);
     else if (tid == 33) prefetch_l2(irec + INTER_TT, 16384);
-    if (!load_raw_wait(cx)) { failed = true; break; }
-    cumsum_span(cx);
+    if (__syncthreads_or(!mbar_wait_lim(bar_raw, w_raw & 1, polls))) { failed = true; break; }
+    ++w_raw;
+    if (L < C) {  // rows past the sequence (a packed batch's next sequence) count as zero
+      for (int x = tid; x < (C - L) * 16; x += NTH) {  // 16-byte pieces of the bf16 rows
+        const int i = L + (x >> 4), p = x & 15;
+        const uint32_t o = (uint32_t)((p >> 3) * 8192 + i * 128 + (((p & 7) ^ (i & 7)) << 4));
+        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(sm + RAW_Q + o) = z;
+        *reinterpret_cast<uint4*>(sm + RAW_K + o) = z;
+        *reinterpret_cast<uint4*>(sm + RAW_X + o) = z;
+        *reinterpret_cast<uint4*>(sm + OP_V + o) = z;
+      }
+      for (int x = tid; x < (C - L) * 32; x += NTH) {  // and of the fp32 g rows
+        const int i = L + (x >> 5), p = x & 31;
+        *reinterpret_cast<uint4*>(tC + (p >> 3) * 8192 + i * 128 + (((p & 7) ^ (i & 7)) << 4)) =
+            make_uint4(0u, 0u, 0u, 0u);
+      }
+      __syncthreads();
+    }
+    {  // cumulative decay (times log2 e) in place: channel tid % 128, rows 32 (tid / 128) ..
+      const int f = tid & 127, hh = tid >> 7;
+      float v[32], run = 0.f;
+#pragma unroll
+      for (int r = 0; r < 32; ++r) {
+        run += ldf(tC, hh * 32 + r, f);
+        v[r] = run;
+      }
+      if (hh == 0) sCarry[f] = run;
+      __syncthreads();
+      const float carry = hh ? sCarry[f] : 0.f;
+#pragma unroll
+      for (int r = 0; r < 32; ++r) *reinterpret_cast<float*>(tC + ft_off(hh * 32 + r, f)) = (v[r] + carry) * LOG2E;
+      __syncthreads();
+    }
 
     // ---------------------------------------------------------------- K o e^c, K o e^{c_last-c}, dO, dO^T
     {
       const int fq = item_f(cx);
-      const float4 c63v = ld4(sC + 63 * LDCF + fq);
+      const float4 c63v = *reinterpret_cast<const float4*>(tC + ft_off(63, fq));
       const float c63[4] = {c63v.x, c63v.y, c63v.z, c63v.w};
       for (int m = 0; m < 8; ++m) {
         const int i = item_row(cx, m);
-        const float4 c4 = ld4(sC + i * LDCF + fq);
+        const float4 c4 = *reinterpret_cast<const float4*>(tC + ft_off(i, fq));
         const float c[4] = {c4.x, c4.y, c4.z, c4.w};
         float kf[4], df[4];
-        bf16x4(sm + RAW_K + raw_off(i, fq), kf);
-        bf16x4(sm + RAW_X + raw_off(i, fq), df);
+        bf16x4(sm + RAW_K + bt_off(i, fq), kf);
+        bf16x4(sm + RAW_X + bt_off(i, fq), df);
         float e[4], ed[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -539,9 +588,7 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
       }
       uint32_t r[32];
 #pragma unroll
-      for (int jj = 0; jj < 32; ++jj)
-        r[jj] = tf32_rna(__bfloat162float(
-              *reinterpret_cast<const __nv_bfloat16*>(sm + RAW_X + raw_off(hcol * 32 + jj, Lr))));
+      for (int jj = 0; jj < 32; ++jj) r[jj] = tf32_rna(ldb(sm + RAW_X, hcol * 32 + jj, Lr));
       tmem_st32(tm + lo + TM_DOT + hcol * 32, r);
       tmem_wait_st();
     }
@@ -595,9 +642,8 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
       uint32_t r[32];
       tmem_ld32(tm + lo + TM_X + hcol * 32, x);
 #pragma unroll
-      const __nv_bfloat16* sV = reinterpret_cast<const __nv_bfloat16*>(sm + OP_V);
       for (int jj = 0; jj < 32; ++jj) {
-        xs[jj] = __bfloat162float(sV[(hcol * 32 + jj) * VD + Lr]) - x[jj];
+        xs[jj] = ldb(sm + OP_V, hcol * 32 + jj, Lr) - x[jj];
         r[jj] = tf32_rna(sBeta[hcol * 32 + jj] * xs[jj]);
       }
       tmem_st32(tm + lo + TM_X + hcol * 32, r);
@@ -697,11 +743,16 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(BwdArgs a) {
       }
     }
     // the record's shared-memory sources are read and every TMEM read-out is
-    // complete before the next item overwrites them
+    // complete before the next item overwrites them (its tiles by TMA)
     fence_before();
+    fence_async_smem();
     __syncthreads();
   }
 
+  if (failed && tid == 0) {  // the raw tiles and the products still in flight end before the memory goes
+    while (w_raw < n_raw) mbar_wait_lim(bar_raw, (w_raw++) & 1, 1u << 24);
+    mbar_wait_lim(bar, (phase ^ 1) & 1, 1u << 24);  // (wait_mma flips the phase even when it gives up)
+  }
   fence_before();
   __syncthreads();
   if (cx.warp == 0) tmem_dealloc(tm, 512);
@@ -721,7 +772,10 @@ static int launch_bwd_grads_tc(const BwdArgs& a, cudaStream_t stream) {
   // (An L2 prefetch of the inputs of the item one SM count further on, as
   // the assembly does, measured 0.36 ms slower per fwd+bwd step at B = 2,
   // H = 96, T = 4096.)
-  kda_bwd_grads_tc_kernel<<<(int)items, tcc::NTH, tcc::SMEM_BYTES, stream>>>(a);
+  RawMaps maps;
+  const int rc = make_raw_maps(&maps, a.q, a.k, a.dO, a.g, a.v, a.ctab ? 1 : a.B, a.T, a.H, a.HV);
+  if (rc) return rc;
+  kda_bwd_grads_tc_kernel<<<(int)items, tcc::NTH, tcc::SMEM_BYTES, stream>>>(maps, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return set_cuda_error("kda_bwd: tensor-core gradient launch", e);
   return 0;

@@ -866,13 +866,14 @@ int launch_t(const FwdArgs& a, cudaStream_t stream) {
 }
 }  // namespace
 
-int make_raw_maps(RawMaps4* m, const void* q, const void* k, const void* x, const float* g, int rows, int T, int H,
-                  int HV) {
+int make_raw_maps(RawMaps* m, const void* q, const void* k, const void* x, const float* g, const void* v, int rows,
+                  int T, int H, int HV) {
   static_assert(sizeof(CUtensorMap) == 128 && alignof(CUtensorMap) <= 64, "tensor map size");
   int rc = head_map(reinterpret_cast<CUtensorMap*>(m->q), q, true, rows, T, H, 64);
   if (!rc) rc = head_map(reinterpret_cast<CUtensorMap*>(m->k), k, true, rows, T, H, 64);
   if (!rc) rc = head_map(reinterpret_cast<CUtensorMap*>(m->x), x, true, rows, T, HV, 64);
   if (!rc) rc = head_map(reinterpret_cast<CUtensorMap*>(m->g), g, false, rows, T, HV, 32);
+  if (!rc && v) rc = head_map(reinterpret_cast<CUtensorMap*>(m->v), v, true, rows, T, HV, 64);
   return rc;
 }
 

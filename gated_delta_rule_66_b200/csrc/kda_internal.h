@@ -206,14 +206,14 @@ int set_wait_polls(unsigned polls);
 int set_bwd_wait_polls(unsigned polls);
 // 4-D TMA tensor maps [rows, T, heads, 128] (rows = B, or 1 for packed
 // sequences; CUtensorMap, 128 bytes each) of raw rows: q and k over the
-// query/key heads and x over the value heads as bf16 with 64-channel boxes,
-// g as fp32 with 32-channel boxes; 64 steps x one head per box, 128-byte
-// swizzle, zero fill past the tensor.
-struct alignas(64) RawMaps4 {
-  unsigned char q[128], k[128], x[128], g[128];
+// query/key heads, x (dO) and v over the value heads as bf16 with 64-channel
+// boxes, g as fp32 with 32-channel boxes; 64 steps x one head per box,
+// 128-byte swizzle, zero fill past the tensor.  (v may be null: no map.)
+struct alignas(64) RawMaps {
+  unsigned char q[128], k[128], x[128], g[128], v[128];
 };
-int make_raw_maps(RawMaps4* m, const void* q, const void* k, const void* x, const float* g, int rows, int T, int H,
-                  int HV);
+int make_raw_maps(RawMaps* m, const void* q, const void* k, const void* x, const float* g, const void* v, int rows,
+                  int T, int H, int HV);
 int take_device_error(unsigned* out);
 int take_bwd_device_error(unsigned* out);
 int launch_bwd(const BwdArgs& a, int dtype, cudaStream_t stream);
