@@ -304,6 +304,20 @@ def test_bwd_tc_strong_unbounded_decay(kda):
     check_bwd(kda, inp, w.scale, w.torch_dtype, "tc_strong_decay")
 
 
+@pytest.mark.parametrize("mag", [1e5, 1e-4], ids=["states_1e5", "states_1e-4"])
+def test_bwd_tc_state_range(kda, mag):
+    """The tensor-core path stores the chunk states and their gradients as
+    fp16 with a power-of-two scale per value column and 32 key channels.
+    v and S0 scaled by 1e5 put the states far past fp16's range (65504), and
+    scaled by 1e-4 into its subnormals; with the scales both keep the bf16
+    bar (the forward's states are reused by the backward, as in training)."""
+    w = BY_NAME["fwdbwd"].with_sizes(B=1, T=130, H=2, HV=2, s0_std=0.5)
+    inp = make_inputs(w, with_do=True)
+    inp["v"] = (inp["v"].float() * mag).to(inp["v"].dtype)
+    inp["S0"] = inp["S0"] * mag
+    check_bwd(kda, inp, w.scale, w.torch_dtype, f"tc_state_range_{mag:g}", reuse=True)
+
+
 def test_bwd_misaligned_dO_after_tensor_core_forward(kda):
     """A dO that is not 16-byte aligned keeps the backward off the tensor-core
     path; with states_from_fwd it must then not rely on the tensor-core
