@@ -59,12 +59,12 @@ __device__ __forceinline__ void store4(__nv_bfloat16* p, float x, float y, float
 // (256 threads; seg is 8 x KQ scratch; `base` is added to every element of a
 // reverse sum).  Ends with a barrier.
 
-// four consecutive fp16 record elements (8-byte aligned) as floats
-__device__ __forceinline__ float4 ld4h(const __half* p) {
+// four consecutive fp16 record elements (8-byte aligned) as floats, times their group's scale
+__device__ __forceinline__ float4 ld4h(const __half* p, float sc) {
   const uint2 u = *reinterpret_cast<const uint2*>(p);
   const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
   const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&u.y));
-  return make_float4(lo.x, lo.y, hi.x, hi.y);
+  return make_float4(lo.x * sc, lo.y * sc, hi.x * sc, hi.y * sc);
 }
 template <bool REVERSE>
 __device__ __forceinline__ void cumsum64(float* a, float* seg, const float* base) {
@@ -100,13 +100,14 @@ __device__ __forceinline__ void prefetch_assembly(const BwdArgs& a, int ch, int 
   const int tid = threadIdx.x, G = a.HV / a.H, h = hv / G, b = row_of(a, sq);
   const int2 sp = chunk_span(a, ch);
   const size_t gc = chunk_gc(a, sq, hv, ch);
-  if (tid < 17) {  // GREC floats = 16 pieces of 4096 bytes + 768
+  if (tid < 17) {  // GREC floats = 16 pieces of 4096 bytes + the rest
+    static_assert(GREC * 4 > 16 * 4096 && GREC * 4 - 16 * 4096 <= 4096 && GREC * 4 % 16 == 0, "record pieces");
     const uint32_t bytes = tid < 16 ? 4096u : (uint32_t)(GREC * 4 - 16 * 4096);
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a.gws + gc * GREC + tid * 1024), "r"(bytes)
                  : "memory");
     return;
   }
-  if (tid >= 20 && tid < 24) {
+  if (tid >= 20 && tid < 24) {  // (Ah: 4 pieces)
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a.inter + gc * INTER_REC + INTER_AH +
                                                                     (tid - 20) * 1024),
                  "r"(4096u)
@@ -151,11 +152,14 @@ __device__ __forceinline__ void assemble_quarter(const BwdArgs& a, float* smem, 
                                                             (16 * fq4 + (tid >> 4)) * 64 + (tid & 15) * 4)
                          : make_float4(0.f, 0.f, 0.f, 0.f);
   float qe[8], ke[8], kd[8];
+  // the fp16 record's block scales: [dQE; dKE'] and dKEd of this quarter, [dP; dA] of both column groups
+  const float sq_e = rec[G_SC + 4 + fq4], sk_e = rec[G_SC + 8 + fq4], sd_e = rec[G_SC + 12 + fq4];
+  const float sp_0 = rec[G_SC + 0], sp_1 = rec[G_SC + 1], sa_0 = rec[G_SC + 2], sa_1 = rec[G_SC + 3];
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
-    qe[u] = __half2float(rech[GH_QK + rec_off(ei + u, f0 + ef, 128)]);
-    ke[u] = __half2float(rech[GH_QK + rec_off(64 + ei + u, f0 + ef, 128)]);
-    kd[u] = __half2float(rech[GH_KED + rec_off(ei + u, f0 + ef, 128)]);
+    qe[u] = __half2float(rech[GH_QK + rec_off(ei + u, f0 + ef, 128)]) * sq_e;
+    ke[u] = __half2float(rech[GH_QK + rec_off(64 + ei + u, f0 + ef, 128)]) * sk_e;
+    kd[u] = __half2float(rech[GH_KED + rec_off(ei + u, f0 + ef, 128)]) * sd_e;
   }
   {  // inputs of this channel quarter (4 channels per item) and the C x C adjoints; loads first
     float4 gv[2], dp[4], da[4];
@@ -178,8 +182,8 @@ __device__ __forceinline__ void assemble_quarter(const BwdArgs& a, float* smem, 
       const int idx = tid + m * NTHREADS, i = idx >> 4, j4 = (idx & 15) * 4;
       // only the lower triangle is used (dP: j <= i, dA: j < i): wholly upper pieces are not read
       const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
-      dp[m] = (j4 <= i) ? ld4h(rech + GH_PA + rec_off(i, j4, 64)) : z4;
-      da[m] = (j4 <= i) ? ld4h(rech + GH_PA + rec_off(64 + i, j4, 64)) : z4;
+      dp[m] = (j4 <= i) ? ld4h(rech + GH_PA + rec_off(i, j4, 64), j4 < 32 ? sp_0 : sp_1) : z4;
+      da[m] = (j4 <= i) ? ld4h(rech + GH_PA + rec_off(64 + i, j4, 64), j4 < 32 ? sa_0 : sa_1) : z4;
     }
     float bt[4];  // beta of the rows of the [dA] items
 #pragma unroll

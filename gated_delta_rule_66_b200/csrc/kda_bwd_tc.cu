@@ -29,13 +29,28 @@ namespace kda {
 
 __device__ unsigned int g_kda_bwd_device_error;  // this file's kernels (one flag per translation unit)
 
-// four fp32 values rounded to fp16 into 8 bytes of shared memory
-__device__ __forceinline__ void st4h(__half* p, const float* v) {
-  const __half2 lo = __floats2half2_rn(v[0], v[1]), hi = __floats2half2_rn(v[2], v[3]);
+// four fp32 values times `up`, rounded to fp16, into 8 bytes of shared memory
+__device__ __forceinline__ void st4h(__half* p, const float* v, float up) {
+  const __half2 lo = __floats2half2_rn(v[0] * up, v[1] * up), hi = __floats2half2_rn(v[2] * up, v[3] * up);
   uint2 u;
   u.x = *reinterpret_cast<const unsigned*>(&lo);
   u.y = *reinterpret_cast<const unsigned*>(&hi);
   *reinterpret_cast<uint2*>(p) = u;
+}
+// The largest magnitude of v[0..31] over the warp's lanes (lanes < n), as float bits
+__device__ __forceinline__ unsigned warp_absmax32(const float (&v)[32], int lane, int n = 32) {
+  float m = 0.f;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) m = fmaxf(m, fabsf(v[j]));
+  return __reduce_max_sync(0xffffffffu, lane < n ? __float_as_uint(m) : 0u);  // (non-negative floats order as ints)
+}
+// The power-of-two factor that puts magnitude m (float bits) in [2^14, 2^15)
+// (the fp16 record's block scale is its inverse, written to *inv)
+__device__ __forceinline__ float block_up(unsigned mbits, float* inv) {
+  const int ex = (int)((mbits >> 23) & 0xff) - 126;
+  const int e = min(126, max(-126, 15 - ex));
+  if (inv) *inv = __int_as_float((127 - e) << 23);
+  return __int_as_float((127 + e) << 23);
 }
 // Warp-specialised, 544 threads (17 warps), one CTA per (sequence, value head):
 //   issuer warp 0 (lane 0): the three products of every chunk and the P^T,
@@ -420,6 +435,9 @@ constexpr uint32_t OP_DV = OP + 48128;
 static_assert(OP_DV >= OP_PBR + 1024 && OP_DV + 16384 <= OP_KED + 32768 && OP_DV >= 4 * 32768,
               "dv staging");
 constexpr uint32_t R_TT = 16384, R_MB = 0;
+// the record's scales are staged over the spent T image (above the fp16 record staging)
+constexpr uint32_t SC_STAGE = 65536;
+static_assert(SC_STAGE >= 65536 && SC_STAGE + 64 + 160 <= OP, "record scale staging");
 constexpr uint32_t PAD_SBO = 128 * 36;  // bytes per 8 rows of a padded 128-wide K tile
 static_assert(OP_DO + 2 * 64 * PAD_SBO / 8 <= SMALL && OP_PBR + 1024 <= OP_DO && R_MB + 16 * PAD_SBO <= OP &&
                   R_TT + 16384 <= R_P,
@@ -713,22 +731,58 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(const __grid_c
     // ---------------------------------------------------------------- record
     {  // the record staged in shared memory (now free) in its global layout, then bulk-stored
       __half* st = reinterpret_cast<__half*>(sm);  // fp16 [dP; dA] | [dQE; dKE'] | dKEd, as in the record
+      // their 16 block scales, as in the record, and the per-warp maxima they come from
+      float* ssc = reinterpret_cast<float*>(sm + SC_STAGE);
+      unsigned* wmax = reinterpret_cast<unsigned*>(sm + SC_STAGE + 64);  // [warp][5]
       static_assert(2 * (GH_KED + 8192) <= OP_DO, "record staging below [dO; -dR]");
       static_assert(2 * (GH_KED + 8192) == 4 * G_DBR, "fp32 tail follows the fp16 matrices");
+      static_assert(GREC == G_SC + 16, "record scales");
+      const int warp = cx.warp, half = cx.sub >> 1;  // rows 64 half .. of [dP; dA] and [dQE; dKE']
       float v[32];
+      {  // block maxima: [dP; dA] (half, hcol), [dQE; dKE'] (half, 2 hcol + cb), dKEd (2 hcol + cb)
+        tmem_ld32(tm + lo + TM_PA + hcol * 32, v);
+        unsigned m0 = warp_absmax32(v, lane);
+        unsigned mq[2], mk[2];
+        for (int cb = 0; cb < 2; ++cb) {
+          tmem_ld32(tm + lo + TM_QK + hcol * 64 + cb * 32, v);
+          mq[cb] = warp_absmax32(v, lane);
+          tmem_ld32(tm + lo + TM_KED + hcol * 64 + cb * 32, v);
+          mk[cb] = warp_absmax32(v, lane, 16);  // (M = 64 accumulator: lanes < 16)
+        }
+        if (lane == 0) {
+          wmax[warp * 5 + 0] = m0;
+          wmax[warp * 5 + 1] = mq[0];
+          wmax[warp * 5 + 2] = mq[1];
+          wmax[warp * 5 + 3] = mk[0];
+          wmax[warp * 5 + 4] = mk[1];
+        }
+      }
+      __syncthreads();
+      // warp w = 4 hcol + sub: the blocks of rows half (sub / 2) come from warps 4 hcol + 2 half + {0, 1};
+      // dKEd's from the four warps 4 hcol + {0 .. 3}
+      const int w0 = 4 * hcol + 2 * half, wk = 4 * hcol;
+      float inv;
+      float up = block_up(max(wmax[w0 * 5 + 0], wmax[(w0 + 1) * 5 + 0]), &inv);
+      if (cx.sub == 2 * half && lane == 0) ssc[half * 2 + hcol] = inv;
       tmem_ld32(tm + lo + TM_PA + hcol * 32, v);
 #pragma unroll
-      for (int q4 = 0; q4 < 8; ++q4) st4h(st + GH_PA + rec_off(Lr, hcol * 32 + 4 * q4, 64), v + 4 * q4);
+      for (int q4 = 0; q4 < 8; ++q4) st4h(st + GH_PA + rec_off(Lr, hcol * 32 + 4 * q4, 64), v + 4 * q4, up);
       for (int cb = 0; cb < 2; ++cb) {
         const int f0 = hcol * 64 + cb * 32;
+        up = block_up(max(wmax[w0 * 5 + 1 + cb], wmax[(w0 + 1) * 5 + 1 + cb]), &inv);
+        if (cx.sub == 2 * half && lane == 0) ssc[4 + half * 4 + f0 / 32] = inv;
         tmem_ld32(tm + lo + TM_QK + f0, v);
 #pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) st4h(st + GH_QK + rec_off(Lr, f0 + 4 * q4, 128), v + 4 * q4);
+        for (int q4 = 0; q4 < 8; ++q4) st4h(st + GH_QK + rec_off(Lr, f0 + 4 * q4, 128), v + 4 * q4, up);
+        const unsigned mk = max(max(wmax[wk * 5 + 3 + cb], wmax[(wk + 1) * 5 + 3 + cb]),
+                                max(wmax[(wk + 2) * 5 + 3 + cb], wmax[(wk + 3) * 5 + 3 + cb]));
+        up = block_up(mk, &inv);
+        if (cx.sub == 0 && lane == 0) ssc[12 + f0 / 32] = inv;
         tmem_ld32(tm + lo + TM_KED + f0, v);
         if (lane < 16) {
           const int r = cx.sub * 16 + lane;  // M = 64 accumulator layout
 #pragma unroll
-          for (int q4 = 0; q4 < 8; ++q4) st4h(st + GH_KED + rec_off(r, f0 + 4 * q4, 128), v + 4 * q4);
+          for (int q4 = 0; q4 < 8; ++q4) st4h(st + GH_KED + rec_off(r, f0 + 4 * q4, 128), v + 4 * q4, up);
         }
       }
       fence_async_smem();
@@ -738,6 +792,7 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_grads_tc_kernel(const __grid_c
         bulk_s2g(rec + 8192, sb + 32768, 32768);
         bulk_s2g(rec + G_DBR, sb + S_EMID, 256);
         bulk_s2g(rec + G_DEL, sb + S_EL, 512);
+        bulk_s2g(rec + G_SC, sb + SC_STAGE, 64);
         bulk_commit();
         bulk_wait_read();
       }

@@ -14,9 +14,15 @@ constexpr int FWD_VBLOCK = 32;   // V columns per CTA in the chunked kernels
 // r % 8 (element (r, c) of a row of n at rec_off(r, c, n)): [dP; dA] as [i'][j]
 // (128 x 64, i' < 64 dP) at half offset GH_PA, [dQE; dKE'] as [i'][f] (128 x
 // 128, i' < 64 dQE) at GH_QK, dKEd as [i][f] (64 x 128) at GH_KED; then fp32
-// dbeta_R [64] and dEl [128] at float offsets G_DBR, G_DEL; GREC floats per
-// chunk.  (fp16 keeps 11 significant bits: about 3e-4 relative RMS added to
-// the gradients, against their 2e-3 bar; the range covers these sums.)
+// dbeta_R [64] and dEl [128] at float offsets G_DBR, G_DEL; then 16 fp32
+// power-of-two scales of the fp16 values (value = half * scale), one per
+// 64-row half and group of 32 columns: [dP; dA] as [half][2] at G_SC,
+// [dQE; dKE'] as [half][4] at G_SC + 4, dKEd as [4] at G_SC + 12; GREC floats
+// per chunk.  (The scale puts each block's largest magnitude in [2^14,
+// 2^15): fp16 keeps 11 significant bits down to 2^-29 of it, about 3e-4
+// relative RMS added to the gradients against their 2e-3 bar, whatever the
+// gradients' range.)
+constexpr int GH_PA = 0, GH_QK = 8192, GH_KED = 24576, G_DBR = 16384, G_DEL = 16448, G_SC = 16576, GREC = 16592;
 // Per-(b, hv, 64-step chunk) interaction record that the tensor-core forward
 // stores with a workspace (floats).  Three 64 x 64 tf32 operand images in the
 // K-major canonical layout of the tensor-core kernels (element (r, k) at
@@ -33,7 +39,6 @@ constexpr int INTER_T = 4096, INTER_AH = 8192, INTER_TT = 12288, INTER_REC = 163
 // for the state pass (64 x 64 tf32 each, K-major canonical layout,
 // (r, k) = T[r][k] and P[r][k]).
 constexpr unsigned FWR_T = 0, FWR_P = 16384, FWI_BYTES = 32768;
-constexpr int GH_PA = 0, GH_QK = 8192, GH_KED = 24576, G_DBR = 16384, G_DEL = 16448, GREC = 16576;
 
 // Chunk geometry of the tensor-core kernels (Args: FwdArgs or BwdArgs).
 // Uniform batches: sequence s = batch row, NT = ceil(T / 64) chunks each, the

@@ -121,9 +121,10 @@ size_t kda_fwd_scratch_bytes(int B, int T, int HV, int K, int V);
  * kda_fwd_workspace_bytes lays them out), then the larger of the forward's
  * scratch and [gradients of the state leaving every 32 steps (state layout);
  * when HV > H fp32 per-value-head partials of dq and dk [B, T, HV, K] each;
- * per-chunk gradient records (K = V = 128; 66,304 bytes per 64-step chunk:
- * the chunk's C x C and C x K adjoints in fp16, its per-row and per-channel
- * terms in fp32)]; 0 if a size is invalid.  This is
+ * per-chunk gradient records (K = V = 128; 66,368 bytes per 64-step chunk:
+ * the chunk's C x C and C x K adjoints in fp16 with a power-of-two scale
+ * per 64 rows and 32 columns, its per-row and per-channel terms in fp32)];
+ * 0 if a size is invalid.  This is
  * at least kda_fwd_workspace_bytes(), so one buffer serves both calls. */
 size_t kda_bwd_workspace_bytes(int B, int T, int H, int HV, int K, int V);
 

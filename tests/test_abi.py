@@ -138,7 +138,7 @@ def test_tensor_core_workspace_sizes(lib):
     img = max(B * HV * nt64 * 32768, B * HV * nt32 * fma_rec_bytes(K))
     assert lib.kda_fwd_scratch_bytes(B, T, HV, K, V) == img
     assert lib.kda_fwd_workspace_bytes(B, T, HV, K, V) == states + inter + img
-    tail = states + 2 * B * T * HV * K * 4 + B * HV * nt64 * 16576 * 4  # state grads, dq/dk partials, records
+    tail = states + 2 * B * T * HV * K * 4 + B * HV * nt64 * 16592 * 4  # state grads, dq/dk partials, records
     assert lib.kda_bwd_workspace_bytes(B, T, H, HV, K, V) == states + inter + max(tail, img)
     assert lib.kda_bwd_workspace_bytes(B, T, H, HV, K, V) >= lib.kda_fwd_workspace_bytes(B, T, HV, K, V)
     assert lib.kda_fwd_scratch_bytes(B, T, HV, 64, 64) == B * HV * nt32 * (fma_rec_bytes(64) + 4 * (64 * 64 + 32 * 64))
